@@ -1,0 +1,175 @@
+"""Float32 op-by-op reference of the grid fit, the projection and the fused
+ADMM-Q epilogue (TEST INFRASTRUCTURE ONLY; see oracle/__init__.py).
+
+The D-update of ADMM-Q is a projection onto a per-group asymmetric integer
+grid whose scale and zero-point are refreshed from the current iterate
+(ADMM-Q technical summary, Methodology section 2: D-update and grid refresh).
+Where a float decides an integer, the CUDA kernels and the oracle must take
+that decision in the same precision, so the decision is spelled out here as a
+sequence of IEEE float32 operations, each rounded to nearest-even on its own
+(no fused multiply-add), with rint = round half to even.  Given the same
+float32 inputs the kernels must reproduce these outputs bit for bit.
+
+Grid semantics (our reading; the pages do not define the fit):
+  minmax  mn = min(0, min y), mx = max(0, max y), s = (mx - mn) / L,
+          z = rint(-mn / s); an all-zero group gets s = 1, z = 0.
+  lsq     codes on the previous grid, then one weighted least-squares refit of
+          y ~ s (q - z) with weights w = diag(H) (the metric of the scaled
+          problem): first slope and offset, then the integer zero point, then
+          the slope again for that zero point.  Groups whose fit is degenerate
+          keep the previous grid.
+  rounding q = clamp(rint(y / s) + z, 0, L);  D = s (q - z).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+f32 = np.float32
+
+
+def _f(x):
+    return np.asarray(x, dtype=np.float32)
+
+
+def fit_minmax(yg: np.ndarray, L: int):
+    """(scale, zero) per group; yg has one group per row."""
+    yg = _f(yg)
+    mn = np.minimum(yg.min(axis=1), f32(0))
+    mx = np.maximum(yg.max(axis=1), f32(0))
+    s = _f(np.subtract(mx, mn, dtype=f32) / f32(L))
+    zero_range = s == f32(0)
+    s_safe = np.where(zero_range, f32(1), s).astype(f32)
+    z = np.rint(_f(np.negative(mn) / s_safe)).astype(f32)
+    z = np.where(zero_range, f32(0), z).astype(f32)
+    return s_safe, z
+
+
+def fit_lsq(yg: np.ndarray, wg: np.ndarray, s_prev: np.ndarray, z_prev: np.ndarray, L: int):
+    """Weighted least-squares grid refit, sums taken in element order."""
+    yg, wg = _f(yg), _f(wg)
+    s0, z0 = _f(s_prev), _f(z_prev)
+    q = round_to_grid(yg, s0, z0, L)
+    G, g = yg.shape
+    Sw = np.zeros(G, f32); Sq = np.zeros(G, f32); Sqq = np.zeros(G, f32)
+    Sy = np.zeros(G, f32); Sqy = np.zeros(G, f32)
+    for i in range(g):
+        w, qi, yi = wg[:, i], q[:, i], yg[:, i]
+        wq = _f(w * qi)
+        Sw = _f(Sw + w)
+        Sq = _f(Sq + wq)
+        Sqq = _f(Sqq + _f(wq * qi))
+        Sy = _f(Sy + _f(w * yi))
+        Sqy = _f(Sqy + _f(wq * yi))
+    qm = _f(Sq / Sw)
+    ym = _f(Sy / Sw)
+    var = _f(Sqq - _f(Sq * qm))
+    cov = _f(Sqy - _f(Sq * ym))
+    ok = (var > 0) & (cov > 0)
+    s1 = _f(cov / np.where(ok, var, f32(1)))
+    zc = np.clip(np.rint(_f(qm - _f(ym / np.where(ok, s1, f32(1))))), f32(0), f32(L)).astype(f32)
+    num = _f(Sqy - _f(zc * Sy))
+    den = _f(_f(Sqq - _f(_f(f32(2) * zc) * Sq)) + _f(_f(zc * zc) * Sw))
+    ok2 = (den > 0) & (num > 0)
+    s2 = np.where(ok2, _f(num / np.where(ok2, den, f32(1))), s1).astype(f32)
+    s = np.where(ok, s2, s0).astype(f32)
+    z = np.where(ok, zc, z0).astype(f32)
+    return s, z
+
+
+def round_to_grid(yg: np.ndarray, s: np.ndarray, z: np.ndarray, L: int) -> np.ndarray:
+    """q = clamp(rint(y / s) + z, 0, L), as float32 integers."""
+    r = np.rint(_f(_f(yg) / _f(s)[:, None]))
+    return np.clip(_f(r + _f(z)[:, None]), f32(0), f32(L)).astype(f32)
+
+
+def dequantize(q: np.ndarray, s: np.ndarray, z: np.ndarray) -> np.ndarray:
+    """D = s (q - z) in float32 (q - z is an exact small integer)."""
+    return _f(_f(s)[:, None] * _f(_f(q) - _f(z)[:, None]))
+
+
+def bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 to bfloat16, nearest-even; returns the 16-bit patterns."""
+    b = _f(x).view(np.uint32).astype(np.uint64)
+    lsb = (b >> 16) & 1
+    return (((b + 0x7FFF + lsb) >> 16) & 0xFFFF).astype(np.uint16)
+
+
+def bf16_value(bits: np.ndarray) -> np.ndarray:
+    return (np.asarray(bits, np.uint32) << 16).view(np.float32)
+
+
+def split_bf16(x: np.ndarray):
+    """x ~= hi + lo with hi = bf16(x), lo = bf16(x - hi) (the split-precision
+    operand planes of the eigenbasis GEMMs)."""
+    hi = bf16_bits(x)
+    lo = bf16_bits(_f(_f(x) - bf16_value(hi)))
+    return hi, lo
+
+
+def _rows_to_groups(A: np.ndarray, g: int) -> np.ndarray:
+    m, d = A.shape
+    return A.reshape(m * (d // g), g)
+
+
+def init_step(W_rows: np.ndarray, rsig: np.ndarray, bits: int, group: int):
+    """RTN start of the iteration in memory layout ([d_out][d_in]).
+
+    y = W_hat; minmax grid; D = s (q - z); D~ = D * rsig (rsig = sqrt(diag H)),
+    V~ = 0 and P = D~ - V~ = D~.
+    """
+    L = (1 << bits) - 1
+    m, d = W_rows.shape
+    yg = _rows_to_groups(_f(W_rows), group)
+    s, z = fit_minmax(yg, L)
+    q = round_to_grid(yg, s, z, L)
+    D = dequantize(q, s, z).reshape(m, d)
+    Dt = _f(D * _f(rsig)[None, :])
+    hi, lo = split_bf16(Dt)
+    return dict(codes=q.reshape(m, d).astype(np.uint8), scale=s.reshape(m, d // group),
+                zero=z.reshape(m, d // group), P=Dt, P_hi=hi, P_lo=lo)
+
+
+def epilogue_step(W_acc: np.ndarray, V: np.ndarray, sigma: np.ndarray, rsig: np.ndarray,
+                  hdiag: np.ndarray, s_prev: np.ndarray, z_prev: np.ndarray,
+                  codes_prev: np.ndarray, bits: int, group: int, mode: str):
+    """One fused projection + dual update in memory layout ([d_out][d_in]).
+
+    Per element (i = input channel):
+      t  = W~ + V~          y  = sigma_i t
+      grid (minmax | lsq | frozen) per group of `group` columns of one row
+      q  = clamp(rint(y/s) + z, 0, L),  D = s (q - z),  D~ = D * rsig_i
+      V~' = t - D~          P  = D~ - V~'   (split into bf16 hi/lo planes)
+    Residual sums (float64 here; the kernels sum in float32, compared with a
+    tolerance): r2 = sum (W~ - D~)^2 and s2 = sum (D~ - D~_prev)^2 where
+    D~_prev = s_prev (q_prev - z_prev) * rsig.
+    """
+    L = (1 << bits) - 1
+    m, d = W_acc.shape
+    W_acc, V = _f(W_acc), _f(V)
+    t = _f(W_acc + V)
+    y = _f(_f(sigma)[None, :] * t)
+    yg = _rows_to_groups(y, group)
+    sp = _f(s_prev).reshape(-1)
+    zp = _f(z_prev).reshape(-1)
+    if mode == "minmax":
+        s, z = fit_minmax(yg, L)
+    elif mode == "lsq":
+        wg = np.broadcast_to(_f(hdiag).reshape(d // group, group)[None],
+                             (m, d // group, group)).reshape(-1, group)
+        s, z = fit_lsq(yg, wg, sp, zp, L)
+    elif mode == "frozen":
+        s, z = sp, zp
+    else:
+        raise ValueError(mode)
+    q = round_to_grid(yg, s, z, L)
+    D = dequantize(q, s, z).reshape(m, d)
+    Dt = _f(D * _f(rsig)[None, :])
+    V_new = _f(t - Dt)
+    P = _f(Dt - V_new)
+    hi, lo = split_bf16(P)
+    qp = _rows_to_groups(_f(codes_prev), group)
+    Dt_prev = _f(dequantize(qp, sp, zp).reshape(m, d) * _f(rsig)[None, :])
+    r2 = float(np.sum((W_acc.astype(np.float64) - Dt) ** 2))
+    s2 = float(np.sum((Dt.astype(np.float64) - Dt_prev) ** 2))
+    return dict(codes=q.reshape(m, d).astype(np.uint8), scale=s.reshape(m, d // group),
+                zero=z.reshape(m, d // group), V=V_new, P=P, P_hi=hi, P_lo=lo, r2=r2, s2=s2)
