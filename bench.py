@@ -1,0 +1,413 @@
+#!/usr/bin/env python
+"""Benchmark of the ADMM-Q layer solve on B200.
+
+One step = the hot path of one layer solve on device-resident inputs:
+  Gram X^T X (tcgen05, bf16 -> fp32)  ->  damping + diagonal scaling  ->
+  C0' GEMM + RTN start  ->  T ADMM iterations (GEMM 1 + GEMM 2 with the fused
+  projection / dual update)  ->  residuals + objective  ->  b-bit packing.
+The one-time eigendecomposition (cuSOLVER, float64) is outside the step: it
+runs during warm-up, is timed on its own and reported as `eigh_s`.
+
+Multi-GPU: layers are independent problems, so every rank solves its own
+layer (seed = rank) with no collective in the data path ("scaling": "weak").
+
+    python bench.py [--gpus N --steps K --warmup W --workload q_proj --grid minmax]
+    python bench.py --impl reference   # the float64 CPU oracle on a bounded sample
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from post_weight_quantization_10_b200 import workloads  # noqa: E402
+
+METRIC = "ADMM-Q layer solve: iters/s, TFLOP/s vs tensor peak; Gram TFLOP/s; s/layer"
+REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return dict(hbm=j["hbm_gbs"], bf16=j["bf16_tflops"],
+                    bf16_sust=j.get("bf16_tflops_sustained", j["bf16_tflops"]), src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, src="fallback")
+
+
+def workload_desc(p, grid):
+    return (f"{p.name}: d_in={p.d_in} d_out={p.d_out} n={p.n} W{p.bits} g{p.group} T={p.iters} "
+            f"grid={grid} (Qwen3-8B-shaped synthetic layer, seed=rank)")
+
+
+# ------------------------------------------------------------------ clocks
+
+
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.gpu)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for name, val in zip(REASONS, parts[4:8]):
+                    if val.lower().startswith("active"):
+                        reasons.add(name)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------- our solver
+
+
+class LayerRun:
+    """Device-resident state of one layer solve through the C ABI binding."""
+
+    def __init__(self, A, p, grid, seed, device):
+        self.A, self.p = A, p
+        self.X = workloads.make_activations(p, seed=seed, device=device)
+        self.W = workloads.make_weights(p, seed=seed, device=device, dtype=torch.bfloat16)
+        self.H = torch.empty((p.d_in, p.d_in), dtype=torch.float32, device=device)
+        self.gram_ws = torch.empty(A.gram_workspace_bytes(p.n, p.d_in), dtype=torch.uint8,
+                                   device=device)
+        prm = A.Params(bits=p.bits, group=p.group, iters=p.iters, rho0=p.rho0, gamma=p.gamma,
+                       lambda_rel=p.lambda_rel, grid=grid)
+        self.s = A.Solver(p.d_in, p.d_out, prm, device=device)
+        self.packed = torch.empty((p.d_out, p.d_in * p.bits // 32), dtype=torch.int32,
+                                  device=device)
+
+    def setup_eigh(self):
+        A = self.A
+        A.build_hessian(self.X, self.H, workspace=self.gram_ws)
+        self.s.prepare(self.H, self.W)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        self.s.eigh()
+        torch.cuda.synchronize()
+        return time.perf_counter() - t0
+
+    def step(self, ev=None):
+        A, p = self.A, self.p
+        mark = (lambda k: ev[k].record()) if ev else (lambda k: None)
+        mark(0)
+        A.build_hessian(self.X, self.H, workspace=self.gram_ws)
+        mark(1)
+        self.s.prepare(self.H, self.W)   # damping + scaling (eigenbasis from setup)
+        self.s.init()
+        mark(2)
+        self.s.iterate(0, p.iters)
+        mark(3)
+        self.s.finish()
+        A.pack(self.s.codes, p.bits, out=self.packed)
+        mark(4)
+
+
+def run_ours(args, rank, world, device):
+    from post_weight_quantization_10_b200 import admmq as A
+    A.lib()
+    p = workloads.PRESETS[args.workload]
+    run = LayerRun(A, p, args.grid, seed=rank, device=device)
+    eigh_s = run.setup_eigh()
+    for _ in range(args.warmup):
+        run.step()
+    torch.cuda.synchronize()
+
+    # ---- device-resident timed region
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    run.s.set_timing(True)
+    n0 = A.launch_count()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for k in range(args.steps):
+        run.step(evs[k])
+    t_end.record()
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    launches = A.launch_count() - n0
+    clk = clocks.stop()
+    ms = t_start.elapsed_time(t_end)
+    gemm_ms, gemm_n = run.s.get_timing()
+    run.s.set_timing(False)
+    phase = np.zeros(4)
+    for e in evs:
+        phase += [e[i].elapsed_time(e[i + 1]) for i in range(4)]
+    phase /= args.steps
+    ms_max = dist_max(ms, world, device)
+
+    # ---- end to end: host buffers, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(A, run, args, world, device)
+
+    if rank != 0:
+        return None
+    pk = peaks()
+    d, m, n, T = p.d_in, p.d_out, p.n, p.iters
+    layers = args.steps * world
+    iters_per_s = T * layers / (ms_max / 1e3)
+    flops_iter = 4.0 * d * d * m
+    admm_ms = phase[2]
+    gram_flops = float(n) * d * (d + 1)
+    # dominant kernel: GEMM 1 or GEMM 2 (same algorithmic flops, 2 d^2 m each)
+    k = 0 if gemm_ms[0] >= gemm_ms[1] else 1
+    avg_ms = gemm_ms[k] / max(gemm_n[k], 1)
+    achieved = 2.0 * d * d * m / (avg_ms / 1e3) / 1e12
+    # 3xTF32: three tf32 MMAs per fp32-accurate product; dense tf32 runs at half
+    # the bf16 rate (nominal 1.1 vs 2.25 PFLOP/s), so the peak is bf16 / 6.
+    peak_split = pk["bf16_sust"] / 6.0
+    line = {
+        "metric": METRIC,
+        "value": iters_per_s,
+        "unit": "iters/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "3xtf32-f32",
+        "data": "synthetic (seeded Qwen3-8B-shaped activations and weights; no dataset)",
+        "config": {"workload": workload_desc(p, args.grid), "parallelism": f"independent layers x{world}",
+                   "l2": "inputs larger than L2 (X is %.1f GiB)" % (n * d * 2 / 2**30),
+                   "eigh": "one-time setup outside the step (eigh_s)"},
+        "s_per_layer": ms_max / 1e3 / args.steps,
+        "s_per_layer_with_eigh": ms_max / 1e3 / args.steps + eigh_s,
+        "eigh_s": eigh_s,
+        "phase_ms": {"gram": phase[0], "scale_init": phase[1], "admm": phase[2],
+                     "finish_pack": phase[3]},
+        "admm_iters_per_s": T / (admm_ms / 1e3),
+        "admm_tflops_fp32_accurate": flops_iter * T / (admm_ms / 1e3) / 1e12,
+        "gram_tflops": gram_flops / (phase[0] / 1e3) / 1e12,
+        "gemm_ms_per_launch": [gemm_ms[0] / max(gemm_n[0], 1), gemm_ms[1] / max(gemm_n[1], 1)],
+        "roofline": {"kernel": ["gemm1_eigscale", "gemm2_project"][k], "bound": "tensor",
+                     "achieved": achieved, "peak": peak_split, "unit": "TFLOP/s",
+                     "frac": achieved / peak_split, "traffic": None,
+                     "peak_note": "bf16 dense %s sustained %.1f TF/s x 1/2 (tf32) / 3 (three "
+                                  "tf32 MMAs per fp32-accurate product)" % (pk["src"], pk["bf16_sust"])},
+        "gpu_launches": launches,
+        "clocks": clk,
+        "e2e": e2e,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(p, args.grid)
+    return line
+
+
+def run_e2e(A, run, args, world, device):
+    p = run.p
+    Xh = torch.empty(run.X.shape, dtype=run.X.dtype, pin_memory=True)
+    Xh.copy_(run.X)
+    Wh = torch.empty(run.W.shape, dtype=run.W.dtype, pin_memory=True)
+    Wh.copy_(run.W)
+    codes_h = torch.empty(run.s.codes.shape, dtype=torch.uint8, pin_memory=True)
+    packed_h = torch.empty(run.packed.shape, dtype=torch.int32, pin_memory=True)
+    scale_h = torch.empty(run.s.scale.shape, dtype=torch.float32, pin_memory=True)
+    zero_h = torch.empty_like(scale_h, pin_memory=True)
+    obj_h = torch.empty(1, dtype=torch.float64, pin_memory=True)
+    h2d = Xh.numel() * Xh.element_size() + Wh.numel() * Wh.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in (codes_h, packed_h, scale_h, zero_h, obj_h))
+
+    def step():
+        run.X.copy_(Xh, non_blocking=True)
+        run.W.copy_(Wh, non_blocking=True)
+        run.step()
+        codes_h.copy_(run.s.codes, non_blocking=True)
+        packed_h.copy_(run.packed, non_blocking=True)
+        scale_h.copy_(run.s.scale, non_blocking=True)
+        zero_h.copy_(run.s.zero, non_blocking=True)
+        obj_h.copy_(run.s.objective, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    ms = dist_max(a.elapsed_time(b), world, device)
+    return {"value": p.iters * args.steps * world / (ms / 1e3), "unit": "iters/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "s_per_layer": ms / 1e3 / args.steps}
+
+
+# --------------------------------------------------- CPU oracle (baseline)
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max((i.get("num_threads", 0) for i in info), default=None)
+    except Exception:
+        return None
+
+
+def cpu_sample(p, grid, seed=0):
+    """Time the float64 oracle on a bounded sample of the layer: the Gram of
+    8192 tokens and one ADMM iteration (W-update, projection, dual update) at
+    the full layer size; extrapolate to the step (n tokens, T iterations)."""
+    from oracle import admmq_oracle as O
+    rng = np.random.default_rng(seed)
+    d, m = p.d_in, p.d_out
+    ns = min(8192, p.n)
+    Xs = rng.standard_normal((ns, d)).astype(np.float32)
+    t0 = time.perf_counter()
+    O.gram(Xs)
+    t_gram = (time.perf_counter() - t0) * (p.n / ns)
+    Q = rng.standard_normal((d, d)) / np.sqrt(d)
+    lam = np.abs(rng.standard_normal(d)) + 0.1
+    B = rng.standard_normal((d, m)) * 0.02
+    Dt = rng.standard_normal((d, m)) * 0.02
+    Vt = rng.standard_normal((d, m)) * 0.002
+    sigma = np.abs(rng.standard_normal(d)) * 0.01 + 0.01
+    hdiag = (1.0 / sigma ** 2).astype(np.float32)
+    s_prev = np.full((d // p.group, m), 0.01, np.float32)
+    z_prev = np.full((d // p.group, m), 3.0, np.float32)
+    t0 = time.perf_counter()
+    Wt = O.w_update(Q, lam, B, 0.1, Dt, Vt)
+    Y = sigma[:, None] * (Wt + Vt)
+    _, _, _, D = O.project(Y, p.bits, p.group, grid, hdiag, s_prev, z_prev)
+    Vt = Vt + Wt - D / sigma[:, None]
+    t_iter = time.perf_counter() - t0
+    step_s = t_gram + p.iters * t_iter
+    return dict(t_gram=t_gram, t_iter=t_iter, step_s=step_s, iters_per_s=p.iters / step_s,
+                sample=f"Gram of {ns} of {p.n} tokens + 1 of {p.iters} ADMM iterations at "
+                       f"d_in={d} d_out={m}, extrapolated linearly (eigh excluded, as on the GPU)")
+
+
+def cpu_baseline(p, grid):
+    r = cpu_sample(p, grid)
+    return {"value": r["iters_per_s"], "unit": "iters/s", "cores": _blas_threads() or os.cpu_count(),
+            "kind": "oracle", "sample": r["sample"], "s_per_layer": r["step_s"]}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    p = workloads.PRESETS[args.workload]
+    for _ in range(args.warmup):
+        cpu_sample(p, args.grid)
+    vals = [cpu_sample(p, args.grid) for _ in range(args.steps)]
+    step_s = float(np.mean([v["step_s"] for v in vals]))
+    value = p.iters / step_s
+    cores = _blas_threads() or os.cpu_count()
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "iters/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_desc(p, args.grid)},
+            "cpu_baseline": {"value": value, "unit": "iters/s", "cores": cores, "kind": "oracle",
+                             "sample": vals[0]["sample"]},
+            "e2e": {"value": value, "unit": "iters/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# ------------------------------------------------------------ distributed
+
+
+def dist_barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def dist_max(v, world, device):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="q_proj", choices=sorted(workloads.PRESETS))
+    ap.add_argument("--grid", default="minmax", choices=["minmax", "lsq", "frozen"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line:
+            print(json.dumps(line), flush=True)
+        return
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    try:
+        line = run_ours(args, rank, world, device)
+        if line:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,206 @@
+/*
+ * admmq.h -- C ABI of the B200 (sm_100a) ADMM-Q layer solve.
+ *
+ * The method (ADMM-Q technical summary, gist.science 2605.11222, Methodology):
+ * for one linear layer with pre-trained weights W_hat (d_in x d_out) and
+ * calibration activations X (n x d_in), minimise
+ *     1/2 Tr((W - W_hat)^T H (W - W_hat))   s.t.  W on a per-group integer grid,
+ * with H = X^T X + lambda I (section 1).  The solve scales by
+ * Sigma = Diag(H)^(-1/2), eigendecomposes the scaled Hessian once, and runs
+ * ADMM under rho_t = rho0 * gamma^t: an eigenbasis W-update, a D-update that
+ * projects onto a per-group asymmetric grid refreshed from the current iterate,
+ * and the dual update V += W - D (section 2).
+ *
+ * Conventions for every entry point:
+ *   - Pointers named *_dev are DEVICE pointers owned by the caller; the
+ *     library never frees them and keeps no reference after the call returns,
+ *     except the context, which keeps the workspace pointer and the W_hat
+ *     pointer given to admmq_prepare() until admmq_destroy().
+ *   - `stream` is a cudaStream_t passed as void*; NULL means the legacy default
+ *     stream.  Calls are asynchronous on that stream unless stated otherwise.
+ *   - Matrices are row-major.  W_hat and codes use the torch nn.Linear layout
+ *     [d_out][d_in] (the pages' d_in x d_out matrix stored column-major).
+ *     A quantization group is `group` consecutive input channels of one output
+ *     row; scale/zero are [d_out][d_in / group].
+ *   - Return value: ADMMQ_OK (0) or a negative ADMMQ_ERR_* code.  Nothing is
+ *     launched when an argument check fails.  No exception crosses the ABI.
+ *   - Sizes: d_in a multiple of 32 and of `group`; group in {32, 64, 128};
+ *     bits in 1..8; d_out >= 1; n >= 0.
+ */
+#ifndef ADMMQ_H_
+#define ADMMQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  ADMMQ_OK = 0,
+  ADMMQ_ERR_INVALID_ARG = -1, /* a size, pointer or parameter is out of range   */
+  ADMMQ_ERR_CUDA = -2,        /* a CUDA runtime call or kernel launch failed      */
+  ADMMQ_ERR_EIG = -3,         /* the eigensolver reported failure (info != 0)    */
+  ADMMQ_ERR_NOT_PD = -4,      /* a diagonal entry of H is not positive           */
+  ADMMQ_ERR_NONFINITE = -5,   /* NaN/Inf found in H's diagonal or the eigenvalues */
+  ADMMQ_ERR_TIMEOUT = -6,     /* a kernel's bounded pipeline wait gave up        */
+  ADMMQ_ERR_WORKSPACE = -7,   /* the workspace is smaller than required          */
+  ADMMQ_ERR_UNSUPPORTED = -8  /* device is not sm_100 or a shape is unsupported  */
+};
+
+/* Grid refresh used by the D-update (the pages do not fix the fit). */
+enum {
+  ADMMQ_GRID_MINMAX = 0, /* scale/zero from the group's min/max, 0 included    */
+  ADMMQ_GRID_LSQ = 1,    /* weighted least-squares refit, weights diag(H)       */
+  ADMMQ_GRID_FROZEN = 2  /* keep the start grid (RTN grid of W_hat)             */
+};
+
+enum { ADMMQ_DTYPE_F32 = 0, ADMMQ_DTYPE_BF16 = 1 };
+
+typedef struct admmq_params {
+  int bits;         /* b: codes in [0, 2^b - 1]                                  */
+  int group;        /* g: input channels per quantization group                 */
+  int iters;        /* T: ADMM iterations                                        */
+  float rho0;       /* penalty at t = 0                                          */
+  float gamma;      /* penalty growth: rho_t = rho0 * gamma^t                    */
+  float lambda_rel; /* damping: lambda = lambda_rel * mean(diag(X^T X))          */
+  int grid_mode;    /* ADMMQ_GRID_*                                              */
+} admmq_params;
+
+typedef struct admmq_ctx admmq_ctx; /* opaque; host memory owned by the library */
+
+/* Status code -> static English string (never NULL). */
+const char* admmq_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int admmq_version(void);
+
+/* Number of CUDA kernels this library has launched in this process (all
+ * devices, all contexts); cuSOLVER's own kernels are not counted. */
+int64_t admmq_launch_count(void);
+
+/* ---------------------------------------------------------------- Hessian --
+ * Gram of the calibration activations, H = X^T X  (ADMM-Q summary, Methodology
+ * section 1: H = X^T X + lambda I; damping is added later by admmq_prepare).
+ *   X_dev      bf16 [n][d_in], row-major (token-major), 16-byte aligned.
+ *   H_dev      fp32 [d_in][d_in]; written in full (both triangles), or, with
+ *              accumulate != 0, the Gram of this chunk is added to its contents
+ *              (so X may be streamed in chunks of tokens).
+ *   ws_dev     scratch of at least admmq_gram_workspace_bytes(n, d_in) bytes.
+ * bf16 products are exact in fp32; sums are fp32 (tensor cores), combined in a
+ * fixed order, so the result is deterministic for a given device and shape. */
+size_t admmq_gram_workspace_bytes(int64_t n, int d_in);
+int admmq_build_hessian(const void* X_dev, int64_t n, int d_in, float* H_dev, int accumulate,
+                        void* ws_dev, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------- context --
+ * One context per layer solve.  ws_dev (caller-allocated device memory of at
+ * least admmq_workspace_bytes() bytes) holds all solver state; the context
+ * only stores pointers into it.  admmq_create() validates the parameters and
+ * creates the eigensolver handle; it launches nothing. */
+size_t admmq_workspace_bytes(int d_in, int d_out, const admmq_params* p);
+int admmq_create(admmq_ctx** ctx, int d_in, int d_out, const admmq_params* p, void* ws_dev,
+                 size_t ws_bytes);
+void admmq_destroy(admmq_ctx* ctx);
+
+/* Damping and diagonal scaling (Methodology section 1 and section 2,
+ * "diagonal scaling"): lambda = lambda_rel * mean(diag G), H = G + lambda I,
+ * sigma_i = H_ii^(-1/2), H~ = Sigma H Sigma (float64, into the workspace) and
+ * the scaled weights W^~ = Sigma^-1 W_hat as tf32 hi/lo planes (fp32 words).
+ *   G_dev      fp32 [d_in][d_in], X^T X WITHOUT damping (admmq_build_hessian).
+ *   W_hat_dev  [d_out][d_in], fp32 or bf16 (w_dtype); must stay valid until
+ *              admmq_destroy (the objective reads it).
+ * Returns ADMMQ_ERR_NOT_PD / _NONFINITE after a host sync if diag(H) is bad. */
+int admmq_prepare(admmq_ctx* ctx, const float* G_dev, const void* W_hat_dev, int w_dtype,
+                  void* stream);
+
+/* One-time eigendecomposition H~ = Q Lambda Q^T (Methodology section 2,
+ * W-update) with cuSOLVER's float64 divide-and-conquer solver, then the tf32
+ * hi/lo planes of Q^T and Q for the split-precision (3xTF32) GEMMs.  Synchronises the
+ * stream once to read the solver's info (ADMMQ_ERR_EIG if non-zero). */
+int admmq_eigh(admmq_ctx* ctx, void* stream);
+
+/* admmq_prepare + admmq_eigh. */
+int admmq_setup(admmq_ctx** ctx_out, const float* G_dev, const void* W_hat_dev, int w_dtype,
+                int d_in, int d_out, const admmq_params* p, void* ws_dev, size_t ws_bytes,
+                void* stream);
+
+/* Start of the iteration: C0' = Lambda Q^T W^~ (so that Q^T H~ W^~ = C0') and
+ * the RTN start D_0 = RTN(W_hat) on its min/max grid, V~_0 = 0.
+ *   codes_dev  u8 [d_out][d_in]; scale_dev, zero_dev fp32 [d_out][d_in/group]. */
+int admmq_init(admmq_ctx* ctx, uint8_t* codes_dev, float* scale_dev, float* zero_dev,
+               void* stream);
+
+/* ADMM iterations t = t0 .. t0+count-1 with rho_t = rho0 gamma^t:
+ *   T  = diag(1/(Lambda+rho)) (C0' + rho Q^T (D~ - V~))          (GEMM 1)
+ *   W~ = Q T;  D = grid projection of Sigma (W~ + V~);  V~ += W~ - D~  (GEMM 2
+ *        with the projection, the dual update and residual sums fused)
+ * codes/scale/zero are updated in place (they hold D).  t0 + count <= iters. */
+int admmq_iterate(admmq_ctx* ctx, int t0, int count, uint8_t* codes_dev, float* scale_dev,
+                  float* zero_dev, void* stream);
+
+/* After the last iteration: the objective 1/2 Tr((D - W_hat)^T H (D - W_hat))
+ * (H with damping) and the residual history.
+ *   resid_dev   optional fp64 [iters][2]: ||W~_t - D~_t||_F and
+ *               rho_t ||D~_t - D~_{t-1}||_F (scaled coordinates); NULL to skip.
+ *   objective_dev optional fp64 [1] (device); NULL to skip. */
+int admmq_finish(admmq_ctx* ctx, const uint8_t* codes_dev, const float* scale_dev,
+                 const float* zero_dev, double* resid_dev, double* objective_dev, void* stream);
+
+/* admmq_init + admmq_iterate(0, iters) + admmq_finish. */
+int admmq_solve(admmq_ctx* ctx, uint8_t* codes_dev, float* scale_dev, float* zero_dev,
+                double* resid_dev, double* objective_dev, void* stream);
+
+/* Pack codes u8 [d_out][d_in] into a little-endian b-bit stream per row:
+ * code k of a row occupies bits [b k, b k + b) of the row, in uint32 words;
+ * packed_dev is uint32 [d_out][d_in * bits / 32].  Codes must be < 2^bits.
+ * (Our reading of "same format as GPTQ", ADMM-Q summary, Experimental results
+ * section 3; the pages do not define the bit layout.) */
+int admmq_pack(const uint8_t* codes_dev, int d_in, int d_out, int bits, uint32_t* packed_dev,
+               void* stream);
+
+/* ------------------------------------------------------------ inspection --
+ * Device buffers inside the workspace, for tests and diagnostics.  Layouts:
+ *   ADMMQ_BUF_SIGMA, _RSIG, _HDIAG, _LAMBDA : fp32 [d_in]
+ *   ADMMQ_BUF_V      fp32 [d_out][d_in]  scaled dual V~
+ *   ADMMQ_BUF_C0     fp32 [d_out][d_in]  C0' = Lambda Q^T W^~ (row j, column k)
+ *   ADMMQ_BUF_P_HI/_P_LO  fp32 [d_out][d_in]  P = D~ - V~ as tf32 hi/lo planes
+ *   ADMMQ_BUF_T_HI/_T_LO  fp32 [d_out][d_in]  GEMM-1 output, tf32 hi/lo planes
+ *   ADMMQ_BUF_E_HI/_E_LO  fp32 [d_in][d_in]   row k = k-th eigenvector of H~ (tf32 planes)
+ *   ADMMQ_BUF_HT     fp64 [d_in][d_in]   H~ before admmq_eigh, Q^T after
+ *   ADMMQ_BUF_STATUS int32 [4]           kernel status words (0 = ok)     */
+enum {
+  ADMMQ_BUF_SIGMA = 0, ADMMQ_BUF_RSIG, ADMMQ_BUF_HDIAG, ADMMQ_BUF_LAMBDA, ADMMQ_BUF_V,
+  ADMMQ_BUF_C0, ADMMQ_BUF_P_HI, ADMMQ_BUF_P_LO, ADMMQ_BUF_T_HI, ADMMQ_BUF_T_LO,
+  ADMMQ_BUF_E_HI, ADMMQ_BUF_E_LO, ADMMQ_BUF_HT, ADMMQ_BUF_STATUS, ADMMQ_BUF_COUNT
+};
+int admmq_get_buffer(admmq_ctx* ctx, int which, void** ptr_dev, size_t* bytes);
+
+/* When wtilde_dev is non-NULL, the next GEMM-2 launches also write the raw
+ * fp32 product W~ [d_out][d_in] there (tests compare the fused projection with
+ * its float32 specification on exactly these values).  NULL turns it off. */
+int admmq_debug_dump_wtilde(admmq_ctx* ctx, float* wtilde_dev);
+
+/* Per-kernel timing with CUDA events recorded on the launch stream around
+ * every GEMM launch of admmq_iterate.  enable != 0 clears and starts it.
+ * admmq_get_timing returns the summed milliseconds and launch counts of
+ * GEMM 1 (index 0) and GEMM 2 (index 1); it synchronises on the events. */
+int admmq_set_timing(admmq_ctx* ctx, int enable);
+int admmq_get_timing(admmq_ctx* ctx, double ms[2], int launches[2]);
+
+/* Standalone projection kernel (the fused GEMM-2 epilogue reading W~ from
+ * memory instead of tensor memory); same per-element float32 arithmetic.
+ * All pointers device; V_dev is updated in place; P_hi/P_lo receive P as
+ * tf32 hi/lo planes in fp32 words (hi = tf32(P), lo = tf32(P - hi));
+ * codes/scale/zero hold the previous D on entry and the new D on exit;
+ * resid_dev fp64 [2] receives the two residual sums of squares. */
+int admmq_project(const float* wtilde_dev, float* V_dev, const float* sigma_dev,
+                  const float* rsig_dev, const float* hdiag_dev, int d_in, int d_out, int bits,
+                  int group, int grid_mode, uint8_t* codes_dev, float* scale_dev, float* zero_dev,
+                  float* P_hi_dev, float* P_lo_dev, double* resid_dev, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ADMMQ_H_ */

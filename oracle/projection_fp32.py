@@ -10,6 +10,9 @@ sequence of IEEE float32 operations, each rounded to nearest-even on its own
 (no fused multiply-add), with rint = round half to even.  Given the same
 float32 inputs the kernels must reproduce these outputs bit for bit.
 
+Signed zeros: every clamp and every zero point is followed by "+ 0", which
+turns -0 into +0, so results never depend on which zero a min/max returns.
+
 Grid semantics (our reading; the pages do not define the fit):
   minmax  mn = min(0, min y), mx = max(0, max y), s = (mx - mn) / L,
           z = rint(-mn / s); an all-zero group gets s = 1, z = 0.
@@ -39,7 +42,7 @@ def fit_minmax(yg: np.ndarray, L: int):
     s = _f(np.subtract(mx, mn, dtype=f32) / f32(L))
     zero_range = s == f32(0)
     s_safe = np.where(zero_range, f32(1), s).astype(f32)
-    z = np.rint(_f(np.negative(mn) / s_safe)).astype(f32)
+    z = _f(np.rint(_f(np.negative(mn) / s_safe)) + f32(0))
     z = np.where(zero_range, f32(0), z).astype(f32)
     return s_safe, z
 
@@ -66,7 +69,7 @@ def fit_lsq(yg: np.ndarray, wg: np.ndarray, s_prev: np.ndarray, z_prev: np.ndarr
     cov = _f(Sqy - _f(Sq * ym))
     ok = (var > 0) & (cov > 0)
     s1 = _f(cov / np.where(ok, var, f32(1)))
-    zc = np.clip(np.rint(_f(qm - _f(ym / np.where(ok, s1, f32(1))))), f32(0), f32(L)).astype(f32)
+    zc = _f(np.clip(np.rint(_f(qm - _f(ym / np.where(ok, s1, f32(1))))), f32(0), f32(L)) + f32(0))
     num = _f(Sqy - _f(zc * Sy))
     den = _f(_f(Sqq - _f(_f(f32(2) * zc) * Sq)) + _f(_f(zc * zc) * Sw))
     ok2 = (den > 0) & (num > 0)
@@ -79,7 +82,7 @@ def fit_lsq(yg: np.ndarray, wg: np.ndarray, s_prev: np.ndarray, z_prev: np.ndarr
 def round_to_grid(yg: np.ndarray, s: np.ndarray, z: np.ndarray, L: int) -> np.ndarray:
     """q = clamp(rint(y / s) + z, 0, L), as float32 integers."""
     r = np.rint(_f(_f(yg) / _f(s)[:, None]))
-    return np.clip(_f(r + _f(z)[:, None]), f32(0), f32(L)).astype(f32)
+    return _f(np.clip(_f(r + _f(z)[:, None]), f32(0), f32(L)) + f32(0))
 
 
 def dequantize(q: np.ndarray, s: np.ndarray, z: np.ndarray) -> np.ndarray:
@@ -99,10 +102,26 @@ def bf16_value(bits: np.ndarray) -> np.ndarray:
 
 
 def split_bf16(x: np.ndarray):
-    """x ~= hi + lo with hi = bf16(x), lo = bf16(x - hi) (the split-precision
-    operand planes of the eigenbasis GEMMs)."""
+    """x ~= hi + lo with hi = bf16(x), lo = bf16(x - hi); returns bit patterns."""
     hi = bf16_bits(x)
     lo = bf16_bits(_f(_f(x) - bf16_value(hi)))
+    return hi, lo
+
+
+def tf32_round(x: np.ndarray) -> np.ndarray:
+    """Round float32 to tf32 (10 explicit mantissa bits), nearest-even; the
+    result is a float32 whose 13 low mantissa bits are zero."""
+    b = _f(x).view(np.uint32).astype(np.uint64)
+    lsb = (b >> 13) & 1
+    r = (((b + 0xFFF + lsb) >> 13) << 13) & 0xFFFFFFFF
+    return r.astype(np.uint32).view(np.float32)
+
+
+def split_tf32(x: np.ndarray):
+    """x ~= hi + lo with hi = tf32(x), lo = tf32(x - hi): the operand planes of
+    the 3xTF32 eigenbasis GEMMs (float32 arrays)."""
+    hi = tf32_round(x)
+    lo = tf32_round(_f(_f(x) - hi))
     return hi, lo
 
 
@@ -124,7 +143,7 @@ def init_step(W_rows: np.ndarray, rsig: np.ndarray, bits: int, group: int):
     q = round_to_grid(yg, s, z, L)
     D = dequantize(q, s, z).reshape(m, d)
     Dt = _f(D * _f(rsig)[None, :])
-    hi, lo = split_bf16(Dt)
+    hi, lo = split_tf32(Dt)
     return dict(codes=q.reshape(m, d).astype(np.uint8), scale=s.reshape(m, d // group),
                 zero=z.reshape(m, d // group), P=Dt, P_hi=hi, P_lo=lo)
 
@@ -138,7 +157,7 @@ def epilogue_step(W_acc: np.ndarray, V: np.ndarray, sigma: np.ndarray, rsig: np.
       t  = W~ + V~          y  = sigma_i t
       grid (minmax | lsq | frozen) per group of `group` columns of one row
       q  = clamp(rint(y/s) + z, 0, L),  D = s (q - z),  D~ = D * rsig_i
-      V~' = t - D~          P  = D~ - V~'   (split into bf16 hi/lo planes)
+      V~' = t - D~          P  = D~ - V~'   (split into tf32 hi/lo planes)
     Residual sums (float64 here; the kernels sum in float32, compared with a
     tolerance): r2 = sum (W~ - D~)^2 and s2 = sum (D~ - D~_prev)^2 where
     D~_prev = s_prev (q_prev - z_prev) * rsig.
@@ -166,7 +185,7 @@ def epilogue_step(W_acc: np.ndarray, V: np.ndarray, sigma: np.ndarray, rsig: np.
     Dt = _f(D * _f(rsig)[None, :])
     V_new = _f(t - Dt)
     P = _f(Dt - V_new)
-    hi, lo = split_bf16(P)
+    hi, lo = split_tf32(P)
     qp = _rows_to_groups(_f(codes_prev), group)
     Dt_prev = _f(dequantize(qp, sp, zp).reshape(m, d) * _f(rsig)[None, :])
     r2 = float(np.sum((W_acc.astype(np.float64) - Dt) ** 2))

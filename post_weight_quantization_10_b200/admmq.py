@@ -1,0 +1,290 @@
+"""Thin Python binding of libadmmq.so (C ABI in include/admmq.h).
+
+Argument marshalling only: torch provides device memory and streams, every
+step of the solve runs in the library's CUDA kernels (and cuSOLVER for the
+one-time eigendecomposition).  A missing library raises; there is no
+fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+from .build import LIB
+
+OK = 0
+GRID_MINMAX, GRID_LSQ, GRID_FROZEN = 0, 1, 2
+GRID_MODES = {"minmax": GRID_MINMAX, "lsq": GRID_LSQ, "frozen": GRID_FROZEN}
+DTYPE_F32, DTYPE_BF16 = 0, 1
+BUFFERS = ["sigma", "rsig", "hdiag", "lambda", "V", "C0", "P_hi", "P_lo", "T_hi", "T_lo",
+           "E_hi", "E_lo", "Ht", "status"]
+
+
+class AdmmqError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+class _Params(ctypes.Structure):
+    _fields_ = [("bits", ctypes.c_int), ("group", ctypes.c_int), ("iters", ctypes.c_int),
+                ("rho0", ctypes.c_float), ("gamma", ctypes.c_float),
+                ("lambda_rel", ctypes.c_float), ("grid_mode", ctypes.c_int)]
+
+
+@dataclass
+class Params:
+    bits: int = 3
+    group: int = 128
+    iters: int = 100
+    rho0: float = 0.1
+    gamma: float = 1.05
+    lambda_rel: float = 0.01
+    grid: str = "minmax"
+
+    def c(self) -> _Params:
+        return _Params(self.bits, self.group, self.iters, self.rho0, self.gamma, self.lambda_rel,
+                       GRID_MODES[self.grid])
+
+
+_lib = None
+_vp, _i, _i64, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+
+
+def _preload_solver_runtime():
+    """Use the cuSOLVER build that matches torch's cuBLAS when torch ships one,
+    so one process never mixes two cuBLAS versions."""
+    try:
+        import nvidia.cusolver  # type: ignore
+        for base in nvidia.cusolver.__path__:
+            p = os.path.join(base, "lib", "libcusolver.so.11")
+            if os.path.exists(p):
+                ctypes.CDLL(p, mode=ctypes.RTLD_GLOBAL)
+                return
+    except Exception:
+        pass
+
+
+def lib():
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB):
+        raise RuntimeError(f"{LIB} is missing: build it with "
+                           "`python -m post_weight_quantization_10_b200.build`")
+    torch.cuda.init() if torch.cuda.is_available() else None
+    _preload_solver_runtime()
+    L = ctypes.CDLL(LIB)
+    sig = {
+        "admmq_status_string": (ctypes.c_char_p, [_i]),
+        "admmq_version": (_i, []),
+        "admmq_launch_count": (ctypes.c_int64, []),
+        "admmq_gram_workspace_bytes": (_sz, [_i64, _i]),
+        "admmq_build_hessian": (_i, [_vp, _i64, _i, _vp, _i, _vp, _sz, _vp]),
+        "admmq_workspace_bytes": (_sz, [_i, _i, ctypes.POINTER(_Params)]),
+        "admmq_create": (_i, [ctypes.POINTER(_vp), _i, _i, ctypes.POINTER(_Params), _vp, _sz]),
+        "admmq_destroy": (None, [_vp]),
+        "admmq_prepare": (_i, [_vp, _vp, _vp, _i, _vp]),
+        "admmq_eigh": (_i, [_vp, _vp]),
+        "admmq_setup": (_i, [ctypes.POINTER(_vp), _vp, _vp, _i, _i, _i, ctypes.POINTER(_Params),
+                             _vp, _sz, _vp]),
+        "admmq_init": (_i, [_vp, _vp, _vp, _vp, _vp]),
+        "admmq_iterate": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp]),
+        "admmq_finish": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+        "admmq_solve": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+        "admmq_pack": (_i, [_vp, _i, _i, _i, _vp, _vp]),
+        "admmq_get_buffer": (_i, [_vp, _i, ctypes.POINTER(_vp), ctypes.POINTER(_sz)]),
+        "admmq_debug_dump_wtilde": (_i, [_vp, _vp]),
+        "admmq_set_timing": (_i, [_vp, _i]),
+        "admmq_get_timing": (_i, [_vp, ctypes.POINTER(ctypes.c_double),
+                                  ctypes.POINTER(ctypes.c_int)]),
+        "admmq_project": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp,
+                               _vp, _vp, _vp]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = L
+    return L
+
+
+def launch_count() -> int:
+    """Kernels launched by libadmmq.so in this process."""
+    return int(lib().admmq_launch_count())
+
+
+def status_string(s: int) -> str:
+    return lib().admmq_status_string(s).decode()
+
+
+def _check(rc: int, where: str):
+    if rc != OK:
+        raise AdmmqError(rc, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+# ------------------------------------------------------------------ Hessian
+
+
+def gram_workspace_bytes(n: int, d_in: int) -> int:
+    return int(lib().admmq_gram_workspace_bytes(n, d_in))
+
+
+def build_hessian(X: torch.Tensor, H: torch.Tensor | None = None, accumulate: bool = False,
+                  workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """H = X^T X (fp32, both triangles) from bf16 activations X [n][d_in]."""
+    assert X.is_cuda and X.dtype == torch.bfloat16 and X.dim() == 2 and X.is_contiguous()
+    n, d = X.shape
+    if H is None:
+        H = torch.empty((d, d), dtype=torch.float32, device=X.device)
+    need = gram_workspace_bytes(n, d)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
+    _check(lib().admmq_build_hessian(_ptr(X), n, d, _ptr(H), int(accumulate), _ptr(workspace),
+                                     workspace.numel(), _stream(stream)), "admmq_build_hessian")
+    return H
+
+
+# ------------------------------------------------------------------- solver
+
+
+class Solver:
+    """One layer solve: owns the workspace tensor and the C context."""
+
+    def __init__(self, d_in: int, d_out: int, params: Params, device="cuda"):
+        self.d_in, self.d_out, self.params = d_in, d_out, params
+        self._cp = params.c()
+        need = int(lib().admmq_workspace_bytes(d_in, d_out, ctypes.byref(self._cp)))
+        if need == 0:
+            raise AdmmqError(-1, "admmq_workspace_bytes")
+        self.workspace = torch.empty(need, dtype=torch.uint8, device=device)
+        self._ctx = ctypes.c_void_p()
+        _check(lib().admmq_create(ctypes.byref(self._ctx), d_in, d_out, ctypes.byref(self._cp),
+                                  _ptr(self.workspace), need), "admmq_create")
+        self._W_hat = None
+        ng = d_in // params.group
+        self.codes = torch.empty((d_out, d_in), dtype=torch.uint8, device=device)
+        self.scale = torch.empty((d_out, ng), dtype=torch.float32, device=device)
+        self.zero = torch.empty((d_out, ng), dtype=torch.float32, device=device)
+        self.resid = torch.zeros((max(params.iters, 1), 2), dtype=torch.float64, device=device)
+        self.objective = torch.zeros(1, dtype=torch.float64, device=device)
+
+    def close(self):
+        if self._ctx:
+            lib().admmq_destroy(self._ctx)
+            self._ctx = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def prepare(self, G: torch.Tensor, W_hat: torch.Tensor, stream=None):
+        assert G.dtype == torch.float32 and G.shape == (self.d_in, self.d_in) and G.is_contiguous()
+        assert W_hat.shape == (self.d_out, self.d_in) and W_hat.is_contiguous()
+        dt = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16}[W_hat.dtype]
+        self._W_hat = W_hat  # the library reads it again in finish()
+        _check(lib().admmq_prepare(self._ctx, _ptr(G), _ptr(W_hat), dt, _stream(stream)),
+               "admmq_prepare")
+
+    def eigh(self, stream=None):
+        _check(lib().admmq_eigh(self._ctx, _stream(stream)), "admmq_eigh")
+
+    def init(self, stream=None):
+        _check(lib().admmq_init(self._ctx, _ptr(self.codes), _ptr(self.scale), _ptr(self.zero),
+                                _stream(stream)), "admmq_init")
+
+    def iterate(self, t0: int, count: int, stream=None):
+        _check(lib().admmq_iterate(self._ctx, t0, count, _ptr(self.codes), _ptr(self.scale),
+                                   _ptr(self.zero), _stream(stream)), "admmq_iterate")
+
+    def finish(self, resid=True, objective=True, stream=None):
+        _check(lib().admmq_finish(self._ctx, _ptr(self.codes), _ptr(self.scale), _ptr(self.zero),
+                                  _ptr(self.resid) if resid else None,
+                                  _ptr(self.objective) if objective else None, _stream(stream)),
+               "admmq_finish")
+
+    def solve(self, stream=None):
+        _check(lib().admmq_solve(self._ctx, _ptr(self.codes), _ptr(self.scale), _ptr(self.zero),
+                                 _ptr(self.resid), _ptr(self.objective), _stream(stream)),
+               "admmq_solve")
+
+    def buffer(self, name: str) -> torch.Tensor:
+        """A torch view of a workspace buffer (see include/admmq.h for layouts)."""
+        which = BUFFERS.index(name)
+        p, nb = ctypes.c_void_p(), ctypes.c_size_t()
+        _check(lib().admmq_get_buffer(self._ctx, which, ctypes.byref(p), ctypes.byref(nb)),
+               "admmq_get_buffer")
+        off = p.value - self.workspace.data_ptr()
+        raw = self.workspace[off:off + nb.value]
+        d, m = self.d_in, self.d_out
+        if name in ("sigma", "rsig", "hdiag", "lambda"):
+            return raw.view(torch.float32)
+        if name in ("V", "C0"):
+            return raw.view(torch.float32).view(m, d)
+        if name in ("P_hi", "P_lo", "T_hi", "T_lo"):
+            return raw.view(torch.float32).view(m, d)
+        if name in ("E_hi", "E_lo"):
+            return raw.view(torch.float32).view(d, d)
+        if name == "Ht":
+            return raw.view(torch.float64).view(d, d)
+        return raw.view(torch.int32)
+
+    def dump_wtilde(self, out: torch.Tensor | None):
+        _check(lib().admmq_debug_dump_wtilde(self._ctx, _ptr(out)), "admmq_debug_dump_wtilde")
+
+    def set_timing(self, enable: bool):
+        _check(lib().admmq_set_timing(self._ctx, int(enable)), "admmq_set_timing")
+
+    def get_timing(self):
+        ms = (ctypes.c_double * 2)()
+        n = (ctypes.c_int * 2)()
+        _check(lib().admmq_get_timing(self._ctx, ms, n), "admmq_get_timing")
+        return [ms[0], ms[1]], [n[0], n[1]]
+
+
+# --------------------------------------------------------------- pack etc.
+
+
+def pack(codes: torch.Tensor, bits: int, out: torch.Tensor | None = None, stream=None):
+    m, d = codes.shape
+    if out is None:
+        out = torch.empty((m, d * bits // 32), dtype=torch.int32, device=codes.device)
+    _check(lib().admmq_pack(_ptr(codes), d, m, bits, _ptr(out), _stream(stream)), "admmq_pack")
+    return out
+
+
+def project(wtilde, V, sigma, rsig, hdiag, bits, group, grid, codes, scale, zero, P_hi, P_lo,
+            resid=None, stream=None):
+    m, d = wtilde.shape
+    if resid is None:
+        resid = torch.zeros(2, dtype=torch.float64, device=wtilde.device)
+    _check(lib().admmq_project(_ptr(wtilde), _ptr(V), _ptr(sigma), _ptr(rsig), _ptr(hdiag), d, m,
+                               bits, group, GRID_MODES[grid], _ptr(codes), _ptr(scale),
+                               _ptr(zero), _ptr(P_hi), _ptr(P_lo), _ptr(resid), _stream(stream)),
+           "admmq_project")
+    return resid
+
+
+def solve_layer(X: torch.Tensor, W_hat: torch.Tensor, params: Params, stream=None) -> Solver:
+    """Gram -> setup -> solve for one layer; the Solver holds codes/scale/zero,
+    the residual history and the objective."""
+    H = build_hessian(X, stream=stream)
+    s = Solver(X.shape[1], W_hat.shape[0], params, device=X.device)
+    s.prepare(H, W_hat, stream)
+    s.eigh(stream)
+    s.solve(stream)
+    return s

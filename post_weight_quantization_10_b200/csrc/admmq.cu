@@ -1,0 +1,1046 @@
+// admmq.cu -- the ADMM-Q layer solve for B200 (sm_100a): setup kernels,
+// packing, reductions, the tcgen05 GEMM instantiations and the C ABI
+// declared in include/admmq.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <cusolverDn.h>
+
+#include <math.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <vector>
+
+#include "../../include/admmq.h"
+#include "kernels.cuh"
+
+using namespace admmq;
+
+namespace {
+
+constexpr int kBM = 128;
+unsigned long long g_launches = 0;  // kernels launched by this library
+inline void count_launch() { __atomic_fetch_add(&g_launches, 1ull, __ATOMIC_RELAXED); }
+// X^T X: bf16, both operands MN-major (X is token-major).
+using GramCfg = GemmCfg<KIND_BF16, 256, 1, true, true, 4>;
+// Eigenbasis GEMMs: 3xTF32 split precision, K-major operands.
+using EigCfg = GemmCfg<KIND_TF32, 128, 2, false, false, 3>;
+
+// Setup status words (ws status[1]).
+enum { SETUP_OK = 0, SETUP_NONFINITE = 1, SETUP_NOT_PD = 2 };
+
+// ------------------------------------------------------------------ kernels
+
+__global__ void k_diag_stats(const float* __restrict__ G, int d, float lambda_rel,
+                             double* __restrict__ lam_out, double* __restrict__ sig64,
+                             float* __restrict__ hdiag, float* __restrict__ sigma,
+                             float* __restrict__ rsig, int* __restrict__ status) {
+  __shared__ double red[1024];
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) acc += (double)G[(long long)i * d + i];
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  for (int s = blockDim.x / 2; s > 0; s >>= 1) {
+    if ((int)threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
+    __syncthreads();
+  }
+  const double lam = (double)lambda_rel * red[0] / (double)d;
+  if (threadIdx.x == 0) *lam_out = lam;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    const double h = (double)G[(long long)i * d + i] + lam;
+    if (!isfinite(h)) {
+      atomicExch(&status[1], SETUP_NONFINITE);
+    } else if (h <= 0.0) {
+      atomicExch(&status[1], SETUP_NOT_PD);
+    }
+    const double sg = 1.0 / sqrt(h);
+    sig64[i] = sg;
+    hdiag[i] = (float)h;
+    sigma[i] = (float)sg;
+    rsig[i] = (float)sqrt(h);
+  }
+}
+
+// H~ = Sigma (G + lambda I) Sigma in float64.
+__global__ void k_scale_hessian(const float* __restrict__ G, int d, const double* __restrict__ lam,
+                                const double* __restrict__ sig64, double* __restrict__ Ht) {
+  const long long total = (long long)d * d;
+  const double l = *lam;
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int i = (int)(idx / d), j = (int)(idx - (long long)i * d);
+    const double h = (double)G[idx] + (i == j ? l : 0.0);
+    Ht[idx] = sig64[i] * h * sig64[j];
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ float load_w(const T* p, long long i);
+template <>
+__device__ __forceinline__ float load_w<float>(const float* p, long long i) {
+  return p[i];
+}
+template <>
+__device__ __forceinline__ float load_w<__nv_bfloat16>(const __nv_bfloat16* p, long long i) {
+  return __bfloat162float(p[i]);
+}
+
+// W^~ = Sigma^-1 W_hat (rows = output channels), split into tf32 hi/lo planes.
+template <typename T>
+__global__ void k_scale_weights(const T* __restrict__ W, const float* __restrict__ rsig, int d,
+                                long long total, float* __restrict__ hi, float* __restrict__ lo) {
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int i = (int)(idx % d);
+    const float w = __fmul_rn(load_w<T>(W, idx), rsig[i]);
+    float h, l;
+    split2(w, h, l);
+    hi[idx] = h;
+    lo[idx] = l;
+  }
+}
+
+// Eigenvector buffer (row k = k-th eigenvector, from the column-major solver
+// output) -> tf32 hi/lo planes of E = Q^T [k][i] and of Q [i][k].
+__global__ void k_split_eigvecs(const double* __restrict__ Evec, int d, float* __restrict__ e_hi,
+                                float* __restrict__ e_lo, float* __restrict__ q_hi,
+                                float* __restrict__ q_lo) {
+  __shared__ float th[32][33], tl[32][33];
+  const int k0 = blockIdx.y * 32, i0 = blockIdx.x * 32;
+  for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+    const int k = k0 + r, i = i0 + threadIdx.x;
+    float h = 0.f, l = 0.f;
+    if (k < d && i < d) {
+      const double e = Evec[(long long)k * d + i];
+      h = tf32_rne((float)e);
+      l = tf32_rne((float)(e - (double)h));
+      e_hi[(long long)k * d + i] = h;
+      e_lo[(long long)k * d + i] = l;
+    }
+    th[r][threadIdx.x] = h;
+    tl[r][threadIdx.x] = l;
+  }
+  __syncthreads();
+  for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+    const int i = i0 + r, k = k0 + threadIdx.x;
+    if (k < d && i < d) {
+      q_hi[(long long)i * d + k] = th[threadIdx.x][r];
+      q_lo[(long long)i * d + k] = tl[threadIdx.x][r];
+    }
+  }
+}
+
+__global__ void k_eigvals(const double* __restrict__ ev, int d, float* __restrict__ lam32,
+                          int* __restrict__ status) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < d; i += gridDim.x * blockDim.x) {
+    const double v = ev[i];
+    if (!isfinite(v)) atomicExch(&status[2], 1);
+    lam32[i] = (float)v;
+  }
+}
+
+// RTN start: D_0 = min/max-grid rounding of W_hat, V~ = 0, P = D~_0.
+template <typename T>
+__global__ void k_init_rtn(const T* __restrict__ W, const float* __restrict__ rsig, int m, int d,
+                           int g, int L, uint8_t* __restrict__ codes, float* __restrict__ scale,
+                           float* __restrict__ zero, float* __restrict__ V,
+                           float* __restrict__ p_hi, float* __restrict__ p_lo) {
+  const int ngr = d / g;
+  const long long total = (long long)m * ngr;
+  const float Lf = (float)L;
+  for (long long gi = blockIdx.x * (long long)blockDim.x + threadIdx.x; gi < total;
+       gi += (long long)gridDim.x * blockDim.x) {
+    const long long row = gi / ngr;
+    const int col0 = (int)(gi - row * ngr) * g;
+    const long long base = row * d + col0;
+    float mn = 0.f, mx = 0.f;
+    for (int e = 0; e < g; ++e) {
+      const float y = load_w<T>(W, base + e);
+      mn = fminf(mn, y);
+      mx = fmaxf(mx, y);
+    }
+    float s = __fdiv_rn(__fsub_rn(mx, mn), Lf), z;
+    if (s == 0.f) {
+      s = 1.f;
+      z = 0.f;
+    } else {
+      z = __fadd_rn(rintf(__fdiv_rn(-mn, s)), 0.f);
+    }
+    for (int e = 0; e < g; ++e) {
+      const float y = load_w<T>(W, base + e);
+      const float q = clampq(__fadd_rn(rintf(__fdiv_rn(y, s)), z), Lf);
+      const float D = __fmul_rn(s, __fsub_rn(q, z));
+      const float dt = __fmul_rn(D, rsig[col0 + e]);
+      float h, l;
+      split2(dt, h, l);
+      codes[base + e] = (uint8_t)q;
+      V[base + e] = 0.f;
+      p_hi[base + e] = h;
+      p_lo[base + e] = l;
+    }
+    scale[gi] = s;
+    zero[gi] = z;
+  }
+}
+
+// Delta~ = D~ - W^~ (scaled coordinates) as tf32 planes, for the objective.
+template <typename T>
+__global__ void k_delta_planes(const T* __restrict__ W, const uint8_t* __restrict__ codes,
+                               const float* __restrict__ scale, const float* __restrict__ zero,
+                               const float* __restrict__ rsig, int d, int g, long long total,
+                               float* __restrict__ hi, float* __restrict__ lo) {
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const long long row = idx / d;
+    const int i = (int)(idx - row * d);
+    const long long gi = row * (d / g) + i / g;
+    const float D = __fmul_rn(scale[gi], __fsub_rn((float)codes[idx], zero[gi]));
+    const float dt = __fmul_rn(D, rsig[i]);
+    const float wt = __fmul_rn(load_w<T>(W, idx), rsig[i]);
+    float h, l;
+    split2(__fsub_rn(dt, wt), h, l);
+    hi[idx] = h;
+    lo[idx] = l;
+  }
+}
+
+// Fixed-order float64 reduction of per-tile partials.
+__global__ void k_reduce_objective(const float* __restrict__ part, int count,
+                                   double* __restrict__ out) {
+  __shared__ double red[256];
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < count; i += blockDim.x) acc += (double)part[i];
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  for (int s = blockDim.x / 2; s > 0; s >>= 1) {
+    if ((int)threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) out[0] = 0.5 * red[0];
+}
+
+__global__ void k_reduce_resid(const float* __restrict__ part, int per_iter, double rho0,
+                               double gamma, double* __restrict__ out) {
+  __shared__ double r2s[256], s2s[256];
+  const int t = blockIdx.x;
+  const float* p = part + (long long)t * per_iter * 2;
+  double a = 0.0, b = 0.0;
+  for (int i = threadIdx.x; i < per_iter; i += blockDim.x) {
+    a += (double)p[2 * i];
+    b += (double)p[2 * i + 1];
+  }
+  r2s[threadIdx.x] = a;
+  s2s[threadIdx.x] = b;
+  __syncthreads();
+  for (int s = blockDim.x / 2; s > 0; s >>= 1) {
+    if ((int)threadIdx.x < s) {
+      r2s[threadIdx.x] += r2s[threadIdx.x + s];
+      s2s[threadIdx.x] += s2s[threadIdx.x + s];
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    out[2 * t] = sqrt(r2s[0]);
+    out[2 * t + 1] = rho0 * pow(gamma, (double)t) * sqrt(s2s[0]);
+  }
+}
+
+// H = sum of the k-split partials over the upper triangle, mirrored; diagonal
+// 32x32 blocks take every value from their upper half so H is symmetric.
+__global__ void k_gram_finalize(const float* __restrict__ part, int splits, long long split_stride,
+                                int d, float* __restrict__ H, int accumulate,
+                                const int* __restrict__ status) {
+  const int I = blockIdx.y, J = blockIdx.x;
+  if (I > J) return;
+  __shared__ float tile[32][33];
+  const bool bad = status[0] != 0;
+  for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+    const int i = I * 32 + r, j = J * 32 + threadIdx.x;
+    float v = 0.f;
+    if (i < d && j < d) {
+      const long long off = (long long)i * d + j;
+      for (int s = 0; s < splits; ++s) v += part[s * split_stride + off];
+    }
+    tile[r][threadIdx.x] = v;
+  }
+  __syncthreads();
+  for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+    const int c = threadIdx.x;
+    // upper block (I, J): H[I*32 + r][J*32 + c]
+    {
+      const int i = I * 32 + r, j = J * 32 + c;
+      if (i < d && j < d) {
+        float v = (I == J && r > c) ? tile[c][r] : tile[r][c];
+        if (bad && i == j) v = __int_as_float(0x7fc00000);
+        const long long off = (long long)i * d + j;
+        H[off] = accumulate ? H[off] + v : v;
+      }
+    }
+    if (I != J) {  // mirrored block (J, I): H[J*32 + r][I*32 + c] = tile[c][r]
+      const int i = J * 32 + r, j = I * 32 + c;
+      if (i < d && j < d) {
+        const long long off = (long long)i * d + j;
+        H[off] = accumulate ? H[off] + tile[c][r] : tile[c][r];
+      }
+    }
+  }
+}
+
+// Pack CH codes per thread into CH*BITS/32 little-endian words.
+template <int BITS, int CH>
+__global__ void k_pack(const uint8_t* __restrict__ codes, long long chunks, int chunks_per_row,
+                       int d, uint32_t* __restrict__ out) {
+  constexpr int WPC = 32 * BITS / 32;  // words per 32 codes
+  constexpr uint32_t MASK = (1u << BITS) - 1u;
+  const long long wpr = (long long)d * BITS / 32;
+  for (long long ch = blockIdx.x * (long long)blockDim.x + threadIdx.x; ch < chunks;
+       ch += (long long)gridDim.x * blockDim.x) {
+    const long long row = ch / chunks_per_row;
+    const int c = (int)(ch - row * chunks_per_row);
+    const uint8_t* src = codes + row * d + (long long)c * CH;
+    uint32_t* dst = out + row * wpr + (long long)c * (CH / 32) * WPC;
+#pragma unroll
+    for (int sub = 0; sub < CH / 32; ++sub) {
+      uint32_t in[8];
+      const uint4 a = reinterpret_cast<const uint4*>(src + sub * 32)[0];
+      const uint4 b = reinterpret_cast<const uint4*>(src + sub * 32)[1];
+      in[0] = a.x; in[1] = a.y; in[2] = a.z; in[3] = a.w;
+      in[4] = b.x; in[5] = b.y; in[6] = b.z; in[7] = b.w;
+      uint32_t w[WPC];
+#pragma unroll
+      for (int k = 0; k < WPC; ++k) w[k] = 0u;
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        const uint32_t v = (in[k >> 2] >> (8 * (k & 3))) & MASK;
+        const int pos = k * BITS;
+        w[pos >> 5] |= v << (pos & 31);
+        if ((pos & 31) + BITS > 32) w[(pos >> 5) + 1] |= v >> (32 - (pos & 31));
+      }
+      uint32_t* o = dst + sub * WPC;
+      if (WPC % 4 == 0) {
+#pragma unroll
+        for (int k = 0; k < WPC; k += 4) reinterpret_cast<uint4*>(o)[k / 4] = make_uint4(w[k], w[k + 1], w[k + 2], w[k + 3]);
+      } else if (WPC % 2 == 0) {
+#pragma unroll
+        for (int k = 0; k < WPC; k += 2) reinterpret_cast<uint2*>(o)[k / 2] = make_uint2(w[k], w[k + 1]);
+      } else {
+#pragma unroll
+        for (int k = 0; k < WPC; ++k) o[k] = w[k];
+      }
+    }
+  }
+}
+
+// Standalone projection: one thread per (row, group), W~ read from memory.
+template <int MODE>
+__global__ void k_project(const float* __restrict__ wt, float* V, const float* __restrict__ sig,
+                          const float* __restrict__ rsig, const float* __restrict__ hd, int m, int d,
+                          int g, int L, uint8_t* codes, float* scale, float* zero, float* p_hi,
+                          float* p_lo, double* resid) {
+  const int row = blockIdx.x * blockDim.x + threadIdx.x;
+  const int grp = blockIdx.y;
+  const bool valid = row < m;
+  const int col0 = grp * g;
+  const long long off = (long long)(valid ? row : 0) * d + col0;
+  const long long goff = (long long)(valid ? row : 0) * (d / g) + grp;
+  ProjRow r;
+  r.V = V + off;
+  r.sig = sig + col0;
+  r.rsig = rsig + col0;
+  r.hd = hd + col0;
+  r.codes = codes + off;
+  r.phi = p_hi + off;
+  r.plo = p_lo + off;
+  r.scale = scale + goff;
+  r.zero = zero + goff;
+  r.wdump = nullptr;
+  r.valid = valid;
+  auto loadw = [&](int c, float (&w)[32]) {
+#pragma unroll
+    for (int k = 0; k < 32; k += 4) {
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (valid) v = *reinterpret_cast<const float4*>(wt + off + c + k);
+      w[k] = v.x; w[k + 1] = v.y; w[k + 2] = v.z; w[k + 3] = v.w;
+    }
+  };
+  float r2 = 0.f, s2 = 0.f;
+  project_group<MODE>(loadw, r, g, L, r2, s2);
+  r2 = warp_sum(r2);
+  s2 = warp_sum(s2);
+  if ((threadIdx.x & 31) == 0) {
+    atomicAdd(&resid[0], (double)r2);
+    atomicAdd(&resid[1], (double)s2);
+  }
+}
+
+// ------------------------------------------------------------- host utils
+
+int num_sms() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 1;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// Row-major [outer][inner] tensor of bf16 or fp32, box {128 bytes, box_outer},
+// 128-byte swizzle, out-of-bounds elements read as zero.
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_outer,
+              bool fp32) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const uint32_t es = fp32 ? 4 : 2;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * es};
+  cuuint32_t box[2] = {128 / es, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+GemmGeom make_geom(int M, int N, long long K, int BN, int BK, int splits, bool triangle,
+                   int* status) {
+  GemmGeom g;
+  g.M = M;
+  g.N = N;
+  g.K = (int)K;
+  g.tiles_m = cdiv(M, kBM);
+  g.tiles_n = cdiv(N, BN);
+  g.kblocks = cdiv(K, BK);
+  g.splits = splits;
+  g.triangle = triangle ? 1 : 0;
+  if (!triangle) {
+    g.tiles = g.tiles_m * g.tiles_n;
+  } else {
+    int t = 0;
+    for (int tn = 0; tn < g.tiles_n; ++tn) {
+      int cnt = cdiv((long long)(tn + 1) * BN, kBM);
+      t += cnt < g.tiles_m ? cnt : g.tiles_m;
+    }
+    g.tiles = t;
+  }
+  g.units = g.tiles * splits;
+  g.status = status;
+  return g;
+}
+
+template <class Cfg, class Epi>
+cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0,
+                        const CUtensorMap& b1, const GemmGeom& g, const typename Epi::Params& ep,
+                        cudaStream_t st) {
+  auto kern = k_gemm<Cfg, Epi>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+  if (e != cudaSuccess) return e;
+  int grid = g.units < num_sms() ? g.units : num_sms();
+  if (grid <= 0) return cudaSuccess;
+  count_launch();
+  kern<<<grid, 192, Cfg::SMEM, st>>>(a0, a1, b0, b1, g, ep);
+  return cudaGetLastError();
+}
+
+int device_ok() {
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ADMMQ_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return ADMMQ_ERR_CUDA;
+  return major == 10 ? ADMMQ_OK : ADMMQ_ERR_UNSUPPORTED;
+}
+
+int grid_for(long long work, int per_block = 256) {
+  long long b = (work + per_block - 1) / per_block;
+  long long cap = (long long)num_sms() * 8;
+  if (b > cap) b = cap;
+  return b < 1 ? 1 : (int)b;
+}
+
+// Gram k-split count: the smallest split (1..8) whose units fill the SMs best.
+int gram_splits(long long n, int d, int nsm) {
+  GemmGeom g = make_geom(d, d, n, GramCfg::BN, GramCfg::BK, 1, true, nullptr);
+  int best = 1;
+  double best_eff = -1.0;
+  for (int s = 1; s <= 8; ++s) {
+    if (s > g.kblocks) break;
+    long long units = (long long)g.tiles * s;
+    long long waves = (units + nsm - 1) / nsm;
+    double eff = (double)units / (double)(waves * nsm);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = s;
+    }
+  }
+  return best;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+}  // namespace
+
+// =================================================================== C ABI
+
+struct admmq_ctx {
+  int d, m, L, dev;
+  admmq_params p;
+  uint8_t* ws;
+  size_t ws_bytes;
+  int* status;          // [4]
+  double* lam64;        // damping lambda
+  double* sig64;        // [d]
+  float *hdiag, *sigma, *rsig, *lam32;
+  double* Ht;           // [d][d]  H~, then eigenvectors (row k = eigenvector k)
+  double* evals;        // [d]
+  double* work;
+  int lwork;
+  int* devinfo;
+  float *E_hi, *E_lo, *Q_hi, *Q_lo;          // [d][d] tf32 planes
+  float *Wt_hi, *Wt_lo, *P_hi, *P_lo, *T_hi, *T_lo;     // [m][d] tf32 planes
+  float *C0, *V;                               // [m][d]
+  float* resid_part;    // [iters][tiles][4][2]
+  float* obj_part;      // [tiles][4]
+  int tiles_eig;
+  const void* W_hat;
+  int w_dtype;
+  float* wdump;
+  cusolverDnHandle_t solver;
+  CUtensorMap mWt[2], mP[2], mT[2], mE[2], mQ[2];
+  bool timing;
+  std::vector<cudaEvent_t> ev;   // triples per iteration
+  bool prepared, eig_done, inited;
+};
+
+namespace {
+
+struct Layout {
+  size_t status, lam64, sig64, hdiag, sigma, rsig, lam32, Ht, evals, work, devinfo;
+  size_t E_hi, E_lo, Q_hi, Q_lo, Wt_hi, Wt_lo, P_hi, P_lo, T_hi, T_lo, C0, V;
+  size_t resid_part, obj_part, total;
+};
+
+Layout make_layout(int d, int m, int iters, int lwork) {
+  Layout L;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = o;
+    o = align256(o + bytes);
+    return at;
+  };
+  const size_t dd = (size_t)d * d, md = (size_t)m * d;
+  const int tiles = cdiv(m, kBM) * cdiv(d, EigCfg::BN);
+  L.status = take(16);
+  L.lam64 = take(8);
+  L.sig64 = take(8 * (size_t)d);
+  L.hdiag = take(4 * (size_t)d);
+  L.sigma = take(4 * (size_t)d);
+  L.rsig = take(4 * (size_t)d);
+  L.lam32 = take(4 * (size_t)d);
+  L.Ht = take(8 * dd);
+  L.evals = take(8 * (size_t)d);
+  L.work = take(8 * (size_t)(lwork > 0 ? lwork : 1));
+  L.devinfo = take(16);
+  L.E_hi = take(4 * dd);
+  L.E_lo = take(4 * dd);
+  L.Q_hi = take(4 * dd);
+  L.Q_lo = take(4 * dd);
+  L.Wt_hi = take(4 * md);
+  L.Wt_lo = take(4 * md);
+  L.P_hi = take(4 * md);
+  L.P_lo = take(4 * md);
+  L.T_hi = take(4 * md);
+  L.T_lo = take(4 * md);
+  L.C0 = take(4 * md);
+  L.V = take(4 * md);
+  L.resid_part = take(4 * (size_t)(iters > 0 ? iters : 1) * tiles * 8);
+  L.obj_part = take(4 * (size_t)tiles * 4);
+  L.total = o;
+  return L;
+}
+
+int check_params(int d, int m, const admmq_params* p) {
+  if (!p) return ADMMQ_ERR_INVALID_ARG;
+  if (d <= 0 || m <= 0 || d % 32 != 0) return ADMMQ_ERR_INVALID_ARG;
+  if (!(p->group == 32 || p->group == 64 || p->group == 128) || d % p->group != 0)
+    return ADMMQ_ERR_INVALID_ARG;
+  if (p->bits < 1 || p->bits > 8 || p->iters < 0) return ADMMQ_ERR_INVALID_ARG;
+  if (!(p->rho0 > 0.f) || !(p->gamma > 0.f) || !(p->lambda_rel >= 0.f)) return ADMMQ_ERR_INVALID_ARG;
+  if (p->grid_mode < ADMMQ_GRID_MINMAX || p->grid_mode > ADMMQ_GRID_FROZEN)
+    return ADMMQ_ERR_INVALID_ARG;
+  return ADMMQ_OK;
+}
+
+int syevd_lwork(int d) {
+  static cusolverDnHandle_t h = nullptr;
+  if (!h && cusolverDnCreate(&h) != CUSOLVER_STATUS_SUCCESS) return -1;
+  int lwork = 0;
+  if (cusolverDnDsyevd_bufferSize(h, CUSOLVER_EIG_MODE_VECTOR, CUBLAS_FILL_MODE_UPPER, d, nullptr,
+                                  d, nullptr, &lwork) != CUSOLVER_STATUS_SUCCESS)
+    return -1;
+  return lwork;
+}
+
+#define CK(x)                                      \
+  do {                                             \
+    if ((x) != cudaSuccess) return ADMMQ_ERR_CUDA; \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char* admmq_status_string(int s) {
+  switch (s) {
+    case ADMMQ_OK: return "ok";
+    case ADMMQ_ERR_INVALID_ARG: return "invalid argument";
+    case ADMMQ_ERR_CUDA: return "CUDA error";
+    case ADMMQ_ERR_EIG: return "eigensolver failed";
+    case ADMMQ_ERR_NOT_PD: return "Hessian diagonal not positive";
+    case ADMMQ_ERR_NONFINITE: return "non-finite value in the Hessian or its eigenvalues";
+    case ADMMQ_ERR_TIMEOUT: return "kernel pipeline wait timed out";
+    case ADMMQ_ERR_WORKSPACE: return "workspace too small";
+    case ADMMQ_ERR_UNSUPPORTED: return "unsupported device or shape";
+    default: return "unknown status";
+  }
+}
+
+int admmq_version(void) { return 100; }
+
+int64_t admmq_launch_count(void) { return (int64_t)__atomic_load_n(&g_launches, __ATOMIC_RELAXED); }
+
+size_t admmq_gram_workspace_bytes(int64_t n, int d_in) {
+  if (d_in <= 0 || d_in % 32 != 0 || n < 0) return 0;
+  const int s = gram_splits(n > 0 ? n : 1, d_in, num_sms());
+  return 256 + (size_t)s * d_in * d_in * 4;
+}
+
+int admmq_build_hessian(const void* X, int64_t n, int d, float* H, int accumulate, void* ws,
+                        size_t ws_bytes, void* stream) {
+  if ((!X && n > 0) || !H || d <= 0 || d % 32 != 0 || n < 0 || !ws) return ADMMQ_ERR_INVALID_ARG;
+  if (((uintptr_t)X & 15) != 0) return ADMMQ_ERR_INVALID_ARG;
+  int rc = device_ok();
+  if (rc) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t dd4 = (size_t)d * d * 4;
+  if (ws_bytes < 256 + dd4) return ADMMQ_ERR_WORKSPACE;
+  if (n == 0) {
+    if (!accumulate) CK(cudaMemsetAsync(H, 0, dd4, st));
+    return ADMMQ_OK;
+  }
+  int splits = gram_splits(n, d, num_sms());
+  while (splits > 1 && ws_bytes < 256 + (size_t)splits * dd4) --splits;
+  int* status = (int*)ws;
+  float* part = (float*)((uint8_t*)ws + 256);
+  CK(cudaMemsetAsync(status, 0, 16, st));
+  CUtensorMap mx;
+  if (!make_map(&mx, X, (uint64_t)d, (uint64_t)n, GramCfg::BK, false)) return ADMMQ_ERR_CUDA;
+  GemmGeom g = make_geom(d, d, n, GramCfg::BN, GramCfg::BK, splits, true, status);
+  EpiGramPartial<GramCfg::BN>::Params ep{part, (long long)d * d, d};
+  CK((launch_gemm<GramCfg, EpiGramPartial<GramCfg::BN>>(mx, mx, mx, mx, g, ep, st)));
+  const int nb = d / 32;
+  count_launch(), k_gram_finalize<<<dim3(nb, nb), dim3(32, 8), 0, st>>>(part, splits, (long long)d * d, d, H,
+                                                        accumulate, status);
+  CK(cudaGetLastError());
+  return ADMMQ_OK;
+}
+
+size_t admmq_workspace_bytes(int d_in, int d_out, const admmq_params* p) {
+  if (check_params(d_in, d_out, p)) return 0;
+  const int lwork = syevd_lwork(d_in);
+  if (lwork < 0) return 0;
+  return make_layout(d_in, d_out, p->iters, lwork).total;
+}
+
+int admmq_create(admmq_ctx** out, int d, int m, const admmq_params* p, void* ws, size_t ws_bytes) {
+  if (!out) return ADMMQ_ERR_INVALID_ARG;
+  *out = nullptr;
+  int rc = check_params(d, m, p);
+  if (rc) return rc;
+  if (!ws || ((uintptr_t)ws & 255) != 0) return ADMMQ_ERR_INVALID_ARG;
+  rc = device_ok();
+  if (rc) return rc;
+  const int lwork = syevd_lwork(d);
+  if (lwork < 0) return ADMMQ_ERR_EIG;
+  Layout L = make_layout(d, m, p->iters, lwork);
+  if (ws_bytes < L.total) return ADMMQ_ERR_WORKSPACE;
+  admmq_ctx* c = new admmq_ctx();
+  c->d = d;
+  c->m = m;
+  c->p = *p;
+  c->L = (1 << p->bits) - 1;
+  cudaGetDevice(&c->dev);
+  c->ws = (uint8_t*)ws;
+  c->ws_bytes = ws_bytes;
+  uint8_t* b = c->ws;
+  c->status = (int*)(b + L.status);
+  c->lam64 = (double*)(b + L.lam64);
+  c->sig64 = (double*)(b + L.sig64);
+  c->hdiag = (float*)(b + L.hdiag);
+  c->sigma = (float*)(b + L.sigma);
+  c->rsig = (float*)(b + L.rsig);
+  c->lam32 = (float*)(b + L.lam32);
+  c->Ht = (double*)(b + L.Ht);
+  c->evals = (double*)(b + L.evals);
+  c->work = (double*)(b + L.work);
+  c->lwork = lwork;
+  c->devinfo = (int*)(b + L.devinfo);
+  c->E_hi = (float*)(b + L.E_hi);
+  c->E_lo = (float*)(b + L.E_lo);
+  c->Q_hi = (float*)(b + L.Q_hi);
+  c->Q_lo = (float*)(b + L.Q_lo);
+  c->Wt_hi = (float*)(b + L.Wt_hi);
+  c->Wt_lo = (float*)(b + L.Wt_lo);
+  c->P_hi = (float*)(b + L.P_hi);
+  c->P_lo = (float*)(b + L.P_lo);
+  c->T_hi = (float*)(b + L.T_hi);
+  c->T_lo = (float*)(b + L.T_lo);
+  c->C0 = (float*)(b + L.C0);
+  c->V = (float*)(b + L.V);
+  c->resid_part = (float*)(b + L.resid_part);
+  c->obj_part = (float*)(b + L.obj_part);
+  c->tiles_eig = cdiv(m, kBM) * cdiv(d, EigCfg::BN);
+  bool ok = true;
+  ok &= make_map(&c->mWt[0], c->Wt_hi, d, m, kBM, true) && make_map(&c->mWt[1], c->Wt_lo, d, m, kBM, true);
+  ok &= make_map(&c->mP[0], c->P_hi, d, m, kBM, true) && make_map(&c->mP[1], c->P_lo, d, m, kBM, true);
+  ok &= make_map(&c->mT[0], c->T_hi, d, m, kBM, true) && make_map(&c->mT[1], c->T_lo, d, m, kBM, true);
+  ok &= make_map(&c->mE[0], c->E_hi, d, d, EigCfg::BN, true) &&
+        make_map(&c->mE[1], c->E_lo, d, d, EigCfg::BN, true);
+  ok &= make_map(&c->mQ[0], c->Q_hi, d, d, EigCfg::BN, true) &&
+        make_map(&c->mQ[1], c->Q_lo, d, d, EigCfg::BN, true);
+  if (!ok || cusolverDnCreate(&c->solver) != CUSOLVER_STATUS_SUCCESS) {
+    delete c;
+    return ADMMQ_ERR_CUDA;
+  }
+  *out = c;
+  return ADMMQ_OK;
+}
+
+void admmq_destroy(admmq_ctx* c) {
+  if (!c) return;
+  for (auto e : c->ev) cudaEventDestroy(e);
+  if (c->solver) cusolverDnDestroy(c->solver);
+  delete c;
+}
+
+int admmq_prepare(admmq_ctx* c, const float* G, const void* W_hat, int w_dtype, void* stream) {
+  if (!c || !G || !W_hat) return ADMMQ_ERR_INVALID_ARG;
+  if (w_dtype != ADMMQ_DTYPE_F32 && w_dtype != ADMMQ_DTYPE_BF16) return ADMMQ_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int d = c->d, m = c->m;
+  c->W_hat = W_hat;
+  c->w_dtype = w_dtype;
+  CK(cudaMemsetAsync(c->status, 0, 16, st));
+  count_launch(), k_diag_stats<<<1, 1024, 0, st>>>(G, d, c->p.lambda_rel, c->lam64, c->sig64, c->hdiag, c->sigma,
+                                   c->rsig, c->status);
+  CK(cudaGetLastError());
+  count_launch(), k_scale_hessian<<<grid_for((long long)d * d), 256, 0, st>>>(G, d, c->lam64, c->sig64, c->Ht);
+  CK(cudaGetLastError());
+  const long long md = (long long)m * d;
+  if (w_dtype == ADMMQ_DTYPE_F32)
+    count_launch(), k_scale_weights<float><<<grid_for(md), 256, 0, st>>>((const float*)W_hat, c->rsig, d, md,
+                                                         c->Wt_hi, c->Wt_lo);
+  else
+    count_launch(), k_scale_weights<__nv_bfloat16><<<grid_for(md), 256, 0, st>>>(
+        (const __nv_bfloat16*)W_hat, c->rsig, d, md, c->Wt_hi, c->Wt_lo);
+  CK(cudaGetLastError());
+  c->prepared = true;
+  return ADMMQ_OK;
+}
+
+int admmq_eigh(admmq_ctx* c, void* stream) {
+  if (!c || !c->prepared) return ADMMQ_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int d = c->d;
+  int host_status[4] = {0, 0, 0, 0};
+  CK(cudaMemcpyAsync(host_status, c->status, 16, cudaMemcpyDeviceToHost, st));
+  CK(cudaStreamSynchronize(st));
+  if (host_status[1] == SETUP_NONFINITE) return ADMMQ_ERR_NONFINITE;
+  if (host_status[1] == SETUP_NOT_PD) return ADMMQ_ERR_NOT_PD;
+  if (cusolverDnSetStream(c->solver, st) != CUSOLVER_STATUS_SUCCESS) return ADMMQ_ERR_CUDA;
+  if (cusolverDnDsyevd(c->solver, CUSOLVER_EIG_MODE_VECTOR, CUBLAS_FILL_MODE_UPPER, d, c->Ht, d,
+                       c->evals, c->work, c->lwork, c->devinfo) != CUSOLVER_STATUS_SUCCESS)
+    return ADMMQ_ERR_EIG;
+  count_launch(), k_eigvals<<<grid_for(d), 256, 0, st>>>(c->evals, d, c->lam32, c->status);
+  CK(cudaGetLastError());
+  count_launch(), k_split_eigvecs<<<dim3(cdiv(d, 32), cdiv(d, 32)), dim3(32, 8), 0, st>>>(c->Ht, d, c->E_hi, c->E_lo,
+                                                                          c->Q_hi, c->Q_lo);
+  CK(cudaGetLastError());
+  int info = 0;
+  CK(cudaMemcpyAsync(&info, c->devinfo, sizeof(int), cudaMemcpyDeviceToHost, st));
+  CK(cudaMemcpyAsync(host_status, c->status, 16, cudaMemcpyDeviceToHost, st));
+  CK(cudaStreamSynchronize(st));
+  if (info != 0) return ADMMQ_ERR_EIG;
+  if (host_status[2] != 0) return ADMMQ_ERR_NONFINITE;
+  c->eig_done = true;
+  return ADMMQ_OK;
+}
+
+int admmq_setup(admmq_ctx** out, const float* G, const void* W_hat, int w_dtype, int d, int m,
+                const admmq_params* p, void* ws, size_t ws_bytes, void* stream) {
+  int rc = admmq_create(out, d, m, p, ws, ws_bytes);
+  if (rc) return rc;
+  rc = admmq_prepare(*out, G, W_hat, w_dtype, stream);
+  if (!rc) rc = admmq_eigh(*out, stream);
+  if (rc) {
+    admmq_destroy(*out);
+    *out = nullptr;
+  }
+  return rc;
+}
+
+int admmq_init(admmq_ctx* c, uint8_t* codes, float* scale, float* zero, void* stream) {
+  if (!c || !c->eig_done || !codes || !scale || !zero) return ADMMQ_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int d = c->d, m = c->m;
+  // C0' = Lambda Q^T W^~   (row j, column k)
+  GemmGeom g = make_geom(m, d, d, EigCfg::BN, EigCfg::BK, 1, false, c->status);
+  EpiScaleStore<EigCfg::BN>::Params ep{c->C0, c->lam32, d};
+  CK((launch_gemm<EigCfg, EpiScaleStore<EigCfg::BN>>(c->mWt[0], c->mWt[1], c->mE[0], c->mE[1], g,
+                                                      ep, st)));
+  const long long groups = (long long)m * (d / c->p.group);
+  if (c->w_dtype == ADMMQ_DTYPE_F32)
+    count_launch(), k_init_rtn<float><<<grid_for(groups, 128), 128, 0, st>>>(
+        (const float*)c->W_hat, c->rsig, m, d, c->p.group, c->L, codes, scale, zero, c->V,
+        c->P_hi, c->P_lo);
+  else
+    count_launch(), k_init_rtn<__nv_bfloat16><<<grid_for(groups, 128), 128, 0, st>>>(
+        (const __nv_bfloat16*)c->W_hat, c->rsig, m, d, c->p.group, c->L, codes, scale, zero,
+        c->V, c->P_hi, c->P_lo);
+  CK(cudaGetLastError());
+  c->inited = true;
+  return ADMMQ_OK;
+}
+
+int admmq_iterate(admmq_ctx* c, int t0, int count, uint8_t* codes, float* scale, float* zero,
+                  void* stream) {
+  if (!c || !c->inited || !codes || !scale || !zero) return ADMMQ_ERR_INVALID_ARG;
+  if (t0 < 0 || count < 0 || t0 + count > c->p.iters) return ADMMQ_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int d = c->d, m = c->m;
+  GemmGeom g = make_geom(m, d, d, EigCfg::BN, EigCfg::BK, 1, false, c->status);
+  for (int t = t0; t < t0 + count; ++t) {
+    const float rho = (float)((double)c->p.rho0 * pow((double)c->p.gamma, (double)t));
+    cudaEvent_t e0 = nullptr, e1 = nullptr, e2 = nullptr;
+    if (c->timing) {
+      for (int k = 0; k < 3; ++k) {
+        cudaEvent_t e;
+        CK(cudaEventCreate(&e));
+        c->ev.push_back(e);
+      }
+      e0 = c->ev[c->ev.size() - 3];
+      e1 = c->ev[c->ev.size() - 2];
+      e2 = c->ev[c->ev.size() - 1];
+      CK(cudaEventRecord(e0, st));
+    }
+    EpiTUpdate<EigCfg::BN>::Params p1{c->C0, c->lam32, c->T_hi, c->T_lo, rho, d};
+    CK((launch_gemm<EigCfg, EpiTUpdate<EigCfg::BN>>(c->mP[0], c->mP[1], c->mE[0], c->mE[1], g, p1,
+                                                     st)));
+    if (c->timing) CK(cudaEventRecord(e1, st));
+    ProjParams p2;
+    p2.V = c->V;
+    p2.codes = codes;
+    p2.scale = scale;
+    p2.zero = zero;
+    p2.p_hi = c->P_hi;
+    p2.p_lo = c->P_lo;
+    p2.sig = c->sigma;
+    p2.rsig = c->rsig;
+    p2.hd = c->hdiag;
+    p2.part = c->resid_part + (size_t)t * c->tiles_eig * 8;
+    p2.wdump = c->wdump;
+    p2.ld = d;
+    p2.group = c->p.group;
+    p2.L = c->L;
+    cudaError_t e;
+    switch (c->p.grid_mode) {
+      case ADMMQ_GRID_MINMAX:
+        e = launch_gemm<EigCfg, EpiProject<EigCfg::BN, GRID_MINMAX>>(c->mT[0], c->mT[1], c->mQ[0],
+                                                                     c->mQ[1], g, p2, st);
+        break;
+      case ADMMQ_GRID_LSQ:
+        e = launch_gemm<EigCfg, EpiProject<EigCfg::BN, GRID_LSQ>>(c->mT[0], c->mT[1], c->mQ[0],
+                                                                  c->mQ[1], g, p2, st);
+        break;
+      default:
+        e = launch_gemm<EigCfg, EpiProject<EigCfg::BN, GRID_FROZEN>>(c->mT[0], c->mT[1], c->mQ[0],
+                                                                     c->mQ[1], g, p2, st);
+        break;
+    }
+    CK(e);
+    if (c->timing) CK(cudaEventRecord(e2, st));
+  }
+  return ADMMQ_OK;
+}
+
+int admmq_finish(admmq_ctx* c, const uint8_t* codes, const float* scale, const float* zero,
+                 double* resid, double* objective, void* stream) {
+  if (!c || !c->inited) return ADMMQ_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int d = c->d, m = c->m;
+  if (resid && c->p.iters > 0) {
+    count_launch(), k_reduce_resid<<<c->p.iters, 256, 0, st>>>(c->resid_part, c->tiles_eig * 4, (double)c->p.rho0,
+                                               (double)c->p.gamma, resid);
+    CK(cudaGetLastError());
+  }
+  if (objective) {
+    if (!codes || !scale || !zero) return ADMMQ_ERR_INVALID_ARG;
+    const long long md = (long long)m * d;
+    if (c->w_dtype == ADMMQ_DTYPE_F32)
+      count_launch(), k_delta_planes<float><<<grid_for(md), 256, 0, st>>>((const float*)c->W_hat, codes, scale,
+                                                          zero, c->rsig, d, c->p.group, md,
+                                                          c->T_hi, c->T_lo);
+    else
+      count_launch(), k_delta_planes<__nv_bfloat16><<<grid_for(md), 256, 0, st>>>(
+          (const __nv_bfloat16*)c->W_hat, codes, scale, zero, c->rsig, d, c->p.group, md, c->T_hi,
+          c->T_lo);
+    CK(cudaGetLastError());
+    GemmGeom g = make_geom(m, d, d, EigCfg::BN, EigCfg::BK, 1, false, c->status);
+    EpiObjective<EigCfg::BN>::Params ep{c->lam32, c->obj_part};
+    CK((launch_gemm<EigCfg, EpiObjective<EigCfg::BN>>(c->mT[0], c->mT[1], c->mE[0], c->mE[1], g,
+                                                       ep, st)));
+    count_launch(), k_reduce_objective<<<1, 256, 0, st>>>(c->obj_part, c->tiles_eig * 4, objective);
+    CK(cudaGetLastError());
+  }
+  return ADMMQ_OK;
+}
+
+int admmq_solve(admmq_ctx* c, uint8_t* codes, float* scale, float* zero, double* resid,
+                double* objective, void* stream) {
+  int rc = admmq_init(c, codes, scale, zero, stream);
+  if (!rc) rc = admmq_iterate(c, 0, c->p.iters, codes, scale, zero, stream);
+  if (!rc) rc = admmq_finish(c, codes, scale, zero, resid, objective, stream);
+  return rc;
+}
+
+int admmq_pack(const uint8_t* codes, int d, int m, int bits, uint32_t* packed, void* stream) {
+  if (!codes || !packed || d <= 0 || m <= 0 || d % 32 != 0 || bits < 1 || bits > 8)
+    return ADMMQ_ERR_INVALID_ARG;
+  if (((uintptr_t)codes & 15) || ((uintptr_t)packed & 15)) return ADMMQ_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  const bool big = d % 128 == 0;
+  const int ch = big ? 128 : 32;
+  const int cpr = d / ch;
+  const long long chunks = (long long)m * cpr;
+  const int grid = grid_for(chunks, 256);
+#define PACK_CASE(B)                                                                      \
+  case B:                                                                                 \
+    if (big)                                                                              \
+      count_launch(), k_pack<B, 128><<<grid, 256, 0, st>>>(codes, chunks, cpr, d, packed);                \
+    else                                                                                  \
+      count_launch(), k_pack<B, 32><<<grid, 256, 0, st>>>(codes, chunks, cpr, d, packed);                 \
+    break;
+  switch (bits) {
+    PACK_CASE(1)
+    PACK_CASE(2)
+    PACK_CASE(3)
+    PACK_CASE(4)
+    PACK_CASE(5)
+    PACK_CASE(6)
+    PACK_CASE(7)
+    PACK_CASE(8)
+  }
+#undef PACK_CASE
+  CK(cudaGetLastError());
+  return ADMMQ_OK;
+}
+
+int admmq_get_buffer(admmq_ctx* c, int which, void** ptr, size_t* bytes) {
+  if (!c || !ptr) return ADMMQ_ERR_INVALID_ARG;
+  const size_t d = c->d, md = (size_t)c->m * c->d, dd = d * d;
+  void* p = nullptr;
+  size_t b = 0;
+  switch (which) {
+    case ADMMQ_BUF_SIGMA: p = c->sigma; b = 4 * d; break;
+    case ADMMQ_BUF_RSIG: p = c->rsig; b = 4 * d; break;
+    case ADMMQ_BUF_HDIAG: p = c->hdiag; b = 4 * d; break;
+    case ADMMQ_BUF_LAMBDA: p = c->lam32; b = 4 * d; break;
+    case ADMMQ_BUF_V: p = c->V; b = 4 * md; break;
+    case ADMMQ_BUF_C0: p = c->C0; b = 4 * md; break;
+    case ADMMQ_BUF_P_HI: p = c->P_hi; b = 4 * md; break;
+    case ADMMQ_BUF_P_LO: p = c->P_lo; b = 4 * md; break;
+    case ADMMQ_BUF_T_HI: p = c->T_hi; b = 4 * md; break;
+    case ADMMQ_BUF_T_LO: p = c->T_lo; b = 4 * md; break;
+    case ADMMQ_BUF_E_HI: p = c->E_hi; b = 4 * dd; break;
+    case ADMMQ_BUF_E_LO: p = c->E_lo; b = 4 * dd; break;
+    case ADMMQ_BUF_HT: p = c->Ht; b = 8 * dd; break;
+    case ADMMQ_BUF_STATUS: p = c->status; b = 16; break;
+    default: return ADMMQ_ERR_INVALID_ARG;
+  }
+  *ptr = p;
+  if (bytes) *bytes = b;
+  return ADMMQ_OK;
+}
+
+int admmq_debug_dump_wtilde(admmq_ctx* c, float* wtilde) {
+  if (!c) return ADMMQ_ERR_INVALID_ARG;
+  c->wdump = wtilde;
+  return ADMMQ_OK;
+}
+
+int admmq_set_timing(admmq_ctx* c, int enable) {
+  if (!c) return ADMMQ_ERR_INVALID_ARG;
+  for (auto e : c->ev) cudaEventDestroy(e);
+  c->ev.clear();
+  c->timing = enable != 0;
+  return ADMMQ_OK;
+}
+
+int admmq_get_timing(admmq_ctx* c, double ms[2], int launches[2]) {
+  if (!c || !ms || !launches) return ADMMQ_ERR_INVALID_ARG;
+  ms[0] = ms[1] = 0.0;
+  launches[0] = launches[1] = 0;
+  for (size_t i = 0; i + 2 < c->ev.size(); i += 3) {
+    float a = 0.f, b = 0.f;
+    CK(cudaEventSynchronize(c->ev[i + 2]));
+    CK(cudaEventElapsedTime(&a, c->ev[i], c->ev[i + 1]));
+    CK(cudaEventElapsedTime(&b, c->ev[i + 1], c->ev[i + 2]));
+    ms[0] += a;
+    ms[1] += b;
+    launches[0] += 1;
+    launches[1] += 1;
+  }
+  return ADMMQ_OK;
+}
+
+int admmq_project(const float* wt, float* V, const float* sig, const float* rsig,
+                  const float* hd, int d, int m, int bits, int g, int mode, uint8_t* codes,
+                  float* scale, float* zero, float* p_hi, float* p_lo, double* resid,
+                  void* stream) {
+  if (!wt || !V || !sig || !rsig || !hd || !codes || !scale || !zero || !p_hi || !p_lo || !resid)
+    return ADMMQ_ERR_INVALID_ARG;
+  if (d <= 0 || m <= 0 || d % 32 != 0 || !(g == 32 || g == 64 || g == 128) || d % g != 0 ||
+      bits < 1 || bits > 8 || mode < 0 || mode > 2)
+    return ADMMQ_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  CK(cudaMemsetAsync(resid, 0, 2 * sizeof(double), st));
+  dim3 grid(cdiv(m, 128), d / g);
+  const int L = (1 << bits) - 1;
+  if (mode == ADMMQ_GRID_MINMAX)
+    count_launch(), k_project<GRID_MINMAX><<<grid, 128, 0, st>>>(wt, V, sig, rsig, hd, m, d, g, L, codes, scale,
+                                                 zero, p_hi, p_lo, resid);
+  else if (mode == ADMMQ_GRID_LSQ)
+    count_launch(), k_project<GRID_LSQ><<<grid, 128, 0, st>>>(wt, V, sig, rsig, hd, m, d, g, L, codes, scale, zero,
+                                              p_hi, p_lo, resid);
+  else
+    count_launch(), k_project<GRID_FROZEN><<<grid, 128, 0, st>>>(wt, V, sig, rsig, hd, m, d, g, L, codes, scale,
+                                                 zero, p_hi, p_lo, resid);
+  CK(cudaGetLastError());
+  return ADMMQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,256 @@
+// gemm.cuh -- persistent tcgen05 GEMM engine for sm_100a.
+//
+// D[M x N] = A[M x K] * B[K x N] with operands staged in shared memory by TMA
+// (128-byte swizzle, no multicast) and fp32 accumulators in tensor memory.
+// Operands are bf16 (kind::f16) or tf32 held in fp32 words (kind::tf32); a
+// shared-memory row is always 128 bytes (64 bf16 or 32 fp32 along K) and one
+// MMA always consumes 32 bytes of K.
+// NPL = 2 runs the split-precision product used for fp32-accurate GEMMs
+// (3xTF32): every operand is stored as two tf32 planes (hi, lo) with
+// x ~= hi + lo, and each k-step issues A_hi*B_hi + A_hi*B_lo + A_lo*B_hi into
+// one accumulator.
+//
+// Warp roles (192 threads, one CTA per SM):
+//   warp 0      TMA producer (one thread)
+//   warp 1      tensor-memory owner and MMA issuer (one thread)
+//   warps 2..5  epilogue: thread = accumulator row, reads 32 columns at a time
+// The accumulator is double-buffered (2 x BN columns) so the epilogue of one
+// tile overlaps the main loop of the next.  Work units (tile, k-split) are
+// dealt to CTAs round-robin; all waits are bounded (see ptx.cuh).
+#pragma once
+#include "ptx.cuh"
+
+namespace admmq {
+
+struct GemmGeom {
+  int M, N, K;        // output rows / columns, reduction length
+  int tiles_m, tiles_n;
+  int splits;         // k-splits per tile (units = tiles * splits)
+  int kblocks;        // ceil(K / BK)
+  int triangle;       // 1: only tiles that meet the upper triangle (i <= j)
+  int tiles;          // number of tiles visited
+  int units;          // tiles * splits
+  int* status;        // kernel status word (device)
+};
+
+enum { KIND_BF16 = 1, KIND_TF32 = 2 };  // instruction-descriptor operand format
+
+template <int KIND_, int BN_, int NPL_, bool A_MN_, bool B_MN_, int STAGES_>
+struct GemmCfg {
+  static constexpr int KIND = KIND_;
+  static constexpr int ELEM = KIND == KIND_BF16 ? 2 : 4;  // bytes per operand element
+  static constexpr int BM = 128, BN = BN_, BK = 128 / ELEM, NPL = NPL_, STAGES = STAGES_;
+  static constexpr int UK = 32 / ELEM;                     // K per MMA instruction
+  static constexpr bool A_MN = A_MN_, B_MN = B_MN_;
+  static constexpr int A_PLANE = BM * 128;  // bytes per operand plane per stage
+  static constexpr int B_PLANE = BN * 128;
+  static constexpr int STAGE = NPL * (A_PLANE + B_PLANE);
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5) + 16;
+  static constexpr int SMEM = STAGES * STAGE + 1024 + BAR_BYTES;
+  static_assert(BN == 128 || BN == 256, "BN must be 128 or 256");
+  static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+// Unit -> (tile row, tile column, k-block range).  Splits are the outer index
+// so that CTAs running at the same time work on the same k-range of different
+// tiles (their A and B panels share L2).
+template <int BM, int BN>
+__device__ __forceinline__ void decode_unit(const GemmGeom& g, int u, int& tm, int& tn, int& split,
+                                            int& kb0, int& kb1) {
+  split = u / g.tiles;
+  int t = u - split * g.tiles;
+  if (!g.triangle) {
+    tm = t % g.tiles_m;
+    tn = t / g.tiles_m;
+  } else {
+    tn = 0;
+    for (;;) {
+      int cnt = ((tn + 1) * BN + BM - 1) / BM;
+      if (cnt > g.tiles_m) cnt = g.tiles_m;
+      if (t < cnt) break;
+      t -= cnt;
+      ++tn;
+    }
+    tm = t;
+  }
+  kb0 = (int)(((long long)split * g.kblocks) / g.splits);
+  kb1 = (int)(((long long)(split + 1) * g.kblocks) / g.splits);
+}
+
+template <class Cfg, class Epi>
+__global__ void __launch_bounds__(192, 1)
+    k_gemm(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ CUtensorMap tA1,
+           const __grid_constant__ CUtensorMap tB0, const __grid_constant__ CUtensorMap tB1,
+           const GemmGeom g, const typename Epi::Params ep) {
+  constexpr int BM = Cfg::BM, BN = Cfg::BN, STAGES = Cfg::STAGES, NPL = Cfg::NPL;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&tfull[a]), 1);
+      mbar_init(smem_u32(&tempty[a]), 128);
+    }
+    mbar_init(smem_u32(drain), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tA0);
+    prefetch_tmap(&tB0);
+    if (NPL == 2) {
+      prefetch_tmap(&tA1);
+      prefetch_tmap(&tB1);
+    }
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), Cfg::TMEM_COLS);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const CUtensorMap* mapA[2] = {&tA0, &tA1};
+      const CUtensorMap* mapB[2] = {&tB0, &tB1};
+      int it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < g.units && ok; u += gridDim.x) {
+        int tm, tn, split, kb0, kb1;
+        decode_unit<BM, BN>(g, u, tm, tn, split, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, abort_flag, g.status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(&full[s]);
+          mbar_arrive_expect_tx(fb, Cfg::STAGE);
+          const uint32_t st = smem_u32(smem + s * Cfg::STAGE);
+          const int k0 = kb * Cfg::BK;
+#pragma unroll
+          for (int p = 0; p < NPL; ++p) {
+            const uint32_t dA = st + p * Cfg::A_PLANE;
+            if (!Cfg::A_MN) {
+              tma_load_2d(dA, mapA[p], k0, tm * BM, fb);
+            } else {
+#pragma unroll
+              for (int b = 0; b < BM / (128 / Cfg::ELEM); ++b) tma_load_2d(dA + b * Cfg::BK * 128, mapA[p], tm * BM + (128 / Cfg::ELEM) * b, k0, fb);
+            }
+          }
+#pragma unroll
+          for (int p = 0; p < NPL; ++p) {
+            const uint32_t dB = st + NPL * Cfg::A_PLANE + p * Cfg::B_PLANE;
+            if (!Cfg::B_MN) {
+              tma_load_2d(dB, mapB[p], k0, tn * BN, fb);
+            } else {
+#pragma unroll
+              for (int b = 0; b < BN / (128 / Cfg::ELEM); ++b) tma_load_2d(dB + b * Cfg::BK * 128, mapB[p], tn * BN + (128 / Cfg::ELEM) * b, k0, fb);
+            }
+          }
+        }
+      }
+      if (!ok) {
+        // Let the copies already in flight land before the CTA retires.
+        for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
+          mbar_wait_drain(smem_u32(&full[j % STAGES]), (uint32_t)(j / STAGES) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    // --------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_f32acc(Cfg::KIND, BM, BN, Cfg::A_MN, Cfg::B_MN);
+      // MN-major: blocks of 128 bytes along MN, BK K-rows each, LBO apart
+      constexpr uint32_t LBO_A = Cfg::A_MN ? Cfg::BK * 128 : 16;
+      constexpr uint32_t LBO_B = Cfg::B_MN ? Cfg::BK * 128 : 16;
+      int it = 0, lu = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < g.units && ok; u += gridDim.x, ++lu) {
+        int tm, tn, split, kb0, kb1;
+        decode_unit<BM, BN>(g, u, tm, tn, split, kb0, kb1);
+        const int acc = lu & 1;
+        const uint32_t aph = (uint32_t)(lu >> 1) & 1u;
+        if (!mbar_wait(smem_u32(&tempty[acc]), aph ^ 1u, abort_flag, g.status)) break;
+        tc_fence_after();
+        const uint32_t dt = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          if (!mbar_wait(smem_u32(&full[s]), ph, abort_flag, g.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = smem_u32(smem + s * Cfg::STAGE);
+#pragma unroll
+          for (int kk = 0; kk < Cfg::BK / Cfg::UK; ++kk) {
+#pragma unroll
+            for (int pr = 0; pr < (NPL == 2 ? 3 : 1); ++pr) {
+              const int pa = (pr == 2) ? 1 : 0;  // (hi,hi), (hi,lo), (lo,hi)
+              const int pb = (pr == 1) ? 1 : 0;
+              const uint32_t a_addr =
+                  st + pa * Cfg::A_PLANE + (Cfg::A_MN ? kk * Cfg::UK * 128 : kk * 32);
+              const uint32_t b_addr = st + NPL * Cfg::A_PLANE + pb * Cfg::B_PLANE +
+                                      (Cfg::B_MN ? kk * Cfg::UK * 128 : kk * 32);
+              const uint64_t ad = smem_desc_sw128(a_addr, LBO_A, 1024);
+              const uint64_t bd = smem_desc_sw128(b_addr, LBO_B, 1024);
+              const uint32_t accum = (kb > kb0 || kk > 0 || pr > 0) ? 1u : 0u;
+              if (Cfg::KIND == KIND_BF16)
+                mma_bf16(dt, ad, bd, IDESC, accum);
+              else
+                mma_tf32(dt, ad, bd, IDESC, accum);
+            }
+          }
+          mma_commit(smem_u32(&empty[s]));
+        }
+        if (!ok) break;
+        mma_commit(smem_u32(&tfull[acc]));
+      }
+      // Every MMA issued above is complete once this arrives.
+      mma_commit(smem_u32(drain));
+      mbar_wait_drain(smem_u32(drain), 0);
+    }
+  } else {
+    // ----------------------------------------------------------- epilogue
+    const int q = warp & 3;  // tensor-memory lane quarter this warp may access
+    int lu = 0;
+    for (int u = blockIdx.x; u < g.units; u += gridDim.x, ++lu) {
+      int tm, tn, split, kb0, kb1;
+      decode_unit<BM, BN>(g, u, tm, tn, split, kb0, kb1);
+      const int acc = lu & 1;
+      const uint32_t aph = (uint32_t)(lu >> 1) & 1u;
+      // warp-uniform decision: tcgen05.ld below needs all 32 lanes
+      const bool ok = mbar_wait(smem_u32(&tfull[acc]), aph, abort_flag, g.status);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      Epi::apply(ep, g, taddr, tm, tn, split, q, lane);
+      tc_fence_before();
+      mbar_arrive(smem_u32(&tempty[acc]));
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+}  // namespace admmq

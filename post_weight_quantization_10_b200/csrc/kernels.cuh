@@ -1,0 +1,380 @@
+// kernels.cuh -- element-wise, reduction and epilogue kernels of the ADMM-Q
+// layer solve (everything that is not the tcgen05 main loop).
+#pragma once
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "gemm.cuh"
+
+namespace admmq {
+
+enum { GRID_MINMAX = 0, GRID_LSQ = 1, GRID_FROZEN = 2 };
+
+// ------------------------------------------------------------ small helpers
+
+__device__ __forceinline__ uint16_t bf16_bits(float x) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+// Round a float32 to tf32 (10 explicit mantissa bits), nearest-even, kept in
+// a float32 word with the 13 low bits zero.
+__device__ __forceinline__ float tf32_rne(float x) {
+  uint32_t b = __float_as_uint(x);
+  b = (b + 0xFFFu + ((b >> 13) & 1u)) & ~0x1FFFu;
+  return __uint_as_float(b);
+}
+// x ~= hi + lo: hi = tf32(x), lo = tf32(x - hi)  (the 3xTF32 operand planes).
+__device__ __forceinline__ void split2(float x, float& hi, float& lo) {
+  hi = tf32_rne(x);
+  lo = tf32_rne(__fsub_rn(x, hi));
+}
+// clamp to [0, L]; adding +0 turns a -0 into +0 so the result never depends
+// on which zero fmaxf returns for (-0, +0)
+__device__ __forceinline__ float clampq(float q, float L) {
+  return __fadd_rn(fminf(fmaxf(q, 0.f), L), 0.f);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// ------------------------------------------- grid fit + projection (fp32)
+//
+// The D-update's float32 arithmetic, one thread per (row, group).  Every
+// operation is an explicitly rounded IEEE op (no contraction) so that the
+// result is reproducible bit for bit by a float32 reference:
+//   t = W~ + V~,  y = sigma t
+//   minmax: mn = min(0, min y), mx = max(0, max y), s = (mx - mn)/L,
+//           z = rint(-mn/s)   (s = 1, z = 0 when mx = mn)
+//   lsq:    q0 = clamp(rint(y/s_prev) + z_prev); weighted sums (w = diag H)
+//           in element order; slope/offset, integer zero point, slope again
+//   q = clamp(rint(y/s) + z, 0, L);  D = s (q - z);  D~ = D rsig
+//   V~' = t - D~;  P = D~ - V~'  (stored as tf32 hi/lo planes)
+
+struct ProjRow {
+  float* V;            // this row's V~ at the group's first column
+  const float* sig;    // sigma, rsig, diag(H) at the group's first column
+  const float* rsig;
+  const float* hd;
+  uint8_t* codes;
+  float* phi;
+  float* plo;
+  float* scale;        // this group's scale / zero
+  float* zero;
+  float* wdump;        // optional raw W~ output
+  bool valid;
+};
+
+template <int MODE, class LoadW>
+__device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, int g, int L,
+                                              float& r2, float& s2) {
+  const float Lf = (float)L;
+  float s0 = 1.f, z0 = 0.f;
+  if (r.valid) {
+    s0 = *r.scale;
+    z0 = *r.zero;
+  }
+  float s = s0, z = z0;
+  if (MODE != GRID_FROZEN) {
+    float mn = 0.f, mx = 0.f;
+    float Sw = 0.f, Sq = 0.f, Sqq = 0.f, Sy = 0.f, Sqy = 0.f;
+    for (int c = 0; c < g; c += 32) {
+      float w[32];
+      loadw(c, w);
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) {
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r.valid) v = *reinterpret_cast<const float4*>(r.V + c + e);
+        const float4 sg = __ldg(reinterpret_cast<const float4*>(r.sig + c + e));
+        float4 hd = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (MODE == GRID_LSQ) hd = __ldg(reinterpret_cast<const float4*>(r.hd + c + e));
+        const float vv[4] = {v.x, v.y, v.z, v.w}, ss[4] = {sg.x, sg.y, sg.z, sg.w};
+        const float hh[4] = {hd.x, hd.y, hd.z, hd.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float t = __fadd_rn(w[e + k], vv[k]);
+          const float y = __fmul_rn(ss[k], t);
+          if (MODE == GRID_MINMAX) {
+            mn = fminf(mn, y);
+            mx = fmaxf(mx, y);
+          } else {
+            const float q0 = clampq(__fadd_rn(rintf(__fdiv_rn(y, s0)), z0), Lf);
+            const float wi = hh[k];
+            const float wq = __fmul_rn(wi, q0);
+            Sw = __fadd_rn(Sw, wi);
+            Sq = __fadd_rn(Sq, wq);
+            Sqq = __fadd_rn(Sqq, __fmul_rn(wq, q0));
+            Sy = __fadd_rn(Sy, __fmul_rn(wi, y));
+            Sqy = __fadd_rn(Sqy, __fmul_rn(wq, y));
+          }
+        }
+      }
+    }
+    if (MODE == GRID_MINMAX) {
+      s = __fdiv_rn(__fsub_rn(mx, mn), Lf);
+      if (s == 0.f) {
+        s = 1.f;
+        z = 0.f;
+      } else {
+        z = __fadd_rn(rintf(__fdiv_rn(-mn, s)), 0.f);
+      }
+    } else {
+      const float qm = __fdiv_rn(Sq, Sw);
+      const float ym = __fdiv_rn(Sy, Sw);
+      const float var = __fsub_rn(Sqq, __fmul_rn(Sq, qm));
+      const float cov = __fsub_rn(Sqy, __fmul_rn(Sq, ym));
+      if (var > 0.f && cov > 0.f) {
+        const float s1 = __fdiv_rn(cov, var);
+        const float zc = clampq(rintf(__fsub_rn(qm, __fdiv_rn(ym, s1))), Lf);
+        const float num = __fsub_rn(Sqy, __fmul_rn(zc, Sy));
+        const float den = __fadd_rn(__fsub_rn(Sqq, __fmul_rn(__fmul_rn(2.f, zc), Sq)),
+                                    __fmul_rn(__fmul_rn(zc, zc), Sw));
+        s = (den > 0.f && num > 0.f) ? __fdiv_rn(num, den) : s1;
+        z = zc;
+      }
+    }
+  }
+  for (int c = 0; c < g; c += 32) {
+    float w[32];
+    loadw(c, w);
+#pragma unroll
+    for (int e = 0; e < 32; e += 4) {
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      uint32_t cp = 0;
+      if (r.valid) {
+        v = *reinterpret_cast<const float4*>(r.V + c + e);
+        cp = *reinterpret_cast<const uint32_t*>(r.codes + c + e);
+      }
+      const float4 sg = __ldg(reinterpret_cast<const float4*>(r.sig + c + e));
+      const float4 rs = __ldg(reinterpret_cast<const float4*>(r.rsig + c + e));
+      const float vv[4] = {v.x, v.y, v.z, v.w}, ss[4] = {sg.x, sg.y, sg.z, sg.w};
+      const float rr[4] = {rs.x, rs.y, rs.z, rs.w};
+      float vn[4];
+      uint32_t qc = 0;
+      float hi[4], lo[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float t = __fadd_rn(w[e + k], vv[k]);
+        const float y = __fmul_rn(ss[k], t);
+        const float q = clampq(__fadd_rn(rintf(__fdiv_rn(y, s)), z), Lf);
+        const float D = __fmul_rn(s, __fsub_rn(q, z));
+        const float dt = __fmul_rn(D, rr[k]);
+        vn[k] = __fsub_rn(t, dt);
+        const float p = __fsub_rn(dt, vn[k]);
+        split2(p, hi[k], lo[k]);
+        qc |= (uint32_t)q << (8 * k);
+        const float e1 = w[e + k] - dt;
+        r2 += e1 * e1;
+        const float qp = (float)((cp >> (8 * k)) & 0xFFu);
+        const float dtp = __fmul_rn(__fmul_rn(s0, __fsub_rn(qp, z0)), rr[k]);
+        const float e2 = dt - dtp;
+        s2 += e2 * e2;
+      }
+      if (r.valid) {
+        *reinterpret_cast<float4*>(r.V + c + e) = make_float4(vn[0], vn[1], vn[2], vn[3]);
+        *reinterpret_cast<uint32_t*>(r.codes + c + e) = qc;
+        *reinterpret_cast<float4*>(r.phi + c + e) = make_float4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<float4*>(r.plo + c + e) = make_float4(lo[0], lo[1], lo[2], lo[3]);
+        if (r.wdump)
+          *reinterpret_cast<float4*>(r.wdump + c + e) = make_float4(w[e], w[e + 1], w[e + 2], w[e + 3]);
+      }
+    }
+  }
+  if (r.valid) {
+    *r.scale = s;
+    *r.zero = z;
+  }
+  if (!r.valid) {  // rows past d_out contribute nothing
+    r2 = 0.f;
+    s2 = 0.f;
+  }
+}
+
+// -------------------------------------------------------------- epilogues
+// Each epilogue thread owns accumulator row (tm*128 + 32q + lane) and reads
+// 32 fp32 columns per tensor-memory load.
+
+// Gram: raw fp32 tile into the k-split's partial buffer (upper part used).
+template <int BN>
+struct EpiGramPartial {
+  struct Params {
+    float* part;
+    long long split_stride;  // elements between k-split buffers
+    int ld;
+  };
+  __device__ static void apply(const Params& p, const GemmGeom& g, uint32_t taddr, int tm, int tn,
+                               int split, int q, int lane) {
+    const int row = tm * 128 + q * 32 + lane;
+    float* out = p.part + split * p.split_stride + (long long)row * p.ld;
+    for (int c = 0; c < BN; c += 32) {
+      const int col = tn * BN + c;
+      if (col >= g.N) break;
+      float v[32];
+      tmem_ld32(taddr + c, v);
+      if (row < g.M) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          *reinterpret_cast<float4*>(out + col + 4 * k) =
+              make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+      }
+    }
+  }
+};
+
+// C0' = Lambda (Q^T W^~): column k scaled by lambda_k, stored fp32.
+template <int BN>
+struct EpiScaleStore {
+  struct Params {
+    float* out;
+    const float* lam;
+    int ld;
+  };
+  __device__ static void apply(const Params& p, const GemmGeom& g, uint32_t taddr, int tm, int tn,
+                               int, int q, int lane) {
+    const int row = tm * 128 + q * 32 + lane;
+    for (int c = 0; c < BN; c += 32) {
+      const int col = tn * BN + c;
+      if (col >= g.N) break;
+      float v[32];
+      tmem_ld32(taddr + c, v);
+      if (row < g.M) {
+        float* o = p.out + (long long)row * p.ld + col;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float4 l = __ldg(reinterpret_cast<const float4*>(p.lam + col + 4 * k));
+          *reinterpret_cast<float4*>(o + 4 * k) =
+              make_float4(__fmul_rn(l.x, v[4 * k]), __fmul_rn(l.y, v[4 * k + 1]),
+                          __fmul_rn(l.z, v[4 * k + 2]), __fmul_rn(l.w, v[4 * k + 3]));
+        }
+      }
+    }
+  }
+};
+
+// GEMM 1 epilogue: T = (C0' + rho acc) / (lambda + rho), split to tf32 planes.
+template <int BN>
+struct EpiTUpdate {
+  struct Params {
+    const float* c0;
+    const float* lam;
+    float* t_hi;
+    float* t_lo;
+    float rho;
+    int ld;
+  };
+  __device__ static void apply(const Params& p, const GemmGeom& g, uint32_t taddr, int tm, int tn,
+                               int, int q, int lane) {
+    const int row = tm * 128 + q * 32 + lane;
+    for (int c = 0; c < BN; c += 32) {
+      const int col = tn * BN + c;
+      if (col >= g.N) break;
+      float v[32];
+      tmem_ld32(taddr + c, v);
+      if (row < g.M) {
+        const long long off = (long long)row * p.ld + col;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float4 c0 = *reinterpret_cast<const float4*>(p.c0 + off + 4 * k);
+          const float4 l = __ldg(reinterpret_cast<const float4*>(p.lam + col + 4 * k));
+          const float cc[4] = {c0.x, c0.y, c0.z, c0.w}, ll[4] = {l.x, l.y, l.z, l.w};
+          float hi[4], lo[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float inv = __frcp_rn(__fadd_rn(ll[j], p.rho));
+            const float t = __fmul_rn(__fadd_rn(cc[j], __fmul_rn(p.rho, v[4 * k + j])), inv);
+            split2(t, hi[j], lo[j]);
+          }
+          *reinterpret_cast<float4*>(p.t_hi + off + 4 * k) = make_float4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<float4*>(p.t_lo + off + 4 * k) = make_float4(lo[0], lo[1], lo[2], lo[3]);
+        }
+      }
+    }
+  }
+};
+
+// GEMM 2 epilogue: W~ = Q T from tensor memory, fused grid refresh,
+// projection, dual update and residual partial sums (one per tile and warp).
+struct ProjParams {
+  float* V;
+  uint8_t* codes;
+  float* scale;
+  float* zero;
+  float* p_hi;
+  float* p_lo;
+  const float* sig;
+  const float* rsig;
+  const float* hd;
+  float* part;    // [tiles][4][2] for this iteration
+  float* wdump;   // optional
+  int ld;         // d_in
+  int group;
+  int L;
+};
+
+template <int BN, int MODE>
+struct EpiProject {
+  using Params = ProjParams;
+  __device__ static void apply(const Params& p, const GemmGeom& g, uint32_t taddr, int tm, int tn,
+                               int, int q, int lane) {
+    const int row = tm * 128 + q * 32 + lane;
+    const bool valid = row < g.M;
+    const int ngrp_row = p.ld / p.group;
+    float r2 = 0.f, s2 = 0.f;
+    for (int c0 = 0; c0 < BN; c0 += p.group) {
+      const int col0 = tn * BN + c0;
+      if (col0 >= g.N) break;
+      const long long off = (long long)(valid ? row : 0) * p.ld + col0;
+      const long long goff = (long long)(valid ? row : 0) * ngrp_row + col0 / p.group;
+      ProjRow r;
+      r.V = p.V + off;
+      r.sig = p.sig + col0;
+      r.rsig = p.rsig + col0;
+      r.hd = p.hd + col0;
+      r.codes = p.codes + off;
+      r.phi = p.p_hi + off;
+      r.plo = p.p_lo + off;
+      r.scale = p.scale + goff;
+      r.zero = p.zero + goff;
+      r.wdump = p.wdump ? p.wdump + off : nullptr;
+      r.valid = valid;
+      auto loadw = [&](int c, float (&w)[32]) { tmem_ld32(taddr + c0 + c, w); };
+      project_group<MODE>(loadw, r, p.group, p.L, r2, s2);
+    }
+    r2 = warp_sum(r2);
+    s2 = warp_sum(s2);
+    if (lane == 0) {
+      const int tile = tn * g.tiles_m + tm;
+      p.part[(tile * 4 + q) * 2 + 0] = r2;
+      p.part[(tile * 4 + q) * 2 + 1] = s2;
+    }
+  }
+};
+
+// Objective: sum_k lambda_k acc_{jk}^2 per tile and warp.
+template <int BN>
+struct EpiObjective {
+  struct Params {
+    const float* lam;
+    float* part;  // [tiles][4]
+  };
+  __device__ static void apply(const Params& p, const GemmGeom& g, uint32_t taddr, int tm, int tn,
+                               int, int q, int lane) {
+    const int row = tm * 128 + q * 32 + lane;
+    float acc = 0.f;
+    for (int c = 0; c < BN; c += 32) {
+      const int col = tn * BN + c;
+      if (col >= g.N) break;
+      float v[32];
+      tmem_ld32(taddr + c, v);
+      if (row < g.M) {
+#pragma unroll
+        for (int k = 0; k < 32; ++k) acc += __ldg(p.lam + col + k) * v[k] * v[k];
+      }
+    }
+    acc = warp_sum(acc);
+    if (lane == 0) p.part[(tn * g.tiles_m + tm) * 4 + q] = acc;
+  }
+};
+
+}  // namespace admmq

@@ -1,0 +1,126 @@
+"""Kernel-level parity of the CUDA path against the oracle (needs a B200).
+
+Inputs come from seeded generators only; expected values come from oracle/.
+Bit-exact where the work is integer or an explicitly specified float32
+sequence (projection, RTN start, packing); Gram within 1e-4 relative
+Frobenius (fp32 tensor-core sums of exact bf16 products).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import admmq_oracle as O
+from oracle import projection_fp32 as P
+from post_weight_quantization_10_b200 import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def A():
+    from post_weight_quantization_10_b200 import admmq
+    admmq.lib()
+    return admmq
+
+
+# ------------------------------------------------------------------- Gram
+
+
+@pytest.mark.parametrize("n,d", [(512, 64), (1000, 192), (4133, 384), (20000, 512)])
+def test_gram_matches_oracle(A, n, d):
+    p = workloads.scaled(workloads.PRESETS["q_proj"], n, d, 8, rank=8)
+    X = workloads.make_activations(p, seed=3, device="cuda")
+    H = A.build_hessian(X)
+    torch.cuda.synchronize()
+    G = O.gram(X.float().cpu().numpy())
+    Hc = H.cpu().numpy().astype(np.float64)
+    assert np.array_equal(Hc, Hc.T)
+    err = np.linalg.norm(Hc - G) / np.linalg.norm(G)
+    assert err <= 1e-4, err
+
+
+def test_gram_accumulate_and_empty(A):
+    p = workloads.scaled(workloads.PRESETS["q_proj"], 3000, 256, 8, rank=8)
+    X = workloads.make_activations(p, seed=4, device="cuda")
+    H = A.build_hessian(X[:1700])
+    A.build_hessian(X[1700:], H=H, accumulate=True)
+    A.build_hessian(X[:0], H=H, accumulate=True)
+    torch.cuda.synchronize()
+    G = O.gram(X.float().cpu().numpy())
+    assert np.linalg.norm(H.cpu().numpy() - G) / np.linalg.norm(G) <= 1e-4
+    Z = A.build_hessian(X[:0])
+    torch.cuda.synchronize()
+    assert float(Z.abs().max()) == 0.0
+
+
+def test_gram_tiny_layer(A):
+    Xn, _ = workloads.tiny_layer(0)
+    X = torch.from_numpy(Xn).to(torch.bfloat16).cuda()
+    H = A.build_hessian(X)
+    torch.cuda.synchronize()
+    G = O.gram(Xn)
+    assert np.linalg.norm(H.cpu().numpy() - G) / np.linalg.norm(G) <= 1e-5
+
+
+# ------------------------------------------------------ projection, bit-exact
+
+
+def _proj_inputs(m, d, g, bits, seed):
+    rng = np.random.default_rng(seed)
+    L = (1 << bits) - 1
+    sig = np.exp(rng.standard_normal(d)).astype(np.float32) * 0.05
+    rsig = (1.0 / sig).astype(np.float32)
+    hd = (rsig.astype(np.float64) ** 2).astype(np.float32)
+    W = (rng.standard_normal((m, d)) * 2).astype(np.float32)
+    V = (rng.standard_normal((m, d)) * 0.3).astype(np.float32)
+    s0 = (rng.random((m, d // g)) * 0.05 + 0.01).astype(np.float32)
+    z0 = rng.integers(0, L + 1, (m, d // g)).astype(np.float32)
+    c0 = rng.integers(0, L + 1, (m, d)).astype(np.uint8)
+    W[0, :g] = 0.0            # an all-zero group (zero range) when V is zero there
+    V[0, :g] = 0.0
+    return dict(W=W, V=V, sig=sig, rsig=rsig, hd=hd, s0=s0, z0=z0, c0=c0)
+
+
+@pytest.mark.parametrize("grid", ["minmax", "lsq", "frozen"])
+@pytest.mark.parametrize("bits,g,m,d", [(3, 128, 200, 384), (2, 64, 33, 128), (4, 32, 130, 96),
+                                        (3, 64, 32, 64)])
+def test_projection_kernel_bitexact(A, grid, bits, g, m, d):
+    x = _proj_inputs(m, d, g, bits, seed=bits * 100 + g + m)
+    ref = P.epilogue_step(x["W"], x["V"], x["sig"], x["rsig"], x["hd"], x["s0"], x["z0"], x["c0"],
+                          bits, g, grid)
+    cu = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    V = cu(x["V"])
+    codes, scale, zero = cu(x["c0"]), cu(x["s0"]), cu(x["z0"])
+    phi = torch.empty((m, d), dtype=torch.float32, device="cuda")
+    plo = torch.empty_like(phi)
+    resid = A.project(cu(x["W"]), V, cu(x["sig"]), cu(x["rsig"]), cu(x["hd"]), bits, g, grid,
+                      codes, scale, zero, phi, plo)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(codes.cpu().numpy(), ref["codes"])
+    np.testing.assert_array_equal(scale.cpu().numpy().view(np.uint32), ref["scale"].view(np.uint32))
+    np.testing.assert_array_equal(zero.cpu().numpy().view(np.uint32), ref["zero"].view(np.uint32))
+    np.testing.assert_array_equal(V.cpu().numpy().view(np.uint32), ref["V"].view(np.uint32))
+    np.testing.assert_array_equal(phi.cpu().numpy().view(np.uint32), ref["P_hi"].view(np.uint32))
+    np.testing.assert_array_equal(plo.cpu().numpy().view(np.uint32), ref["P_lo"].view(np.uint32))
+    r = resid.cpu().numpy()
+    assert r[0] == pytest.approx(ref["r2"], rel=1e-4)
+    assert r[1] == pytest.approx(ref["s2"], rel=1e-4, abs=1e-12)
+
+
+# ------------------------------------------------------------------ packing
+
+
+@pytest.mark.parametrize("bits", range(1, 9))
+@pytest.mark.parametrize("m,d", [(7, 32), (5, 96), (3, 128), (33, 384)])
+def test_pack_bitexact(A, bits, m, d):
+    rng = np.random.default_rng(bits * 1000 + d + m)
+    codes = rng.integers(0, 1 << bits, (m, d)).astype(np.uint8)
+    out = A.pack(torch.from_numpy(codes).cuda(), bits)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(out.cpu().numpy().view(np.uint32), O.pack(codes, bits))
+
+
+def test_pack_rejects_bad_shapes(A):
+    c = torch.zeros((4, 48), dtype=torch.uint8, device="cuda")
+    with pytest.raises(A.AdmmqError):
+        A.pack(c, 3, out=torch.empty((4, 8), dtype=torch.int32, device="cuda"))

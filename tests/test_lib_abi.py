@@ -1,0 +1,58 @@
+"""The C-ABI library loads and exports every entry point include/admmq.h
+declares; argument checks that need no GPU reject bad input."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    src = open(os.path.join(ROOT, "include", "admmq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(admmq_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from post_weight_quantization_10_b200 import admmq, build
+    build.build()
+    return admmq.lib()
+
+
+def test_exports_every_declared_function(lib):
+    names = _header_functions()
+    assert len(names) >= 10
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings(lib):
+    from post_weight_quantization_10_b200 import admmq
+    for code in range(0, -9, -1):
+        s = admmq.status_string(code)
+        assert s and s != "unknown status"
+    assert admmq.status_string(-99) == "unknown status"
+    assert lib.admmq_version() >= 100
+
+
+def test_argument_checks_without_gpu(lib):
+    from post_weight_quantization_10_b200 import admmq
+    p = admmq.Params(bits=3, group=128, iters=10).c()
+    # d_in not a multiple of the group / of 32, bad bits, bad group
+    assert lib.admmq_workspace_bytes(100, 8, ctypes.byref(p)) == 0
+    bad = admmq.Params(bits=9, group=128).c()
+    assert lib.admmq_workspace_bytes(256, 8, ctypes.byref(bad)) == 0
+    bad = admmq.Params(bits=3, group=48).c()
+    assert lib.admmq_workspace_bytes(96, 8, ctypes.byref(bad)) == 0
+    assert lib.admmq_gram_workspace_bytes(100, 30) == 0
+    assert lib.admmq_pack(None, 64, 4, 3, None, None) == admmq.ADMMQ_ERR_INVALID_ARG if hasattr(admmq, "ADMMQ_ERR_INVALID_ARG") else -1
+    assert lib.admmq_pack(ctypes.c_void_p(16), 48, 4, 3, ctypes.c_void_p(16), None) == -1
+    assert lib.admmq_build_hessian(None, 10, 64, None, 0, None, 0, None) == -1
+    ctx = ctypes.c_void_p()
+    assert lib.admmq_create(ctypes.byref(ctx), 100, 8, ctypes.byref(p), None, 0) == -1
+    assert lib.admmq_init(None, None, None, None, None) == -1
+    assert lib.admmq_iterate(None, 0, 1, None, None, None, None) == -1
+    lib.admmq_destroy(None)

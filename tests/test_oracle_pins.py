@@ -298,6 +298,21 @@ def test_lsq_refit_does_not_increase_weighted_error():
     assert e1.sum() < e0.sum()
 
 
+def test_tf32_split_reconstructs_float32():
+    """3xTF32 operand planes: hi and lo carry 11 significant bits each, so
+    hi + lo holds x to about 2^-22 relative, and hi is the nearest tf32."""
+    rng = np.random.default_rng(10)
+    x = (rng.standard_normal(10000) * np.exp(rng.standard_normal(10000) * 3)).astype(np.float32)
+    hi, lo = P.split_tf32(x)
+    assert np.all((hi.view(np.uint32) & 0x1FFF) == 0) and np.all((lo.view(np.uint32) & 0x1FFF) == 0)
+    rec = hi.astype(np.float64) + lo
+    assert np.max(np.abs(rec - x) / np.abs(x)) < 2.0 ** -21
+    assert np.all(np.abs(x - hi.astype(np.float64)) <= np.abs(x) * 2.0 ** -11)
+    # hand example: 1 + 2^-11 is a tie between 1 and 1 + 2^-10 -> even (1.0)
+    t = np.array([1 + 2.0 ** -11, 1 + 3 * 2.0 ** -11], np.float32)
+    np.testing.assert_array_equal(P.tf32_round(t), np.array([1.0, 1 + 2.0 ** -9], np.float32))
+
+
 def test_bf16_split_reconstructs_float32():
     rng = np.random.default_rng(9)
     x = (rng.standard_normal(10000) * np.exp(rng.standard_normal(10000) * 3)).astype(np.float32)
