@@ -152,6 +152,8 @@ def run_ours(args, rank, world, device):
     from post_weight_quantization_10_b200 import admmq as A
     A.lib()
     p = workloads.PRESETS[args.workload]
+    if args.tokens:
+        p = workloads.scaled(p, args.tokens, p.d_in, p.d_out)
     run = LayerRun(A, p, args.grid, seed=rank, device=device)
     eigh_s = run.setup_eigh()
     for _ in range(args.warmup):
@@ -383,6 +385,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="q_proj", choices=sorted(workloads.PRESETS))
     ap.add_argument("--grid", default="minmax", choices=["minmax", "lsq", "frozen"])
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override the calibration token count n (profiling captures only; "
+                         "the eigenbasis GEMMs do not depend on n)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

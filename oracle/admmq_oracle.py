@@ -169,7 +169,7 @@ def w_update(Q: np.ndarray, lam: np.ndarray, B: np.ndarray, rho: float,
 
 def admm_q(H: np.ndarray, W_hat: np.ndarray, bits: int, group: int, iters: int,
            rho0: float = 0.1, gamma: float = 1.05, grid: str = "minmax",
-           scaling: bool = True, eig=None, grid0=None) -> dict:
+           scaling: bool = True, eig=None, grid0=None, trace=None) -> dict:
     """The ADMM-Q layer solve, step by step in the pages' order.
 
     1. Sigma = Diag(H)^(-1/2); H~ = Sigma H Sigma; W^~ = Sigma^-1 W_hat.
@@ -208,11 +208,19 @@ def admm_q(H: np.ndarray, W_hat: np.ndarray, bits: int, group: int, iters: int,
     Wt = Wt_hat
     for t in range(iters):
         rho = rho0 * gamma ** t
+        entry = None
+        if trace is not None:
+            entry = dict(t=t, rho=rho, Dt=Dt.copy(), Vt=Vt.copy(), codes=codes.copy(),
+                         scale=s.copy(), zero=z.copy())
         Wt = w_update(Q, lam, B, rho, Dt, Vt)
         Y = sigma[:, None] * (Wt + Vt)
         codes_new, s, z, D = project(Y, bits, group, grid, hdiag, s, z)
         Dt_new = D / sigma[:, None]
         Vt = Vt + Wt - Dt_new
+        if entry is not None:
+            entry.update(W_tilde=Wt.copy(), Y=Y.copy(), codes_out=codes_new.copy(),
+                         scale_out=s.copy(), zero_out=z.copy(), Vt_out=Vt.copy())
+            trace.append(entry)
         r_hist.append(float(np.linalg.norm(Wt - Dt_new)))
         s_hist.append(float(rho * np.linalg.norm(Dt_new - Dt)))
         code_changes.append(int(np.count_nonzero(codes_new != codes)))
