@@ -94,6 +94,32 @@ size_t admmq_gram_workspace_bytes(int64_t n, int d_in);
 int admmq_build_hessian(const void* X_dev, int64_t n, int d_in, float* H_dev, int accumulate,
                         void* ws_dev, size_t ws_bytes, void* stream);
 
+/* No-allocation variant of admmq_build_hessian (the pages have no counterpart:
+ * this is an interface for callers, not a step of the method).
+ * Some callers cannot allocate device memory at the moment they need the
+ * Hessian: a serving or training framework that has already reserved all
+ * device memory for its own pool, or code that must not call cudaMalloc
+ * (it can synchronise the device and is not allowed while a stream is being
+ * captured).  This entry point takes no workspace: its scratch (the k-split
+ * partial sums and a status word) lives in one file-scope device array of
+ * ADMMQ_STATIC_SCRATCH_BYTES, which every GPU that loads the library holds
+ * until the process exits.  It computes the same X^T X as
+ * admmq_build_hessian (same kernels; the k-split count may be smaller so that
+ * the partials fit, which only changes the order of fp32 additions).
+ *   Limit: 256 + d_in * d_in * 4 bytes must fit in ADMMQ_STATIC_SCRATCH_BYTES
+ *   (d_in <= 4096); larger d_in returns ADMMQ_ERR_WORKSPACE before anything
+ *   is launched.
+ *   The first call on a device looks the array's device address up
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.  Nothing is allocated, here or later.
+ *   All calls share the array and it keeps the last call's contents (the
+ *   status word is cleared at the start of every call): calls that overlap on
+ *   the GPU -- on different streams, or from different threads -- race on it
+ *   and must be serialised by the caller. */
+#define ADMMQ_STATIC_SCRATCH_BYTES ((size_t)64 * 1024 * 1024 + 256)
+int admmq_build_hessian_static(const void* X_dev, int64_t n, int d_in, float* H_dev,
+                               int accumulate, void* stream);
+
 /* ---------------------------------------------------------------- context --
  * One context per layer solve.  ws_dev (caller-allocated device memory of at
  * least admmq_workspace_bytes() bytes) holds all solver state; the context

@@ -1043,4 +1043,67 @@ int admmq_project(const float* wt, float* V, const float* sig, const float* rsig
   return ADMMQ_OK;
 }
 
+// ------------------------------------------- no-allocation Gram variant
+
 }  // extern "C"
+
+namespace {
+
+// Scratch of admmq_build_hessian_static: a status word (first 256 bytes) and
+// the k-split partial sums.  Shared by every call on a device.
+__device__ __align__(256) uint8_t g_static_scratch[ADMMQ_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+void* g_static_ptr[kMaxDevices] = {};
+bool g_static_ready[kMaxDevices] = {};
+
+// Device address of g_static_scratch for the current device (looked up once
+// per device with that device current).
+int static_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ADMMQ_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return ADMMQ_ERR_UNSUPPORTED;
+  if (!__atomic_load_n(&g_static_ready[dev], __ATOMIC_ACQUIRE)) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return ADMMQ_ERR_CUDA;
+    g_static_ptr[dev] = p;
+    __atomic_store_n(&g_static_ready[dev], true, __ATOMIC_RELEASE);
+  }
+  *out = g_static_ptr[dev];
+  return ADMMQ_OK;
+}
+
+}  // namespace
+
+extern "C" int admmq_build_hessian_static(const void* X, int64_t n, int d, float* H,
+                                          int accumulate, void* stream) {
+  if ((!X && n > 0) || !H || d <= 0 || d % 32 != 0 || n < 0) return ADMMQ_ERR_INVALID_ARG;
+  if (((uintptr_t)X & 15) != 0) return ADMMQ_ERR_INVALID_ARG;
+  const size_t dd4 = (size_t)d * d * 4;
+  if (256 + dd4 > ADMMQ_STATIC_SCRATCH_BYTES) return ADMMQ_ERR_WORKSPACE;
+  int rc = device_ok();
+  if (rc) return rc;
+  void* base = nullptr;
+  rc = static_scratch(&base);
+  if (rc) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (n == 0) {
+    if (!accumulate) CK(cudaMemsetAsync(H, 0, dd4, st));
+    return ADMMQ_OK;
+  }
+  int splits = gram_splits(n, d, num_sms());
+  while (splits > 1 && 256 + (size_t)splits * dd4 > ADMMQ_STATIC_SCRATCH_BYTES) --splits;
+  int* status = (int*)base;
+  float* part = (float*)((uint8_t*)base + 256);
+  CK(cudaMemsetAsync(status, 0, 16, st));
+  CUtensorMap mx;
+  if (!make_map(&mx, X, (uint64_t)d, (uint64_t)n, GramCfg::BK, false)) return ADMMQ_ERR_CUDA;
+  GemmGeom g = make_geom(d, d, n, GramCfg::BN, GramCfg::BK, splits, true, status);
+  EpiGramPartial<GramCfg::BN>::Params ep{part, (long long)d * d, d};
+  CK((launch_gemm<GramCfg, EpiGramPartial<GramCfg::BN>>(mx, mx, mx, mx, g, ep, st)));
+  const int nb = d / 32;
+  count_launch(), k_gram_finalize<<<dim3(nb, nb), dim3(32, 8), 0, st>>>(part, splits, (long long)d * d, d, H,
+                                                                          accumulate, status);
+  CK(cudaGetLastError());
+  return ADMMQ_OK;
+}

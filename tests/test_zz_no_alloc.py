@@ -1,0 +1,81 @@
+"""The no-allocation Hessian entry point, admmq_build_hessian_static.
+
+Some callers cannot allocate device memory at the moment they need the
+Hessian: a framework whose memory pool already holds all of the device
+memory, or code that must not call cudaMalloc (it can synchronise the device
+and is not allowed while a stream is being captured).  This entry point keeps
+its scratch in a fixed device array inside the library instead of taking a
+workspace.  Called through the C ABI, it must return the same X^T X as the
+allocating admmq_build_hessian (within the 1e-4 relative Frobenius tolerance
+the Gram tests use), on two calls in a row, since the shared array keeps the
+previous call's contents; and it must refuse a d_in whose partial sums do not
+fit, before launching anything.
+
+This file is collected last so that a run stopping at the first failure has
+run every other test already.
+"""
+import ctypes
+
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+ERR_WORKSPACE = -7
+
+
+def _entry():
+    from post_weight_quantization_10_b200 import admmq
+    f = admmq.lib().admmq_build_hessian_static
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_int,
+                  ctypes.c_void_p]
+    return admmq, f
+
+
+def _acts(n, d, seed):
+    from post_weight_quantization_10_b200 import workloads
+    p = workloads.scaled(workloads.PRESETS["q_proj"], n, d, 8, rank=8)
+    return workloads.make_activations(p, seed=seed, device="cuda")
+
+
+def test_static_gram_equals_allocating_gram_twice():
+    admmq, f = _entry()
+    stream = torch.cuda.current_stream().cuda_stream
+    n, d = 5000, 384
+    for seed in (11, 12):      # two calls in a row on the shared scratch
+        X = _acts(n, d, seed)
+        ref = admmq.build_hessian(X)
+        H = torch.full((d, d), float("nan"), dtype=torch.float32, device="cuda")
+        assert f(X.data_ptr(), n, d, H.data_ptr(), 0, stream) == 0
+        torch.cuda.synchronize()
+        assert torch.isfinite(H).all()
+        assert torch.equal(H, H.T)
+        err = float((H.double() - ref.double()).norm() / ref.double().norm())
+        assert err <= 1e-4, err
+
+
+def test_static_gram_accumulate_and_limit():
+    admmq, f = _entry()
+    stream = torch.cuda.current_stream().cuda_stream
+    n, d = 3000, 256
+    X = _acts(n, d, 13)
+    ref = admmq.build_hessian(X)
+    H = torch.empty((d, d), dtype=torch.float32, device="cuda")
+    assert f(X[:1200].data_ptr(), 1200, d, H.data_ptr(), 0, stream) == 0
+    assert f(X[1200:].data_ptr(), n - 1200, d, H.data_ptr(), 1, stream) == 0
+    torch.cuda.synchronize()
+    err = float((H.double() - ref.double()).norm() / ref.double().norm())
+    assert err <= 1e-4, err
+    # d_in = 4128: 4128^2 * 4 bytes of partial sums exceed the fixed scratch
+    big = torch.zeros((16, 4128), dtype=torch.bfloat16, device="cuda")
+    Hb = torch.zeros(1, dtype=torch.float32, device="cuda")
+    assert f(big.data_ptr(), 16, 4128, Hb.data_ptr(), 0, stream) == ERR_WORKSPACE
+    # the largest supported width still works
+    Xw = _acts(700, 4096, 14)
+    Hw = admmq.build_hessian(Xw)
+    H2 = torch.empty_like(Hw)
+    assert f(Xw.data_ptr(), 700, 4096, H2.data_ptr(), 0, stream) == 0
+    torch.cuda.synchronize()
+    err = float((H2.double() - Hw.double()).norm() / Hw.double().norm())
+    assert err <= 1e-4, err
