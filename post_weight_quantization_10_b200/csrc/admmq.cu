@@ -24,9 +24,11 @@ constexpr int kBM = 128;
 unsigned long long g_launches = 0;  // kernels launched by this library
 inline void count_launch() { __atomic_fetch_add(&g_launches, 1ull, __ATOMIC_RELAXED); }
 // X^T X: bf16, both operands MN-major (X is token-major).
-using GramCfg = GemmCfg<KIND_BF16, 256, 1, true, true, 4>;
+// Promoted every 4 k-blocks (16 MMAs of K = 16).
+using GramCfg = GemmCfg<KIND_BF16, 256, 1, true, true, 4, 4>;
 // Eigenbasis GEMMs: 3xTF32 split precision, K-major operands.
-using EigCfg = GemmCfg<KIND_TF32, 128, 2, false, false, 3>;
+// Promoted every 2 k-blocks (24 MMAs of K = 8).
+using EigCfg = GemmCfg<KIND_TF32, 128, 2, false, false, 3, 2>;
 
 // Setup status words (ws status[1]).
 enum { SETUP_OK = 0, SETUP_NONFINITE = 1, SETUP_NOT_PD = 2 };
@@ -439,6 +441,7 @@ GemmGeom make_geom(int M, int N, long long K, int BN, int BK, int splits, bool t
     g.tiles = t;
   }
   g.units = g.tiles * splits;
+  g.band = g.tiles_m < 12 ? g.tiles_m : 12;  // 12 x 12 tiles in flight ~ 100 MB of operands
   g.status = status;
   return g;
 }
@@ -453,7 +456,7 @@ cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
   int grid = g.units < num_sms() ? g.units : num_sms();
   if (grid <= 0) return cudaSuccess;
   count_launch();
-  kern<<<grid, 192, Cfg::SMEM, st>>>(a0, a1, b0, b1, g, ep);
+  kern<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(a0, a1, b0, b1, g, ep);
   return cudaGetLastError();
 }
 

@@ -1,22 +1,32 @@
 // gemm.cuh -- persistent tcgen05 GEMM engine for sm_100a.
 //
 // D[M x N] = A[M x K] * B[K x N] with operands staged in shared memory by TMA
-// (128-byte swizzle, no multicast) and fp32 accumulators in tensor memory.
-// Operands are bf16 (kind::f16) or tf32 held in fp32 words (kind::tf32); a
-// shared-memory row is always 128 bytes (64 bf16 or 32 fp32 along K) and one
-// MMA always consumes 32 bytes of K.
-// NPL = 2 runs the split-precision product used for fp32-accurate GEMMs
+// (128-byte swizzle, no multicast) and fp32 accumulation.  Operands are bf16
+// (kind::f16) or tf32 held in fp32 words (kind::tf32); a shared-memory row is
+// always 128 bytes (64 bf16 or 32 fp32 along K) and one MMA consumes 32 bytes
+// of K.  NPL = 2 runs the split-precision product used for fp32-accurate GEMMs
 // (3xTF32): every operand is stored as two tf32 planes (hi, lo) with
-// x ~= hi + lo, and each k-step issues A_hi*B_hi + A_hi*B_lo + A_lo*B_hi into
-// one accumulator.
+// x ~= hi + lo, and each k-step issues A_hi*B_hi + A_hi*B_lo + A_lo*B_hi.
 //
-// Warp roles (192 threads, one CTA per SM):
+// Promoted accumulation.  The tensor core adds every MMA into its fp32
+// accumulator with a small one-sided rounding error, so a long K sum drifts by
+// a relative amount proportional to the number of MMAs (measured 2.9e-5 for
+// K = 4096 with 3xTF32).  The MMA therefore writes each chunk of KC k-blocks
+// into a fresh tensor-memory slot, and the consumer warps add the chunks into
+// fp32 registers with round-to-nearest: the drift is bounded by one chunk.
+//
+// Warp roles (320 threads, one CTA per SM, 512 tensor-memory columns):
 //   warp 0      TMA producer (one thread)
 //   warp 1      tensor-memory owner and MMA issuer (one thread)
-//   warps 2..5  epilogue: thread = accumulator row, reads 32 columns at a time
-// The accumulator is double-buffered (2 x BN columns) so the epilogue of one
-// tile overlaps the main loop of the next.  Work units (tile, k-split) are
-// dealt to CTAs round-robin; all waits are bounded (see ptx.cuh).
+//   warps 2..9  two consumer warpgroups; thread = accumulator row
+//     BN = 128: the warpgroups take alternate tiles; the owner adds the chunks
+//               from a 2-slot ring, writes the sum to its private final slot
+//               and runs the tile epilogue from there, while the other
+//               warpgroup accumulates the next tile.
+//     BN = 256: both warpgroups take every tile, 128 columns each, and store
+//               the tile from registers (Gram partial sums).
+// Work units (tile, k-split) are dealt to CTAs round-robin; all waits are
+// bounded (see ptx.cuh).
 #pragma once
 #include "ptx.cuh"
 
@@ -30,23 +40,27 @@ struct GemmGeom {
   int triangle;       // 1: only tiles that meet the upper triangle (i <= j)
   int tiles;          // number of tiles visited
   int units;          // tiles * splits
+  int band;           // tile rows per band of the visiting order (L2 reuse)
   int* status;        // kernel status word (device)
 };
 
 enum { KIND_BF16 = 1, KIND_TF32 = 2 };  // instruction-descriptor operand format
 
-template <int KIND_, int BN_, int NPL_, bool A_MN_, bool B_MN_, int STAGES_>
+template <int KIND_, int BN_, int NPL_, bool A_MN_, bool B_MN_, int STAGES_, int KC_>
 struct GemmCfg {
   static constexpr int KIND = KIND_;
   static constexpr int ELEM = KIND == KIND_BF16 ? 2 : 4;  // bytes per operand element
   static constexpr int BM = 128, BN = BN_, BK = 128 / ELEM, NPL = NPL_, STAGES = STAGES_;
   static constexpr int UK = 32 / ELEM;                     // K per MMA instruction
+  static constexpr int KC = KC_;                           // k-blocks per promoted chunk
   static constexpr bool A_MN = A_MN_, B_MN = B_MN_;
+  static constexpr bool SPLITCOL = BN == 256;
   static constexpr int A_PLANE = BM * 128;  // bytes per operand plane per stage
   static constexpr int B_PLANE = BN * 128;
   static constexpr int STAGE = NPL * (A_PLANE + B_PLANE);
-  static constexpr int TMEM_COLS = 2 * BN;
-  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5) + 16;
+  static constexpr int TMEM_COLS = 512;     // ring 2 x BN (+ final 2 x 128 when BN = 128)
+  static constexpr int THREADS = 320;
+  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 9) + 16;
   static constexpr int SMEM = STAGES * STAGE + 1024 + BAR_BYTES;
   static_assert(BN == 128 || BN == 256, "BN must be 128 or 256");
   static_assert(SMEM <= 232448, "shared memory budget");
@@ -54,15 +68,20 @@ struct GemmCfg {
 
 // Unit -> (tile row, tile column, k-block range).  Splits are the outer index
 // so that CTAs running at the same time work on the same k-range of different
-// tiles (their A and B panels share L2).
+// tiles.  Full grids are visited in bands of `band` tile rows, column by
+// column inside a band, so that the tiles in flight share A rows and B
+// columns in L2.
 template <int BM, int BN>
 __device__ __forceinline__ void decode_unit(const GemmGeom& g, int u, int& tm, int& tn, int& split,
                                             int& kb0, int& kb1) {
   split = u / g.tiles;
   int t = u - split * g.tiles;
   if (!g.triangle) {
-    tm = t % g.tiles_m;
-    tn = t / g.tiles_m;
+    const int b = t / (g.band * g.tiles_n);
+    const int rows = min(g.band, g.tiles_m - b * g.band);
+    const int r = t - b * g.band * g.tiles_n;
+    tn = r / rows;
+    tm = b * g.band + (r - tn * rows);
   } else {
     tn = 0;
     for (;;) {
@@ -79,20 +98,24 @@ __device__ __forceinline__ void decode_unit(const GemmGeom& g, int u, int& tm, i
 }
 
 template <class Cfg, class Epi>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     k_gemm(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ CUtensorMap tA1,
            const __grid_constant__ CUtensorMap tB0, const __grid_constant__ CUtensorMap tB1,
            const GemmGeom g, const typename Epi::Params ep) {
-  constexpr int BM = Cfg::BM, BN = Cfg::BN, STAGES = Cfg::STAGES, NPL = Cfg::NPL;
+  constexpr int BM = Cfg::BM, BN = Cfg::BN, STAGES = Cfg::STAGES, NPL = Cfg::NPL, KC = Cfg::KC;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
-  uint64_t* tfull = bars + 2 * STAGES;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
+  // Ring-slot barriers per (consumer warpgroup, slot): [2 * wg + slot].  Each
+  // warpgroup waits only on its own chunks, in order, so no waiter is ever
+  // more than one phase away from its barrier.  (BN = 256 uses wg 0 only:
+  // both warpgroups consume every chunk.)
+  uint64_t* rfull = bars + 2 * STAGES;  // slot holds a finished chunk
+  uint64_t* rempty = rfull + 4;         // slot drained by its consumers
+  uint64_t* drain = rempty + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -103,9 +126,9 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1);
     }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(smem_u32(&tfull[a]), 1);
-      mbar_init(smem_u32(&tempty[a]), 128);
+    for (int a = 0; a < 4; ++a) {
+      mbar_init(smem_u32(&rfull[a]), 1);
+      mbar_init(smem_u32(&rempty[a]), Cfg::SPLITCOL ? 256 : 128);
     }
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
@@ -152,7 +175,8 @@ __global__ void __launch_bounds__(192, 1)
               tma_load_2d(dA, mapA[p], k0, tm * BM, fb);
             } else {
 #pragma unroll
-              for (int b = 0; b < BM / (128 / Cfg::ELEM); ++b) tma_load_2d(dA + b * Cfg::BK * 128, mapA[p], tm * BM + (128 / Cfg::ELEM) * b, k0, fb);
+              for (int b = 0; b < BM / (128 / Cfg::ELEM); ++b)
+                tma_load_2d(dA + b * Cfg::BK * 128, mapA[p], tm * BM + (128 / Cfg::ELEM) * b, k0, fb);
             }
           }
 #pragma unroll
@@ -162,7 +186,8 @@ __global__ void __launch_bounds__(192, 1)
               tma_load_2d(dB, mapB[p], k0, tn * BN, fb);
             } else {
 #pragma unroll
-              for (int b = 0; b < BN / (128 / Cfg::ELEM); ++b) tma_load_2d(dB + b * Cfg::BK * 128, mapB[p], tn * BN + (128 / Cfg::ELEM) * b, k0, fb);
+              for (int b = 0; b < BN / (128 / Cfg::ELEM); ++b)
+                tma_load_2d(dB + b * Cfg::BK * 128, mapB[p], tn * BN + (128 / Cfg::ELEM) * b, k0, fb);
             }
           }
         }
@@ -181,69 +206,122 @@ __global__ void __launch_bounds__(192, 1)
       constexpr uint32_t LBO_A = Cfg::A_MN ? Cfg::BK * 128 : 16;
       constexpr uint32_t LBO_B = Cfg::B_MN ? Cfg::BK * 128 : 16;
       int it = 0, lu = 0;
+      uint32_t q = 0;                      // chunks issued by this CTA
+      uint32_t use[4] = {0, 0, 0, 0};      // chunks issued per (warpgroup, slot)
+      int prev[2] = {-1, -1};              // warpgroup of the chunk last put in a slot
       bool ok = true;
       for (int u = blockIdx.x; u < g.units && ok; u += gridDim.x, ++lu) {
         int tm, tn, split, kb0, kb1;
         decode_unit<BM, BN>(g, u, tm, tn, split, kb0, kb1);
-        const int acc = lu & 1;
-        const uint32_t aph = (uint32_t)(lu >> 1) & 1u;
-        if (!mbar_wait(smem_u32(&tempty[acc]), aph ^ 1u, abort_flag, g.status)) break;
-        tc_fence_after();
-        const uint32_t dt = tmem_base + (uint32_t)(acc * BN);
-        for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!mbar_wait(smem_u32(&full[s]), ph, abort_flag, g.status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t st = smem_u32(smem + s * Cfg::STAGE);
-#pragma unroll
-          for (int kk = 0; kk < Cfg::BK / Cfg::UK; ++kk) {
-#pragma unroll
-            for (int pr = 0; pr < (NPL == 2 ? 3 : 1); ++pr) {
-              const int pa = (pr == 2) ? 1 : 0;  // (hi,hi), (hi,lo), (lo,hi)
-              const int pb = (pr == 1) ? 1 : 0;
-              const uint32_t a_addr =
-                  st + pa * Cfg::A_PLANE + (Cfg::A_MN ? kk * Cfg::UK * 128 : kk * 32);
-              const uint32_t b_addr = st + NPL * Cfg::A_PLANE + pb * Cfg::B_PLANE +
-                                      (Cfg::B_MN ? kk * Cfg::UK * 128 : kk * 32);
-              const uint64_t ad = smem_desc_sw128(a_addr, LBO_A, 1024);
-              const uint64_t bd = smem_desc_sw128(b_addr, LBO_B, 1024);
-              const uint32_t accum = (kb > kb0 || kk > 0 || pr > 0) ? 1u : 0u;
-              if (Cfg::KIND == KIND_BF16)
-                mma_bf16(dt, ad, bd, IDESC, accum);
-              else
-                mma_tf32(dt, ad, bd, IDESC, accum);
+        const int owner = Cfg::SPLITCOL ? 0 : (lu & 1);
+        for (int c0 = kb0; c0 < kb1 && ok; c0 += KC, ++q) {
+          const int c1 = min(c0 + KC, kb1);
+          const uint32_t slot = q & 1u;
+          if (prev[slot] >= 0) {
+            // wait until the slot's previous chunk has been drained
+            const int b = 2 * prev[slot] + (int)slot;
+            if (!mbar_wait(smem_u32(&rempty[b]), (use[b] - 1u) & 1u, abort_flag, g.status)) {
+              ok = false;
+              break;
             }
           }
-          mma_commit(smem_u32(&empty[s]));
+          tc_fence_after();
+          const uint32_t dt = tmem_base + slot * BN;
+          for (int kb = c0; kb < c1; ++kb, ++it) {
+            const int s = it % STAGES;
+            const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+            if (!mbar_wait(smem_u32(&full[s]), ph, abort_flag, g.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t st = smem_u32(smem + s * Cfg::STAGE);
+#pragma unroll
+            for (int kk = 0; kk < Cfg::BK / Cfg::UK; ++kk) {
+#pragma unroll
+              for (int pr = 0; pr < (NPL == 2 ? 3 : 1); ++pr) {
+                const int pa = (pr == 2) ? 1 : 0;  // (hi,hi), (hi,lo), (lo,hi)
+                const int pb = (pr == 1) ? 1 : 0;
+                const uint32_t a_addr =
+                    st + pa * Cfg::A_PLANE + (Cfg::A_MN ? kk * Cfg::UK * 128 : kk * 32);
+                const uint32_t b_addr = st + NPL * Cfg::A_PLANE + pb * Cfg::B_PLANE +
+                                        (Cfg::B_MN ? kk * Cfg::UK * 128 : kk * 32);
+                const uint64_t ad = smem_desc_sw128(a_addr, LBO_A, 1024);
+                const uint64_t bd = smem_desc_sw128(b_addr, LBO_B, 1024);
+                const uint32_t accum = (kb > c0 || kk > 0 || pr > 0) ? 1u : 0u;
+                if (Cfg::KIND == KIND_BF16)
+                  mma_bf16(dt, ad, bd, IDESC, accum);
+                else
+                  mma_tf32(dt, ad, bd, IDESC, accum);
+              }
+            }
+            mma_commit(smem_u32(&empty[s]));
+          }
+          if (!ok) break;
+          const int b = 2 * owner + (int)slot;
+          mma_commit(smem_u32(&rfull[b]));
+          ++use[b];
+          prev[slot] = owner;
         }
-        if (!ok) break;
-        mma_commit(smem_u32(&tfull[acc]));
       }
       // Every MMA issued above is complete once this arrives.
       mma_commit(smem_u32(drain));
       mbar_wait_drain(smem_u32(drain), 0);
     }
   } else {
-    // ----------------------------------------------------------- epilogue
-    const int q = warp & 3;  // tensor-memory lane quarter this warp may access
+    // ---------------------------------------------------------- consumers
+    const int wg = (warp - 2) >> 2;  // consumer warpgroup 0 or 1
+    const int qtr = warp & 3;        // tensor-memory lane quarter this warp may access
+    const uint32_t lane_off = (uint32_t)(qtr * 32) << 16;
+    const uint32_t col_off = Cfg::SPLITCOL ? (uint32_t)(wg * 128) : 0u;
+    const int bw = Cfg::SPLITCOL ? 0 : wg;  // barrier set of this warpgroup
+    uint32_t q = 0;
+    uint32_t my_use[2] = {0, 0};            // own chunks consumed per slot
     int lu = 0;
-    for (int u = blockIdx.x; u < g.units; u += gridDim.x, ++lu) {
+    bool ok = true;
+    for (int u = blockIdx.x; u < g.units && ok; u += gridDim.x, ++lu) {
       int tm, tn, split, kb0, kb1;
       decode_unit<BM, BN>(g, u, tm, tn, split, kb0, kb1);
-      const int acc = lu & 1;
-      const uint32_t aph = (uint32_t)(lu >> 1) & 1u;
-      // warp-uniform decision: tcgen05.ld below needs all 32 lanes
-      const bool ok = mbar_wait(smem_u32(&tfull[acc]), aph, abort_flag, g.status);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
-      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      Epi::apply(ep, g, taddr, tm, tn, split, q, lane);
-      tc_fence_before();
-      mbar_arrive(smem_u32(&tempty[acc]));
+      const bool mine = Cfg::SPLITCOL || ((lu & 1) == wg);
+      float acc[128];
+#pragma unroll
+      for (int i = 0; i < 128; ++i) acc[i] = 0.f;
+      for (int c0 = kb0; c0 < kb1; c0 += KC, ++q) {
+        if (!mine) continue;
+        const uint32_t slot = q & 1u;
+        const int b = 2 * bw + (int)slot;
+        const bool got = mbar_wait(smem_u32(&rfull[b]), my_use[slot] & 1u, abort_flag, g.status);
+        if (!__all_sync(0xffffffffu, got)) {  // tcgen05.ld needs all 32 lanes
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t ta = tmem_base + lane_off + slot * BN + col_off;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float v[16];
+          tmem_ld16(ta + 16 * j, v);
+#pragma unroll
+          for (int k = 0; k < 16; ++k) acc[16 * j + k] += v[k];
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&rempty[b]));
+        ++my_use[slot];
+      }
+      if (!ok || !mine) continue;
+      if constexpr (Cfg::SPLITCOL) {
+        Epi::apply_regs(ep, g, acc, tm, tn, split, qtr * 32 + lane, tn * BN + wg * 128);
+      } else {
+        const uint32_t fin = tmem_base + lane_off + 2 * BN + wg * 128;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float v[32];
+#pragma unroll
+          for (int k = 0; k < 32; ++k) v[k] = acc[32 * j + k];
+          tmem_st32(fin + 32 * j, v);
+        }
+        Epi::apply(ep, g, fin, tm, tn, split, qtr, lane);
+      }
     }
   }
   __syncthreads();

@@ -203,6 +203,24 @@ struct EpiGramPartial {
     long long split_stride;  // elements between k-split buffers
     int ld;
   };
+  // From registers: 128 columns starting at col0 of tile row `rit`.
+  __device__ static void apply_regs(const Params& p, const GemmGeom& g, const float (&acc)[128],
+                                    int tm, int, int split, int rit, int col0) {
+    const int row = tm * 128 + rit;
+    if (row >= g.M) return;
+    float* out = p.part + split * p.split_stride + (long long)row * p.ld;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int col = col0 + 32 * j;
+      if (col < g.N) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          *reinterpret_cast<float4*>(out + col + 4 * k) =
+              make_float4(acc[32 * j + 4 * k], acc[32 * j + 4 * k + 1], acc[32 * j + 4 * k + 2],
+                          acc[32 * j + 4 * k + 3]);
+      }
+    }
+  }
   __device__ static void apply(const Params& p, const GemmGeom& g, uint32_t taddr, int tm, int tn,
                                int split, int q, int lane) {
     const int row = tm * 128 + q * 32 + lane;
