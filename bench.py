@@ -31,6 +31,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from post_weight_quantization_10_b200 import dist as D  # noqa: E402
 from post_weight_quantization_10_b200 import workloads  # noqa: E402
 
 METRIC = "ADMM-Q layer solve: iters/s, TFLOP/s vs tensor peak; Gram TFLOP/s; s/layer"
@@ -365,16 +366,11 @@ def run_reference(args, rank, world):
 
 
 def dist_barrier(world):
-    if world > 1:
-        torch.distributed.barrier()
+    D.barrier(world)
 
 
 def dist_max(v, world, device):
-    if world == 1:
-        return v
-    t = torch.tensor([v], dtype=torch.float64, device=device)
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    return float(t.item())
+    return D.max_over_ranks(v, world, device)
 
 
 def main():
@@ -391,9 +387,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = D.world()
     if args.impl == "reference":
         line = run_reference(args, rank, world)
         if line:
