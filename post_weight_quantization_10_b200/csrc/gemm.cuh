@@ -20,11 +20,13 @@
 //   warp 1      tensor-memory owner and MMA issuer (one thread)
 //   warps 2..9  two consumer warpgroups; thread = accumulator row
 //     BN = 128: the warpgroups take alternate tiles; the owner adds the chunks
-//               from a 2-slot ring, writes the sum to its private final slot
-//               and runs the tile epilogue from there, while the other
-//               warpgroup accumulates the next tile.
-//     BN = 256: both warpgroups take every tile, 128 columns each, and store
-//               the tile from registers (Gram partial sums).
+//               from a 3-slot ring, writes the sum to the final slot and runs
+//               the tile epilogue from there, while the other warpgroup
+//               accumulates the next tile.  The final slot passes from one
+//               tile's owner to the next through the `fin` barrier.
+//     BN = 256: both warpgroups take every tile, 128 columns each, from a
+//               2-slot ring, and store the tile from registers (Gram partial
+//               sums).
 // Work units (tile, k-split) are dealt to CTAs round-robin; all waits are
 // bounded (see ptx.cuh).
 #pragma once
@@ -58,9 +60,10 @@ struct GemmCfg {
   static constexpr int A_PLANE = BM * 128;  // bytes per operand plane per stage
   static constexpr int B_PLANE = BN * 128;
   static constexpr int STAGE = NPL * (A_PLANE + B_PLANE);
-  static constexpr int TMEM_COLS = 512;     // ring 2 x BN (+ final 2 x 128 when BN = 128)
+  static constexpr int RING = SPLITCOL ? 2 : 3;  // chunk slots in tensor memory
+  static constexpr int TMEM_COLS = 512;          // RING x BN (+ one final 128-column slot)
   static constexpr int THREADS = 320;
-  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 9) + 16;
+  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 4 * RING + 2) + 16;
   static constexpr int SMEM = STAGES * STAGE + 1024 + BAR_BYTES;
   static_assert(BN == 128 || BN == 256, "BN must be 128 or 256");
   static_assert(SMEM <= 232448, "shared memory budget");
@@ -113,9 +116,11 @@ __global__ void __launch_bounds__(320, 1)
   // warpgroup waits only on its own chunks, in order, so no waiter is ever
   // more than one phase away from its barrier.  (BN = 256 uses wg 0 only:
   // both warpgroups consume every chunk.)
-  uint64_t* rfull = bars + 2 * STAGES;  // slot holds a finished chunk
-  uint64_t* rempty = rfull + 4;         // slot drained by its consumers
-  uint64_t* drain = rempty + 4;
+  constexpr int R = Cfg::RING;
+  uint64_t* rfull = bars + 2 * STAGES;  // [R * wg + slot]: slot holds a finished chunk
+  uint64_t* rempty = rfull + 2 * R;     // [R * wg + slot]: slot drained by its consumers
+  uint64_t* fin = rempty + 2 * R;       // final slot released by the previous tile's owner
+  uint64_t* drain = fin + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -126,10 +131,11 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1);
     }
-    for (int a = 0; a < 4; ++a) {
+    for (int a = 0; a < 2 * R; ++a) {
       mbar_init(smem_u32(&rfull[a]), 1);
       mbar_init(smem_u32(&rempty[a]), Cfg::SPLITCOL ? 256 : 128);
     }
+    mbar_init(smem_u32(fin), 128);
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -207,8 +213,10 @@ __global__ void __launch_bounds__(320, 1)
       constexpr uint32_t LBO_B = Cfg::B_MN ? Cfg::BK * 128 : 16;
       int it = 0, lu = 0;
       uint32_t q = 0;                      // chunks issued by this CTA
-      uint32_t use[4] = {0, 0, 0, 0};      // chunks issued per (warpgroup, slot)
-      int prev[2] = {-1, -1};              // warpgroup of the chunk last put in a slot
+      uint32_t use[2 * R] = {};            // chunks issued per (warpgroup, slot)
+      int prev[R];                         // warpgroup of the chunk last put in a slot
+#pragma unroll
+      for (int i = 0; i < R; ++i) prev[i] = -1;
       bool ok = true;
       for (int u = blockIdx.x; u < g.units && ok; u += gridDim.x, ++lu) {
         int tm, tn, split, kb0, kb1;
@@ -216,10 +224,10 @@ __global__ void __launch_bounds__(320, 1)
         const int owner = Cfg::SPLITCOL ? 0 : (lu & 1);
         for (int c0 = kb0; c0 < kb1 && ok; c0 += KC, ++q) {
           const int c1 = min(c0 + KC, kb1);
-          const uint32_t slot = q & 1u;
+          const uint32_t slot = q % R;
           if (prev[slot] >= 0) {
             // wait until the slot's previous chunk has been drained
-            const int b = 2 * prev[slot] + (int)slot;
+            const int b = R * prev[slot] + (int)slot;
             if (!mbar_wait(smem_u32(&rempty[b]), (use[b] - 1u) & 1u, abort_flag, g.status)) {
               ok = false;
               break;
@@ -258,7 +266,7 @@ __global__ void __launch_bounds__(320, 1)
             mma_commit(smem_u32(&empty[s]));
           }
           if (!ok) break;
-          const int b = 2 * owner + (int)slot;
+          const int b = R * owner + (int)slot;
           mma_commit(smem_u32(&rfull[b]));
           ++use[b];
           prev[slot] = owner;
@@ -276,7 +284,7 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t col_off = Cfg::SPLITCOL ? (uint32_t)(wg * 128) : 0u;
     const int bw = Cfg::SPLITCOL ? 0 : wg;  // barrier set of this warpgroup
     uint32_t q = 0;
-    uint32_t my_use[2] = {0, 0};            // own chunks consumed per slot
+    uint32_t my_use[R] = {};                // own chunks consumed per slot
     int lu = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < g.units && ok; u += gridDim.x, ++lu) {
@@ -288,8 +296,8 @@ __global__ void __launch_bounds__(320, 1)
       for (int i = 0; i < 128; ++i) acc[i] = 0.f;
       for (int c0 = kb0; c0 < kb1; c0 += KC, ++q) {
         if (!mine) continue;
-        const uint32_t slot = q & 1u;
-        const int b = 2 * bw + (int)slot;
+        const uint32_t slot = q % R;
+        const int b = R * bw + (int)slot;
         const bool got = mbar_wait(smem_u32(&rfull[b]), my_use[slot] & 1u, abort_flag, g.status);
         if (!__all_sync(0xffffffffu, got)) {  // tcgen05.ld needs all 32 lanes
           ok = false;
@@ -312,15 +320,27 @@ __global__ void __launch_bounds__(320, 1)
       if constexpr (Cfg::SPLITCOL) {
         Epi::apply_regs(ep, g, acc, tm, tn, split, qtr * 32 + lane, tn * BN + wg * 128);
       } else {
-        const uint32_t fin = tmem_base + lane_off + 2 * BN + wg * 128;
+        // The final slot is free once the previous tile's owner (the other
+        // warpgroup) has finished its epilogue: phase lu - 1 of `fin`.
+        if (lu > 0) {
+          const bool freed = mbar_wait(smem_u32(fin), (uint32_t)(lu - 1) & 1u, abort_flag, g.status);
+          if (!__all_sync(0xffffffffu, freed)) {
+            ok = false;
+            continue;
+          }
+          tc_fence_after();
+        }
+        const uint32_t fslot = tmem_base + lane_off + R * BN;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           float v[32];
 #pragma unroll
           for (int k = 0; k < 32; ++k) v[k] = acc[32 * j + k];
-          tmem_st32(fin + 32 * j, v);
+          tmem_st32(fslot + 32 * j, v);
         }
-        Epi::apply(ep, g, fin, tm, tn, split, qtr, lane);
+        Epi::apply(ep, g, fslot, tm, tn, split, qtr, lane);
+        tc_fence_before();
+        mbar_arrive(smem_u32(fin));
       }
     }
   }
