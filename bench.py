@@ -48,6 +48,27 @@ def peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, src="fallback")
 
 
+def source_hash():
+    """Short hash of the CUDA sources (matches the ncu captures in profiles/)."""
+    import hashlib
+    csrc = os.path.join(ROOT, "post_weight_quantization_10_b200", "csrc")
+    per = [hashlib.sha1(open(os.path.join(csrc, f), "rb").read()).hexdigest() + "  " + f
+           for f in sorted(os.listdir(csrc)) if f.endswith((".cu", ".cuh"))]
+    return hashlib.sha1(("\n".join(per) + "\n").encode()).hexdigest()[:12]
+
+
+def measured_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu capture, or None when the
+    kernel sources changed since that capture."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            t = json.load(f)[kernel]
+    except (OSError, KeyError, ValueError):
+        return None
+    return t["dram_bytes_per_launch"] if t["source_hash"] == source_hash() else None
+
+
 def workload_desc(p, grid):
     return (f"{p.name}: d_in={p.d_in} d_out={p.d_out} n={p.n} W{p.bits} g{p.group} T={p.iters} "
             f"grid={grid} (Qwen3-8B-shaped synthetic layer, seed=rank)")
@@ -236,7 +257,8 @@ def run_ours(args, rank, world, device):
         "gemm_ms_per_launch": [gemm_ms[0] / max(gemm_n[0], 1), gemm_ms[1] / max(gemm_n[1], 1)],
         "roofline": {"kernel": ["gemm1_eigscale", "gemm2_project"][k], "bound": "tensor",
                      "achieved": achieved, "peak": peak_split, "unit": "TFLOP/s",
-                     "frac": achieved / peak_split, "traffic": None,
+                     "frac": achieved / peak_split,
+                     "traffic": measured_traffic(["gemm1_eigscale", "gemm2_project"][k]),
                      "peak_note": "bf16 dense %s sustained %.1f TF/s x 1/2 (tf32) / 3 (three "
                                   "tf32 MMAs per fp32-accurate product)" % (pk["src"], pk["bf16_sust"])},
         "gpu_launches": launches,
