@@ -154,7 +154,9 @@ int admmq_setup(admmq_ctx** ctx_out, const float* G_dev, const void* W_hat_dev, 
 
 /* Start of the iteration: C0' = Lambda Q^T W^~ (so that Q^T H~ W^~ = C0') and
  * the RTN start D_0 = RTN(W_hat) on its min/max grid, V~_0 = 0.
- *   codes_dev  u8 [d_out][d_in]; scale_dev, zero_dev fp32 [d_out][d_in/group]. */
+ *   codes_dev  u8 [d_out][d_in], 32-byte aligned (the epilogues move 32 codes
+ *              per 256-bit access); scale_dev, zero_dev fp32 [d_out][d_in/group].
+ * A misaligned codes_dev returns ADMMQ_ERR_INVALID_ARG (also for iterate). */
 int admmq_init(admmq_ctx* ctx, uint8_t* codes_dev, float* scale_dev, float* zero_dev,
                void* stream);
 
@@ -205,7 +207,8 @@ int admmq_get_buffer(admmq_ctx* ctx, int which, void** ptr_dev, size_t* bytes);
 
 /* When wtilde_dev is non-NULL, the next GEMM-2 launches also write the raw
  * fp32 product W~ [d_out][d_in] there (tests compare the fused projection with
- * its float32 specification on exactly these values).  NULL turns it off. */
+ * its float32 specification on exactly these values).  NULL turns it off;
+ * a pointer that is not 32-byte aligned returns ADMMQ_ERR_INVALID_ARG. */
 int admmq_debug_dump_wtilde(admmq_ctx* ctx, float* wtilde_dev);
 
 /* Per-kernel timing with CUDA events recorded on the launch stream around
@@ -220,7 +223,10 @@ int admmq_get_timing(admmq_ctx* ctx, double ms[2], int launches[2]);
  * All pointers device; V_dev is updated in place; P_hi/P_lo receive P as
  * tf32 hi/lo planes in fp32 words (hi = tf32(P), lo = tf32(P - hi));
  * codes/scale/zero hold the previous D on entry and the new D on exit;
- * resid_dev fp64 [2] receives the two residual sums of squares. */
+ * resid_dev fp64 [2] receives the two residual sums of squares.
+ * V_dev, codes_dev, P_hi_dev, P_lo_dev, sigma_dev, rsig_dev and hdiag_dev
+ * must be 32-byte aligned, wtilde_dev 16-byte aligned (ADMMQ_ERR_INVALID_ARG
+ * otherwise). */
 int admmq_project(const float* wtilde_dev, float* V_dev, const float* sigma_dev,
                   const float* rsig_dev, const float* hdiag_dev, int d_in, int d_out, int bits,
                   int group, int grid_mode, uint8_t* codes_dev, float* scale_dev, float* zero_dev,

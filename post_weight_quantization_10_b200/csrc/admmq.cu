@@ -494,6 +494,7 @@ int gram_splits(long long n, int d, int nsm) {
 }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+bool aligned32(const void* p) { return ((uintptr_t)p & 31) == 0; }
 
 }  // namespace
 
@@ -808,6 +809,7 @@ int admmq_setup(admmq_ctx** out, const float* G, const void* W_hat, int w_dtype,
 
 int admmq_init(admmq_ctx* c, uint8_t* codes, float* scale, float* zero, void* stream) {
   if (!c || !c->eig_done || !codes || !scale || !zero) return ADMMQ_ERR_INVALID_ARG;
+  if (!aligned32(codes)) return ADMMQ_ERR_INVALID_ARG;
   cudaStream_t st = (cudaStream_t)stream;
   const int d = c->d, m = c->m;
   // C0' = Lambda Q^T W^~   (row j, column k)
@@ -832,6 +834,7 @@ int admmq_init(admmq_ctx* c, uint8_t* codes, float* scale, float* zero, void* st
 int admmq_iterate(admmq_ctx* c, int t0, int count, uint8_t* codes, float* scale, float* zero,
                   void* stream) {
   if (!c || !c->inited || !codes || !scale || !zero) return ADMMQ_ERR_INVALID_ARG;
+  if (!aligned32(codes)) return ADMMQ_ERR_INVALID_ARG;
   if (t0 < 0 || count < 0 || t0 + count > c->p.iters) return ADMMQ_ERR_INVALID_ARG;
   cudaStream_t st = (cudaStream_t)stream;
   const int d = c->d, m = c->m;
@@ -990,7 +993,7 @@ int admmq_get_buffer(admmq_ctx* c, int which, void** ptr, size_t* bytes) {
 }
 
 int admmq_debug_dump_wtilde(admmq_ctx* c, float* wtilde) {
-  if (!c) return ADMMQ_ERR_INVALID_ARG;
+  if (!c || !aligned32(wtilde)) return ADMMQ_ERR_INVALID_ARG;
   c->wdump = wtilde;
   return ADMMQ_OK;
 }
@@ -1028,6 +1031,9 @@ int admmq_project(const float* wt, float* V, const float* sig, const float* rsig
     return ADMMQ_ERR_INVALID_ARG;
   if (d <= 0 || m <= 0 || d % 32 != 0 || !(g == 32 || g == 64 || g == 128) || d % g != 0 ||
       bits < 1 || bits > 8 || mode < 0 || mode > 2)
+    return ADMMQ_ERR_INVALID_ARG;
+  if (!aligned32(V) || !aligned32(codes) || !aligned32(p_hi) || !aligned32(p_lo) ||
+      ((uintptr_t)wt & 15) || ((uintptr_t)sig & 31) || ((uintptr_t)rsig & 31) || ((uintptr_t)hd & 31))
     return ADMMQ_ERR_INVALID_ARG;
   cudaStream_t st = (cudaStream_t)stream;
   CK(cudaMemsetAsync(resid, 0, 2 * sizeof(double), st));

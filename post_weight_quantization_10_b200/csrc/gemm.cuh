@@ -211,6 +211,12 @@ __global__ void __launch_bounds__(320, 1)
       // MN-major: blocks of 128 bytes along MN, BK K-rows each, LBO apart
       constexpr uint32_t LBO_A = Cfg::A_MN ? Cfg::BK * 128 : 16;
       constexpr uint32_t LBO_B = Cfg::B_MN ? Cfg::BK * 128 : 16;
+      constexpr int kStageStep = Cfg::STAGE >> 4, kAPlane = Cfg::A_PLANE >> 4;
+      constexpr int kBPlane = Cfg::B_PLANE >> 4;
+      constexpr int kKStepA = (Cfg::A_MN ? Cfg::UK * 128 : 32) >> 4;
+      constexpr int kKStepB = (Cfg::B_MN ? Cfg::UK * 128 : 32) >> 4;
+      const uint64_t descA0 = smem_desc_sw128(smem_u32(smem), LBO_A, 1024);
+      const uint64_t descB0 = smem_desc_sw128(smem_u32(smem + NPL * Cfg::A_PLANE), LBO_B, 1024);
       int it = 0, lu = 0;
       uint32_t q = 0;                      // chunks issued by this CTA
       uint32_t use[2 * R] = {};            // chunks issued per (warpgroup, slot)
@@ -243,20 +249,20 @@ __global__ void __launch_bounds__(320, 1)
               break;
             }
             tc_fence_after();
-            const uint32_t st = smem_u32(smem + s * Cfg::STAGE);
+            // descriptors of this stage: the start-address field counts
+            // 16-byte units, so planes, stages and K steps are plain adds
+            const uint64_t a0 = descA0 + (uint64_t)s * kStageStep;
+            const uint64_t b0 = descB0 + (uint64_t)s * kStageStep;
+            const uint32_t acc0 = (kb > c0) ? 1u : 0u;
 #pragma unroll
             for (int kk = 0; kk < Cfg::BK / Cfg::UK; ++kk) {
 #pragma unroll
               for (int pr = 0; pr < (NPL == 2 ? 3 : 1); ++pr) {
                 const int pa = (pr == 2) ? 1 : 0;  // (hi,hi), (hi,lo), (lo,hi)
                 const int pb = (pr == 1) ? 1 : 0;
-                const uint32_t a_addr =
-                    st + pa * Cfg::A_PLANE + (Cfg::A_MN ? kk * Cfg::UK * 128 : kk * 32);
-                const uint32_t b_addr = st + NPL * Cfg::A_PLANE + pb * Cfg::B_PLANE +
-                                        (Cfg::B_MN ? kk * Cfg::UK * 128 : kk * 32);
-                const uint64_t ad = smem_desc_sw128(a_addr, LBO_A, 1024);
-                const uint64_t bd = smem_desc_sw128(b_addr, LBO_B, 1024);
-                const uint32_t accum = (kb > c0 || kk > 0 || pr > 0) ? 1u : 0u;
+                const uint64_t ad = a0 + (uint64_t)(pa * kAPlane + kk * kKStepA);
+                const uint64_t bd = b0 + (uint64_t)(pb * kBPlane + kk * kKStepB);
+                const uint32_t accum = (kk > 0 || pr > 0) ? 1u : acc0;
                 if (Cfg::KIND == KIND_BF16)
                   mma_bf16(dt, ad, bd, IDESC, accum);
                 else

@@ -33,6 +33,14 @@ __device__ __forceinline__ float clampq(float q, float L) {
   return __fadd_rn(fminf(fmaxf(q, 0.f), L), 0.f);
 }
 
+// eight consecutive read-only floats (per-column vectors: sigma, 1/sigma, diag H)
+__device__ __forceinline__ void load8_ro(const float* p, float (&v)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p + 4));
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -83,16 +91,14 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, i
       float w[32];
       loadw(c, w);
 #pragma unroll
-      for (int e = 0; e < 32; e += 4) {
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (r.valid) v = *reinterpret_cast<const float4*>(r.V + c + e);
-        const float4 sg = __ldg(reinterpret_cast<const float4*>(r.sig + c + e));
-        float4 hd = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (MODE == GRID_LSQ) hd = __ldg(reinterpret_cast<const float4*>(r.hd + c + e));
-        const float vv[4] = {v.x, v.y, v.z, v.w}, ss[4] = {sg.x, sg.y, sg.z, sg.w};
-        const float hh[4] = {hd.x, hd.y, hd.z, hd.w};
+      for (int e = 0; e < 32; e += 8) {
+        float vv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (r.valid) ld_v8f(r.V + c + e, vv);
+        float ss[8], hh[8];
+        load8_ro(r.sig + c + e, ss);
+        if (MODE == GRID_LSQ) load8_ro(r.hd + c + e, hh);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < 8; ++k) {
           const float t = __fadd_rn(w[e + k], vv[k]);
           const float y = __fmul_rn(ss[k], t);
           if (MODE == GRID_MINMAX) {
@@ -138,23 +144,19 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, i
   for (int c = 0; c < g; c += 32) {
     float w[32];
     loadw(c, w);
+    uint32_t cw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // the 32 previous codes
+    if (r.valid) ld_v8(r.codes + c, cw);
+    uint32_t qw[8];
 #pragma unroll
-    for (int e = 0; e < 32; e += 4) {
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      uint32_t cp = 0;
-      if (r.valid) {
-        v = *reinterpret_cast<const float4*>(r.V + c + e);
-        cp = *reinterpret_cast<const uint32_t*>(r.codes + c + e);
-      }
-      const float4 sg = __ldg(reinterpret_cast<const float4*>(r.sig + c + e));
-      const float4 rs = __ldg(reinterpret_cast<const float4*>(r.rsig + c + e));
-      const float vv[4] = {v.x, v.y, v.z, v.w}, ss[4] = {sg.x, sg.y, sg.z, sg.w};
-      const float rr[4] = {rs.x, rs.y, rs.z, rs.w};
-      float vn[4];
-      uint32_t qc = 0;
-      float hi[4], lo[4];
+    for (int e = 0; e < 32; e += 8) {
+      float vv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (r.valid) ld_v8f(r.V + c + e, vv);
+      float ss[8], rr[8];
+      load8_ro(r.sig + c + e, ss);
+      load8_ro(r.rsig + c + e, rr);
+      float vn[8], hi[8], lo[8];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+      for (int k = 0; k < 8; ++k) {
         const float t = __fadd_rn(w[e + k], vv[k]);
         const float y = __fmul_rn(ss[k], t);
         const float q = clampq(__fadd_rn(rintf(__fdiv_rn(y, s)), z), Lf);
@@ -163,23 +165,29 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, i
         vn[k] = __fsub_rn(t, dt);
         const float p = __fsub_rn(dt, vn[k]);
         split2(p, hi[k], lo[k]);
-        qc |= (uint32_t)q << (8 * k);
+        const int wi = (e + k) >> 2, sh = 8 * ((e + k) & 3);
+        if (sh == 0) qw[wi] = 0u;
+        qw[wi] |= (uint32_t)q << sh;
         const float e1 = w[e + k] - dt;
         r2 += e1 * e1;
-        const float qp = (float)((cp >> (8 * k)) & 0xFFu);
+        const float qp = (float)((cw[wi] >> sh) & 0xFFu);
         const float dtp = __fmul_rn(__fmul_rn(s0, __fsub_rn(qp, z0)), rr[k]);
         const float e2 = dt - dtp;
         s2 += e2 * e2;
       }
       if (r.valid) {
-        *reinterpret_cast<float4*>(r.V + c + e) = make_float4(vn[0], vn[1], vn[2], vn[3]);
-        *reinterpret_cast<uint32_t*>(r.codes + c + e) = qc;
-        *reinterpret_cast<float4*>(r.phi + c + e) = make_float4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<float4*>(r.plo + c + e) = make_float4(lo[0], lo[1], lo[2], lo[3]);
-        if (r.wdump)
-          *reinterpret_cast<float4*>(r.wdump + c + e) = make_float4(w[e], w[e + 1], w[e + 2], w[e + 3]);
+        st_v8f(r.V + c + e, vn);
+        st_v8f(r.phi + c + e, hi);
+        st_v8f(r.plo + c + e, lo);
+        if (r.wdump) {
+          float wd[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) wd[k] = w[e + k];
+          st_v8f(r.wdump + c + e, wd);
+        }
       }
     }
+    if (r.valid) st_v8(r.codes + c, qw);
   }
   if (r.valid) {
     *r.scale = s;
@@ -292,19 +300,20 @@ struct EpiTUpdate {
       if (row < g.M) {
         const long long off = (long long)row * p.ld + col;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const float4 c0 = *reinterpret_cast<const float4*>(p.c0 + off + 4 * k);
-          const float4 l = __ldg(reinterpret_cast<const float4*>(p.lam + col + 4 * k));
-          const float cc[4] = {c0.x, c0.y, c0.z, c0.w}, ll[4] = {l.x, l.y, l.z, l.w};
-          float hi[4], lo[4];
+        for (int k = 0; k < 4; ++k) {
+          float cc[8], hi[8], lo[8];
+          ld_v8f(p.c0 + off + 8 * k, cc);
+          const float4 l0 = __ldg(reinterpret_cast<const float4*>(p.lam + col + 8 * k));
+          const float4 l1 = __ldg(reinterpret_cast<const float4*>(p.lam + col + 8 * k + 4));
+          const float ll[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
+          for (int j = 0; j < 8; ++j) {
             const float inv = __frcp_rn(__fadd_rn(ll[j], p.rho));
-            const float t = __fmul_rn(__fadd_rn(cc[j], __fmul_rn(p.rho, v[4 * k + j])), inv);
+            const float t = __fmul_rn(__fadd_rn(cc[j], __fmul_rn(p.rho, v[8 * k + j])), inv);
             split2(t, hi[j], lo[j]);
           }
-          *reinterpret_cast<float4*>(p.t_hi + off + 4 * k) = make_float4(hi[0], hi[1], hi[2], hi[3]);
-          *reinterpret_cast<float4*>(p.t_lo + off + 4 * k) = make_float4(lo[0], lo[1], lo[2], lo[3]);
+          st_v8f(p.t_hi + off + 8 * k, hi);
+          st_v8f(p.t_lo + off + 8 * k, lo);
         }
       }
     }

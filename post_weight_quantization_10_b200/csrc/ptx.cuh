@@ -209,6 +209,35 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// 256-bit global accesses (sm_100): eight 32-bit words from / to a 32-byte
+// aligned address, without allocating in L1.  The epilogues give each thread
+// one accumulator row, so a warp's access touches 32 different rows; wider
+// accesses halve the L1 transactions per byte next to the main loop.
+__device__ __forceinline__ void ld_v8(const void* p, uint32_t (&v)[8]) {
+  asm volatile("ld.global.L1::no_allocate.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+                 "=r"(v[6]), "=r"(v[7])
+               : "l"(p));
+}
+__device__ __forceinline__ void ld_v8f(const float* p, float (&v)[8]) {
+  uint32_t u[8];
+  ld_v8(p, u);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(u[i]);
+}
+__device__ __forceinline__ void st_v8(void* p, const uint32_t (&v)[8]) {
+  asm volatile("st.global.L1::no_allocate.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+               ::"l"(p), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]),
+               "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+__device__ __forceinline__ void st_v8f(float* p, const float (&v)[8]) {
+  uint32_t u[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) u[i] = __float_as_uint(v[i]);
+  st_v8(p, u);
+}
+
 // Instruction descriptor with fp32 D: kind::f16 with bf16 A/B (fmt 1) or
 // kind::tf32 (fmt 2).
 __host__ __device__ constexpr uint32_t idesc_f32acc(uint32_t fmt, int M, int N, bool a_mn, bool b_mn) {
