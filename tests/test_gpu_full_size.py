@@ -1,0 +1,143 @@
+"""Parity at the full q_proj sizes, in the launch configuration the benchmark
+times (d_in = d_out = 4096, group 128, 3 bits, T = 100), on sampled outputs
+that the float64 oracle computes one by one (needs a B200).
+
+- Gram over the full n = 262144 tokens: sampled entries H_ij against float64
+  dot products of the same bf16 columns.
+- ADMM-Q iterations: every output row follows its own trajectory (the
+  W-update, the grid projection and the dual update act row by row), so the
+  oracle runs the solve for a few sampled rows on the same H~ and the GPU
+  runs all 4096.  The Hessian here comes from n = 8192 tokens, which the
+  oracle forms in full; the iteration kernels do not depend on n.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import admmq_oracle as O
+from oracle import projection_fp32 as P
+from post_weight_quantization_10_b200 import workloads
+
+pytestmark = pytest.mark.gpu
+
+D = 4096
+ROWS = np.array([0, 1, 77, 128, 1000, 2047, 2048, 3001, 3500, 4000, 4094, 4095])
+STEPS = (0, 1, 30, 60, 99)
+
+
+@pytest.fixture(scope="module")
+def A():
+    from post_weight_quantization_10_b200 import admmq
+    admmq.lib()
+    return admmq
+
+
+def test_full_gram_sampled(A):
+    """H = X^T X over 262144 tokens x 4096 features: 24 x 24 sampled entries
+    (the diagonal among them) within 1e-5 of sqrt(H_ii H_jj)."""
+    p = workloads.PRESETS["q_proj"]
+    X = workloads.make_activations(p, seed=0, device="cuda")
+    H = A.build_hessian(X)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(11)
+    I = np.sort(rng.choice(D, 20, replace=False))
+    I = np.unique(np.concatenate([I, [0, 127, 128, D - 1]]))
+    cols = torch.from_numpy(I).cuda()
+    Xc = X[:, cols].float().cpu().numpy().astype(np.float64)
+    del X
+    ref = Xc.T @ Xc
+    got = H[cols][:, cols].cpu().numpy().astype(np.float64)
+    dg = np.sqrt(np.outer(np.diag(ref), np.diag(ref)))
+    err = np.max(np.abs(got - ref) / dg)
+    assert err <= 1e-5, err
+    assert np.array_equal(got, got.T)
+
+
+@pytest.fixture(scope="module")
+def full_layer(A):
+    p = workloads.scaled(workloads.PRESETS["q_proj"], 8192, D, D)
+    X = workloads.make_activations(p, seed=0, device="cuda")
+    W = workloads.make_weights(p, seed=0, device="cuda", dtype=torch.float32)
+    Xn = X.float().cpu().numpy()
+    H = O.hessian(Xn, p.lambda_rel)
+    Wm = W[torch.from_numpy(ROWS).cuda()].cpu().numpy().T.astype(np.float64)
+    trace = []
+    res = O.admm_q(H, Wm, p.bits, p.group, p.iters, rho0=p.rho0, gamma=p.gamma, grid="minmax",
+                   trace=trace)
+    return p, X, W, H, Wm, res, trace
+
+
+def _solver(A, p, X, W):
+    prm = A.Params(bits=p.bits, group=p.group, iters=p.iters, rho0=p.rho0, gamma=p.gamma,
+                   lambda_rel=p.lambda_rel, grid="minmax")
+    G = A.build_hessian(X)
+    s = A.Solver(D, D, prm)
+    s.prepare(G, W)
+    s.eigh()
+    return s
+
+
+def test_full_size_teacher_forced(A, full_layer):
+    """RTN start bit-exact on the sampled rows; then, at sampled iterations,
+    the oracle's state of those rows is loaded into the GPU's state and one
+    GPU iteration runs: W~ within 1e-4 relative, codes equal on >= 99.9%,
+    mismatches one level apart where the grid agrees."""
+    p, X, W, H, Wm, res, trace = full_layer
+    s = _solver(A, p, X, W)
+    s.init()
+    torch.cuda.synchronize()
+    rows = torch.from_numpy(ROWS).cuda()
+    np.testing.assert_array_equal(s.codes[rows].cpu().numpy(), trace[0]["codes"].T)
+    np.testing.assert_array_equal(s.scale[rows].cpu().numpy(), trace[0]["scale"].T)
+    wt = torch.empty((D, D), dtype=torch.float32, device="cuda")
+    s.dump_wtilde(wt)
+    cu = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    for t in STEPS:
+        e = trace[t]
+        if t > 0:
+            hi, lo = P.split_tf32((e["Dt"] - e["Vt"]).T.astype(np.float32))
+            s.buffer("V")[rows] = cu(e["Vt"].T.astype(np.float32))
+            s.buffer("P_hi")[rows] = cu(hi)
+            s.buffer("P_lo")[rows] = cu(lo)
+            s.codes[rows] = cu(e["codes"].T)
+            s.scale[rows] = cu(e["scale"].T.astype(np.float32))
+            s.zero[rows] = cu(e["zero"].T.astype(np.float32))
+        s.iterate(t, 1)
+        torch.cuda.synchronize()
+        ref = e["W_tilde"].T
+        got = wt[rows].cpu().numpy().astype(np.float64)
+        err = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+        assert err <= 1e-4, (t, err)
+        c = s.codes[rows].cpu().numpy().astype(int)
+        co = e["codes_out"].T.astype(int)
+        assert np.mean(c != co) <= 1e-3, (t, np.mean(c != co))
+        same_grid = np.repeat(s.zero[rows].cpu().numpy() == e["zero_out"].T, p.group, axis=1)
+        assert np.all(np.abs(c - co)[same_grid] <= 1), t
+        print(f"full-size step {t}: W~ rel err {err:.2e}, code mismatches {np.mean(c != co):.2e}")
+    s.dump_wtilde(None)
+
+
+def test_full_size_free_running(A, full_layer):
+    """The whole T = 100 solve at 4096 x 4096: valid codes and grids, and on
+    the sampled rows an objective inside the spread the method itself shows.
+    At this size the min/max-grid trajectory is chaotic: the float64 oracle,
+    given relative noise of 1e-6 (4e-6) in its W-update, agrees with its own
+    noise-free run on 81-93% (70-75%) of these rows' codes and its objective
+    moves by -10%..+2% (-13%..+4%).  Step parity is the teacher-forced test
+    above; here the bar is that spread, with margin."""
+    p, X, W, H, Wm, res, trace = full_layer
+    s = _solver(A, p, X, W)
+    s.solve()
+    torch.cuda.synchronize()
+    rows = torch.from_numpy(ROWS).cuda()
+    codes = s.codes[rows].cpu().numpy()
+    sc, ze = s.scale[rows].cpu().numpy(), s.zero[rows].cpu().numpy()
+    L = (1 << p.bits) - 1
+    assert codes.max() <= L and np.all(sc > 0)
+    assert np.all((ze >= 0) & (ze <= L) & (ze == np.rint(ze)))
+    Dg = np.repeat(sc, p.group, axis=1) * (codes - np.repeat(ze, p.group, axis=1))
+    obj_gpu = O.objective(H, Dg.T.astype(np.float64), Wm)
+    rel = obj_gpu / res["objective"] - 1.0
+    agree = float(np.mean(codes == res["codes"].T))
+    print(f"full-size free-running: codes agree {agree:.5f}, objective rel {rel:+.3e}")
+    assert agree >= 0.6 and abs(rel) <= 0.2
