@@ -214,6 +214,13 @@ def run_ours(args, rank, world, device):
     if not args.no_e2e:
         e2e = run_e2e(A, run, args, world, device)
 
+    # objective 1/2 Tr((D - W_hat)^T H (D - W_hat)) of the solve just timed,
+    # next to that of its RTN start (same layer, same H)
+    obj_admm = float(run.s.objective.cpu())
+    run.s.init()
+    run.s.finish(resid=False)
+    obj_rtn = float(run.s.objective.cpu())
+
     if rank != 0:
         return None
     pk = peaks()
@@ -261,13 +268,61 @@ def run_ours(args, rank, world, device):
                      "traffic": measured_traffic(["gemm1_eigscale", "gemm2_project"][k]),
                      "peak_note": "bf16 dense %s sustained %.1f TF/s x 1/2 (tf32) / 3 (three "
                                   "tf32 MMAs per fp32-accurate product)" % (pk["src"], pk["bf16_sust"])},
+        "objective": {"admm_q": obj_admm, "rtn": obj_rtn, "admm_over_rtn": obj_admm / obj_rtn},
         "gpu_launches": launches,
         "clocks": clk,
         "e2e": e2e,
     }
+    if not args.no_stream_kernels:
+        line["stream_kernels"] = stream_kernels(A, args.grid, device)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(p, args.grid)
     return line
+
+
+def stream_kernels(A, grid, device, reps=10):
+    """HBM-bound kernels timed on their own, on buffers larger than L2: the
+    standalone projection (the fused epilogue's float32 arithmetic reading W~
+    from memory) and the b-bit pack.  Algorithmic bytes per element: W~ 4,
+    V 4 + 4, codes 1 + 1, P planes 8 (projection); codes 1 + b/8 (pack)."""
+    pk = peaks()
+    m, d, g, bits = 25600, 5120, 128, 3          # the up_proj 32B layer shape
+    gen = torch.Generator(device=device).manual_seed(7)
+    wt = torch.randn((m, d), generator=gen, device=device) * 0.02
+    V = torch.randn((m, d), generator=gen, device=device) * 0.002
+    sig = torch.rand(d, generator=gen, device=device) + 0.5
+    rsig = 1.0 / sig
+    hd = rsig * rsig
+    L = (1 << bits) - 1
+    codes = torch.randint(0, L + 1, (m, d), generator=gen, device=device, dtype=torch.uint8)
+    scale = torch.full((m, d // g), 0.01, device=device)
+    zero = torch.full((m, d // g), 3.0, device=device)
+    phi = torch.empty((m, d), device=device)
+    plo = torch.empty((m, d), device=device)
+    resid = torch.zeros(2, dtype=torch.float64, device=device)
+    big = torch.randint(0, L + 1, (4 * m, d), generator=gen, device=device, dtype=torch.uint8)
+    packed = torch.empty((4 * m, d * bits // 32), dtype=torch.int32, device=device)
+    out = {}
+    for name, fn, nbytes, shape in (
+            ("project", lambda: A.project(wt, V, sig, rsig, hd, bits, g, grid, codes, scale, zero,
+                                          phi, plo, resid=resid), 22.0 * m * d, [m, d]),
+            ("pack", lambda: A.pack(big, bits, out=packed), (1 + bits / 8) * 4 * m * d, [4 * m, d])):
+        fn()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / reps
+        gbs = nbytes / (ms / 1e3) / 1e9
+        out[name] = {"shape": shape, "bits": bits, "alg_bytes": nbytes, "ms": ms, "gbs": gbs,
+                     "frac_hbm": gbs / pk["hbm"], "traffic": measured_traffic(name)}
+    del wt, V, codes, phi, plo, big, packed
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_e2e(A, run, args, world, device):
@@ -402,12 +457,14 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="q_proj", choices=sorted(workloads.PRESETS))
-    ap.add_argument("--grid", default="minmax", choices=["minmax", "lsq", "frozen"])
+    ap.add_argument("--grid", default="lsq", choices=["lsq", "minmax", "frozen"])
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the calibration token count n (profiling captures only; "
                          "the eigenbasis GEMMs do not depend on n)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-stream-kernels", action="store_true",
+                    help="skip the stand-alone projection / pack bandwidth measurement")
     args = ap.parse_args()
     rank, world, local = D.world()
     if args.impl == "reference":

@@ -43,7 +43,7 @@ class Params:
     rho0: float = 0.1
     gamma: float = 1.05
     lambda_rel: float = 0.01
-    grid: str = "minmax"
+    grid: str = "lsq"
 
     def c(self) -> _Params:
         return _Params(self.bits, self.group, self.iters, self.rho0, self.gamma, self.lambda_rel,

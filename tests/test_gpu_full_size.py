@@ -4,7 +4,8 @@ that the float64 oracle computes one by one (needs a B200).
 
 - Gram over the full n = 262144 tokens: sampled entries H_ij against float64
   dot products of the same bf16 columns.
-- ADMM-Q iterations: every output row follows its own trajectory (the
+- ADMM-Q iterations (least-squares and min/max grid refresh): every output
+  row follows its own trajectory (the
   W-update, the grid projection and the dual update act row by row), so the
   oracle runs the solve for a few sampled rows on the same H~ and the GPU
   runs all 4096.  The Hessian here comes from n = 8192 tokens, which the
@@ -54,22 +55,29 @@ def test_full_gram_sampled(A):
 
 
 @pytest.fixture(scope="module")
-def full_layer(A):
+def full_setup(A):
     p = workloads.scaled(workloads.PRESETS["q_proj"], 8192, D, D)
     X = workloads.make_activations(p, seed=0, device="cuda")
     W = workloads.make_weights(p, seed=0, device="cuda", dtype=torch.float32)
-    Xn = X.float().cpu().numpy()
-    H = O.hessian(Xn, p.lambda_rel)
+    H = O.hessian(X.float().cpu().numpy(), p.lambda_rel)
     Wm = W[torch.from_numpy(ROWS).cuda()].cpu().numpy().T.astype(np.float64)
-    trace = []
-    res = O.admm_q(H, Wm, p.bits, p.group, p.iters, rho0=p.rho0, gamma=p.gamma, grid="minmax",
-                   trace=trace)
-    return p, X, W, H, Wm, res, trace
+    eig = np.linalg.eigh(O.diagonal_scaling(H)[1])
+    return p, X, W, H, Wm, eig, {}
 
 
-def _solver(A, p, X, W):
+def _oracle_run(full_setup, grid):
+    p, X, W, H, Wm, eig, cache = full_setup
+    if grid not in cache:
+        trace = []
+        res = O.admm_q(H, Wm, p.bits, p.group, p.iters, rho0=p.rho0, gamma=p.gamma, grid=grid,
+                       eig=eig, trace=trace)
+        cache[grid] = (res, trace)
+    return cache[grid]
+
+
+def _solver(A, p, X, W, grid):
     prm = A.Params(bits=p.bits, group=p.group, iters=p.iters, rho0=p.rho0, gamma=p.gamma,
-                   lambda_rel=p.lambda_rel, grid="minmax")
+                   lambda_rel=p.lambda_rel, grid=grid)
     G = A.build_hessian(X)
     s = A.Solver(D, D, prm)
     s.prepare(G, W)
@@ -77,13 +85,15 @@ def _solver(A, p, X, W):
     return s
 
 
-def test_full_size_teacher_forced(A, full_layer):
+@pytest.mark.parametrize("grid", ["lsq", "minmax"])
+def test_full_size_teacher_forced(A, full_setup, grid):
     """RTN start bit-exact on the sampled rows; then, at sampled iterations,
     the oracle's state of those rows is loaded into the GPU's state and one
     GPU iteration runs: W~ within 1e-4 relative, codes equal on >= 99.9%,
     mismatches one level apart where the grid agrees."""
-    p, X, W, H, Wm, res, trace = full_layer
-    s = _solver(A, p, X, W)
+    p, X, W, H, Wm, _, _ = full_setup
+    res, trace = _oracle_run(full_setup, grid)
+    s = _solver(A, p, X, W, grid)
     s.init()
     torch.cuda.synchronize()
     rows = torch.from_numpy(ROWS).cuda()
@@ -113,20 +123,46 @@ def test_full_size_teacher_forced(A, full_layer):
         assert np.mean(c != co) <= 1e-3, (t, np.mean(c != co))
         same_grid = np.repeat(s.zero[rows].cpu().numpy() == e["zero_out"].T, p.group, axis=1)
         assert np.all(np.abs(c - co)[same_grid] <= 1), t
-        print(f"full-size step {t}: W~ rel err {err:.2e}, code mismatches {np.mean(c != co):.2e}")
+        print(f"full-size {grid} step {t}: W~ rel err {err:.2e}, code mismatches {np.mean(c != co):.2e}")
     s.dump_wtilde(None)
 
 
-def test_full_size_free_running(A, full_layer):
+def _oracle_spread(full_setup, grid, res, monkeypatch, rel_noise=4e-6, seeds=(0, 1, 2)):
+    """How far the float64 oracle's own result moves on this layer when its
+    W-update carries relative noise of `rel_noise` (the GPU's per-step W~
+    error at this size is ~4e-6): (lowest code agreement, largest objective
+    change) over a few noise seeds."""
+    p, X, W, H, Wm, eig, _ = full_setup
+    w_update = O.w_update
+    agrees, rels = [], []
+    for seed in seeds:
+        rng = np.random.default_rng(seed)
+
+        def noisy(*a, rng=rng):
+            Wt = w_update(*a)
+            return Wt * (1.0 + rel_noise * rng.standard_normal(Wt.shape))
+
+        monkeypatch.setattr(O, "w_update", noisy)
+        r = O.admm_q(H, Wm, p.bits, p.group, p.iters, rho0=p.rho0, gamma=p.gamma, grid=grid,
+                     eig=eig)
+        monkeypatch.setattr(O, "w_update", w_update)
+        agrees.append(float(np.mean(r["codes"] == res["codes"])))
+        rels.append(abs(r["objective"] / res["objective"] - 1.0))
+    return min(agrees), max(rels)
+
+
+@pytest.mark.parametrize("grid", ["lsq", "minmax"])
+def test_full_size_free_running(A, full_setup, grid, monkeypatch):
     """The whole T = 100 solve at 4096 x 4096: valid codes and grids, and on
-    the sampled rows an objective inside the spread the method itself shows.
-    At this size the min/max-grid trajectory is chaotic: the float64 oracle,
-    given relative noise of 1e-6 (4e-6) in its W-update, agrees with its own
-    noise-free run on 81-93% (70-75%) of these rows' codes and its objective
-    moves by -10%..+2% (-13%..+4%).  Step parity is the teacher-forced test
-    above; here the bar is that spread, with margin."""
-    p, X, W, H, Wm, res, trace = full_layer
-    s = _solver(A, p, X, W)
+    the sampled rows codes and objective inside the spread the method itself
+    shows at this size.  The trajectory amplifies last-bit differences (step
+    parity is the teacher-forced test above), so the bar is the oracle's own
+    spread on this layer under W-update noise of the GPU's size, with margin:
+    codes agree >= (lowest noisy agreement - 0.05), objective within
+    2 x (largest noisy change) + 1e-3."""
+    p, X, W, H, Wm, _, _ = full_setup
+    res, _ = _oracle_run(full_setup, grid)
+    s = _solver(A, p, X, W, grid)
     s.solve()
     torch.cuda.synchronize()
     rows = torch.from_numpy(ROWS).cuda()
@@ -139,5 +175,8 @@ def test_full_size_free_running(A, full_layer):
     obj_gpu = O.objective(H, Dg.T.astype(np.float64), Wm)
     rel = obj_gpu / res["objective"] - 1.0
     agree = float(np.mean(codes == res["codes"].T))
-    print(f"full-size free-running: codes agree {agree:.5f}, objective rel {rel:+.3e}")
-    assert agree >= 0.6 and abs(rel) <= 0.2
+    min_agree, max_rel = _oracle_spread(full_setup, grid, res, monkeypatch)
+    print(f"full-size free-running {grid}: codes agree {agree:.5f}, objective rel {rel:+.3e}; "
+          f"oracle under noise: agree >= {min_agree:.5f}, |rel| <= {max_rel:.3e}")
+    assert agree >= min_agree - 0.05
+    assert abs(rel) <= 2.0 * max_rel + 1e-3
