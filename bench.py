@@ -220,6 +220,14 @@ def run_ours(args, rank, world, device):
     run.s.init()
     run.s.finish(resid=False)
     obj_rtn = float(run.s.objective.cpu())
+    # GPTQ (Algorithm 1, float64, the same fixed grid as RTN) on the same layer
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    g_codes, g_scale, g_zero = A.gptq(run.H, run.W, p.bits, p.group, p.lambda_rel)
+    torch.cuda.synchronize()
+    gptq_s = time.perf_counter() - t0
+    obj_gptq = run.s.objective_of(g_codes, g_scale, g_zero)
+    del g_codes, g_scale, g_zero
 
     if rank != 0:
         return None
@@ -268,7 +276,11 @@ def run_ours(args, rank, world, device):
                      "traffic": measured_traffic(["gemm1_eigscale", "gemm2_project"][k]),
                      "peak_note": "bf16 dense %s sustained %.1f TF/s x 1/2 (tf32) / 3 (three "
                                   "tf32 MMAs per fp32-accurate product)" % (pk["src"], pk["bf16_sust"])},
-        "objective": {"admm_q": obj_admm, "rtn": obj_rtn, "admm_over_rtn": obj_admm / obj_rtn},
+        "objective": {"admm_q": obj_admm, "rtn": obj_rtn, "gptq": obj_gptq,
+                      "admm_over_rtn": obj_admm / obj_rtn, "admm_over_gptq": obj_admm / obj_gptq,
+                      "gptq_s": gptq_s,
+                      "note": "1/2 Tr((D - W_hat)^T H (D - W_hat)), H = X^T X + lambda I; RTN and "
+                              "GPTQ on the min/max grid of W_hat, ADMM-Q with its refreshed grid"},
         "gpu_launches": launches,
         "clocks": clk,
         "e2e": e2e,

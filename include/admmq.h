@@ -232,6 +232,33 @@ int admmq_project(const float* wtilde_dev, float* V_dev, const float* sigma_dev,
                   int group, int grid_mode, uint8_t* codes_dev, float* scale_dev, float* zero_dev,
                   float* P_hi_dev, float* P_lo_dev, double* resid_dev, void* stream);
 
+/* ---------------------------------------------------------------- GPTQ ----
+ * The baseline the ADMM-Q objective is reported against: GPTQ, Algorithm 1
+ * of "GPTQ: Accurate Post-Training Quantization for Generative Pre-trained
+ * Transformers" (sections 2-3), on a fixed grid (the min/max grid of W_hat
+ * per output row and group, the RTN grid), columns in natural order, blocks
+ * of `block` columns, float64 arithmetic.  R is the upper Cholesky factor of
+ * H^-1 with H = G + lambda I and lambda = lambda_rel * mean(diag G), the same
+ * damping as admmq_prepare.
+ *
+ * admmq_gptq_workspace_bytes: bytes of device workspace for d_in x d_out with
+ * that block size (block in {32, 64, 128}); 0 for invalid sizes.
+ *
+ * admmq_gptq:
+ *   G_dev       fp32 [d_in][d_in] Gram X^T X (read only).
+ *   W_hat_dev   [d_out][d_in], fp32 or bf16 per w_dtype (read only).
+ *   codes_dev   u8 [d_out][d_in] out; scale_dev, zero_dev fp32
+ *               [d_out][d_in/group] out (the fixed grid).
+ *   ws_dev      workspace, 256-byte aligned, ws_bytes >= the size above.
+ * Synchronises the stream three times (status words and factorisation info).
+ * ADMMQ_ERR_NOT_PD when H or H^-1 is not positive definite,
+ * ADMMQ_ERR_NONFINITE for a non-finite diagonal, ADMMQ_ERR_WORKSPACE when
+ * ws_bytes is too small. */
+size_t admmq_gptq_workspace_bytes(int d_in, int d_out, int block);
+int admmq_gptq(const float* G_dev, const void* W_hat_dev, int w_dtype, int d_in, int d_out,
+               int bits, int group, float lambda_rel, int block, uint8_t* codes_dev,
+               float* scale_dev, float* zero_dev, void* ws_dev, size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

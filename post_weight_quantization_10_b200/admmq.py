@@ -103,6 +103,9 @@ def lib():
                                   ctypes.POINTER(ctypes.c_int)]),
         "admmq_project": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp,
                                _vp, _vp, _vp]),
+        "admmq_gptq_workspace_bytes": (_sz, [_i, _i, _i]),
+        "admmq_gptq": (_i, [_vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float, _i, _vp, _vp, _vp, _vp,
+                            _sz, _vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -217,6 +220,14 @@ class Solver:
                                   _ptr(self.objective) if objective else None, _stream(stream)),
                "admmq_finish")
 
+    def objective_of(self, codes, scale, zero, stream=None) -> float:
+        """1/2 Tr((D - W_hat)^T H (D - W_hat)) of any codes on any grid of this
+        layer (e.g. a GPTQ result), through the same eigenbasis GEMM."""
+        out = torch.zeros(1, dtype=torch.float64, device=codes.device)
+        _check(lib().admmq_finish(self._ctx, _ptr(codes), _ptr(scale), _ptr(zero), None,
+                                  _ptr(out), _stream(stream)), "admmq_finish")
+        return float(out.cpu())
+
     def solve(self, stream=None):
         _check(lib().admmq_solve(self._ctx, _ptr(self.codes), _ptr(self.scale), _ptr(self.zero),
                                  _ptr(self.resid), _ptr(self.objective), _stream(stream)),
@@ -277,6 +288,26 @@ def project(wtilde, V, sigma, rsig, hdiag, bits, group, grid, codes, scale, zero
                                _ptr(zero), _ptr(P_hi), _ptr(P_lo), _ptr(resid), _stream(stream)),
            "admmq_project")
     return resid
+
+
+def gptq(G: torch.Tensor, W_hat: torch.Tensor, bits: int, group: int, lambda_rel: float = 0.01,
+         block: int = 128, stream=None):
+    """GPTQ on the fixed min/max grid of W_hat: returns (codes, scale, zero)."""
+    m, d = W_hat.shape
+    assert G.dtype == torch.float32 and G.shape == (d, d) and G.is_contiguous()
+    assert W_hat.is_contiguous()
+    dt = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16}[W_hat.dtype]
+    need = int(lib().admmq_gptq_workspace_bytes(d, m, block))
+    if need == 0:
+        raise AdmmqError(-1, "admmq_gptq_workspace_bytes")
+    ws = torch.empty(need, dtype=torch.uint8, device=W_hat.device)
+    codes = torch.empty((m, d), dtype=torch.uint8, device=W_hat.device)
+    scale = torch.empty((m, d // group), dtype=torch.float32, device=W_hat.device)
+    zero = torch.empty_like(scale)
+    _check(lib().admmq_gptq(_ptr(G), _ptr(W_hat), dt, d, m, bits, group, lambda_rel, block,
+                            _ptr(codes), _ptr(scale), _ptr(zero), _ptr(ws), need, _stream(stream)),
+           "admmq_gptq")
+    return codes, scale, zero
 
 
 def solve_layer(X: torch.Tensor, W_hat: torch.Tensor, params: Params, stream=None) -> Solver:

@@ -16,7 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libadmmq.so")
 SOURCES = ["admmq.cu"]
-HEADERS = ["ptx.cuh", "gemm.cuh", "kernels.cuh"]
+HEADERS = ["ptx.cuh", "gemm.cuh", "kernels.cuh", "gptq.cuh"]
 INCLUDE = os.path.join(os.path.dirname(HERE), "include", "admmq.h")
 
 
@@ -44,7 +44,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
     cmd = [nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
            "-Xcompiler", "-fPIC,-O2", "-shared", "--expt-relaxed-constexpr",
            "-o", LIB + ".tmp"] + [os.path.join(CSRC, s) for s in SOURCES] + [
-           "-L" + libdir, "-lcusolver", "-Xlinker", "-rpath," + libdir]
+           "-L" + libdir, "-lcusolver", "-lcublas", "-Xlinker", "-rpath," + libdir]
     if ptxas_info:
         cmd += ["-Xptxas", "-v"]
     if verbose:

@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
+#include <cublas_v2.h>
 #include <cusolverDn.h>
 
 #include <math.h>
@@ -88,6 +89,8 @@ template <>
 __device__ __forceinline__ float load_w<__nv_bfloat16>(const __nv_bfloat16* p, long long i) {
   return __bfloat162float(p[i]);
 }
+
+#include "gptq.cuh"
 
 // W^~ = Sigma^-1 W_hat (rows = output channels), split into tf32 hi/lo planes.
 template <typename T>
@@ -290,48 +293,52 @@ __global__ void k_gram_finalize(const float* __restrict__ part, int splits, long
   }
 }
 
-// Pack CH codes per thread into CH*BITS/32 little-endian words.
-template <int BITS, int CH>
-__global__ void k_pack(const uint8_t* __restrict__ codes, long long chunks, int chunks_per_row,
-                       int d, uint32_t* __restrict__ out) {
-  constexpr int WPC = 32 * BITS / 32;  // words per 32 codes
+// Pack codes into a little-endian BITS-bit stream per row.  With d % 32 == 0
+// the codes are a flat sequence of 32-code groups whose packed words (BITS
+// per group) are contiguous as well, rows included.  A warp takes 32
+// consecutive groups: lane l reads group l (32 bytes; the warp reads 1 KB
+// contiguous), builds its BITS words, stages them in shared memory, and the
+// warp writes its 32 x BITS words back as contiguous 16-byte stores.
+template <int BITS>
+__global__ void __launch_bounds__(256) k_pack(const uint8_t* __restrict__ codes, long long groups,
+                                              uint32_t* __restrict__ out) {
   constexpr uint32_t MASK = (1u << BITS) - 1u;
-  const long long wpr = (long long)d * BITS / 32;
-  for (long long ch = blockIdx.x * (long long)blockDim.x + threadIdx.x; ch < chunks;
-       ch += (long long)gridDim.x * blockDim.x) {
-    const long long row = ch / chunks_per_row;
-    const int c = (int)(ch - row * chunks_per_row);
-    const uint8_t* src = codes + row * d + (long long)c * CH;
-    uint32_t* dst = out + row * wpr + (long long)c * (CH / 32) * WPC;
-#pragma unroll
-    for (int sub = 0; sub < CH / 32; ++sub) {
-      uint32_t in[8];
-      const uint4 a = reinterpret_cast<const uint4*>(src + sub * 32)[0];
-      const uint4 b = reinterpret_cast<const uint4*>(src + sub * 32)[1];
+  __shared__ __align__(16) uint32_t stage[8][32 * BITS];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  uint32_t* buf = stage[wib];
+  const long long nwarps = (long long)gridDim.x * 8;
+  for (long long base = ((long long)blockIdx.x * 8 + wib) * 32; base < groups; base += nwarps * 32) {
+    const long long grp = base + lane;
+    uint32_t in[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    if (grp < groups) {
+      const uint4* src = reinterpret_cast<const uint4*>(codes + grp * 32);
+      const uint4 a = __ldcs(src), b = __ldcs(src + 1);
       in[0] = a.x; in[1] = a.y; in[2] = a.z; in[3] = a.w;
       in[4] = b.x; in[5] = b.y; in[6] = b.z; in[7] = b.w;
-      uint32_t w[WPC];
-#pragma unroll
-      for (int k = 0; k < WPC; ++k) w[k] = 0u;
-#pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const uint32_t v = (in[k >> 2] >> (8 * (k & 3))) & MASK;
-        const int pos = k * BITS;
-        w[pos >> 5] |= v << (pos & 31);
-        if ((pos & 31) + BITS > 32) w[(pos >> 5) + 1] |= v >> (32 - (pos & 31));
-      }
-      uint32_t* o = dst + sub * WPC;
-      if (WPC % 4 == 0) {
-#pragma unroll
-        for (int k = 0; k < WPC; k += 4) reinterpret_cast<uint4*>(o)[k / 4] = make_uint4(w[k], w[k + 1], w[k + 2], w[k + 3]);
-      } else if (WPC % 2 == 0) {
-#pragma unroll
-        for (int k = 0; k < WPC; k += 2) reinterpret_cast<uint2*>(o)[k / 2] = make_uint2(w[k], w[k + 1]);
-      } else {
-#pragma unroll
-        for (int k = 0; k < WPC; ++k) o[k] = w[k];
-      }
     }
+    uint32_t w[BITS];
+#pragma unroll
+    for (int k = 0; k < BITS; ++k) w[k] = 0u;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      const uint32_t v = (in[k >> 2] >> (8 * (k & 3))) & MASK;
+      const int pos = k * BITS;
+      w[pos >> 5] |= v << (pos & 31);
+      if ((pos & 31) + BITS > 32) w[(pos >> 5) + 1] |= v >> (32 - (pos & 31));
+    }
+#pragma unroll
+    for (int k = 0; k < BITS; ++k) buf[lane * BITS + k] = w[k];
+    __syncwarp();
+    const long long valid = groups - base < 32 ? groups - base : 32;
+    uint32_t* dst = out + base * BITS;
+    if (valid == 32) {
+      // 32 * BITS words = 8 * BITS 16-byte vectors
+      for (int v = lane; v < 8 * BITS; v += 32)
+        __stcs(reinterpret_cast<uint4*>(dst) + v, reinterpret_cast<const uint4*>(buf)[v]);
+    } else {
+      for (int k = lane; k < valid * BITS; k += 32) dst[k] = buf[k];
+    }
+    __syncwarp();
   }
 }
 
@@ -597,6 +604,63 @@ int syevd_lwork(int d) {
                                   d, nullptr, &lwork) != CUSOLVER_STATUS_SUCCESS)
     return -1;
   return lwork;
+}
+
+// ------------------------------------------------------------ GPTQ host side
+
+// Library handles for the GPTQ baseline (created on first use, for the
+// device current at that time).
+cusolverDnHandle_t gptq_solver() {
+  static cusolverDnHandle_t h = nullptr;
+  if (!h && cusolverDnCreate(&h) != CUSOLVER_STATUS_SUCCESS) h = nullptr;
+  return h;
+}
+cublasHandle_t gptq_blas() {
+  static cublasHandle_t h = nullptr;
+  if (!h && cublasCreate(&h) != CUBLAS_STATUS_SUCCESS) h = nullptr;
+  return h;
+}
+
+int gptq_lwork(int d) {
+  cusolverDnHandle_t h = gptq_solver();
+  if (!h) return -1;
+  int l1 = 0, l2 = 0;
+  if (cusolverDnDpotrf_bufferSize(h, CUBLAS_FILL_MODE_LOWER, d, nullptr, d, &l1) !=
+          CUSOLVER_STATUS_SUCCESS ||
+      cusolverDnDpotri_bufferSize(h, CUBLAS_FILL_MODE_LOWER, d, nullptr, d, &l2) !=
+          CUSOLVER_STATUS_SUCCESS)
+    return -1;
+  return l1 > l2 ? l1 : l2;
+}
+
+// GPTQ workspace: status words, lambda and the damping kernel's per-column
+// outputs, H in float64 (factorised in place into R), the float64 working
+// weights, one block of errors E, the solver's work area.
+struct GptqLayout {
+  size_t status, lam64, sig64, hdiag, sigma, rsig, Hd, Wd, E, work, devinfo, total;
+};
+
+GptqLayout gptq_layout(int d, int m, int block, int lwork) {
+  GptqLayout L;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = o;
+    o = align256(o + bytes);
+    return at;
+  };
+  L.status = take(16);
+  L.lam64 = take(8);
+  L.sig64 = take(8 * (size_t)d);
+  L.hdiag = take(4 * (size_t)d);
+  L.sigma = take(4 * (size_t)d);
+  L.rsig = take(4 * (size_t)d);
+  L.Hd = take(8 * (size_t)d * d);
+  L.Wd = take(8 * (size_t)d * m);
+  L.E = take(8 * (size_t)m * block);
+  L.work = take(8 * (size_t)(lwork > 0 ? lwork : 1));
+  L.devinfo = take(16);
+  L.total = o;
+  return L;
 }
 
 #define CK(x)                                      \
@@ -938,17 +1002,11 @@ int admmq_pack(const uint8_t* codes, int d, int m, int bits, uint32_t* packed, v
     return ADMMQ_ERR_INVALID_ARG;
   if (((uintptr_t)codes & 15) || ((uintptr_t)packed & 15)) return ADMMQ_ERR_INVALID_ARG;
   cudaStream_t st = (cudaStream_t)stream;
-  const bool big = d % 128 == 0;
-  const int ch = big ? 128 : 32;
-  const int cpr = d / ch;
-  const long long chunks = (long long)m * cpr;
-  const int grid = grid_for(chunks, 256);
-#define PACK_CASE(B)                                                                      \
-  case B:                                                                                 \
-    if (big)                                                                              \
-      count_launch(), k_pack<B, 128><<<grid, 256, 0, st>>>(codes, chunks, cpr, d, packed);                \
-    else                                                                                  \
-      count_launch(), k_pack<B, 32><<<grid, 256, 0, st>>>(codes, chunks, cpr, d, packed);                 \
+  const long long groups = (long long)m * (d / 32);
+  const int grid = grid_for(groups, 256);  // one group per thread, 8 warps per block
+#define PACK_CASE(B)                                                         \
+  case B:                                                                    \
+    count_launch(), k_pack<B><<<grid, 256, 0, st>>>(codes, groups, packed);  \
     break;
   switch (bits) {
     PACK_CASE(1)
@@ -1048,6 +1106,111 @@ int admmq_project(const float* wt, float* V, const float* sig, const float* rsig
   else
     count_launch(), k_project<GRID_FROZEN><<<grid, 128, 0, st>>>(wt, V, sig, rsig, hd, m, d, g, L, codes, scale,
                                                  zero, p_hi, p_lo, resid);
+  CK(cudaGetLastError());
+  return ADMMQ_OK;
+}
+
+// ------------------------------------------------------------------ GPTQ
+
+size_t admmq_gptq_workspace_bytes(int d, int m, int block) {
+  if (d <= 0 || m <= 0 || d % 32 != 0 || !(block == 32 || block == 64 || block == 128)) return 0;
+  const int lw = gptq_lwork(d);
+  if (lw < 0) return 0;
+  return gptq_layout(d, m, block, lw).total;
+}
+
+int admmq_gptq(const float* G, const void* W_hat, int w_dtype, int d, int m, int bits, int group,
+               float lambda_rel, int block, uint8_t* codes, float* scale, float* zero, void* ws,
+               size_t ws_bytes, void* stream) {
+  if (!G || !W_hat || !codes || !scale || !zero || !ws) return ADMMQ_ERR_INVALID_ARG;
+  if (d <= 0 || m <= 0 || d % 32 != 0 || !(group == 32 || group == 64 || group == 128) ||
+      d % group != 0 || bits < 1 || bits > 8 || !(lambda_rel >= 0.f) ||
+      !(block == 32 || block == 64 || block == 128) ||
+      (w_dtype != ADMMQ_DTYPE_F32 && w_dtype != ADMMQ_DTYPE_BF16))
+    return ADMMQ_ERR_INVALID_ARG;
+  if (((uintptr_t)ws & 255) != 0) return ADMMQ_ERR_INVALID_ARG;
+  const int lw = gptq_lwork(d);
+  if (lw < 0) return ADMMQ_ERR_CUDA;
+  const GptqLayout Lo = gptq_layout(d, m, block, lw);
+  if (ws_bytes < Lo.total) return ADMMQ_ERR_WORKSPACE;
+  int rc = device_ok();
+  if (rc) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  uint8_t* base = (uint8_t*)ws;
+  int* status = (int*)(base + Lo.status);
+  double* lam64 = (double*)(base + Lo.lam64);
+  double* Hd = (double*)(base + Lo.Hd);
+  double* Wd = (double*)(base + Lo.Wd);
+  double* E = (double*)(base + Lo.E);
+  double* work = (double*)(base + Lo.work);
+  int* devinfo = (int*)(base + Lo.devinfo);
+  const int L = (1 << bits) - 1;
+
+  // H = X^T X + lambda I (lambda as in the ADMM-Q setup) and the fixed grid
+  CK(cudaMemsetAsync(status, 0, 16, st));
+  count_launch(), k_diag_stats<<<1, 1024, 0, st>>>(G, d, lambda_rel, lam64, (double*)(base + Lo.sig64),
+                                                   (float*)(base + Lo.hdiag), (float*)(base + Lo.sigma),
+                                                   (float*)(base + Lo.rsig), status);
+  CK(cudaGetLastError());
+  count_launch(), k_gptq_hessian<<<grid_for((long long)d * d), 256, 0, st>>>(G, d, lam64, Hd);
+  CK(cudaGetLastError());
+  const long long groups = (long long)m * (d / group);
+  if (w_dtype == ADMMQ_DTYPE_F32)
+    count_launch(), k_gptq_start<float><<<grid_for(groups, 128), 128, 0, st>>>(
+        (const float*)W_hat, m, d, group, L, scale, zero, Wd);
+  else
+    count_launch(), k_gptq_start<__nv_bfloat16><<<grid_for(groups, 128), 128, 0, st>>>(
+        (const __nv_bfloat16*)W_hat, m, d, group, L, scale, zero, Wd);
+  CK(cudaGetLastError());
+  int host_status[4] = {0, 0, 0, 0};
+  CK(cudaMemcpyAsync(host_status, status, 16, cudaMemcpyDeviceToHost, st));
+  CK(cudaStreamSynchronize(st));
+  if (host_status[1] == SETUP_NONFINITE) return ADMMQ_ERR_NONFINITE;
+  if (host_status[1] == SETUP_NOT_PD) return ADMMQ_ERR_NOT_PD;
+
+  // R = upper Cholesky factor of H^-1.  cuSOLVER is column-major: the lower
+  // factor it writes is, read row-major, the upper factor R with R^T R = A.
+  cusolverDnHandle_t sv = gptq_solver();
+  cublasHandle_t bl = gptq_blas();
+  if (!sv || !bl) return ADMMQ_ERR_CUDA;
+  if (cusolverDnSetStream(sv, st) != CUSOLVER_STATUS_SUCCESS ||
+      cublasSetStream(bl, st) != CUBLAS_STATUS_SUCCESS)
+    return ADMMQ_ERR_CUDA;
+  auto info_ok = [&]() -> int {
+    int info = 0;
+    if (cudaMemcpyAsync(&info, devinfo, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+      return ADMMQ_ERR_CUDA;
+    return info == 0 ? ADMMQ_OK : ADMMQ_ERR_NOT_PD;
+  };
+  if (cusolverDnDpotrf(sv, CUBLAS_FILL_MODE_LOWER, d, Hd, d, work, lw, devinfo) !=
+      CUSOLVER_STATUS_SUCCESS)
+    return ADMMQ_ERR_CUDA;
+  if ((rc = info_ok())) return rc;
+  if (cusolverDnDpotri(sv, CUBLAS_FILL_MODE_LOWER, d, Hd, d, work, lw, devinfo) !=
+      CUSOLVER_STATUS_SUCCESS)
+    return ADMMQ_ERR_CUDA;
+  if ((rc = info_ok())) return rc;
+  if (cusolverDnDpotrf(sv, CUBLAS_FILL_MODE_LOWER, d, Hd, d, work, lw, devinfo) !=
+      CUSOLVER_STATUS_SUCCESS)
+    return ADMMQ_ERR_CUDA;
+  if ((rc = info_ok())) return rc;
+
+  // column blocks: the sequential block kernel, then the trailing update
+  //   W[:, b:] -= E R[a:b, b:]   (row-major; column-major C^T = R^T-block E^T)
+  const double minus_one = -1.0, one = 1.0;
+  for (int a = 0; a < d; a += block) {
+    const int bw = d - a < block ? d - a : block;
+    count_launch(), k_gptq_block<<<cdiv(m, 8), 256, 0, st>>>(Wd, Hd, scale, zero, m, d, group, L, a,
+                                                            bw, codes, E, block);
+    CK(cudaGetLastError());
+    const int b = a + bw;
+    if (b < d) {
+      if (cublasDgemm(bl, CUBLAS_OP_N, CUBLAS_OP_N, d - b, m, bw, &minus_one, Hd + (size_t)a * d + b,
+                      d, E, block, &one, Wd + b, d) != CUBLAS_STATUS_SUCCESS)
+        return ADMMQ_ERR_CUDA;
+    }
+  }
   CK(cudaGetLastError());
   return ADMMQ_OK;
 }

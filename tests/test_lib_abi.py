@@ -74,3 +74,20 @@ def test_alignment_checks_without_gpu(lib):
     bad[0] = ctypes.c_void_p(ok[0].value + 8)  # W~ needs 16 bytes
     assert call(bad) == -1
     assert lib.admmq_debug_dump_wtilde(None, None) == -1
+
+
+def test_gptq_argument_checks_without_gpu(lib):
+    """GPTQ entry points reject bad sizes and pointers before touching a device."""
+    fake = ctypes.c_void_p(0x10000)
+    assert lib.admmq_gptq_workspace_bytes(100, 8, 128) == 0      # d_in % 32
+    assert lib.admmq_gptq_workspace_bytes(256, 8, 96) == 0       # block
+    assert lib.admmq_gptq_workspace_bytes(256, 0, 128) == 0
+    args = [fake, fake, 0, 256, 8, 3, 128, 0.01, 128, fake, fake, fake, fake, 1 << 30, None]
+    for k, bad in ((0, None), (1, None), (9, None), (12, None),    # null pointers
+                   (3, 200), (6, 96), (5, 9), (8, 16), (2, 5), (7, -1.0)):
+        a = list(args)
+        a[k] = bad
+        assert lib.admmq_gptq(*a) == -1, k
+    a = list(args)
+    a[12] = ctypes.c_void_p(0x10000 + 64)                       # workspace alignment
+    assert lib.admmq_gptq(*a) == -1
