@@ -131,7 +131,7 @@ class ClockSampler:
 class LayerRun:
     """Device-resident state of one layer solve through the C ABI binding."""
 
-    def __init__(self, A, p, grid, seed, device):
+    def __init__(self, A, p, grid, seed, device, split="auto"):
         self.A, self.p = A, p
         self.X = workloads.make_activations(p, seed=seed, device=device)
         self.W = workloads.make_weights(p, seed=seed, device=device, dtype=torch.bfloat16)
@@ -139,7 +139,7 @@ class LayerRun:
         self.gram_ws = torch.empty(A.gram_workspace_bytes(p.n, p.d_in), dtype=torch.uint8,
                                    device=device)
         prm = A.Params(bits=p.bits, group=p.group, iters=p.iters, rho0=p.rho0, gamma=p.gamma,
-                       lambda_rel=p.lambda_rel, grid=grid)
+                       lambda_rel=p.lambda_rel, grid=grid, split=split)
         self.s = A.Solver(p.d_in, p.d_out, prm, device=device)
         self.packed = torch.empty((p.d_out, p.d_in * p.bits // 32), dtype=torch.int32,
                                   device=device)
@@ -176,7 +176,7 @@ def run_ours(args, rank, world, device):
     p = workloads.PRESETS[args.workload]
     if args.tokens:
         p = workloads.scaled(p, args.tokens, p.d_in, p.d_out)
-    run = LayerRun(A, p, args.grid, seed=rank, device=device)
+    run = LayerRun(A, p, args.grid, seed=rank, device=device, split=args.split)
     eigh_s = run.setup_eigh()
     for _ in range(args.warmup):
         run.step()
@@ -242,9 +242,13 @@ def run_ours(args, rank, world, device):
     k = 0 if gemm_ms[0] >= gemm_ms[1] else 1
     avg_ms = gemm_ms[k] / max(gemm_n[k], 1)
     achieved = 2.0 * d * d * m / (avg_ms / 1e3) / 1e12
-    # 3xTF32: three tf32 MMAs per fp32-accurate product; dense tf32 runs at half
-    # the bf16 rate (nominal 1.1 vs 2.25 PFLOP/s), so the peak is bf16 / 6.
-    peak_split = pk["bf16_sust"] / 6.0
+    # Tensor work per fp32-accurate product, in bf16-MMA units (dense tf32 runs
+    # at half the bf16 rate, nominal 1.1 vs 2.25 PFLOP/s): 3xTF32 = three tf32
+    # MMAs = 6; mixed split = one tf32 MMA (2) + one bf16 MMA over the doubled
+    # K of the correction rows (2) = 4.  Peak = bf16 peak / that.
+    split = run.s.split
+    per_product = 4.0 if split == "mixed" else 6.0
+    peak_split = pk["bf16_sust"] / per_product
     line = {
         "metric": METRIC,
         "value": iters_per_s,
@@ -256,11 +260,12 @@ def run_ours(args, rank, world, device):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "3xtf32-f32",
+        "dtype": "f32 via tf32+bf16 split" if split == "mixed" else "f32 via 3xtf32",
         "data": "synthetic (seeded Qwen3-8B-shaped activations and weights; no dataset)",
         "config": {"workload": workload_desc(p, args.grid), "parallelism": f"independent layers x{world}",
                    "l2": "inputs larger than L2 (X is %.1f GiB)" % (n * d * 2 / 2**30),
-                   "eigh": "one-time setup outside the step (eigh_s)"},
+                   "eigh": "one-time setup outside the step (eigh_s)",
+                   "split": split},
         "s_per_layer": ms_max / 1e3 / args.steps,
         "s_per_layer_with_eigh": ms_max / 1e3 / args.steps + eigh_s,
         "eigh_s": eigh_s,
@@ -274,8 +279,9 @@ def run_ours(args, rank, world, device):
                      "achieved": achieved, "peak": peak_split, "unit": "TFLOP/s",
                      "frac": achieved / peak_split,
                      "traffic": measured_traffic(["gemm1_eigscale", "gemm2_project"][k]),
-                     "peak_note": "bf16 dense %s sustained %.1f TF/s x 1/2 (tf32) / 3 (three "
-                                  "tf32 MMAs per fp32-accurate product)" % (pk["src"], pk["bf16_sust"])},
+                     "peak_note": "bf16 dense %s sustained %.1f TF/s / %d (bf16-MMA units of tensor "
+                                  "work per fp32-accurate product, %s split)" % (
+                                      pk["src"], pk["bf16_sust"], per_product, split)},
         "objective": {"admm_q": obj_admm, "rtn": obj_rtn, "gptq": obj_gptq,
                       "admm_over_rtn": obj_admm / obj_rtn, "admm_over_gptq": obj_admm / obj_gptq,
                       "gptq_s": gptq_s,
@@ -310,7 +316,7 @@ def stream_kernels(A, grid, device, reps=10):
     scale = torch.full((m, d // g), 0.01, device=device)
     zero = torch.full((m, d // g), 3.0, device=device)
     phi = torch.empty((m, d), device=device)
-    plo = torch.empty((m, d), device=device)
+    plo = torch.empty((m, 2 * d), dtype=torch.int16, device=device)  # bf16 correction rows
     resid = torch.zeros(2, dtype=torch.float64, device=device)
     big = torch.randint(0, L + 1, (4 * m, d), generator=gen, device=device, dtype=torch.uint8)
     packed = torch.empty((4 * m, d * bits // 32), dtype=torch.int32, device=device)
@@ -470,6 +476,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="q_proj", choices=sorted(workloads.PRESETS))
     ap.add_argument("--grid", default="lsq", choices=["lsq", "minmax", "frozen"])
+    ap.add_argument("--split", default="auto", choices=["auto", "mixed", "3xtf32"],
+                    help="split precision of the eigenbasis GEMMs (auto: mixed from d_in 2048)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the calibration token count n (profiling captures only; "
                          "the eigenbasis GEMMs do not depend on n)")

@@ -58,6 +58,14 @@ enum {
 
 enum { ADMMQ_DTYPE_F32 = 0, ADMMQ_DTYPE_BF16 = 1 };
 
+/* Split precision of the eigenbasis GEMMs (fp32-accurate products on tf32 /
+ * bf16 tensor cores; see "operand encoding" below). */
+enum {
+  ADMMQ_SPLIT_AUTO = 0,   /* mixed from d_in >= 2048, else 3xTF32                 */
+  ADMMQ_SPLIT_3XTF32 = 1, /* hi.hi + hi.lo + lo.hi, three tf32 products           */
+  ADMMQ_SPLIT_MIXED = 2   /* tf32 hi.hi + one bf16 product for hi.lo + lo.hi      */
+};
+
 typedef struct admmq_params {
   int bits;         /* b: codes in [0, 2^b - 1]                                  */
   int group;        /* g: input channels per quantization group                 */
@@ -66,6 +74,7 @@ typedef struct admmq_params {
   float gamma;      /* penalty growth: rho_t = rho0 * gamma^t                    */
   float lambda_rel; /* damping: lambda = lambda_rel * mean(diag(X^T X))          */
   int grid_mode;    /* ADMMQ_GRID_*                                              */
+  int split_mode;   /* ADMMQ_SPLIT_*                                             */
 } admmq_params;
 
 typedef struct admmq_ctx admmq_ctx; /* opaque; host memory owned by the library */
@@ -133,7 +142,8 @@ void admmq_destroy(admmq_ctx* ctx);
 /* Damping and diagonal scaling (Methodology section 1 and section 2,
  * "diagonal scaling"): lambda = lambda_rel * mean(diag G), H = G + lambda I,
  * sigma_i = H_ii^(-1/2), H~ = Sigma H Sigma (float64, into the workspace) and
- * the scaled weights W^~ = Sigma^-1 W_hat as tf32 hi/lo planes (fp32 words).
+ * the scaled weights W^~ = Sigma^-1 W_hat as split-precision operand planes
+ * (see "operand encoding" below).
  *   G_dev      fp32 [d_in][d_in], X^T X WITHOUT damping (admmq_build_hessian).
  *   W_hat_dev  [d_out][d_in], fp32 or bf16 (w_dtype); must stay valid until
  *              admmq_destroy (the objective reads it).
@@ -142,9 +152,9 @@ int admmq_prepare(admmq_ctx* ctx, const float* G_dev, const void* W_hat_dev, int
                   void* stream);
 
 /* One-time eigendecomposition H~ = Q Lambda Q^T (Methodology section 2,
- * W-update) with cuSOLVER's float64 divide-and-conquer solver, then the tf32
- * hi/lo planes of Q^T and Q for the split-precision (3xTF32) GEMMs.  Synchronises the
- * stream once to read the solver's info (ADMMQ_ERR_EIG if non-zero). */
+ * W-update) with cuSOLVER's float64 divide-and-conquer solver, then the
+ * split-precision operand planes of Q^T and Q.  Synchronises the stream once
+ * to read the solver's info (ADMMQ_ERR_EIG if non-zero). */
 int admmq_eigh(admmq_ctx* ctx, void* stream);
 
 /* admmq_prepare + admmq_eigh. */
@@ -189,13 +199,24 @@ int admmq_pack(const uint8_t* codes_dev, int d_in, int d_out, int bits, uint32_t
                void* stream);
 
 /* ------------------------------------------------------------ inspection --
- * Device buffers inside the workspace, for tests and diagnostics.  Layouts:
+ * Device buffers inside the workspace, for tests and diagnostics.
+ * Operand encoding of the eigenbasis GEMMs (fp32-accurate split precision,
+ * per admmq_split_mode): a matrix x [rows][K] is stored as plane HI, fp32
+ * [rows][K] with hi = tf32(x), and plane LO:
+ *   ADMMQ_SPLIT_3XTF32: fp32 [rows][K], lo = tf32(x - hi);
+ *   ADMMQ_SPLIT_MIXED:  u16 [rows][2K] of bfloat16 bit patterns: per 32
+ *     columns c0..c0+31 of a row, for operands on the A side (W^~, P, T) the
+ *     32 values bf16(hi) then the 32 values bf16(x - hi); on the B side
+ *     (Q^T, Q) the two halves swapped.
+ * All roundings nearest-even.  Both encodings take 4 bytes per element.
+ * Layouts:
  *   ADMMQ_BUF_SIGMA, _RSIG, _HDIAG, _LAMBDA : fp32 [d_in]
  *   ADMMQ_BUF_V      fp32 [d_out][d_in]  scaled dual V~
  *   ADMMQ_BUF_C0     fp32 [d_out][d_in]  C0' = Lambda Q^T W^~ (row j, column k)
- *   ADMMQ_BUF_P_HI/_P_LO  fp32 [d_out][d_in]  P = D~ - V~ as tf32 hi/lo planes
- *   ADMMQ_BUF_T_HI/_T_LO  fp32 [d_out][d_in]  GEMM-1 output, tf32 hi/lo planes
- *   ADMMQ_BUF_E_HI/_E_LO  fp32 [d_in][d_in]   row k = k-th eigenvector of H~ (tf32 planes)
+ *   ADMMQ_BUF_P_HI/_P_LO  P = D~ - V~, encoded planes (A side)
+ *   ADMMQ_BUF_T_HI/_T_LO  GEMM-1 output T, encoded planes (A side)
+ *   ADMMQ_BUF_E_HI/_E_LO  E = Q^T (row k = k-th eigenvector of H~), encoded
+ *                         planes (B side)
  *   ADMMQ_BUF_HT     fp64 [d_in][d_in]   H~ before admmq_eigh, Q^T after
  *   ADMMQ_BUF_STATUS int32 [4]           kernel status words (0 = ok)     */
 enum {
@@ -220,17 +241,26 @@ int admmq_get_timing(admmq_ctx* ctx, double ms[2], int launches[2]);
 
 /* Standalone projection kernel (the fused GEMM-2 epilogue reading W~ from
  * memory instead of tensor memory); same per-element float32 arithmetic.
- * All pointers device; V_dev is updated in place; P_hi/P_lo receive P as
- * tf32 hi/lo planes in fp32 words (hi = tf32(P), lo = tf32(P - hi));
- * codes/scale/zero hold the previous D on entry and the new D on exit;
- * resid_dev fp64 [2] receives the two residual sums of squares.
+ * All pointers device; V_dev is updated in place; P is written in the
+ * eigenbasis GEMMs' operand encoding of `split_mode` (ADMMQ_SPLIT_3XTF32 or
+ * ADMMQ_SPLIT_MIXED, A side): P_hi_dev fp32 [d_out][d_in] and P_lo_dev
+ * (fp32 [d_out][d_in] or u16 [d_out][2 d_in]); codes/scale/zero hold the
+ * previous D on entry and the new D on exit; resid_dev fp64 [2] receives the
+ * two residual sums of squares.
  * V_dev, codes_dev, P_hi_dev, P_lo_dev, sigma_dev, rsig_dev and hdiag_dev
  * must be 32-byte aligned, wtilde_dev 16-byte aligned (ADMMQ_ERR_INVALID_ARG
  * otherwise). */
 int admmq_project(const float* wtilde_dev, float* V_dev, const float* sigma_dev,
                   const float* rsig_dev, const float* hdiag_dev, int d_in, int d_out, int bits,
-                  int group, int grid_mode, uint8_t* codes_dev, float* scale_dev, float* zero_dev,
-                  float* P_hi_dev, float* P_lo_dev, double* resid_dev, void* stream);
+                  int group, int grid_mode, int split_mode, uint8_t* codes_dev, float* scale_dev,
+                  float* zero_dev, float* P_hi_dev, void* P_lo_dev, double* resid_dev,
+                  void* stream);
+
+/* The split precision a context runs its eigenbasis GEMMs in
+ * (ADMMQ_SPLIT_3XTF32 or ADMMQ_SPLIT_MIXED; ADMMQ_SPLIT_AUTO resolved by
+ * d_in), which fixes the encoding of its P/T/E buffers; ADMMQ_ERR_INVALID_ARG
+ * for a NULL context. */
+int admmq_split_mode(const admmq_ctx* ctx);
 
 /* ---------------------------------------------------------------- GPTQ ----
  * The baseline the ADMM-Q objective is reported against: GPTQ, Algorithm 1

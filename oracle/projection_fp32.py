@@ -125,12 +125,39 @@ def split_tf32(x: np.ndarray):
     return hi, lo
 
 
+def split_mix(x: np.ndarray, side: str = "A"):
+    """The eigenbasis GEMMs' operand encoding of a float32 matrix x [rows][K]
+    (K % 32 == 0): plane 0 = hi = tf32(x) (float32); plane 1 = uint16 bf16
+    bit patterns [rows][2K], per 32 columns the 32 values bf16(hi) then the
+    32 values bf16(lo) with lo = x - hi (exact in float32) for side "A", the
+    two halves swapped for side "B".  One tf32 product of the hi planes plus
+    one bf16 product of the correction rows gives hi.hi + hi.lo + lo.hi."""
+    x = _f(x)
+    rows, K = x.shape
+    hi = tf32_round(x)
+    lo = _f(x - hi)
+    hb = bf16_bits(hi).reshape(rows, K // 32, 32)
+    lb = bf16_bits(lo).reshape(rows, K // 32, 32)
+    first, second = (hb, lb) if side == "A" else (lb, hb)
+    return hi, np.concatenate([first, second], axis=2).reshape(rows, 2 * K)
+
+
 def _rows_to_groups(A: np.ndarray, g: int) -> np.ndarray:
     m, d = A.shape
     return A.reshape(m * (d // g), g)
 
 
-def init_step(W_rows: np.ndarray, rsig: np.ndarray, bits: int, group: int):
+def encode_operand(x: np.ndarray, split: str, side: str = "A"):
+    """The eigenbasis GEMMs' operand planes of x in the given split precision:
+    "3xtf32" -> (tf32(x), tf32(x - tf32(x))) as float32; "mixed" -> split_mix."""
+    if split == "3xtf32":
+        return split_tf32(x)
+    if split == "mixed":
+        return split_mix(x, side)
+    raise ValueError(split)
+
+
+def init_step(W_rows: np.ndarray, rsig: np.ndarray, bits: int, group: int, split: str = "mixed"):
     """RTN start of the iteration in memory layout ([d_out][d_in]).
 
     y = W_hat; minmax grid; D = s (q - z); D~ = D * rsig (rsig = sqrt(diag H)),
@@ -143,21 +170,22 @@ def init_step(W_rows: np.ndarray, rsig: np.ndarray, bits: int, group: int):
     q = round_to_grid(yg, s, z, L)
     D = dequantize(q, s, z).reshape(m, d)
     Dt = _f(D * _f(rsig)[None, :])
-    hi, lo = split_tf32(Dt)
+    hi, pc = encode_operand(Dt, split, "A")
     return dict(codes=q.reshape(m, d).astype(np.uint8), scale=s.reshape(m, d // group),
-                zero=z.reshape(m, d // group), P=Dt, P_hi=hi, P_lo=lo)
+                zero=z.reshape(m, d // group), P=Dt, P_hi=hi, P_lo=pc)
 
 
 def epilogue_step(W_acc: np.ndarray, V: np.ndarray, sigma: np.ndarray, rsig: np.ndarray,
                   hdiag: np.ndarray, s_prev: np.ndarray, z_prev: np.ndarray,
-                  codes_prev: np.ndarray, bits: int, group: int, mode: str):
+                  codes_prev: np.ndarray, bits: int, group: int, mode: str,
+                  split: str = "mixed"):
     """One fused projection + dual update in memory layout ([d_out][d_in]).
 
     Per element (i = input channel):
       t  = W~ + V~          y  = sigma_i t
       grid (minmax | lsq | frozen) per group of `group` columns of one row
       q  = clamp(rint(y/s) + z, 0, L),  D = s (q - z),  D~ = D * rsig_i
-      V~' = t - D~          P  = D~ - V~'   (split into tf32 hi/lo planes)
+      V~' = t - D~          P  = D~ - V~'   (in the operand encoding of `split`)
     Residual sums (float64 here; the kernels sum in float32, compared with a
     tolerance): r2 = sum (W~ - D~)^2 and s2 = sum (D~ - D~_prev)^2 where
     D~_prev = s_prev (q_prev - z_prev) * rsig.
@@ -185,7 +213,7 @@ def epilogue_step(W_acc: np.ndarray, V: np.ndarray, sigma: np.ndarray, rsig: np.
     Dt = _f(D * _f(rsig)[None, :])
     V_new = _f(t - Dt)
     P = _f(Dt - V_new)
-    hi, lo = split_tf32(P)
+    hi, lo = encode_operand(P, split, "A")
     qp = _rows_to_groups(_f(codes_prev), group)
     Dt_prev = _f(dequantize(qp, sp, zp).reshape(m, d) * _f(rsig)[None, :])
     r2 = float(np.sum((W_acc.astype(np.float64) - Dt) ** 2))

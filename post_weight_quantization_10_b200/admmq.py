@@ -18,6 +18,7 @@ from .build import LIB
 OK = 0
 GRID_MINMAX, GRID_LSQ, GRID_FROZEN = 0, 1, 2
 GRID_MODES = {"minmax": GRID_MINMAX, "lsq": GRID_LSQ, "frozen": GRID_FROZEN}
+SPLIT_MODES = {"auto": 0, "3xtf32": 1, "mixed": 2}
 DTYPE_F32, DTYPE_BF16 = 0, 1
 BUFFERS = ["sigma", "rsig", "hdiag", "lambda", "V", "C0", "P_hi", "P_lo", "T_hi", "T_lo",
            "E_hi", "E_lo", "Ht", "status"]
@@ -32,7 +33,8 @@ class AdmmqError(RuntimeError):
 class _Params(ctypes.Structure):
     _fields_ = [("bits", ctypes.c_int), ("group", ctypes.c_int), ("iters", ctypes.c_int),
                 ("rho0", ctypes.c_float), ("gamma", ctypes.c_float),
-                ("lambda_rel", ctypes.c_float), ("grid_mode", ctypes.c_int)]
+                ("lambda_rel", ctypes.c_float), ("grid_mode", ctypes.c_int),
+                ("split_mode", ctypes.c_int)]
 
 
 @dataclass
@@ -44,10 +46,11 @@ class Params:
     gamma: float = 1.05
     lambda_rel: float = 0.01
     grid: str = "lsq"
+    split: str = "auto"   # eigenbasis GEMM split precision: auto | 3xtf32 | mixed
 
     def c(self) -> _Params:
         return _Params(self.bits, self.group, self.iters, self.rho0, self.gamma, self.lambda_rel,
-                       GRID_MODES[self.grid])
+                       GRID_MODES[self.grid], SPLIT_MODES[self.split])
 
 
 _lib = None
@@ -101,8 +104,9 @@ def lib():
         "admmq_set_timing": (_i, [_vp, _i]),
         "admmq_get_timing": (_i, [_vp, ctypes.POINTER(ctypes.c_double),
                                   ctypes.POINTER(ctypes.c_int)]),
-        "admmq_project": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp,
-                               _vp, _vp, _vp]),
+        "admmq_project": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp,
+                               _vp, _vp, _vp, _vp]),
+        "admmq_split_mode": (_i, [_vp]),
         "admmq_gptq_workspace_bytes": (_sz, [_i, _i, _i]),
         "admmq_gptq": (_i, [_vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float, _i, _vp, _vp, _vp, _vp,
                             _sz, _vp]),
@@ -246,13 +250,24 @@ class Solver:
             return raw.view(torch.float32)
         if name in ("V", "C0"):
             return raw.view(torch.float32).view(m, d)
-        if name in ("P_hi", "P_lo", "T_hi", "T_lo"):
+        mixed = self.split == "mixed"
+        if name in ("P_hi", "T_hi") or (name in ("P_lo", "T_lo") and not mixed):
             return raw.view(torch.float32).view(m, d)
-        if name in ("E_hi", "E_lo"):
+        if name in ("P_lo", "T_lo"):   # bf16 correction rows (bit patterns)
+            return raw.view(torch.int16).view(m, 2 * d)
+        if name == "E_hi" or (name == "E_lo" and not mixed):
             return raw.view(torch.float32).view(d, d)
+        if name == "E_lo":
+            return raw.view(torch.int16).view(d, 2 * d)
         if name == "Ht":
             return raw.view(torch.float64).view(d, d)
         return raw.view(torch.int32)
+
+    @property
+    def split(self) -> str:
+        """The eigenbasis GEMMs' split precision ("3xtf32" or "mixed")."""
+        mode = int(lib().admmq_split_mode(self._ctx))
+        return {1: "3xtf32", 2: "mixed"}[mode]
 
     def dump_wtilde(self, out: torch.Tensor | None):
         _check(lib().admmq_debug_dump_wtilde(self._ctx, _ptr(out)), "admmq_debug_dump_wtilde")
@@ -279,13 +294,16 @@ def pack(codes: torch.Tensor, bits: int, out: torch.Tensor | None = None, stream
 
 
 def project(wtilde, V, sigma, rsig, hdiag, bits, group, grid, codes, scale, zero, P_hi, P_lo,
-            resid=None, stream=None):
+            resid=None, split="mixed", stream=None):
+    """Stand-alone projection; P_lo is fp32 [m][d] for split "3xtf32", int16
+    (bf16 bit patterns) [m][2d] for "mixed"."""
     m, d = wtilde.shape
     if resid is None:
         resid = torch.zeros(2, dtype=torch.float64, device=wtilde.device)
     _check(lib().admmq_project(_ptr(wtilde), _ptr(V), _ptr(sigma), _ptr(rsig), _ptr(hdiag), d, m,
-                               bits, group, GRID_MODES[grid], _ptr(codes), _ptr(scale),
-                               _ptr(zero), _ptr(P_hi), _ptr(P_lo), _ptr(resid), _stream(stream)),
+                               bits, group, GRID_MODES[grid], SPLIT_MODES[split], _ptr(codes),
+                               _ptr(scale), _ptr(zero), _ptr(P_hi), _ptr(P_lo), _ptr(resid),
+                               _stream(stream)),
            "admmq_project")
     return resid
 

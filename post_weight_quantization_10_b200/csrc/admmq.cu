@@ -12,6 +12,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <type_traits>
 #include <vector>
 
 #include "../../include/admmq.h"
@@ -27,9 +28,15 @@ inline void count_launch() { __atomic_fetch_add(&g_launches, 1ull, __ATOMIC_RELA
 // X^T X: bf16, both operands MN-major (X is token-major).
 // Promoted every 4 k-blocks (16 MMAs of K = 16).
 using GramCfg = GemmCfg<KIND_BF16, 256, 1, true, true, 4, 4>;
-// Eigenbasis GEMMs: 3xTF32 split precision, K-major operands.
-// Promoted every 8 k-blocks (96 MMAs of K = 8): drift ~2e-6 per product.
-using EigCfg = GemmCfg<KIND_TF32, 128, 2, false, false, 3, 8>;
+// Eigenbasis GEMMs, K-major operands, promoted every 8 k-blocks:
+//   mixed split (tf32 hi.hi + one bf16 product for the corrections, 64 MMAs
+//   per chunk) for large layers, 3xTF32 (96 MMAs per chunk) where the
+//   reduction is short enough that the split's own rounding would dominate.
+using EigCfg = GemmCfg<KIND_MIX, 128, 2, false, false, 3, 8>;
+using EigCfg3 = GemmCfg<KIND_TF32, 128, 2, false, false, 3, 8>;
+static_assert(EigCfg::BN == EigCfg3::BN && EigCfg::BK == EigCfg3::BK, "same tile geometry");
+// d_in from which the automatic split mode picks the mixed split
+constexpr int kMixedFromDin = 2048;
 
 // Setup status words (ws status[1]).
 enum { SETUP_OK = 0, SETUP_NONFINITE = 1, SETUP_NOT_PD = 2 };
@@ -92,26 +99,26 @@ __device__ __forceinline__ float load_w<__nv_bfloat16>(const __nv_bfloat16* p, l
 
 #include "gptq.cuh"
 
-// W^~ = Sigma^-1 W_hat (rows = output channels), split into tf32 hi/lo planes.
+// W^~ = Sigma^-1 W_hat (rows = output channels) in the operand encoding (A side).
 template <typename T>
 __global__ void k_scale_weights(const T* __restrict__ W, const float* __restrict__ rsig, int d,
-                                long long total, float* __restrict__ hi, float* __restrict__ lo) {
+                                long long total, float* __restrict__ hi, void* lo, bool mix) {
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
        idx += (long long)gridDim.x * blockDim.x) {
-    const int i = (int)(idx % d);
+    const long long row = idx / d;
+    const int i = (int)(idx - row * d);
     const float w = __fmul_rn(load_w<T>(W, idx), rsig[i]);
-    float h, l;
-    split2(w, h, l);
-    hi[idx] = h;
-    lo[idx] = l;
+    const float h = tf32_rne(w);
+    put_operand1(mix, false, hi + row * d, mix ? lo_row<true>(lo, row, d) : lo_row<false>(lo, row, d),
+                 i, h, __fsub_rn(w, h));
   }
 }
 
 // Eigenvector buffer (row k = k-th eigenvector, from the column-major solver
-// output) -> tf32 hi/lo planes of E = Q^T [k][i] and of Q [i][k].
+// output) -> operand planes (B side) of E = Q^T [k][i] and of Q [i][k]; the
+// lo part comes from the float64 value (e - hi).
 __global__ void k_split_eigvecs(const double* __restrict__ Evec, int d, float* __restrict__ e_hi,
-                                float* __restrict__ e_lo, float* __restrict__ q_hi,
-                                float* __restrict__ q_lo) {
+                                void* e_lo, float* __restrict__ q_hi, void* q_lo, bool mix) {
   __shared__ float th[32][33], tl[32][33];
   const int k0 = blockIdx.y * 32, i0 = blockIdx.x * 32;
   for (int r = threadIdx.y; r < 32; r += blockDim.y) {
@@ -120,9 +127,9 @@ __global__ void k_split_eigvecs(const double* __restrict__ Evec, int d, float* _
     if (k < d && i < d) {
       const double e = Evec[(long long)k * d + i];
       h = tf32_rne((float)e);
-      l = tf32_rne((float)(e - (double)h));
-      e_hi[(long long)k * d + i] = h;
-      e_lo[(long long)k * d + i] = l;
+      l = (float)(e - (double)h);
+      put_operand1(mix, true, e_hi + (long long)k * d,
+                   mix ? lo_row<true>(e_lo, k, d) : lo_row<false>(e_lo, k, d), i, h, l);
     }
     th[r][threadIdx.x] = h;
     tl[r][threadIdx.x] = l;
@@ -130,10 +137,10 @@ __global__ void k_split_eigvecs(const double* __restrict__ Evec, int d, float* _
   __syncthreads();
   for (int r = threadIdx.y; r < 32; r += blockDim.y) {
     const int i = i0 + r, k = k0 + threadIdx.x;
-    if (k < d && i < d) {
-      q_hi[(long long)i * d + k] = th[threadIdx.x][r];
-      q_lo[(long long)i * d + k] = tl[threadIdx.x][r];
-    }
+    if (k < d && i < d)
+      put_operand1(mix, true, q_hi + (long long)i * d,
+                   mix ? lo_row<true>(q_lo, i, d) : lo_row<false>(q_lo, i, d), k,
+                   th[threadIdx.x][r], tl[threadIdx.x][r]);
   }
 }
 
@@ -146,12 +153,13 @@ __global__ void k_eigvals(const double* __restrict__ ev, int d, float* __restric
   }
 }
 
-// RTN start: D_0 = min/max-grid rounding of W_hat, V~ = 0, P = D~_0.
+// RTN start: D_0 = min/max-grid rounding of W_hat, V~ = 0, P = D~_0 (operand
+// encoding, A side).
 template <typename T>
 __global__ void k_init_rtn(const T* __restrict__ W, const float* __restrict__ rsig, int m, int d,
                            int g, int L, uint8_t* __restrict__ codes, float* __restrict__ scale,
                            float* __restrict__ zero, float* __restrict__ V,
-                           float* __restrict__ p_hi, float* __restrict__ p_lo) {
+                           float* __restrict__ p_hi, void* p_lo, bool mix) {
   const int ngr = d / g;
   const long long total = (long long)m * ngr;
   const float Lf = (float)L;
@@ -178,24 +186,25 @@ __global__ void k_init_rtn(const T* __restrict__ W, const float* __restrict__ rs
       const float q = clampq(__fadd_rn(rintf(__fdiv_rn(y, s)), z), Lf);
       const float D = __fmul_rn(s, __fsub_rn(q, z));
       const float dt = __fmul_rn(D, rsig[col0 + e]);
-      float h, l;
-      split2(dt, h, l);
+      const float h = tf32_rne(dt);
       codes[base + e] = (uint8_t)q;
       V[base + e] = 0.f;
-      p_hi[base + e] = h;
-      p_lo[base + e] = l;
+      put_operand1(mix, false, p_hi + row * d,
+                   mix ? lo_row<true>(p_lo, row, d) : lo_row<false>(p_lo, row, d), col0 + e, h,
+                   __fsub_rn(dt, h));
     }
     scale[gi] = s;
     zero[gi] = z;
   }
 }
 
-// Delta~ = D~ - W^~ (scaled coordinates) as tf32 planes, for the objective.
+// Delta~ = D~ - W^~ (scaled coordinates) in the operand encoding (A side),
+// for the objective.
 template <typename T>
 __global__ void k_delta_planes(const T* __restrict__ W, const uint8_t* __restrict__ codes,
                                const float* __restrict__ scale, const float* __restrict__ zero,
                                const float* __restrict__ rsig, int d, int g, long long total,
-                               float* __restrict__ hi, float* __restrict__ lo) {
+                               float* __restrict__ hi, void* lo, bool mix) {
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
        idx += (long long)gridDim.x * blockDim.x) {
     const long long row = idx / d;
@@ -204,10 +213,9 @@ __global__ void k_delta_planes(const T* __restrict__ W, const uint8_t* __restric
     const float D = __fmul_rn(scale[gi], __fsub_rn((float)codes[idx], zero[gi]));
     const float dt = __fmul_rn(D, rsig[i]);
     const float wt = __fmul_rn(load_w<T>(W, idx), rsig[i]);
-    float h, l;
-    split2(__fsub_rn(dt, wt), h, l);
-    hi[idx] = h;
-    lo[idx] = l;
+    const float x = __fsub_rn(dt, wt), h = tf32_rne(x);
+    put_operand1(mix, false, hi + row * d, mix ? lo_row<true>(lo, row, d) : lo_row<false>(lo, row, d),
+                 i, h, __fsub_rn(x, h));
   }
 }
 
@@ -343,11 +351,11 @@ __global__ void __launch_bounds__(256) k_pack(const uint8_t* __restrict__ codes,
 }
 
 // Standalone projection: one thread per (row, group), W~ read from memory.
-template <int MODE>
+template <int MODE, bool MIX>
 __global__ void k_project(const float* __restrict__ wt, float* V, const float* __restrict__ sig,
                           const float* __restrict__ rsig, const float* __restrict__ hd, int m, int d,
                           int g, int L, uint8_t* codes, float* scale, float* zero, float* p_hi,
-                          float* p_lo, double* resid) {
+                          void* p_lo, double* resid) {
   const int row = blockIdx.x * blockDim.x + threadIdx.x;
   const int grp = blockIdx.y;
   const bool valid = row < m;
@@ -361,7 +369,8 @@ __global__ void k_project(const float* __restrict__ wt, float* V, const float* _
   r.hd = hd + col0;
   r.codes = codes + off;
   r.phi = p_hi + off;
-  r.plo = p_lo + off;
+  r.plo = MIX ? (void*)(reinterpret_cast<uint16_t*>(p_lo) + (long long)(valid ? row : 0) * 2 * d + 2 * col0)
+              : (void*)(reinterpret_cast<float*>(p_lo) + off);
   r.scale = scale + goff;
   r.zero = zero + goff;
   r.wdump = nullptr;
@@ -375,7 +384,7 @@ __global__ void k_project(const float* __restrict__ wt, float* V, const float* _
     }
   };
   float r2 = 0.f, s2 = 0.f;
-  project_group<MODE>(loadw, r, g, L, r2, s2);
+  project_group<MODE, MIX>(loadw, r, g, L, r2, s2);
   r2 = warp_sum(r2);
   s2 = warp_sum(s2);
   if ((threadIdx.x & 31) == 0) {
@@ -467,6 +476,16 @@ cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
   return cudaGetLastError();
 }
 
+// An eigenbasis GEMM (A and B operand maps, plane 0 and 1) with the split
+// precision of the context: EpiM for the mixed split, Epi3 for 3xTF32.
+template <class Epi3, class EpiM>
+cudaError_t launch_eig(bool mix, const CUtensorMap (&a)[2], const CUtensorMap (&b)[2],
+                       const GemmGeom& g, const typename EpiM::Params& ep, cudaStream_t st) {
+  static_assert(std::is_same<typename Epi3::Params, typename EpiM::Params>::value, "same params");
+  return mix ? launch_gemm<EigCfg, EpiM>(a[0], a[1], b[0], b[1], g, ep, st)
+             : launch_gemm<EigCfg3, Epi3>(a[0], a[1], b[0], b[1], g, ep, st);
+}
+
 int device_ok() {
   int dev = 0, major = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return ADMMQ_ERR_CUDA;
@@ -521,8 +540,14 @@ struct admmq_ctx {
   double* work;
   int lwork;
   int* devinfo;
-  float *E_hi, *E_lo, *Q_hi, *Q_lo;          // [d][d] tf32 planes
-  float *Wt_hi, *Wt_lo, *P_hi, *P_lo, *T_hi, *T_lo;     // [m][d] tf32 planes
+  // operand planes: *_hi tf32 in fp32 words [rows][d]; *_lo the tf32 lo
+  // plane [rows][d] (3xTF32) or the bf16 correction rows [rows][2d] (mixed);
+  // A side: Wt, P, T; B side: E, Q
+  bool mix;
+  float *E_hi, *Q_hi;                          // [d][d]
+  void *E_lo, *Q_lo;
+  float *Wt_hi, *P_hi, *T_hi;                  // [m][d]
+  void *Wt_lo, *P_lo, *T_lo;
   float *C0, *V;                               // [m][d]
   float* resid_part;    // [iters][tiles][4][2]
   float* obj_part;      // [tiles][4]
@@ -592,6 +617,8 @@ int check_params(int d, int m, const admmq_params* p) {
   if (p->bits < 1 || p->bits > 8 || p->iters < 0) return ADMMQ_ERR_INVALID_ARG;
   if (!(p->rho0 > 0.f) || !(p->gamma > 0.f) || !(p->lambda_rel >= 0.f)) return ADMMQ_ERR_INVALID_ARG;
   if (p->grid_mode < ADMMQ_GRID_MINMAX || p->grid_mode > ADMMQ_GRID_FROZEN)
+    return ADMMQ_ERR_INVALID_ARG;
+  if (p->split_mode < ADMMQ_SPLIT_AUTO || p->split_mode > ADMMQ_SPLIT_MIXED)
     return ADMMQ_ERR_INVALID_ARG;
   return ADMMQ_OK;
 }
@@ -751,6 +778,8 @@ int admmq_create(admmq_ctx** out, int d, int m, const admmq_params* p, void* ws,
   c->m = m;
   c->p = *p;
   c->L = (1 << p->bits) - 1;
+  c->mix = p->split_mode == ADMMQ_SPLIT_MIXED ||
+           (p->split_mode == ADMMQ_SPLIT_AUTO && d >= kMixedFromDin);
   cudaGetDevice(&c->dev);
   c->ws = (uint8_t*)ws;
   c->ws_bytes = ws_bytes;
@@ -768,28 +797,28 @@ int admmq_create(admmq_ctx** out, int d, int m, const admmq_params* p, void* ws,
   c->lwork = lwork;
   c->devinfo = (int*)(b + L.devinfo);
   c->E_hi = (float*)(b + L.E_hi);
-  c->E_lo = (float*)(b + L.E_lo);
+  c->E_lo = (void*)(b + L.E_lo);
   c->Q_hi = (float*)(b + L.Q_hi);
-  c->Q_lo = (float*)(b + L.Q_lo);
+  c->Q_lo = (void*)(b + L.Q_lo);
   c->Wt_hi = (float*)(b + L.Wt_hi);
-  c->Wt_lo = (float*)(b + L.Wt_lo);
+  c->Wt_lo = (void*)(b + L.Wt_lo);
   c->P_hi = (float*)(b + L.P_hi);
-  c->P_lo = (float*)(b + L.P_lo);
+  c->P_lo = (void*)(b + L.P_lo);
   c->T_hi = (float*)(b + L.T_hi);
-  c->T_lo = (float*)(b + L.T_lo);
+  c->T_lo = (void*)(b + L.T_lo);
   c->C0 = (float*)(b + L.C0);
   c->V = (float*)(b + L.V);
   c->resid_part = (float*)(b + L.resid_part);
   c->obj_part = (float*)(b + L.obj_part);
   c->tiles_eig = cdiv(m, kBM) * cdiv(d, EigCfg::BN);
   bool ok = true;
-  ok &= make_map(&c->mWt[0], c->Wt_hi, d, m, kBM, true) && make_map(&c->mWt[1], c->Wt_lo, d, m, kBM, true);
-  ok &= make_map(&c->mP[0], c->P_hi, d, m, kBM, true) && make_map(&c->mP[1], c->P_lo, d, m, kBM, true);
-  ok &= make_map(&c->mT[0], c->T_hi, d, m, kBM, true) && make_map(&c->mT[1], c->T_lo, d, m, kBM, true);
+  ok &= make_map(&c->mWt[0], c->Wt_hi, d, m, kBM, true) && make_map(&c->mWt[1], c->Wt_lo, c->mix ? 2 * (uint64_t)d : (uint64_t)d, m, kBM, !c->mix);
+  ok &= make_map(&c->mP[0], c->P_hi, d, m, kBM, true) && make_map(&c->mP[1], c->P_lo, c->mix ? 2 * (uint64_t)d : (uint64_t)d, m, kBM, !c->mix);
+  ok &= make_map(&c->mT[0], c->T_hi, d, m, kBM, true) && make_map(&c->mT[1], c->T_lo, c->mix ? 2 * (uint64_t)d : (uint64_t)d, m, kBM, !c->mix);
   ok &= make_map(&c->mE[0], c->E_hi, d, d, EigCfg::BN, true) &&
-        make_map(&c->mE[1], c->E_lo, d, d, EigCfg::BN, true);
+        make_map(&c->mE[1], c->E_lo, c->mix ? 2 * (uint64_t)d : (uint64_t)d, d, EigCfg::BN, !c->mix);
   ok &= make_map(&c->mQ[0], c->Q_hi, d, d, EigCfg::BN, true) &&
-        make_map(&c->mQ[1], c->Q_lo, d, d, EigCfg::BN, true);
+        make_map(&c->mQ[1], c->Q_lo, c->mix ? 2 * (uint64_t)d : (uint64_t)d, d, EigCfg::BN, !c->mix);
   if (!ok || cusolverDnCreate(&c->solver) != CUSOLVER_STATUS_SUCCESS) {
     delete c;
     return ADMMQ_ERR_CUDA;
@@ -821,10 +850,10 @@ int admmq_prepare(admmq_ctx* c, const float* G, const void* W_hat, int w_dtype, 
   const long long md = (long long)m * d;
   if (w_dtype == ADMMQ_DTYPE_F32)
     count_launch(), k_scale_weights<float><<<grid_for(md), 256, 0, st>>>((const float*)W_hat, c->rsig, d, md,
-                                                         c->Wt_hi, c->Wt_lo);
+                                                         c->Wt_hi, c->Wt_lo, c->mix);
   else
     count_launch(), k_scale_weights<__nv_bfloat16><<<grid_for(md), 256, 0, st>>>(
-        (const __nv_bfloat16*)W_hat, c->rsig, d, md, c->Wt_hi, c->Wt_lo);
+        (const __nv_bfloat16*)W_hat, c->rsig, d, md, c->Wt_hi, c->Wt_lo, c->mix);
   CK(cudaGetLastError());
   c->prepared = true;
   return ADMMQ_OK;
@@ -846,7 +875,7 @@ int admmq_eigh(admmq_ctx* c, void* stream) {
   count_launch(), k_eigvals<<<grid_for(d), 256, 0, st>>>(c->evals, d, c->lam32, c->status);
   CK(cudaGetLastError());
   count_launch(), k_split_eigvecs<<<dim3(cdiv(d, 32), cdiv(d, 32)), dim3(32, 8), 0, st>>>(c->Ht, d, c->E_hi, c->E_lo,
-                                                                          c->Q_hi, c->Q_lo);
+                                                                          c->Q_hi, c->Q_lo, c->mix);
   CK(cudaGetLastError());
   int info = 0;
   CK(cudaMemcpyAsync(&info, c->devinfo, sizeof(int), cudaMemcpyDeviceToHost, st));
@@ -879,17 +908,17 @@ int admmq_init(admmq_ctx* c, uint8_t* codes, float* scale, float* zero, void* st
   // C0' = Lambda Q^T W^~   (row j, column k)
   GemmGeom g = make_geom(m, d, d, EigCfg::BN, EigCfg::BK, 1, false, c->status);
   EpiScaleStore<EigCfg::BN>::Params ep{c->C0, c->lam32, d};
-  CK((launch_gemm<EigCfg, EpiScaleStore<EigCfg::BN>>(c->mWt[0], c->mWt[1], c->mE[0], c->mE[1], g,
-                                                      ep, st)));
+  CK((launch_eig<EpiScaleStore<EigCfg::BN>, EpiScaleStore<EigCfg::BN>>(c->mix, c->mWt, c->mE, g, ep,
+                                                                         st)));
   const long long groups = (long long)m * (d / c->p.group);
   if (c->w_dtype == ADMMQ_DTYPE_F32)
     count_launch(), k_init_rtn<float><<<grid_for(groups, 128), 128, 0, st>>>(
         (const float*)c->W_hat, c->rsig, m, d, c->p.group, c->L, codes, scale, zero, c->V,
-        c->P_hi, c->P_lo);
+        c->P_hi, c->P_lo, c->mix);
   else
     count_launch(), k_init_rtn<__nv_bfloat16><<<grid_for(groups, 128), 128, 0, st>>>(
         (const __nv_bfloat16*)c->W_hat, c->rsig, m, d, c->p.group, c->L, codes, scale, zero,
-        c->V, c->P_hi, c->P_lo);
+        c->V, c->P_hi, c->P_lo, c->mix);
   CK(cudaGetLastError());
   c->inited = true;
   return ADMMQ_OK;
@@ -917,9 +946,9 @@ int admmq_iterate(admmq_ctx* c, int t0, int count, uint8_t* codes, float* scale,
       e2 = c->ev[c->ev.size() - 1];
       CK(cudaEventRecord(e0, st));
     }
-    EpiTUpdate<EigCfg::BN>::Params p1{c->C0, c->lam32, c->T_hi, c->T_lo, rho, d};
-    CK((launch_gemm<EigCfg, EpiTUpdate<EigCfg::BN>>(c->mP[0], c->mP[1], c->mE[0], c->mE[1], g, p1,
-                                                     st)));
+    TUpdateParams p1{c->C0, c->lam32, c->T_hi, c->T_lo, rho, d};
+    CK((launch_eig<EpiTUpdate<EigCfg::BN, false>, EpiTUpdate<EigCfg::BN, true>>(c->mix, c->mP, c->mE,
+                                                                                g, p1, st)));
     if (c->timing) CK(cudaEventRecord(e1, st));
     ProjParams p2;
     p2.V = c->V;
@@ -939,16 +968,16 @@ int admmq_iterate(admmq_ctx* c, int t0, int count, uint8_t* codes, float* scale,
     cudaError_t e;
     switch (c->p.grid_mode) {
       case ADMMQ_GRID_MINMAX:
-        e = launch_gemm<EigCfg, EpiProject<EigCfg::BN, GRID_MINMAX>>(c->mT[0], c->mT[1], c->mQ[0],
-                                                                     c->mQ[1], g, p2, st);
+        e = launch_eig<EpiProject<EigCfg::BN, GRID_MINMAX, false>,
+                       EpiProject<EigCfg::BN, GRID_MINMAX, true>>(c->mix, c->mT, c->mQ, g, p2, st);
         break;
       case ADMMQ_GRID_LSQ:
-        e = launch_gemm<EigCfg, EpiProject<EigCfg::BN, GRID_LSQ>>(c->mT[0], c->mT[1], c->mQ[0],
-                                                                  c->mQ[1], g, p2, st);
+        e = launch_eig<EpiProject<EigCfg::BN, GRID_LSQ, false>,
+                       EpiProject<EigCfg::BN, GRID_LSQ, true>>(c->mix, c->mT, c->mQ, g, p2, st);
         break;
       default:
-        e = launch_gemm<EigCfg, EpiProject<EigCfg::BN, GRID_FROZEN>>(c->mT[0], c->mT[1], c->mQ[0],
-                                                                     c->mQ[1], g, p2, st);
+        e = launch_eig<EpiProject<EigCfg::BN, GRID_FROZEN, false>,
+                       EpiProject<EigCfg::BN, GRID_FROZEN, true>>(c->mix, c->mT, c->mQ, g, p2, st);
         break;
     }
     CK(e);
@@ -973,16 +1002,16 @@ int admmq_finish(admmq_ctx* c, const uint8_t* codes, const float* scale, const f
     if (c->w_dtype == ADMMQ_DTYPE_F32)
       count_launch(), k_delta_planes<float><<<grid_for(md), 256, 0, st>>>((const float*)c->W_hat, codes, scale,
                                                           zero, c->rsig, d, c->p.group, md,
-                                                          c->T_hi, c->T_lo);
+                                                          c->T_hi, c->T_lo, c->mix);
     else
       count_launch(), k_delta_planes<__nv_bfloat16><<<grid_for(md), 256, 0, st>>>(
           (const __nv_bfloat16*)c->W_hat, codes, scale, zero, c->rsig, d, c->p.group, md, c->T_hi,
-          c->T_lo);
+          c->T_lo, c->mix);
     CK(cudaGetLastError());
     GemmGeom g = make_geom(m, d, d, EigCfg::BN, EigCfg::BK, 1, false, c->status);
     EpiObjective<EigCfg::BN>::Params ep{c->lam32, c->obj_part};
-    CK((launch_gemm<EigCfg, EpiObjective<EigCfg::BN>>(c->mT[0], c->mT[1], c->mE[0], c->mE[1], g,
-                                                       ep, st)));
+    CK((launch_eig<EpiObjective<EigCfg::BN>, EpiObjective<EigCfg::BN>>(c->mix, c->mT, c->mE, g, ep,
+                                                                         st)));
     count_launch(), k_reduce_objective<<<1, 256, 0, st>>>(c->obj_part, c->tiles_eig * 4, objective);
     CK(cudaGetLastError());
   }
@@ -1082,13 +1111,14 @@ int admmq_get_timing(admmq_ctx* c, double ms[2], int launches[2]) {
 }
 
 int admmq_project(const float* wt, float* V, const float* sig, const float* rsig,
-                  const float* hd, int d, int m, int bits, int g, int mode, uint8_t* codes,
-                  float* scale, float* zero, float* p_hi, float* p_lo, double* resid,
-                  void* stream) {
+                  const float* hd, int d, int m, int bits, int g, int mode, int split,
+                  uint8_t* codes, float* scale, float* zero, float* p_hi, void* p_lo,
+                  double* resid, void* stream) {
   if (!wt || !V || !sig || !rsig || !hd || !codes || !scale || !zero || !p_hi || !p_lo || !resid)
     return ADMMQ_ERR_INVALID_ARG;
   if (d <= 0 || m <= 0 || d % 32 != 0 || !(g == 32 || g == 64 || g == 128) || d % g != 0 ||
-      bits < 1 || bits > 8 || mode < 0 || mode > 2)
+      bits < 1 || bits > 8 || mode < 0 || mode > 2 ||
+      !(split == ADMMQ_SPLIT_3XTF32 || split == ADMMQ_SPLIT_MIXED))
     return ADMMQ_ERR_INVALID_ARG;
   if (!aligned32(V) || !aligned32(codes) || !aligned32(p_hi) || !aligned32(p_lo) ||
       ((uintptr_t)wt & 15) || ((uintptr_t)sig & 31) || ((uintptr_t)rsig & 31) || ((uintptr_t)hd & 31))
@@ -1097,17 +1127,29 @@ int admmq_project(const float* wt, float* V, const float* sig, const float* rsig
   CK(cudaMemsetAsync(resid, 0, 2 * sizeof(double), st));
   dim3 grid(cdiv(m, 128), d / g);
   const int L = (1 << bits) - 1;
-  if (mode == ADMMQ_GRID_MINMAX)
-    count_launch(), k_project<GRID_MINMAX><<<grid, 128, 0, st>>>(wt, V, sig, rsig, hd, m, d, g, L, codes, scale,
-                                                 zero, p_hi, p_lo, resid);
-  else if (mode == ADMMQ_GRID_LSQ)
-    count_launch(), k_project<GRID_LSQ><<<grid, 128, 0, st>>>(wt, V, sig, rsig, hd, m, d, g, L, codes, scale, zero,
-                                              p_hi, p_lo, resid);
-  else
-    count_launch(), k_project<GRID_FROZEN><<<grid, 128, 0, st>>>(wt, V, sig, rsig, hd, m, d, g, L, codes, scale,
-                                                 zero, p_hi, p_lo, resid);
+  const bool mix = split == ADMMQ_SPLIT_MIXED;
+#define PROJECT_CASE(MODE)                                                                   \
+  if (mix)                                                                                   \
+    count_launch(), k_project<MODE, true><<<grid, 128, 0, st>>>(wt, V, sig, rsig, hd, m, d, g, L, \
+                                                                codes, scale, zero, p_hi, p_lo, resid); \
+  else                                                                                       \
+    count_launch(), k_project<MODE, false><<<grid, 128, 0, st>>>(wt, V, sig, rsig, hd, m, d, g, L, \
+                                                                 codes, scale, zero, p_hi, p_lo, resid);
+  if (mode == ADMMQ_GRID_MINMAX) {
+    PROJECT_CASE(GRID_MINMAX)
+  } else if (mode == ADMMQ_GRID_LSQ) {
+    PROJECT_CASE(GRID_LSQ)
+  } else {
+    PROJECT_CASE(GRID_FROZEN)
+  }
+#undef PROJECT_CASE
   CK(cudaGetLastError());
   return ADMMQ_OK;
+}
+
+int admmq_split_mode(const admmq_ctx* c) {
+  if (!c) return ADMMQ_ERR_INVALID_ARG;
+  return c->mix ? ADMMQ_SPLIT_MIXED : ADMMQ_SPLIT_3XTF32;
 }
 
 // ------------------------------------------------------------------ GPTQ

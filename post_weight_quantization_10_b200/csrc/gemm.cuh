@@ -7,6 +7,13 @@
 // of K.  NPL = 2 runs the split-precision product used for fp32-accurate GEMMs
 // (3xTF32): every operand is stored as two tf32 planes (hi, lo) with
 // x ~= hi + lo, and each k-step issues A_hi*B_hi + A_hi*B_lo + A_lo*B_hi.
+// KIND_MIX is the cheaper split: plane 0 holds hi = tf32(x) (fp32 words),
+// plane 1 holds bf16 correction rows, each 128-byte row covering the same 32
+// K-elements as plane 0's row: [bf16(hi) x32 | bf16(lo) x32] for A and
+// [bf16(lo) x32 | bf16(hi) x32] for B, lo = x - hi.  Each k-step issues one
+// tf32 MMA on plane 0 and one bf16 MMA on plane 1, whose K = 16 runs over
+// hi(A).lo(B) and lo(A).hi(B): the same three terms in ~2/3 of the tensor
+// time, with the correction terms carried to bf16 precision.
 //
 // Promoted accumulation.  The tensor core adds every MMA into its fp32
 // accumulator with a small one-sided rounding error, so a long K sum drifts by
@@ -46,12 +53,15 @@ struct GemmGeom {
   int* status;        // kernel status word (device)
 };
 
-enum { KIND_BF16 = 1, KIND_TF32 = 2 };  // instruction-descriptor operand format
+// Operand kinds: KIND_BF16 / KIND_TF32 are the instruction-descriptor formats
+// of plain products.  KIND_MIX is the split-precision product with one tf32
+// plane and one bf16 correction plane per operand (see GemmCfg).
+enum { KIND_BF16 = 1, KIND_TF32 = 2, KIND_MIX = 3 };
 
 template <int KIND_, int BN_, int NPL_, bool A_MN_, bool B_MN_, int STAGES_, int KC_>
 struct GemmCfg {
   static constexpr int KIND = KIND_;
-  static constexpr int ELEM = KIND == KIND_BF16 ? 2 : 4;  // bytes per operand element
+  static constexpr int ELEM = KIND == KIND_BF16 ? 2 : 4;  // bytes per (plane-0) operand element
   static constexpr int BM = 128, BN = BN_, BK = 128 / ELEM, NPL = NPL_, STAGES = STAGES_;
   static constexpr int UK = 32 / ELEM;                     // K per MMA instruction
   static constexpr int KC = KC_;                           // k-blocks per promoted chunk
@@ -66,6 +76,10 @@ struct GemmCfg {
   static constexpr int BAR_BYTES = 8 * (2 * STAGES + 4 * RING + 2) + 16;
   static constexpr int SMEM = STAGES * STAGE + 1024 + BAR_BYTES;
   static_assert(BN == 128 || BN == 256, "BN must be 128 or 256");
+  static_assert(KIND != KIND_MIX || (NPL == 2 && !A_MN && !B_MN), "mixed split: two K-major planes");
+  // products per K step: 3xTF32 (hi.hi, hi.lo, lo.hi), mixed (tf32 hi.hi +
+  // one bf16 product over the [hi|lo] x [lo|hi] correction row), or one
+  static constexpr int PRODUCTS = KIND == KIND_MIX ? 2 : (NPL == 2 ? 3 : 1);
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -178,7 +192,8 @@ __global__ void __launch_bounds__(320, 1)
           for (int p = 0; p < NPL; ++p) {
             const uint32_t dA = st + p * Cfg::A_PLANE;
             if (!Cfg::A_MN) {
-              tma_load_2d(dA, mapA[p], k0, tm * BM, fb);
+              // a mixed correction plane holds two bf16 per K-element
+              tma_load_2d(dA, mapA[p], (Cfg::KIND == KIND_MIX && p == 1) ? 2 * k0 : k0, tm * BM, fb);
             } else {
 #pragma unroll
               for (int b = 0; b < BM / (128 / Cfg::ELEM); ++b)
@@ -189,7 +204,7 @@ __global__ void __launch_bounds__(320, 1)
           for (int p = 0; p < NPL; ++p) {
             const uint32_t dB = st + NPL * Cfg::A_PLANE + p * Cfg::B_PLANE;
             if (!Cfg::B_MN) {
-              tma_load_2d(dB, mapB[p], k0, tn * BN, fb);
+              tma_load_2d(dB, mapB[p], (Cfg::KIND == KIND_MIX && p == 1) ? 2 * k0 : k0, tn * BN, fb);
             } else {
 #pragma unroll
               for (int b = 0; b < BN / (128 / Cfg::ELEM); ++b)
@@ -207,7 +222,9 @@ __global__ void __launch_bounds__(320, 1)
   } else if (warp == 1) {
     // --------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t IDESC = idesc_f32acc(Cfg::KIND, BM, BN, Cfg::A_MN, Cfg::B_MN);
+      constexpr uint32_t IDESC = idesc_f32acc(Cfg::KIND == KIND_MIX ? (uint32_t)KIND_TF32 : Cfg::KIND,
+                                              BM, BN, Cfg::A_MN, Cfg::B_MN);
+      constexpr uint32_t IDESC16 = idesc_f32acc(KIND_BF16, BM, BN, Cfg::A_MN, Cfg::B_MN);
       // MN-major: blocks of 128 bytes along MN, BK K-rows each, LBO apart
       constexpr uint32_t LBO_A = Cfg::A_MN ? Cfg::BK * 128 : 16;
       constexpr uint32_t LBO_B = Cfg::B_MN ? Cfg::BK * 128 : 16;
@@ -257,14 +274,15 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
             for (int kk = 0; kk < Cfg::BK / Cfg::UK; ++kk) {
 #pragma unroll
-              for (int pr = 0; pr < (NPL == 2 ? 3 : 1); ++pr) {
-                const int pa = (pr == 2) ? 1 : 0;  // (hi,hi), (hi,lo), (lo,hi)
-                const int pb = (pr == 1) ? 1 : 0;
+              for (int pr = 0; pr < Cfg::PRODUCTS; ++pr) {
+                // 3xTF32: (hi,hi), (hi,lo), (lo,hi); mixed: (0,0) tf32, (1,1) bf16
+                const int pa = Cfg::KIND == KIND_MIX ? pr : ((pr == 2) ? 1 : 0);
+                const int pb = Cfg::KIND == KIND_MIX ? pr : ((pr == 1) ? 1 : 0);
                 const uint64_t ad = a0 + (uint64_t)(pa * kAPlane + kk * kKStepA);
                 const uint64_t bd = b0 + (uint64_t)(pb * kBPlane + kk * kKStepB);
                 const uint32_t accum = (kk > 0 || pr > 0) ? 1u : acc0;
-                if (Cfg::KIND == KIND_BF16)
-                  mma_bf16(dt, ad, bd, IDESC, accum);
+                if (Cfg::KIND == KIND_BF16 || (Cfg::KIND == KIND_MIX && pr == 1))
+                  mma_bf16(dt, ad, bd, Cfg::KIND == KIND_MIX ? IDESC16 : IDESC, accum);
                 else
                   mma_tf32(dt, ad, bd, IDESC, accum);
               }

@@ -22,10 +22,76 @@ __device__ __forceinline__ float tf32_rne(float x) {
   b = (b + 0xFFFu + ((b >> 13) & 1u)) & ~0x1FFFu;
   return __uint_as_float(b);
 }
-// x ~= hi + lo: hi = tf32(x), lo = tf32(x - hi)  (the 3xTF32 operand planes).
+// Operand encodings of the eigenbasis GEMMs.  Plane 0 always holds
+// hi = tf32(x) in an fp32 word.  Plane 1:
+//   3xTF32 (GemmCfg KIND_TF32, NPL 2): lo = tf32(x - hi), fp32 [rows][K];
+//   mixed  (GemmCfg KIND_MIX): bf16(hi) and bf16(lo), lo = x - hi (exact in
+//          float32), in correction rows of 64 bf16 per 32 columns,
+//          [rows][2K]: A operands [hi x32 | lo x32], B operands [lo x32 | hi x32].
+// x ~= hi + lo: hi = tf32(x), lo = tf32(x - hi)  (the 3xTF32 planes).
 __device__ __forceinline__ void split2(float x, float& hi, float& lo) {
   hi = tf32_rne(x);
   lo = tf32_rne(__fsub_rn(x, hi));
+}
+__device__ __forceinline__ void split_mix(float x, float& hi, uint16_t& hb, uint16_t& lb) {
+  hi = tf32_rne(x);
+  hb = bf16_bits(hi);
+  lb = bf16_bits(__fsub_rn(x, hi));
+}
+// Index of column c's hi entry in its correction row (lo is 32 further on
+// for A operands, 32 before for B operands).
+__device__ __forceinline__ long long cplane_hi(long long c, bool b_side) {
+  return 64 * (c >> 5) + (c & 31) + (b_side ? 32 : 0);
+}
+// Eight consecutive bf16 (16 bytes, 16-byte aligned).
+__device__ __forceinline__ void st_bf16x8(uint16_t* p, const uint16_t (&v)[8]) {
+  uint4 u;
+  u.x = (uint32_t)v[0] | ((uint32_t)v[1] << 16);
+  u.y = (uint32_t)v[2] | ((uint32_t)v[3] << 16);
+  u.z = (uint32_t)v[4] | ((uint32_t)v[5] << 16);
+  u.w = (uint32_t)v[6] | ((uint32_t)v[7] << 16);
+  *reinterpret_cast<uint4*>(p) = u;
+}
+// Plane-1 address of row `row` (ld = K columns) in either encoding.
+template <bool MIX>
+__device__ __forceinline__ void* lo_row(void* plane1, long long row, int ld) {
+  return MIX ? (void*)(reinterpret_cast<uint16_t*>(plane1) + row * 2 * ld)
+             : (void*)(reinterpret_cast<float*>(plane1) + row * ld);
+}
+// Columns c..c+7 (c % 8 == 0) of one A-side operand row in the encoding:
+// hi_row / lo_row point at the row's start in planes 0 / 1.
+template <bool MIX>
+__device__ __forceinline__ void put_operand8(float* hi_row, void* lo_row_p, long long c,
+                                             const float (&x)[8]) {
+  float hi[8];
+  if (MIX) {
+    uint16_t hb[8], lb[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) split_mix(x[k], hi[k], hb[k], lb[k]);
+    uint16_t* cr = reinterpret_cast<uint16_t*>(lo_row_p) + cplane_hi(c, false);
+    st_bf16x8(cr, hb);
+    st_bf16x8(cr + 32, lb);
+  } else {
+    float lo[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) split2(x[k], hi[k], lo[k]);
+    st_v8f(reinterpret_cast<float*>(lo_row_p) + c, lo);
+  }
+  st_v8f(hi_row + c, hi);
+}
+// One element (column c of a row) in the encoding, for element-wise kernels.
+// `lo_from` is the value whose rounding is stored as lo (x - hi, or a more
+// accurate residual when the source is float64).
+__device__ __forceinline__ void put_operand1(bool mix, bool b_side, float* hi_row, void* lo_row_p,
+                                             long long c, float hi, float lo_from) {
+  hi_row[c] = hi;
+  if (mix) {
+    uint16_t* cr = reinterpret_cast<uint16_t*>(lo_row_p) + cplane_hi(c, b_side);
+    cr[0] = bf16_bits(hi);
+    cr[b_side ? -32 : 32] = bf16_bits(lo_from);
+  } else {
+    reinterpret_cast<float*>(lo_row_p)[c] = tf32_rne(lo_from);
+  }
 }
 // clamp to [0, L]; adding +0 turns a -0 into +0 so the result never depends
 // on which zero fmaxf returns for (-0, +0)
@@ -58,7 +124,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 //   lsq:    q0 = clamp(rint(y/s_prev) + z_prev); weighted sums (w = diag H)
 //           in element order; slope/offset, integer zero point, slope again
 //   q = clamp(rint(y/s) + z, 0, L);  D = s (q - z);  D~ = D rsig
-//   V~' = t - D~;  P = D~ - V~'  (stored as tf32 hi/lo planes)
+//   V~' = t - D~;  P = D~ - V~'  (stored in the GEMM operand encoding)
 
 struct ProjRow {
   float* V;            // this row's V~ at the group's first column
@@ -66,15 +132,15 @@ struct ProjRow {
   const float* rsig;
   const float* hd;
   uint8_t* codes;
-  float* phi;
-  float* plo;
+  float* phi;          // P plane 0 at the group's first column
+  void* plo;           // P plane 1 at the group's first column (either encoding)
   float* scale;        // this group's scale / zero
   float* zero;
   float* wdump;        // optional raw W~ output
   bool valid;
 };
 
-template <int MODE, class LoadW>
+template <int MODE, bool MIX, class LoadW>
 __device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, int g, int L,
                                               float& r2, float& s2) {
   const float Lf = (float)L;
@@ -154,7 +220,7 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, i
       float ss[8], rr[8];
       load8_ro(r.sig + c + e, ss);
       load8_ro(r.rsig + c + e, rr);
-      float vn[8], hi[8], lo[8];
+      float vn[8], pv[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         const float t = __fadd_rn(w[e + k], vv[k]);
@@ -163,8 +229,7 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, i
         const float D = __fmul_rn(s, __fsub_rn(q, z));
         const float dt = __fmul_rn(D, rr[k]);
         vn[k] = __fsub_rn(t, dt);
-        const float p = __fsub_rn(dt, vn[k]);
-        split2(p, hi[k], lo[k]);
+        pv[k] = __fsub_rn(dt, vn[k]);
         const int wi = (e + k) >> 2, sh = 8 * ((e + k) & 3);
         if (sh == 0) qw[wi] = 0u;
         qw[wi] |= (uint32_t)q << sh;
@@ -177,8 +242,7 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, i
       }
       if (r.valid) {
         st_v8f(r.V + c + e, vn);
-        st_v8f(r.phi + c + e, hi);
-        st_v8f(r.plo + c + e, lo);
+        put_operand8<MIX>(r.phi, r.plo, c + e, pv);  // P, A side
         if (r.wdump) {
           float wd[8];
 #pragma unroll
@@ -278,17 +342,20 @@ struct EpiScaleStore {
   }
 };
 
-// GEMM 1 epilogue: T = (C0' + rho acc) / (lambda + rho), split to tf32 planes.
-template <int BN>
+// GEMM 1 epilogue: T = (C0' + rho acc) / (lambda + rho), stored in the
+// operand encoding (A side).
+struct TUpdateParams {
+  const float* c0;
+  const float* lam;
+  float* t_hi;
+  void* t_lo;      // plane 1 (encoding per the epilogue's MIX)
+  float rho;
+  int ld;
+};
+
+template <int BN, bool MIX>
 struct EpiTUpdate {
-  struct Params {
-    const float* c0;
-    const float* lam;
-    float* t_hi;
-    float* t_lo;
-    float rho;
-    int ld;
-  };
+  using Params = TUpdateParams;
   __device__ static void apply(const Params& p, const GemmGeom& g, uint32_t taddr, int tm, int tn,
                                int, int q, int lane) {
     const int row = tm * 128 + q * 32 + lane;
@@ -301,7 +368,7 @@ struct EpiTUpdate {
         const long long off = (long long)row * p.ld + col;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          float cc[8], hi[8], lo[8];
+          float cc[8], tv[8];
           ld_v8f(p.c0 + off + 8 * k, cc);
           const float4 l0 = __ldg(reinterpret_cast<const float4*>(p.lam + col + 8 * k));
           const float4 l1 = __ldg(reinterpret_cast<const float4*>(p.lam + col + 8 * k + 4));
@@ -310,10 +377,10 @@ struct EpiTUpdate {
           for (int j = 0; j < 8; ++j) {
             const float inv = __frcp_rn(__fadd_rn(ll[j], p.rho));
             const float t = __fmul_rn(__fadd_rn(cc[j], __fmul_rn(p.rho, v[8 * k + j])), inv);
-            split2(t, hi[j], lo[j]);
+            tv[j] = t;
           }
-          st_v8f(p.t_hi + off + 8 * k, hi);
-          st_v8f(p.t_lo + off + 8 * k, lo);
+          put_operand8<MIX>(p.t_hi + (long long)row * p.ld, lo_row<MIX>(p.t_lo, row, p.ld),
+                            col + 8 * k, tv);
         }
       }
     }
@@ -328,7 +395,7 @@ struct ProjParams {
   float* scale;
   float* zero;
   float* p_hi;
-  float* p_lo;
+  void* p_lo;     // plane 1 (encoding per the epilogue's MIX)
   const float* sig;
   const float* rsig;
   const float* hd;
@@ -339,7 +406,7 @@ struct ProjParams {
   int L;
 };
 
-template <int BN, int MODE>
+template <int BN, int MODE, bool MIX>
 struct EpiProject {
   using Params = ProjParams;
   __device__ static void apply(const Params& p, const GemmGeom& g, uint32_t taddr, int tm, int tn,
@@ -360,13 +427,15 @@ struct EpiProject {
       r.hd = p.hd + col0;
       r.codes = p.codes + off;
       r.phi = p.p_hi + off;
-      r.plo = p.p_lo + off;
+      r.plo = MIX ? (void*)(reinterpret_cast<uint16_t*>(p.p_lo) + (long long)(valid ? row : 0) * 2 * p.ld +
+                            2 * col0)
+                  : (void*)(reinterpret_cast<float*>(p.p_lo) + off);
       r.scale = p.scale + goff;
       r.zero = p.zero + goff;
       r.wdump = p.wdump ? p.wdump + off : nullptr;
       r.valid = valid;
       auto loadw = [&](int c, float (&w)[32]) { tmem_ld32(taddr + c0 + c, w); };
-      project_group<MODE>(loadw, r, p.group, p.L, r2, s2);
+      project_group<MODE, MIX>(loadw, r, p.group, p.L, r2, s2);
     }
     r2 = warp_sum(r2);
     s2 = warp_sum(s2);

@@ -75,9 +75,9 @@ def _oracle_run(full_setup, grid):
     return cache[grid]
 
 
-def _solver(A, p, X, W, grid):
+def _solver(A, p, X, W, grid, split="auto"):
     prm = A.Params(bits=p.bits, group=p.group, iters=p.iters, rho0=p.rho0, gamma=p.gamma,
-                   lambda_rel=p.lambda_rel, grid=grid)
+                   lambda_rel=p.lambda_rel, grid=grid, split=split)
     G = A.build_hessian(X)
     s = A.Solver(D, D, prm)
     s.prepare(G, W)
@@ -85,15 +85,17 @@ def _solver(A, p, X, W, grid):
     return s
 
 
-@pytest.mark.parametrize("grid", ["lsq", "minmax"])
-def test_full_size_teacher_forced(A, full_setup, grid):
+@pytest.mark.parametrize("grid,split", [("lsq", "auto"), ("minmax", "auto"), ("lsq", "3xtf32")])
+def test_full_size_teacher_forced(A, full_setup, grid, split):
     """RTN start bit-exact on the sampled rows; then, at sampled iterations,
     the oracle's state of those rows is loaded into the GPU's state and one
     GPU iteration runs: W~ within 1e-4 relative, codes equal on >= 99.9%,
-    mismatches one level apart where the grid agrees."""
+    mismatches one level apart where the grid agrees.  At this size the
+    automatic split precision is the mixed one; 3xTF32 is forced once."""
     p, X, W, H, Wm, _, _ = full_setup
     res, trace = _oracle_run(full_setup, grid)
-    s = _solver(A, p, X, W, grid)
+    s = _solver(A, p, X, W, grid, split)
+    assert s.split == ("3xtf32" if split == "3xtf32" else "mixed")
     s.init()
     torch.cuda.synchronize()
     rows = torch.from_numpy(ROWS).cuda()
@@ -105,10 +107,10 @@ def test_full_size_teacher_forced(A, full_setup, grid):
     for t in STEPS:
         e = trace[t]
         if t > 0:
-            hi, lo = P.split_tf32((e["Dt"] - e["Vt"]).T.astype(np.float32))
+            hi, lo = P.encode_operand((e["Dt"] - e["Vt"]).T.astype(np.float32), s.split, "A")
             s.buffer("V")[rows] = cu(e["Vt"].T.astype(np.float32))
             s.buffer("P_hi")[rows] = cu(hi)
-            s.buffer("P_lo")[rows] = cu(lo)
+            s.buffer("P_lo")[rows] = cu(lo.view(np.int16) if s.split == "mixed" else lo)
             s.codes[rows] = cu(e["codes"].T)
             s.scale[rows] = cu(e["scale"].T.astype(np.float32))
             s.zero[rows] = cu(e["zero"].T.astype(np.float32))
@@ -123,7 +125,7 @@ def test_full_size_teacher_forced(A, full_setup, grid):
         assert np.mean(c != co) <= 1e-3, (t, np.mean(c != co))
         same_grid = np.repeat(s.zero[rows].cpu().numpy() == e["zero_out"].T, p.group, axis=1)
         assert np.all(np.abs(c - co)[same_grid] <= 1), t
-        print(f"full-size {grid} step {t}: W~ rel err {err:.2e}, code mismatches {np.mean(c != co):.2e}")
+        print(f"full-size {grid}/{s.split} step {t}: W~ rel err {err:.2e}, code mismatches {np.mean(c != co):.2e}")
     s.dump_wtilde(None)
 
 

@@ -81,27 +81,29 @@ def _proj_inputs(m, d, g, bits, seed):
     return dict(W=W, V=V, sig=sig, rsig=rsig, hd=hd, s0=s0, z0=z0, c0=c0)
 
 
+@pytest.mark.parametrize("split", ["mixed", "3xtf32"])
 @pytest.mark.parametrize("grid", ["minmax", "lsq", "frozen"])
 @pytest.mark.parametrize("bits,g,m,d", [(3, 128, 200, 384), (2, 64, 33, 128), (4, 32, 130, 96),
                                         (3, 64, 32, 64)])
-def test_projection_kernel_bitexact(A, grid, bits, g, m, d):
+def test_projection_kernel_bitexact(A, grid, bits, g, m, d, split):
     x = _proj_inputs(m, d, g, bits, seed=bits * 100 + g + m)
     ref = P.epilogue_step(x["W"], x["V"], x["sig"], x["rsig"], x["hd"], x["s0"], x["z0"], x["c0"],
-                          bits, g, grid)
+                          bits, g, grid, split)
     cu = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
     V = cu(x["V"])
     codes, scale, zero = cu(x["c0"]), cu(x["s0"]), cu(x["z0"])
     phi = torch.empty((m, d), dtype=torch.float32, device="cuda")
-    plo = torch.empty_like(phi)
+    plo = (torch.empty((m, 2 * d), dtype=torch.int16, device="cuda") if split == "mixed"
+           else torch.empty((m, d), dtype=torch.float32, device="cuda"))
     resid = A.project(cu(x["W"]), V, cu(x["sig"]), cu(x["rsig"]), cu(x["hd"]), bits, g, grid,
-                      codes, scale, zero, phi, plo)
+                      codes, scale, zero, phi, plo, split=split)
     torch.cuda.synchronize()
     np.testing.assert_array_equal(codes.cpu().numpy(), ref["codes"])
     np.testing.assert_array_equal(scale.cpu().numpy().view(np.uint32), ref["scale"].view(np.uint32))
     np.testing.assert_array_equal(zero.cpu().numpy().view(np.uint32), ref["zero"].view(np.uint32))
     np.testing.assert_array_equal(V.cpu().numpy().view(np.uint32), ref["V"].view(np.uint32))
     np.testing.assert_array_equal(phi.cpu().numpy().view(np.uint32), ref["P_hi"].view(np.uint32))
-    np.testing.assert_array_equal(plo.cpu().numpy().view(np.uint32), ref["P_lo"].view(np.uint32))
+    np.testing.assert_array_equal(plo.cpu().numpy().view(np.uint16), ref["P_lo"].view(np.uint16))
     r = resid.cpu().numpy()
     assert r[0] == pytest.approx(ref["r2"], rel=1e-4)
     assert r[1] == pytest.approx(ref["s2"], rel=1e-4, abs=1e-12)

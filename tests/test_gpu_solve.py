@@ -51,9 +51,9 @@ def _oracle(p, X, W, grid, iters=None):
     return H, Wm, res
 
 
-def _solver(A, p, X, W, grid, iters=None):
+def _solver(A, p, X, W, grid, iters=None, split="auto"):
     prm = A.Params(bits=p.bits, group=p.group, iters=p.iters if iters is None else iters,
-                   rho0=p.rho0, gamma=p.gamma, lambda_rel=p.lambda_rel, grid=grid)
+                   rho0=p.rho0, gamma=p.gamma, lambda_rel=p.lambda_rel, grid=grid, split=split)
     G = A.build_hessian(X)
     s = A.Solver(X.shape[1], W.shape[0], prm)
     s.prepare(G, W)
@@ -117,9 +117,9 @@ def test_first_iteration_w_update(A, name, grid):
     V = V0.clone()
     codes, scale, zero = c0.clone(), s0.clone(), z0.clone()
     phi = torch.empty_like(s.buffer("P_hi"))
-    plo = torch.empty_like(phi)
+    plo = torch.empty_like(s.buffer("P_lo"))
     A.project(wt, V, s.buffer("sigma"), s.buffer("rsig"), s.buffer("hdiag"), p.bits, p.group,
-              grid, codes, scale, zero, phi, plo)
+              grid, codes, scale, zero, phi, plo, split=s.split)
     torch.cuda.synchronize()
     assert torch.equal(codes, s.codes) and torch.equal(scale, s.scale) and torch.equal(zero, s.zero)
     assert torch.equal(V, s.buffer("V"))
@@ -133,31 +133,37 @@ def _load_state(s, e):
     """Oracle state entering iteration t -> the GPU's state buffers."""
     Vt = e["Vt"].T.astype(np.float32)
     Pm = (e["Dt"] - e["Vt"]).T.astype(np.float32)
-    hi, lo = P.split_tf32(Pm)
+    hi, lo = P.encode_operand(Pm, s.split, "A")
     cu = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
     s.buffer("V").copy_(cu(Vt))
     s.buffer("P_hi").copy_(cu(hi))
-    s.buffer("P_lo").copy_(cu(lo))
+    s.buffer("P_lo").copy_(cu(lo.view(np.int16) if s.split == "mixed" else lo))
     s.codes.copy_(cu(e["codes"].T))
     s.scale.copy_(cu(e["scale"].T.astype(np.float32)))
     s.zero.copy_(cu(e["zero"].T.astype(np.float32)))
 
 
-@pytest.mark.parametrize("name", ["tiny", "ragged", "down_small"])
-@pytest.mark.parametrize("grid", ["minmax", "lsq", "frozen"])
-def test_teacher_forced_iterations(A, name, grid):
+TEACHER_CASES = [(n, g, "auto") for n in ("tiny", "ragged", "down_small")
+                 for g in ("minmax", "lsq", "frozen")] + \
+                [(n, g, "mixed") for n in ("tiny", "ragged") for g in ("minmax", "lsq")]
+
+
+@pytest.mark.parametrize("name,grid,split", TEACHER_CASES)
+def test_teacher_forced_iterations(A, name, grid, split):
     """Step parity along the oracle's trajectory: at sampled iterations t the
     oracle's state (D~_t, V~_t, grid) is loaded into the GPU, one GPU iteration
     runs, and W~ must be within 1e-4 relative and the codes must agree on
     >= 99.9% of entries, mismatches being adjacent levels (decisions at a
-    rounding tie)."""
+    rounding tie).  These small layers run 3xTF32 by default; the mixed split
+    is forced on two of them as well."""
     p, X, W = _layer(name)
     trace = []
     Xn = X.float().cpu().numpy()
     H = O.hessian(Xn, p.lambda_rel)
     Wm = W.float().cpu().numpy().T.astype(np.float64)
     O.admm_q(H, Wm, p.bits, p.group, p.iters, rho0=p.rho0, gamma=p.gamma, grid=grid, trace=trace)
-    s = _solver(A, p, X, W, grid)
+    s = _solver(A, p, X, W, grid, split=split)
+    assert s.split == ("mixed" if split == "mixed" else "3xtf32")
     s.init()
     wt = torch.empty((W.shape[0], X.shape[1]), dtype=torch.float32, device="cuda")
     s.dump_wtilde(wt)

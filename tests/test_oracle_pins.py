@@ -313,6 +313,45 @@ def test_tf32_split_reconstructs_float32():
     np.testing.assert_array_equal(P.tf32_round(t), np.array([1.0, 1 + 2.0 ** -9], np.float32))
 
 
+def test_mixed_split_encoding():
+    """Operand encoding of the eigenbasis GEMMs: hi = tf32(x) is the plane-0
+    value, lo = x - hi is exact in float32, and the correction rows hold
+    bf16(hi) / bf16(lo) in blocks of 32 columns, swapped on the B side, so
+    that one tf32 product plus one bf16 product over a row pair gives
+    hi.hi + hi.lo + lo.hi to ~2^-19 relative."""
+    rng = np.random.default_rng(12)
+    x = (rng.standard_normal((3, 64)) * np.exp(rng.standard_normal((3, 64)))).astype(np.float32)
+    hi, ca = P.split_mix(x, "A")
+    _, cb = P.split_mix(x, "B")
+    np.testing.assert_array_equal(hi, P.tf32_round(x))
+    lo = (x.astype(np.float64) - hi).astype(np.float32)
+    assert np.array_equal(hi.astype(np.float64) + lo, x.astype(np.float64))   # exact split
+    assert ca.shape == (3, 128) and ca.dtype == np.uint16
+    for b in range(2):                       # blocks of 32 columns
+        blk = slice(32 * b, 32 * b + 32)
+        np.testing.assert_array_equal(ca[:, 64 * b:64 * b + 32], P.bf16_bits(hi[:, blk]))
+        np.testing.assert_array_equal(ca[:, 64 * b + 32:64 * b + 64], P.bf16_bits(lo[:, blk]))
+        np.testing.assert_array_equal(cb[:, 64 * b:64 * b + 32], ca[:, 64 * b + 32:64 * b + 64])
+        np.testing.assert_array_equal(cb[:, 64 * b + 32:64 * b + 64], ca[:, 64 * b:64 * b + 32])
+    # hand example: x = 1 + 2^-11 + 2^-20 -> hi = 1 + 2^-10 (round up past the
+    # tie), lo = -2^-11 + 2^-20, bf16(lo) = -2^-11 (2^-20 is below bf16's 8 bits)
+    t = np.zeros((1, 32), np.float32)
+    t[0, 0] = np.float32(1 + 2.0 ** -11 + 2.0 ** -20)
+    th, tc = P.split_mix(t, "A")
+    assert th[0, 0] == np.float32(1 + 2.0 ** -10)
+    assert P.bf16_value(tc[0, 32]) == np.float32(-(2.0 ** -11))
+    # the two products reproduce x_a . x_b to the bf16 level of the corrections
+    a = (rng.standard_normal((4, 256))).astype(np.float32)
+    bm = (rng.standard_normal((5, 256))).astype(np.float32)
+    ha, cA = P.split_mix(a, "A")
+    hb, cB = P.split_mix(bm, "B")
+    prod = ha.astype(np.float64) @ hb.T.astype(np.float64) + \
+        P.bf16_value(cA).astype(np.float64) @ P.bf16_value(cB).T.astype(np.float64)
+    exact = a.astype(np.float64) @ bm.T.astype(np.float64)
+    scale = np.abs(a).astype(np.float64) @ np.abs(bm).T.astype(np.float64)
+    assert np.max(np.abs(prod - exact) / scale) < 2.0 ** -18
+
+
 def test_bf16_split_reconstructs_float32():
     rng = np.random.default_rng(9)
     x = (rng.standard_normal(10000) * np.exp(rng.standard_normal(10000) * 3)).astype(np.float32)
