@@ -32,9 +32,13 @@ using GramCfg = GemmCfg<KIND_BF16, 256, 1, true, true, 4, 4>;
 //   mixed split (tf32 hi.hi + one bf16 product for the corrections, 64 MMAs
 //   per chunk) for large layers, 3xTF32 (96 MMAs per chunk) where the
 //   reduction is short enough that the split's own rounding would dominate.
-using EigCfg = GemmCfg<KIND_MIX, 128, 2, false, false, 3, 8>;
-using EigCfg3 = GemmCfg<KIND_TF32, 128, 2, false, false, 3, 8>;
-static_assert(EigCfg::BN == EigCfg3::BN && EigCfg::BK == EigCfg3::BK, "same tile geometry");
+// Both run on CTA pairs (2-SM MMAs of 256 x 128; each SM stages half of B,
+// which cuts the shared-memory traffic per MMA by a quarter) with 4 stages.
+using EigCfg = GemmCfg<KIND_MIX, 256, 2, false, false, 3, 16, true>;
+using EigCfg3 = GemmCfg<KIND_TF32, 256, 2, false, false, 3, 16, true>;
+static_assert(EigCfg::BN == EigCfg3::BN && EigCfg::BK == EigCfg3::BK &&
+                  EigCfg::UNIT_M == EigCfg3::UNIT_M && EigCfg::B_ROWS == EigCfg3::B_ROWS,
+              "same tile geometry");
 // d_in from which the automatic split mode picks the mixed split
 constexpr int kMixedFromDin = 2048;
 
@@ -435,19 +439,27 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, u
 
 int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
 
+// 128-row x BN tiles of an eigenbasis GEMM output [m][d] (per-tile partials)
+int eig_tiles(int m, int d) {
+  return cdiv(m, EigCfg::UNIT_M) * (EigCfg::UNIT_M / kBM) * cdiv(d, 128);
+}
+
 GemmGeom make_geom(int M, int N, long long K, int BN, int BK, int splits, bool triangle,
-                   int* status) {
+                   int* status, int unit_m = kBM) {
   GemmGeom g;
   g.M = M;
   g.N = N;
   g.K = (int)K;
-  g.tiles_m = cdiv(M, kBM);
+  // 128-row tiles, counted up to whole units (a CTA pair's second tile may
+  // lie past M: its epilogue masks every row, its partial sums are zeros)
+  g.tiles_mu = cdiv(M, unit_m);
+  g.tiles_m = g.tiles_mu * (unit_m / kBM);
   g.tiles_n = cdiv(N, BN);
   g.kblocks = cdiv(K, BK);
   g.splits = splits;
   g.triangle = triangle ? 1 : 0;
   if (!triangle) {
-    g.tiles = g.tiles_m * g.tiles_n;
+    g.tiles = g.tiles_mu * g.tiles_n;
   } else {
     int t = 0;
     for (int tn = 0; tn < g.tiles_n; ++tn) {
@@ -457,7 +469,7 @@ GemmGeom make_geom(int M, int N, long long K, int BN, int BK, int splits, bool t
     g.tiles = t;
   }
   g.units = g.tiles * splits;
-  g.band = g.tiles_m < 12 ? g.tiles_m : 12;  // 12 x 12 tiles in flight ~ 100 MB of operands
+  g.band = g.tiles_mu < 12 ? g.tiles_mu : 12;  // 12 x 12 tiles in flight ~ 100 MB of operands
   g.status = status;
   return g;
 }
@@ -469,10 +481,30 @@ cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
   auto kern = k_gemm<Cfg, Epi>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
   if (e != cudaSuccess) return e;
-  int grid = g.units < num_sms() ? g.units : num_sms();
-  if (grid <= 0) return cudaSuccess;
+  if (g.units <= 0) return cudaSuccess;
+  if (!Cfg::PAIR) {
+    const int grid = g.units < num_sms() ? g.units : num_sms();
+    count_launch();
+    kern<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(a0, a1, b0, b1, g, ep);
+    return cudaGetLastError();
+  }
+  // CTA pairs: clusters of two, one work unit per cluster at a time
+  const int pairs = num_sms() / 2;
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(2 * (g.units < pairs ? g.units : pairs));
+  lc.blockDim = dim3(Cfg::THREADS);
+  lc.dynamicSmemBytes = Cfg::SMEM;
+  lc.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
   count_launch();
-  kern<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(a0, a1, b0, b1, g, ep);
+  e = cudaLaunchKernelEx(&lc, kern, a0, a1, b0, b1, g, ep);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -579,7 +611,7 @@ Layout make_layout(int d, int m, int iters, int lwork) {
     return at;
   };
   const size_t dd = (size_t)d * d, md = (size_t)m * d;
-  const int tiles = cdiv(m, kBM) * cdiv(d, EigCfg::BN);
+  const int tiles = eig_tiles(m, d);
   L.status = take(16);
   L.lam64 = take(8);
   L.sig64 = take(8 * (size_t)d);
@@ -810,15 +842,15 @@ int admmq_create(admmq_ctx** out, int d, int m, const admmq_params* p, void* ws,
   c->V = (float*)(b + L.V);
   c->resid_part = (float*)(b + L.resid_part);
   c->obj_part = (float*)(b + L.obj_part);
-  c->tiles_eig = cdiv(m, kBM) * cdiv(d, EigCfg::BN);
+  c->tiles_eig = eig_tiles(m, d);
   bool ok = true;
   ok &= make_map(&c->mWt[0], c->Wt_hi, d, m, kBM, true) && make_map(&c->mWt[1], c->Wt_lo, c->mix ? 2 * (uint64_t)d : (uint64_t)d, m, kBM, !c->mix);
   ok &= make_map(&c->mP[0], c->P_hi, d, m, kBM, true) && make_map(&c->mP[1], c->P_lo, c->mix ? 2 * (uint64_t)d : (uint64_t)d, m, kBM, !c->mix);
   ok &= make_map(&c->mT[0], c->T_hi, d, m, kBM, true) && make_map(&c->mT[1], c->T_lo, c->mix ? 2 * (uint64_t)d : (uint64_t)d, m, kBM, !c->mix);
-  ok &= make_map(&c->mE[0], c->E_hi, d, d, EigCfg::BN, true) &&
-        make_map(&c->mE[1], c->E_lo, c->mix ? 2 * (uint64_t)d : (uint64_t)d, d, EigCfg::BN, !c->mix);
-  ok &= make_map(&c->mQ[0], c->Q_hi, d, d, EigCfg::BN, true) &&
-        make_map(&c->mQ[1], c->Q_lo, c->mix ? 2 * (uint64_t)d : (uint64_t)d, d, EigCfg::BN, !c->mix);
+  ok &= make_map(&c->mE[0], c->E_hi, d, d, EigCfg::B_ROWS, true) &&
+        make_map(&c->mE[1], c->E_lo, c->mix ? 2 * (uint64_t)d : (uint64_t)d, d, EigCfg::B_ROWS, !c->mix);
+  ok &= make_map(&c->mQ[0], c->Q_hi, d, d, EigCfg::B_ROWS, true) &&
+        make_map(&c->mQ[1], c->Q_lo, c->mix ? 2 * (uint64_t)d : (uint64_t)d, d, EigCfg::B_ROWS, !c->mix);
   if (!ok || cusolverDnCreate(&c->solver) != CUSOLVER_STATUS_SUCCESS) {
     delete c;
     return ADMMQ_ERR_CUDA;
@@ -906,7 +938,7 @@ int admmq_init(admmq_ctx* c, uint8_t* codes, float* scale, float* zero, void* st
   cudaStream_t st = (cudaStream_t)stream;
   const int d = c->d, m = c->m;
   // C0' = Lambda Q^T W^~   (row j, column k)
-  GemmGeom g = make_geom(m, d, d, EigCfg::BN, EigCfg::BK, 1, false, c->status);
+  GemmGeom g = make_geom(m, d, d, EigCfg::BN, EigCfg::BK, 1, false, c->status, EigCfg::UNIT_M);
   EpiScaleStore<EigCfg::BN>::Params ep{c->C0, c->lam32, d};
   CK((launch_eig<EpiScaleStore<EigCfg::BN>, EpiScaleStore<EigCfg::BN>>(c->mix, c->mWt, c->mE, g, ep,
                                                                          st)));
@@ -931,7 +963,7 @@ int admmq_iterate(admmq_ctx* c, int t0, int count, uint8_t* codes, float* scale,
   if (t0 < 0 || count < 0 || t0 + count > c->p.iters) return ADMMQ_ERR_INVALID_ARG;
   cudaStream_t st = (cudaStream_t)stream;
   const int d = c->d, m = c->m;
-  GemmGeom g = make_geom(m, d, d, EigCfg::BN, EigCfg::BK, 1, false, c->status);
+  GemmGeom g = make_geom(m, d, d, EigCfg::BN, EigCfg::BK, 1, false, c->status, EigCfg::UNIT_M);
   for (int t = t0; t < t0 + count; ++t) {
     const float rho = (float)((double)c->p.rho0 * pow((double)c->p.gamma, (double)t));
     cudaEvent_t e0 = nullptr, e1 = nullptr, e2 = nullptr;
@@ -1008,7 +1040,7 @@ int admmq_finish(admmq_ctx* c, const uint8_t* codes, const float* scale, const f
           (const __nv_bfloat16*)c->W_hat, codes, scale, zero, c->rsig, d, c->p.group, md, c->T_hi,
           c->T_lo, c->mix);
     CK(cudaGetLastError());
-    GemmGeom g = make_geom(m, d, d, EigCfg::BN, EigCfg::BK, 1, false, c->status);
+    GemmGeom g = make_geom(m, d, d, EigCfg::BN, EigCfg::BK, 1, false, c->status, EigCfg::UNIT_M);
     EpiObjective<EigCfg::BN>::Params ep{c->lam32, c->obj_part};
     CK((launch_eig<EpiObjective<EigCfg::BN>, EpiObjective<EigCfg::BN>>(c->mix, c->mT, c->mE, g, ep,
                                                                          st)));

@@ -43,7 +43,8 @@ namespace admmq {
 
 struct GemmGeom {
   int M, N, K;        // output rows / columns, reduction length
-  int tiles_m, tiles_n;
+  int tiles_m, tiles_n;  // 128-row and BN-column output tiles
+  int tiles_mu;          // unit rows: 128-row tiles, or 256-row tile pairs (CTA-pair configs)
   int splits;         // k-splits per tile (units = tiles * splits)
   int kblocks;        // ceil(K / BK)
   int triangle;       // 1: only tiles that meet the upper triangle (i <= j)
@@ -58,7 +59,8 @@ struct GemmGeom {
 // plane and one bf16 correction plane per operand (see GemmCfg).
 enum { KIND_BF16 = 1, KIND_TF32 = 2, KIND_MIX = 3 };
 
-template <int KIND_, int BN_, int NPL_, bool A_MN_, bool B_MN_, int STAGES_, int KC_>
+template <int KIND_, int BN_, int NPL_, bool A_MN_, bool B_MN_, int STAGES_, int KC_,
+          bool PAIR_ = false>
 struct GemmCfg {
   static constexpr int KIND = KIND_;
   static constexpr int ELEM = KIND == KIND_BF16 ? 2 : 4;  // bytes per (plane-0) operand element
@@ -67,15 +69,25 @@ struct GemmCfg {
   static constexpr int KC = KC_;                           // k-blocks per promoted chunk
   static constexpr bool A_MN = A_MN_, B_MN = B_MN_;
   static constexpr bool SPLITCOL = BN == 256;
+  // PAIR: a cluster of two CTAs runs 2-SM MMAs of 256 x BN; each CTA stages
+  // its 128 A rows and half of the BN B rows.
+  static constexpr bool PAIR = PAIR_;
+  static constexpr int UNIT_M = PAIR ? 2 * BM : BM;   // output rows per work unit
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;   // B rows staged per CTA
   static constexpr int A_PLANE = BM * 128;  // bytes per operand plane per stage
-  static constexpr int B_PLANE = BN * 128;
+  static constexpr int B_PLANE = B_ROWS * 128;
   static constexpr int STAGE = NPL * (A_PLANE + B_PLANE);
   static constexpr int RING = SPLITCOL ? 2 : 3;  // chunk slots in tensor memory
   static constexpr int TMEM_COLS = 512;          // RING x BN (+ one final 128-column slot)
   static constexpr int THREADS = 320;
+  static constexpr int CONS_WARP0 = 2;  // first consumer warp
   static constexpr int BAR_BYTES = 8 * (2 * STAGES + 4 * RING + 2) + 16;
+  // arrivals that release a ring slot: every consumer thread of the CTA, or
+  // one per consumer warp of both CTAs of a pair
+  static constexpr int SLOT_ARRIVALS = PAIR ? (SPLITCOL ? 16 : 8) : (SPLITCOL ? 256 : 128);
   static constexpr int SMEM = STAGES * STAGE + 1024 + BAR_BYTES;
   static_assert(BN == 128 || BN == 256, "BN must be 128 or 256");
+  static_assert(!PAIR || (!A_MN && !B_MN), "CTA pairs: K-major operands");
   static_assert(KIND != KIND_MIX || (NPL == 2 && !A_MN && !B_MN), "mixed split: two K-major planes");
   // products per K step: 3xTF32 (hi.hi, hi.lo, lo.hi), mixed (tf32 hi.hi +
   // one bf16 product over the [hi|lo] x [lo|hi] correction row), or one
@@ -95,7 +107,7 @@ __device__ __forceinline__ void decode_unit(const GemmGeom& g, int u, int& tm, i
   int t = u - split * g.tiles;
   if (!g.triangle) {
     const int b = t / (g.band * g.tiles_n);
-    const int rows = min(g.band, g.tiles_m - b * g.band);
+    const int rows = min(g.band, g.tiles_mu - b * g.band);
     const int r = t - b * g.band * g.tiles_n;
     tn = r / rows;
     tm = b * g.band + (r - tn * rows);
@@ -103,7 +115,7 @@ __device__ __forceinline__ void decode_unit(const GemmGeom& g, int u, int& tm, i
     tn = 0;
     for (;;) {
       int cnt = ((tn + 1) * BN + BM - 1) / BM;
-      if (cnt > g.tiles_m) cnt = g.tiles_m;
+      if (cnt > g.tiles_mu) cnt = g.tiles_mu;
       if (t < cnt) break;
       t -= cnt;
       ++tn;
@@ -115,7 +127,7 @@ __device__ __forceinline__ void decode_unit(const GemmGeom& g, int u, int& tm, i
 }
 
 template <class Cfg, class Epi>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(Cfg::THREADS, 1)
     k_gemm(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ CUtensorMap tA1,
            const __grid_constant__ CUtensorMap tB0, const __grid_constant__ CUtensorMap tB1,
            const GemmGeom g, const typename Epi::Params ep) {
@@ -139,6 +151,11 @@ __global__ void __launch_bounds__(320, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // CTA pairs: rank in the cluster (0 = leader, issues the MMAs); work units
+  // are dealt per cluster.
+  const uint32_t rank = Cfg::PAIR ? cluster_rank() : 0u;
+  const int unit0 = Cfg::PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int unit_step = Cfg::PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -147,7 +164,7 @@ __global__ void __launch_bounds__(320, 1)
     }
     for (int a = 0; a < 2 * R; ++a) {
       mbar_init(smem_u32(&rfull[a]), 1);
-      mbar_init(smem_u32(&rempty[a]), Cfg::SPLITCOL ? 256 : 128);
+      mbar_init(smem_u32(&rempty[a]), Cfg::SLOT_ARRIVALS);
     }
     mbar_init(smem_u32(fin), 128);
     mbar_init(smem_u32(drain), 1);
@@ -162,9 +179,16 @@ __global__ void __launch_bounds__(320, 1)
       prefetch_tmap(&tB1);
     }
   }
-  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), Cfg::TMEM_COLS);
+  if (warp == 1) {
+    if (Cfg::PAIR)
+      tmem_alloc_pair(smem_u32(tmem_slot), Cfg::TMEM_COLS);
+    else
+      tmem_alloc(smem_u32(tmem_slot), Cfg::TMEM_COLS);
+  }
   __syncthreads();
+  if (Cfg::PAIR) cluster_sync();  // both CTAs' barriers exist before any remote use
   tc_fence_after();
+
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
@@ -174,9 +198,11 @@ __global__ void __launch_bounds__(320, 1)
       const CUtensorMap* mapB[2] = {&tB0, &tB1};
       int it = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < g.units && ok; u += gridDim.x) {
+      for (int u = unit0; u < g.units && ok; u += unit_step) {
         int tm, tn, split, kb0, kb1;
         decode_unit<BM, BN>(g, u, tm, tn, split, kb0, kb1);
+        const int a_row = tm * Cfg::UNIT_M + (int)rank * BM;        // this CTA's A rows
+        const int b_row = tn * BN + (int)rank * Cfg::B_ROWS;        // this CTA's B rows
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
@@ -184,8 +210,15 @@ __global__ void __launch_bounds__(320, 1)
             ok = false;
             break;
           }
-          const uint32_t fb = smem_u32(&full[s]);
-          mbar_arrive_expect_tx(fb, Cfg::STAGE);
+          // A pair's loads all count on the leader's barrier, which expects
+          // the bytes of both CTAs.
+          uint32_t fb = smem_u32(&full[s]);
+          if (Cfg::PAIR) {
+            if (rank == 0) mbar_arrive_expect_tx(fb, 2 * Cfg::STAGE);
+            fb = cluster_addr(fb, 0);
+          } else {
+            mbar_arrive_expect_tx(fb, Cfg::STAGE);
+          }
           const uint32_t st = smem_u32(smem + s * Cfg::STAGE);
           const int k0 = kb * Cfg::BK;
 #pragma unroll
@@ -193,18 +226,26 @@ __global__ void __launch_bounds__(320, 1)
             const uint32_t dA = st + p * Cfg::A_PLANE;
             if (!Cfg::A_MN) {
               // a mixed correction plane holds two bf16 per K-element
-              tma_load_2d(dA, mapA[p], (Cfg::KIND == KIND_MIX && p == 1) ? 2 * k0 : k0, tm * BM, fb);
+              const int xa = (Cfg::KIND == KIND_MIX && p == 1) ? 2 * k0 : k0;
+              if (Cfg::PAIR)
+                tma_load_2d_pair(dA, mapA[p], xa, a_row, fb);
+              else
+                tma_load_2d(dA, mapA[p], xa, a_row, fb);
             } else {
 #pragma unroll
               for (int b = 0; b < BM / (128 / Cfg::ELEM); ++b)
-                tma_load_2d(dA + b * Cfg::BK * 128, mapA[p], tm * BM + (128 / Cfg::ELEM) * b, k0, fb);
+                tma_load_2d(dA + b * Cfg::BK * 128, mapA[p], a_row + (128 / Cfg::ELEM) * b, k0, fb);
             }
           }
 #pragma unroll
           for (int p = 0; p < NPL; ++p) {
             const uint32_t dB = st + NPL * Cfg::A_PLANE + p * Cfg::B_PLANE;
             if (!Cfg::B_MN) {
-              tma_load_2d(dB, mapB[p], (Cfg::KIND == KIND_MIX && p == 1) ? 2 * k0 : k0, tn * BN, fb);
+              const int xb = (Cfg::KIND == KIND_MIX && p == 1) ? 2 * k0 : k0;
+              if (Cfg::PAIR)
+                tma_load_2d_pair(dB, mapB[p], xb, b_row, fb);
+              else
+                tma_load_2d(dB, mapB[p], xb, b_row, fb);
             } else {
 #pragma unroll
               for (int b = 0; b < BN / (128 / Cfg::ELEM); ++b)
@@ -214,17 +255,36 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       if (!ok) {
-        // Let the copies already in flight land before the CTA retires.
-        for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
-          mbar_wait_drain(smem_u32(&full[j % STAGES]), (uint32_t)(j / STAGES) & 1u);
+        // Let the copies already in flight land before the CTA retires.  A
+        // pair member's copies count on the leader's barriers: it waits a
+        // fixed ~1 ms instead.
+        if (!Cfg::PAIR || rank == 0) {
+          for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
+            mbar_wait_drain(smem_u32(&full[j % STAGES]), (uint32_t)(j / STAGES) & 1u);
+        } else {
+          const long long t0 = clock64();
+          while (clock64() - t0 < 2000000LL) {
+          }
+        }
       }
     }
   } else if (warp == 1) {
     // --------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // (a pair's MMAs, 256 rows of the unit, are issued by its leader alone)
+    if (lane == 0 && (!Cfg::PAIR || rank == 0)) {
       constexpr uint32_t IDESC = idesc_f32acc(Cfg::KIND == KIND_MIX ? (uint32_t)KIND_TF32 : Cfg::KIND,
-                                              BM, BN, Cfg::A_MN, Cfg::B_MN);
-      constexpr uint32_t IDESC16 = idesc_f32acc(KIND_BF16, BM, BN, Cfg::A_MN, Cfg::B_MN);
+                                              Cfg::UNIT_M, BN, Cfg::A_MN, Cfg::B_MN);
+      constexpr uint32_t IDESC16 = idesc_f32acc(KIND_BF16, Cfg::UNIT_M, BN, Cfg::A_MN, Cfg::B_MN);
+      // a completed group of MMAs is announced on the barrier at the same
+      // offset in each CTA of the pair (or in this CTA)
+      auto commit_all = [&](uint64_t* bar) {
+        if (Cfg::PAIR) {
+          mma_commit_pair(cluster_addr(smem_u32(bar), 0));
+          mma_commit_pair(cluster_addr(smem_u32(bar), 1));
+        } else {
+          mma_commit(smem_u32(bar));
+        }
+      };
       // MN-major: blocks of 128 bytes along MN, BK K-rows each, LBO apart
       constexpr uint32_t LBO_A = Cfg::A_MN ? Cfg::BK * 128 : 16;
       constexpr uint32_t LBO_B = Cfg::B_MN ? Cfg::BK * 128 : 16;
@@ -241,7 +301,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
       for (int i = 0; i < R; ++i) prev[i] = -1;
       bool ok = true;
-      for (int u = blockIdx.x; u < g.units && ok; u += gridDim.x, ++lu) {
+      for (int u = unit0; u < g.units && ok; u += unit_step, ++lu) {
         int tm, tn, split, kb0, kb1;
         decode_unit<BM, BN>(g, u, tm, tn, split, kb0, kb1);
         const int owner = Cfg::SPLITCOL ? 0 : (lu & 1);
@@ -281,28 +341,40 @@ __global__ void __launch_bounds__(320, 1)
                 const uint64_t ad = a0 + (uint64_t)(pa * kAPlane + kk * kKStepA);
                 const uint64_t bd = b0 + (uint64_t)(pb * kBPlane + kk * kKStepB);
                 const uint32_t accum = (kk > 0 || pr > 0) ? 1u : acc0;
-                if (Cfg::KIND == KIND_BF16 || (Cfg::KIND == KIND_MIX && pr == 1))
-                  mma_bf16(dt, ad, bd, Cfg::KIND == KIND_MIX ? IDESC16 : IDESC, accum);
-                else
-                  mma_tf32(dt, ad, bd, IDESC, accum);
+                const bool b16 = Cfg::KIND == KIND_BF16 || (Cfg::KIND == KIND_MIX && pr == 1);
+                const uint32_t id = Cfg::KIND == KIND_MIX && pr == 1 ? IDESC16 : IDESC;
+                if (Cfg::PAIR) {
+                  if (b16)
+                    mma_bf16_pair(dt, ad, bd, id, accum);
+                  else
+                    mma_tf32_pair(dt, ad, bd, id, accum);
+                } else {
+                  if (b16)
+                    mma_bf16(dt, ad, bd, id, accum);
+                  else
+                    mma_tf32(dt, ad, bd, id, accum);
+                }
               }
             }
-            mma_commit(smem_u32(&empty[s]));
+            commit_all(&empty[s]);
           }
           if (!ok) break;
           const int b = R * owner + (int)slot;
-          mma_commit(smem_u32(&rfull[b]));
+          commit_all(&rfull[b]);
           ++use[b];
           prev[slot] = owner;
         }
       }
       // Every MMA issued above is complete once this arrives.
-      mma_commit(smem_u32(drain));
+      if (Cfg::PAIR)
+        mma_commit_pair(cluster_addr(smem_u32(drain), 0));
+      else
+        mma_commit(smem_u32(drain));
       mbar_wait_drain(smem_u32(drain), 0);
     }
-  } else {
+  } else if (warp >= Cfg::CONS_WARP0) {
     // ---------------------------------------------------------- consumers
-    const int wg = (warp - 2) >> 2;  // consumer warpgroup 0 or 1
+    const int wg = (warp - Cfg::CONS_WARP0) >> 2;  // consumer warpgroup 0 or 1
     const int qtr = warp & 3;        // tensor-memory lane quarter this warp may access
     const uint32_t lane_off = (uint32_t)(qtr * 32) << 16;
     const uint32_t col_off = Cfg::SPLITCOL ? (uint32_t)(wg * 128) : 0u;
@@ -311,13 +383,27 @@ __global__ void __launch_bounds__(320, 1)
     uint32_t my_use[R] = {};                // own chunks consumed per slot
     int lu = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < g.units && ok; u += gridDim.x, ++lu) {
+    // a pair member drains its slots for the leader's MMA issuer
+    const uint32_t rempty_leader = Cfg::PAIR ? cluster_addr(smem_u32(rempty), 0) : 0u;
+    for (int u = unit0; u < g.units && ok; u += unit_step, ++lu) {
       int tm, tn, split, kb0, kb1;
       decode_unit<BM, BN>(g, u, tm, tn, split, kb0, kb1);
+      const int tile_m = Cfg::PAIR ? 2 * tm + (int)rank : tm;  // this CTA's 128-row tile
       const bool mine = Cfg::SPLITCOL || ((lu & 1) == wg);
       float acc[128];
 #pragma unroll
       for (int i = 0; i < 128; ++i) acc[i] = 0.f;
+      // releases ring slot b for the MMA issuer (of this CTA or of the pair)
+      auto release = [&](int b) {
+        if (Cfg::PAIR) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(rempty_leader + 8u * (uint32_t)b);
+        } else {
+          mbar_arrive(smem_u32(&rempty[b]));
+        }
+      };
+      int kept_b = 0;
+      uint32_t kept_slot = 0;
       for (int c0 = kb0; c0 < kb1; c0 += KC, ++q) {
         if (!mine) continue;
         const uint32_t slot = q % R;
@@ -337,12 +423,33 @@ __global__ void __launch_bounds__(320, 1)
           for (int k = 0; k < 16; ++k) acc[16 * j + k] += v[k];
         }
         tc_fence_before();
-        mbar_arrive(smem_u32(&rempty[b]));
+        // An epilogue that reads the tile from tensor memory keeps the last
+        // chunk's slot: the summed accumulator goes back into it below.
+        if (Cfg::SPLITCOL && Epi::FROM_TMEM && c0 + KC >= kb1) {
+          kept_b = b;
+          kept_slot = slot;
+        } else {
+          release(b);
+        }
         ++my_use[slot];
       }
       if (!ok || !mine) continue;
       if constexpr (Cfg::SPLITCOL) {
-        Epi::apply_regs(ep, g, acc, tm, tn, split, qtr * 32 + lane, tn * BN + wg * 128);
+        if constexpr (Epi::FROM_TMEM) {
+          const uint32_t ta = tmem_base + lane_off + kept_slot * BN + col_off;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            float v[32];
+#pragma unroll
+            for (int k = 0; k < 32; ++k) v[k] = acc[32 * j + k];
+            tmem_st32(ta + 32 * j, v);
+          }
+          Epi::apply_tmem(ep, g, ta, tile_m, qtr * 32 + lane, tn * BN + wg * 128);
+          tc_fence_before();
+          release(kept_b);
+        } else {
+          Epi::apply_regs(ep, g, acc, tile_m, tn, split, qtr * 32 + lane, tn * BN + wg * 128);
+        }
       } else {
         // The final slot is free once the previous tile's owner (the other
         // warpgroup) has finished its epilogue: phase lu - 1 of `fin`.
@@ -362,16 +469,20 @@ __global__ void __launch_bounds__(320, 1)
           for (int k = 0; k < 32; ++k) v[k] = acc[32 * j + k];
           tmem_st32(fslot + 32 * j, v);
         }
-        Epi::apply(ep, g, fslot, tm, tn, split, qtr, lane);
+        Epi::apply(ep, g, fslot, tile_m, tn, split, qtr, lane);
         tc_fence_before();
         mbar_arrive(smem_u32(fin));
       }
     }
   }
   __syncthreads();
+  if (Cfg::PAIR) cluster_sync();  // the peer's last remote arrivals have landed
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+    if (Cfg::PAIR)
+      tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+    else
+      tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
   }
 }
 

@@ -153,6 +153,7 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, i
   if (MODE != GRID_FROZEN) {
     float mn = 0.f, mx = 0.f;
     float Sw = 0.f, Sq = 0.f, Sqq = 0.f, Sy = 0.f, Sqy = 0.f;
+#pragma unroll
     for (int c = 0; c < g; c += 32) {
       float w[32];
       loadw(c, w);
@@ -207,6 +208,7 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, i
       }
     }
   }
+#pragma unroll
   for (int c = 0; c < g; c += 32) {
     float w[32];
     loadw(c, w);
@@ -270,6 +272,7 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, i
 // Gram: raw fp32 tile into the k-split's partial buffer (upper part used).
 template <int BN>
 struct EpiGramPartial {
+  static constexpr bool FROM_TMEM = false;
   struct Params {
     float* part;
     long long split_stride;  // elements between k-split buffers
@@ -315,11 +318,30 @@ struct EpiGramPartial {
 // C0' = Lambda (Q^T W^~): column k scaled by lambda_k, stored fp32.
 template <int BN>
 struct EpiScaleStore {
+  static constexpr bool FROM_TMEM = false;
   struct Params {
     float* out;
     const float* lam;
     int ld;
   };
+  // From registers: 128 columns of tile row `rit`, starting at column col0.
+  __device__ static void apply_regs(const Params& p, const GemmGeom& g, const float (&acc)[128],
+                                    int tm, int, int, int rit, int col0) {
+    const int row = tm * 128 + rit;
+    if (row >= g.M) return;
+    float* o = p.out + (long long)row * p.ld;
+#pragma unroll
+    for (int c = 0; c < 128; c += 8) {
+      const int col = col0 + c;
+      if (col < g.N) {
+        float l[8], v[8];
+        load8_ro(p.lam + col, l);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = __fmul_rn(l[k], acc[c + k]);
+        st_v8f(o + col, v);
+      }
+    }
+  }
   __device__ static void apply(const Params& p, const GemmGeom& g, uint32_t taddr, int tm, int tn,
                                int, int q, int lane) {
     const int row = tm * 128 + q * 32 + lane;
@@ -355,7 +377,30 @@ struct TUpdateParams {
 
 template <int BN, bool MIX>
 struct EpiTUpdate {
+  static constexpr bool FROM_TMEM = false;
   using Params = TUpdateParams;
+  __device__ static void apply_regs(const Params& p, const GemmGeom& g, const float (&acc)[128],
+                                    int tm, int, int, int rit, int col0) {
+    const int row = tm * 128 + rit;
+    if (row >= g.M) return;
+    const long long rb = (long long)row * p.ld;
+    void* lo = lo_row<MIX>(p.t_lo, row, p.ld);
+#pragma unroll
+    for (int c = 0; c < 128; c += 8) {
+      const int col = col0 + c;
+      if (col < g.N) {
+        float cc[8], ll[8], tv[8];
+        ld_v8f(p.c0 + rb + col, cc);
+        load8_ro(p.lam + col, ll);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float inv = __frcp_rn(__fadd_rn(ll[j], p.rho));
+          tv[j] = __fmul_rn(__fadd_rn(cc[j], __fmul_rn(p.rho, acc[c + j])), inv);
+        }
+        put_operand8<MIX>(p.t_hi + rb, lo, col, tv);
+      }
+    }
+  }
   __device__ static void apply(const Params& p, const GemmGeom& g, uint32_t taddr, int tm, int tn,
                                int, int q, int lane) {
     const int row = tm * 128 + q * 32 + lane;
@@ -408,27 +453,32 @@ struct ProjParams {
 
 template <int BN, int MODE, bool MIX>
 struct EpiProject {
+  // The projection keeps a whole group of one row in flight twice (refit and
+  // projection passes): it reads the tile from tensor memory, where the
+  // engine leaves the summed accumulator, instead of 128 live registers.
+  static constexpr bool FROM_TMEM = true;
   using Params = ProjParams;
-  __device__ static void apply(const Params& p, const GemmGeom& g, uint32_t taddr, int tm, int tn,
-                               int, int q, int lane) {
-    const int row = tm * 128 + q * 32 + lane;
+  // Tile row `rit` of 128-row tile tm, columns col0 .. col0 + 127 at taddr.
+  __device__ static void apply_tmem(const Params& p, const GemmGeom& g, uint32_t taddr, int tm,
+                                    int rit, int col0) {
+    const int row = tm * 128 + rit;
     const bool valid = row < g.M;
     const int ngrp_row = p.ld / p.group;
     float r2 = 0.f, s2 = 0.f;
-    for (int c0 = 0; c0 < BN; c0 += p.group) {
-      const int col0 = tn * BN + c0;
-      if (col0 >= g.N) break;
-      const long long off = (long long)(valid ? row : 0) * p.ld + col0;
-      const long long goff = (long long)(valid ? row : 0) * ngrp_row + col0 / p.group;
+    for (int c0 = 0; c0 < 128; c0 += p.group) {
+      const int col = col0 + c0;
+      if (col >= g.N) break;
+      const long long off = (long long)(valid ? row : 0) * p.ld + col;
+      const long long goff = (long long)(valid ? row : 0) * ngrp_row + col / p.group;
       ProjRow r;
       r.V = p.V + off;
-      r.sig = p.sig + col0;
-      r.rsig = p.rsig + col0;
-      r.hd = p.hd + col0;
+      r.sig = p.sig + col;
+      r.rsig = p.rsig + col;
+      r.hd = p.hd + col;
       r.codes = p.codes + off;
       r.phi = p.p_hi + off;
       r.plo = MIX ? (void*)(reinterpret_cast<uint16_t*>(p.p_lo) + (long long)(valid ? row : 0) * 2 * p.ld +
-                            2 * col0)
+                            2 * col)
                   : (void*)(reinterpret_cast<float*>(p.p_lo) + off);
       r.scale = p.scale + goff;
       r.zero = p.zero + goff;
@@ -439,10 +489,10 @@ struct EpiProject {
     }
     r2 = warp_sum(r2);
     s2 = warp_sum(s2);
-    if (lane == 0) {
-      const int tile = tn * g.tiles_m + tm;
-      p.part[(tile * 4 + q) * 2 + 0] = r2;
-      p.part[(tile * 4 + q) * 2 + 1] = s2;
+    if ((rit & 31) == 0) {
+      const int tile = (col0 >> 7) * g.tiles_m + tm;  // 128 x 128 tile of the output
+      p.part[(tile * 4 + (rit >> 5)) * 2 + 0] = r2;
+      p.part[(tile * 4 + (rit >> 5)) * 2 + 1] = s2;
     }
   }
 };
@@ -450,10 +500,29 @@ struct EpiProject {
 // Objective: sum_k lambda_k acc_{jk}^2 per tile and warp.
 template <int BN>
 struct EpiObjective {
+  static constexpr bool FROM_TMEM = false;
   struct Params {
     const float* lam;
-    float* part;  // [tiles][4]
+    float* part;  // [128-row tiles x 128-column tiles][4]
   };
+  __device__ static void apply_regs(const Params& p, const GemmGeom& g, const float (&acc)[128],
+                                    int tm, int, int, int rit, int col0) {
+    const int row = tm * 128 + rit;
+    float s = 0.f;
+    if (row < g.M) {
+#pragma unroll
+      for (int c = 0; c < 128; c += 8) {
+        if (col0 + c < g.N) {
+          float l[8];
+          load8_ro(p.lam + col0 + c, l);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) s += l[k] * acc[c + k] * acc[c + k];
+        }
+      }
+    }
+    s = warp_sum(s);
+    if ((rit & 31) == 0) p.part[((col0 >> 7) * g.tiles_m + tm) * 4 + (rit >> 5)] = s;
+  }
   __device__ static void apply(const Params& p, const GemmGeom& g, uint32_t taddr, int tm, int tn,
                                int, int q, int lane) {
     const int row = tm * 128 + q * 32 + lane;
