@@ -27,15 +27,15 @@ unsigned long long g_launches = 0;  // kernels launched by this library
 inline void count_launch() { __atomic_fetch_add(&g_launches, 1ull, __ATOMIC_RELAXED); }
 // X^T X: bf16, both operands MN-major (X is token-major).
 // Promoted every 4 k-blocks (16 MMAs of K = 16).
-using GramCfg = GemmCfg<KIND_BF16, 256, 1, true, true, 4, 4>;
+using GramCfg = GemmCfg<KIND_BF16, 1, true, true, 4, 4, false>;
 // Eigenbasis GEMMs, K-major operands, promoted every 8 k-blocks:
 //   mixed split (tf32 hi.hi + one bf16 product for the corrections, 64 MMAs
 //   per chunk) for large layers, 3xTF32 (96 MMAs per chunk) where the
 //   reduction is short enough that the split's own rounding would dominate.
 // Both run on CTA pairs (2-SM MMAs of 256 x 128; each SM stages half of B,
 // which cuts the shared-memory traffic per MMA by a quarter) with 4 stages.
-using EigCfg = GemmCfg<KIND_MIX, 256, 2, false, false, 3, 16, true>;
-using EigCfg3 = GemmCfg<KIND_TF32, 256, 2, false, false, 3, 16, true>;
+using EigCfg = GemmCfg<KIND_MIX, 2, false, false, 3, 16, true>;
+using EigCfg3 = GemmCfg<KIND_TF32, 2, false, false, 3, 16, true>;
 static_assert(EigCfg::BN == EigCfg3::BN && EigCfg::BK == EigCfg3::BK &&
                   EigCfg::UNIT_M == EigCfg3::UNIT_M && EigCfg::B_ROWS == EigCfg3::B_ROWS,
               "same tile geometry");
@@ -777,8 +777,8 @@ int admmq_build_hessian(const void* X, int64_t n, int d, float* H, int accumulat
   CUtensorMap mx;
   if (!make_map(&mx, X, (uint64_t)d, (uint64_t)n, GramCfg::BK, false)) return ADMMQ_ERR_CUDA;
   GemmGeom g = make_geom(d, d, n, GramCfg::BN, GramCfg::BK, splits, true, status);
-  EpiGramPartial<GramCfg::BN>::Params ep{part, (long long)d * d, d};
-  CK((launch_gemm<GramCfg, EpiGramPartial<GramCfg::BN>>(mx, mx, mx, mx, g, ep, st)));
+  EpiGramPartial::Params ep{part, (long long)d * d, d};
+  CK((launch_gemm<GramCfg, EpiGramPartial>(mx, mx, mx, mx, g, ep, st)));
   const int nb = d / 32;
   count_launch(), k_gram_finalize<<<dim3(nb, nb), dim3(32, 8), 0, st>>>(part, splits, (long long)d * d, d, H,
                                                         accumulate, status);
@@ -939,8 +939,8 @@ int admmq_init(admmq_ctx* c, uint8_t* codes, float* scale, float* zero, void* st
   const int d = c->d, m = c->m;
   // C0' = Lambda Q^T W^~   (row j, column k)
   GemmGeom g = make_geom(m, d, d, EigCfg::BN, EigCfg::BK, 1, false, c->status, EigCfg::UNIT_M);
-  EpiScaleStore<EigCfg::BN>::Params ep{c->C0, c->lam32, d};
-  CK((launch_eig<EpiScaleStore<EigCfg::BN>, EpiScaleStore<EigCfg::BN>>(c->mix, c->mWt, c->mE, g, ep,
+  EpiScaleStore::Params ep{c->C0, c->lam32, d};
+  CK((launch_eig<EpiScaleStore, EpiScaleStore>(c->mix, c->mWt, c->mE, g, ep,
                                                                          st)));
   const long long groups = (long long)m * (d / c->p.group);
   if (c->w_dtype == ADMMQ_DTYPE_F32)
@@ -979,7 +979,7 @@ int admmq_iterate(admmq_ctx* c, int t0, int count, uint8_t* codes, float* scale,
       CK(cudaEventRecord(e0, st));
     }
     TUpdateParams p1{c->C0, c->lam32, c->T_hi, c->T_lo, rho, d};
-    CK((launch_eig<EpiTUpdate<EigCfg::BN, false>, EpiTUpdate<EigCfg::BN, true>>(c->mix, c->mP, c->mE,
+    CK((launch_eig<EpiTUpdate<false>, EpiTUpdate<true>>(c->mix, c->mP, c->mE,
                                                                                 g, p1, st)));
     if (c->timing) CK(cudaEventRecord(e1, st));
     ProjParams p2;
@@ -1000,16 +1000,16 @@ int admmq_iterate(admmq_ctx* c, int t0, int count, uint8_t* codes, float* scale,
     cudaError_t e;
     switch (c->p.grid_mode) {
       case ADMMQ_GRID_MINMAX:
-        e = launch_eig<EpiProject<EigCfg::BN, GRID_MINMAX, false>,
-                       EpiProject<EigCfg::BN, GRID_MINMAX, true>>(c->mix, c->mT, c->mQ, g, p2, st);
+        e = launch_eig<EpiProject<GRID_MINMAX, false>,
+                       EpiProject<GRID_MINMAX, true>>(c->mix, c->mT, c->mQ, g, p2, st);
         break;
       case ADMMQ_GRID_LSQ:
-        e = launch_eig<EpiProject<EigCfg::BN, GRID_LSQ, false>,
-                       EpiProject<EigCfg::BN, GRID_LSQ, true>>(c->mix, c->mT, c->mQ, g, p2, st);
+        e = launch_eig<EpiProject<GRID_LSQ, false>,
+                       EpiProject<GRID_LSQ, true>>(c->mix, c->mT, c->mQ, g, p2, st);
         break;
       default:
-        e = launch_eig<EpiProject<EigCfg::BN, GRID_FROZEN, false>,
-                       EpiProject<EigCfg::BN, GRID_FROZEN, true>>(c->mix, c->mT, c->mQ, g, p2, st);
+        e = launch_eig<EpiProject<GRID_FROZEN, false>,
+                       EpiProject<GRID_FROZEN, true>>(c->mix, c->mT, c->mQ, g, p2, st);
         break;
     }
     CK(e);
@@ -1041,8 +1041,8 @@ int admmq_finish(admmq_ctx* c, const uint8_t* codes, const float* scale, const f
           c->T_lo, c->mix);
     CK(cudaGetLastError());
     GemmGeom g = make_geom(m, d, d, EigCfg::BN, EigCfg::BK, 1, false, c->status, EigCfg::UNIT_M);
-    EpiObjective<EigCfg::BN>::Params ep{c->lam32, c->obj_part};
-    CK((launch_eig<EpiObjective<EigCfg::BN>, EpiObjective<EigCfg::BN>>(c->mix, c->mT, c->mE, g, ep,
+    EpiObjective::Params ep{c->lam32, c->obj_part};
+    CK((launch_eig<EpiObjective, EpiObjective>(c->mix, c->mT, c->mE, g, ep,
                                                                          st)));
     count_launch(), k_reduce_objective<<<1, 256, 0, st>>>(c->obj_part, c->tiles_eig * 4, objective);
     CK(cudaGetLastError());
@@ -1345,8 +1345,8 @@ extern "C" int admmq_build_hessian_static(const void* X, int64_t n, int d, float
   CUtensorMap mx;
   if (!make_map(&mx, X, (uint64_t)d, (uint64_t)n, GramCfg::BK, false)) return ADMMQ_ERR_CUDA;
   GemmGeom g = make_geom(d, d, n, GramCfg::BN, GramCfg::BK, splits, true, status);
-  EpiGramPartial<GramCfg::BN>::Params ep{part, (long long)d * d, d};
-  CK((launch_gemm<GramCfg, EpiGramPartial<GramCfg::BN>>(mx, mx, mx, mx, g, ep, st)));
+  EpiGramPartial::Params ep{part, (long long)d * d, d};
+  CK((launch_gemm<GramCfg, EpiGramPartial>(mx, mx, mx, mx, g, ep, st)));
   const int nb = d / 32;
   count_launch(), k_gram_finalize<<<dim3(nb, nb), dim3(32, 8), 0, st>>>(part, splits, (long long)d * d, d, H,
                                                                           accumulate, status);

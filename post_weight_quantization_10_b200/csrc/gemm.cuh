@@ -4,38 +4,42 @@
 // (128-byte swizzle, no multicast) and fp32 accumulation.  Operands are bf16
 // (kind::f16) or tf32 held in fp32 words (kind::tf32); a shared-memory row is
 // always 128 bytes (64 bf16 or 32 fp32 along K) and one MMA consumes 32 bytes
-// of K.  NPL = 2 runs the split-precision product used for fp32-accurate GEMMs
-// (3xTF32): every operand is stored as two tf32 planes (hi, lo) with
-// x ~= hi + lo, and each k-step issues A_hi*B_hi + A_hi*B_lo + A_lo*B_hi.
-// KIND_MIX is the cheaper split: plane 0 holds hi = tf32(x) (fp32 words),
-// plane 1 holds bf16 correction rows, each 128-byte row covering the same 32
-// K-elements as plane 0's row: [bf16(hi) x32 | bf16(lo) x32] for A and
-// [bf16(lo) x32 | bf16(hi) x32] for B, lo = x - hi.  Each k-step issues one
-// tf32 MMA on plane 0 and one bf16 MMA on plane 1, whose K = 16 runs over
-// hi(A).lo(B) and lo(A).hi(B): the same three terms in ~2/3 of the tensor
-// time, with the correction terms carried to bf16 precision.
+// of K.  Split-precision products for fp32-accurate GEMMs (NPL = 2 planes):
+//   3xTF32 (KIND_TF32): planes hi = tf32(x), lo = tf32(x - hi); each K step
+//     issues A_hi*B_hi + A_hi*B_lo + A_lo*B_hi.
+//   mixed (KIND_MIX): plane 0 holds hi = tf32(x); plane 1 holds bf16
+//     correction rows, each 128-byte row covering the same 32 K-elements as
+//     plane 0's row: [bf16(hi) x32 | bf16(lo) x32] for A and
+//     [bf16(lo) x32 | bf16(hi) x32] for B, lo = x - hi.  Each K step issues
+//     one tf32 MMA on plane 0 and one bf16 MMA on plane 1, whose K = 16 runs
+//     over hi(A).lo(B) and lo(A).hi(B): the same three terms in ~2/3 of the
+//     tensor time, the correction terms carried to bf16 precision.
 //
 // Promoted accumulation.  The tensor core adds every MMA into its fp32
 // accumulator with a small one-sided rounding error, so a long K sum drifts by
 // a relative amount proportional to the number of MMAs (measured 2.9e-5 for
 // K = 4096 with 3xTF32).  The MMA therefore writes each chunk of KC k-blocks
-// into a fresh tensor-memory slot, and the consumer warps add the chunks into
-// fp32 registers with round-to-nearest: the drift is bounded by one chunk.
+// into a fresh tensor-memory slot (a ring of two 256-column slots), and the
+// consumer warps add the chunks into fp32 registers with round-to-nearest:
+// the drift is bounded by one chunk.
 //
-// Warp roles (320 threads, one CTA per SM, 512 tensor-memory columns):
+// Tiles are 128 (CTA pairs: 256) rows x 256 columns.  Warp roles (320
+// threads, one CTA per SM, 512 tensor-memory columns):
 //   warp 0      TMA producer (one thread)
 //   warp 1      tensor-memory owner and MMA issuer (one thread)
-//   warps 2..9  two consumer warpgroups; thread = accumulator row
-//     BN = 128: the warpgroups take alternate tiles; the owner adds the chunks
-//               from a 3-slot ring, writes the sum to the final slot and runs
-//               the tile epilogue from there, while the other warpgroup
-//               accumulates the next tile.  The final slot passes from one
-//               tile's owner to the next through the `fin` barrier.
-//     BN = 256: both warpgroups take every tile, 128 columns each, from a
-//               2-slot ring, and store the tile from registers (Gram partial
-//               sums).
-// Work units (tile, k-split) are dealt to CTAs round-robin; all waits are
-// bounded (see ptx.cuh).
+//   warps 2..9  two consumer warpgroups: thread = accumulator row, each
+//               warpgroup 128 of the tile's 256 columns, summed in registers;
+//               the epilogue runs from those registers (apply_regs) or, for
+//               an epilogue that reads the tile twice (FROM_TMEM), from the
+//               last chunk's slot, where the sum is written back and which
+//               is released only afterwards (apply_tmem).
+// CTA pairs (PAIR): a cluster of two CTAs runs 2-SM MMAs (cta_group::2) of
+// 256 x 256: each CTA stages its 128 A rows and 128 of the 256 B rows; the
+// leader (rank 0) issues the MMAs and commits to the barriers of both CTAs;
+// both CTAs' TMA loads count on the leader's stage barrier; consumers release
+// ring slots to the leader with remote arrivals.
+// Work units (tile, k-split) are dealt to CTAs (or pairs) round-robin; every
+// wait on a barrier is bounded (see ptx.cuh).
 #pragma once
 #include "ptx.cuh"
 
@@ -43,8 +47,9 @@ namespace admmq {
 
 struct GemmGeom {
   int M, N, K;        // output rows / columns, reduction length
-  int tiles_m, tiles_n;  // 128-row and BN-column output tiles
-  int tiles_mu;          // unit rows: 128-row tiles, or 256-row tile pairs (CTA-pair configs)
+  int tiles_m;        // 128-row output tiles (counted up to whole units)
+  int tiles_n;        // 256-column output tiles
+  int tiles_mu;       // unit rows: 128-row tiles, or 256-row tile pairs
   int splits;         // k-splits per tile (units = tiles * splits)
   int kblocks;        // ceil(K / BK)
   int triangle;       // 1: only tiles that meet the upper triangle (i <= j)
@@ -56,37 +61,31 @@ struct GemmGeom {
 
 // Operand kinds: KIND_BF16 / KIND_TF32 are the instruction-descriptor formats
 // of plain products.  KIND_MIX is the split-precision product with one tf32
-// plane and one bf16 correction plane per operand (see GemmCfg).
+// plane and one bf16 correction plane per operand (see above).
 enum { KIND_BF16 = 1, KIND_TF32 = 2, KIND_MIX = 3 };
 
-template <int KIND_, int BN_, int NPL_, bool A_MN_, bool B_MN_, int STAGES_, int KC_,
-          bool PAIR_ = false>
+template <int KIND_, int NPL_, bool A_MN_, bool B_MN_, int STAGES_, int KC_, bool PAIR_>
 struct GemmCfg {
   static constexpr int KIND = KIND_;
   static constexpr int ELEM = KIND == KIND_BF16 ? 2 : 4;  // bytes per (plane-0) operand element
-  static constexpr int BM = 128, BN = BN_, BK = 128 / ELEM, NPL = NPL_, STAGES = STAGES_;
+  static constexpr int BM = 128, BN = 256, BK = 128 / ELEM, NPL = NPL_, STAGES = STAGES_;
   static constexpr int UK = 32 / ELEM;                     // K per MMA instruction
   static constexpr int KC = KC_;                           // k-blocks per promoted chunk
   static constexpr bool A_MN = A_MN_, B_MN = B_MN_;
-  static constexpr bool SPLITCOL = BN == 256;
-  // PAIR: a cluster of two CTAs runs 2-SM MMAs of 256 x BN; each CTA stages
-  // its 128 A rows and half of the BN B rows.
   static constexpr bool PAIR = PAIR_;
   static constexpr int UNIT_M = PAIR ? 2 * BM : BM;   // output rows per work unit
   static constexpr int B_ROWS = PAIR ? BN / 2 : BN;   // B rows staged per CTA
   static constexpr int A_PLANE = BM * 128;  // bytes per operand plane per stage
   static constexpr int B_PLANE = B_ROWS * 128;
   static constexpr int STAGE = NPL * (A_PLANE + B_PLANE);
-  static constexpr int RING = SPLITCOL ? 2 : 3;  // chunk slots in tensor memory
-  static constexpr int TMEM_COLS = 512;          // RING x BN (+ one final 128-column slot)
+  static constexpr int RING = 2;                 // 256-column chunk slots in tensor memory
+  static constexpr int TMEM_COLS = RING * BN;    // 512
   static constexpr int THREADS = 320;
-  static constexpr int CONS_WARP0 = 2;  // first consumer warp
-  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 4 * RING + 2) + 16;
+  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 2 * RING + 1) + 16;
   // arrivals that release a ring slot: every consumer thread of the CTA, or
   // one per consumer warp of both CTAs of a pair
-  static constexpr int SLOT_ARRIVALS = PAIR ? (SPLITCOL ? 16 : 8) : (SPLITCOL ? 256 : 128);
+  static constexpr int SLOT_ARRIVALS = PAIR ? 16 : 256;
   static constexpr int SMEM = STAGES * STAGE + 1024 + BAR_BYTES;
-  static_assert(BN == 128 || BN == 256, "BN must be 128 or 256");
   static_assert(!PAIR || (!A_MN && !B_MN), "CTA pairs: K-major operands");
   static_assert(KIND != KIND_MIX || (NPL == 2 && !A_MN && !B_MN), "mixed split: two K-major planes");
   // products per K step: 3xTF32 (hi.hi, hi.lo, lo.hi), mixed (tf32 hi.hi +
@@ -97,9 +96,10 @@ struct GemmCfg {
 
 // Unit -> (tile row, tile column, k-block range).  Splits are the outer index
 // so that CTAs running at the same time work on the same k-range of different
-// tiles.  Full grids are visited in bands of `band` tile rows, column by
+// tiles.  Full grids are visited in bands of `band` unit rows, column by
 // column inside a band, so that the tiles in flight share A rows and B
-// columns in L2.
+// columns in L2.  Triangle mode (square Gram) visits the 128-row tiles that
+// meet the upper triangle, column by column.
 template <int BM, int BN>
 __device__ __forceinline__ void decode_unit(const GemmGeom& g, int u, int& tm, int& tn, int& split,
                                             int& kb0, int& kb1) {
@@ -138,15 +138,11 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
-  // Ring-slot barriers per (consumer warpgroup, slot): [2 * wg + slot].  Each
-  // warpgroup waits only on its own chunks, in order, so no waiter is ever
-  // more than one phase away from its barrier.  (BN = 256 uses wg 0 only:
-  // both warpgroups consume every chunk.)
+  // Ring-slot barriers: both consumer warpgroups drain every chunk.
   constexpr int R = Cfg::RING;
-  uint64_t* rfull = bars + 2 * STAGES;  // [R * wg + slot]: slot holds a finished chunk
-  uint64_t* rempty = rfull + 2 * R;     // [R * wg + slot]: slot drained by its consumers
-  uint64_t* fin = rempty + 2 * R;       // final slot released by the previous tile's owner
-  uint64_t* drain = fin + 1;
+  uint64_t* rfull = bars + 2 * STAGES;  // [slot]: slot holds a finished chunk
+  uint64_t* rempty = rfull + R;         // [slot]: slot drained by its consumers
+  uint64_t* drain = rempty + R;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -162,11 +158,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1);
     }
-    for (int a = 0; a < 2 * R; ++a) {
+    for (int a = 0; a < R; ++a) {
       mbar_init(smem_u32(&rfull[a]), 1);
       mbar_init(smem_u32(&rempty[a]), Cfg::SLOT_ARRIVALS);
     }
-    mbar_init(smem_u32(fin), 128);
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -294,24 +289,18 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       constexpr int kKStepB = (Cfg::B_MN ? Cfg::UK * 128 : 32) >> 4;
       const uint64_t descA0 = smem_desc_sw128(smem_u32(smem), LBO_A, 1024);
       const uint64_t descB0 = smem_desc_sw128(smem_u32(smem + NPL * Cfg::A_PLANE), LBO_B, 1024);
-      int it = 0, lu = 0;
-      uint32_t q = 0;                      // chunks issued by this CTA
-      uint32_t use[2 * R] = {};            // chunks issued per (warpgroup, slot)
-      int prev[R];                         // warpgroup of the chunk last put in a slot
-#pragma unroll
-      for (int i = 0; i < R; ++i) prev[i] = -1;
+      int it = 0;
+      uint32_t q = 0;  // chunks issued: chunk q goes to slot q % R, use q / R of it
       bool ok = true;
-      for (int u = unit0; u < g.units && ok; u += unit_step, ++lu) {
+      for (int u = unit0; u < g.units && ok; u += unit_step) {
         int tm, tn, split, kb0, kb1;
         decode_unit<BM, BN>(g, u, tm, tn, split, kb0, kb1);
-        const int owner = Cfg::SPLITCOL ? 0 : (lu & 1);
         for (int c0 = kb0; c0 < kb1 && ok; c0 += KC, ++q) {
           const int c1 = min(c0 + KC, kb1);
           const uint32_t slot = q % R;
-          if (prev[slot] >= 0) {
+          if (q >= (uint32_t)R) {
             // wait until the slot's previous chunk has been drained
-            const int b = R * prev[slot] + (int)slot;
-            if (!mbar_wait(smem_u32(&rempty[b]), (use[b] - 1u) & 1u, abort_flag, g.status)) {
+            if (!mbar_wait(smem_u32(&rempty[slot]), (q / R - 1u) & 1u, abort_flag, g.status)) {
               ok = false;
               break;
             }
@@ -359,10 +348,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             commit_all(&empty[s]);
           }
           if (!ok) break;
-          const int b = R * owner + (int)slot;
-          commit_all(&rfull[b]);
-          ++use[b];
-          prev[slot] = owner;
+          commit_all(&rfull[slot]);
         }
       }
       // Every MMA issued above is complete once this arrives.
@@ -372,43 +358,36 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         mma_commit(smem_u32(drain));
       mbar_wait_drain(smem_u32(drain), 0);
     }
-  } else if (warp >= Cfg::CONS_WARP0) {
+  } else {
     // ---------------------------------------------------------- consumers
-    const int wg = (warp - Cfg::CONS_WARP0) >> 2;  // consumer warpgroup 0 or 1
+    const int wg = (warp - 2) >> 2;  // consumer warpgroup 0 or 1: columns 128 wg ..
     const int qtr = warp & 3;        // tensor-memory lane quarter this warp may access
     const uint32_t lane_off = (uint32_t)(qtr * 32) << 16;
-    const uint32_t col_off = Cfg::SPLITCOL ? (uint32_t)(wg * 128) : 0u;
-    const int bw = Cfg::SPLITCOL ? 0 : wg;  // barrier set of this warpgroup
-    uint32_t q = 0;
-    uint32_t my_use[R] = {};                // own chunks consumed per slot
-    int lu = 0;
+    const uint32_t col_off = (uint32_t)(wg * 128);
+    uint32_t q = 0;  // chunks consumed: chunk q is use q / R of slot q % R
     bool ok = true;
     // a pair member drains its slots for the leader's MMA issuer
     const uint32_t rempty_leader = Cfg::PAIR ? cluster_addr(smem_u32(rempty), 0) : 0u;
-    for (int u = unit0; u < g.units && ok; u += unit_step, ++lu) {
+    // releases ring slot `slot` for the MMA issuer (of this CTA or of the pair)
+    auto release = [&](uint32_t slot) {
+      if (Cfg::PAIR) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(rempty_leader + 8u * slot);
+      } else {
+        mbar_arrive(smem_u32(&rempty[slot]));
+      }
+    };
+    for (int u = unit0; u < g.units && ok; u += unit_step) {
       int tm, tn, split, kb0, kb1;
       decode_unit<BM, BN>(g, u, tm, tn, split, kb0, kb1);
       const int tile_m = Cfg::PAIR ? 2 * tm + (int)rank : tm;  // this CTA's 128-row tile
-      const bool mine = Cfg::SPLITCOL || ((lu & 1) == wg);
       float acc[128];
 #pragma unroll
       for (int i = 0; i < 128; ++i) acc[i] = 0.f;
-      // releases ring slot b for the MMA issuer (of this CTA or of the pair)
-      auto release = [&](int b) {
-        if (Cfg::PAIR) {
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(rempty_leader + 8u * (uint32_t)b);
-        } else {
-          mbar_arrive(smem_u32(&rempty[b]));
-        }
-      };
-      int kept_b = 0;
-      uint32_t kept_slot = 0;
+      uint32_t kept = 0;
       for (int c0 = kb0; c0 < kb1; c0 += KC, ++q) {
-        if (!mine) continue;
         const uint32_t slot = q % R;
-        const int b = R * bw + (int)slot;
-        const bool got = mbar_wait(smem_u32(&rfull[b]), my_use[slot] & 1u, abort_flag, g.status);
+        const bool got = mbar_wait(smem_u32(&rfull[slot]), (q / R) & 1u, abort_flag, g.status);
         if (!__all_sync(0xffffffffu, got)) {  // tcgen05.ld needs all 32 lanes
           ok = false;
           break;
@@ -425,53 +404,26 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         tc_fence_before();
         // An epilogue that reads the tile from tensor memory keeps the last
         // chunk's slot: the summed accumulator goes back into it below.
-        if (Cfg::SPLITCOL && Epi::FROM_TMEM && c0 + KC >= kb1) {
-          kept_b = b;
-          kept_slot = slot;
-        } else {
-          release(b);
-        }
-        ++my_use[slot];
+        if (Epi::FROM_TMEM && c0 + KC >= kb1)
+          kept = slot;
+        else
+          release(slot);
       }
-      if (!ok || !mine) continue;
-      if constexpr (Cfg::SPLITCOL) {
-        if constexpr (Epi::FROM_TMEM) {
-          const uint32_t ta = tmem_base + lane_off + kept_slot * BN + col_off;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            float v[32];
-#pragma unroll
-            for (int k = 0; k < 32; ++k) v[k] = acc[32 * j + k];
-            tmem_st32(ta + 32 * j, v);
-          }
-          Epi::apply_tmem(ep, g, ta, tile_m, qtr * 32 + lane, tn * BN + wg * 128);
-          tc_fence_before();
-          release(kept_b);
-        } else {
-          Epi::apply_regs(ep, g, acc, tile_m, tn, split, qtr * 32 + lane, tn * BN + wg * 128);
-        }
-      } else {
-        // The final slot is free once the previous tile's owner (the other
-        // warpgroup) has finished its epilogue: phase lu - 1 of `fin`.
-        if (lu > 0) {
-          const bool freed = mbar_wait(smem_u32(fin), (uint32_t)(lu - 1) & 1u, abort_flag, g.status);
-          if (!__all_sync(0xffffffffu, freed)) {
-            ok = false;
-            continue;
-          }
-          tc_fence_after();
-        }
-        const uint32_t fslot = tmem_base + lane_off + R * BN;
+      if (!ok) continue;
+      if constexpr (Epi::FROM_TMEM) {
+        const uint32_t ta = tmem_base + lane_off + kept * BN + col_off;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           float v[32];
 #pragma unroll
           for (int k = 0; k < 32; ++k) v[k] = acc[32 * j + k];
-          tmem_st32(fslot + 32 * j, v);
+          tmem_st32(ta + 32 * j, v);
         }
-        Epi::apply(ep, g, fslot, tile_m, tn, split, qtr, lane);
+        Epi::apply_tmem(ep, g, ta, tile_m, qtr * 32 + lane, tn * BN + wg * 128);
         tc_fence_before();
-        mbar_arrive(smem_u32(fin));
+        release(kept);
+      } else {
+        Epi::apply_regs(ep, g, acc, tile_m, tn, split, qtr * 32 + lane, tn * BN + wg * 128);
       }
     }
   }

@@ -266,11 +266,12 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, i
 }
 
 // -------------------------------------------------------------- epilogues
-// Each epilogue thread owns accumulator row (tm*128 + 32q + lane) and reads
-// 32 fp32 columns per tensor-memory load.
+// Each epilogue thread owns one accumulator row (tile row rit = 32 q + lane
+// of 128-row tile tm) and 128 consecutive columns col0 .. col0 + 127: from
+// registers (apply_regs) or from tensor memory (apply_tmem, 32 columns per
+// load).
 
 // Gram: raw fp32 tile into the k-split's partial buffer (upper part used).
-template <int BN>
 struct EpiGramPartial {
   static constexpr bool FROM_TMEM = false;
   struct Params {
@@ -296,27 +297,9 @@ struct EpiGramPartial {
       }
     }
   }
-  __device__ static void apply(const Params& p, const GemmGeom& g, uint32_t taddr, int tm, int tn,
-                               int split, int q, int lane) {
-    const int row = tm * 128 + q * 32 + lane;
-    float* out = p.part + split * p.split_stride + (long long)row * p.ld;
-    for (int c = 0; c < BN; c += 32) {
-      const int col = tn * BN + c;
-      if (col >= g.N) break;
-      float v[32];
-      tmem_ld32(taddr + c, v);
-      if (row < g.M) {
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          *reinterpret_cast<float4*>(out + col + 4 * k) =
-              make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
-      }
-    }
-  }
 };
 
 // C0' = Lambda (Q^T W^~): column k scaled by lambda_k, stored fp32.
-template <int BN>
 struct EpiScaleStore {
   static constexpr bool FROM_TMEM = false;
   struct Params {
@@ -342,26 +325,6 @@ struct EpiScaleStore {
       }
     }
   }
-  __device__ static void apply(const Params& p, const GemmGeom& g, uint32_t taddr, int tm, int tn,
-                               int, int q, int lane) {
-    const int row = tm * 128 + q * 32 + lane;
-    for (int c = 0; c < BN; c += 32) {
-      const int col = tn * BN + c;
-      if (col >= g.N) break;
-      float v[32];
-      tmem_ld32(taddr + c, v);
-      if (row < g.M) {
-        float* o = p.out + (long long)row * p.ld + col;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const float4 l = __ldg(reinterpret_cast<const float4*>(p.lam + col + 4 * k));
-          *reinterpret_cast<float4*>(o + 4 * k) =
-              make_float4(__fmul_rn(l.x, v[4 * k]), __fmul_rn(l.y, v[4 * k + 1]),
-                          __fmul_rn(l.z, v[4 * k + 2]), __fmul_rn(l.w, v[4 * k + 3]));
-        }
-      }
-    }
-  }
 };
 
 // GEMM 1 epilogue: T = (C0' + rho acc) / (lambda + rho), stored in the
@@ -375,7 +338,7 @@ struct TUpdateParams {
   int ld;
 };
 
-template <int BN, bool MIX>
+template <bool MIX>
 struct EpiTUpdate {
   static constexpr bool FROM_TMEM = false;
   using Params = TUpdateParams;
@@ -401,35 +364,6 @@ struct EpiTUpdate {
       }
     }
   }
-  __device__ static void apply(const Params& p, const GemmGeom& g, uint32_t taddr, int tm, int tn,
-                               int, int q, int lane) {
-    const int row = tm * 128 + q * 32 + lane;
-    for (int c = 0; c < BN; c += 32) {
-      const int col = tn * BN + c;
-      if (col >= g.N) break;
-      float v[32];
-      tmem_ld32(taddr + c, v);
-      if (row < g.M) {
-        const long long off = (long long)row * p.ld + col;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          float cc[8], tv[8];
-          ld_v8f(p.c0 + off + 8 * k, cc);
-          const float4 l0 = __ldg(reinterpret_cast<const float4*>(p.lam + col + 8 * k));
-          const float4 l1 = __ldg(reinterpret_cast<const float4*>(p.lam + col + 8 * k + 4));
-          const float ll[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float inv = __frcp_rn(__fadd_rn(ll[j], p.rho));
-            const float t = __fmul_rn(__fadd_rn(cc[j], __fmul_rn(p.rho, v[8 * k + j])), inv);
-            tv[j] = t;
-          }
-          put_operand8<MIX>(p.t_hi + (long long)row * p.ld, lo_row<MIX>(p.t_lo, row, p.ld),
-                            col + 8 * k, tv);
-        }
-      }
-    }
-  }
 };
 
 // GEMM 2 epilogue: W~ = Q T from tensor memory, fused grid refresh,
@@ -451,7 +385,7 @@ struct ProjParams {
   int L;
 };
 
-template <int BN, int MODE, bool MIX>
+template <int MODE, bool MIX>
 struct EpiProject {
   // The projection keeps a whole group of one row in flight twice (refit and
   // projection passes): it reads the tile from tensor memory, where the
@@ -498,7 +432,6 @@ struct EpiProject {
 };
 
 // Objective: sum_k lambda_k acc_{jk}^2 per tile and warp.
-template <int BN>
 struct EpiObjective {
   static constexpr bool FROM_TMEM = false;
   struct Params {
@@ -522,23 +455,6 @@ struct EpiObjective {
     }
     s = warp_sum(s);
     if ((rit & 31) == 0) p.part[((col0 >> 7) * g.tiles_m + tm) * 4 + (rit >> 5)] = s;
-  }
-  __device__ static void apply(const Params& p, const GemmGeom& g, uint32_t taddr, int tm, int tn,
-                               int, int q, int lane) {
-    const int row = tm * 128 + q * 32 + lane;
-    float acc = 0.f;
-    for (int c = 0; c < BN; c += 32) {
-      const int col = tn * BN + c;
-      if (col >= g.N) break;
-      float v[32];
-      tmem_ld32(taddr + c, v);
-      if (row < g.M) {
-#pragma unroll
-        for (int k = 0; k < 32; ++k) acc += __ldg(p.lam + col + k) * v[k] * v[k];
-      }
-    }
-    acc = warp_sum(acc);
-    if (lane == 0) p.part[(tn * g.tiles_m + tm) * 4 + q] = acc;
   }
 };
 
