@@ -170,6 +170,83 @@ class LayerRun:
         mark(4)
 
 
+def objective_report(A, run):
+    """Objective of the solve just run next to its RTN start and GPTQ on the
+    same layer (same H, same fixed min/max grid for RTN and GPTQ)."""
+    p = run.p
+    obj_admm = float(run.s.objective.cpu())
+    run.s.init()
+    run.s.finish(resid=False)
+    obj_rtn = float(run.s.objective.cpu())
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    g_codes, g_scale, g_zero = A.gptq(run.H, run.W, p.bits, p.group, p.lambda_rel)
+    torch.cuda.synchronize()
+    gptq_s = time.perf_counter() - t0
+    obj_gptq = run.s.objective_of(g_codes, g_scale, g_zero)
+    del g_codes, g_scale, g_zero
+    return {"admm_q": obj_admm, "rtn": obj_rtn, "gptq": obj_gptq,
+            "admm_over_rtn": obj_admm / obj_rtn, "admm_over_gptq": obj_admm / obj_gptq,
+            "gptq_s": gptq_s}
+
+
+def run_decoder(args, rank, world, device):
+    """One Qwen3-8B-shaped decoder layer per rank: its four solves (q/k/v and
+    gate/up stacked on their shared inputs), each timed like the single-layer
+    step; the value is the layer's solve time (sum over the four)."""
+    from post_weight_quantization_10_b200 import admmq as A
+    A.lib()
+    bits = args.bits or 3
+    solves = []
+    n0 = A.launch_count()
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    for label, p, seed in workloads.decoder_layer(bits):
+        if args.tokens:
+            p = workloads.scaled(p, args.tokens, p.d_in, p.d_out)
+        run = LayerRun(A, p, args.grid, seed=seed + 1000 * rank, device=device, split=args.split)
+        eigh_s = run.setup_eigh()
+        for _ in range(args.warmup):
+            run.step()
+        torch.cuda.synchronize()
+        dist_barrier(world)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.steps):
+            run.step()
+        b.record()
+        torch.cuda.synchronize()
+        ms = dist_max(a.elapsed_time(b), world, device) / args.steps
+        obj = objective_report(A, run)
+        solves.append({"solve": label, "d_in": p.d_in, "d_out": p.d_out, "bits": p.bits,
+                       "iters": p.iters, "s": ms / 1e3, "eigh_s": eigh_s, "split": run.s.split,
+                       "iters_per_s": p.iters / (ms / 1e3), "objective": obj})
+        del run
+        torch.cuda.empty_cache()
+    clk = clocks.stop()
+    if rank != 0:
+        return None
+    s_layer = sum(x["s"] for x in solves)
+    return {
+        "metric": "ADMM-Q decoder-layer solve: s/layer (four solves, eigh separate)",
+        "value": s_layer, "unit": "s/layer", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": s_layer * 1e3, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32 via tf32+bf16 split",
+        "data": "synthetic (seeded Qwen3-8B-shaped activations and weights; no dataset)",
+        "config": {"workload": "Qwen3-8B-shaped decoder layer: qkv 4096->6144, o 4096->4096, "
+                               "gate_up 4096->24576, down 12288->4096; W%d g128 T=%d grid=%s"
+                               % (bits, solves[0]["iters"], args.grid),
+                   "parallelism": f"independent decoder layers x{world}",
+                   "l2": "inputs larger than L2"},
+        "s_per_layer_with_eigh": s_layer + sum(x["eigh_s"] for x in solves),
+        "solves": solves,
+        "gpu_launches": A.launch_count() - n0,
+        "clocks": clk,
+    }
+
+
 def run_ours(args, rank, world, device):
     from post_weight_quantization_10_b200 import admmq as A
     A.lib()
@@ -215,19 +292,8 @@ def run_ours(args, rank, world, device):
         e2e = run_e2e(A, run, args, world, device)
 
     # objective 1/2 Tr((D - W_hat)^T H (D - W_hat)) of the solve just timed,
-    # next to that of its RTN start (same layer, same H)
-    obj_admm = float(run.s.objective.cpu())
-    run.s.init()
-    run.s.finish(resid=False)
-    obj_rtn = float(run.s.objective.cpu())
-    # GPTQ (Algorithm 1, float64, the same fixed grid as RTN) on the same layer
-    torch.cuda.synchronize()
-    t0 = time.perf_counter()
-    g_codes, g_scale, g_zero = A.gptq(run.H, run.W, p.bits, p.group, p.lambda_rel)
-    torch.cuda.synchronize()
-    gptq_s = time.perf_counter() - t0
-    obj_gptq = run.s.objective_of(g_codes, g_scale, g_zero)
-    del g_codes, g_scale, g_zero
+    # next to its RTN start and GPTQ on the same layer
+    obj = objective_report(A, run)
 
     if rank != 0:
         return None
@@ -282,11 +348,9 @@ def run_ours(args, rank, world, device):
                      "peak_note": "bf16 dense %s sustained %.1f TF/s / %d (bf16-MMA units of tensor "
                                   "work per fp32-accurate product, %s split)" % (
                                       pk["src"], pk["bf16_sust"], per_product, split)},
-        "objective": {"admm_q": obj_admm, "rtn": obj_rtn, "gptq": obj_gptq,
-                      "admm_over_rtn": obj_admm / obj_rtn, "admm_over_gptq": obj_admm / obj_gptq,
-                      "gptq_s": gptq_s,
-                      "note": "1/2 Tr((D - W_hat)^T H (D - W_hat)), H = X^T X + lambda I; RTN and "
-                              "GPTQ on the min/max grid of W_hat, ADMM-Q with its refreshed grid"},
+        "objective": dict(obj, note="1/2 Tr((D - W_hat)^T H (D - W_hat)), H = X^T X + lambda I; "
+                                    "RTN and GPTQ on the min/max grid of W_hat, ADMM-Q with its "
+                                    "refreshed grid"),
         "gpu_launches": launches,
         "clocks": clk,
         "e2e": e2e,
@@ -436,9 +500,34 @@ def cpu_baseline(p, grid):
             "kind": "oracle", "sample": r["sample"], "s_per_layer": r["step_s"]}
 
 
+def run_reference_decoder(args, world):
+    """The oracle on the decoder-layer workload: the bounded sample of each of
+    the four solves, summed (seconds per decoder layer)."""
+    bits = args.bits or 3
+    layers = workloads.decoder_layer(bits)
+    for _ in range(args.warmup):
+        cpu_sample(layers[0][1], args.grid)
+    vals = [sum(cpu_sample(p, args.grid)["step_s"] for _, p, _ in layers) for _ in range(args.steps)]
+    value = float(np.mean(vals))
+    cores = _blas_threads() or os.cpu_count()
+    sample = ("per solve: Gram of 8192 tokens + 1 ADMM iteration at full size, extrapolated "
+              "linearly to n and T; summed over the four solves")
+    return {"impl": "reference", "metric": "ADMM-Q decoder-layer solve: s/layer (four solves, eigh separate)",
+            "value": value, "unit": "s/layer", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": value * 1e3, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "Qwen3-8B-shaped decoder layer, W%d g128" % bits},
+            "cpu_baseline": {"value": value, "unit": "s/layer", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "s/layer", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
+    if args.workload == "decoder":
+        return run_reference_decoder(args, world)
     p = workloads.PRESETS[args.workload]
     for _ in range(args.warmup):
         cpu_sample(p, args.grid)
@@ -474,7 +563,9 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="q_proj", choices=sorted(workloads.PRESETS))
+    ap.add_argument("--workload", default="q_proj", choices=sorted(workloads.PRESETS) + ["decoder"],
+                    help="a single layer preset, or 'decoder': a whole decoder layer's four solves")
+    ap.add_argument("--bits", type=int, default=0, help="decoder workload: W2/W3/W4 (default 3)")
     ap.add_argument("--grid", default="lsq", choices=["lsq", "minmax", "frozen"])
     ap.add_argument("--split", default="auto", choices=["auto", "mixed", "3xtf32"],
                     help="split precision of the eigenbasis GEMMs (auto: mixed from d_in 2048)")
@@ -499,7 +590,7 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=device)
     try:
-        line = run_ours(args, rank, world, device)
+        line = (run_decoder if args.workload == "decoder" else run_ours)(args, rank, world, device)
         if line:
             print(json.dumps(line), flush=True)
     finally:

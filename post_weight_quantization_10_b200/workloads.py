@@ -64,6 +64,25 @@ PRESETS = {
 }
 
 
+def decoder_layer(bits: int = 3, n: int = 262144):
+    """A Qwen3-8B-shaped decoder layer as four solves, one per distinct input
+    (and Hessian): q/k/v (4096 -> 4096 + 1024 + 1024) and gate/up (4096 ->
+    12288 + 12288) share their input, so each pair of stacked output rows is
+    one problem; o (4096 -> 4096) and down (12288 -> 4096) stand alone.  The
+    attention-side inputs use the q_proj activation recipe, the MLP's down
+    input the SiLU-gated one.  T = 100 iterations (150 for 2 bits).
+    Returns [(label, preset, seed)]."""
+    T = 150 if bits == 2 else 100
+    q, dn = PRESETS["q_proj"], PRESETS["down_proj"]
+    mk = lambda base, name, d_in, d_out: LayerPreset(
+        **{**base.__dict__, "name": name, "n": n, "d_in": d_in, "d_out": d_out, "bits": bits,
+           "iters": T})
+    return [("qkv", mk(q, "qkv", 4096, 6144), 0),
+            ("o", mk(q, "o", 4096, 4096), 10),
+            ("gate_up", mk(q, "gate_up", 4096, 24576), 20),
+            ("down", mk(dn, "down", 12288, 4096), 30)]
+
+
 def scaled(preset: LayerPreset, n: int, d_in: int, d_out: int, **kw) -> LayerPreset:
     """The same recipe at other sizes (used for parity cases the oracle finishes)."""
     fields = dict(preset.__dict__)
