@@ -190,6 +190,115 @@ def objective_report(A, run):
             "gptq_s": gptq_s}
 
 
+class ShardRun(LayerRun):
+    """One layer split over the ranks: this rank's block of calibration tokens
+    and of output rows; H is the all-reduced sum of the ranks' partial Grams
+    (the layer's one exchange step), every rank eigendecomposes it and solves
+    its rows."""
+
+    def __init__(self, A, p, grid, rank, world, device, split="auto"):
+        from post_weight_quantization_10_b200 import sharded
+        X = workloads.make_activations(p, seed=0, device=device)
+        W = workloads.make_weights(p, seed=0, device=device, dtype=torch.bfloat16)
+        t0, t1 = sharded.block(p.n, world, rank)
+        self.rows = sharded.block(p.d_out, world, rank)
+        self.A, self.p, self.world = A, p, world
+        self.X = X[t0:t1].contiguous()
+        self.W = W[self.rows[0]:self.rows[1]].contiguous()
+        del X, W
+        torch.cuda.empty_cache()
+        self.H = torch.empty((p.d_in, p.d_in), dtype=torch.float32, device=device)
+        self.gram_ws = torch.empty(A.gram_workspace_bytes(self.X.shape[0], p.d_in),
+                                   dtype=torch.uint8, device=device)
+        prm = A.Params(bits=p.bits, group=p.group, iters=p.iters, rho0=p.rho0, gamma=p.gamma,
+                       lambda_rel=p.lambda_rel, grid=grid, split=split)
+        self.s = A.Solver(p.d_in, self.W.shape[0], prm, device=device)
+        self.packed = torch.empty((self.W.shape[0], p.d_in * p.bits // 32), dtype=torch.int32,
+                                  device=device)
+
+    def _gram(self):
+        self.A.build_hessian(self.X, self.H, workspace=self.gram_ws)
+        if self.world > 1:
+            torch.distributed.all_reduce(self.H, op=torch.distributed.ReduceOp.SUM)
+
+    def setup_eigh(self):
+        self._gram()
+        self.s.prepare(self.H, self.W)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        self.s.eigh()
+        torch.cuda.synchronize()
+        return time.perf_counter() - t0
+
+    def step(self, ev=None):
+        mark = (lambda k: ev[k].record()) if ev else (lambda k: None)
+        mark(0)
+        self._gram()
+        mark(1)
+        self.s.prepare(self.H, self.W)
+        self.s.init()
+        mark(2)
+        self.s.iterate(0, self.p.iters)
+        mark(3)
+        self.s.finish()
+        self.A.pack(self.s.codes, self.p.bits, out=self.packed)
+        mark(4)
+
+
+def run_sharded(args, rank, world, device):
+    """One layer over all ranks (strong scaling): value = ADMM iterations of
+    the whole layer per second, from the slowest rank's step time."""
+    from post_weight_quantization_10_b200 import admmq as A
+    A.lib()
+    p = workloads.PRESETS[args.workload]
+    if args.tokens:
+        p = workloads.scaled(p, args.tokens, p.d_in, p.d_out)
+    run = ShardRun(A, p, args.grid, rank, world, device, split=args.split)
+    eigh_s = run.setup_eigh()
+    for _ in range(args.warmup):
+        run.step()
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    n0 = A.launch_count()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for k in range(args.steps):
+        run.step(evs[k])
+    b.record()
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    clk = clocks.stop()
+    ms = dist_max(a.elapsed_time(b), world, device)
+    phase = np.zeros(4)
+    for e in evs:
+        phase += [e[i].elapsed_time(e[i + 1]) for i in range(4)]
+    phase /= args.steps
+    obj = D.sum_over_ranks(float(run.s.objective.cpu()), world, device)
+    if rank != 0:
+        return None
+    return {
+        "metric": METRIC, "value": p.iters * args.steps / (ms / 1e3), "unit": "iters/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None,
+        "dtype": "f32 via tf32+bf16 split" if run.s.split == "mixed" else "f32 via 3xtf32",
+        "data": "synthetic (seeded Qwen3-8B-shaped activations and weights; no dataset)",
+        "config": {"workload": workload_desc(p, args.grid) + " (one layer split over the ranks)",
+                   "parallelism": f"tokens and output rows split over {world} ranks, "
+                                  "H all-reduced", "split": run.s.split,
+                   "l2": "inputs larger than L2"},
+        "s_per_layer": ms / 1e3 / args.steps, "eigh_s": eigh_s,
+        "phase_ms_rank0": {"gram_allreduce": phase[0], "scale_init": phase[1], "admm": phase[2],
+                           "finish_pack": phase[3]},
+        "objective": obj, "gpu_launches": A.launch_count() - n0, "clocks": clk,
+    }
+
+
 def run_decoder(args, rank, world, device):
     """One Qwen3-8B-shaped decoder layer per rank: its four solves (q/k/v and
     gate/up stacked on their shared inputs), each timed like the single-layer
@@ -566,6 +675,8 @@ def main():
     ap.add_argument("--workload", default="q_proj", choices=sorted(workloads.PRESETS) + ["decoder"],
                     help="a single layer preset, or 'decoder': a whole decoder layer's four solves")
     ap.add_argument("--bits", type=int, default=0, help="decoder workload: W2/W3/W4 (default 3)")
+    ap.add_argument("--shard", action="store_true",
+                    help="split ONE layer over the ranks (tokens and output rows; H all-reduced)")
     ap.add_argument("--grid", default="lsq", choices=["lsq", "minmax", "frozen"])
     ap.add_argument("--split", default="auto", choices=["auto", "mixed", "3xtf32"],
                     help="split precision of the eigenbasis GEMMs (auto: mixed from d_in 2048)")
@@ -590,7 +701,8 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=device)
     try:
-        line = (run_decoder if args.workload == "decoder" else run_ours)(args, rank, world, device)
+        runner = run_decoder if args.workload == "decoder" else (run_sharded if args.shard else run_ours)
+        line = runner(args, rank, world, device)
         if line:
             print(json.dumps(line), flush=True)
     finally:
