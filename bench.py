@@ -131,7 +131,7 @@ class ClockSampler:
 class LayerRun:
     """Device-resident state of one layer solve through the C ABI binding."""
 
-    def __init__(self, A, p, grid, seed, device, split="auto"):
+    def __init__(self, A, p, grid, seed, device, split="auto", scaling=True):
         self.A, self.p = A, p
         self.X = workloads.make_activations(p, seed=seed, device=device)
         self.W = workloads.make_weights(p, seed=seed, device=device, dtype=torch.bfloat16)
@@ -139,7 +139,7 @@ class LayerRun:
         self.gram_ws = torch.empty(A.gram_workspace_bytes(p.n, p.d_in), dtype=torch.uint8,
                                    device=device)
         prm = A.Params(bits=p.bits, group=p.group, iters=p.iters, rho0=p.rho0, gamma=p.gamma,
-                       lambda_rel=p.lambda_rel, grid=grid, split=split)
+                       lambda_rel=p.lambda_rel, grid=grid, split=split, scaling=scaling)
         self.s = A.Solver(p.d_in, p.d_out, prm, device=device)
         self.packed = torch.empty((p.d_out, p.d_in * p.bits // 32), dtype=torch.int32,
                                   device=device)
@@ -362,7 +362,8 @@ def run_ours(args, rank, world, device):
     p = workloads.PRESETS[args.workload]
     if args.tokens:
         p = workloads.scaled(p, args.tokens, p.d_in, p.d_out)
-    run = LayerRun(A, p, args.grid, seed=rank, device=device, split=args.split)
+    run = LayerRun(A, p, args.grid, seed=rank, device=device, split=args.split,
+                   scaling=not args.no_scaling)
     eigh_s = run.setup_eigh()
     for _ in range(args.warmup):
         run.step()
@@ -437,7 +438,9 @@ def run_ours(args, rank, world, device):
         "vs_baseline": None,
         "dtype": "f32 via tf32+bf16 split" if split == "mixed" else "f32 via 3xtf32",
         "data": "synthetic (seeded Qwen3-8B-shaped activations and weights; no dataset)",
-        "config": {"workload": workload_desc(p, args.grid), "parallelism": f"independent layers x{world}",
+        "config": {"workload": workload_desc(p, args.grid) + (" Sigma=I (unscaled ablation)"
+                                                              if args.no_scaling else ""),
+                   "parallelism": f"independent layers x{world}",
                    "l2": "inputs larger than L2 (X is %.1f GiB)" % (n * d * 2 / 2**30),
                    "eigh": "one-time setup outside the step (eigh_s)",
                    "split": split},
@@ -675,6 +678,8 @@ def main():
     ap.add_argument("--workload", default="q_proj", choices=sorted(workloads.PRESETS) + ["decoder"],
                     help="a single layer preset, or 'decoder': a whole decoder layer's four solves")
     ap.add_argument("--bits", type=int, default=0, help="decoder workload: W2/W3/W4 (default 3)")
+    ap.add_argument("--no-scaling", action="store_true",
+                    help="Sigma = I: the unscaled ablation (objective comparison)")
     ap.add_argument("--shard", action="store_true",
                     help="split ONE layer over the ranks (tokens and output rows; H all-reduced)")
     ap.add_argument("--grid", default="lsq", choices=["lsq", "minmax", "frozen"])

@@ -75,6 +75,8 @@ typedef struct admmq_params {
   float lambda_rel; /* damping: lambda = lambda_rel * mean(diag(X^T X))          */
   int grid_mode;    /* ADMMQ_GRID_*                                              */
   int split_mode;   /* ADMMQ_SPLIT_*                                             */
+  int no_scaling;   /* 1: Sigma = I, the unscaled ablation ([ADMM-Q] Methodology
+                       section 2 reports what removing the scaling costs); 0 */
 } admmq_params;
 
 typedef struct admmq_ctx admmq_ctx; /* opaque; host memory owned by the library */
@@ -141,7 +143,8 @@ void admmq_destroy(admmq_ctx* ctx);
 
 /* Damping and diagonal scaling (Methodology section 1 and section 2,
  * "diagonal scaling"): lambda = lambda_rel * mean(diag G), H = G + lambda I,
- * sigma_i = H_ii^(-1/2), H~ = Sigma H Sigma (float64, into the workspace) and
+ * sigma_i = H_ii^(-1/2) (1 with params.no_scaling), H~ = Sigma H Sigma
+ * (float64, into the workspace) and
  * the scaled weights W^~ = Sigma^-1 W_hat as split-precision operand planes
  * (see "operand encoding" below).
  *   G_dev      fp32 [d_in][d_in], X^T X WITHOUT damping (admmq_build_hessian).

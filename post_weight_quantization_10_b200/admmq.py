@@ -34,7 +34,7 @@ class _Params(ctypes.Structure):
     _fields_ = [("bits", ctypes.c_int), ("group", ctypes.c_int), ("iters", ctypes.c_int),
                 ("rho0", ctypes.c_float), ("gamma", ctypes.c_float),
                 ("lambda_rel", ctypes.c_float), ("grid_mode", ctypes.c_int),
-                ("split_mode", ctypes.c_int)]
+                ("split_mode", ctypes.c_int), ("no_scaling", ctypes.c_int)]
 
 
 @dataclass
@@ -47,10 +47,11 @@ class Params:
     lambda_rel: float = 0.01
     grid: str = "lsq"
     split: str = "auto"   # eigenbasis GEMM split precision: auto | 3xtf32 | mixed
+    scaling: bool = True  # False: Sigma = I (the unscaled ablation)
 
     def c(self) -> _Params:
         return _Params(self.bits, self.group, self.iters, self.rho0, self.gamma, self.lambda_rel,
-                       GRID_MODES[self.grid], SPLIT_MODES[self.split])
+                       GRID_MODES[self.grid], SPLIT_MODES[self.split], int(not self.scaling))
 
 
 _lib = None

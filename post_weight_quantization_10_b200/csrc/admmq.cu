@@ -47,7 +47,9 @@ enum { SETUP_OK = 0, SETUP_NONFINITE = 1, SETUP_NOT_PD = 2 };
 
 // ------------------------------------------------------------------ kernels
 
-__global__ void k_diag_stats(const float* __restrict__ G, int d, float lambda_rel,
+// sigma = Diag(H)^(-1/2), or 1 with scale == 0 (the unscaled ablation: the
+// iteration then runs on H itself; diag H is still the refit's weight).
+__global__ void k_diag_stats(const float* __restrict__ G, int d, float lambda_rel, int scale,
                              double* __restrict__ lam_out, double* __restrict__ sig64,
                              float* __restrict__ hdiag, float* __restrict__ sigma,
                              float* __restrict__ rsig, int* __restrict__ status) {
@@ -69,11 +71,11 @@ __global__ void k_diag_stats(const float* __restrict__ G, int d, float lambda_re
     } else if (h <= 0.0) {
       atomicExch(&status[1], SETUP_NOT_PD);
     }
-    const double sg = 1.0 / sqrt(h);
+    const double sg = scale ? 1.0 / sqrt(h) : 1.0;
     sig64[i] = sg;
     hdiag[i] = (float)h;
     sigma[i] = (float)sg;
-    rsig[i] = (float)sqrt(h);
+    rsig[i] = scale ? (float)sqrt(h) : 1.f;
   }
 }
 
@@ -652,6 +654,7 @@ int check_params(int d, int m, const admmq_params* p) {
     return ADMMQ_ERR_INVALID_ARG;
   if (p->split_mode < ADMMQ_SPLIT_AUTO || p->split_mode > ADMMQ_SPLIT_MIXED)
     return ADMMQ_ERR_INVALID_ARG;
+  if (p->no_scaling != 0 && p->no_scaling != 1) return ADMMQ_ERR_INVALID_ARG;
   return ADMMQ_OK;
 }
 
@@ -874,7 +877,7 @@ int admmq_prepare(admmq_ctx* c, const float* G, const void* W_hat, int w_dtype, 
   c->W_hat = W_hat;
   c->w_dtype = w_dtype;
   CK(cudaMemsetAsync(c->status, 0, 16, st));
-  count_launch(), k_diag_stats<<<1, 1024, 0, st>>>(G, d, c->p.lambda_rel, c->lam64, c->sig64, c->hdiag, c->sigma,
+  count_launch(), k_diag_stats<<<1, 1024, 0, st>>>(G, d, c->p.lambda_rel, !c->p.no_scaling, c->lam64, c->sig64, c->hdiag, c->sigma,
                                    c->rsig, c->status);
   CK(cudaGetLastError());
   count_launch(), k_scale_hessian<<<grid_for((long long)d * d), 256, 0, st>>>(G, d, c->lam64, c->sig64, c->Ht);
@@ -1222,7 +1225,7 @@ int admmq_gptq(const float* G, const void* W_hat, int w_dtype, int d, int m, int
 
   // H = X^T X + lambda I (lambda as in the ADMM-Q setup) and the fixed grid
   CK(cudaMemsetAsync(status, 0, 16, st));
-  count_launch(), k_diag_stats<<<1, 1024, 0, st>>>(G, d, lambda_rel, lam64, (double*)(base + Lo.sig64),
+  count_launch(), k_diag_stats<<<1, 1024, 0, st>>>(G, d, lambda_rel, 1, lam64, (double*)(base + Lo.sig64),
                                                    (float*)(base + Lo.hdiag), (float*)(base + Lo.sigma),
                                                    (float*)(base + Lo.rsig), status);
   CK(cudaGetLastError());

@@ -51,9 +51,10 @@ def _oracle(p, X, W, grid, iters=None):
     return H, Wm, res
 
 
-def _solver(A, p, X, W, grid, iters=None, split="auto"):
+def _solver(A, p, X, W, grid, iters=None, split="auto", scaling=True):
     prm = A.Params(bits=p.bits, group=p.group, iters=p.iters if iters is None else iters,
-                   rho0=p.rho0, gamma=p.gamma, lambda_rel=p.lambda_rel, grid=grid, split=split)
+                   rho0=p.rho0, gamma=p.gamma, lambda_rel=p.lambda_rel, grid=grid, split=split,
+                   scaling=scaling)
     G = A.build_hessian(X)
     s = A.Solver(X.shape[1], W.shape[0], prm)
     s.prepare(G, W)
@@ -213,3 +214,31 @@ def test_free_running_solve(A, name, grid):
     r = s.resid.cpu().numpy()[: p.iters]
     np.testing.assert_allclose(r[:3, 0], res["r"][:3], rtol=1e-3)
     assert agree >= 0.9 and abs(rel) <= 0.2
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged"])
+def test_unscaled_ablation_teacher_forced(A, name):
+    """Sigma = I (the pages' ablation of the diagonal scaling): step parity
+    against the oracle run with scaling=False, as in the scaled case."""
+    p, X, W = _layer(name)
+    trace = []
+    H = O.hessian(X.float().cpu().numpy(), p.lambda_rel)
+    Wm = W.float().cpu().numpy().T.astype(np.float64)
+    O.admm_q(H, Wm, p.bits, p.group, p.iters, rho0=p.rho0, gamma=p.gamma, grid="lsq",
+             scaling=False, trace=trace)
+    s = _solver(A, p, X, W, "lsq", scaling=False)
+    assert float(s.buffer("sigma").max()) == 1.0 and float(s.buffer("sigma").min()) == 1.0
+    s.init()
+    wt = torch.empty((W.shape[0], X.shape[1]), dtype=torch.float32, device="cuda")
+    s.dump_wtilde(wt)
+    for t in STEPS[name]:
+        e = trace[t]
+        _load_state(s, e)
+        s.iterate(t, 1)
+        torch.cuda.synchronize()
+        ref = e["W_tilde"].T
+        err = np.linalg.norm(wt.cpu().numpy() - ref) / np.linalg.norm(ref)
+        assert err <= 1e-4, (t, err)
+        mism = np.mean(s.codes.cpu().numpy() != e["codes_out"].T)
+        assert mism <= 1e-3, (t, mism)
+    s.dump_wtilde(None)
