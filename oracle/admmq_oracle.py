@@ -127,6 +127,10 @@ def project(Y: np.ndarray, bits: int, group: int, mode: str, hdiag: np.ndarray,
       "minmax": scale/zero refitted from the group's min/max (with 0 included);
       "lsq":    one weighted least-squares refit in the scaled metric
                 (weights diag H), warm-started from the previous grid;
+      "mse":    the clipped min/max grid with the smallest squared error over
+                the ratios of oracle.projection_fp32.CLIP_RATIOS (a clipping
+                heuristic by MSE grid search, [ADMM-Q] Methodology section 3,
+                modularity);
       "frozen": the previous grid is kept (GPTQ-style fixed grid).
     Returns (codes, scale, zero, D) like rtn().
     """
@@ -141,6 +145,8 @@ def project(Y: np.ndarray, bits: int, group: int, mode: str, hdiag: np.ndarray,
         wg = np.broadcast_to(np.asarray(hdiag, np.float32).reshape(d // group, group)[None],
                              (m, d // group, group)).reshape(-1, group)
         s, z = p32.fit_lsq(yg, wg, sp, zp, L)
+    elif mode == "mse":
+        s, z = p32.fit_mse(yg, L)
     elif mode == "frozen":
         s, z = sp, zp
     else:

@@ -21,6 +21,11 @@ Grid semantics (our reading; the pages do not define the fit):
           problem): first slope and offset, then the integer zero point, then
           the slope again for that zero point.  Groups whose fit is degenerate
           keep the previous grid.
+  mse     clipping search: for each ratio a in CLIP_RATIOS (1, 31/32, ..., 17/32,
+          exact in float32) the min/max grid of the clipped range
+          (a * mn, a * mx); each candidate's squared error sum (y - D)^2 is
+          summed in element order, and the first smallest one wins.  The
+          ratio 1 candidate is the min/max grid itself.
   rounding q = clamp(rint(y / s) + z, 0, L);  D = s (q - z).
 """
 from __future__ import annotations
@@ -34,17 +39,53 @@ def _f(x):
     return np.asarray(x, dtype=np.float32)
 
 
-def fit_minmax(yg: np.ndarray, L: int):
-    """(scale, zero) per group; yg has one group per row."""
-    yg = _f(yg)
-    mn = np.minimum(yg.min(axis=1), f32(0))
-    mx = np.maximum(yg.max(axis=1), f32(0))
+CLIP_RATIOS = tuple((32 - k) / 32 for k in range(16))
+
+
+def _range_grid(mn: np.ndarray, mx: np.ndarray, L: int):
+    """Grid spanning [mn, mx] (mn <= 0 <= mx): s = (mx - mn) / L, z = rint(-mn / s)."""
     s = _f(np.subtract(mx, mn, dtype=f32) / f32(L))
     zero_range = s == f32(0)
     s_safe = np.where(zero_range, f32(1), s).astype(f32)
     z = _f(np.rint(_f(np.negative(mn) / s_safe)) + f32(0))
     z = np.where(zero_range, f32(0), z).astype(f32)
     return s_safe, z
+
+
+def _group_range(yg: np.ndarray):
+    yg = _f(yg)
+    return np.minimum(yg.min(axis=1), f32(0)), np.maximum(yg.max(axis=1), f32(0))
+
+
+def fit_minmax(yg: np.ndarray, L: int):
+    """(scale, zero) per group; yg has one group per row."""
+    return _range_grid(*_group_range(yg), L)
+
+
+def fit_mse(yg: np.ndarray, L: int, return_error: bool = False):
+    """Clipping search: the candidate grid with the smallest squared error.
+
+    Candidate a spans (a * mn, a * mx); its error is sum_i (y_i - D_i)^2 with
+    each square and each partial sum rounded to float32 in element order.  A
+    later candidate replaces the best one only when strictly smaller."""
+    yg = _f(yg)
+    mn, mx = _group_range(yg)
+    best = None
+    for a in CLIP_RATIOS:
+        a = f32(a)
+        s, z = _range_grid(_f(a * mn), _f(a * mx), L)
+        d = _f(yg - dequantize(round_to_grid(yg, s, z, L), s, z))
+        d2 = _f(d * d)
+        e = np.zeros(yg.shape[0], f32)
+        for i in range(yg.shape[1]):
+            e = _f(e + d2[:, i])
+        if best is None:
+            best = [s, z, e]
+        else:
+            take = e < best[2]
+            best = [np.where(take, s, best[0]).astype(f32), np.where(take, z, best[1]).astype(f32),
+                    np.where(take, e, best[2]).astype(f32)]
+    return tuple(best) if return_error else (best[0], best[1])
 
 
 def fit_lsq(yg: np.ndarray, wg: np.ndarray, s_prev: np.ndarray, z_prev: np.ndarray, L: int):
@@ -183,7 +224,7 @@ def epilogue_step(W_acc: np.ndarray, V: np.ndarray, sigma: np.ndarray, rsig: np.
 
     Per element (i = input channel):
       t  = W~ + V~          y  = sigma_i t
-      grid (minmax | lsq | frozen) per group of `group` columns of one row
+      grid (minmax | lsq | mse | frozen) per group of `group` columns of one row
       q  = clamp(rint(y/s) + z, 0, L),  D = s (q - z),  D~ = D * rsig_i
       V~' = t - D~          P  = D~ - V~'   (in the operand encoding of `split`)
     Residual sums (float64 here; the kernels sum in float32, compared with a
@@ -204,6 +245,8 @@ def epilogue_step(W_acc: np.ndarray, V: np.ndarray, sigma: np.ndarray, rsig: np.
         wg = np.broadcast_to(_f(hdiag).reshape(d // group, group)[None],
                              (m, d // group, group)).reshape(-1, group)
         s, z = fit_lsq(yg, wg, sp, zp, L)
+    elif mode == "mse":
+        s, z = fit_mse(yg, L)
     elif mode == "frozen":
         s, z = sp, zp
     else:

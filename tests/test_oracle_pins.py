@@ -240,6 +240,79 @@ def test_minmax_grid_all_zero_group():
     np.testing.assert_array_equal(P.round_to_grid(y, s, z, 7), 0)
 
 
+def test_mse_clip_hand_example():
+    """2 bits, one group of 128: a zero, 126 ones and one outlier 3.2.  The
+    min/max grid (s = 3.2/3) misses every 1 by 1/15: error 126/225 = 0.56.  The
+    ratio 30/32 clips the range to [0, 3]: s = 1 puts every 1 on the grid
+    and costs only (3.2 - 3)^2 = 0.04 at the outlier, less than any other
+    ratio (31/32 leaves 126 * (1/30)^2 = 0.14 on the ones).  Mirrored, the
+    zero point moves to 3."""
+    y = np.ones((1, 128), np.float32)
+    y[0, 0], y[0, -1] = 0.0, 3.2
+    s, z, e = P.fit_mse(y, 3, return_error=True)
+    assert (s[0], z[0]) == (1.0, 0.0)
+    assert abs(e[0] - 0.04) < 1e-6
+    s_mm, _ = P.fit_minmax(y, 3)
+    assert abs(s_mm[0] - 3.2 / 3) < 1e-6
+    s, z = P.fit_mse(-y, 3)
+    assert (s[0], z[0]) == (1.0, 3.0)
+
+
+def test_mse_clip_all_zero_group():
+    y = np.zeros((2, 16), np.float32)
+    s, z = P.fit_mse(y, 7)
+    np.testing.assert_array_equal(s, 1.0)
+    np.testing.assert_array_equal(z, 0.0)
+
+
+def test_mse_clip_exact_grid_keeps_minmax():
+    """Points that fill a grid from level 0 to level L are reproduced exactly
+    by the min/max grid, so the search keeps it (later ratios tie or lose)."""
+    rng = np.random.default_rng(11)
+    L = 7
+    G, g = 30, 32
+    s_true = (2.0 ** -rng.integers(3, 9, G)).astype(np.float32)
+    z_true = rng.integers(1, L, G).astype(np.float32)
+    q = rng.integers(0, L + 1, (G, g)).astype(np.float32)
+    q[:, 0], q[:, 1] = 0, L
+    y = P.dequantize(q, s_true, z_true)
+    s, z, e = P.fit_mse(y, L, return_error=True)
+    np.testing.assert_array_equal(s, s_true)
+    np.testing.assert_array_equal(z, z_true)
+    np.testing.assert_array_equal(e, 0.0)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_mse_clip_search_against_float64(bits):
+    """Heavy-tailed groups: the chosen grid is never worse than min/max and
+    is, within float32 rounding of the error sums, the best of the clipped
+    grids, each evaluated here in float64 by brute force over its levels."""
+    rng = np.random.default_rng(100 + bits)
+    L = (1 << bits) - 1
+    G, g = 300, 64
+    y = (rng.standard_t(3, (G, g)) * 0.02).astype(np.float32)
+    s, z = P.fit_mse(y, L)
+    y64 = y.astype(np.float64)
+
+    def err64(sg, zg):
+        lev = sg[:, None] * (np.arange(L + 1)[None, :] - zg[:, None])
+        return (np.abs(y64[:, :, None] - lev[:, None, :]).min(axis=2) ** 2).sum(axis=1)
+
+    e_pick = err64(s.astype(np.float64), z.astype(np.float64))
+    mn = np.minimum(y64.min(axis=1), 0.0)
+    mx = np.maximum(y64.max(axis=1), 0.0)
+    e_all = []
+    for k in range(16):
+        a = 1.0 - k / 32.0
+        sk = (a * mx - a * mn) / L
+        zk = np.rint(-a * mn / sk)
+        e_all.append(err64(sk, zk))
+    e_all = np.array(e_all)
+    assert np.all(e_pick <= e_all[0] * (1 + 1e-5) + 1e-12)
+    assert np.all(e_pick <= e_all.min(axis=0) * (1 + 1e-4) + 1e-12)
+    assert np.mean(e_pick < e_all[0] * (1 - 1e-3)) > 0.5   # clipping pays on t(3) tails
+
+
 @pytest.mark.parametrize("bits", [2, 3, 4])
 def test_projection_is_nearest_grid_point(bits):
     """On a fixed grid the D-update rounds each entry to its nearest level
@@ -381,7 +454,7 @@ def test_diagonal_hessian_frozen_grid_gives_rtn():
         np.testing.assert_array_equal(res["codes"], c_rtn)
 
 
-@pytest.mark.parametrize("grid", ["minmax", "lsq", "frozen"])
+@pytest.mark.parametrize("grid", ["minmax", "lsq", "mse", "frozen"])
 def test_admm_converges_to_common_limit(grid):
     """Under rho_t = rho0 gamma^t the continuous and discrete iterates reach
     the same limit: once rho >> lambda_max(H~) the primal residual vanishes
