@@ -682,7 +682,7 @@ def main():
                     help="Sigma = I: the unscaled ablation (objective comparison)")
     ap.add_argument("--shard", action="store_true",
                     help="split ONE layer over the ranks (tokens and output rows; H all-reduced)")
-    ap.add_argument("--grid", default="lsq", choices=["lsq", "minmax", "frozen"])
+    ap.add_argument("--grid", default="lsq", choices=["lsq", "minmax", "mse", "frozen"])
     ap.add_argument("--split", default="auto", choices=["auto", "mixed", "3xtf32"],
                     help="split precision of the eigenbasis GEMMs (auto: mixed from d_in 2048)")
     ap.add_argument("--tokens", type=int, default=0,

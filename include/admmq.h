@@ -53,7 +53,12 @@ enum {
 enum {
   ADMMQ_GRID_MINMAX = 0, /* scale/zero from the group's min/max, 0 included    */
   ADMMQ_GRID_LSQ = 1,    /* weighted least-squares refit, weights diag(H)       */
-  ADMMQ_GRID_FROZEN = 2  /* keep the start grid (RTN grid of W_hat)             */
+  ADMMQ_GRID_FROZEN = 2, /* keep the start grid (RTN grid of W_hat)             */
+  ADMMQ_GRID_MSE = 3     /* MSE clipping search: the min/max grid of the range
+                            clipped by a = (32 - k) / 32, k < 16, whose float32
+                            squared error (summed in element order) is the
+                            first smallest (ADMM-Q technical summary,
+                            Methodology section 3: clipping heuristics)       */
 };
 
 enum { ADMMQ_DTYPE_F32 = 0, ADMMQ_DTYPE_BF16 = 1 };

@@ -16,8 +16,8 @@ import torch
 from .build import LIB
 
 OK = 0
-GRID_MINMAX, GRID_LSQ, GRID_FROZEN = 0, 1, 2
-GRID_MODES = {"minmax": GRID_MINMAX, "lsq": GRID_LSQ, "frozen": GRID_FROZEN}
+GRID_MINMAX, GRID_LSQ, GRID_FROZEN, GRID_MSE = 0, 1, 2, 3
+GRID_MODES = {"minmax": GRID_MINMAX, "lsq": GRID_LSQ, "frozen": GRID_FROZEN, "mse": GRID_MSE}
 SPLIT_MODES = {"auto": 0, "3xtf32": 1, "mixed": 2}
 DTYPE_F32, DTYPE_BF16 = 0, 1
 BUFFERS = ["sigma", "rsig", "hdiag", "lambda", "V", "C0", "P_hi", "P_lo", "T_hi", "T_lo",

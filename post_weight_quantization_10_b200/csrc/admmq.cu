@@ -650,7 +650,7 @@ int check_params(int d, int m, const admmq_params* p) {
     return ADMMQ_ERR_INVALID_ARG;
   if (p->bits < 1 || p->bits > 8 || p->iters < 0) return ADMMQ_ERR_INVALID_ARG;
   if (!(p->rho0 > 0.f) || !(p->gamma > 0.f) || !(p->lambda_rel >= 0.f)) return ADMMQ_ERR_INVALID_ARG;
-  if (p->grid_mode < ADMMQ_GRID_MINMAX || p->grid_mode > ADMMQ_GRID_FROZEN)
+  if (p->grid_mode < ADMMQ_GRID_MINMAX || p->grid_mode > ADMMQ_GRID_MSE)
     return ADMMQ_ERR_INVALID_ARG;
   if (p->split_mode < ADMMQ_SPLIT_AUTO || p->split_mode > ADMMQ_SPLIT_MIXED)
     return ADMMQ_ERR_INVALID_ARG;
@@ -1010,6 +1010,10 @@ int admmq_iterate(admmq_ctx* c, int t0, int count, uint8_t* codes, float* scale,
         e = launch_eig<EpiProject<GRID_LSQ, false>,
                        EpiProject<GRID_LSQ, true>>(c->mix, c->mT, c->mQ, g, p2, st);
         break;
+      case ADMMQ_GRID_MSE:
+        e = launch_eig<EpiProject<GRID_MSE, false>,
+                       EpiProject<GRID_MSE, true>>(c->mix, c->mT, c->mQ, g, p2, st);
+        break;
       default:
         e = launch_eig<EpiProject<GRID_FROZEN, false>,
                        EpiProject<GRID_FROZEN, true>>(c->mix, c->mT, c->mQ, g, p2, st);
@@ -1152,7 +1156,7 @@ int admmq_project(const float* wt, float* V, const float* sig, const float* rsig
   if (!wt || !V || !sig || !rsig || !hd || !codes || !scale || !zero || !p_hi || !p_lo || !resid)
     return ADMMQ_ERR_INVALID_ARG;
   if (d <= 0 || m <= 0 || d % 32 != 0 || !(g == 32 || g == 64 || g == 128) || d % g != 0 ||
-      bits < 1 || bits > 8 || mode < 0 || mode > 2 ||
+      bits < 1 || bits > 8 || mode < ADMMQ_GRID_MINMAX || mode > ADMMQ_GRID_MSE ||
       !(split == ADMMQ_SPLIT_3XTF32 || split == ADMMQ_SPLIT_MIXED))
     return ADMMQ_ERR_INVALID_ARG;
   if (!aligned32(V) || !aligned32(codes) || !aligned32(p_hi) || !aligned32(p_lo) ||
@@ -1174,6 +1178,8 @@ int admmq_project(const float* wt, float* V, const float* sig, const float* rsig
     PROJECT_CASE(GRID_MINMAX)
   } else if (mode == ADMMQ_GRID_LSQ) {
     PROJECT_CASE(GRID_LSQ)
+  } else if (mode == ADMMQ_GRID_MSE) {
+    PROJECT_CASE(GRID_MSE)
   } else {
     PROJECT_CASE(GRID_FROZEN)
   }

@@ -8,7 +8,10 @@
 
 namespace admmq {
 
-enum { GRID_MINMAX = 0, GRID_LSQ = 1, GRID_FROZEN = 2 };
+enum { GRID_MINMAX = 0, GRID_LSQ = 1, GRID_FROZEN = 2, GRID_MSE = 3 };
+
+// Clipping search of the MSE grid refresh: ratios (32 - k) / 32, k < 16.
+constexpr int kClipCandidates = 16;
 
 // ------------------------------------------------------------ small helpers
 
@@ -140,6 +143,69 @@ struct ProjRow {
   bool valid;
 };
 
+// Grid spanning [mn, mx] (mn <= 0 <= mx): s = (mx - mn) / L, z = rint(-mn / s);
+// an empty range gets s = 1, z = 0.
+__device__ __forceinline__ void range_grid(float mn, float mx, float Lf, float& s, float& z) {
+  s = __fdiv_rn(__fsub_rn(mx, mn), Lf);
+  if (s == 0.f) {
+    s = 1.f;
+    z = 0.f;
+  } else {
+    z = __fadd_rn(rintf(__fdiv_rn(-mn, s)), 0.f);
+  }
+}
+
+// MSE clipping search over one group: candidate k is the grid of the clipped
+// range (a mn, a mx), a = (32 - k) / 32; its error sum (y - D)^2 is accumulated
+// in element order with every product and sum rounded on its own; the first
+// smallest error wins.  The group is read once per 32-column chunk; the
+// candidates run in an outer loop over the chunk's y held in registers.
+template <class LoadW>
+__device__ __forceinline__ void mse_clip_grid(LoadW& loadw, const ProjRow& r, int g, float Lf,
+                                              float mn, float mx, float& s, float& z) {
+  float ce[kClipCandidates];
+#pragma unroll
+  for (int k = 0; k < kClipCandidates; ++k) ce[k] = 0.f;
+#pragma unroll 1
+  for (int c = 0; c < g; c += 32) {
+    float y[32];
+    loadw(c, y);
+#pragma unroll
+    for (int e = 0; e < 32; e += 8) {
+      float vv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (r.valid) ld_v8f(r.V + c + e, vv);
+      float ss[8];
+      load8_ro(r.sig + c + e, ss);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) y[e + j] = __fmul_rn(ss[j], __fadd_rn(y[e + j], vv[j]));
+    }
+#pragma unroll 1
+    for (int k = 0; k < kClipCandidates; ++k) {
+      const float a = __fmul_rn((float)(32 - k), 0.03125f);
+      float sk, zk;
+      range_grid(__fmul_rn(a, mn), __fmul_rn(a, mx), Lf, sk, zk);
+      float ek = ce[k];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float q = clampq(__fadd_rn(rintf(__fdiv_rn(y[j], sk)), zk), Lf);
+        const float dd = __fsub_rn(y[j], __fmul_rn(sk, __fsub_rn(q, zk)));
+        ek = __fadd_rn(ek, __fmul_rn(dd, dd));
+      }
+      ce[k] = ek;
+    }
+  }
+  float best = ce[0];
+  range_grid(mn, mx, Lf, s, z);
+#pragma unroll 1
+  for (int k = 1; k < kClipCandidates; ++k) {
+    if (ce[k] < best) {
+      best = ce[k];
+      const float a = __fmul_rn((float)(32 - k), 0.03125f);
+      range_grid(__fmul_rn(a, mn), __fmul_rn(a, mx), Lf, s, z);
+    }
+  }
+}
+
 template <int MODE, bool MIX, class LoadW>
 __device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, int g, int L,
                                               float& r2, float& s2) {
@@ -168,7 +234,7 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, i
         for (int k = 0; k < 8; ++k) {
           const float t = __fadd_rn(w[e + k], vv[k]);
           const float y = __fmul_rn(ss[k], t);
-          if (MODE == GRID_MINMAX) {
+          if (MODE == GRID_MINMAX || MODE == GRID_MSE) {
             mn = fminf(mn, y);
             mx = fmaxf(mx, y);
           } else {
@@ -185,13 +251,9 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, i
       }
     }
     if (MODE == GRID_MINMAX) {
-      s = __fdiv_rn(__fsub_rn(mx, mn), Lf);
-      if (s == 0.f) {
-        s = 1.f;
-        z = 0.f;
-      } else {
-        z = __fadd_rn(rintf(__fdiv_rn(-mn, s)), 0.f);
-      }
+      range_grid(mn, mx, Lf, s, z);
+    } else if (MODE == GRID_MSE) {
+      mse_clip_grid(loadw, r, g, Lf, mn, mx, s, z);
     } else {
       const float qm = __fdiv_rn(Sq, Sw);
       const float ym = __fdiv_rn(Sy, Sw);

@@ -85,7 +85,8 @@ def _solver(A, p, X, W, grid, split="auto"):
     return s
 
 
-@pytest.mark.parametrize("grid,split", [("lsq", "auto"), ("minmax", "auto"), ("lsq", "3xtf32")])
+@pytest.mark.parametrize("grid,split", [("lsq", "auto"), ("minmax", "auto"), ("mse", "auto"),
+                                        ("lsq", "3xtf32")])
 def test_full_size_teacher_forced(A, full_setup, grid, split):
     """RTN start bit-exact on the sampled rows; then, at sampled iterations,
     the oracle's state of those rows is loaded into the GPU's state and one

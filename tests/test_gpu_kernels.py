@@ -82,7 +82,7 @@ def _proj_inputs(m, d, g, bits, seed):
 
 
 @pytest.mark.parametrize("split", ["mixed", "3xtf32"])
-@pytest.mark.parametrize("grid", ["minmax", "lsq", "frozen"])
+@pytest.mark.parametrize("grid", ["minmax", "lsq", "mse", "frozen"])
 @pytest.mark.parametrize("bits,g,m,d", [(3, 128, 200, 384), (2, 64, 33, 128), (4, 32, 130, 96),
                                         (3, 64, 32, 64)])
 def test_projection_kernel_bitexact(A, grid, bits, g, m, d, split):

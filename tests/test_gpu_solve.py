@@ -145,8 +145,8 @@ def _load_state(s, e):
 
 
 TEACHER_CASES = [(n, g, "auto") for n in ("tiny", "ragged", "down_small")
-                 for g in ("minmax", "lsq", "frozen")] + \
-                [(n, g, "mixed") for n in ("tiny", "ragged") for g in ("minmax", "lsq")]
+                 for g in ("minmax", "lsq", "mse", "frozen")] + \
+                [(n, g, "mixed") for n in ("tiny", "ragged") for g in ("minmax", "lsq", "mse")]
 
 
 @pytest.mark.parametrize("name,grid,split", TEACHER_CASES)
@@ -187,7 +187,7 @@ def test_teacher_forced_iterations(A, name, grid, split):
 
 
 @pytest.mark.parametrize("name", ["tiny", "ragged", "down_small"])
-@pytest.mark.parametrize("grid", ["minmax", "lsq", "frozen"])
+@pytest.mark.parametrize("grid", ["minmax", "lsq", "mse", "frozen"])
 def test_free_running_solve(A, name, grid):
     """The whole solve, free-running on both sides.  The trajectory is
     sensitive to rounding at the 1e-7 level (the float64 oracle itself only

@@ -47,6 +47,9 @@ def test_argument_checks_without_gpu(lib):
     assert lib.admmq_workspace_bytes(256, 8, ctypes.byref(bad)) == 0
     bad = admmq.Params(bits=3, group=48).c()
     assert lib.admmq_workspace_bytes(96, 8, ctypes.byref(bad)) == 0
+    bad = admmq.Params(bits=3, group=128).c()
+    bad.grid_mode = 4
+    assert lib.admmq_workspace_bytes(256, 8, ctypes.byref(bad)) == 0
     assert lib.admmq_gram_workspace_bytes(100, 30) == 0
     assert lib.admmq_pack(None, 64, 4, 3, None, None) == -1
     assert lib.admmq_pack(ctypes.c_void_p(16), 48, 4, 3, ctypes.c_void_p(16), None) == -1
@@ -64,8 +67,8 @@ def test_alignment_checks_without_gpu(lib):
     device (the pointers below are never dereferenced)."""
     ok = [ctypes.c_void_p(0x10000 * (i + 1)) for i in range(12)]
     # wt V sig rsig hd | d m bits g mode split | codes scale zero p_hi p_lo resid stream
-    def call(ptrs, split=2):
-        return lib.admmq_project(*ptrs[:5], 256, 8, 3, 128, 0, split, *ptrs[5:11], None)
+    def call(ptrs, split=2, mode=0):
+        return lib.admmq_project(*ptrs[:5], 256, 8, 3, 128, mode, split, *ptrs[5:11], None)
     for k in (1, 5, 8, 9):  # V, codes, P_hi, P_lo off by 16 bytes
         bad = list(ok)
         bad[k] = ctypes.c_void_p(ok[k].value + 16)
@@ -75,6 +78,8 @@ def test_alignment_checks_without_gpu(lib):
     assert call(bad) == -1
     for split in (0, 3, -1):                   # the kernel needs a concrete split precision
         assert call(list(ok), split) == -1, split
+    for mode in (-1, 4):                       # grid modes are 0 (minmax) .. 3 (mse)
+        assert call(list(ok), mode=mode) == -1, mode
     assert lib.admmq_split_mode(None) == -1
     assert lib.admmq_debug_dump_wtilde(None, None) == -1
 
