@@ -131,7 +131,7 @@ class ClockSampler:
 class LayerRun:
     """Device-resident state of one layer solve through the C ABI binding."""
 
-    def __init__(self, A, p, grid, seed, device, split="auto", scaling=True):
+    def __init__(self, A, p, grid, seed, device, split="auto", scaling=True, schedule="fused"):
         self.A, self.p = A, p
         self.X = workloads.make_activations(p, seed=seed, device=device)
         self.W = workloads.make_weights(p, seed=seed, device=device, dtype=torch.bfloat16)
@@ -139,7 +139,8 @@ class LayerRun:
         self.gram_ws = torch.empty(A.gram_workspace_bytes(p.n, p.d_in), dtype=torch.uint8,
                                    device=device)
         prm = A.Params(bits=p.bits, group=p.group, iters=p.iters, rho0=p.rho0, gamma=p.gamma,
-                       lambda_rel=p.lambda_rel, grid=grid, split=split, scaling=scaling)
+                       lambda_rel=p.lambda_rel, grid=grid, split=split, scaling=scaling,
+                       schedule=schedule)
         self.s = A.Solver(p.d_in, p.d_out, prm, device=device)
         self.packed = torch.empty((p.d_out, p.d_in * p.bits // 32), dtype=torch.int32,
                                   device=device)
@@ -196,7 +197,7 @@ class ShardRun(LayerRun):
     (the layer's one exchange step), every rank eigendecomposes it and solves
     its rows."""
 
-    def __init__(self, A, p, grid, rank, world, device, split="auto"):
+    def __init__(self, A, p, grid, rank, world, device, split="auto", schedule="fused"):
         from post_weight_quantization_10_b200 import sharded
         X = workloads.make_activations(p, seed=0, device=device)
         W = workloads.make_weights(p, seed=0, device=device, dtype=torch.bfloat16)
@@ -211,7 +212,7 @@ class ShardRun(LayerRun):
         self.gram_ws = torch.empty(A.gram_workspace_bytes(self.X.shape[0], p.d_in),
                                    dtype=torch.uint8, device=device)
         prm = A.Params(bits=p.bits, group=p.group, iters=p.iters, rho0=p.rho0, gamma=p.gamma,
-                       lambda_rel=p.lambda_rel, grid=grid, split=split)
+                       lambda_rel=p.lambda_rel, grid=grid, split=split, schedule=schedule)
         self.s = A.Solver(p.d_in, self.W.shape[0], prm, device=device)
         self.packed = torch.empty((self.W.shape[0], p.d_in * p.bits // 32), dtype=torch.int32,
                                   device=device)
@@ -253,7 +254,7 @@ def run_sharded(args, rank, world, device):
     p = workloads.PRESETS[args.workload]
     if args.tokens:
         p = workloads.scaled(p, args.tokens, p.d_in, p.d_out)
-    run = ShardRun(A, p, args.grid, rank, world, device, split=args.split)
+    run = ShardRun(A, p, args.grid, rank, world, device, split=args.split, schedule=args.schedule)
     eigh_s = run.setup_eigh()
     for _ in range(args.warmup):
         run.step()
@@ -313,7 +314,8 @@ def run_decoder(args, rank, world, device):
     for label, p, seed in workloads.decoder_layer(bits):
         if args.tokens:
             p = workloads.scaled(p, args.tokens, p.d_in, p.d_out)
-        run = LayerRun(A, p, args.grid, seed=seed + 1000 * rank, device=device, split=args.split)
+        run = LayerRun(A, p, args.grid, seed=seed + 1000 * rank, device=device, split=args.split,
+                       schedule=args.schedule)
         eigh_s = run.setup_eigh()
         for _ in range(args.warmup):
             run.step()
@@ -363,7 +365,7 @@ def run_ours(args, rank, world, device):
     if args.tokens:
         p = workloads.scaled(p, args.tokens, p.d_in, p.d_out)
     run = LayerRun(A, p, args.grid, seed=rank, device=device, split=args.split,
-                   scaling=not args.no_scaling)
+                   scaling=not args.no_scaling, schedule=args.schedule)
     eigh_s = run.setup_eigh()
     for _ in range(args.warmup):
         run.step()
@@ -388,7 +390,7 @@ def run_ours(args, rank, world, device):
     launches = A.launch_count() - n0
     clk = clocks.stop()
     ms = t_start.elapsed_time(t_end)
-    gemm_ms, gemm_n = run.s.get_timing()
+    gemm_ms, gemm_n, gemm_iters = run.s.get_timing()
     run.s.set_timing(False)
     phase = np.zeros(4)
     for e in evs:
@@ -414,10 +416,22 @@ def run_ours(args, rank, world, device):
     flops_iter = 4.0 * d * d * m
     admm_ms = phase[2]
     gram_flops = float(n) * d * (d + 1)
-    # dominant kernel: GEMM 1 or GEMM 2 (same algorithmic flops, 2 d^2 m each)
-    k = 0 if gemm_ms[0] >= gemm_ms[1] else 1
-    avg_ms = gemm_ms[k] / max(gemm_n[k], 1)
-    achieved = 2.0 * d * d * m / (avg_ms / 1e3) / 1e12
+    if gemm_n[1] == 0:
+        # fused schedule: one launch runs GEMM 1 and GEMM 2 of every iteration
+        # of the solve (4 d^2 m flops per iteration)
+        kname = "admm_loop"
+        avg_ms = gemm_ms[0] / max(gemm_n[0], 1)
+        flops_launch = flops_iter * gemm_iters / max(gemm_n[0], 1)
+        per_launch = {"admm_loop": avg_ms, "iters_per_launch": gemm_iters / max(gemm_n[0], 1)}
+    else:
+        # dominant kernel: GEMM 1 or GEMM 2 (same algorithmic flops, 2 d^2 m each)
+        k = 0 if gemm_ms[0] >= gemm_ms[1] else 1
+        kname = ["gemm1_eigscale", "gemm2_project"][k]
+        avg_ms = gemm_ms[k] / max(gemm_n[k], 1)
+        flops_launch = 2.0 * d * d * m
+        per_launch = {"gemm1_eigscale": gemm_ms[0] / max(gemm_n[0], 1),
+                      "gemm2_project": gemm_ms[1] / max(gemm_n[1], 1)}
+    achieved = flops_launch / (avg_ms / 1e3) / 1e12
     # Tensor work per fp32-accurate product, in bf16-MMA units (dense tf32 runs
     # at half the bf16 rate, nominal 1.1 vs 2.25 PFLOP/s): 3xTF32 = three tf32
     # MMAs = 6; mixed split = one tf32 MMA (2) + one bf16 MMA over the doubled
@@ -443,7 +457,7 @@ def run_ours(args, rank, world, device):
                    "parallelism": f"independent layers x{world}",
                    "l2": "inputs larger than L2 (X is %.1f GiB)" % (n * d * 2 / 2**30),
                    "eigh": "one-time setup outside the step (eigh_s)",
-                   "split": split},
+                   "split": split, "schedule": args.schedule},
         "s_per_layer": ms_max / 1e3 / args.steps,
         "s_per_layer_with_eigh": ms_max / 1e3 / args.steps + eigh_s,
         "eigh_s": eigh_s,
@@ -452,11 +466,11 @@ def run_ours(args, rank, world, device):
         "admm_iters_per_s": T / (admm_ms / 1e3),
         "admm_tflops_fp32_accurate": flops_iter * T / (admm_ms / 1e3) / 1e12,
         "gram_tflops": gram_flops / (phase[0] / 1e3) / 1e12,
-        "gemm_ms_per_launch": [gemm_ms[0] / max(gemm_n[0], 1), gemm_ms[1] / max(gemm_n[1], 1)],
-        "roofline": {"kernel": ["gemm1_eigscale", "gemm2_project"][k], "bound": "tensor",
+        "ms_per_launch": per_launch,
+        "roofline": {"kernel": kname, "bound": "tensor",
                      "achieved": achieved, "peak": peak_split, "unit": "TFLOP/s",
                      "frac": achieved / peak_split,
-                     "traffic": measured_traffic(["gemm1_eigscale", "gemm2_project"][k]),
+                     "traffic": measured_traffic(kname),
                      "peak_note": "bf16 dense %s sustained %.1f TF/s / %d (bf16-MMA units of tensor "
                                   "work per fp32-accurate product, %s split)" % (
                                       pk["src"], pk["bf16_sust"], per_product, split)},
@@ -685,6 +699,9 @@ def main():
     ap.add_argument("--grid", default="lsq", choices=["lsq", "minmax", "mse", "frozen"])
     ap.add_argument("--split", default="auto", choices=["auto", "mixed", "3xtf32"],
                     help="split precision of the eigenbasis GEMMs (auto: mixed from d_in 2048)")
+    ap.add_argument("--schedule", default="fused", choices=["fused", "per_gemm"],
+                    help="fused: GEMM 1 and GEMM 2 of all iterations in one launch; "
+                         "per_gemm: two launches per iteration")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the calibration token count n (profiling captures only; "
                          "the eigenbasis GEMMs do not depend on n)")

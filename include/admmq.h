@@ -71,6 +71,16 @@ enum {
   ADMMQ_SPLIT_MIXED = 2   /* tf32 hi.hi + one bf16 product for hi.lo + lo.hi      */
 };
 
+/* How admmq_iterate launches the iterations.  Every step of an iteration acts
+ * on rows, so GEMM 1 and GEMM 2 of an iteration can run in one persistent
+ * launch whose GEMM-2 tiles wait until the row block of T they read is
+ * complete (the default: one tail instead of two per iteration); or GEMM 1
+ * and GEMM 2 are launched separately.  Both give the same bits. */
+enum {
+  ADMMQ_SCHEDULE_FUSED = 0,   /* GEMM 1 + GEMM 2 of an iteration in one launch */
+  ADMMQ_SCHEDULE_PER_GEMM = 1 /* two launches per iteration                   */
+};
+
 typedef struct admmq_params {
   int bits;         /* b: codes in [0, 2^b - 1]                                  */
   int group;        /* g: input channels per quantization group                 */
@@ -82,6 +92,7 @@ typedef struct admmq_params {
   int split_mode;   /* ADMMQ_SPLIT_*                                             */
   int no_scaling;   /* 1: Sigma = I, the unscaled ablation ([ADMM-Q] Methodology
                        section 2 reports what removing the scaling costs); 0 */
+  int schedule;     /* ADMMQ_SCHEDULE_*                                          */
 } admmq_params;
 
 typedef struct admmq_ctx admmq_ctx; /* opaque; host memory owned by the library */
@@ -182,7 +193,11 @@ int admmq_init(admmq_ctx* ctx, uint8_t* codes_dev, float* scale_dev, float* zero
  *   T  = diag(1/(Lambda+rho)) (C0' + rho Q^T (D~ - V~))          (GEMM 1)
  *   W~ = Q T;  D = grid projection of Sigma (W~ + V~);  V~ += W~ - D~  (GEMM 2
  *        with the projection, the dual update and residual sums fused)
- * codes/scale/zero are updated in place (they hold D).  t0 + count <= iters. */
+ * codes/scale/zero are updated in place (they hold D).  t0 + count <= iters.
+ * With ADMMQ_SCHEDULE_FUSED each iteration is one kernel launch.  Its waits for
+ * other units are bounded like the pipeline waits: one that gives up sets the
+ * kernel status word (ADMMQ_BUF_STATUS[0] = 1, "timed out") and the launch
+ * ends. */
 int admmq_iterate(admmq_ctx* ctx, int t0, int count, uint8_t* codes_dev, float* scale_dev,
                   float* zero_dev, void* stream);
 
@@ -243,9 +258,12 @@ int admmq_debug_dump_wtilde(admmq_ctx* ctx, float* wtilde_dev);
 /* Per-kernel timing with CUDA events recorded on the launch stream around
  * every GEMM launch of admmq_iterate.  enable != 0 clears and starts it.
  * admmq_get_timing returns the summed milliseconds and launch counts of
- * GEMM 1 (index 0) and GEMM 2 (index 1); it synchronises on the events. */
+ * GEMM 1 (index 0) and GEMM 2 (index 1), or, with ADMMQ_SCHEDULE_FUSED, of
+ * the fused launches (index 0; index 1 is zero); iters_timed (optional)
+ * receives the number of iterations those launches ran.  It synchronises on
+ * the events. */
 int admmq_set_timing(admmq_ctx* ctx, int enable);
-int admmq_get_timing(admmq_ctx* ctx, double ms[2], int launches[2]);
+int admmq_get_timing(admmq_ctx* ctx, double ms[2], int launches[2], int* iters_timed);
 
 /* Standalone projection kernel (the fused GEMM-2 epilogue reading W~ from
  * memory instead of tensor memory); same per-element float32 arithmetic.

@@ -19,6 +19,7 @@ OK = 0
 GRID_MINMAX, GRID_LSQ, GRID_FROZEN, GRID_MSE = 0, 1, 2, 3
 GRID_MODES = {"minmax": GRID_MINMAX, "lsq": GRID_LSQ, "frozen": GRID_FROZEN, "mse": GRID_MSE}
 SPLIT_MODES = {"auto": 0, "3xtf32": 1, "mixed": 2}
+SCHEDULES = {"fused": 0, "per_gemm": 1}
 DTYPE_F32, DTYPE_BF16 = 0, 1
 BUFFERS = ["sigma", "rsig", "hdiag", "lambda", "V", "C0", "P_hi", "P_lo", "T_hi", "T_lo",
            "E_hi", "E_lo", "Ht", "status"]
@@ -34,7 +35,8 @@ class _Params(ctypes.Structure):
     _fields_ = [("bits", ctypes.c_int), ("group", ctypes.c_int), ("iters", ctypes.c_int),
                 ("rho0", ctypes.c_float), ("gamma", ctypes.c_float),
                 ("lambda_rel", ctypes.c_float), ("grid_mode", ctypes.c_int),
-                ("split_mode", ctypes.c_int), ("no_scaling", ctypes.c_int)]
+                ("split_mode", ctypes.c_int), ("no_scaling", ctypes.c_int),
+                ("schedule", ctypes.c_int)]
 
 
 @dataclass
@@ -48,10 +50,12 @@ class Params:
     grid: str = "lsq"
     split: str = "auto"   # eigenbasis GEMM split precision: auto | 3xtf32 | mixed
     scaling: bool = True  # False: Sigma = I (the unscaled ablation)
+    schedule: str = "fused"  # fused: one launch per iterate call | per_gemm: two per iteration
 
     def c(self) -> _Params:
         return _Params(self.bits, self.group, self.iters, self.rho0, self.gamma, self.lambda_rel,
-                       GRID_MODES[self.grid], SPLIT_MODES[self.split], int(not self.scaling))
+                       GRID_MODES[self.grid], SPLIT_MODES[self.split], int(not self.scaling),
+                       SCHEDULES[self.schedule])
 
 
 _lib = None
@@ -104,7 +108,7 @@ def lib():
         "admmq_debug_dump_wtilde": (_i, [_vp, _vp]),
         "admmq_set_timing": (_i, [_vp, _i]),
         "admmq_get_timing": (_i, [_vp, ctypes.POINTER(ctypes.c_double),
-                                  ctypes.POINTER(ctypes.c_int)]),
+                                  ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
         "admmq_project": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp,
                                _vp, _vp, _vp, _vp]),
         "admmq_split_mode": (_i, [_vp]),
@@ -238,6 +242,11 @@ class Solver:
                                  _ptr(self.resid), _ptr(self.objective), _stream(stream)),
                "admmq_solve")
 
+    def kernel_status(self) -> int:
+        """The kernels' status word (0 = ok, 1 = a bounded wait gave up);
+        synchronises with the device."""
+        return int(self.buffer("status")[0].item())
+
     def buffer(self, name: str) -> torch.Tensor:
         """A torch view of a workspace buffer (see include/admmq.h for layouts)."""
         which = BUFFERS.index(name)
@@ -277,10 +286,13 @@ class Solver:
         _check(lib().admmq_set_timing(self._ctx, int(enable)), "admmq_set_timing")
 
     def get_timing(self):
+        """([ms GEMM 1, ms GEMM 2], [launches, launches], iterations timed); with
+        the fused schedule index 0 is the fused launches and index 1 is zero."""
         ms = (ctypes.c_double * 2)()
         n = (ctypes.c_int * 2)()
-        _check(lib().admmq_get_timing(self._ctx, ms, n), "admmq_get_timing")
-        return [ms[0], ms[1]], [n[0], n[1]]
+        iters = ctypes.c_int(0)
+        _check(lib().admmq_get_timing(self._ctx, ms, n, ctypes.byref(iters)), "admmq_get_timing")
+        return [ms[0], ms[1]], [n[0], n[1]], iters.value
 
 
 # --------------------------------------------------------------- pack etc.

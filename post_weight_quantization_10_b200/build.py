@@ -16,7 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libadmmq.so")
 SOURCES = ["admmq.cu"]
-HEADERS = ["ptx.cuh", "gemm.cuh", "kernels.cuh", "gptq.cuh"]
+HEADERS = ["ptx.cuh", "gemm.cuh", "kernels.cuh", "admm_loop.cuh", "gptq.cuh"]
 INCLUDE = os.path.join(os.path.dirname(HERE), "include", "admmq.h")
 
 

@@ -17,12 +17,16 @@
 
 #include "../../include/admmq.h"
 #include "kernels.cuh"
+#include "admm_loop.cuh"
 
 using namespace admmq;
 
 namespace {
 
 constexpr int kBM = 128;
+// Iterations per launch of the fused schedule (one: measured fastest under
+// the power cap, see admm_loop.cuh).
+constexpr int kFusedIters = 1;
 unsigned long long g_launches = 0;  // kernels launched by this library
 inline void count_launch() { __atomic_fetch_add(&g_launches, 1ull, __ATOMIC_RELAXED); }
 // X^T X: bf16, both operands MN-major (X is token-major).
@@ -476,24 +480,34 @@ GemmGeom make_geom(int M, int N, long long K, int BN, int BK, int splits, bool t
   return g;
 }
 
-template <class Cfg, class Epi>
-cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0,
-                        const CUtensorMap& b1, const GemmGeom& g, const typename Epi::Params& ep,
-                        cudaStream_t st) {
-  auto kern = k_gemm<Cfg, Epi>;
+// Launches k_gemm<Cfg, Work> over `units` work units: one CTA per SM, or one
+// pair of CTAs per two SMs.  A policy whose units wait on earlier units of the
+// same launch needs every CTA of the launch resident at once, so its grid is
+// capped by the occupancy query.
+template <class Cfg, class Work>
+cudaError_t launch_work(const typename Work::Args& args, int units, cudaStream_t st) {
+  auto kern = k_gemm<Cfg, Work>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
   if (e != cudaSuccess) return e;
-  if (g.units <= 0) return cudaSuccess;
+  if (units <= 0) return cudaSuccess;
   if (!Cfg::PAIR) {
-    const int grid = g.units < num_sms() ? g.units : num_sms();
+    int grid = num_sms();
+    if (Work::SIGNALS) {
+      int per_sm = 0;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Cfg::THREADS, Cfg::SMEM);
+      if (e != cudaSuccess) return e;
+      if (per_sm < 1) return cudaErrorInvalidConfiguration;
+      grid = per_sm * num_sms();
+    }
+    if (units < grid) grid = units;
     count_launch();
-    kern<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(a0, a1, b0, b1, g, ep);
+    kern<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(args);
     return cudaGetLastError();
   }
   // CTA pairs: clusters of two, one work unit per cluster at a time
-  const int pairs = num_sms() / 2;
+  int pairs = num_sms() / 2;
   cudaLaunchConfig_t lc = {};
-  lc.gridDim = dim3(2 * (g.units < pairs ? g.units : pairs));
+  lc.gridDim = dim3(2 * pairs);
   lc.blockDim = dim3(Cfg::THREADS);
   lc.dynamicSmemBytes = Cfg::SMEM;
   lc.stream = st;
@@ -504,10 +518,32 @@ cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
   attr[0].val.clusterDim.z = 1;
   lc.attrs = attr;
   lc.numAttrs = 1;
+  if (Work::SIGNALS) {
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, kern, &lc);
+    if (e != cudaSuccess) return e;
+    if (clusters < 1) return cudaErrorInvalidConfiguration;
+    if (clusters < pairs) pairs = clusters;
+  }
+  lc.gridDim = dim3(2 * (units < pairs ? units : pairs));
   count_launch();
-  e = cudaLaunchKernelEx(&lc, kern, a0, a1, b0, b1, g, ep);
+  e = cudaLaunchKernelEx(&lc, kern, args);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+template <class Cfg, class Epi>
+cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0,
+                        const CUtensorMap& b1, const GemmGeom& g, const typename Epi::Params& ep,
+                        cudaStream_t st) {
+  typename OneGemm<Epi>::Args x;
+  x.a[0] = a0;
+  x.a[1] = a1;
+  x.b[0] = b0;
+  x.b[1] = b1;
+  x.g = g;
+  x.ep = ep;
+  return launch_work<Cfg, OneGemm<Epi>>(x, g.units, st);
 }
 
 // An eigenbasis GEMM (A and B operand maps, plane 0 and 1) with the split
@@ -585,6 +621,9 @@ struct admmq_ctx {
   float *C0, *V;                               // [m][d]
   float* resid_part;    // [iters][tiles][4][2]
   float* obj_part;      // [tiles][4]
+  float* rho_tab;       // [iters] rho_t, as the host computes it
+  int* ready;           // [2][unit rows] ready counters of the fused schedule
+  int ready_base;       // iterations counted in `ready` since admmq_init zeroed it
   int tiles_eig;
   const void* W_hat;
   int w_dtype;
@@ -592,7 +631,12 @@ struct admmq_ctx {
   cusolverDnHandle_t solver;
   CUtensorMap mWt[2], mP[2], mT[2], mE[2], mQ[2];
   bool timing;
-  std::vector<cudaEvent_t> ev;   // triples per iteration
+  struct TimingRec {
+    cudaEvent_t a, b, c;  // GEMM 1 = a..b, GEMM 2 = b..c; fused: a..b, c unused
+    bool fused;
+    int iters;
+  };
+  std::vector<TimingRec> ev;
   bool prepared, eig_done, inited;
 };
 
@@ -601,7 +645,7 @@ namespace {
 struct Layout {
   size_t status, lam64, sig64, hdiag, sigma, rsig, lam32, Ht, evals, work, devinfo;
   size_t E_hi, E_lo, Q_hi, Q_lo, Wt_hi, Wt_lo, P_hi, P_lo, T_hi, T_lo, C0, V;
-  size_t resid_part, obj_part, total;
+  size_t resid_part, obj_part, rho_tab, ready, total;
 };
 
 Layout make_layout(int d, int m, int iters, int lwork) {
@@ -639,8 +683,24 @@ Layout make_layout(int d, int m, int iters, int lwork) {
   L.V = take(4 * md);
   L.resid_part = take(4 * (size_t)(iters > 0 ? iters : 1) * tiles * 8);
   L.obj_part = take(4 * (size_t)tiles * 4);
+  L.rho_tab = take(4 * (size_t)(iters > 0 ? iters : 1));
+  L.ready = take(4 * 2 * (size_t)cdiv(m, 2 * kBM));
   L.total = o;
   return L;
+}
+
+void destroy_events(admmq_ctx* c) {
+  for (auto& r : c->ev) {
+    if (r.a) cudaEventDestroy(r.a);
+    if (r.b) cudaEventDestroy(r.b);
+    if (r.c) cudaEventDestroy(r.c);
+  }
+  c->ev.clear();
+}
+
+// rho_t = rho0 gamma^t, evaluated in double and rounded once to float.
+float rho_at(const admmq_params& p, int t) {
+  return (float)((double)p.rho0 * pow((double)p.gamma, (double)t));
 }
 
 int check_params(int d, int m, const admmq_params* p) {
@@ -655,6 +715,8 @@ int check_params(int d, int m, const admmq_params* p) {
   if (p->split_mode < ADMMQ_SPLIT_AUTO || p->split_mode > ADMMQ_SPLIT_MIXED)
     return ADMMQ_ERR_INVALID_ARG;
   if (p->no_scaling != 0 && p->no_scaling != 1) return ADMMQ_ERR_INVALID_ARG;
+  if (p->schedule != ADMMQ_SCHEDULE_FUSED && p->schedule != ADMMQ_SCHEDULE_PER_GEMM)
+    return ADMMQ_ERR_INVALID_ARG;
   return ADMMQ_OK;
 }
 
@@ -729,6 +791,41 @@ GptqLayout gptq_layout(int d, int m, int block, int lwork) {
   do {                                             \
     if ((x) != cudaSuccess) return ADMMQ_ERR_CUDA; \
   } while (0)
+
+// GEMM 1 and GEMM 2 of iterations t0 .. t0+count-1 in one launch.
+template <class Cfg, class E1, class E2>
+cudaError_t launch_admm_loop(const admmq_ctx* c, const GemmGeom& g, const TUpdateParams& p1,
+                             const ProjParams& p2, int t0, int count, cudaStream_t st) {
+  using W = AdmmLoop<E1, E2>;
+  typename W::Args x;
+  for (int p = 0; p < 2; ++p) {
+    x.a[0][p] = c->mP[p];
+    x.b[0][p] = c->mE[p];
+    x.a[1][p] = c->mT[p];
+    x.b[1][p] = c->mQ[p];
+  }
+  x.g = g;
+  x.p1 = p1;
+  x.p2 = p2;
+  x.rho = c->rho_tab;
+  x.part0 = c->resid_part;
+  x.part_stride = (long long)c->tiles_eig * 8;
+  x.ready = c->ready;
+  x.base = c->ready_base;
+  x.ctas = Cfg::PAIR ? 2 : 1;
+  x.t0 = t0;
+  x.count = count;
+  return launch_work<Cfg, W>(x, count * 2 * g.units, st);
+}
+
+template <int MODE>
+cudaError_t launch_admm_loop_split(const admmq_ctx* c, const GemmGeom& g, const TUpdateParams& p1,
+                                   const ProjParams& p2, int t0, int count, cudaStream_t st) {
+  return c->mix ? launch_admm_loop<EigCfg, EpiTUpdate<true>, EpiProject<MODE, true>>(c, g, p1, p2, t0,
+                                                                                     count, st)
+                : launch_admm_loop<EigCfg3, EpiTUpdate<false>, EpiProject<MODE, false>>(c, g, p1, p2,
+                                                                                       t0, count, st);
+}
 
 }  // namespace
 
@@ -845,6 +942,8 @@ int admmq_create(admmq_ctx** out, int d, int m, const admmq_params* p, void* ws,
   c->V = (float*)(b + L.V);
   c->resid_part = (float*)(b + L.resid_part);
   c->obj_part = (float*)(b + L.obj_part);
+  c->rho_tab = (float*)(b + L.rho_tab);
+  c->ready = (int*)(b + L.ready);
   c->tiles_eig = eig_tiles(m, d);
   bool ok = true;
   ok &= make_map(&c->mWt[0], c->Wt_hi, d, m, kBM, true) && make_map(&c->mWt[1], c->Wt_lo, c->mix ? 2 * (uint64_t)d : (uint64_t)d, m, kBM, !c->mix);
@@ -864,7 +963,7 @@ int admmq_create(admmq_ctx** out, int d, int m, const admmq_params* p, void* ws,
 
 void admmq_destroy(admmq_ctx* c) {
   if (!c) return;
-  for (auto e : c->ev) cudaEventDestroy(e);
+  destroy_events(c);
   if (c->solver) cusolverDnDestroy(c->solver);
   delete c;
 }
@@ -955,6 +1054,13 @@ int admmq_init(admmq_ctx* c, uint8_t* codes, float* scale, float* zero, void* st
         (const __nv_bfloat16*)c->W_hat, c->rsig, m, d, c->p.group, c->L, codes, scale, zero,
         c->V, c->P_hi, c->P_lo, c->mix);
   CK(cudaGetLastError());
+  if (c->p.iters > 0) {
+    std::vector<float> rho(c->p.iters);
+    for (int t = 0; t < c->p.iters; ++t) rho[t] = rho_at(c->p, t);
+    CK(cudaMemcpyAsync(c->rho_tab, rho.data(), sizeof(float) * rho.size(), cudaMemcpyHostToDevice, st));
+  }
+  CK(cudaMemsetAsync(c->ready, 0, sizeof(int) * 2 * cdiv(m, 2 * kBM), st));
+  c->ready_base = 0;
   c->inited = true;
   return ADMMQ_OK;
 }
@@ -964,42 +1070,76 @@ int admmq_iterate(admmq_ctx* c, int t0, int count, uint8_t* codes, float* scale,
   if (!c || !c->inited || !codes || !scale || !zero) return ADMMQ_ERR_INVALID_ARG;
   if (!aligned32(codes)) return ADMMQ_ERR_INVALID_ARG;
   if (t0 < 0 || count < 0 || t0 + count > c->p.iters) return ADMMQ_ERR_INVALID_ARG;
+  if (count == 0) return ADMMQ_OK;
   cudaStream_t st = (cudaStream_t)stream;
   const int d = c->d, m = c->m;
   GemmGeom g = make_geom(m, d, d, EigCfg::BN, EigCfg::BK, 1, false, c->status, EigCfg::UNIT_M);
-  for (int t = t0; t < t0 + count; ++t) {
-    const float rho = (float)((double)c->p.rho0 * pow((double)c->p.gamma, (double)t));
-    cudaEvent_t e0 = nullptr, e1 = nullptr, e2 = nullptr;
-    if (c->timing) {
-      for (int k = 0; k < 3; ++k) {
-        cudaEvent_t e;
-        CK(cudaEventCreate(&e));
-        c->ev.push_back(e);
+  TUpdateParams p1{c->C0, c->lam32, c->T_hi, c->T_lo, 0.f, d};
+  ProjParams p2;
+  p2.V = c->V;
+  p2.codes = codes;
+  p2.scale = scale;
+  p2.zero = zero;
+  p2.p_hi = c->P_hi;
+  p2.p_lo = c->P_lo;
+  p2.sig = c->sigma;
+  p2.rsig = c->rsig;
+  p2.hd = c->hdiag;
+  p2.part = nullptr;
+  p2.wdump = c->wdump;
+  p2.ld = d;
+  p2.group = c->p.group;
+  p2.L = c->L;
+  auto new_event = [&](cudaEvent_t& e) -> int {
+    CK(cudaEventCreate(&e));
+    return ADMMQ_OK;
+  };
+  if (c->p.schedule == ADMMQ_SCHEDULE_FUSED) {
+    for (int t = t0; t < t0 + count; t += kFusedIters) {
+      const int n = t0 + count - t < kFusedIters ? t0 + count - t : kFusedIters;
+      admmq_ctx::TimingRec rec{nullptr, nullptr, nullptr, true, n};
+      if (c->timing) {
+        int rc = new_event(rec.a);
+        if (!rc) rc = new_event(rec.b);
+        if (rc) return rc;
+        c->ev.push_back(rec);
+        CK(cudaEventRecord(rec.a, st));
       }
-      e0 = c->ev[c->ev.size() - 3];
-      e1 = c->ev[c->ev.size() - 2];
-      e2 = c->ev[c->ev.size() - 1];
-      CK(cudaEventRecord(e0, st));
+      cudaError_t e;
+      switch (c->p.grid_mode) {
+        case ADMMQ_GRID_MINMAX:
+          e = launch_admm_loop_split<GRID_MINMAX>(c, g, p1, p2, t, n, st);
+          break;
+        case ADMMQ_GRID_LSQ:
+          e = launch_admm_loop_split<GRID_LSQ>(c, g, p1, p2, t, n, st);
+          break;
+        case ADMMQ_GRID_MSE:
+          e = launch_admm_loop_split<GRID_MSE>(c, g, p1, p2, t, n, st);
+          break;
+        default:
+          e = launch_admm_loop_split<GRID_FROZEN>(c, g, p1, p2, t, n, st);
+          break;
+      }
+      CK(e);
+      c->ready_base += n;
+      if (c->timing) CK(cudaEventRecord(rec.b, st));
     }
-    TUpdateParams p1{c->C0, c->lam32, c->T_hi, c->T_lo, rho, d};
-    CK((launch_eig<EpiTUpdate<false>, EpiTUpdate<true>>(c->mix, c->mP, c->mE,
-                                                                                g, p1, st)));
-    if (c->timing) CK(cudaEventRecord(e1, st));
-    ProjParams p2;
-    p2.V = c->V;
-    p2.codes = codes;
-    p2.scale = scale;
-    p2.zero = zero;
-    p2.p_hi = c->P_hi;
-    p2.p_lo = c->P_lo;
-    p2.sig = c->sigma;
-    p2.rsig = c->rsig;
-    p2.hd = c->hdiag;
+    return ADMMQ_OK;
+  }
+  for (int t = t0; t < t0 + count; ++t) {
+    admmq_ctx::TimingRec rec{nullptr, nullptr, nullptr, false, 1};
+    if (c->timing) {
+      int rc = new_event(rec.a);
+      if (!rc) rc = new_event(rec.b);
+      if (!rc) rc = new_event(rec.c);
+      if (rc) return rc;
+      c->ev.push_back(rec);
+      CK(cudaEventRecord(rec.a, st));
+    }
+    p1.rho = rho_at(c->p, t);
+    CK((launch_eig<EpiTUpdate<false>, EpiTUpdate<true>>(c->mix, c->mP, c->mE, g, p1, st)));
+    if (c->timing) CK(cudaEventRecord(rec.b, st));
     p2.part = c->resid_part + (size_t)t * c->tiles_eig * 8;
-    p2.wdump = c->wdump;
-    p2.ld = d;
-    p2.group = c->p.group;
-    p2.L = c->L;
     cudaError_t e;
     switch (c->p.grid_mode) {
       case ADMMQ_GRID_MINMAX:
@@ -1020,7 +1160,7 @@ int admmq_iterate(admmq_ctx* c, int t0, int count, uint8_t* codes, float* scale,
         break;
     }
     CK(e);
-    if (c->timing) CK(cudaEventRecord(e2, st));
+    if (c->timing) CK(cudaEventRecord(rec.c, st));
   }
   return ADMMQ_OK;
 }
@@ -1126,26 +1266,30 @@ int admmq_debug_dump_wtilde(admmq_ctx* c, float* wtilde) {
 
 int admmq_set_timing(admmq_ctx* c, int enable) {
   if (!c) return ADMMQ_ERR_INVALID_ARG;
-  for (auto e : c->ev) cudaEventDestroy(e);
-  c->ev.clear();
+  destroy_events(c);
   c->timing = enable != 0;
   return ADMMQ_OK;
 }
 
-int admmq_get_timing(admmq_ctx* c, double ms[2], int launches[2]) {
+int admmq_get_timing(admmq_ctx* c, double ms[2], int launches[2], int* iters_timed) {
   if (!c || !ms || !launches) return ADMMQ_ERR_INVALID_ARG;
   ms[0] = ms[1] = 0.0;
   launches[0] = launches[1] = 0;
-  for (size_t i = 0; i + 2 < c->ev.size(); i += 3) {
+  int iters = 0;
+  for (const auto& r : c->ev) {
     float a = 0.f, b = 0.f;
-    CK(cudaEventSynchronize(c->ev[i + 2]));
-    CK(cudaEventElapsedTime(&a, c->ev[i], c->ev[i + 1]));
-    CK(cudaEventElapsedTime(&b, c->ev[i + 1], c->ev[i + 2]));
+    CK(cudaEventSynchronize(r.fused ? r.b : r.c));
+    CK(cudaEventElapsedTime(&a, r.a, r.b));
     ms[0] += a;
-    ms[1] += b;
     launches[0] += 1;
-    launches[1] += 1;
+    if (!r.fused) {
+      CK(cudaEventElapsedTime(&b, r.b, r.c));
+      ms[1] += b;
+      launches[1] += 1;
+    }
+    iters += r.iters;
   }
+  if (iters_timed) *iters_timed = iters;
   return ADMMQ_OK;
 }
 

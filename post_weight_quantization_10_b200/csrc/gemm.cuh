@@ -38,8 +38,12 @@
 // leader (rank 0) issues the MMAs and commits to the barriers of both CTAs;
 // both CTAs' TMA loads count on the leader's stage barrier; consumers release
 // ring slots to the leader with remote arrivals.
-// Work units (tile, k-split) are dealt to CTAs (or pairs) round-robin; every
-// wait on a barrier is bounded (see ptx.cuh).
+// Work units are dealt to CTAs (or pairs) round-robin in index order.  What a
+// unit is comes from the Work policy: OneGemm (below) runs the (tile, k-split)
+// units of one GEMM with one epilogue; a policy may also chain several GEMMs
+// in one launch, with units whose operands are produced by earlier units of
+// the same launch (ready counters, see ptx.cuh: wait_counter).  Every wait is
+// bounded.
 #pragma once
 #include "ptx.cuh"
 
@@ -81,7 +85,9 @@ struct GemmCfg {
   static constexpr int RING = 2;                 // 256-column chunk slots in tensor memory
   static constexpr int TMEM_COLS = RING * BN;    // 512
   static constexpr int THREADS = 320;
-  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 2 * RING + 1) + 16;
+  // mbarriers, then tensor-memory address, abort flag, 2 spare words and the
+  // four unit-completion counters of the consumer warps
+  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 2 * RING + 1) + 32;
   // arrivals that release a ring slot: every consumer thread of the CTA, or
   // one per consumer warp of both CTAs of a pair
   static constexpr int SLOT_ARRIVALS = PAIR ? 16 : 256;
@@ -126,12 +132,55 @@ __device__ __forceinline__ void decode_unit(const GemmGeom& g, int u, int& tm, i
   kb1 = (int)(((long long)(split + 1) * g.kblocks) / g.splits);
 }
 
-template <class Cfg, class Epi>
+// One work unit: which GEMM of the launch (phase), which iteration (t), the
+// output tile and the k-block range.
+struct Unit {
+  int phase, t, tm, tn, split, kb0, kb1;
+};
+
+// Work policy of a plain GEMM: the (tile, k-split) units of one geometry, one
+// pair of operand maps per operand (planes 0 and 1), one epilogue.
+template <class Epi>
+struct OneGemm {
+  struct Args {
+    CUtensorMap a[2], b[2];
+    GemmGeom g;
+    typename Epi::Params ep;
+  };
+  static constexpr bool SIGNALS = false;
+  __device__ static int units(const Args& x) { return x.g.units; }
+  template <class Cfg>
+  __device__ static void decode(const Args& x, int u, Unit& w) {
+    w.phase = 0;
+    w.t = 0;
+    decode_unit<Cfg::BM, Cfg::BN>(x.g, u, w.tm, w.tn, w.split, w.kb0, w.kb1);
+  }
+  __device__ static const CUtensorMap* map_a(const Args& x, const Unit&, int p) { return &x.a[p]; }
+  __device__ static const CUtensorMap* map_b(const Args& x, const Unit&, int p) { return &x.b[p]; }
+  __device__ static void prefetch(const Args& x, int npl) {
+    for (int p = 0; p < npl; ++p) {
+      prefetch_tmap(&x.a[p]);
+      prefetch_tmap(&x.b[p]);
+    }
+  }
+  __device__ static bool ready(const Args&, const Unit&, volatile int*) { return true; }
+  __device__ static bool from_tmem(const Unit&) { return Epi::FROM_TMEM; }
+  __device__ static void epi_regs(const Args& x, const Unit& w, const float (&acc)[128], int tile_m,
+                                  int rit, int col0) {
+    if constexpr (!Epi::FROM_TMEM) Epi::apply_regs(x.ep, x.g, acc, tile_m, w.tn, w.split, rit, col0);
+  }
+  __device__ static void epi_tmem(const Args& x, const Unit&, uint32_t ta, int tile_m, int rit,
+                                  int col0) {
+    if constexpr (Epi::FROM_TMEM) Epi::apply_tmem(x.ep, x.g, ta, tile_m, rit, col0);
+  }
+  __device__ static int* done_counter(const Args&, const Unit&) { return nullptr; }
+};
+
+template <class Cfg, class Work>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
-    k_gemm(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ CUtensorMap tA1,
-           const __grid_constant__ CUtensorMap tB0, const __grid_constant__ CUtensorMap tB1,
-           const GemmGeom g, const typename Epi::Params ep) {
+    k_gemm(const __grid_constant__ typename Work::Args args) {
   constexpr int BM = Cfg::BM, BN = Cfg::BN, STAGES = Cfg::STAGES, NPL = Cfg::NPL, KC = Cfg::KC;
+  const GemmGeom& g = args.g;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -145,6 +194,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   uint64_t* drain = rempty + R;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* epi_count = reinterpret_cast<int*>(tmem_slot + 4);  // [4], by unit sequence number & 3
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // CTA pairs: rank in the cluster (0 = leader, issues the MMAs); work units
@@ -152,6 +202,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   const uint32_t rank = Cfg::PAIR ? cluster_rank() : 0u;
   const int unit0 = Cfg::PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int unit_step = Cfg::PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  const int nunits = Work::units(args);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -164,16 +215,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     }
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
+    for (int k = 0; k < 4; ++k) epi_count[k] = 0;
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tA0);
-    prefetch_tmap(&tB0);
-    if (NPL == 2) {
-      prefetch_tmap(&tA1);
-      prefetch_tmap(&tB1);
-    }
-  }
+  if (warp == 0 && lane == 0) Work::prefetch(args, NPL);
   if (warp == 1) {
     if (Cfg::PAIR)
       tmem_alloc_pair(smem_u32(tmem_slot), Cfg::TMEM_COLS);
@@ -189,16 +234,19 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const CUtensorMap* mapA[2] = {&tA0, &tA1};
-      const CUtensorMap* mapB[2] = {&tB0, &tB1};
       int it = 0;
       bool ok = true;
-      for (int u = unit0; u < g.units && ok; u += unit_step) {
-        int tm, tn, split, kb0, kb1;
-        decode_unit<BM, BN>(g, u, tm, tn, split, kb0, kb1);
-        const int a_row = tm * Cfg::UNIT_M + (int)rank * BM;        // this CTA's A rows
-        const int b_row = tn * BN + (int)rank * Cfg::B_ROWS;        // this CTA's B rows
-        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+      for (int u = unit0; u < nunits && ok; u += unit_step) {
+        Unit w;
+        Work::template decode<Cfg>(args, u, w);
+        // operands written earlier in this launch are published first
+        if (!Work::ready(args, w, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const int a_row = w.tm * Cfg::UNIT_M + (int)rank * BM;        // this CTA's A rows
+        const int b_row = w.tn * BN + (int)rank * Cfg::B_ROWS;        // this CTA's B rows
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
           if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, abort_flag, g.status)) {
@@ -219,32 +267,34 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 #pragma unroll
           for (int p = 0; p < NPL; ++p) {
             const uint32_t dA = st + p * Cfg::A_PLANE;
+            const CUtensorMap* ma = Work::map_a(args, w, p);
             if (!Cfg::A_MN) {
               // a mixed correction plane holds two bf16 per K-element
               const int xa = (Cfg::KIND == KIND_MIX && p == 1) ? 2 * k0 : k0;
               if (Cfg::PAIR)
-                tma_load_2d_pair(dA, mapA[p], xa, a_row, fb);
+                tma_load_2d_pair(dA, ma, xa, a_row, fb);
               else
-                tma_load_2d(dA, mapA[p], xa, a_row, fb);
+                tma_load_2d(dA, ma, xa, a_row, fb);
             } else {
 #pragma unroll
               for (int b = 0; b < BM / (128 / Cfg::ELEM); ++b)
-                tma_load_2d(dA + b * Cfg::BK * 128, mapA[p], a_row + (128 / Cfg::ELEM) * b, k0, fb);
+                tma_load_2d(dA + b * Cfg::BK * 128, ma, a_row + (128 / Cfg::ELEM) * b, k0, fb);
             }
           }
 #pragma unroll
           for (int p = 0; p < NPL; ++p) {
             const uint32_t dB = st + NPL * Cfg::A_PLANE + p * Cfg::B_PLANE;
+            const CUtensorMap* mb = Work::map_b(args, w, p);
             if (!Cfg::B_MN) {
               const int xb = (Cfg::KIND == KIND_MIX && p == 1) ? 2 * k0 : k0;
               if (Cfg::PAIR)
-                tma_load_2d_pair(dB, mapB[p], xb, b_row, fb);
+                tma_load_2d_pair(dB, mb, xb, b_row, fb);
               else
-                tma_load_2d(dB, mapB[p], xb, b_row, fb);
+                tma_load_2d(dB, mb, xb, b_row, fb);
             } else {
 #pragma unroll
               for (int b = 0; b < BN / (128 / Cfg::ELEM); ++b)
-                tma_load_2d(dB + b * Cfg::BK * 128, mapB[p], tn * BN + (128 / Cfg::ELEM) * b, k0, fb);
+                tma_load_2d(dB + b * Cfg::BK * 128, mb, w.tn * BN + (128 / Cfg::ELEM) * b, k0, fb);
             }
           }
         }
@@ -292,9 +342,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       int it = 0;
       uint32_t q = 0;  // chunks issued: chunk q goes to slot q % R, use q / R of it
       bool ok = true;
-      for (int u = unit0; u < g.units && ok; u += unit_step) {
-        int tm, tn, split, kb0, kb1;
-        decode_unit<BM, BN>(g, u, tm, tn, split, kb0, kb1);
+      for (int u = unit0; u < nunits && ok; u += unit_step) {
+        Unit w;
+        Work::template decode<Cfg>(args, u, w);
+        const int kb0 = w.kb0, kb1 = w.kb1;
         for (int c0 = kb0; c0 < kb1 && ok; c0 += KC, ++q) {
           const int c1 = min(c0 + KC, kb1);
           const uint32_t slot = q % R;
@@ -377,10 +428,13 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         mbar_arrive(smem_u32(&rempty[slot]));
       }
     };
-    for (int u = unit0; u < g.units && ok; u += unit_step) {
-      int tm, tn, split, kb0, kb1;
-      decode_unit<BM, BN>(g, u, tm, tn, split, kb0, kb1);
-      const int tile_m = Cfg::PAIR ? 2 * tm + (int)rank : tm;  // this CTA's 128-row tile
+    int seq = 0;  // units this CTA has taken
+    for (int u = unit0; u < nunits && ok; u += unit_step, ++seq) {
+      Unit w;
+      Work::template decode<Cfg>(args, u, w);
+      const int kb0 = w.kb0, kb1 = w.kb1;
+      const bool from_tmem = Work::from_tmem(w);
+      const int tile_m = Cfg::PAIR ? 2 * w.tm + (int)rank : w.tm;  // this CTA's 128-row tile
       float acc[128];
 #pragma unroll
       for (int i = 0; i < 128; ++i) acc[i] = 0.f;
@@ -404,13 +458,14 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         tc_fence_before();
         // An epilogue that reads the tile from tensor memory keeps the last
         // chunk's slot: the summed accumulator goes back into it below.
-        if (Epi::FROM_TMEM && c0 + KC >= kb1)
+        if (from_tmem && c0 + KC >= kb1)
           kept = slot;
         else
           release(slot);
       }
       if (!ok) continue;
-      if constexpr (Epi::FROM_TMEM) {
+      const int col0 = w.tn * BN + wg * 128;
+      if (from_tmem) {
         const uint32_t ta = tmem_base + lane_off + kept * BN + col_off;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -419,11 +474,26 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           for (int k = 0; k < 32; ++k) v[k] = acc[32 * j + k];
           tmem_st32(ta + 32 * j, v);
         }
-        Epi::apply_tmem(ep, g, ta, tile_m, qtr * 32 + lane, tn * BN + wg * 128);
+        Work::epi_tmem(args, w, ta, tile_m, qtr * 32 + lane, col0);
         tc_fence_before();
         release(kept);
       } else {
-        Epi::apply_regs(ep, g, acc, tile_m, tn, split, qtr * 32 + lane, tn * BN + wg * 128);
+        Work::epi_regs(args, w, acc, tile_m, qtr * 32 + lane, col0);
+      }
+      if constexpr (Work::SIGNALS) {
+        // Publish this unit's stores: every thread makes them visible to the
+        // GPU (and to TMA reads); the last of the CTA's eight consumer warps
+        // to finish the unit adds one to its ready counter.  Warps never
+        // drift four units apart (each chunk's slot is released by all of
+        // them), so four counters indexed by the unit's sequence number keep
+        // the arrivals of different units apart.
+        fence_proxy_async_global();
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) {
+          const int old = atom_add_acq_rel_cta(smem_u32(&epi_count[seq & 3]), 1);
+          if ((old & 7) == 7) red_release_gpu_add(Work::done_counter(args, w), 1);
+        }
       }
     }
   }

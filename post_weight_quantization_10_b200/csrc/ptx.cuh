@@ -316,6 +316,57 @@ __device__ __forceinline__ void st_v8f(float* p, const float (&v)[8]) {
   st_v8(p, u);
 }
 
+// Ordering between the CTAs of one persistent launch.  A unit's epilogue
+// publishes its stores with a release add on a ready counter; a producer that
+// needs them polls the counter with acquire loads and then orders its TMA
+// reads (async proxy) after what it has observed (generic proxy).
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_gpu_add(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int atom_add_acq_rel_cta(uint32_t smem_addr, int v) {
+  int old;
+  asm volatile("atom.acq_rel.cta.shared::cta.add.s32 %0, [%1], %2;"
+               : "=r"(old)
+               : "r"(smem_addr), "r"(v)
+               : "memory");
+  return old;
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Bounded wait until *cnt >= target (acquire), then a proxy fence so that
+// later TMA reads see what the counter published.  Gives up, like mbar_wait,
+// after kWaitCycles or as soon as this CTA or any other has recorded a failure.
+__device__ __forceinline__ bool wait_counter(const int* cnt, int target, volatile int* abort_flag,
+                                             int* status) {
+  if (ld_acquire_gpu(cnt) < target) {
+    const long long t0 = clock64();
+    for (uint32_t i = 1;; ++i) {
+      __nanosleep(32);
+      if (ld_acquire_gpu(cnt) >= target) break;
+      if ((i & 63u) == 0) {
+        if (*abort_flag || *(volatile int*)status != KSTAT_OK) {
+          *abort_flag = 1;
+          return false;
+        }
+        if (clock64() - t0 > kWaitCycles) {
+          *abort_flag = 1;
+          atomicExch(status, KSTAT_TIMEOUT);
+          return false;
+        }
+      }
+    }
+  }
+  fence_proxy_async_global();
+  return true;
+}
+
 // Instruction descriptor with fp32 D: kind::f16 with bf16 A/B (fmt 1) or
 // kind::tf32 (fmt 2).
 __host__ __device__ constexpr uint32_t idesc_f32acc(uint32_t fmt, int M, int N, bool a_mn, bool b_mn) {

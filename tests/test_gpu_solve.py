@@ -51,10 +51,10 @@ def _oracle(p, X, W, grid, iters=None):
     return H, Wm, res
 
 
-def _solver(A, p, X, W, grid, iters=None, split="auto", scaling=True):
+def _solver(A, p, X, W, grid, iters=None, split="auto", scaling=True, schedule="fused"):
     prm = A.Params(bits=p.bits, group=p.group, iters=p.iters if iters is None else iters,
                    rho0=p.rho0, gamma=p.gamma, lambda_rel=p.lambda_rel, grid=grid, split=split,
-                   scaling=scaling)
+                   scaling=scaling, schedule=schedule)
     G = A.build_hessian(X)
     s = A.Solver(X.shape[1], W.shape[0], prm)
     s.prepare(G, W)
@@ -242,3 +242,38 @@ def test_unscaled_ablation_teacher_forced(A, name):
         mism = np.mean(s.codes.cpu().numpy() != e["codes_out"].T)
         assert mism <= 1e-3, (t, mism)
     s.dump_wtilde(None)
+
+
+@pytest.mark.parametrize("name,grid,split", [("tiny", "lsq", "auto"), ("ragged", "lsq", "auto"),
+                                             ("ragged", "mse", "mixed"),
+                                             ("down_small", "minmax", "auto")])
+def test_fused_schedule_matches_per_gemm(A, name, grid, split):
+    """The fused schedule runs GEMM 1 and GEMM 2 of all iterations in one
+    launch, each unit waiting for the row block it reads; every unit keeps the
+    arithmetic of the separate launches, so codes, grids, dual, objective and
+    residual history equal the per-GEMM schedule's bit for bit -- also when the
+    iterations are split over several calls."""
+    p, X, W = _layer(name)
+    runs = {}
+    for sched in ("per_gemm", "fused", "fused_in_parts"):
+        s = _solver(A, p, X, W, grid, split=split,
+                    schedule="per_gemm" if sched == "per_gemm" else "fused")
+        if sched == "fused_in_parts":
+            s.init()
+            t = 0
+            for n in (1, 2, 7, p.iters):
+                n = min(n, p.iters - t)
+                s.iterate(t, n)
+                t += n
+            s.finish()
+        else:
+            s.solve()
+        torch.cuda.synchronize()
+        assert s.kernel_status() == 0, sched
+        runs[sched] = {k: v.cpu().clone() for k, v in (
+            ("codes", s.codes), ("scale", s.scale), ("zero", s.zero), ("V", s.buffer("V")),
+            ("resid", s.resid), ("objective", s.objective))}
+    ref = runs["per_gemm"]
+    for sched in ("fused", "fused_in_parts"):
+        for k, v in runs[sched].items():
+            assert torch.equal(v, ref[k]), (sched, k)
