@@ -34,6 +34,8 @@ sys.path.insert(0, ROOT)
 from post_weight_quantization_10_b200 import dist as D  # noqa: E402
 from post_weight_quantization_10_b200 import workloads  # noqa: E402
 
+DTYPES = {"mixed": "f32 via tf32+bf16 split", "3xtf32": "f32 via 3xtf32",
+          "f16": "f32 via fp16x3 split (power-of-two scaled)"}
 METRIC = "ADMM-Q layer solve: iters/s, TFLOP/s vs tensor peak; Gram TFLOP/s; s/layer"
 REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
@@ -287,7 +289,7 @@ def run_sharded(args, rank, world, device):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "strong",
         "vs_baseline": None,
-        "dtype": "f32 via tf32+bf16 split" if run.s.split == "mixed" else "f32 via 3xtf32",
+        "dtype": DTYPES[run.s.split],
         "data": "synthetic (seeded Qwen3-8B-shaped activations and weights; no dataset)",
         "config": {"workload": workload_desc(p, args.grid) + " (one layer split over the ranks)",
                    "parallelism": f"tokens and output rows split over {world} ranks, "
@@ -389,6 +391,7 @@ def run_ours(args, rank, world, device):
     dist_barrier(world)
     launches = A.launch_count() - n0
     clk = clocks.stop()
+    run.s.check()   # a timed-out wait or an fp16 range overflow invalidates the run
     ms = t_start.elapsed_time(t_end)
     gemm_ms, gemm_n, gemm_iters = run.s.get_timing()
     run.s.set_timing(False)
@@ -434,10 +437,11 @@ def run_ours(args, rank, world, device):
     achieved = flops_launch / (avg_ms / 1e3) / 1e12
     # Tensor work per fp32-accurate product, in bf16-MMA units (dense tf32 runs
     # at half the bf16 rate, nominal 1.1 vs 2.25 PFLOP/s): 3xTF32 = three tf32
-    # MMAs = 6; mixed split = one tf32 MMA (2) + one bf16 MMA over the doubled
+    # MMAs = 6; fp16 x3 = three full-rate fp16 MMAs = 3; mixed split = one
+    # tf32 MMA (2) + one bf16 MMA over the doubled
     # K of the correction rows (2) = 4.  Peak = bf16 peak / that.
     split = run.s.split
-    per_product = 4.0 if split == "mixed" else 6.0
+    per_product = {"mixed": 4.0, "3xtf32": 6.0, "f16": 3.0}[split]
     peak_split = pk["bf16_sust"] / per_product
     line = {
         "metric": METRIC,
@@ -450,7 +454,7 @@ def run_ours(args, rank, world, device):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f32 via tf32+bf16 split" if split == "mixed" else "f32 via 3xtf32",
+        "dtype": DTYPES[split],
         "data": "synthetic (seeded Qwen3-8B-shaped activations and weights; no dataset)",
         "config": {"workload": workload_desc(p, args.grid) + (" Sigma=I (unscaled ablation)"
                                                               if args.no_scaling else ""),
@@ -697,8 +701,8 @@ def main():
     ap.add_argument("--shard", action="store_true",
                     help="split ONE layer over the ranks (tokens and output rows; H all-reduced)")
     ap.add_argument("--grid", default="lsq", choices=["lsq", "minmax", "mse", "frozen"])
-    ap.add_argument("--split", default="auto", choices=["auto", "mixed", "3xtf32"],
-                    help="split precision of the eigenbasis GEMMs (auto: mixed from d_in 2048)")
+    ap.add_argument("--split", default="auto", choices=["auto", "f16", "mixed", "3xtf32"],
+                    help="split precision of the eigenbasis GEMMs (auto: f16 from d_in 2048)")
     ap.add_argument("--schedule", default="fused", choices=["fused", "per_gemm"],
                     help="fused: GEMM 1 and GEMM 2 of all iterations in one launch; "
                          "per_gemm: two launches per iteration")

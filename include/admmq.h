@@ -46,7 +46,8 @@ enum {
   ADMMQ_ERR_NONFINITE = -5,   /* NaN/Inf found in H's diagonal or the eigenvalues */
   ADMMQ_ERR_TIMEOUT = -6,     /* a kernel's bounded pipeline wait gave up        */
   ADMMQ_ERR_WORKSPACE = -7,   /* the workspace is smaller than required          */
-  ADMMQ_ERR_UNSUPPORTED = -8  /* device is not sm_100 or a shape is unsupported  */
+  ADMMQ_ERR_UNSUPPORTED = -8, /* device is not sm_100 or a shape is unsupported  */
+  ADMMQ_ERR_RANGE = -9        /* an fp16-split operand left fp16's range          */
 };
 
 /* Grid refresh used by the D-update (the pages do not fix the fit). */
@@ -66,9 +67,12 @@ enum { ADMMQ_DTYPE_F32 = 0, ADMMQ_DTYPE_BF16 = 1 };
 /* Split precision of the eigenbasis GEMMs (fp32-accurate products on tf32 /
  * bf16 tensor cores; see "operand encoding" below). */
 enum {
-  ADMMQ_SPLIT_AUTO = 0,   /* mixed from d_in >= 2048, else 3xTF32                 */
+  ADMMQ_SPLIT_AUTO = 0,   /* fp16 x3 from d_in >= 2048, else 3xTF32               */
   ADMMQ_SPLIT_3XTF32 = 1, /* hi.hi + hi.lo + lo.hi, three tf32 products           */
-  ADMMQ_SPLIT_MIXED = 2   /* tf32 hi.hi + one bf16 product for hi.lo + lo.hi      */
+  ADMMQ_SPLIT_MIXED = 2,  /* tf32 hi.hi + one bf16 product for hi.lo + lo.hi      */
+  ADMMQ_SPLIT_F16 = 3     /* hi.hi + hi.lo + lo.hi, three fp16 products on
+                             power-of-two scaled operands (22 bits like 3xTF32,
+                             at the full 16-bit rate)                           */
 };
 
 /* How admmq_iterate launches the iterations.  Every step of an iteration acts
@@ -224,14 +228,20 @@ int admmq_pack(const uint8_t* codes_dev, int d_in, int d_out, int bits, uint32_t
 /* ------------------------------------------------------------ inspection --
  * Device buffers inside the workspace, for tests and diagnostics.
  * Operand encoding of the eigenbasis GEMMs (fp32-accurate split precision,
- * per admmq_split_mode): a matrix x [rows][K] is stored as plane HI, fp32
- * [rows][K] with hi = tf32(x), and plane LO:
- *   ADMMQ_SPLIT_3XTF32: fp32 [rows][K], lo = tf32(x - hi);
- *   ADMMQ_SPLIT_MIXED:  u16 [rows][2K] of bfloat16 bit patterns: per 32
- *     columns c0..c0+31 of a row, for operands on the A side (W^~, P, T) the
- *     32 values bf16(hi) then the 32 values bf16(x - hi); on the B side
- *     (Q^T, Q) the two halves swapped.
- * All roundings nearest-even.  Both encodings take 4 bytes per element.
+ * per admmq_split_mode): a matrix x [rows][K] is stored as planes HI and LO:
+ *   ADMMQ_SPLIT_3XTF32: HI fp32 [rows][K] with hi = tf32(x); LO fp32
+ *     [rows][K], lo = tf32(x - hi);
+ *   ADMMQ_SPLIT_MIXED: HI as for 3XTF32; LO u16 [rows][2K] of bfloat16 bit
+ *     patterns: per 32 columns c0..c0+31 of a row, for operands on the A side
+ *     (W^~, P, T, Delta~) the 32 values bf16(hi) then the 32 values
+ *     bf16(x - hi); on the B side (Q^T, Q) the two halves swapped;
+ *   ADMMQ_SPLIT_F16: HI and LO u16 [rows][K] of IEEE fp16 bit patterns,
+ *     hi = fp16(x s), lo = fp16(x s - hi), with s = 2^14 on the B side
+ *     (|entries| <= 1) and s = ADMMQ_BUF_ROW_IN[row] on the A side: a power
+ *     of two with s ||W^~_row|| in [2^9, 2^10).  A scaled A-side value at or
+ *     beyond 65504 sets status word 3 (admmq_check: ADMMQ_ERR_RANGE).
+ * All roundings nearest-even.  Every encoding fits 4 bytes per element per
+ * plane.
  * Layouts:
  *   ADMMQ_BUF_SIGMA, _RSIG, _HDIAG, _LAMBDA : fp32 [d_in]
  *   ADMMQ_BUF_V      fp32 [d_out][d_in]  scaled dual V~
@@ -241,11 +251,18 @@ int admmq_pack(const uint8_t* codes_dev, int d_in, int d_out, int bits, uint32_t
  *   ADMMQ_BUF_E_HI/_E_LO  E = Q^T (row k = k-th eigenvector of H~), encoded
  *                         planes (B side)
  *   ADMMQ_BUF_HT     fp64 [d_in][d_in]   H~ before admmq_eigh, Q^T after
- *   ADMMQ_BUF_STATUS int32 [4]           kernel status words (0 = ok)     */
+ *   ADMMQ_BUF_STATUS int32 [4]           kernel status words (0 = ok): [0]
+ *                    a bounded wait gave up, [1] setup, [2] eigenvalues,
+ *                    [3] fp16-split range
+ *   ADMMQ_BUF_ROW_IN fp32 [d_out]        A-side operand scale per row
+ *                                        (1 unless ADMMQ_SPLIT_F16)
+ *   ADMMQ_BUF_ROW_OUT fp32 [d_out]       factor that unscales a GEMM result
+ *                                        row (1 / (ROW_IN 2^14) for fp16) */
 enum {
   ADMMQ_BUF_SIGMA = 0, ADMMQ_BUF_RSIG, ADMMQ_BUF_HDIAG, ADMMQ_BUF_LAMBDA, ADMMQ_BUF_V,
   ADMMQ_BUF_C0, ADMMQ_BUF_P_HI, ADMMQ_BUF_P_LO, ADMMQ_BUF_T_HI, ADMMQ_BUF_T_LO,
-  ADMMQ_BUF_E_HI, ADMMQ_BUF_E_LO, ADMMQ_BUF_HT, ADMMQ_BUF_STATUS, ADMMQ_BUF_COUNT
+  ADMMQ_BUF_E_HI, ADMMQ_BUF_E_LO, ADMMQ_BUF_HT, ADMMQ_BUF_STATUS, ADMMQ_BUF_ROW_IN,
+  ADMMQ_BUF_ROW_OUT, ADMMQ_BUF_COUNT
 };
 int admmq_get_buffer(admmq_ctx* ctx, int which, void** ptr_dev, size_t* bytes);
 
@@ -268,25 +285,32 @@ int admmq_get_timing(admmq_ctx* ctx, double ms[2], int launches[2], int* iters_t
 /* Standalone projection kernel (the fused GEMM-2 epilogue reading W~ from
  * memory instead of tensor memory); same per-element float32 arithmetic.
  * All pointers device; V_dev is updated in place; P is written in the
- * eigenbasis GEMMs' operand encoding of `split_mode` (ADMMQ_SPLIT_3XTF32 or
- * ADMMQ_SPLIT_MIXED, A side): P_hi_dev fp32 [d_out][d_in] and P_lo_dev
- * (fp32 [d_out][d_in] or u16 [d_out][2 d_in]); codes/scale/zero hold the
- * previous D on entry and the new D on exit; resid_dev fp64 [2] receives the
- * two residual sums of squares.
+ * eigenbasis GEMMs' operand encoding of `split_mode` (ADMMQ_SPLIT_3XTF32,
+ * ADMMQ_SPLIT_MIXED or ADMMQ_SPLIT_F16, A side; see "operand encoding"):
+ * P_hi_dev / P_lo_dev as that encoding lays them out; row_scale_dev
+ * (optional, fp32 [d_out]) is the fp16 split's per-row scale (1 when NULL);
+ * range_flag_dev (optional, int32) is set to 1 when a scaled value leaves
+ * fp16's range; codes/scale/zero hold the previous D on entry and the new D
+ * on exit; resid_dev fp64 [2] receives the two residual sums of squares.
  * V_dev, codes_dev, P_hi_dev, P_lo_dev, sigma_dev, rsig_dev and hdiag_dev
- * must be 32-byte aligned, wtilde_dev 16-byte aligned (ADMMQ_ERR_INVALID_ARG
- * otherwise). */
+ * must be 32-byte aligned, wtilde_dev 16-byte aligned, row_scale_dev and
+ * range_flag_dev 4-byte aligned (ADMMQ_ERR_INVALID_ARG otherwise). */
 int admmq_project(const float* wtilde_dev, float* V_dev, const float* sigma_dev,
                   const float* rsig_dev, const float* hdiag_dev, int d_in, int d_out, int bits,
                   int group, int grid_mode, int split_mode, uint8_t* codes_dev, float* scale_dev,
-                  float* zero_dev, float* P_hi_dev, void* P_lo_dev, double* resid_dev,
-                  void* stream);
+                  float* zero_dev, void* P_hi_dev, void* P_lo_dev, const float* row_scale_dev,
+                  int* range_flag_dev, double* resid_dev, void* stream);
 
 /* The split precision a context runs its eigenbasis GEMMs in
- * (ADMMQ_SPLIT_3XTF32 or ADMMQ_SPLIT_MIXED; ADMMQ_SPLIT_AUTO resolved by
- * d_in), which fixes the encoding of its P/T/E buffers; ADMMQ_ERR_INVALID_ARG
- * for a NULL context. */
+ * (ADMMQ_SPLIT_3XTF32, ADMMQ_SPLIT_MIXED or ADMMQ_SPLIT_F16; ADMMQ_SPLIT_AUTO
+ * resolved by d_in), which fixes the encoding of its P/T/E buffers;
+ * ADMMQ_ERR_INVALID_ARG for a NULL context. */
 int admmq_split_mode(const admmq_ctx* ctx);
+
+/* Synchronises the stream and reads the kernel status words: ADMMQ_OK,
+ * ADMMQ_ERR_TIMEOUT (a bounded wait gave up) or ADMMQ_ERR_RANGE (an fp16-split
+ * operand left fp16's range; rerun with ADMMQ_SPLIT_MIXED or _3XTF32). */
+int admmq_check(admmq_ctx* ctx, void* stream);
 
 /* ---------------------------------------------------------------- GPTQ ----
  * The baseline the ADMM-Q objective is reported against: GPTQ, Algorithm 1

@@ -188,17 +188,58 @@ def _rows_to_groups(A: np.ndarray, g: int) -> np.ndarray:
     return A.reshape(m * (d // g), g)
 
 
-def encode_operand(x: np.ndarray, split: str, side: str = "A"):
+F16_B_SCALE = np.float32(2.0 ** 14)
+F16_LIMIT = np.float32(65504.0)
+
+
+def split_f16(x: np.ndarray, s):
+    """fp16 pair of x scaled by s (a power of two, per row or scalar): hi =
+    fp16(x s), lo = fp16(x s - hi), nearest-even, as uint16 bit patterns, and
+    whether any |x s| reached fp16's largest finite value (the range flag).
+    hi + lo carries 22 significant bits; each product of two fp16 values is
+    exact in float32, so hi.hi + hi.lo + lo.hi gives the fp32-accurate
+    product as three fp16 tensor-core products."""
+    x = _f(x)
+    s = _f(s)
+    xs = _f(x * (s[:, None] if s.ndim == 1 else s))
+    with np.errstate(over="ignore"):
+        hi = xs.astype(np.float16)
+        lo = _f(xs - hi.astype(np.float32)).astype(np.float16)
+    bad = bool(np.any(~(np.abs(xs) < F16_LIMIT)))
+    return hi.view(np.uint16), lo.view(np.uint16), bad
+
+
+def row_scales_f16(W_tilde_rows: np.ndarray):
+    """Per-row power-of-two scale of the A operands under the fp16 split: 2^e
+    with 2^e ||row|| in [2^9, 2^10) (row norms of W^~ = Sigma^-1 W_hat,
+    rows = output channels, computed in float64), e clamped to [-60, 60];
+    1 for a zero row."""
+    n = np.sqrt(np.sum(np.asarray(W_tilde_rows, np.float64) ** 2, axis=1))
+    e = np.zeros(n.shape, np.int64)
+    ok = (n > 0) & np.isfinite(n)
+    _, k = np.frexp(n[ok])
+    e[ok] = np.clip(10 - k, -60, 60)
+    return np.ldexp(np.float32(1), e).astype(np.float32)
+
+
+def encode_operand(x: np.ndarray, split: str, side: str = "A", row_scale=None):
     """The eigenbasis GEMMs' operand planes of x in the given split precision:
-    "3xtf32" -> (tf32(x), tf32(x - tf32(x))) as float32; "mixed" -> split_mix."""
+    "3xtf32" -> (tf32(x), tf32(x - tf32(x))) as float32; "mixed" -> split_mix;
+    "f16" -> split_f16 with the rows' scales (side "A", row_scale) or 2^14
+    (side "B")."""
     if split == "3xtf32":
         return split_tf32(x)
     if split == "mixed":
         return split_mix(x, side)
+    if split == "f16":
+        s = F16_B_SCALE if side == "B" else np.asarray(row_scale, np.float32)
+        hi, lo, _ = split_f16(x, s)
+        return hi, lo
     raise ValueError(split)
 
 
-def init_step(W_rows: np.ndarray, rsig: np.ndarray, bits: int, group: int, split: str = "mixed"):
+def init_step(W_rows: np.ndarray, rsig: np.ndarray, bits: int, group: int, split: str = "mixed",
+              row_scale=None):
     """RTN start of the iteration in memory layout ([d_out][d_in]).
 
     y = W_hat; minmax grid; D = s (q - z); D~ = D * rsig (rsig = sqrt(diag H)),
@@ -211,7 +252,7 @@ def init_step(W_rows: np.ndarray, rsig: np.ndarray, bits: int, group: int, split
     q = round_to_grid(yg, s, z, L)
     D = dequantize(q, s, z).reshape(m, d)
     Dt = _f(D * _f(rsig)[None, :])
-    hi, pc = encode_operand(Dt, split, "A")
+    hi, pc = encode_operand(Dt, split, "A", row_scale)
     return dict(codes=q.reshape(m, d).astype(np.uint8), scale=s.reshape(m, d // group),
                 zero=z.reshape(m, d // group), P=Dt, P_hi=hi, P_lo=pc)
 
@@ -219,7 +260,7 @@ def init_step(W_rows: np.ndarray, rsig: np.ndarray, bits: int, group: int, split
 def epilogue_step(W_acc: np.ndarray, V: np.ndarray, sigma: np.ndarray, rsig: np.ndarray,
                   hdiag: np.ndarray, s_prev: np.ndarray, z_prev: np.ndarray,
                   codes_prev: np.ndarray, bits: int, group: int, mode: str,
-                  split: str = "mixed"):
+                  split: str = "mixed", row_scale=None):
     """One fused projection + dual update in memory layout ([d_out][d_in]).
 
     Per element (i = input channel):
@@ -256,7 +297,7 @@ def epilogue_step(W_acc: np.ndarray, V: np.ndarray, sigma: np.ndarray, rsig: np.
     Dt = _f(D * _f(rsig)[None, :])
     V_new = _f(t - Dt)
     P = _f(Dt - V_new)
-    hi, lo = encode_operand(P, split, "A")
+    hi, lo = encode_operand(P, split, "A", row_scale)
     qp = _rows_to_groups(_f(codes_prev), group)
     Dt_prev = _f(dequantize(qp, sp, zp).reshape(m, d) * _f(rsig)[None, :])
     r2 = float(np.sum((W_acc.astype(np.float64) - Dt) ** 2))

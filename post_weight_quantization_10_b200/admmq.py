@@ -18,11 +18,12 @@ from .build import LIB
 OK = 0
 GRID_MINMAX, GRID_LSQ, GRID_FROZEN, GRID_MSE = 0, 1, 2, 3
 GRID_MODES = {"minmax": GRID_MINMAX, "lsq": GRID_LSQ, "frozen": GRID_FROZEN, "mse": GRID_MSE}
-SPLIT_MODES = {"auto": 0, "3xtf32": 1, "mixed": 2}
+SPLIT_MODES = {"auto": 0, "3xtf32": 1, "mixed": 2, "f16": 3}
 SCHEDULES = {"fused": 0, "per_gemm": 1}
 DTYPE_F32, DTYPE_BF16 = 0, 1
 BUFFERS = ["sigma", "rsig", "hdiag", "lambda", "V", "C0", "P_hi", "P_lo", "T_hi", "T_lo",
-           "E_hi", "E_lo", "Ht", "status"]
+           "E_hi", "E_lo", "Ht", "status", "row_in", "row_out"]
+ERR_TIMEOUT, ERR_RANGE = -6, -9
 
 
 class AdmmqError(RuntimeError):
@@ -48,7 +49,7 @@ class Params:
     gamma: float = 1.05
     lambda_rel: float = 0.01
     grid: str = "lsq"
-    split: str = "auto"   # eigenbasis GEMM split precision: auto | 3xtf32 | mixed
+    split: str = "auto"   # eigenbasis GEMM split precision: auto | 3xtf32 | mixed | f16
     scaling: bool = True  # False: Sigma = I (the unscaled ablation)
     schedule: str = "fused"  # fused: one launch per iterate call | per_gemm: two per iteration
 
@@ -110,8 +111,9 @@ def lib():
         "admmq_get_timing": (_i, [_vp, ctypes.POINTER(ctypes.c_double),
                                   ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
         "admmq_project": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp,
-                               _vp, _vp, _vp, _vp]),
+                               _vp, _vp, _vp, _vp, _vp, _vp]),
         "admmq_split_mode": (_i, [_vp]),
+        "admmq_check": (_i, [_vp, _vp]),
         "admmq_gptq_workspace_bytes": (_sz, [_i, _i, _i]),
         "admmq_gptq": (_i, [_vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float, _i, _vp, _vp, _vp, _vp,
                             _sz, _vp]),
@@ -247,6 +249,11 @@ class Solver:
         synchronises with the device."""
         return int(self.buffer("status")[0].item())
 
+    def check(self, stream=None):
+        """Synchronise and raise AdmmqError if a kernel's bounded wait gave up
+        (ERR_TIMEOUT) or an fp16-split operand left fp16's range (ERR_RANGE)."""
+        _check(lib().admmq_check(self._ctx, _stream(stream)), "admmq_check")
+
     def buffer(self, name: str) -> torch.Tensor:
         """A torch view of a workspace buffer (see include/admmq.h for layouts)."""
         which = BUFFERS.index(name)
@@ -256,11 +263,15 @@ class Solver:
         off = p.value - self.workspace.data_ptr()
         raw = self.workspace[off:off + nb.value]
         d, m = self.d_in, self.d_out
-        if name in ("sigma", "rsig", "hdiag", "lambda"):
+        if name in ("sigma", "rsig", "hdiag", "lambda", "row_in", "row_out"):
             return raw.view(torch.float32)
         if name in ("V", "C0"):
             return raw.view(torch.float32).view(m, d)
         mixed = self.split == "mixed"
+        if self.split == "f16" and name in ("P_hi", "P_lo", "T_hi", "T_lo"):   # fp16 bit patterns
+            return raw[:2 * m * d].view(torch.int16).view(m, d)
+        if self.split == "f16" and name in ("E_hi", "E_lo"):
+            return raw[:2 * d * d].view(torch.int16).view(d, d)
         if name in ("P_hi", "T_hi") or (name in ("P_lo", "T_lo") and not mixed):
             return raw.view(torch.float32).view(m, d)
         if name in ("P_lo", "T_lo"):   # bf16 correction rows (bit patterns)
@@ -277,7 +288,7 @@ class Solver:
     def split(self) -> str:
         """The eigenbasis GEMMs' split precision ("3xtf32" or "mixed")."""
         mode = int(lib().admmq_split_mode(self._ctx))
-        return {1: "3xtf32", 2: "mixed"}[mode]
+        return {1: "3xtf32", 2: "mixed", 3: "f16"}[mode]
 
     def dump_wtilde(self, out: torch.Tensor | None):
         _check(lib().admmq_debug_dump_wtilde(self._ctx, _ptr(out)), "admmq_debug_dump_wtilde")
@@ -307,16 +318,18 @@ def pack(codes: torch.Tensor, bits: int, out: torch.Tensor | None = None, stream
 
 
 def project(wtilde, V, sigma, rsig, hdiag, bits, group, grid, codes, scale, zero, P_hi, P_lo,
-            resid=None, split="mixed", stream=None):
-    """Stand-alone projection; P_lo is fp32 [m][d] for split "3xtf32", int16
-    (bf16 bit patterns) [m][2d] for "mixed"."""
+            resid=None, split="mixed", row_scale=None, range_flag=None, stream=None):
+    """Stand-alone projection; P planes in the encoding of `split`: "3xtf32"
+    fp32 [m][d] x2, "mixed" fp32 [m][d] + int16 (bf16 bit patterns) [m][2d],
+    "f16" int16 (fp16 bit patterns) [m][d] x2 with the rows' scales
+    `row_scale` (fp32 [m]; None = 1) and an optional int32 range flag."""
     m, d = wtilde.shape
     if resid is None:
         resid = torch.zeros(2, dtype=torch.float64, device=wtilde.device)
     _check(lib().admmq_project(_ptr(wtilde), _ptr(V), _ptr(sigma), _ptr(rsig), _ptr(hdiag), d, m,
                                bits, group, GRID_MODES[grid], SPLIT_MODES[split], _ptr(codes),
-                               _ptr(scale), _ptr(zero), _ptr(P_hi), _ptr(P_lo), _ptr(resid),
-                               _stream(stream)),
+                               _ptr(scale), _ptr(zero), _ptr(P_hi), _ptr(P_lo), _ptr(row_scale),
+                               _ptr(range_flag), _ptr(resid), _stream(stream)),
            "admmq_project")
     return resid
 

@@ -32,19 +32,23 @@ inline void count_launch() { __atomic_fetch_add(&g_launches, 1ull, __ATOMIC_RELA
 // X^T X: bf16, both operands MN-major (X is token-major).
 // Promoted every 4 k-blocks (16 MMAs of K = 16).
 using GramCfg = GemmCfg<KIND_BF16, 1, true, true, 4, 4, false>;
-// Eigenbasis GEMMs, K-major operands, promoted every 8 k-blocks:
-//   mixed split (tf32 hi.hi + one bf16 product for the corrections, 64 MMAs
-//   per chunk) for large layers, 3xTF32 (96 MMAs per chunk) where the
-//   reduction is short enough that the split's own rounding would dominate.
-// Both run on CTA pairs (2-SM MMAs of 256 x 128; each SM stages half of B,
-// which cuts the shared-memory traffic per MMA by a quarter) with 4 stages.
+// Eigenbasis GEMMs: K-major operands on CTA pairs (2-SM MMAs of 256 x 256
+// tiles), 3 stages of 64 KB, promoted every KC k-blocks (K = 512 per chunk):
+//   fp16 x3 (three full-rate fp16 products per K step, 96 MMAs per chunk):
+//     the default for large layers;
+//   mixed split (tf32 hi.hi + one bf16 product for the corrections, 128 MMAs
+//     per chunk);
+//   3xTF32 (three tf32 products, 192 MMAs per chunk): the default where the
+//     reduction is short.
 using EigCfg = GemmCfg<KIND_MIX, 2, false, false, 3, 16, true>;
 using EigCfg3 = GemmCfg<KIND_TF32, 2, false, false, 3, 16, true>;
-static_assert(EigCfg::BN == EigCfg3::BN && EigCfg::BK == EigCfg3::BK &&
-                  EigCfg::UNIT_M == EigCfg3::UNIT_M && EigCfg::B_ROWS == EigCfg3::B_ROWS,
-              "same tile geometry");
-// d_in from which the automatic split mode picks the mixed split
-constexpr int kMixedFromDin = 2048;
+using EigCfgF = GemmCfg<KIND_F16X3, 2, false, false, 3, 8, true>;
+static_assert(EigCfg::BN == EigCfg3::BN && EigCfg::BK == EigCfg3::BK && EigCfg::BN == EigCfgF::BN &&
+                  EigCfg::UNIT_M == EigCfg3::UNIT_M && EigCfg::UNIT_M == EigCfgF::UNIT_M &&
+                  EigCfg::B_ROWS == EigCfg3::B_ROWS && EigCfg::B_ROWS == EigCfgF::B_ROWS,
+              "same tile geometry (K per stage differs: 32 fp32 or 64 fp16 elements)");
+// d_in from which the automatic split mode picks the fp16 split
+constexpr int kSplitFromDin = 2048;
 
 // Setup status words (ws status[1]).
 enum { SETUP_OK = 0, SETUP_NONFINITE = 1, SETUP_NOT_PD = 2 };
@@ -109,48 +113,83 @@ __device__ __forceinline__ float load_w<__nv_bfloat16>(const __nv_bfloat16* p, l
 
 #include "gptq.cuh"
 
+// Power-of-two operand scale of each output row for the fp16 split.  Every
+// A operand of the eigenbasis GEMMs is a row of the W~ family (W^~, P =
+// D~ - V~, T, Delta~), whose entries stay within a small multiple of the
+// row's norm ||W^~_j||; with 2^e_j ||W^~_j|| in [2^9, 2^10) they keep 64x
+// headroom below fp16's largest value (an overflow raises the range flag)
+// while the fp16 pair's absolute resolution stays far below what the
+// row's products need.  row_out = 2^(-e_j - 14) undoes e_j and the B
+// operands' 2^14 on a GEMM result.  Other encodings: 1 and 1.  One warp per
+// row; the norm is summed in float64.
+template <typename T>
+__global__ void k_row_scales(const T* __restrict__ W, const float* __restrict__ rsig, int m, int d,
+                             int enc, float* __restrict__ row_in, float* __restrict__ row_out) {
+  const int warps = (int)(blockDim.x >> 5), lane = (int)(threadIdx.x & 31);
+  for (long long row = blockIdx.x * (long long)warps + (threadIdx.x >> 5); row < m;
+       row += (long long)gridDim.x * warps) {
+    double n2 = 0.0;
+    for (int i = lane; i < d; i += 32) {
+      const double w = (double)__fmul_rn(load_w<T>(W, row * d + i), rsig[i]);
+      n2 += w * w;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) n2 += __shfl_xor_sync(0xffffffffu, n2, o);
+    if (lane == 0) {
+      int e = 0;
+      if (enc == ENC_F16) {
+        const double nrm = sqrt(n2);
+        if (nrm > 0.0 && isfinite(nrm)) {
+          int k = 0;
+          frexp(nrm, &k);  // nrm in [2^(k-1), 2^k)
+          e = 10 - k;
+          e = e < -60 ? -60 : (e > 60 ? 60 : e);
+        }
+        row_in[row] = ldexpf(1.f, e);
+        row_out[row] = ldexpf(1.f, -e - kBScaleExp);
+      } else {
+        row_in[row] = 1.f;
+        row_out[row] = 1.f;
+      }
+    }
+  }
+}
+
 // W^~ = Sigma^-1 W_hat (rows = output channels) in the operand encoding (A side).
 template <typename T>
 __global__ void k_scale_weights(const T* __restrict__ W, const float* __restrict__ rsig, int d,
-                                long long total, float* __restrict__ hi, void* lo, bool mix) {
+                                long long total, void* hi, void* lo, int enc,
+                                const float* __restrict__ row_in, int* flag) {
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
        idx += (long long)gridDim.x * blockDim.x) {
     const long long row = idx / d;
     const int i = (int)(idx - row * d);
     const float w = __fmul_rn(load_w<T>(W, idx), rsig[i]);
-    const float h = tf32_rne(w);
-    put_operand1(mix, false, hi + row * d, mix ? lo_row<true>(lo, row, d) : lo_row<false>(lo, row, d),
-                 i, h, __fsub_rn(w, h));
+    put_a1(enc, plane0_row(enc, hi, row, d), plane1_row(enc, lo, row, d), i, w, row_in[row], flag);
   }
 }
 
 // Eigenvector buffer (row k = k-th eigenvector, from the column-major solver
 // output) -> operand planes (B side) of E = Q^T [k][i] and of Q [i][k]; the
-// lo part comes from the float64 value (e - hi).
-__global__ void k_split_eigvecs(const double* __restrict__ Evec, int d, float* __restrict__ e_hi,
-                                void* e_lo, float* __restrict__ q_hi, void* q_lo, bool mix) {
-  __shared__ float th[32][33], tl[32][33];
+// low part comes from the float64 value.
+__global__ void k_split_eigvecs(const double* __restrict__ Evec, int d, void* e_hi, void* e_lo,
+                                void* q_hi, void* q_lo, int enc) {
+  __shared__ double tv[32][33];
   const int k0 = blockIdx.y * 32, i0 = blockIdx.x * 32;
   for (int r = threadIdx.y; r < 32; r += blockDim.y) {
     const int k = k0 + r, i = i0 + threadIdx.x;
-    float h = 0.f, l = 0.f;
+    double e = 0.0;
     if (k < d && i < d) {
-      const double e = Evec[(long long)k * d + i];
-      h = tf32_rne((float)e);
-      l = (float)(e - (double)h);
-      put_operand1(mix, true, e_hi + (long long)k * d,
-                   mix ? lo_row<true>(e_lo, k, d) : lo_row<false>(e_lo, k, d), i, h, l);
+      e = Evec[(long long)k * d + i];
+      put_b1(enc, plane0_row(enc, e_hi, k, d), plane1_row(enc, e_lo, k, d), i, e);
     }
-    th[r][threadIdx.x] = h;
-    tl[r][threadIdx.x] = l;
+    tv[r][threadIdx.x] = e;
   }
   __syncthreads();
   for (int r = threadIdx.y; r < 32; r += blockDim.y) {
     const int i = i0 + r, k = k0 + threadIdx.x;
     if (k < d && i < d)
-      put_operand1(mix, true, q_hi + (long long)i * d,
-                   mix ? lo_row<true>(q_lo, i, d) : lo_row<false>(q_lo, i, d), k,
-                   th[threadIdx.x][r], tl[threadIdx.x][r]);
+      put_b1(enc, plane0_row(enc, q_hi, i, d), plane1_row(enc, q_lo, i, d), k, tv[threadIdx.x][r]);
   }
 }
 
@@ -168,8 +207,8 @@ __global__ void k_eigvals(const double* __restrict__ ev, int d, float* __restric
 template <typename T>
 __global__ void k_init_rtn(const T* __restrict__ W, const float* __restrict__ rsig, int m, int d,
                            int g, int L, uint8_t* __restrict__ codes, float* __restrict__ scale,
-                           float* __restrict__ zero, float* __restrict__ V,
-                           float* __restrict__ p_hi, void* p_lo, bool mix) {
+                           float* __restrict__ zero, float* __restrict__ V, void* p_hi,
+                           void* p_lo, int enc, const float* __restrict__ row_in, int* flag) {
   const int ngr = d / g;
   const long long total = (long long)m * ngr;
   const float Lf = (float)L;
@@ -196,12 +235,10 @@ __global__ void k_init_rtn(const T* __restrict__ W, const float* __restrict__ rs
       const float q = clampq(__fadd_rn(rintf(__fdiv_rn(y, s)), z), Lf);
       const float D = __fmul_rn(s, __fsub_rn(q, z));
       const float dt = __fmul_rn(D, rsig[col0 + e]);
-      const float h = tf32_rne(dt);
       codes[base + e] = (uint8_t)q;
       V[base + e] = 0.f;
-      put_operand1(mix, false, p_hi + row * d,
-                   mix ? lo_row<true>(p_lo, row, d) : lo_row<false>(p_lo, row, d), col0 + e, h,
-                   __fsub_rn(dt, h));
+      put_a1(enc, plane0_row(enc, p_hi, row, d), plane1_row(enc, p_lo, row, d), col0 + e, dt,
+             row_in[row], flag);
     }
     scale[gi] = s;
     zero[gi] = z;
@@ -214,7 +251,8 @@ template <typename T>
 __global__ void k_delta_planes(const T* __restrict__ W, const uint8_t* __restrict__ codes,
                                const float* __restrict__ scale, const float* __restrict__ zero,
                                const float* __restrict__ rsig, int d, int g, long long total,
-                               float* __restrict__ hi, void* lo, bool mix) {
+                               void* hi, void* lo, int enc, const float* __restrict__ row_in,
+                               int* flag) {
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
        idx += (long long)gridDim.x * blockDim.x) {
     const long long row = idx / d;
@@ -223,9 +261,8 @@ __global__ void k_delta_planes(const T* __restrict__ W, const uint8_t* __restric
     const float D = __fmul_rn(scale[gi], __fsub_rn((float)codes[idx], zero[gi]));
     const float dt = __fmul_rn(D, rsig[i]);
     const float wt = __fmul_rn(load_w<T>(W, idx), rsig[i]);
-    const float x = __fsub_rn(dt, wt), h = tf32_rne(x);
-    put_operand1(mix, false, hi + row * d, mix ? lo_row<true>(lo, row, d) : lo_row<false>(lo, row, d),
-                 i, h, __fsub_rn(x, h));
+    put_a1(enc, plane0_row(enc, hi, row, d), plane1_row(enc, lo, row, d), i, __fsub_rn(dt, wt),
+           row_in[row], flag);
   }
 }
 
@@ -361,11 +398,11 @@ __global__ void __launch_bounds__(256) k_pack(const uint8_t* __restrict__ codes,
 }
 
 // Standalone projection: one thread per (row, group), W~ read from memory.
-template <int MODE, bool MIX>
+template <int MODE, int ENC>
 __global__ void k_project(const float* __restrict__ wt, float* V, const float* __restrict__ sig,
                           const float* __restrict__ rsig, const float* __restrict__ hd, int m, int d,
-                          int g, int L, uint8_t* codes, float* scale, float* zero, float* p_hi,
-                          void* p_lo, double* resid) {
+                          int g, int L, uint8_t* codes, float* scale, float* zero, void* p_hi,
+                          void* p_lo, const float* __restrict__ row_in, int* flag, double* resid) {
   const int row = blockIdx.x * blockDim.x + threadIdx.x;
   const int grp = blockIdx.y;
   const bool valid = row < m;
@@ -378,12 +415,13 @@ __global__ void k_project(const float* __restrict__ wt, float* V, const float* _
   r.rsig = rsig + col0;
   r.hd = hd + col0;
   r.codes = codes + off;
-  r.phi = p_hi + off;
-  r.plo = MIX ? (void*)(reinterpret_cast<uint16_t*>(p_lo) + (long long)(valid ? row : 0) * 2 * d + 2 * col0)
-              : (void*)(reinterpret_cast<float*>(p_lo) + off);
+  r.phi = plane0_at(ENC, p_hi, valid ? row : 0, d, col0);
+  r.plo = plane1_at(ENC, p_lo, valid ? row : 0, d, col0);
   r.scale = scale + goff;
   r.zero = zero + goff;
   r.wdump = nullptr;
+  r.rs = (valid && row_in) ? row_in[row] : 1.f;
+  r.flag = flag;
   r.valid = valid;
   auto loadw = [&](int c, float (&w)[32]) {
 #pragma unroll
@@ -394,7 +432,7 @@ __global__ void k_project(const float* __restrict__ wt, float* V, const float* _
     }
   };
   float r2 = 0.f, s2 = 0.f;
-  project_group<MODE, MIX>(loadw, r, g, L, r2, s2);
+  project_group<MODE, ENC>(loadw, r, g, L, r2, s2);
   r2 = warp_sum(r2);
   s2 = warp_sum(s2);
   if ((threadIdx.x & 31) == 0) {
@@ -425,22 +463,35 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// Row-major [outer][inner] tensor of bf16 or fp32, box {128 bytes, box_outer},
-// 128-byte swizzle, out-of-bounds elements read as zero.
+// Row-major [outer][inner] tensor of fp32, bf16 or fp16, box {128 bytes,
+// box_outer}, 128-byte swizzle, out-of-bounds elements read as zero.
 bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_outer,
-              bool fp32) {
+              CUtensorMapDataType dt) {
   auto fn = encode_fn();
   if (!fn) return false;
-  const uint32_t es = fp32 ? 4 : 2;
+  const uint32_t es = dt == CU_TENSOR_MAP_DATA_TYPE_FLOAT32 ? 4 : 2;
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {inner * es};
   cuuint32_t box[2] = {128 / es, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+  CUresult r = fn(m, dt, 2,
                   const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// The two planes of an operand [rows][d] in encoding `enc` (see kernels.cuh).
+bool make_plane_maps(CUtensorMap (&mp)[2], void* hi, void* lo, uint64_t d, uint64_t rows,
+                     uint32_t box_rows, int enc) {
+  if (enc == ENC_F16)
+    return make_map(&mp[0], hi, d, rows, box_rows, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) &&
+           make_map(&mp[1], lo, d, rows, box_rows, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+  if (enc == ENC_MIX)
+    return make_map(&mp[0], hi, d, rows, box_rows, CU_TENSOR_MAP_DATA_TYPE_FLOAT32) &&
+           make_map(&mp[1], lo, 2 * d, rows, box_rows, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+  return make_map(&mp[0], hi, d, rows, box_rows, CU_TENSOR_MAP_DATA_TYPE_FLOAT32) &&
+         make_map(&mp[1], lo, d, rows, box_rows, CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
 }
 
 int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
@@ -484,6 +535,13 @@ GemmGeom make_geom(int M, int N, long long K, int BN, int BK, int splits, bool t
 // pair of CTAs per two SMs.  A policy whose units wait on earlier units of the
 // same launch needs every CTA of the launch resident at once, so its grid is
 // capped by the occupancy query.
+// Geometry of an eigenbasis GEMM [rows][d] x [d][d] for an encoding (its K
+// per stage: 32 fp32 or 64 fp16 elements).
+GemmGeom eig_geom(int enc, int rows, int d, int* status) {
+  return enc == ENC_F16 ? make_geom(rows, d, d, EigCfgF::BN, EigCfgF::BK, 1, false, status, EigCfgF::UNIT_M)
+                        : make_geom(rows, d, d, EigCfg::BN, EigCfg::BK, 1, false, status, EigCfg::UNIT_M);
+}
+
 template <class Cfg, class Work>
 cudaError_t launch_work(const typename Work::Args& args, int units, cudaStream_t st) {
   auto kern = k_gemm<Cfg, Work>;
@@ -547,13 +605,17 @@ cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
 }
 
 // An eigenbasis GEMM (A and B operand maps, plane 0 and 1) with the split
-// precision of the context: EpiM for the mixed split, Epi3 for 3xTF32.
-template <class Epi3, class EpiM>
-cudaError_t launch_eig(bool mix, const CUtensorMap (&a)[2], const CUtensorMap (&b)[2],
+// precision of the context: Epi3 for 3xTF32, EpiM for the mixed split, EpiF
+// for the fp16 split.
+template <class Epi3, class EpiM, class EpiF>
+cudaError_t launch_eig(int enc, const CUtensorMap (&a)[2], const CUtensorMap (&b)[2],
                        const GemmGeom& g, const typename EpiM::Params& ep, cudaStream_t st) {
-  static_assert(std::is_same<typename Epi3::Params, typename EpiM::Params>::value, "same params");
-  return mix ? launch_gemm<EigCfg, EpiM>(a[0], a[1], b[0], b[1], g, ep, st)
-             : launch_gemm<EigCfg3, Epi3>(a[0], a[1], b[0], b[1], g, ep, st);
+  static_assert(std::is_same<typename Epi3::Params, typename EpiM::Params>::value &&
+                    std::is_same<typename EpiF::Params, typename EpiM::Params>::value,
+                "same params");
+  if (enc == ENC_F16) return launch_gemm<EigCfgF, EpiF>(a[0], a[1], b[0], b[1], g, ep, st);
+  if (enc == ENC_MIX) return launch_gemm<EigCfg, EpiM>(a[0], a[1], b[0], b[1], g, ep, st);
+  return launch_gemm<EigCfg3, Epi3>(a[0], a[1], b[0], b[1], g, ep, st);
 }
 
 int device_ok() {
@@ -610,14 +672,14 @@ struct admmq_ctx {
   double* work;
   int lwork;
   int* devinfo;
-  // operand planes: *_hi tf32 in fp32 words [rows][d]; *_lo the tf32 lo
-  // plane [rows][d] (3xTF32) or the bf16 correction rows [rows][2d] (mixed);
-  // A side: Wt, P, T; B side: E, Q
-  bool mix;
-  float *E_hi, *Q_hi;                          // [d][d]
+  // operand planes in the encoding `enc` (ENC_*, kernels.cuh): A side Wt, P,
+  // T [m][d]; B side E, Q [d][d]
+  int enc;
+  void *E_hi, *Q_hi;
   void *E_lo, *Q_lo;
-  float *Wt_hi, *P_hi, *T_hi;                  // [m][d]
+  void *Wt_hi, *P_hi, *T_hi;
   void *Wt_lo, *P_lo, *T_lo;
+  float *row_in, *row_out;  // [m] per-row operand scale and result factor (fp16 split)
   float *C0, *V;                               // [m][d]
   float* resid_part;    // [iters][tiles][4][2]
   float* obj_part;      // [tiles][4]
@@ -645,7 +707,7 @@ namespace {
 struct Layout {
   size_t status, lam64, sig64, hdiag, sigma, rsig, lam32, Ht, evals, work, devinfo;
   size_t E_hi, E_lo, Q_hi, Q_lo, Wt_hi, Wt_lo, P_hi, P_lo, T_hi, T_lo, C0, V;
-  size_t resid_part, obj_part, rho_tab, ready, total;
+  size_t resid_part, obj_part, rho_tab, ready, row_in, row_out, total;
 };
 
 Layout make_layout(int d, int m, int iters, int lwork) {
@@ -685,6 +747,8 @@ Layout make_layout(int d, int m, int iters, int lwork) {
   L.obj_part = take(4 * (size_t)tiles * 4);
   L.rho_tab = take(4 * (size_t)(iters > 0 ? iters : 1));
   L.ready = take(4 * 2 * (size_t)cdiv(m, 2 * kBM));
+  L.row_in = take(4 * (size_t)m);
+  L.row_out = take(4 * (size_t)m);
   L.total = o;
   return L;
 }
@@ -712,7 +776,7 @@ int check_params(int d, int m, const admmq_params* p) {
   if (!(p->rho0 > 0.f) || !(p->gamma > 0.f) || !(p->lambda_rel >= 0.f)) return ADMMQ_ERR_INVALID_ARG;
   if (p->grid_mode < ADMMQ_GRID_MINMAX || p->grid_mode > ADMMQ_GRID_MSE)
     return ADMMQ_ERR_INVALID_ARG;
-  if (p->split_mode < ADMMQ_SPLIT_AUTO || p->split_mode > ADMMQ_SPLIT_MIXED)
+  if (p->split_mode < ADMMQ_SPLIT_AUTO || p->split_mode > ADMMQ_SPLIT_F16)
     return ADMMQ_ERR_INVALID_ARG;
   if (p->no_scaling != 0 && p->no_scaling != 1) return ADMMQ_ERR_INVALID_ARG;
   if (p->schedule != ADMMQ_SCHEDULE_FUSED && p->schedule != ADMMQ_SCHEDULE_PER_GEMM)
@@ -821,10 +885,14 @@ cudaError_t launch_admm_loop(const admmq_ctx* c, const GemmGeom& g, const TUpdat
 template <int MODE>
 cudaError_t launch_admm_loop_split(const admmq_ctx* c, const GemmGeom& g, const TUpdateParams& p1,
                                    const ProjParams& p2, int t0, int count, cudaStream_t st) {
-  return c->mix ? launch_admm_loop<EigCfg, EpiTUpdate<true>, EpiProject<MODE, true>>(c, g, p1, p2, t0,
-                                                                                     count, st)
-                : launch_admm_loop<EigCfg3, EpiTUpdate<false>, EpiProject<MODE, false>>(c, g, p1, p2,
-                                                                                       t0, count, st);
+  if (c->enc == ENC_F16)
+    return launch_admm_loop<EigCfgF, EpiTUpdate<ENC_F16>, EpiProject<MODE, ENC_F16>>(c, g, p1, p2, t0,
+                                                                                     count, st);
+  if (c->enc == ENC_MIX)
+    return launch_admm_loop<EigCfg, EpiTUpdate<ENC_MIX>, EpiProject<MODE, ENC_MIX>>(c, g, p1, p2, t0,
+                                                                                    count, st);
+  return launch_admm_loop<EigCfg3, EpiTUpdate<ENC_TF32X3>, EpiProject<MODE, ENC_TF32X3>>(c, g, p1, p2,
+                                                                                         t0, count, st);
 }
 
 }  // namespace
@@ -842,6 +910,7 @@ const char* admmq_status_string(int s) {
     case ADMMQ_ERR_TIMEOUT: return "kernel pipeline wait timed out";
     case ADMMQ_ERR_WORKSPACE: return "workspace too small";
     case ADMMQ_ERR_UNSUPPORTED: return "unsupported device or shape";
+    case ADMMQ_ERR_RANGE: return "an fp16-split operand left fp16's range";
     default: return "unknown status";
   }
 }
@@ -875,7 +944,7 @@ int admmq_build_hessian(const void* X, int64_t n, int d, float* H, int accumulat
   float* part = (float*)((uint8_t*)ws + 256);
   CK(cudaMemsetAsync(status, 0, 16, st));
   CUtensorMap mx;
-  if (!make_map(&mx, X, (uint64_t)d, (uint64_t)n, GramCfg::BK, false)) return ADMMQ_ERR_CUDA;
+  if (!make_map(&mx, X, (uint64_t)d, (uint64_t)n, GramCfg::BK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)) return ADMMQ_ERR_CUDA;
   GemmGeom g = make_geom(d, d, n, GramCfg::BN, GramCfg::BK, splits, true, status);
   EpiGramPartial::Params ep{part, (long long)d * d, d};
   CK((launch_gemm<GramCfg, EpiGramPartial>(mx, mx, mx, mx, g, ep, st)));
@@ -910,8 +979,10 @@ int admmq_create(admmq_ctx** out, int d, int m, const admmq_params* p, void* ws,
   c->m = m;
   c->p = *p;
   c->L = (1 << p->bits) - 1;
-  c->mix = p->split_mode == ADMMQ_SPLIT_MIXED ||
-           (p->split_mode == ADMMQ_SPLIT_AUTO && d >= kMixedFromDin);
+  c->enc = p->split_mode == ADMMQ_SPLIT_MIXED    ? ENC_MIX
+           : p->split_mode == ADMMQ_SPLIT_3XTF32 ? ENC_TF32X3
+           : p->split_mode == ADMMQ_SPLIT_F16    ? ENC_F16
+           : (d >= kSplitFromDin ? ENC_F16 : ENC_TF32X3);
   cudaGetDevice(&c->dev);
   c->ws = (uint8_t*)ws;
   c->ws_bytes = ws_bytes;
@@ -928,15 +999,15 @@ int admmq_create(admmq_ctx** out, int d, int m, const admmq_params* p, void* ws,
   c->work = (double*)(b + L.work);
   c->lwork = lwork;
   c->devinfo = (int*)(b + L.devinfo);
-  c->E_hi = (float*)(b + L.E_hi);
+  c->E_hi = (void*)(b + L.E_hi);
   c->E_lo = (void*)(b + L.E_lo);
-  c->Q_hi = (float*)(b + L.Q_hi);
+  c->Q_hi = (void*)(b + L.Q_hi);
   c->Q_lo = (void*)(b + L.Q_lo);
-  c->Wt_hi = (float*)(b + L.Wt_hi);
+  c->Wt_hi = (void*)(b + L.Wt_hi);
   c->Wt_lo = (void*)(b + L.Wt_lo);
-  c->P_hi = (float*)(b + L.P_hi);
+  c->P_hi = (void*)(b + L.P_hi);
   c->P_lo = (void*)(b + L.P_lo);
-  c->T_hi = (float*)(b + L.T_hi);
+  c->T_hi = (void*)(b + L.T_hi);
   c->T_lo = (void*)(b + L.T_lo);
   c->C0 = (float*)(b + L.C0);
   c->V = (float*)(b + L.V);
@@ -946,13 +1017,13 @@ int admmq_create(admmq_ctx** out, int d, int m, const admmq_params* p, void* ws,
   c->ready = (int*)(b + L.ready);
   c->tiles_eig = eig_tiles(m, d);
   bool ok = true;
-  ok &= make_map(&c->mWt[0], c->Wt_hi, d, m, kBM, true) && make_map(&c->mWt[1], c->Wt_lo, c->mix ? 2 * (uint64_t)d : (uint64_t)d, m, kBM, !c->mix);
-  ok &= make_map(&c->mP[0], c->P_hi, d, m, kBM, true) && make_map(&c->mP[1], c->P_lo, c->mix ? 2 * (uint64_t)d : (uint64_t)d, m, kBM, !c->mix);
-  ok &= make_map(&c->mT[0], c->T_hi, d, m, kBM, true) && make_map(&c->mT[1], c->T_lo, c->mix ? 2 * (uint64_t)d : (uint64_t)d, m, kBM, !c->mix);
-  ok &= make_map(&c->mE[0], c->E_hi, d, d, EigCfg::B_ROWS, true) &&
-        make_map(&c->mE[1], c->E_lo, c->mix ? 2 * (uint64_t)d : (uint64_t)d, d, EigCfg::B_ROWS, !c->mix);
-  ok &= make_map(&c->mQ[0], c->Q_hi, d, d, EigCfg::B_ROWS, true) &&
-        make_map(&c->mQ[1], c->Q_lo, c->mix ? 2 * (uint64_t)d : (uint64_t)d, d, EigCfg::B_ROWS, !c->mix);
+  c->row_in = (float*)(b + L.row_in);
+  c->row_out = (float*)(b + L.row_out);
+  ok &= make_plane_maps(c->mWt, c->Wt_hi, c->Wt_lo, d, m, kBM, c->enc);
+  ok &= make_plane_maps(c->mP, c->P_hi, c->P_lo, d, m, kBM, c->enc);
+  ok &= make_plane_maps(c->mT, c->T_hi, c->T_lo, d, m, kBM, c->enc);
+  ok &= make_plane_maps(c->mE, c->E_hi, c->E_lo, d, d, EigCfg::B_ROWS, c->enc);
+  ok &= make_plane_maps(c->mQ, c->Q_hi, c->Q_lo, d, d, EigCfg::B_ROWS, c->enc);
   if (!ok || cusolverDnCreate(&c->solver) != CUSOLVER_STATUS_SUCCESS) {
     delete c;
     return ADMMQ_ERR_CUDA;
@@ -982,12 +1053,18 @@ int admmq_prepare(admmq_ctx* c, const float* G, const void* W_hat, int w_dtype, 
   count_launch(), k_scale_hessian<<<grid_for((long long)d * d), 256, 0, st>>>(G, d, c->lam64, c->sig64, c->Ht);
   CK(cudaGetLastError());
   const long long md = (long long)m * d;
-  if (w_dtype == ADMMQ_DTYPE_F32)
-    count_launch(), k_scale_weights<float><<<grid_for(md), 256, 0, st>>>((const float*)W_hat, c->rsig, d, md,
-                                                         c->Wt_hi, c->Wt_lo, c->mix);
-  else
+  int* flag = c->status + 3;
+  if (w_dtype == ADMMQ_DTYPE_F32) {
+    count_launch(), k_row_scales<float><<<grid_for(m, 8), 256, 0, st>>>((const float*)W_hat, c->rsig, m, d,
+                                                                        c->enc, c->row_in, c->row_out);
+    count_launch(), k_scale_weights<float><<<grid_for(md), 256, 0, st>>>(
+        (const float*)W_hat, c->rsig, d, md, c->Wt_hi, c->Wt_lo, c->enc, c->row_in, flag);
+  } else {
+    count_launch(), k_row_scales<__nv_bfloat16><<<grid_for(m, 8), 256, 0, st>>>(
+        (const __nv_bfloat16*)W_hat, c->rsig, m, d, c->enc, c->row_in, c->row_out);
     count_launch(), k_scale_weights<__nv_bfloat16><<<grid_for(md), 256, 0, st>>>(
-        (const __nv_bfloat16*)W_hat, c->rsig, d, md, c->Wt_hi, c->Wt_lo, c->mix);
+        (const __nv_bfloat16*)W_hat, c->rsig, d, md, c->Wt_hi, c->Wt_lo, c->enc, c->row_in, flag);
+  }
   CK(cudaGetLastError());
   c->prepared = true;
   return ADMMQ_OK;
@@ -1009,7 +1086,7 @@ int admmq_eigh(admmq_ctx* c, void* stream) {
   count_launch(), k_eigvals<<<grid_for(d), 256, 0, st>>>(c->evals, d, c->lam32, c->status);
   CK(cudaGetLastError());
   count_launch(), k_split_eigvecs<<<dim3(cdiv(d, 32), cdiv(d, 32)), dim3(32, 8), 0, st>>>(c->Ht, d, c->E_hi, c->E_lo,
-                                                                          c->Q_hi, c->Q_lo, c->mix);
+                                                                          c->Q_hi, c->Q_lo, c->enc);
   CK(cudaGetLastError());
   int info = 0;
   CK(cudaMemcpyAsync(&info, c->devinfo, sizeof(int), cudaMemcpyDeviceToHost, st));
@@ -1040,19 +1117,19 @@ int admmq_init(admmq_ctx* c, uint8_t* codes, float* scale, float* zero, void* st
   cudaStream_t st = (cudaStream_t)stream;
   const int d = c->d, m = c->m;
   // C0' = Lambda Q^T W^~   (row j, column k)
-  GemmGeom g = make_geom(m, d, d, EigCfg::BN, EigCfg::BK, 1, false, c->status, EigCfg::UNIT_M);
-  EpiScaleStore::Params ep{c->C0, c->lam32, d};
-  CK((launch_eig<EpiScaleStore, EpiScaleStore>(c->mix, c->mWt, c->mE, g, ep,
-                                                                         st)));
+  GemmGeom g = eig_geom(c->enc, m, d, c->status);
+  EpiScaleStore::Params ep{c->C0, c->lam32, c->row_out, d};
+  CK((launch_eig<EpiScaleStore, EpiScaleStore, EpiScaleStore>(c->enc, c->mWt, c->mE, g, ep, st)));
   const long long groups = (long long)m * (d / c->p.group);
+  int* flag = c->status + 3;
   if (c->w_dtype == ADMMQ_DTYPE_F32)
     count_launch(), k_init_rtn<float><<<grid_for(groups, 128), 128, 0, st>>>(
         (const float*)c->W_hat, c->rsig, m, d, c->p.group, c->L, codes, scale, zero, c->V,
-        c->P_hi, c->P_lo, c->mix);
+        c->P_hi, c->P_lo, c->enc, c->row_in, flag);
   else
     count_launch(), k_init_rtn<__nv_bfloat16><<<grid_for(groups, 128), 128, 0, st>>>(
         (const __nv_bfloat16*)c->W_hat, c->rsig, m, d, c->p.group, c->L, codes, scale, zero,
-        c->V, c->P_hi, c->P_lo, c->mix);
+        c->V, c->P_hi, c->P_lo, c->enc, c->row_in, flag);
   CK(cudaGetLastError());
   if (c->p.iters > 0) {
     std::vector<float> rho(c->p.iters);
@@ -1073,8 +1150,9 @@ int admmq_iterate(admmq_ctx* c, int t0, int count, uint8_t* codes, float* scale,
   if (count == 0) return ADMMQ_OK;
   cudaStream_t st = (cudaStream_t)stream;
   const int d = c->d, m = c->m;
-  GemmGeom g = make_geom(m, d, d, EigCfg::BN, EigCfg::BK, 1, false, c->status, EigCfg::UNIT_M);
-  TUpdateParams p1{c->C0, c->lam32, c->T_hi, c->T_lo, 0.f, d};
+  GemmGeom g = eig_geom(c->enc, m, d, c->status);
+  int* flag = c->status + 3;
+  TUpdateParams p1{c->C0, c->lam32, c->T_hi, c->T_lo, c->row_in, c->row_out, flag, 0.f, d};
   ProjParams p2;
   p2.V = c->V;
   p2.codes = codes;
@@ -1082,6 +1160,9 @@ int admmq_iterate(admmq_ctx* c, int t0, int count, uint8_t* codes, float* scale,
   p2.zero = zero;
   p2.p_hi = c->P_hi;
   p2.p_lo = c->P_lo;
+  p2.row_in = c->row_in;
+  p2.row_out = c->row_out;
+  p2.flag = flag;
   p2.sig = c->sigma;
   p2.rsig = c->rsig;
   p2.hd = c->hdiag;
@@ -1137,26 +1218,27 @@ int admmq_iterate(admmq_ctx* c, int t0, int count, uint8_t* codes, float* scale,
       CK(cudaEventRecord(rec.a, st));
     }
     p1.rho = rho_at(c->p, t);
-    CK((launch_eig<EpiTUpdate<false>, EpiTUpdate<true>>(c->mix, c->mP, c->mE, g, p1, st)));
+    CK((launch_eig<EpiTUpdate<ENC_TF32X3>, EpiTUpdate<ENC_MIX>, EpiTUpdate<ENC_F16>>(c->enc, c->mP,
+                                                                                    c->mE, g, p1, st)));
     if (c->timing) CK(cudaEventRecord(rec.b, st));
     p2.part = c->resid_part + (size_t)t * c->tiles_eig * 8;
     cudaError_t e;
     switch (c->p.grid_mode) {
       case ADMMQ_GRID_MINMAX:
-        e = launch_eig<EpiProject<GRID_MINMAX, false>,
-                       EpiProject<GRID_MINMAX, true>>(c->mix, c->mT, c->mQ, g, p2, st);
+        e = launch_eig<EpiProject<GRID_MINMAX, ENC_TF32X3>, EpiProject<GRID_MINMAX, ENC_MIX>,
+                       EpiProject<GRID_MINMAX, ENC_F16>>(c->enc, c->mT, c->mQ, g, p2, st);
         break;
       case ADMMQ_GRID_LSQ:
-        e = launch_eig<EpiProject<GRID_LSQ, false>,
-                       EpiProject<GRID_LSQ, true>>(c->mix, c->mT, c->mQ, g, p2, st);
+        e = launch_eig<EpiProject<GRID_LSQ, ENC_TF32X3>, EpiProject<GRID_LSQ, ENC_MIX>,
+                       EpiProject<GRID_LSQ, ENC_F16>>(c->enc, c->mT, c->mQ, g, p2, st);
         break;
       case ADMMQ_GRID_MSE:
-        e = launch_eig<EpiProject<GRID_MSE, false>,
-                       EpiProject<GRID_MSE, true>>(c->mix, c->mT, c->mQ, g, p2, st);
+        e = launch_eig<EpiProject<GRID_MSE, ENC_TF32X3>, EpiProject<GRID_MSE, ENC_MIX>,
+                       EpiProject<GRID_MSE, ENC_F16>>(c->enc, c->mT, c->mQ, g, p2, st);
         break;
       default:
-        e = launch_eig<EpiProject<GRID_FROZEN, false>,
-                       EpiProject<GRID_FROZEN, true>>(c->mix, c->mT, c->mQ, g, p2, st);
+        e = launch_eig<EpiProject<GRID_FROZEN, ENC_TF32X3>, EpiProject<GRID_FROZEN, ENC_MIX>,
+                       EpiProject<GRID_FROZEN, ENC_F16>>(c->enc, c->mT, c->mQ, g, p2, st);
         break;
     }
     CK(e);
@@ -1178,19 +1260,19 @@ int admmq_finish(admmq_ctx* c, const uint8_t* codes, const float* scale, const f
   if (objective) {
     if (!codes || !scale || !zero) return ADMMQ_ERR_INVALID_ARG;
     const long long md = (long long)m * d;
+    int* flag = c->status + 3;
     if (c->w_dtype == ADMMQ_DTYPE_F32)
-      count_launch(), k_delta_planes<float><<<grid_for(md), 256, 0, st>>>((const float*)c->W_hat, codes, scale,
-                                                          zero, c->rsig, d, c->p.group, md,
-                                                          c->T_hi, c->T_lo, c->mix);
+      count_launch(), k_delta_planes<float><<<grid_for(md), 256, 0, st>>>(
+          (const float*)c->W_hat, codes, scale, zero, c->rsig, d, c->p.group, md, c->T_hi, c->T_lo,
+          c->enc, c->row_in, flag);
     else
       count_launch(), k_delta_planes<__nv_bfloat16><<<grid_for(md), 256, 0, st>>>(
           (const __nv_bfloat16*)c->W_hat, codes, scale, zero, c->rsig, d, c->p.group, md, c->T_hi,
-          c->T_lo, c->mix);
+          c->T_lo, c->enc, c->row_in, flag);
     CK(cudaGetLastError());
-    GemmGeom g = make_geom(m, d, d, EigCfg::BN, EigCfg::BK, 1, false, c->status, EigCfg::UNIT_M);
-    EpiObjective::Params ep{c->lam32, c->obj_part};
-    CK((launch_eig<EpiObjective, EpiObjective>(c->mix, c->mT, c->mE, g, ep,
-                                                                         st)));
+    GemmGeom g = eig_geom(c->enc, m, d, c->status);
+    EpiObjective::Params ep{c->lam32, c->row_out, c->obj_part};
+    CK((launch_eig<EpiObjective, EpiObjective, EpiObjective>(c->enc, c->mT, c->mE, g, ep, st)));
     count_launch(), k_reduce_objective<<<1, 256, 0, st>>>(c->obj_part, c->tiles_eig * 4, objective);
     CK(cudaGetLastError());
   }
@@ -1251,6 +1333,8 @@ int admmq_get_buffer(admmq_ctx* c, int which, void** ptr, size_t* bytes) {
     case ADMMQ_BUF_E_LO: p = c->E_lo; b = 4 * dd; break;
     case ADMMQ_BUF_HT: p = c->Ht; b = 8 * dd; break;
     case ADMMQ_BUF_STATUS: p = c->status; b = 16; break;
+    case ADMMQ_BUF_ROW_IN: p = c->row_in; b = 4 * (size_t)c->m; break;
+    case ADMMQ_BUF_ROW_OUT: p = c->row_out; b = 4 * (size_t)c->m; break;
     default: return ADMMQ_ERR_INVALID_ARG;
   }
   *ptr = p;
@@ -1295,29 +1379,35 @@ int admmq_get_timing(admmq_ctx* c, double ms[2], int launches[2], int* iters_tim
 
 int admmq_project(const float* wt, float* V, const float* sig, const float* rsig,
                   const float* hd, int d, int m, int bits, int g, int mode, int split,
-                  uint8_t* codes, float* scale, float* zero, float* p_hi, void* p_lo,
-                  double* resid, void* stream) {
+                  uint8_t* codes, float* scale, float* zero, void* p_hi, void* p_lo,
+                  const float* row_scale, int* range_flag, double* resid, void* stream) {
   if (!wt || !V || !sig || !rsig || !hd || !codes || !scale || !zero || !p_hi || !p_lo || !resid)
     return ADMMQ_ERR_INVALID_ARG;
   if (d <= 0 || m <= 0 || d % 32 != 0 || !(g == 32 || g == 64 || g == 128) || d % g != 0 ||
       bits < 1 || bits > 8 || mode < ADMMQ_GRID_MINMAX || mode > ADMMQ_GRID_MSE ||
-      !(split == ADMMQ_SPLIT_3XTF32 || split == ADMMQ_SPLIT_MIXED))
+      !(split == ADMMQ_SPLIT_3XTF32 || split == ADMMQ_SPLIT_MIXED || split == ADMMQ_SPLIT_F16))
     return ADMMQ_ERR_INVALID_ARG;
   if (!aligned32(V) || !aligned32(codes) || !aligned32(p_hi) || !aligned32(p_lo) ||
-      ((uintptr_t)wt & 15) || ((uintptr_t)sig & 31) || ((uintptr_t)rsig & 31) || ((uintptr_t)hd & 31))
+      ((uintptr_t)wt & 15) || ((uintptr_t)sig & 31) || ((uintptr_t)rsig & 31) || ((uintptr_t)hd & 31) ||
+      ((uintptr_t)row_scale & 3) || ((uintptr_t)range_flag & 3))
     return ADMMQ_ERR_INVALID_ARG;
   cudaStream_t st = (cudaStream_t)stream;
   CK(cudaMemsetAsync(resid, 0, 2 * sizeof(double), st));
   dim3 grid(cdiv(m, 128), d / g);
   const int L = (1 << bits) - 1;
-  const bool mix = split == ADMMQ_SPLIT_MIXED;
-#define PROJECT_CASE(MODE)                                                                   \
-  if (mix)                                                                                   \
-    count_launch(), k_project<MODE, true><<<grid, 128, 0, st>>>(wt, V, sig, rsig, hd, m, d, g, L, \
-                                                                codes, scale, zero, p_hi, p_lo, resid); \
-  else                                                                                       \
-    count_launch(), k_project<MODE, false><<<grid, 128, 0, st>>>(wt, V, sig, rsig, hd, m, d, g, L, \
-                                                                 codes, scale, zero, p_hi, p_lo, resid);
+  const int enc = split == ADMMQ_SPLIT_MIXED ? ENC_MIX : (split == ADMMQ_SPLIT_F16 ? ENC_F16 : ENC_TF32X3);
+#define PROJECT_ENC(MODE, ENC)                                                                  \
+  count_launch(), k_project<MODE, ENC><<<grid, 128, 0, st>>>(wt, V, sig, rsig, hd, m, d, g, L, codes, \
+                                                             scale, zero, p_hi, p_lo, row_scale,     \
+                                                             range_flag, resid);
+#define PROJECT_CASE(MODE)       \
+  if (enc == ENC_MIX) {          \
+    PROJECT_ENC(MODE, ENC_MIX)   \
+  } else if (enc == ENC_F16) {   \
+    PROJECT_ENC(MODE, ENC_F16)   \
+  } else {                       \
+    PROJECT_ENC(MODE, ENC_TF32X3) \
+  }
   if (mode == ADMMQ_GRID_MINMAX) {
     PROJECT_CASE(GRID_MINMAX)
   } else if (mode == ADMMQ_GRID_LSQ) {
@@ -1328,13 +1418,25 @@ int admmq_project(const float* wt, float* V, const float* sig, const float* rsig
     PROJECT_CASE(GRID_FROZEN)
   }
 #undef PROJECT_CASE
+#undef PROJECT_ENC
   CK(cudaGetLastError());
   return ADMMQ_OK;
 }
 
 int admmq_split_mode(const admmq_ctx* c) {
   if (!c) return ADMMQ_ERR_INVALID_ARG;
-  return c->mix ? ADMMQ_SPLIT_MIXED : ADMMQ_SPLIT_3XTF32;
+  return c->enc == ENC_MIX ? ADMMQ_SPLIT_MIXED : (c->enc == ENC_F16 ? ADMMQ_SPLIT_F16 : ADMMQ_SPLIT_3XTF32);
+}
+
+int admmq_check(admmq_ctx* c, void* stream) {
+  if (!c) return ADMMQ_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  int host_status[4] = {0, 0, 0, 0};
+  CK(cudaMemcpyAsync(host_status, c->status, 16, cudaMemcpyDeviceToHost, st));
+  CK(cudaStreamSynchronize(st));
+  if (host_status[0] != KSTAT_OK) return ADMMQ_ERR_TIMEOUT;
+  if (host_status[3] != 0) return ADMMQ_ERR_RANGE;
+  return ADMMQ_OK;
 }
 
 // ------------------------------------------------------------------ GPTQ
@@ -1496,7 +1598,7 @@ extern "C" int admmq_build_hessian_static(const void* X, int64_t n, int d, float
   float* part = (float*)((uint8_t*)base + 256);
   CK(cudaMemsetAsync(status, 0, 16, st));
   CUtensorMap mx;
-  if (!make_map(&mx, X, (uint64_t)d, (uint64_t)n, GramCfg::BK, false)) return ADMMQ_ERR_CUDA;
+  if (!make_map(&mx, X, (uint64_t)d, (uint64_t)n, GramCfg::BK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)) return ADMMQ_ERR_CUDA;
   GemmGeom g = make_geom(d, d, n, GramCfg::BN, GramCfg::BK, splits, true, status);
   EpiGramPartial::Params ep{part, (long long)d * d, d};
   CK((launch_gemm<GramCfg, EpiGramPartial>(mx, mx, mx, mx, g, ep, st)));

@@ -14,6 +14,12 @@
 //     one tf32 MMA on plane 0 and one bf16 MMA on plane 1, whose K = 16 runs
 //     over hi(A).lo(B) and lo(A).hi(B): the same three terms in ~2/3 of the
 //     tensor time, the correction terms carried to bf16 precision.
+//   fp16 x3 (KIND_F16X3): planes hi = fp16(x s), lo = fp16(x s - hi) for a
+//     power-of-two scale s chosen by the encoder (fp16's range is narrow);
+//     each K step issues hi*hi + hi*lo + lo*hi as three kind::f16 MMAs.
+//     fp16 products are exact in the fp32 accumulator and hi + lo carries 22
+//     bits, as in 3xTF32, at the full 16-bit rate: 3 bf16-MMA units of
+//     tensor time per product against 4 for the mixed split.
 //
 // Promoted accumulation.  The tensor core adds every MMA into its fp32
 // accumulator with a small one-sided rounding error, so a long K sum drifts by
@@ -66,12 +72,12 @@ struct GemmGeom {
 // Operand kinds: KIND_BF16 / KIND_TF32 are the instruction-descriptor formats
 // of plain products.  KIND_MIX is the split-precision product with one tf32
 // plane and one bf16 correction plane per operand (see above).
-enum { KIND_BF16 = 1, KIND_TF32 = 2, KIND_MIX = 3 };
+enum { KIND_BF16 = 1, KIND_TF32 = 2, KIND_MIX = 3, KIND_F16X3 = 4 };
 
 template <int KIND_, int NPL_, bool A_MN_, bool B_MN_, int STAGES_, int KC_, bool PAIR_>
 struct GemmCfg {
   static constexpr int KIND = KIND_;
-  static constexpr int ELEM = KIND == KIND_BF16 ? 2 : 4;  // bytes per (plane-0) operand element
+  static constexpr int ELEM = (KIND == KIND_BF16 || KIND == KIND_F16X3) ? 2 : 4;  // bytes per (plane-0) element
   static constexpr int BM = 128, BN = 256, BK = 128 / ELEM, NPL = NPL_, STAGES = STAGES_;
   static constexpr int UK = 32 / ELEM;                     // K per MMA instruction
   static constexpr int KC = KC_;                           // k-blocks per promoted chunk
@@ -94,10 +100,14 @@ struct GemmCfg {
   static constexpr int SMEM = STAGES * STAGE + 1024 + BAR_BYTES;
   static_assert(!PAIR || (!A_MN && !B_MN), "CTA pairs: K-major operands");
   static_assert(KIND != KIND_MIX || (NPL == 2 && !A_MN && !B_MN), "mixed split: two K-major planes");
-  // products per K step: 3xTF32 (hi.hi, hi.lo, lo.hi), mixed (tf32 hi.hi +
-  // one bf16 product over the [hi|lo] x [lo|hi] correction row), or one
+  // products per K step: 3xTF32 / fp16 x3 (hi.hi, hi.lo, lo.hi), mixed (tf32
+  // hi.hi + one bf16 product over the [hi|lo] x [lo|hi] correction row), or one
   static constexpr int PRODUCTS = KIND == KIND_MIX ? 2 : (NPL == 2 ? 3 : 1);
+  static_assert(KIND != KIND_F16X3 || NPL == 2, "fp16 x3: two planes");
   static_assert(SMEM <= 232448, "shared memory budget");
+  // instruction-descriptor A/B format: kind::f16 takes 0 = f16, 1 = bf16;
+  // kind::tf32 takes 2
+  static constexpr uint32_t FMT = KIND == KIND_F16X3 ? 0u : (KIND == KIND_BF16 ? 1u : 2u);
 };
 
 // Unit -> (tile row, tile column, k-block range).  Splits are the outer index
@@ -317,8 +327,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     // --------------------------------------------------------- MMA issuer
     // (a pair's MMAs, 256 rows of the unit, are issued by its leader alone)
     if (lane == 0 && (!Cfg::PAIR || rank == 0)) {
-      constexpr uint32_t IDESC = idesc_f32acc(Cfg::KIND == KIND_MIX ? (uint32_t)KIND_TF32 : Cfg::KIND,
-                                              Cfg::UNIT_M, BN, Cfg::A_MN, Cfg::B_MN);
+      constexpr uint32_t IDESC = idesc_f32acc(Cfg::FMT, Cfg::UNIT_M, BN, Cfg::A_MN, Cfg::B_MN);
       constexpr uint32_t IDESC16 = idesc_f32acc(KIND_BF16, Cfg::UNIT_M, BN, Cfg::A_MN, Cfg::B_MN);
       // a completed group of MMAs is announced on the barrier at the same
       // offset in each CTA of the pair (or in this CTA)
@@ -381,16 +390,18 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                 const uint64_t ad = a0 + (uint64_t)(pa * kAPlane + kk * kKStepA);
                 const uint64_t bd = b0 + (uint64_t)(pb * kBPlane + kk * kKStepB);
                 const uint32_t accum = (kk > 0 || pr > 0) ? 1u : acc0;
-                const bool b16 = Cfg::KIND == KIND_BF16 || (Cfg::KIND == KIND_MIX && pr == 1);
+                // a kind::f16 MMA (bf16 or fp16 operands) or a kind::tf32 one
+                const bool b16 = Cfg::KIND == KIND_BF16 || Cfg::KIND == KIND_F16X3 ||
+                                 (Cfg::KIND == KIND_MIX && pr == 1);
                 const uint32_t id = Cfg::KIND == KIND_MIX && pr == 1 ? IDESC16 : IDESC;
                 if (Cfg::PAIR) {
                   if (b16)
-                    mma_bf16_pair(dt, ad, bd, id, accum);
+                    mma_f16_pair(dt, ad, bd, id, accum);
                   else
                     mma_tf32_pair(dt, ad, bd, id, accum);
                 } else {
                   if (b16)
-                    mma_bf16(dt, ad, bd, id, accum);
+                    mma_f16(dt, ad, bd, id, accum);
                   else
                     mma_tf32(dt, ad, bd, id, accum);
                 }

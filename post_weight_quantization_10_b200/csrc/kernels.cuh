@@ -2,6 +2,7 @@
 // layer solve (everything that is not the tcgen05 main loop).
 #pragma once
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include "gemm.cuh"
@@ -25,12 +26,23 @@ __device__ __forceinline__ float tf32_rne(float x) {
   b = (b + 0xFFFu + ((b >> 13) & 1u)) & ~0x1FFFu;
   return __uint_as_float(b);
 }
-// Operand encodings of the eigenbasis GEMMs.  Plane 0 always holds
-// hi = tf32(x) in an fp32 word.  Plane 1:
-//   3xTF32 (GemmCfg KIND_TF32, NPL 2): lo = tf32(x - hi), fp32 [rows][K];
-//   mixed  (GemmCfg KIND_MIX): bf16(hi) and bf16(lo), lo = x - hi (exact in
-//          float32), in correction rows of 64 bf16 per 32 columns,
-//          [rows][2K]: A operands [hi x32 | lo x32], B operands [lo x32 | hi x32].
+// Operand encodings of the eigenbasis GEMMs (ENC_*, selected by the split
+// precision):
+//   ENC_TF32X3 (GemmCfg KIND_TF32): plane 0 hi = tf32(x) in fp32 words,
+//     plane 1 lo = tf32(x - hi), both fp32 [rows][K];
+//   ENC_MIX (KIND_MIX): plane 0 hi = tf32(x) fp32 [rows][K]; plane 1 bf16(hi)
+//     and bf16(lo), lo = x - hi (exact in float32), in correction rows of 64
+//     bf16 per 32 columns, [rows][2K]: A operands [hi x32 | lo x32], B
+//     operands [lo x32 | hi x32];
+//   ENC_F16 (KIND_F16X3): plane 0 hi = fp16(x s), plane 1 lo = fp16(x s - hi),
+//     both u16 [rows][K], with a power-of-two scale s: 2^14 for B operands
+//     (eigenvector entries, |x| <= 1) and the row's own scale for A operands
+//     (see k_row_scales); a scaled value at or beyond fp16's largest finite
+//     value raises the range flag instead of passing as infinity.
+enum { ENC_TF32X3 = 0, ENC_MIX = 1, ENC_F16 = 2 };
+constexpr int kBScaleExp = 14;       // B operands of the fp16 split are scaled by 2^14
+constexpr float kF16Limit = 65504.f;  // largest finite fp16
+
 // x ~= hi + lo: hi = tf32(x), lo = tf32(x - hi)  (the 3xTF32 planes).
 __device__ __forceinline__ void split2(float x, float& hi, float& lo) {
   hi = tf32_rne(x);
@@ -41,13 +53,20 @@ __device__ __forceinline__ void split_mix(float x, float& hi, uint16_t& hb, uint
   hb = bf16_bits(hi);
   lb = bf16_bits(__fsub_rn(x, hi));
 }
+// fp16 pair of an already scaled value: hi = fp16(xs), lo = fp16(xs - hi)
+// (xs - hi is exact in float32); both round to nearest even.
+__device__ __forceinline__ void split_f16(float xs, uint16_t& hb, uint16_t& lb) {
+  const __half h = __float2half_rn(xs);
+  hb = __half_as_ushort(h);
+  lb = __half_as_ushort(__float2half_rn(__fsub_rn(xs, __half2float(h))));
+}
 // Index of column c's hi entry in its correction row (lo is 32 further on
 // for A operands, 32 before for B operands).
 __device__ __forceinline__ long long cplane_hi(long long c, bool b_side) {
   return 64 * (c >> 5) + (c & 31) + (b_side ? 32 : 0);
 }
-// Eight consecutive bf16 (16 bytes, 16-byte aligned).
-__device__ __forceinline__ void st_bf16x8(uint16_t* p, const uint16_t (&v)[8]) {
+// Eight consecutive 16-bit words (16 bytes, 16-byte aligned).
+__device__ __forceinline__ void st_u16x8(uint16_t* p, const uint16_t (&v)[8]) {
   uint4 u;
   u.x = (uint32_t)v[0] | ((uint32_t)v[1] << 16);
   u.y = (uint32_t)v[2] | ((uint32_t)v[3] << 16);
@@ -55,45 +74,102 @@ __device__ __forceinline__ void st_bf16x8(uint16_t* p, const uint16_t (&v)[8]) {
   u.w = (uint32_t)v[6] | ((uint32_t)v[7] << 16);
   *reinterpret_cast<uint4*>(p) = u;
 }
-// Plane-1 address of row `row` (ld = K columns) in either encoding.
-template <bool MIX>
-__device__ __forceinline__ void* lo_row(void* plane1, long long row, int ld) {
-  return MIX ? (void*)(reinterpret_cast<uint16_t*>(plane1) + row * 2 * ld)
-             : (void*)(reinterpret_cast<float*>(plane1) + row * ld);
+// Start of row `row` (K = ld columns) in plane 0 / plane 1 of an encoding.
+__device__ __forceinline__ void* plane0_row(int enc, void* p0, long long row, int ld) {
+  return enc == ENC_F16 ? (void*)(reinterpret_cast<uint16_t*>(p0) + row * ld)
+                        : (void*)(reinterpret_cast<float*>(p0) + row * ld);
+}
+__device__ __forceinline__ void* plane1_row(int enc, void* p1, long long row, int ld) {
+  return enc == ENC_TF32X3 ? (void*)(reinterpret_cast<float*>(p1) + row * ld)
+                           : (void*)(reinterpret_cast<uint16_t*>(p1) + row * (enc == ENC_MIX ? 2 : 1) * ld);
+}
+// The same for column c (c % 32 == 0 for the mixed correction rows).
+__device__ __forceinline__ void* plane0_at(int enc, void* p0, long long row, int ld, long long c) {
+  return enc == ENC_F16 ? (void*)(reinterpret_cast<uint16_t*>(p0) + row * ld + c)
+                        : (void*)(reinterpret_cast<float*>(p0) + row * ld + c);
+}
+__device__ __forceinline__ void* plane1_at(int enc, void* p1, long long row, int ld, long long c) {
+  if (enc == ENC_TF32X3) return reinterpret_cast<float*>(p1) + row * ld + c;
+  if (enc == ENC_MIX) return reinterpret_cast<uint16_t*>(p1) + row * 2 * ld + 2 * c;
+  return reinterpret_cast<uint16_t*>(p1) + row * ld + c;
 }
 // Columns c..c+7 (c % 8 == 0) of one A-side operand row in the encoding:
-// hi_row / lo_row point at the row's start in planes 0 / 1.
-template <bool MIX>
-__device__ __forceinline__ void put_operand8(float* hi_row, void* lo_row_p, long long c,
-                                             const float (&x)[8]) {
+// hi_row / lo_row point at the row's (or the column block's) start in planes
+// 0 / 1; s is the row's scale (fp16 split only), flag the range flag.
+template <int ENC>
+__device__ __forceinline__ void put_operand8(void* hi_row, void* lo_row, long long c,
+                                             const float (&x)[8], float s, int* flag) {
+  if (ENC == ENC_F16) {
+    uint16_t hb[8], lb[8];
+    bool bad = false;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float xs = __fmul_rn(x[k], s);
+      bad |= !(fabsf(xs) < kF16Limit);
+      split_f16(xs, hb[k], lb[k]);
+    }
+    st_u16x8(reinterpret_cast<uint16_t*>(hi_row) + c, hb);
+    st_u16x8(reinterpret_cast<uint16_t*>(lo_row) + c, lb);
+    if (bad && flag) *flag = 1;
+    return;
+  }
   float hi[8];
-  if (MIX) {
+  if (ENC == ENC_MIX) {
     uint16_t hb[8], lb[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) split_mix(x[k], hi[k], hb[k], lb[k]);
-    uint16_t* cr = reinterpret_cast<uint16_t*>(lo_row_p) + cplane_hi(c, false);
-    st_bf16x8(cr, hb);
-    st_bf16x8(cr + 32, lb);
+    uint16_t* cr = reinterpret_cast<uint16_t*>(lo_row) + cplane_hi(c, false);
+    st_u16x8(cr, hb);
+    st_u16x8(cr + 32, lb);
   } else {
     float lo[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) split2(x[k], hi[k], lo[k]);
-    st_v8f(reinterpret_cast<float*>(lo_row_p) + c, lo);
+    st_v8f(reinterpret_cast<float*>(lo_row) + c, lo);
   }
-  st_v8f(hi_row + c, hi);
+  st_v8f(reinterpret_cast<float*>(hi_row) + c, hi);
 }
-// One element (column c of a row) in the encoding, for element-wise kernels.
-// `lo_from` is the value whose rounding is stored as lo (x - hi, or a more
-// accurate residual when the source is float64).
-__device__ __forceinline__ void put_operand1(bool mix, bool b_side, float* hi_row, void* lo_row_p,
-                                             long long c, float hi, float lo_from) {
-  hi_row[c] = hi;
-  if (mix) {
-    uint16_t* cr = reinterpret_cast<uint16_t*>(lo_row_p) + cplane_hi(c, b_side);
-    cr[0] = bf16_bits(hi);
-    cr[b_side ? -32 : 32] = bf16_bits(lo_from);
+// One A-side element (column c of a row) for element-wise kernels.
+__device__ __forceinline__ void put_a1(int enc, void* hi_row, void* lo_row, long long c, float x,
+                                       float s, int* flag) {
+  if (enc == ENC_F16) {
+    const float xs = __fmul_rn(x, s);
+    if (!(fabsf(xs) < kF16Limit) && flag) *flag = 1;
+    uint16_t hb, lb;
+    split_f16(xs, hb, lb);
+    reinterpret_cast<uint16_t*>(hi_row)[c] = hb;
+    reinterpret_cast<uint16_t*>(lo_row)[c] = lb;
+    return;
+  }
+  const float h = tf32_rne(x), lo = __fsub_rn(x, h);
+  reinterpret_cast<float*>(hi_row)[c] = h;
+  if (enc == ENC_MIX) {
+    uint16_t* cr = reinterpret_cast<uint16_t*>(lo_row) + cplane_hi(c, false);
+    cr[0] = bf16_bits(h);
+    cr[32] = bf16_bits(lo);
   } else {
-    reinterpret_cast<float*>(lo_row_p)[c] = tf32_rne(lo_from);
+    reinterpret_cast<float*>(lo_row)[c] = tf32_rne(lo);
+  }
+}
+// One B-side element from a float64 value (eigenvectors): the low part is
+// taken from the float64 residual.
+__device__ __forceinline__ void put_b1(int enc, void* hi_row, void* lo_row, long long c, double e) {
+  if (enc == ENC_F16) {
+    const double xs = e * (double)(1 << kBScaleExp);
+    const __half h = __double2half(xs);
+    reinterpret_cast<uint16_t*>(hi_row)[c] = __half_as_ushort(h);
+    reinterpret_cast<uint16_t*>(lo_row)[c] =
+        __half_as_ushort(__double2half(xs - (double)__half2float(h)));
+    return;
+  }
+  const float h = tf32_rne((float)e), lo = (float)(e - (double)h);
+  reinterpret_cast<float*>(hi_row)[c] = h;
+  if (enc == ENC_MIX) {
+    uint16_t* cr = reinterpret_cast<uint16_t*>(lo_row) + cplane_hi(c, true);
+    cr[0] = bf16_bits(h);
+    cr[-32] = bf16_bits(lo);
+  } else {
+    reinterpret_cast<float*>(lo_row)[c] = tf32_rne(lo);
   }
 }
 // clamp to [0, L]; adding +0 turns a -0 into +0 so the result never depends
@@ -135,11 +211,13 @@ struct ProjRow {
   const float* rsig;
   const float* hd;
   uint8_t* codes;
-  float* phi;          // P plane 0 at the group's first column
-  void* plo;           // P plane 1 at the group's first column (either encoding)
+  void* phi;           // P plane 0 at the group's first column (any encoding)
+  void* plo;           // P plane 1 at the group's first column
   float* scale;        // this group's scale / zero
   float* zero;
   float* wdump;        // optional raw W~ output
+  float rs;            // the row's operand scale (fp16 split; 1 otherwise)
+  int* flag;           // range flag of the fp16 split
   bool valid;
 };
 
@@ -206,7 +284,7 @@ __device__ __forceinline__ void mse_clip_grid(LoadW& loadw, const ProjRow& r, in
   }
 }
 
-template <int MODE, bool MIX, class LoadW>
+template <int MODE, int ENC, class LoadW>
 __device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, int g, int L,
                                               float& r2, float& s2) {
   const float Lf = (float)L;
@@ -306,7 +384,7 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, i
       }
       if (r.valid) {
         st_v8f(r.V + c + e, vn);
-        put_operand8<MIX>(r.phi, r.plo, c + e, pv);  // P, A side
+        put_operand8<ENC>(r.phi, r.plo, c + e, pv, r.rs, r.flag);  // P, A side
         if (r.wdump) {
           float wd[8];
 #pragma unroll
@@ -367,6 +445,7 @@ struct EpiScaleStore {
   struct Params {
     float* out;
     const float* lam;
+    const float* row_out;  // per-row factor that unscales the GEMM result
     int ld;
   };
   // From registers: 128 columns of tile row `rit`, starting at column col0.
@@ -375,6 +454,7 @@ struct EpiScaleStore {
     const int row = tm * 128 + rit;
     if (row >= g.M) return;
     float* o = p.out + (long long)row * p.ld;
+    const float ro = p.row_out[row];
 #pragma unroll
     for (int c = 0; c < 128; c += 8) {
       const int col = col0 + c;
@@ -382,7 +462,7 @@ struct EpiScaleStore {
         float l[8], v[8];
         load8_ro(p.lam + col, l);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) v[k] = __fmul_rn(l[k], acc[c + k]);
+        for (int k = 0; k < 8; ++k) v[k] = __fmul_rn(l[k], __fmul_rn(acc[c + k], ro));
         st_v8f(o + col, v);
       }
     }
@@ -394,13 +474,16 @@ struct EpiScaleStore {
 struct TUpdateParams {
   const float* c0;
   const float* lam;
-  float* t_hi;
-  void* t_lo;      // plane 1 (encoding per the epilogue's MIX)
+  void* t_hi;             // plane 0 (encoding per the epilogue's ENC)
+  void* t_lo;             // plane 1
+  const float* row_in;    // per-row operand scale of the fp16 split (1 otherwise)
+  const float* row_out;   // per-row factor that unscales a GEMM result row
+  int* flag;              // range flag of the fp16 split
   float rho;
   int ld;
 };
 
-template <bool MIX>
+template <int ENC>
 struct EpiTUpdate {
   static constexpr bool FROM_TMEM = false;
   using Params = TUpdateParams;
@@ -409,7 +492,9 @@ struct EpiTUpdate {
     const int row = tm * 128 + rit;
     if (row >= g.M) return;
     const long long rb = (long long)row * p.ld;
-    void* lo = lo_row<MIX>(p.t_lo, row, p.ld);
+    void* hi = plane0_row(ENC, p.t_hi, row, p.ld);
+    void* lo = plane1_row(ENC, p.t_lo, row, p.ld);
+    const float ro = p.row_out[row], ri = p.row_in[row];
 #pragma unroll
     for (int c = 0; c < 128; c += 8) {
       const int col = col0 + c;
@@ -420,9 +505,10 @@ struct EpiTUpdate {
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const float inv = __frcp_rn(__fadd_rn(ll[j], p.rho));
-          tv[j] = __fmul_rn(__fadd_rn(cc[j], __fmul_rn(p.rho, acc[c + j])), inv);
+          const float a = __fmul_rn(acc[c + j], ro);
+          tv[j] = __fmul_rn(__fadd_rn(cc[j], __fmul_rn(p.rho, a)), inv);
         }
-        put_operand8<MIX>(p.t_hi + rb, lo, col, tv);
+        put_operand8<ENC>(hi, lo, col, tv, ri, p.flag);
       }
     }
   }
@@ -435,8 +521,11 @@ struct ProjParams {
   uint8_t* codes;
   float* scale;
   float* zero;
-  float* p_hi;
-  void* p_lo;     // plane 1 (encoding per the epilogue's MIX)
+  void* p_hi;     // plane 0 (encoding per the epilogue's ENC)
+  void* p_lo;     // plane 1
+  const float* row_in;    // per-row operand scale of the fp16 split (1 otherwise)
+  const float* row_out;   // per-row factor that unscales W~ = Q T
+  int* flag;              // range flag of the fp16 split
   const float* sig;
   const float* rsig;
   const float* hd;
@@ -447,7 +536,7 @@ struct ProjParams {
   int L;
 };
 
-template <int MODE, bool MIX>
+template <int MODE, int ENC>
 struct EpiProject {
   // The projection keeps a whole group of one row in flight twice (refit and
   // projection passes): it reads the tile from tensor memory, where the
@@ -460,6 +549,8 @@ struct EpiProject {
     const int row = tm * 128 + rit;
     const bool valid = row < g.M;
     const int ngrp_row = p.ld / p.group;
+    const float ro = valid ? p.row_out[row] : 1.f;
+    const float ri = valid ? p.row_in[row] : 1.f;
     float r2 = 0.f, s2 = 0.f;
     for (int c0 = 0; c0 < 128; c0 += p.group) {
       const int col = col0 + c0;
@@ -472,16 +563,21 @@ struct EpiProject {
       r.rsig = p.rsig + col;
       r.hd = p.hd + col;
       r.codes = p.codes + off;
-      r.phi = p.p_hi + off;
-      r.plo = MIX ? (void*)(reinterpret_cast<uint16_t*>(p.p_lo) + (long long)(valid ? row : 0) * 2 * p.ld +
-                            2 * col)
-                  : (void*)(reinterpret_cast<float*>(p.p_lo) + off);
+      r.phi = plane0_at(ENC, p.p_hi, valid ? row : 0, p.ld, col);
+      r.plo = plane1_at(ENC, p.p_lo, valid ? row : 0, p.ld, col);
       r.scale = p.scale + goff;
       r.zero = p.zero + goff;
       r.wdump = p.wdump ? p.wdump + off : nullptr;
+      r.rs = ri;
+      r.flag = p.flag;
       r.valid = valid;
-      auto loadw = [&](int c, float (&w)[32]) { tmem_ld32(taddr + c0 + c, w); };
-      project_group<MODE, MIX>(loadw, r, p.group, p.L, r2, s2);
+      // W~ = Q T: the accumulator carries the operands' scales (exact powers of two)
+      auto loadw = [&](int c, float (&w)[32]) {
+        tmem_ld32(taddr + c0 + c, w);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) w[k] = __fmul_rn(w[k], ro);
+      };
+      project_group<MODE, ENC>(loadw, r, p.group, p.L, r2, s2);
     }
     r2 = warp_sum(r2);
     s2 = warp_sum(s2);
@@ -498,20 +594,25 @@ struct EpiObjective {
   static constexpr bool FROM_TMEM = false;
   struct Params {
     const float* lam;
-    float* part;  // [128-row tiles x 128-column tiles][4]
+    const float* row_out;  // per-row factor that unscales the GEMM result
+    float* part;           // [128-row tiles x 128-column tiles][4]
   };
   __device__ static void apply_regs(const Params& p, const GemmGeom& g, const float (&acc)[128],
                                     int tm, int, int, int rit, int col0) {
     const int row = tm * 128 + rit;
     float s = 0.f;
     if (row < g.M) {
+      const float ro = p.row_out[row];
 #pragma unroll
       for (int c = 0; c < 128; c += 8) {
         if (col0 + c < g.N) {
           float l[8];
           load8_ro(p.lam + col0 + c, l);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) s += l[k] * acc[c + k] * acc[c + k];
+          for (int k = 0; k < 8; ++k) {
+            const float a = __fmul_rn(acc[c + k], ro);
+            s += l[k] * a * a;
+          }
         }
       }
     }

@@ -161,8 +161,9 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem], bf16 inputs, fp32 accumulation.
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+// D[tmem] (+)= A[smem] * B[smem], kind::f16 (bf16 or fp16 inputs, same type
+// for A and B, as the descriptor says), fp32 accumulation.
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                          uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -185,7 +186,7 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint6
 
 // 2-SM MMA (issued by the pair leader): A rows split across the pair's shared
 // memories at the same offsets, B columns split likewise, D in both TMEMs.
-__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+__device__ __forceinline__ void mma_f16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                               uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -367,8 +368,8 @@ __device__ __forceinline__ bool wait_counter(const int* cnt, int target, volatil
   return true;
 }
 
-// Instruction descriptor with fp32 D: kind::f16 with bf16 A/B (fmt 1) or
-// kind::tf32 (fmt 2).
+// Instruction descriptor with fp32 D: kind::f16 with f16 A/B (fmt 0) or bf16
+// A/B (fmt 1), or kind::tf32 (fmt 2).
 __host__ __device__ constexpr uint32_t idesc_f32acc(uint32_t fmt, int M, int N, bool a_mn, bool b_mn) {
   return (1u << 4)                       // D format f32
          | (fmt << 7)                    // A format

@@ -86,17 +86,17 @@ def _solver(A, p, X, W, grid, split="auto"):
 
 
 @pytest.mark.parametrize("grid,split", [("lsq", "auto"), ("minmax", "auto"), ("mse", "auto"),
-                                        ("lsq", "3xtf32")])
+                                        ("lsq", "3xtf32"), ("lsq", "mixed")])
 def test_full_size_teacher_forced(A, full_setup, grid, split):
     """RTN start bit-exact on the sampled rows; then, at sampled iterations,
     the oracle's state of those rows is loaded into the GPU's state and one
     GPU iteration runs: W~ within 1e-4 relative, codes equal on >= 99.9%,
     mismatches one level apart where the grid agrees.  At this size the
-    automatic split precision is the mixed one; 3xTF32 is forced once."""
+    automatic split precision is the fp16 one; 3xTF32 and mixed are forced once each."""
     p, X, W, H, Wm, _, _ = full_setup
     res, trace = _oracle_run(full_setup, grid)
     s = _solver(A, p, X, W, grid, split)
-    assert s.split == ("3xtf32" if split == "3xtf32" else "mixed")
+    assert s.split == (split if split != "auto" else "f16")
     s.init()
     torch.cuda.synchronize()
     rows = torch.from_numpy(ROWS).cuda()
@@ -108,10 +108,11 @@ def test_full_size_teacher_forced(A, full_setup, grid, split):
     for t in STEPS:
         e = trace[t]
         if t > 0:
-            hi, lo = P.encode_operand((e["Dt"] - e["Vt"]).T.astype(np.float32), s.split, "A")
+            hi, lo = P.encode_operand((e["Dt"] - e["Vt"]).T.astype(np.float32), s.split, "A",
+                                      s.buffer("row_in")[rows].cpu().numpy())
             s.buffer("V")[rows] = cu(e["Vt"].T.astype(np.float32))
-            s.buffer("P_hi")[rows] = cu(hi)
-            s.buffer("P_lo")[rows] = cu(lo.view(np.int16) if s.split == "mixed" else lo)
+            s.buffer("P_hi")[rows] = cu(hi.view(np.int16) if s.split == "f16" else hi)
+            s.buffer("P_lo")[rows] = cu(lo.view(np.int16) if s.split in ("mixed", "f16") else lo)
             s.codes[rows] = cu(e["codes"].T)
             s.scale[rows] = cu(e["scale"].T.astype(np.float32))
             s.zero[rows] = cu(e["zero"].T.astype(np.float32))

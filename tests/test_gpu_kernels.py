@@ -81,32 +81,67 @@ def _proj_inputs(m, d, g, bits, seed):
     return dict(W=W, V=V, sig=sig, rsig=rsig, hd=hd, s0=s0, z0=z0, c0=c0)
 
 
-@pytest.mark.parametrize("split", ["mixed", "3xtf32"])
+@pytest.mark.parametrize("split", ["mixed", "3xtf32", "f16"])
 @pytest.mark.parametrize("grid", ["minmax", "lsq", "mse", "frozen"])
 @pytest.mark.parametrize("bits,g,m,d", [(3, 128, 200, 384), (2, 64, 33, 128), (4, 32, 130, 96),
                                         (3, 64, 32, 64)])
 def test_projection_kernel_bitexact(A, grid, bits, g, m, d, split):
     x = _proj_inputs(m, d, g, bits, seed=bits * 100 + g + m)
+    rng = np.random.default_rng(m + d)
+    # the fp16 split's per-row powers of two (1 for the other encodings)
+    rs = (np.ldexp(np.float32(1), rng.integers(-4, 5, m)).astype(np.float32) if split == "f16"
+          else None)
     ref = P.epilogue_step(x["W"], x["V"], x["sig"], x["rsig"], x["hd"], x["s0"], x["z0"], x["c0"],
-                          bits, g, grid, split)
+                          bits, g, grid, split, row_scale=rs)
     cu = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
     V = cu(x["V"])
     codes, scale, zero = cu(x["c0"]), cu(x["s0"]), cu(x["z0"])
-    phi = torch.empty((m, d), dtype=torch.float32, device="cuda")
-    plo = (torch.empty((m, 2 * d), dtype=torch.int16, device="cuda") if split == "mixed"
-           else torch.empty((m, d), dtype=torch.float32, device="cuda"))
+    if split == "f16":
+        phi = torch.empty((m, d), dtype=torch.int16, device="cuda")
+        plo = torch.empty((m, d), dtype=torch.int16, device="cuda")
+    else:
+        phi = torch.empty((m, d), dtype=torch.float32, device="cuda")
+        plo = (torch.empty((m, 2 * d), dtype=torch.int16, device="cuda") if split == "mixed"
+               else torch.empty((m, d), dtype=torch.float32, device="cuda"))
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
     resid = A.project(cu(x["W"]), V, cu(x["sig"]), cu(x["rsig"]), cu(x["hd"]), bits, g, grid,
-                      codes, scale, zero, phi, plo, split=split)
+                      codes, scale, zero, phi, plo, split=split,
+                      row_scale=cu(rs) if rs is not None else None, range_flag=flag)
     torch.cuda.synchronize()
     np.testing.assert_array_equal(codes.cpu().numpy(), ref["codes"])
     np.testing.assert_array_equal(scale.cpu().numpy().view(np.uint32), ref["scale"].view(np.uint32))
     np.testing.assert_array_equal(zero.cpu().numpy().view(np.uint32), ref["zero"].view(np.uint32))
     np.testing.assert_array_equal(V.cpu().numpy().view(np.uint32), ref["V"].view(np.uint32))
-    np.testing.assert_array_equal(phi.cpu().numpy().view(np.uint32), ref["P_hi"].view(np.uint32))
+    if split == "f16":
+        np.testing.assert_array_equal(phi.cpu().numpy().view(np.uint16), ref["P_hi"])
+    else:
+        np.testing.assert_array_equal(phi.cpu().numpy().view(np.uint32), ref["P_hi"].view(np.uint32))
     np.testing.assert_array_equal(plo.cpu().numpy().view(np.uint16), ref["P_lo"].view(np.uint16))
+    assert int(flag.item()) == 0
     r = resid.cpu().numpy()
     assert r[0] == pytest.approx(ref["r2"], rel=1e-4)
     assert r[1] == pytest.approx(ref["s2"], rel=1e-4, abs=1e-12)
+
+
+def test_projection_f16_range_flag(A):
+    """An fp16-split operand scaled past fp16's largest value raises the range
+    flag (the kernel writes the rounded planes and carries on)."""
+    m, d, g, bits = 40, 128, 64, 3
+    x = _proj_inputs(m, d, g, bits, seed=5)
+    cu = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    rs = np.ones(m, np.float32)
+    rs[7] = np.float32(2.0 ** 40)           # row 7's P entries land far past 65504
+    ref = P.epilogue_step(x["W"], x["V"], x["sig"], x["rsig"], x["hd"], x["s0"], x["z0"], x["c0"],
+                          bits, g, "lsq", "f16", row_scale=rs)
+    phi = torch.empty((m, d), dtype=torch.int16, device="cuda")
+    plo = torch.empty((m, d), dtype=torch.int16, device="cuda")
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    A.project(cu(x["W"]), cu(x["V"]), cu(x["sig"]), cu(x["rsig"]), cu(x["hd"]), bits, g, "lsq",
+              cu(x["c0"]), cu(x["s0"]), cu(x["z0"]), phi, plo, split="f16", row_scale=cu(rs),
+              range_flag=flag)
+    torch.cuda.synchronize()
+    assert int(flag.item()) == 1
+    np.testing.assert_array_equal(phi.cpu().numpy().view(np.uint16)[:7], ref["P_hi"][:7])
 
 
 # ------------------------------------------------------------------ packing

@@ -120,7 +120,7 @@ def test_first_iteration_w_update(A, name, grid):
     phi = torch.empty_like(s.buffer("P_hi"))
     plo = torch.empty_like(s.buffer("P_lo"))
     A.project(wt, V, s.buffer("sigma"), s.buffer("rsig"), s.buffer("hdiag"), p.bits, p.group,
-              grid, codes, scale, zero, phi, plo, split=s.split)
+              grid, codes, scale, zero, phi, plo, split=s.split, row_scale=s.buffer("row_in"))
     torch.cuda.synchronize()
     assert torch.equal(codes, s.codes) and torch.equal(scale, s.scale) and torch.equal(zero, s.zero)
     assert torch.equal(V, s.buffer("V"))
@@ -134,11 +134,11 @@ def _load_state(s, e):
     """Oracle state entering iteration t -> the GPU's state buffers."""
     Vt = e["Vt"].T.astype(np.float32)
     Pm = (e["Dt"] - e["Vt"]).T.astype(np.float32)
-    hi, lo = P.encode_operand(Pm, s.split, "A")
+    hi, lo = P.encode_operand(Pm, s.split, "A", s.buffer("row_in").cpu().numpy())
     cu = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
     s.buffer("V").copy_(cu(Vt))
-    s.buffer("P_hi").copy_(cu(hi))
-    s.buffer("P_lo").copy_(cu(lo.view(np.int16) if s.split == "mixed" else lo))
+    s.buffer("P_hi").copy_(cu(hi.view(np.int16) if s.split == "f16" else hi))
+    s.buffer("P_lo").copy_(cu(lo.view(np.int16) if s.split in ("mixed", "f16") else lo))
     s.codes.copy_(cu(e["codes"].T))
     s.scale.copy_(cu(e["scale"].T.astype(np.float32)))
     s.zero.copy_(cu(e["zero"].T.astype(np.float32)))
@@ -146,7 +146,8 @@ def _load_state(s, e):
 
 TEACHER_CASES = [(n, g, "auto") for n in ("tiny", "ragged", "down_small")
                  for g in ("minmax", "lsq", "mse", "frozen")] + \
-                [(n, g, "mixed") for n in ("tiny", "ragged") for g in ("minmax", "lsq", "mse")]
+                [(n, g, "mixed") for n in ("tiny", "ragged") for g in ("minmax", "lsq", "mse")] + \
+                [(n, g, "f16") for n in ("tiny", "ragged", "down_small") for g in ("lsq", "mse")]
 
 
 @pytest.mark.parametrize("name,grid,split", TEACHER_CASES)
@@ -155,8 +156,8 @@ def test_teacher_forced_iterations(A, name, grid, split):
     oracle's state (D~_t, V~_t, grid) is loaded into the GPU, one GPU iteration
     runs, and W~ must be within 1e-4 relative and the codes must agree on
     >= 99.9% of entries, mismatches being adjacent levels (decisions at a
-    rounding tie).  These small layers run 3xTF32 by default; the mixed split
-    is forced on two of them as well."""
+    rounding tie).  These small layers run 3xTF32 by default; the mixed and
+    fp16 splits are forced on them as well."""
     p, X, W = _layer(name)
     trace = []
     Xn = X.float().cpu().numpy()
@@ -164,7 +165,7 @@ def test_teacher_forced_iterations(A, name, grid, split):
     Wm = W.float().cpu().numpy().T.astype(np.float64)
     O.admm_q(H, Wm, p.bits, p.group, p.iters, rho0=p.rho0, gamma=p.gamma, grid=grid, trace=trace)
     s = _solver(A, p, X, W, grid, split=split)
-    assert s.split == ("mixed" if split == "mixed" else "3xtf32")
+    assert s.split == (split if split != "auto" else "3xtf32")
     s.init()
     wt = torch.empty((W.shape[0], X.shape[1]), dtype=torch.float32, device="cuda")
     s.dump_wtilde(wt)
@@ -245,7 +246,7 @@ def test_unscaled_ablation_teacher_forced(A, name):
 
 
 @pytest.mark.parametrize("name,grid,split", [("tiny", "lsq", "auto"), ("ragged", "lsq", "auto"),
-                                             ("ragged", "mse", "mixed"),
+                                             ("ragged", "mse", "mixed"), ("ragged", "lsq", "f16"),
                                              ("down_small", "minmax", "auto")])
 def test_fused_schedule_matches_per_gemm(A, name, grid, split):
     """The fused schedule runs GEMM 1 and GEMM 2 of all iterations in one
@@ -270,6 +271,7 @@ def test_fused_schedule_matches_per_gemm(A, name, grid, split):
             s.solve()
         torch.cuda.synchronize()
         assert s.kernel_status() == 0, sched
+        s.check()
         runs[sched] = {k: v.cpu().clone() for k, v in (
             ("codes", s.codes), ("scale", s.scale), ("zero", s.zero), ("V", s.buffer("V")),
             ("resid", s.resid), ("objective", s.objective))}

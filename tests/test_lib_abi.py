@@ -66,9 +66,11 @@ def test_alignment_checks_without_gpu(lib):
     rejects state buffers that are not 32-byte aligned before touching the
     device (the pointers below are never dereferenced)."""
     ok = [ctypes.c_void_p(0x10000 * (i + 1)) for i in range(12)]
-    # wt V sig rsig hd | d m bits g mode split | codes scale zero p_hi p_lo resid stream
-    def call(ptrs, split=2, mode=0):
-        return lib.admmq_project(*ptrs[:5], 256, 8, 3, 128, mode, split, *ptrs[5:11], None)
+    # wt V sig rsig hd | d m bits g mode split | codes scale zero p_hi p_lo | row_scale flag
+    # | resid stream
+    def call(ptrs, split=2, mode=0, row_scale=None, flag=None):
+        return lib.admmq_project(*ptrs[:5], 256, 8, 3, 128, mode, split, *ptrs[5:10], row_scale,
+                                 flag, ptrs[10], None)
     for k in (1, 5, 8, 9):  # V, codes, P_hi, P_lo off by 16 bytes
         bad = list(ok)
         bad[k] = ctypes.c_void_p(ok[k].value + 16)
@@ -76,8 +78,10 @@ def test_alignment_checks_without_gpu(lib):
     bad = list(ok)
     bad[0] = ctypes.c_void_p(ok[0].value + 8)  # W~ needs 16 bytes
     assert call(bad) == -1
-    for split in (0, 3, -1):                   # the kernel needs a concrete split precision
+    for split in (0, 4, -1):                   # the kernel needs a concrete split precision
         assert call(list(ok), split) == -1, split
+    assert call(list(ok), 3, row_scale=ctypes.c_void_p(0x10002)) == -1   # fp32 scales, 4-byte aligned
+    assert call(list(ok), 3, flag=ctypes.c_void_p(0x10001)) == -1
     for mode in (-1, 4):                       # grid modes are 0 (minmax) .. 3 (mse)
         assert call(list(ok), mode=mode) == -1, mode
     assert lib.admmq_split_mode(None) == -1

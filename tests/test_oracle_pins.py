@@ -386,6 +386,59 @@ def test_tf32_split_reconstructs_float32():
     np.testing.assert_array_equal(P.tf32_round(t), np.array([1.0, 1 + 2.0 ** -9], np.float32))
 
 
+def test_f16_split_encoding():
+    """fp16 split of the eigenbasis GEMMs' operands: hi = fp16(x s), lo =
+    fp16(x s - hi) with a power-of-two scale s.  Hand examples: 3 + 2^-9 + 2^-20
+    splits exactly into hi = 3 + 2^-9 (fp16 spacing 2^-9 on [2, 4)) and lo =
+    2^-20 (an fp16 subnormal, 16 * 2^-24); an eigenvector entry 1 scaled by 2^14
+    is 16384; 4 * 2^14 = 65536 is past fp16's largest value and raises the
+    flag.  On random data hi + lo keeps 22 bits and the three fp16 products
+    hi.hi + hi.lo + lo.hi give the dot product to ~2^-20."""
+    t = np.zeros((1, 8), np.float32)
+    t[0, 0] = np.float32(3 + 2.0 ** -9 + 2.0 ** -20)
+    t[0, 1] = 1.0
+    hi, lo, bad = P.split_f16(t, np.float32(1.0))
+    assert not bad
+    assert hi.view(np.float16)[0, 0] == np.float16(3 + 2.0 ** -9)
+    assert lo.view(np.float16)[0, 0].astype(np.float64) == 2.0 ** -20
+    h2, l2, bad2 = P.split_f16(t, P.F16_B_SCALE)
+    assert not bad2 and h2.view(np.float16)[0, 1] == 16384.0 and l2.view(np.float16)[0, 1] == 0.0
+    t[0, 2] = 4.0
+    assert P.split_f16(t, P.F16_B_SCALE)[2]
+    rng = np.random.default_rng(13)
+    x = (rng.standard_normal((6, 256)) * np.exp(rng.standard_normal((6, 256)))).astype(np.float32)
+    s = P.row_scales_f16(x)
+    h, l, bad = P.split_f16(x, s)
+    assert not bad
+    xs = x.astype(np.float64) * s[:, None]
+    rec = h.view(np.float16).astype(np.float64) + l.view(np.float16).astype(np.float64)
+    # 22 bits relative to the value, or the fp16 subnormal step 2^-24 absolute
+    assert np.all(np.abs(rec - xs) <= np.maximum(2.0 ** -22 * np.abs(xs), 2.0 ** -25))
+    b = rng.uniform(-1, 1, (7, 256)).astype(np.float32)       # eigenvector-like entries
+    hb, lb, _ = P.split_f16(b, P.F16_B_SCALE)
+    ha, la = h.view(np.float16).astype(np.float64), l.view(np.float16).astype(np.float64)
+    hbf, lbf = hb.view(np.float16).astype(np.float64), lb.view(np.float16).astype(np.float64)
+    prod = (ha @ hbf.T + ha @ lbf.T + la @ hbf.T) / (s[:, None].astype(np.float64) * 2.0 ** 14)
+    exact = x.astype(np.float64) @ b.astype(np.float64).T
+    scale = np.abs(x.astype(np.float64)) @ np.abs(b.astype(np.float64)).T
+    assert np.max(np.abs(prod - exact) / scale) < 2.0 ** -20
+
+
+def test_f16_row_scales():
+    """The A operands' row scale 2^e puts the row norm of W^~ in [2^9, 2^10)
+    (64x headroom below fp16's 65504 for entries up to the norm), and a zero
+    row gets 1."""
+    rng = np.random.default_rng(14)
+    W = rng.standard_normal((20, 300)) * np.exp(3 * rng.standard_normal((20, 1)))
+    W[3] = 0.0
+    s = P.row_scales_f16(W)
+    n = np.linalg.norm(W, axis=1) * s
+    ok = np.arange(20) != 3
+    assert np.all((n[ok] >= 2.0 ** 9) & (n[ok] < 2.0 ** 10))
+    assert s[3] == 1.0
+    assert np.all(np.log2(s) == np.round(np.log2(s)))      # powers of two
+
+
 def test_mixed_split_encoding():
     """Operand encoding of the eigenbasis GEMMs: hi = tf32(x) is the plane-0
     value, lo = x - hi is exact in float32, and the correction rows hold
