@@ -289,9 +289,9 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, i
                                               float& r2, float& s2) {
   const float Lf = (float)L;
   float s0 = 1.f, z0 = 0.f;
-  if (r.valid) {
-    s0 = *r.scale;
-    z0 = *r.zero;
+  if (r.valid) {  // L2 reads: another SM may have written them in this launch
+    s0 = __ldcg(r.scale);
+    z0 = __ldcg(r.zero);
   }
   float s = s0, z = z0;
   if (MODE != GRID_FROZEN) {
