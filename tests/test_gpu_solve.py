@@ -279,3 +279,27 @@ def test_fused_schedule_matches_per_gemm(A, name, grid, split):
     for sched in ("fused", "fused_in_parts"):
         for k, v in runs[sched].items():
             assert torch.equal(v, ref[k]), (sched, k)
+
+
+def test_pipeline_matches_separate_solves(A):
+    """solve_layers (next layer's inputs copied on a second stream during the
+    current solve) gives each layer the same bits as solving it alone."""
+    from post_weight_quantization_10_b200 import pipeline
+    p = workloads.scaled(workloads.PRESETS["q_proj"], 4096, 384, 200, rank=16)
+    layers = []
+    for seed in range(3):
+        X = workloads.make_activations(p, seed=seed, device="cuda")
+        W = workloads.make_weights(p, seed=seed, device="cuda", dtype=torch.float32)
+        layers.append((X.cpu().pin_memory(), W.cpu().pin_memory()))
+    prm = A.Params(bits=p.bits, group=p.group, iters=40, rho0=p.rho0, gamma=p.gamma,
+                   lambda_rel=p.lambda_rel, grid="lsq")
+    results = list(pipeline.solve_layers(iter(layers), prm))
+    torch.cuda.synchronize()
+    assert len(results) == 3
+    for (Xh, Wh), r in zip(layers, results):
+        s = A.solve_layer(Xh.cuda(), Wh.cuda(), prm)
+        torch.cuda.synchronize()
+        assert torch.equal(r.codes, s.codes.cpu())
+        assert torch.equal(r.scale, s.scale.cpu()) and torch.equal(r.zero, s.zero.cpu())
+        assert torch.equal(r.packed, A.pack(s.codes, p.bits).cpu())
+        assert float(r.objective) == float(s.objective.cpu())
