@@ -59,13 +59,14 @@ def source_hash():
     return hashlib.sha1(("\n".join(per) + "\n").encode()).hexdigest()[:12]
 
 
-def measured_traffic(kernel):
-    """DRAM bytes per launch from the committed ncu capture, or None when the
-    kernel sources changed since that capture."""
+def measured_traffic(kernel, workload):
+    """DRAM bytes per launch of `kernel` on `workload` (a preset name) from
+    the committed ncu capture, or None when there is no capture of that pair
+    or the kernel sources changed since it was taken."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
-            t = json.load(f)[kernel]
+            t = json.load(f)[f"{kernel}@{workload}"]
     except (OSError, KeyError, ValueError):
         return None
     return t["dram_bytes_per_launch"] if t["source_hash"] == source_hash() else None
@@ -477,7 +478,7 @@ def run_ours(args, rank, world, device):
         "roofline": {"kernel": kname, "bound": "tensor",
                      "achieved": achieved, "peak": peak_split, "unit": "TFLOP/s",
                      "frac": achieved / peak_split,
-                     "traffic": measured_traffic(kname),
+                     "traffic": measured_traffic(kname, args.workload),
                      "peak_note": "bf16 dense %s sustained %.1f TF/s / %d (bf16-MMA units of tensor "
                                   "work per fp32-accurate product, %s split)" % (
                                       pk["src"], pk["bf16_sust"], per_product, split)},
@@ -534,7 +535,7 @@ def stream_kernels(A, grid, device, reps=10):
         ms = a.elapsed_time(b) / reps
         gbs = nbytes / (ms / 1e3) / 1e9
         out[name] = {"shape": shape, "bits": bits, "alg_bytes": nbytes, "ms": ms, "gbs": gbs,
-                     "frac_hbm": gbs / pk["hbm"], "traffic": measured_traffic(name)}
+                     "frac_hbm": gbs / pk["hbm"], "traffic": measured_traffic(name, "stream")}
     del wt, V, codes, phi, plo, big, packed
     torch.cuda.empty_cache()
     return out
