@@ -350,7 +350,7 @@ def run_decoder(args, rank, world, device):
         "value": s_layer, "unit": "s/layer", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": s_layer * 1e3, "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32 via tf32+bf16 split",
+        "dtype": " / ".join(sorted({DTYPES[x["split"]] for x in solves})),
         "data": "synthetic (seeded Qwen3-8B-shaped activations and weights; no dataset)",
         "config": {"workload": "Qwen3-8B-shaped decoder layer: qkv 4096->6144, o 4096->4096, "
                                "gate_up 4096->24576, down 12288->4096; W%d g128 T=%d grid=%s"
