@@ -312,6 +312,14 @@ int admmq_split_mode(const admmq_ctx* ctx);
  * operand left fp16's range; rerun with ADMMQ_SPLIT_MIXED or _3XTF32). */
 int admmq_check(admmq_ctx* ctx, void* stream);
 
+/* Test hook for the failure path: pretend `iterations` more iterations have
+ * been counted, so that the next fused launch's GEMM-2 tiles wait for GEMM-1
+ * tiles that never finish.  Their bounded waits run out (about a second),
+ * the launch ends and admmq_check reports ADMMQ_ERR_TIMEOUT; admmq_prepare
+ * clears the status words and admmq_init the counters, after which the
+ * context solves normally.  No fault, trap or endless loop is involved. */
+int admmq_debug_skew_ready(admmq_ctx* ctx, int iterations);
+
 /* ---------------------------------------------------------------- GPTQ ----
  * The baseline the ADMM-Q objective is reported against: GPTQ, Algorithm 1
  * of "GPTQ: Accurate Post-Training Quantization for Generative Pre-trained

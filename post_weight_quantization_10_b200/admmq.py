@@ -114,6 +114,7 @@ def lib():
                                _vp, _vp, _vp, _vp, _vp, _vp]),
         "admmq_split_mode": (_i, [_vp]),
         "admmq_check": (_i, [_vp, _vp]),
+        "admmq_debug_skew_ready": (_i, [_vp, _i]),
         "admmq_gptq_workspace_bytes": (_sz, [_i, _i, _i]),
         "admmq_gptq": (_i, [_vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float, _i, _vp, _vp, _vp, _vp,
                             _sz, _vp]),
@@ -253,6 +254,10 @@ class Solver:
         """Synchronise and raise AdmmqError if a kernel's bounded wait gave up
         (ERR_TIMEOUT) or an fp16-split operand left fp16's range (ERR_RANGE)."""
         _check(lib().admmq_check(self._ctx, _stream(stream)), "admmq_check")
+
+    def debug_skew_ready(self, iterations: int):
+        """Failure-path test hook (see include/admmq.h)."""
+        _check(lib().admmq_debug_skew_ready(self._ctx, iterations), "admmq_debug_skew_ready")
 
     def buffer(self, name: str) -> torch.Tensor:
         """A torch view of a workspace buffer (see include/admmq.h for layouts)."""

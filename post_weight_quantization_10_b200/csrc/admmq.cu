@@ -1428,6 +1428,12 @@ int admmq_split_mode(const admmq_ctx* c) {
   return c->enc == ENC_MIX ? ADMMQ_SPLIT_MIXED : (c->enc == ENC_F16 ? ADMMQ_SPLIT_F16 : ADMMQ_SPLIT_3XTF32);
 }
 
+int admmq_debug_skew_ready(admmq_ctx* c, int iterations) {
+  if (!c || iterations < 0) return ADMMQ_ERR_INVALID_ARG;
+  c->ready_base += iterations;
+  return ADMMQ_OK;
+}
+
 int admmq_check(admmq_ctx* c, void* stream) {
   if (!c) return ADMMQ_ERR_INVALID_ARG;
   cudaStream_t st = (cudaStream_t)stream;

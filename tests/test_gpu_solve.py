@@ -303,3 +303,32 @@ def test_pipeline_matches_separate_solves(A):
         assert torch.equal(r.scale, s.scale.cpu()) and torch.equal(r.zero, s.zero.cpu())
         assert torch.equal(r.packed, A.pack(s.codes, p.bits).cpu())
         assert float(r.objective) == float(s.objective.cpu())
+
+
+@pytest.mark.parametrize("name,split", [("tiny", "auto"), ("ragged", "f16")])
+def test_bounded_wait_timeout_reports_and_recovers(A, name, split):
+    """Failure detection without a GPU fault: the fused launch's GEMM-2 tiles
+    are made to wait for ready counts that nothing will reach.  Their bounded
+    waits give up after about a second, the launch ends, the host reads
+    ADMMQ_ERR_TIMEOUT from the status word, and the same context then solves
+    the layer again to the same bits as a fresh one."""
+    import time
+    p, X, W = _layer(name)
+    s = _solver(A, p, X, W, "lsq", split=split)
+    s.init()
+    s.debug_skew_ready(1000)
+    t0 = time.perf_counter()
+    s.iterate(0, 1)
+    with pytest.raises(A.AdmmqError) as ei:
+        s.check()
+    assert ei.value.status == A.ERR_TIMEOUT
+    assert time.perf_counter() - t0 < 30.0
+    G = A.build_hessian(X)
+    s.prepare(G, W)
+    s.solve()
+    s.check()
+    ref = _solver(A, p, X, W, "lsq", split=split)
+    ref.solve()
+    ref.check()
+    assert torch.equal(s.codes, ref.codes) and torch.equal(s.scale, ref.scale)
+    assert float(s.objective.cpu()) == float(ref.objective.cpu())
