@@ -320,6 +320,13 @@ int admmq_check(admmq_ctx* ctx, void* stream);
  * context solves normally.  No fault, trap or endless loop is involved. */
 int admmq_debug_skew_ready(admmq_ctx* ctx, int iterations);
 
+/* The projection's quotient rounding on its own (tests): out[i] =
+ * rint(y[i] / s[i / 8]) with the quotient correctly rounded first, computed
+ * as the projection does (a reciprocal product, exact division only near a
+ * rounding tie).  Device pointers; n a multiple of 8. */
+int admmq_debug_rint_div(const float* y_dev, const float* s_dev, long long n, float* out_dev,
+                         void* stream);
+
 /* ---------------------------------------------------------------- GPTQ ----
  * The baseline the ADMM-Q objective is reported against: GPTQ, Algorithm 1
  * of "GPTQ: Accurate Post-Training Quantization for Generative Pre-trained

@@ -397,6 +397,21 @@ __global__ void __launch_bounds__(256) k_pack(const uint8_t* __restrict__ codes,
   }
 }
 
+// rint_div8 on batches of eight values with one divisor per batch (tests).
+__global__ void k_rint_div(const float* __restrict__ y, const float* __restrict__ s, long long batches,
+                           float* __restrict__ out) {
+  for (long long b = blockIdx.x * (long long)blockDim.x + threadIdx.x; b < batches;
+       b += (long long)gridDim.x * blockDim.x) {
+    float yy[8], q[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) yy[k] = y[8 * b + k];
+    const float sb = s[b];
+    rint_div8(yy, sb, __frcp_rn(sb), q);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) out[8 * b + k] = q[k];
+  }
+}
+
 // Standalone projection: one thread per (row, group), W~ read from memory.
 template <int MODE, int ENC>
 __global__ void k_project(const float* __restrict__ wt, float* V, const float* __restrict__ sig,
@@ -1426,6 +1441,15 @@ int admmq_project(const float* wt, float* V, const float* sig, const float* rsig
 int admmq_split_mode(const admmq_ctx* c) {
   if (!c) return ADMMQ_ERR_INVALID_ARG;
   return c->enc == ENC_MIX ? ADMMQ_SPLIT_MIXED : (c->enc == ENC_F16 ? ADMMQ_SPLIT_F16 : ADMMQ_SPLIT_3XTF32);
+}
+
+int admmq_debug_rint_div(const float* y, const float* s, long long n, float* out, void* stream) {
+  if (!y || !s || !out || n < 0 || n % 8 != 0) return ADMMQ_ERR_INVALID_ARG;
+  if (n == 0) return ADMMQ_OK;
+  cudaStream_t st = (cudaStream_t)stream;
+  count_launch(), k_rint_div<<<grid_for(n / 8), 256, 0, st>>>(y, s, n / 8, out);
+  CK(cudaGetLastError());
+  return ADMMQ_OK;
 }
 
 int admmq_debug_skew_ready(admmq_ctx* c, int iterations) {

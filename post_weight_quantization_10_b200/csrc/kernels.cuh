@@ -178,6 +178,34 @@ __device__ __forceinline__ float clampq(float q, float L) {
   return __fadd_rn(fminf(fmaxf(q, 0.f), L), 0.f);
 }
 
+// rint(y / s) for eight values sharing the divisor s, with the quotient
+// correctly rounded first (the same integers as rintf(__fdiv_rn(y, s))), from
+// r = __frcp_rn(s).  t = y r differs from the rounded quotient by at most
+// 1.5 * 2^-23 |y / s| (the reciprocal's and the product's roundings, 2^-24
+// each, and the quotient's own), so when t lies farther than 2^-21 |t| from
+// the nearest half-integer both round to the same integer.  Otherwise (a
+// near-tie, or a non-finite t) that value is divided exactly.  The eight
+// fast paths are straight-line code; the exact divisions are rare.
+__device__ __forceinline__ void rint_div8(const float (&y)[8], float s, float r, float (&q)[8]) {
+  bool exact = false;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float t = __fmul_rn(y[k], r);
+    q[k] = rintf(t);
+    const float off = fabsf(__fsub_rn(t, q[k]));
+    exact |= !(off < __fsub_rn(0.5f, __fmul_rn(fabsf(t), 4.76837158203125e-7f)));  // 2^-21
+  }
+  if (exact) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float t = __fmul_rn(y[k], r);
+      const float off = fabsf(__fsub_rn(t, rintf(t)));
+      if (!(off < __fsub_rn(0.5f, __fmul_rn(fabsf(t), 4.76837158203125e-7f))))
+        q[k] = rintf(__fdiv_rn(y[k], s));
+    }
+  }
+}
+
 // eight consecutive read-only floats (per-column vectors: sigma, 1/sigma, diag H)
 __device__ __forceinline__ void load8_ro(const float* p, float (&v)[8]) {
   const float4 a = __ldg(reinterpret_cast<const float4*>(p));
@@ -263,11 +291,19 @@ __device__ __forceinline__ void mse_clip_grid(LoadW& loadw, const ProjRow& r, in
       float sk, zk;
       range_grid(__fmul_rn(a, mn), __fmul_rn(a, mx), Lf, sk, zk);
       float ek = ce[k];
+      const float rk = __frcp_rn(sk);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float q = clampq(__fadd_rn(rintf(__fdiv_rn(y[j], sk)), zk), Lf);
-        const float dd = __fsub_rn(y[j], __fmul_rn(sk, __fsub_rn(q, zk)));
-        ek = __fadd_rn(ek, __fmul_rn(dd, dd));
+      for (int j0 = 0; j0 < 32; j0 += 8) {
+        float y8[8], q8[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) y8[j] = y[j0 + j];
+        rint_div8(y8, sk, rk, q8);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float q = clampq(__fadd_rn(q8[j], zk), Lf);
+          const float dd = __fsub_rn(y8[j], __fmul_rn(sk, __fsub_rn(q, zk)));
+          ek = __fadd_rn(ek, __fmul_rn(dd, dd));
+        }
       }
       ce[k] = ek;
     }
@@ -294,6 +330,7 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, i
     z0 = __ldcg(r.zero);
   }
   float s = s0, z = z0;
+  const float r0 = __frcp_rn(s0);
   if (MODE != GRID_FROZEN) {
     float mn = 0.f, mx = 0.f;
     float Sw = 0.f, Sq = 0.f, Sqq = 0.f, Sy = 0.f, Sqy = 0.f;
@@ -305,18 +342,20 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, i
       for (int e = 0; e < 32; e += 8) {
         float vv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         if (r.valid) ld_v8f(r.V + c + e, vv);
-        float ss[8], hh[8];
+        float ss[8], hh[8], y8[8], q8[8];
         load8_ro(r.sig + c + e, ss);
         if (MODE == GRID_LSQ) load8_ro(r.hd + c + e, hh);
 #pragma unroll
+        for (int k = 0; k < 8; ++k) y8[k] = __fmul_rn(ss[k], __fadd_rn(w[e + k], vv[k]));
+        if (MODE == GRID_LSQ) rint_div8(y8, s0, r0, q8);
+#pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const float t = __fadd_rn(w[e + k], vv[k]);
-          const float y = __fmul_rn(ss[k], t);
+          const float y = y8[k];
           if (MODE == GRID_MINMAX || MODE == GRID_MSE) {
             mn = fminf(mn, y);
             mx = fmaxf(mx, y);
           } else {
-            const float q0 = clampq(__fadd_rn(rintf(__fdiv_rn(y, s0)), z0), Lf);
+            const float q0 = clampq(__fadd_rn(q8[k], z0), Lf);
             const float wi = hh[k];
             const float wq = __fmul_rn(wi, q0);
             Sw = __fadd_rn(Sw, wi);
@@ -348,6 +387,7 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, i
       }
     }
   }
+  const float rs = __frcp_rn(s);
 #pragma unroll
   for (int c = 0; c < g; c += 32) {
     float w[32];
@@ -359,15 +399,20 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, i
     for (int e = 0; e < 32; e += 8) {
       float vv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       if (r.valid) ld_v8f(r.V + c + e, vv);
-      float ss[8], rr[8];
+      float ss[8], rr[8], t8[8], y8[8], q8[8];
       load8_ro(r.sig + c + e, ss);
       load8_ro(r.rsig + c + e, rr);
       float vn[8], pv[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        const float t = __fadd_rn(w[e + k], vv[k]);
-        const float y = __fmul_rn(ss[k], t);
-        const float q = clampq(__fadd_rn(rintf(__fdiv_rn(y, s)), z), Lf);
+        t8[k] = __fadd_rn(w[e + k], vv[k]);
+        y8[k] = __fmul_rn(ss[k], t8[k]);
+      }
+      rint_div8(y8, s, rs, q8);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float t = t8[k];
+        const float q = clampq(__fadd_rn(q8[k], z), Lf);
         const float D = __fmul_rn(s, __fsub_rn(q, z));
         const float dt = __fmul_rn(D, rr[k]);
         vn[k] = __fsub_rn(t, dt);

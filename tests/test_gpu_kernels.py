@@ -161,3 +161,35 @@ def test_pack_rejects_bad_shapes(A):
     c = torch.zeros((4, 48), dtype=torch.uint8, device="cuda")
     with pytest.raises(A.AdmmqError):
         A.pack(c, 3, out=torch.empty((4, 8), dtype=torch.int32, device="cuda"))
+
+
+def test_quotient_rounding_matches_correct_division(A):
+    """The projection rounds y / s through a reciprocal product and divides
+    exactly only near a rounding tie; the integers must equal rint of the
+    correctly rounded float32 quotient (numpy's IEEE division) everywhere:
+    random data over wide magnitudes, exact half-integer quotients, their
+    neighbours a few ulps away, zeros of both signs, tiny and huge values."""
+    rng = np.random.default_rng(21)
+    nb = 200_000
+    s = (np.exp(rng.uniform(-12, 6, nb)) * rng.choice([1.0, 1.5, 1.25, 0.875], nb)).astype(np.float32)
+    y = (rng.standard_normal((nb, 8)) * rng.choice([1.0, 10.0, 300.0], (nb, 1)) * s[:, None]).astype(np.float32)
+    # exact ties (k + 1/2) s for s with short mantissas, and their neighbours
+    t = nb // 4
+    k = rng.integers(-300, 300, (t, 8)).astype(np.float32) + np.float32(0.5)
+    s_short = np.ldexp(np.float32(1), rng.integers(-20, 10, t)).astype(np.float32) * np.float32(1.5)
+    s[:t] = s_short
+    y[:t] = (k * s_short[:, None]).astype(np.float32)
+    for j, steps in enumerate((1, -1, 2, -2, 3, -3)):
+        y[t // 8 * j:t // 8 * (j + 1), 7] = np.nextafter(
+            y[t // 8 * j:t // 8 * (j + 1), 7], np.float32(np.inf) if steps > 0 else np.float32(-np.inf))
+    y[t:t + 100, 0] = 0.0
+    y[t + 100:t + 200, 0] = -0.0
+    y[t + 200:t + 300, 1] = np.float32(1e-40)          # subnormal numerators
+    y[t + 300:t + 400, 2] = np.float32(3e38)           # huge numerators
+    s[t + 400:t + 500] = np.float32(1e-39)             # subnormal divisors
+    out = A.debug_rint_div(torch.from_numpy(y.reshape(-1)).cuda(), torch.from_numpy(s).cuda())
+    torch.cuda.synchronize()
+    with np.errstate(over="ignore", invalid="ignore", divide="ignore"):
+        ref = np.rint(y / s[:, None]).astype(np.float32).reshape(-1)
+    got = out.cpu().numpy()
+    np.testing.assert_array_equal(got.view(np.uint32), ref.view(np.uint32))
