@@ -541,7 +541,9 @@ GemmGeom make_geom(int M, int N, long long K, int BN, int BK, int splits, bool t
     g.tiles = t;
   }
   g.units = g.tiles * splits;
-  g.band = g.tiles_mu < 12 ? g.tiles_mu : 12;  // 12 x 12 tiles in flight ~ 100 MB of operands
+  // bands of 8 unit rows: measured best of 4, 8, 12, 16 for the eigenbasis
+  // GEMMs at q_proj (ms per solve 75.0, 73.8, 75.3, 79.7)
+  g.band = g.tiles_mu < 8 ? g.tiles_mu : 8;
   g.status = status;
   return g;
 }
