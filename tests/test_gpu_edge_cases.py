@@ -109,3 +109,23 @@ def test_zero_iterations_is_the_rtn_start(A, split):
     np.testing.assert_array_equal(s.zero.cpu().numpy(), zero.T.astype(np.float32))
     H = O.hessian(X.float().cpu().numpy(), p.lambda_rel)
     assert float(s.objective.cpu()) == pytest.approx(O.objective(H, D, Wm), rel=1e-4)
+
+
+@pytest.mark.parametrize("bits", [1, 8])
+@pytest.mark.parametrize("split", ["auto", "f16"])
+def test_extreme_bit_widths(A, bits, split):
+    """b = 1 (two levels per group) and b = 8 (256 levels): valid solutions
+    close to the oracle's, with codes spanning the whole range [0, 2^b - 1]."""
+    p = workloads.scaled(BASE, 2048, 256, 64, group=64, bits=bits, iters=40, rank=16)
+    X = workloads.make_activations(p, seed=6, device="cuda")
+    W = workloads.make_weights(p, seed=6, device="cuda", dtype=torch.float32)
+    s = _solve(A, p, split, X, W)
+    H = O.hessian(X.float().cpu().numpy(), p.lambda_rel)
+    Wm = W.float().cpu().numpy().T.astype(np.float64)
+    res = O.admm_q(H, Wm, p.bits, p.group, p.iters, rho0=p.rho0, gamma=p.gamma, grid="lsq")
+    codes, obj = _valid(p, s, H, Wm)
+    assert codes.min() == 0 and codes.max() == (1 << bits) - 1
+    agree = float(np.mean(codes == res["codes"].T))
+    rel = obj / res["objective"] - 1.0
+    print(f"bits {bits} / {s.split}: codes agree {agree:.5f}, objective rel {rel:+.3e}")
+    assert agree >= 0.9 and abs(rel) <= 0.2
