@@ -203,25 +203,39 @@ __global__ void k_eigvals(const double* __restrict__ ev, int d, float* __restric
 }
 
 // RTN start: D_0 = min/max-grid rounding of W_hat, V~ = 0, P = D~_0 (operand
-// encoding, A side).
+// encoding, A side).  One warp per (row, group): lane l takes the group's
+// g/32 consecutive elements from l g/32 on, so the warp's accesses are
+// contiguous; the group's min and max (exact in any order) come from a warp
+// reduction and every lane forms the same grid from them.
 template <typename T>
 __global__ void k_init_rtn(const T* __restrict__ W, const float* __restrict__ rsig, int m, int d,
                            int g, int L, uint8_t* __restrict__ codes, float* __restrict__ scale,
                            float* __restrict__ zero, float* __restrict__ V, void* p_hi,
                            void* p_lo, int enc, const float* __restrict__ row_in, int* flag) {
-  const int ngr = d / g;
+  const int ngr = d / g, per = g / 32;
   const long long total = (long long)m * ngr;
   const float Lf = (float)L;
-  for (long long gi = blockIdx.x * (long long)blockDim.x + threadIdx.x; gi < total;
-       gi += (long long)gridDim.x * blockDim.x) {
+  const int lane = threadIdx.x & 31;
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long gi = blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5); gi < total;
+       gi += warps) {
     const long long row = gi / ngr;
-    const int col0 = (int)(gi - row * ngr) * g;
+    const int col0 = (int)(gi - row * ngr) * g + lane * per;
     const long long base = row * d + col0;
+    float y[4] = {0.f, 0.f, 0.f, 0.f};
     float mn = 0.f, mx = 0.f;
-    for (int e = 0; e < g; ++e) {
-      const float y = load_w<T>(W, base + e);
-      mn = fminf(mn, y);
-      mx = fmaxf(mx, y);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (e < per) {
+        y[e] = load_w<T>(W, base + e);
+        mn = fminf(mn, y[e]);
+        mx = fmaxf(mx, y[e]);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     }
     float s = __fdiv_rn(__fsub_rn(mx, mn), Lf), z;
     if (s == 0.f) {
@@ -230,18 +244,23 @@ __global__ void k_init_rtn(const T* __restrict__ W, const float* __restrict__ rs
     } else {
       z = __fadd_rn(rintf(__fdiv_rn(-mn, s)), 0.f);
     }
-    for (int e = 0; e < g; ++e) {
-      const float y = load_w<T>(W, base + e);
-      const float q = clampq(__fadd_rn(rintf(__fdiv_rn(y, s)), z), Lf);
+    void* hi = plane0_row(enc, p_hi, row, d);
+    void* lo = plane1_row(enc, p_lo, row, d);
+    const float ri = row_in[row];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (e >= per) break;
+      const float q = clampq(__fadd_rn(rintf(__fdiv_rn(y[e], s)), z), Lf);
       const float D = __fmul_rn(s, __fsub_rn(q, z));
       const float dt = __fmul_rn(D, rsig[col0 + e]);
       codes[base + e] = (uint8_t)q;
       V[base + e] = 0.f;
-      put_a1(enc, plane0_row(enc, p_hi, row, d), plane1_row(enc, p_lo, row, d), col0 + e, dt,
-             row_in[row], flag);
+      put_a1(enc, hi, lo, col0 + e, dt, ri, flag);
     }
-    scale[gi] = s;
-    zero[gi] = z;
+    if (lane == 0) {
+      scale[gi] = s;
+      zero[gi] = z;
+    }
   }
 }
 
@@ -1140,11 +1159,11 @@ int admmq_init(admmq_ctx* c, uint8_t* codes, float* scale, float* zero, void* st
   const long long groups = (long long)m * (d / c->p.group);
   int* flag = c->status + 3;
   if (c->w_dtype == ADMMQ_DTYPE_F32)
-    count_launch(), k_init_rtn<float><<<grid_for(groups, 128), 128, 0, st>>>(
+    count_launch(), k_init_rtn<float><<<grid_for(groups, 8), 256, 0, st>>>(
         (const float*)c->W_hat, c->rsig, m, d, c->p.group, c->L, codes, scale, zero, c->V,
         c->P_hi, c->P_lo, c->enc, c->row_in, flag);
   else
-    count_launch(), k_init_rtn<__nv_bfloat16><<<grid_for(groups, 128), 128, 0, st>>>(
+    count_launch(), k_init_rtn<__nv_bfloat16><<<grid_for(groups, 8), 256, 0, st>>>(
         (const __nv_bfloat16*)c->W_hat, c->rsig, m, d, c->p.group, c->L, codes, scale, zero,
         c->V, c->P_hi, c->P_lo, c->enc, c->row_in, flag);
   CK(cudaGetLastError());
