@@ -567,10 +567,6 @@ GemmGeom make_geom(int M, int N, long long K, int BN, int BK, int splits, bool t
   return g;
 }
 
-// Launches k_gemm<Cfg, Work> over `units` work units: one CTA per SM, or one
-// pair of CTAs per two SMs.  A policy whose units wait on earlier units of the
-// same launch needs every CTA of the launch resident at once, so its grid is
-// capped by the occupancy query.
 // Geometry of an eigenbasis GEMM [rows][d] x [d][d] for an encoding (its K
 // per stage: 32 fp32 or 64 fp16 elements).
 GemmGeom eig_geom(int enc, int rows, int d, int* status) {
@@ -578,6 +574,10 @@ GemmGeom eig_geom(int enc, int rows, int d, int* status) {
                         : make_geom(rows, d, d, EigCfg::BN, EigCfg::BK, 1, false, status, EigCfg::UNIT_M);
 }
 
+// Launches k_gemm<Cfg, Work> over `units` work units: one CTA per SM, or one
+// pair of CTAs per two SMs.  A policy whose units wait on earlier units of the
+// same launch needs every CTA of the launch resident at once, so its grid is
+// capped by the occupancy query.
 template <class Cfg, class Work>
 cudaError_t launch_work(const typename Work::Args& args, int units, cudaStream_t st) {
   auto kern = k_gemm<Cfg, Work>;
