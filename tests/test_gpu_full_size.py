@@ -186,15 +186,27 @@ def test_full_size_free_running(A, full_setup, grid, monkeypatch):
     assert abs(rel) <= 2.0 * max_rel + 1e-3
 
 
-def test_down_proj_first_iteration_sampled(A):
-    """The down_proj shape (d_in = 12288, d_out = 4096, W2, group 128; the
-    eigenbasis GEMMs reduce over K = 12288): the RTN start bit-exact on 12
-    sampled rows, then W~ after iteration 0 within 1e-4 relative of the
-    W-update's closed form W~* = (H~ + rho0 I)^-1 (H~ W^~ + rho0 D~_0) solved in
-    float64 for those rows, and the codes of that step equal to the oracle's
-    projection of W~* on >= 99.9% of entries.  H comes from n = 8192 tokens."""
-    p = workloads.scaled(workloads.PRESETS["down_proj"], 8192, 12288, 4096)
-    rows = np.array([0, 1, 500, 1023, 1024, 2047, 2048, 2500, 3071, 3500, 4094, 4095])
+FIRST_ITERATION_SHAPES = {
+    # the eigenbasis GEMMs reduce over K = 12288
+    "down_proj": ("down_proj", 12288, 4096,
+                  [0, 1, 500, 1023, 1024, 2047, 2048, 2500, 3071, 3500, 4094, 4095]),
+    # 25600 rows: 100 unit rows of 256, the largest tile grid of the workloads
+    "up_proj_32b": ("up_proj_32b", 5120, 25600,
+                    [0, 255, 256, 4095, 12799, 12800, 20000, 25343, 25344, 25598, 25599, 7777]),
+}
+
+
+@pytest.mark.parametrize("shape", sorted(FIRST_ITERATION_SHAPES))
+def test_first_iteration_sampled(A, shape):
+    """A deep and a tall layer at their real sizes (the fp16 split): the RTN
+    start bit-exact on 12 sampled rows (across unit-row boundaries), then W~
+    after iteration 0 within 1e-4 relative of the W-update's closed form
+    W~* = (H~ + rho0 I)^-1 (H~ W^~ + rho0 D~_0) solved in float64 for those
+    rows, and the codes of that step equal to the oracle's projection of W~*
+    on >= 99.9% of entries.  H comes from n = 8192 tokens."""
+    preset, d_in, d_out, rows = FIRST_ITERATION_SHAPES[shape]
+    p = workloads.scaled(workloads.PRESETS[preset], 8192, d_in, d_out)
+    rows = np.array(rows)
     X = workloads.make_activations(p, seed=0, device="cuda")
     W = workloads.make_weights(p, seed=0, device="cuda", dtype=torch.float32)
     prm = A.Params(bits=p.bits, group=p.group, iters=p.iters, rho0=p.rho0, gamma=p.gamma,
@@ -202,15 +214,17 @@ def test_down_proj_first_iteration_sampled(A):
     s = A.Solver(p.d_in, p.d_out, prm)
     s.prepare(A.build_hessian(X), W)
     s.eigh()
+    assert s.split == "f16"
     s.init()
     wt = torch.empty((p.d_out, p.d_in), dtype=torch.float32, device="cuda")
     s.dump_wtilde(wt)
     c_init = s.codes[torch.from_numpy(rows).cuda()].cpu().numpy()
     s.iterate(0, 1)
-    torch.cuda.synchronize()
+    s.check()
     s.dump_wtilde(None)
     r_idx = torch.from_numpy(rows).cuda()
     got_w, got_c = wt[r_idx].cpu().numpy().astype(np.float64), s.codes[r_idx].cpu().numpy()
+    del wt
 
     H = O.hessian(X.float().cpu().numpy(), p.lambda_rel)
     del X
@@ -226,6 +240,6 @@ def test_down_proj_first_iteration_sampled(A):
     err = np.linalg.norm(got_w - w_ref.T) / np.linalg.norm(w_ref)
     c_ref = O.project(sigma[:, None] * w_ref, p.bits, p.group, "lsq", hdiag, s0, z0)[0]
     mism = np.mean(got_c != c_ref.T)
-    print(f"down_proj first iteration: W~ rel err {err:.2e}, code mismatches {mism:.2e}")
+    print(f"{shape} first iteration: W~ rel err {err:.2e}, code mismatches {mism:.2e}")
     assert err <= 1e-4
     assert mism <= 1e-3
