@@ -79,7 +79,11 @@ enum {
  * on rows, so GEMM 1 and GEMM 2 of an iteration can run in one persistent
  * launch whose GEMM-2 tiles wait until the row block of T they read is
  * complete (the default: one tail instead of two per iteration); or GEMM 1
- * and GEMM 2 are launched separately.  Both give the same bits. */
+ * and GEMM 2 are launched separately.  Both give the same bits.  The fused
+ * launch needs all its CTAs resident at once (its grid is sized for that):
+ * do not run other kernels on the GPU concurrently with admmq_iterate
+ * (copies on other streams are fine); ADMMQ_SCHEDULE_PER_GEMM has no such
+ * requirement. */
 enum {
   ADMMQ_SCHEDULE_FUSED = 0,   /* GEMM 1 + GEMM 2 of an iteration in one launch */
   ADMMQ_SCHEDULE_PER_GEMM = 1 /* two launches per iteration                   */
