@@ -76,16 +76,15 @@ enum {
 };
 
 /* How admmq_iterate launches the iterations.  Every step of an iteration acts
- * on rows, so GEMM 1 and GEMM 2 of an iteration can run in one persistent
- * launch whose GEMM-2 tiles wait until the row block of T they read is
- * complete (the default: one tail instead of two per iteration); or GEMM 1
- * and GEMM 2 are launched separately.  Both give the same bits.  The fused
- * launch needs all its CTAs resident at once (its grid is sized for that):
- * do not run other kernels on the GPU concurrently with admmq_iterate
- * (copies on other streams are fine); ADMMQ_SCHEDULE_PER_GEMM has no such
- * requirement. */
+ * on rows, so GEMM 1 and GEMM 2 of all the iterations of one admmq_iterate
+ * call can run in one persistent launch whose tiles wait until the row block
+ * they read is complete (the default: one launch and one tail per call); or
+ * GEMM 1 and GEMM 2 of each iteration are launched separately.  Both give the
+ * same bits.  The fused launch hands out its tiles in order from a counter
+ * to whichever CTAs are running, so it needs no particular number of them
+ * resident and may share the GPU with other work. */
 enum {
-  ADMMQ_SCHEDULE_FUSED = 0,   /* GEMM 1 + GEMM 2 of an iteration in one launch */
+  ADMMQ_SCHEDULE_FUSED = 0,   /* every iteration of a call in one launch      */
   ADMMQ_SCHEDULE_PER_GEMM = 1 /* two launches per iteration                   */
 };
 

@@ -5,21 +5,20 @@
 // update): row block r of T needs only row block r of P (GEMM 1); row block r
 // of W~ needs only row block r of T (GEMM 2), whose epilogue refreshes row
 // block r of P, V~ and the codes.  So the units of GEMM 1 and GEMM 2 of
-// several iterations share one launch, ordered (iteration, GEMM, tile) and
-// dealt round-robin to the CTA pairs (the library launches one iteration at a
-// time: over many iterations the pairs drift apart, the tiles in flight stop
-// sharing operands in L2 and the extra HBM traffic costs more than the launch
-// tails it saves).  Before loading, a unit's producer waits
-// until the row block it reads is complete:
+// every iteration share one launch, ordered (iteration, GEMM, tile) and
+// dealt to the CTA pairs in that order from a ticket counter: the units in
+// flight are always a narrow window of consecutive indices, whose tiles share
+// their operand panels in L2, however long the launch.  Before loading, a
+// unit's producer waits until the row block it reads is complete:
 //   GEMM 2 of iteration i, row block r: every GEMM-1 tile of (i, r) is done;
 //   GEMM 1 of iteration i > 0, row block r: every GEMM-2 tile of (i - 1, r).
 // The same waits cover the overwrites: GEMM 1 of i rewrites the T that GEMM 2
 // of i - 1 read, GEMM 2 of i the P that GEMM 1 of i read.
-// Every dependency has a smaller unit index, every CTA takes its units in
-// index order, and all CTAs of the launch are resident at once (the launch is
-// sized by the occupancy query), so the lowest unfinished unit can always
-// proceed; the waits are bounded all the same.  The arithmetic of each unit is
-// that of the separate GEMM launches, so both schedules give the same bits.
+// Every dependency has a smaller unit index and a unit is only taken by a
+// running pair after every smaller one, so the lowest unfinished unit is
+// always held by a running pair and can proceed, however many pairs are
+// resident; the waits are bounded all the same.  The arithmetic of each unit
+// is that of the separate GEMM launches, so both schedules give the same bits.
 #pragma once
 #include "gemm.cuh"
 
@@ -38,10 +37,18 @@ struct AdmmLoop {
     long long part_stride;
     int* ready;                    // [2][tiles_mu] finished CTA tiles per row block
     int base;                      // iterations already counted in `ready`
+    int* ticket;                   // next unit to deal, zero before the launch
+    int* ticket_next;              // the next launch's counter, zeroed by this one
     int ctas;                      // CTAs per unit (2 for CTA pairs)
     int t0, count;
   };
   static constexpr bool SIGNALS = true;
+  static constexpr bool DYNAMIC = true;
+  __device__ static int take_ticket(const Args& x) { return atomicAdd(x.ticket, 1); }
+  // Launches alternate between two counters: each zeroes the other one for
+  // the launch after it (which starts only once this one has ended), so an
+  // aborted launch leaves no stale count behind.
+  __device__ static void begin(const Args& x) { *x.ticket_next = 0; }
   __device__ static int units(const Args& x) { return x.count * 2 * x.g.units; }
   template <class Cfg>
   __device__ static void decode(const Args& x, int u, Unit& w) {

@@ -24,9 +24,6 @@ using namespace admmq;
 namespace {
 
 constexpr int kBM = 128;
-// Iterations per launch of the fused schedule (one: measured fastest under
-// the power cap, see admm_loop.cuh).
-constexpr int kFusedIters = 1;
 unsigned long long g_launches = 0;  // kernels launched by this library
 inline void count_launch() { __atomic_fetch_add(&g_launches, 1ull, __ATOMIC_RELAXED); }
 // X^T X: bf16, both operands MN-major (X is token-major).
@@ -576,8 +573,9 @@ GemmGeom eig_geom(int enc, int rows, int d, int* status) {
 
 // Launches k_gemm<Cfg, Work> over `units` work units: one CTA per SM, or one
 // pair of CTAs per two SMs.  A policy whose units wait on earlier units of the
-// same launch needs every CTA of the launch resident at once, so its grid is
-// capped by the occupancy query.
+// same launch deals them from a counter to the CTAs that are running, so it
+// needs none resident in particular; its grid is the occupancy query's count,
+// the most CTAs that can run at once.
 template <class Cfg, class Work>
 cudaError_t launch_work(const typename Work::Args& args, int units, cudaStream_t st) {
   auto kern = k_gemm<Cfg, Work>;
@@ -722,6 +720,8 @@ struct admmq_ctx {
   float* rho_tab;       // [iters] rho_t, as the host computes it
   int* ready;           // [2][unit rows] ready counters of the fused schedule
   int ready_base;       // iterations counted in `ready` since admmq_init zeroed it
+  int* ticket;          // [2] unit tickets of the fused launches, used alternately
+  unsigned fused_launches;  // fused launches since admmq_init
   int tiles_eig;
   const void* W_hat;
   int w_dtype;
@@ -782,7 +782,7 @@ Layout make_layout(int d, int m, int iters, int lwork) {
   L.resid_part = take(4 * (size_t)(iters > 0 ? iters : 1) * tiles * 8);
   L.obj_part = take(4 * (size_t)tiles * 4);
   L.rho_tab = take(4 * (size_t)(iters > 0 ? iters : 1));
-  L.ready = take(4 * 2 * (size_t)cdiv(m, 2 * kBM));
+  L.ready = take(4 * (2 * (size_t)cdiv(m, 2 * kBM) + 2));  // counters, then 2 tickets
   L.row_in = take(4 * (size_t)m);
   L.row_out = take(4 * (size_t)m);
   L.total = o;
@@ -912,6 +912,8 @@ cudaError_t launch_admm_loop(const admmq_ctx* c, const GemmGeom& g, const TUpdat
   x.part_stride = (long long)c->tiles_eig * 8;
   x.ready = c->ready;
   x.base = c->ready_base;
+  x.ticket = c->ticket + (c->fused_launches & 1u);
+  x.ticket_next = c->ticket + ((c->fused_launches + 1u) & 1u);
   x.ctas = Cfg::PAIR ? 2 : 1;
   x.t0 = t0;
   x.count = count;
@@ -1051,6 +1053,7 @@ int admmq_create(admmq_ctx** out, int d, int m, const admmq_params* p, void* ws,
   c->obj_part = (float*)(b + L.obj_part);
   c->rho_tab = (float*)(b + L.rho_tab);
   c->ready = (int*)(b + L.ready);
+  c->ticket = c->ready + 2 * cdiv(m, 2 * kBM);
   c->tiles_eig = eig_tiles(m, d);
   bool ok = true;
   c->row_in = (float*)(b + L.row_in);
@@ -1172,8 +1175,9 @@ int admmq_init(admmq_ctx* c, uint8_t* codes, float* scale, float* zero, void* st
     for (int t = 0; t < c->p.iters; ++t) rho[t] = rho_at(c->p, t);
     CK(cudaMemcpyAsync(c->rho_tab, rho.data(), sizeof(float) * rho.size(), cudaMemcpyHostToDevice, st));
   }
-  CK(cudaMemsetAsync(c->ready, 0, sizeof(int) * 2 * cdiv(m, 2 * kBM), st));
+  CK(cudaMemsetAsync(c->ready, 0, sizeof(int) * (2 * cdiv(m, 2 * kBM) + 2), st));
   c->ready_base = 0;
+  c->fused_launches = 0;
   c->inited = true;
   return ADMMQ_OK;
 }
@@ -1212,8 +1216,9 @@ int admmq_iterate(admmq_ctx* c, int t0, int count, uint8_t* codes, float* scale,
     return ADMMQ_OK;
   };
   if (c->p.schedule == ADMMQ_SCHEDULE_FUSED) {
-    for (int t = t0; t < t0 + count; t += kFusedIters) {
-      const int n = t0 + count - t < kFusedIters ? t0 + count - t : kFusedIters;
+    // one launch for all the iterations of the call
+    {
+      const int t = t0, n = count;
       admmq_ctx::TimingRec rec{nullptr, nullptr, nullptr, true, n};
       if (c->timing) {
         int rc = new_event(rec.a);
@@ -1239,6 +1244,7 @@ int admmq_iterate(admmq_ctx* c, int t0, int count, uint8_t* codes, float* scale,
       }
       CK(e);
       c->ready_base += n;
+      c->fused_launches += 1;
       if (c->timing) CK(cudaEventRecord(rec.b, st));
     }
     return ADMMQ_OK;

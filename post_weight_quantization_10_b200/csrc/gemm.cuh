@@ -44,12 +44,16 @@
 // leader (rank 0) issues the MMAs and commits to the barriers of both CTAs;
 // both CTAs' TMA loads count on the leader's stage barrier; consumers release
 // ring slots to the leader with remote arrivals.
-// Work units are dealt to CTAs (or pairs) round-robin in index order.  What a
-// unit is comes from the Work policy: OneGemm (below) runs the (tile, k-split)
-// units of one GEMM with one epilogue; a policy may also chain several GEMMs
-// in one launch, with units whose operands are produced by earlier units of
-// the same launch (ready counters, see ptx.cuh: wait_counter).  Every wait is
-// bounded.
+// What a unit is comes from the Work policy: OneGemm (below) runs the (tile,
+// k-split) units of one GEMM with one epilogue, dealt to CTAs (or pairs)
+// round-robin.  A policy may also chain several GEMMs in one launch, with
+// units whose operands are produced by earlier units of the same launch
+// (ready counters, see ptx.cuh: wait_counter); such a policy deals its units
+// dynamically (DYNAMIC): the pair leader's producer takes the next unit from
+// a global ticket counter and passes it to its roles and to its pair member
+// through a four-entry ring in shared memory.  A unit is then only ever taken
+// by a running CTA, after every unit with a smaller index, so units waiting
+// on smaller ones always make progress.  Every wait is bounded.
 #pragma once
 #include "ptx.cuh"
 
@@ -91,9 +95,15 @@ struct GemmCfg {
   static constexpr int RING = 2;                 // 256-column chunk slots in tensor memory
   static constexpr int TMEM_COLS = RING * BN;    // 512
   static constexpr int THREADS = 320;
-  // mbarriers, then tensor-memory address, abort flag, 2 spare words and the
-  // four unit-completion counters of the consumer warps
-  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 2 * RING + 1) + 32;
+  // mbarriers (stages, ring slots, drain, unit ring), then tensor-memory
+  // address, abort flag, 2 spare words, the four unit-completion counters of
+  // the consumer warps and the four unit-ring entries
+  static constexpr int UNIT_RING = 4;
+  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 2 * RING + 1 + 2 * UNIT_RING) + 48;
+  // readers that release a unit-ring entry: the MMA issuer and the eight
+  // consumer warps of the leader, and the producer and eight consumer warps of
+  // its pair member
+  static constexpr int RING_READERS = PAIR ? 18 : 9;
   // arrivals that release a ring slot: every consumer thread of the CTA, or
   // one per consumer warp of both CTAs of a pair
   static constexpr int SLOT_ARRIVALS = PAIR ? 16 : 256;
@@ -158,6 +168,7 @@ struct OneGemm {
     typename Epi::Params ep;
   };
   static constexpr bool SIGNALS = false;
+  static constexpr bool DYNAMIC = false;
   __device__ static int units(const Args& x) { return x.g.units; }
   template <class Cfg>
   __device__ static void decode(const Args& x, int u, Unit& w) {
@@ -202,9 +213,13 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   uint64_t* rfull = bars + 2 * STAGES;  // [slot]: slot holds a finished chunk
   uint64_t* rempty = rfull + R;         // [slot]: slot drained by its consumers
   uint64_t* drain = rempty + R;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  constexpr int UR = Cfg::UNIT_RING;
+  uint64_t* ufull = drain + 1;          // [UR]: unit-ring entry written
+  uint64_t* uempty = ufull + UR;        // [UR]: entry read by every reader (leader's)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(uempty + UR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* epi_count = reinterpret_cast<int*>(tmem_slot + 4);  // [4], by unit sequence number & 3
+  volatile int* unit_ring = reinterpret_cast<volatile int*>(tmem_slot + 8);  // [UR]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // CTA pairs: rank in the cluster (0 = leader, issues the MMAs); work units
@@ -213,6 +228,28 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   const int unit0 = Cfg::PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int unit_step = Cfg::PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   const int nunits = Work::units(args);
+  constexpr bool DYN = Work::DYNAMIC;
+  const bool leader = !Cfg::PAIR || rank == 0;
+  // Dynamic dealing, reader side: the unit of this CTA's seq-th entry, -1 if
+  // the wait gave up.  Every lane of the calling warp calls it (or the one
+  // thread of a single-thread role); one arrival per warp releases the entry
+  // on the leader's barrier.
+  auto take_unit = [&](int seq, bool single) -> int {
+    const int e = seq % UR;
+    const uint32_t par = (uint32_t)(seq / UR) & 1u;
+    const bool got = leader ? mbar_wait(smem_u32(&ufull[e]), par, abort_flag, g.status)
+                            : mbar_wait_cluster(smem_u32(&ufull[e]), par, abort_flag, g.status);
+    if (single ? !got : !__all_sync(0xffffffffu, got)) return -1;
+    const int u = unit_ring[e];
+    if (!single) __syncwarp();
+    if (single || (threadIdx.x & 31) == 0) {
+      if (leader)
+        mbar_arrive(smem_u32(&uempty[e]));
+      else
+        mbar_arrive_cluster(cluster_addr(smem_u32(&uempty[e]), 0));
+    }
+    return u;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -224,6 +261,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       mbar_init(smem_u32(&rempty[a]), Cfg::SLOT_ARRIVALS);
     }
     mbar_init(smem_u32(drain), 1);
+    for (int e = 0; e < UR; ++e) {
+      mbar_init(smem_u32(&ufull[e]), 1);
+      mbar_init(smem_u32(&uempty[e]), Cfg::RING_READERS);
+    }
     *abort_flag = 0;
     for (int k = 0; k < 4; ++k) epi_count[k] = 0;
     fence_barrier_init();
@@ -246,7 +287,37 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     if (lane == 0) {
       int it = 0;
       bool ok = true;
-      for (int u = unit0; u < nunits && ok; u += unit_step) {
+      if constexpr (DYN) {
+        if (blockIdx.x == 0) Work::begin(args);
+      }
+      for (int seq = 0; ok; ++seq) {
+        int u = unit0 + seq * unit_step;
+        if constexpr (DYN) {
+          if (leader) {
+            // take a ticket and pass it to this CTA's roles and to the pair member
+            const int e = seq % UR;
+            if (seq >= UR && !mbar_wait_cluster(smem_u32(&uempty[e]), (uint32_t)(seq / UR - 1) & 1u,
+                                                abort_flag, g.status)) {
+              ok = false;
+              break;
+            }
+            u = Work::take_ticket(args);
+            if (u > nunits) u = nunits;
+            unit_ring[e] = u;
+            mbar_arrive(smem_u32(&ufull[e]));
+            if (Cfg::PAIR) {
+              st_cluster_u32(cluster_addr(smem_u32((const void*)&unit_ring[e]), 1), (uint32_t)u);
+              mbar_arrive_cluster(cluster_addr(smem_u32(&ufull[e]), 1));
+            }
+          } else {
+            u = take_unit(seq, true);
+            if (u < 0) {
+              ok = false;
+              break;
+            }
+          }
+        }
+        if (u >= nunits) break;
         Unit w;
         Work::template decode<Cfg>(args, u, w);
         // operands written earlier in this launch are published first
@@ -351,7 +422,16 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       int it = 0;
       uint32_t q = 0;  // chunks issued: chunk q goes to slot q % R, use q / R of it
       bool ok = true;
-      for (int u = unit0; u < nunits && ok; u += unit_step) {
+      for (int seq = 0; ok; ++seq) {
+        int u = unit0 + seq * unit_step;
+        if constexpr (DYN) {
+          u = take_unit(seq, true);
+          if (u < 0) {
+            ok = false;
+            break;
+          }
+        }
+        if (u >= nunits) break;
         Unit w;
         Work::template decode<Cfg>(args, u, w);
         const int kb0 = w.kb0, kb1 = w.kb1;
@@ -439,8 +519,16 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         mbar_arrive(smem_u32(&rempty[slot]));
       }
     };
-    int seq = 0;  // units this CTA has taken
-    for (int u = unit0; u < nunits && ok; u += unit_step, ++seq) {
+    for (int seq = 0; ok; ++seq) {  // seq: units this CTA has taken
+      int u = unit0 + seq * unit_step;
+      if constexpr (DYN) {
+        u = take_unit(seq, false);
+        if (u < 0) {
+          ok = false;
+          break;
+        }
+      }
+      if (u >= nunits) break;
       Unit w;
       Work::template decode<Cfg>(args, u, w);
       const int kb0 = w.kb0, kb1 = w.kb1;
