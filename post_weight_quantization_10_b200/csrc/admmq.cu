@@ -429,15 +429,54 @@ __global__ void k_rint_div(const float* __restrict__ y, const float* __restrict_
 }
 
 // Standalone projection: one thread per (row, group), W~ read from memory.
-template <int MODE, int ENC>
-__global__ void k_project(const float* __restrict__ wt, float* V, const float* __restrict__ sig,
-                          const float* __restrict__ rsig, const float* __restrict__ hd, int m, int d,
-                          int g, int L, uint8_t* codes, float* scale, float* zero, void* p_hi,
-                          void* p_lo, const float* __restrict__ row_in, int* flag, double* resid) {
-  const int row = blockIdx.x * blockDim.x + threadIdx.x;
+// The passes over a group read each of its elements two or three times, and
+// once enough warps run to cover the memory latency their groups (2 x g
+// floats each) no longer stay in L1, so by default a block is one warp of 32
+// rows that first copies its rows' W~ and V~ segments into shared memory
+// (coalesced 16-byte asynchronous copies, a whole row segment per
+// instruction for g = 128); the passes read them from there and DRAM sees
+// each input once.  The 16-candidate error search of GRID_MSE is bound by
+// arithmetic rather than memory, so it keeps more warps per SM by reading W~
+// and V~ from global memory (STAGED = false, 128-thread blocks).
+constexpr int kProjRows = 32;
+// floats per row slot: W~ (g), V~ (g), 4 of padding so that the rows' 16-byte
+// reads at one column spread over the banks
+__host__ __device__ constexpr int proj_slot(int g) { return 2 * g + 4; }
+
+template <int MODE, int ENC, bool STAGED>
+__global__ void __launch_bounds__(STAGED ? kProjRows : 128) k_project(
+    const float* __restrict__ wt, float* V, const float* __restrict__ sig,
+    const float* __restrict__ rsig, const float* __restrict__ hd, int m, int d, int g, int L,
+    uint8_t* codes, float* scale, float* zero, void* p_hi, void* p_lo,
+    const float* __restrict__ row_in, int* flag, double* resid) {
+  extern __shared__ float4 proj_smem[];
+  float* stage = reinterpret_cast<float*>(proj_smem);
+  const int lane = threadIdx.x & 31;
+  const int row0 = blockIdx.x * blockDim.x;
   const int grp = blockIdx.y;
-  const bool valid = row < m;
   const int col0 = grp * g;
+  const int slot = proj_slot(g);
+  if (STAGED) {
+    // rows past m are filled with zeros (they are projected, never stored)
+    const int per_row = g / 2;  // float4 pieces of W~ and V~ in one row
+    const uint32_t sbase = smem_u32(stage);
+    for (int i = lane; i < kProjRows * per_row; i += 32) {
+      const int rr = i / per_row, piece = i - rr * per_row;
+      const int arr = piece >= g / 4 ? 1 : 0;
+      const int k = 4 * (piece - arr * (g / 4));
+      const int off_s = rr * slot + arr * g + k;
+      if (row0 + rr < m) {
+        const float* src = (arr ? V : wt) + (long long)(row0 + rr) * d + col0 + k;
+        cp_async16(sbase + 4u * (uint32_t)off_s, src);
+      } else {
+        *reinterpret_cast<float4*>(stage + off_s) = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    cp_async_wait_all();
+    __syncwarp();
+  }
+  const int row = row0 + (int)threadIdx.x;
+  const bool valid = row < m;
   const long long off = (long long)(valid ? row : 0) * d + col0;
   const long long goff = (long long)(valid ? row : 0) * (d / g) + grp;
   ProjRow r;
@@ -454,19 +493,33 @@ __global__ void k_project(const float* __restrict__ wt, float* V, const float* _
   r.rs = (valid && row_in) ? row_in[row] : 1.f;
   r.flag = flag;
   r.valid = valid;
+  const float* mine = stage + lane * slot;
   auto loadw = [&](int c, float (&w)[32]) {
 #pragma unroll
     for (int k = 0; k < 32; k += 4) {
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (valid) v = *reinterpret_cast<const float4*>(wt + off + c + k);
+      if (STAGED)
+        v = *reinterpret_cast<const float4*>(mine + c + k);
+      else if (valid)
+        v = *reinterpret_cast<const float4*>(wt + off + c + k);
       w[k] = v.x; w[k + 1] = v.y; w[k + 2] = v.z; w[k + 3] = v.w;
     }
   };
+  auto loadv = [&](int c, float (&v)[8]) {
+    if (STAGED) {
+      const float4 a = *reinterpret_cast<const float4*>(mine + g + c);
+      const float4 b = *reinterpret_cast<const float4*>(mine + g + c + 4);
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+      v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    } else if (valid) {
+      ld_v8f(r.V + c, v);
+    }
+  };
   float r2 = 0.f, s2 = 0.f;
-  project_group<MODE, ENC>(loadw, r, g, L, r2, s2);
+  project_group<MODE, ENC>(loadw, loadv, r, g, L, r2, s2);
   r2 = warp_sum(r2);
   s2 = warp_sum(s2);
-  if ((threadIdx.x & 31) == 0) {
+  if (lane == 0) {
     atomicAdd(&resid[0], (double)r2);
     atomicAdd(&resid[1], (double)s2);
   }
@@ -1435,13 +1488,16 @@ int admmq_project(const float* wt, float* V, const float* sig, const float* rsig
     return ADMMQ_ERR_INVALID_ARG;
   cudaStream_t st = (cudaStream_t)stream;
   CK(cudaMemsetAsync(resid, 0, 2 * sizeof(double), st));
-  dim3 grid(cdiv(m, 128), d / g);
+  const bool staged = mode != ADMMQ_GRID_MSE;
+  const int block = staged ? kProjRows : 128;
+  dim3 grid(cdiv(m, block), d / g);
+  const size_t smem = staged ? sizeof(float) * kProjRows * proj_slot(g) : 0;  // <= 33,280 bytes
   const int L = (1 << bits) - 1;
   const int enc = split == ADMMQ_SPLIT_MIXED ? ENC_MIX : (split == ADMMQ_SPLIT_F16 ? ENC_F16 : ENC_TF32X3);
-#define PROJECT_ENC(MODE, ENC)                                                                  \
-  count_launch(), k_project<MODE, ENC><<<grid, 128, 0, st>>>(wt, V, sig, rsig, hd, m, d, g, L, codes, \
-                                                             scale, zero, p_hi, p_lo, row_scale,     \
-                                                             range_flag, resid);
+#define PROJECT_ENC(MODE, ENC)                                                               \
+  count_launch(), k_project<MODE, ENC, MODE != GRID_MSE><<<grid, block, smem, st>>>(         \
+                      wt, V, sig, rsig, hd, m, d, g, L, codes, scale, zero, p_hi, p_lo,      \
+                      row_scale, range_flag, resid);
 #define PROJECT_CASE(MODE)       \
   if (enc == ENC_MIX) {          \
     PROJECT_ENC(MODE, ENC_MIX)   \

@@ -266,9 +266,9 @@ __device__ __forceinline__ void range_grid(float mn, float mx, float Lf, float& 
 // in element order with every product and sum rounded on its own; the first
 // smallest error wins.  The group is read once per 32-column chunk; the
 // candidates run in an outer loop over the chunk's y held in registers.
-template <class LoadW>
-__device__ __forceinline__ void mse_clip_grid(LoadW& loadw, const ProjRow& r, int g, float Lf,
-                                              float mn, float mx, float& s, float& z) {
+template <class LoadW, class LoadV>
+__device__ __forceinline__ void mse_clip_grid(LoadW& loadw, LoadV& loadv, const ProjRow& r, int g,
+                                              float Lf, float mn, float mx, float& s, float& z) {
   float ce[kClipCandidates];
 #pragma unroll
   for (int k = 0; k < kClipCandidates; ++k) ce[k] = 0.f;
@@ -279,7 +279,7 @@ __device__ __forceinline__ void mse_clip_grid(LoadW& loadw, const ProjRow& r, in
 #pragma unroll
     for (int e = 0; e < 32; e += 8) {
       float vv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      if (r.valid) ld_v8f(r.V + c + e, vv);
+      loadv(c + e, vv);
       float ss[8];
       load8_ro(r.sig + c + e, ss);
 #pragma unroll
@@ -320,9 +320,12 @@ __device__ __forceinline__ void mse_clip_grid(LoadW& loadw, const ProjRow& r, in
   }
 }
 
-template <int MODE, int ENC, class LoadW>
-__device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, int g, int L,
-                                              float& r2, float& s2) {
+// loadw(c, w[32]) gives W~ at columns c .. c + 31 of the group, loadv(c,
+// v[8]) the dual V~ at c .. c + 7 (left at zero for an invalid row); the new
+// V~ is stored through r.V.
+template <int MODE, int ENC, class LoadW, class LoadV>
+__device__ __forceinline__ void project_group(LoadW&& loadw, LoadV&& loadv, const ProjRow& r,
+                                              int g, int L, float& r2, float& s2) {
   const float Lf = (float)L;
   float s0 = 1.f, z0 = 0.f;
   if (r.valid) {  // L2 reads: another SM may have written them in this launch
@@ -341,7 +344,7 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, i
 #pragma unroll
       for (int e = 0; e < 32; e += 8) {
         float vv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (r.valid) ld_v8f(r.V + c + e, vv);
+        loadv(c + e, vv);
         float ss[8], hh[8], y8[8], q8[8];
         load8_ro(r.sig + c + e, ss);
         if (MODE == GRID_LSQ) load8_ro(r.hd + c + e, hh);
@@ -370,7 +373,7 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, i
     if (MODE == GRID_MINMAX) {
       range_grid(mn, mx, Lf, s, z);
     } else if (MODE == GRID_MSE) {
-      mse_clip_grid(loadw, r, g, Lf, mn, mx, s, z);
+      mse_clip_grid(loadw, loadv, r, g, Lf, mn, mx, s, z);
     } else {
       const float qm = __fdiv_rn(Sq, Sw);
       const float ym = __fdiv_rn(Sy, Sw);
@@ -398,7 +401,7 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, const ProjRow& r, i
 #pragma unroll
     for (int e = 0; e < 32; e += 8) {
       float vv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      if (r.valid) ld_v8f(r.V + c + e, vv);
+      loadv(c + e, vv);
       float ss[8], rr[8], t8[8], y8[8], q8[8];
       load8_ro(r.sig + c + e, ss);
       load8_ro(r.rsig + c + e, rr);
@@ -622,7 +625,10 @@ struct EpiProject {
 #pragma unroll
         for (int k = 0; k < 32; ++k) w[k] = __fmul_rn(w[k], ro);
       };
-      project_group<MODE, ENC>(loadw, r, p.group, p.L, r2, s2);
+      auto loadv = [&](int c, float (&v)[8]) {
+        if (valid) ld_v8f(r.V + c, v);
+      };
+      project_group<MODE, ENC>(loadw, loadv, r, p.group, p.L, r2, s2);
     }
     r2 = warp_sum(r2);
     s2 = warp_sum(s2);
