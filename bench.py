@@ -17,6 +17,7 @@ layer (seed = rank) with no collective in the data path ("scaling": "weak").
 from __future__ import annotations
 
 import argparse
+import datetime
 import json
 import os
 import statistics
@@ -81,23 +82,41 @@ def workload_desc(p, grid):
 
 
 class ClockSampler:
-    def __init__(self, gpu_index: int):
+    """SM clock, power and throttle reasons from `nvidia-smi -lms 50`, started
+    before the warm-up (its first sample takes a moment to arrive).  Only the
+    samples whose timestamps fall inside the timed windows (host wall clock,
+    begin() .. end(), taken after a device synchronize on both sides) are
+    reported."""
+
+    def __init__(self, gpu_index: int, interval_ms: int = 50):
         self.gpu = gpu_index
+        self.interval = interval_ms
         self.proc = None
         self.path = None
+        self.windows = []
+        self._t0 = None
 
     def start(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+        q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
              "clocks_event_reasons.sw_power_cap")
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "200",
-                 "-i", str(self.gpu)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms",
+                 str(self.interval), "-i", str(self.gpu)],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+
+    def begin(self):
+        self._t0 = time.time()
+
+    def end(self):
+        if self._t0 is not None:
+            self.windows.append((self._t0, time.time()))
+        self._t0 = None
 
     def stop(self):
         if self.proc is None:
@@ -107,25 +126,30 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-        sm, mx, reasons = [], None, set()
+        rows = []
         with open(self.path) as f:
             for line in f:
                 parts = [x.strip() for x in line.split(",")]
-                if len(parts) < 8:
+                if len(parts) < 9:
                     continue
                 try:
-                    sm.append(float(parts[1]))
-                    mx = float(parts[2])
+                    t = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    rows.append((t, float(parts[2]), float(parts[3]), parts[5:9]))
                 except ValueError:
                     continue
-                for name, val in zip(REASONS, parts[4:8]):
-                    if val.lower().startswith("active"):
-                        reasons.add(name)
         os.unlink(self.path)
-        if not sm:
+        inside = [r for r in rows if any(a <= r[0] <= b for a, b in self.windows)]
+        if not inside:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        sm = [r[1] for r in inside]
+        reasons = set()
+        for r in inside:
+            for name, val in zip(REASONS, r[3]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": inside[-1][2],
+                "reasons": sorted(reasons), "samples": len(inside),
+                "window_s": round(sum(b - a for a, b in self.windows), 3)}
 
 
 # ------------------------------------------------------------- our solver
@@ -261,23 +285,25 @@ def run_sharded(args, rank, world, device):
     if args.tokens:
         p = workloads.scaled(p, args.tokens, p.d_in, p.d_out)
     run = ShardRun(A, p, args.grid, rank, world, device, split=args.split, schedule=args.schedule)
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
     eigh_s = run.setup_eigh()
     for _ in range(args.warmup):
         run.step()
     torch.cuda.synchronize()
     dist_barrier(world)
     torch.cuda.synchronize()
-    clocks = ClockSampler(torch.cuda.current_device())
-    clocks.start()
     n0 = A.launch_count()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
+    clocks.begin()
     a.record()
     for k in range(args.steps):
         run.step(evs[k])
     b.record()
     torch.cuda.synchronize()
+    clocks.end()
     dist_barrier(world)
     clk = clocks.stop()
     ms = dist_max(a.elapsed_time(b), world, device)
@@ -329,11 +355,13 @@ def run_decoder(args, rank, world, device):
         dist_barrier(world)
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
+        clocks.begin()
         a.record()
         for _ in range(args.steps):
             run.step()
         b.record()
         torch.cuda.synchronize()
+        clocks.end()
         ms = dist_max(a.elapsed_time(b), world, device) / args.steps
         obj = objective_report(A, run)
         solves.append({"solve": label, "d_in": p.d_in, "d_out": p.d_out, "bits": p.bits,
@@ -372,6 +400,8 @@ def run_ours(args, rank, world, device):
         p = workloads.scaled(p, args.tokens, p.d_in, p.d_out)
     run = LayerRun(A, p, args.grid, seed=rank, device=device, split=args.split,
                    scaling=not args.no_scaling, schedule=args.schedule)
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
     eigh_s = run.setup_eigh()
     for _ in range(args.warmup):
         run.step()
@@ -380,18 +410,18 @@ def run_ours(args, rank, world, device):
     # ---- device-resident timed region
     dist_barrier(world)
     torch.cuda.synchronize()
-    clocks = ClockSampler(torch.cuda.current_device())
-    clocks.start()
     run.s.set_timing(True)
     n0 = A.launch_count()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    clocks.begin()
     t_start.record()
     for k in range(args.steps):
         run.step(evs[k])
     t_end.record()
     torch.cuda.synchronize()
+    clocks.end()
     dist_barrier(world)
     launches = A.launch_count() - n0
     clk = clocks.stop()
@@ -707,7 +737,7 @@ def dist_max(v, world, device):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="q_proj", choices=sorted(workloads.PRESETS) + ["decoder"],
