@@ -281,6 +281,34 @@ def test_fused_schedule_matches_per_gemm(A, name, grid, split):
             assert torch.equal(v, ref[k]), (sched, k)
 
 
+def test_fused_schedule_shares_the_gpu(A):
+    """The fused launch deals its tiles from a counter to whichever CTAs are
+    running, so it needs no particular number of them resident: while a
+    second stream keeps SMs busy with matrix products, the solve finishes
+    without a wait timing out and gives the bits of a solve run alone."""
+    p = workloads.scaled(workloads.PRESETS["q_proj"], 4096, 1024, 3000, rank=16)
+    X = workloads.make_activations(p, seed=3, device="cuda")
+    W = workloads.make_weights(p, seed=3, device="cuda", dtype=torch.float32)
+    alone = _solver(A, p, X, W, "lsq", schedule="fused")
+    alone.solve()
+    torch.cuda.synchronize()
+    ref = (alone.codes.cpu().clone(), alone.buffer("V").cpu().clone(), alone.objective.cpu().clone())
+    side = torch.cuda.Stream()
+    a = torch.randn(4096, 4096, device="cuda")
+    s = _solver(A, p, X, W, "lsq", schedule="fused")
+    torch.cuda.synchronize()
+    with torch.cuda.stream(side):
+        for _ in range(40):
+            a = torch.tanh(a @ a * 1e-3)
+    s.solve()
+    torch.cuda.synchronize()
+    assert s.kernel_status() == 0
+    s.check()
+    assert torch.equal(s.codes.cpu(), ref[0])
+    assert torch.equal(s.buffer("V").cpu(), ref[1])
+    assert torch.equal(s.objective.cpu(), ref[2])
+
+
 def test_pipeline_matches_separate_solves(A):
     """solve_layers (next layer's inputs copied on a second stream during the
     current solve) gives each layer the same bits as solving it alone."""
