@@ -440,8 +440,10 @@ __global__ void k_rint_div(const float* __restrict__ y, const float* __restrict_
 // and V~ from global memory (STAGED = false, 128-thread blocks).
 constexpr int kProjRows = 32;
 // floats per row slot: W~ (g), V~ (g), 4 of padding so that the rows' 16-byte
-// reads at one column spread over the banks
+// reads at one column spread over the banks; after the 32 row slots, the
+// group's sigma, 1/sigma and diag(H) (g each), shared by the block's rows
 __host__ __device__ constexpr int proj_slot(int g) { return 2 * g + 4; }
+__host__ __device__ constexpr int proj_floats(int g) { return kProjRows * proj_slot(g) + 3 * g; }
 
 template <int MODE, int ENC, bool STAGED>
 __global__ void __launch_bounds__(STAGED ? kProjRows : 128) k_project(
@@ -472,6 +474,14 @@ __global__ void __launch_bounds__(STAGED ? kProjRows : 128) k_project(
         *reinterpret_cast<float4*>(stage + off_s) = make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
+    float* cols = stage + kProjRows * slot;
+    for (int i = lane; i < 3 * (g / 4); i += 32) {
+      const int v = i / (g / 4), k = 4 * (i - v * (g / 4));
+      const float* src = (v == 0 ? sig : v == 1 ? rsig : hd) + col0 + k;
+      cp_async16(smem_u32(cols + v * g + k), src);
+    }
+    // the codes of this lane's row, read in the projection pass
+    if (row0 + lane < m) prefetch_l2_bulk(codes + (long long)(row0 + lane) * d + col0, (uint32_t)g);
     cp_async_wait_all();
     __syncwarp();
   }
@@ -481,9 +491,16 @@ __global__ void __launch_bounds__(STAGED ? kProjRows : 128) k_project(
   const long long goff = (long long)(valid ? row : 0) * (d / g) + grp;
   ProjRow r;
   r.V = V + off;
-  r.sig = sig + col0;
-  r.rsig = rsig + col0;
-  r.hd = hd + col0;
+  if (STAGED) {
+    const float* cols = stage + kProjRows * slot;
+    r.sig = cols;
+    r.rsig = cols + g;
+    r.hd = cols + 2 * g;
+  } else {
+    r.sig = sig + col0;
+    r.rsig = rsig + col0;
+    r.hd = hd + col0;
+  }
   r.codes = codes + off;
   r.phi = plane0_at(ENC, p_hi, valid ? row : 0, d, col0);
   r.plo = plane1_at(ENC, p_lo, valid ? row : 0, d, col0);
@@ -516,7 +533,7 @@ __global__ void __launch_bounds__(STAGED ? kProjRows : 128) k_project(
     }
   };
   float r2 = 0.f, s2 = 0.f;
-  project_group<MODE, ENC>(loadw, loadv, r, g, L, r2, s2);
+  project_group<MODE, ENC, STAGED>(loadw, loadv, r, g, L, r2, s2);
   r2 = warp_sum(r2);
   s2 = warp_sum(s2);
   if (lane == 0) {
@@ -1491,7 +1508,7 @@ int admmq_project(const float* wt, float* V, const float* sig, const float* rsig
   const bool staged = mode != ADMMQ_GRID_MSE;
   const int block = staged ? kProjRows : 128;
   dim3 grid(cdiv(m, block), d / g);
-  const size_t smem = staged ? sizeof(float) * kProjRows * proj_slot(g) : 0;  // <= 33,280 bytes
+  const size_t smem = staged ? sizeof(float) * proj_floats(g) : 0;  // <= 34,816 bytes
   const int L = (1 << bits) - 1;
   const int enc = split == ADMMQ_SPLIT_MIXED ? ENC_MIX : (split == ADMMQ_SPLIT_F16 ? ENC_F16 : ENC_TF32X3);
 #define PROJECT_ENC(MODE, ENC)                                                               \

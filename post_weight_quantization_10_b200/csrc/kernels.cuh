@@ -214,6 +214,20 @@ __device__ __forceinline__ void load8_ro(const float* p, float (&v)[8]) {
   v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
+// Eight floats of a per-column vector (sigma, 1/sigma, diag(H)): through the
+// read-only path from global memory, or from a copy in shared memory.
+template <bool SMEM>
+__device__ __forceinline__ void load8_col(const float* p, float (&v)[8]) {
+  if (SMEM) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    const float4 b = *reinterpret_cast<const float4*>(p + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+    load8_ro(p, v);
+  }
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -266,7 +280,7 @@ __device__ __forceinline__ void range_grid(float mn, float mx, float Lf, float& 
 // in element order with every product and sum rounded on its own; the first
 // smallest error wins.  The group is read once per 32-column chunk; the
 // candidates run in an outer loop over the chunk's y held in registers.
-template <class LoadW, class LoadV>
+template <bool COLS_SMEM, class LoadW, class LoadV>
 __device__ __forceinline__ void mse_clip_grid(LoadW& loadw, LoadV& loadv, const ProjRow& r, int g,
                                               float Lf, float mn, float mx, float& s, float& z) {
   float ce[kClipCandidates];
@@ -281,7 +295,7 @@ __device__ __forceinline__ void mse_clip_grid(LoadW& loadw, LoadV& loadv, const 
       float vv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       loadv(c + e, vv);
       float ss[8];
-      load8_ro(r.sig + c + e, ss);
+      load8_col<COLS_SMEM>(r.sig + c + e, ss);
 #pragma unroll
       for (int j = 0; j < 8; ++j) y[e + j] = __fmul_rn(ss[j], __fadd_rn(y[e + j], vv[j]));
     }
@@ -322,8 +336,9 @@ __device__ __forceinline__ void mse_clip_grid(LoadW& loadw, LoadV& loadv, const 
 
 // loadw(c, w[32]) gives W~ at columns c .. c + 31 of the group, loadv(c,
 // v[8]) the dual V~ at c .. c + 7 (left at zero for an invalid row); the new
-// V~ is stored through r.V.
-template <int MODE, int ENC, class LoadW, class LoadV>
+// V~ is stored through r.V.  COLS_SMEM: r.sig, r.rsig and r.hd point into
+// shared memory.
+template <int MODE, int ENC, bool COLS_SMEM = false, class LoadW, class LoadV>
 __device__ __forceinline__ void project_group(LoadW&& loadw, LoadV&& loadv, const ProjRow& r,
                                               int g, int L, float& r2, float& s2) {
   const float Lf = (float)L;
@@ -346,8 +361,8 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, LoadV&& loadv, cons
         float vv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         loadv(c + e, vv);
         float ss[8], hh[8], y8[8], q8[8];
-        load8_ro(r.sig + c + e, ss);
-        if (MODE == GRID_LSQ) load8_ro(r.hd + c + e, hh);
+        load8_col<COLS_SMEM>(r.sig + c + e, ss);
+        if (MODE == GRID_LSQ) load8_col<COLS_SMEM>(r.hd + c + e, hh);
 #pragma unroll
         for (int k = 0; k < 8; ++k) y8[k] = __fmul_rn(ss[k], __fadd_rn(w[e + k], vv[k]));
         if (MODE == GRID_LSQ) rint_div8(y8, s0, r0, q8);
@@ -373,7 +388,7 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, LoadV&& loadv, cons
     if (MODE == GRID_MINMAX) {
       range_grid(mn, mx, Lf, s, z);
     } else if (MODE == GRID_MSE) {
-      mse_clip_grid(loadw, loadv, r, g, Lf, mn, mx, s, z);
+      mse_clip_grid<COLS_SMEM>(loadw, loadv, r, g, Lf, mn, mx, s, z);
     } else {
       const float qm = __fdiv_rn(Sq, Sw);
       const float ym = __fdiv_rn(Sy, Sw);
@@ -403,8 +418,8 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, LoadV&& loadv, cons
       float vv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       loadv(c + e, vv);
       float ss[8], rr[8], t8[8], y8[8], q8[8];
-      load8_ro(r.sig + c + e, ss);
-      load8_ro(r.rsig + c + e, rr);
+      load8_col<COLS_SMEM>(r.sig + c + e, ss);
+      load8_col<COLS_SMEM>(r.rsig + c + e, rr);
       float vn[8], pv[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
