@@ -201,10 +201,10 @@ int admmq_init(admmq_ctx* ctx, uint8_t* codes_dev, float* scale_dev, float* zero
  *   W~ = Q T;  D = grid projection of Sigma (W~ + V~);  V~ += W~ - D~  (GEMM 2
  *        with the projection, the dual update and residual sums fused)
  * codes/scale/zero are updated in place (they hold D).  t0 + count <= iters.
- * With ADMMQ_SCHEDULE_FUSED each iteration is one kernel launch.  Its waits for
- * other units are bounded like the pipeline waits: one that gives up sets the
- * kernel status word (ADMMQ_BUF_STATUS[0] = 1, "timed out") and the launch
- * ends. */
+ * With ADMMQ_SCHEDULE_FUSED the count iterations are one kernel launch.  Its
+ * waits for other units are bounded like the pipeline waits: one that gives up
+ * sets the kernel status word (ADMMQ_BUF_STATUS[0] = 1, "timed out") and the
+ * launch ends. */
 int admmq_iterate(admmq_ctx* ctx, int t0, int count, uint8_t* codes_dev, float* scale_dev,
                   float* zero_dev, void* stream);
 
