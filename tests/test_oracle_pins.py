@@ -233,6 +233,20 @@ def test_minmax_grid_hand_example():
     np.testing.assert_array_equal(P.dequantize(q, s, z)[0], [-1, 0, 2])
 
 
+def test_minmax_grid_one_signed_groups():
+    """The range always includes 0, so a one-signed group still gets a grid
+    with 0 on it and an integer zero point in [0, L]: y = (0.5, 1, 2), 2 bits:
+    mn = 0, mx = 2, s = 2/3, z = 0, codes (1, 2, 3); y = (-2, -1, -0.5): mn =
+    -2, mx = 0, s = 2/3, z = rint(2 / fl(2/3)) = 3, codes (0, 1, 2) with
+    rint(-1.5) = -2 (ties to even)."""
+    f = np.float32
+    y = np.array([[0.5, 1.0, 2.0], [-2.0, -1.0, -0.5]], f)
+    s, z = P.fit_minmax(y, 3)
+    np.testing.assert_array_equal(s, [f(2) / f(3), f(2) / f(3)])
+    np.testing.assert_array_equal(z, [0.0, 3.0])
+    np.testing.assert_array_equal(P.round_to_grid(y, s, z, 3), [[1, 2, 3], [0, 1, 2]])
+
+
 def test_minmax_grid_all_zero_group():
     y = np.zeros((1, 8), np.float32)
     s, z = P.fit_minmax(y, 7)
@@ -369,6 +383,69 @@ def test_lsq_refit_does_not_increase_weighted_error():
     e0, e1 = err(s0, z0), err(s1, z1)
     assert np.mean(e1 <= e0 * (1 + 1e-6)) > 0.95
     assert e1.sum() < e0.sum()
+
+
+def _epilogue_inputs(m, d, g, bits, seed):
+    """A [d_out][d_in] tile of W~ and V~ with a scaling vector, its inverse,
+    diag(H) = 1/sigma^2, and a previous grid and codes (the min/max RTN grid
+    of a perturbed W~)."""
+    rng = np.random.default_rng(seed)
+    L = (1 << bits) - 1
+    W = (rng.standard_normal((m, d)) * 0.05).astype(np.float32)
+    V = (rng.standard_normal((m, d)) * 0.005).astype(np.float32)
+    sig = (rng.random(d) + 0.5).astype(np.float32)
+    rsig = (1.0 / sig.astype(np.float64)).astype(np.float32)
+    hd = (rsig.astype(np.float64) ** 2).astype(np.float32)
+    prev = (W * 1.1).reshape(m * (d // g), g)
+    s0, z0 = P.fit_minmax(prev, L)
+    c0 = P.round_to_grid(prev, s0, z0, L).reshape(m, d).astype(np.uint8)
+    return W, V, sig, rsig, hd, s0.reshape(m, d // g), z0.reshape(m, d // g), c0
+
+
+@pytest.mark.parametrize("mode", ["minmax", "lsq", "mse", "frozen"])
+@pytest.mark.parametrize("bits,g,m,d", [(3, 32, 5, 96), (2, 64, 3, 128), (4, 32, 4, 64)])
+def test_epilogue_step_follows_the_d_and_dual_updates(mode, bits, g, m, d):
+    """The memory-layout ([d_out][d_in]) statement of one fused step against
+    the D-update of the float64 route (oracle.admmq_oracle.project, the
+    [d_in][d_out] layout) on the same float32 iterate y = sigma (W~ + V~),
+    and against the dual and residual definitions taken in float64:
+    V~' = (W~ + V~) - D~, P = D~ - V~' (so P = 2 D~ - (W~ + V~) up to
+    rounding), D~ = D / sigma, r2 = ||W~ - D~||^2, s2 = ||D~ - D~_prev||^2."""
+    W, V, sig, rsig, hd, s0, z0, c0 = _epilogue_inputs(m, d, g, bits, seed=bits + g + m)
+    out = P.epilogue_step(W, V, sig, rsig, hd, s0, z0, c0, bits, g, mode)
+    t = (W + V).astype(np.float32)
+    y = (sig[None, :] * t).astype(np.float32)
+    codes, sc, ze, D = O.project(y.T, bits, g, mode, hd, s0.T, z0.T)
+    np.testing.assert_array_equal(out["codes"], codes.T)
+    np.testing.assert_array_equal(out["scale"], sc.T)
+    np.testing.assert_array_equal(out["zero"], ze.T)
+    Dt = D.T / sig.astype(np.float64)[None, :]
+    f = np.float64
+    assert np.allclose(out["P"].astype(f) + out["V"].astype(f) - Dt, 0, atol=4e-7 * np.abs(Dt).max())
+    assert np.allclose(out["V"].astype(f), t.astype(f) - Dt, atol=4e-7 * np.abs(t).max())
+    assert np.allclose(out["P"].astype(f), 2 * Dt - t.astype(f), atol=8e-7 * np.abs(t).max())
+    L = (1 << bits) - 1
+    lev_prev = s0.astype(f).repeat(g, axis=1) * (c0.astype(f) - z0.astype(f).repeat(g, axis=1))
+    Dt_prev = lev_prev / sig.astype(f)[None, :]
+    assert out["r2"] == pytest.approx(np.sum((W.astype(f) - Dt) ** 2), rel=1e-5)
+    assert out["s2"] == pytest.approx(np.sum((Dt - Dt_prev) ** 2), rel=1e-5, abs=1e-12)
+    assert out["codes"].max() <= L
+
+
+@pytest.mark.parametrize("bits,g,m,d", [(3, 32, 6, 96), (2, 64, 2, 128), (8, 32, 3, 64)])
+def test_init_step_is_rtn_in_memory_layout(bits, g, m, d):
+    """The RTN start in [d_out][d_in] layout equals oracle.admmq_oracle.rtn on
+    the [d_in][d_out] matrix, with P = D~ = D / sigma and V~ = 0."""
+    rng = np.random.default_rng(bits * 7 + g)
+    Wr = (rng.standard_normal((m, d)) * 0.05).astype(np.float32)
+    sig = (rng.random(d) + 0.5).astype(np.float32)
+    rsig = (1.0 / sig.astype(np.float64)).astype(np.float32)
+    out = P.init_step(Wr, rsig, bits, g)
+    codes, sc, ze, D = O.rtn(Wr.T, bits, g)
+    np.testing.assert_array_equal(out["codes"], codes.T)
+    np.testing.assert_array_equal(out["scale"], sc.T)
+    np.testing.assert_array_equal(out["zero"], ze.T)
+    np.testing.assert_allclose(out["P"], D.T / sig.astype(np.float64)[None, :], rtol=2e-7, atol=0)
 
 
 def test_tf32_split_reconstructs_float32():
