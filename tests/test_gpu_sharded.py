@@ -55,7 +55,12 @@ def test_row_blocks_reproduce_the_whole_layer(A):
         obj += float(s.objective.cpu())
     torch.cuda.synchronize()
     assert torch.equal(torch.cat(parts), whole.codes)
-    assert obj == pytest.approx(float(whole.objective.cpu()), rel=1e-9)
+    # Same codes, hence the same D; the objective is summed from float32
+    # partials per 32-row warp and 128-row tile, and the row blocks start a
+    # tile at row 300 where the whole layer does not, so the two totals
+    # group the rows differently: they agree to the rounding of float32
+    # partial sums of ~160 terms (~1e-6 relative), not bit for bit.
+    assert obj == pytest.approx(float(whole.objective.cpu()), rel=1e-6)
 
 
 def test_token_blocks_sum_to_the_whole_gram(A):
