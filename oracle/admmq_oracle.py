@@ -175,7 +175,8 @@ def w_update(Q: np.ndarray, lam: np.ndarray, B: np.ndarray, rho: float,
 
 def admm_q(H: np.ndarray, W_hat: np.ndarray, bits: int, group: int, iters: int,
            rho0: float = 0.1, gamma: float = 1.05, grid: str = "minmax",
-           scaling: bool = True, eig=None, grid0=None, trace=None) -> dict:
+           scaling: bool = True, eig=None, grid0=None, trace=None,
+           rescale_dual: bool = False) -> dict:
     """The ADMM-Q layer solve, step by step in the pages' order.
 
     1. Sigma = Diag(H)^(-1/2); H~ = Sigma H Sigma; W^~ = Sigma^-1 W_hat.
@@ -188,6 +189,10 @@ def admm_q(H: np.ndarray, W_hat: np.ndarray, bits: int, group: int, iters: int,
     5. Return the last D as codes + per-group scale/zero, and its objective.
 
     `scaling=False` replaces Sigma by the identity (the pages' ablation).
+    `rescale_dual=True` multiplies V~ by rho_t / rho_{t+1} after its update, so
+    that the unscaled dual rho V~ carries over unchanged when the penalty
+    grows (the pages say nothing on this; without the flag V~ is literally
+    V~ + W~ - D~, the reading the default follows).
     `eig` optionally passes a precomputed (Lambda, Q) of H~; `grid0` an
     initial (scale, zero) pair ((d_in/group) x d_out each) replacing the RTN
     grid of W_hat (the start D is then W_hat rounded on that grid).
@@ -223,6 +228,8 @@ def admm_q(H: np.ndarray, W_hat: np.ndarray, bits: int, group: int, iters: int,
         codes_new, s, z, D = project(Y, bits, group, grid, hdiag, s, z)
         Dt_new = D / sigma[:, None]
         Vt = Vt + Wt - Dt_new
+        if rescale_dual:
+            Vt = Vt * (rho / (rho0 * gamma ** (t + 1)))
         if entry is not None:
             entry.update(W_tilde=Wt.copy(), Y=Y.copy(), codes_out=codes_new.copy(),
                          scale_out=s.copy(), zero_out=z.copy(), Vt_out=Vt.copy())

@@ -260,7 +260,7 @@ def init_step(W_rows: np.ndarray, rsig: np.ndarray, bits: int, group: int, split
 def epilogue_step(W_acc: np.ndarray, V: np.ndarray, sigma: np.ndarray, rsig: np.ndarray,
                   hdiag: np.ndarray, s_prev: np.ndarray, z_prev: np.ndarray,
                   codes_prev: np.ndarray, bits: int, group: int, mode: str,
-                  split: str = "mixed", row_scale=None):
+                  split: str = "mixed", row_scale=None, dual_scale=None):
     """One fused projection + dual update in memory layout ([d_out][d_in]).
 
     Per element (i = input channel):
@@ -268,6 +268,8 @@ def epilogue_step(W_acc: np.ndarray, V: np.ndarray, sigma: np.ndarray, rsig: np.
       grid (minmax | lsq | mse | frozen) per group of `group` columns of one row
       q  = clamp(rint(y/s) + z, 0, L),  D = s (q - z),  D~ = D * rsig_i
       V~' = t - D~          P  = D~ - V~'   (in the operand encoding of `split`)
+    With `dual_scale` r (the dual rescaling rho_t / rho_{t+1}, a float32):
+      V~' = (t - D~) r, rounded after the subtraction and after the product.
     Residual sums (float64 here; the kernels sum in float32, compared with a
     tolerance): r2 = sum (W~ - D~)^2 and s2 = sum (D~ - D~_prev)^2 where
     D~_prev = s_prev (q_prev - z_prev) * rsig.
@@ -296,6 +298,8 @@ def epilogue_step(W_acc: np.ndarray, V: np.ndarray, sigma: np.ndarray, rsig: np.
     D = dequantize(q, s, z).reshape(m, d)
     Dt = _f(D * _f(rsig)[None, :])
     V_new = _f(t - Dt)
+    if dual_scale is not None:
+        V_new = _f(V_new * f32(dual_scale))
     P = _f(Dt - V_new)
     hi, lo = encode_operand(P, split, "A", row_scale)
     qp = _rows_to_groups(_f(codes_prev), group)

@@ -33,6 +33,7 @@ struct AdmmLoop {
     typename Epi1::Params p1;      // rho taken per unit from rho[t]
     typename Epi2::Params p2;      // part taken per unit: part0 + t * part_stride
     const float* rho;              // [iterations] rho_t
+    const float* vscale;           // [iterations] dual rescaling after iteration t
     float* part0;
     long long part_stride;
     int* ready;                    // [2][tiles_mu] finished CTA tiles per row block
@@ -91,6 +92,7 @@ struct AdmmLoop {
                                   int col0) {
     typename Epi2::Params p = x.p2;
     p.part = x.part0 + (long long)w.t * x.part_stride;
+    p.vs = x.vscale[w.t];
     Epi2::apply_tmem(p, x.g, ta, tile_m, rit, col0);
   }
   __device__ static int* done_counter(const Args& x, const Unit& w) {

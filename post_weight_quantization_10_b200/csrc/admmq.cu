@@ -451,7 +451,7 @@ __global__ void __launch_bounds__(STAGED ? kProjRows : 128) k_project(
     const float* __restrict__ wt, float* V, const float* __restrict__ sig,
     const float* __restrict__ rsig, const float* __restrict__ hd, int m, int d, int g, int L,
     uint8_t* codes, float* scale, float* zero, void* p_hi, void* p_lo,
-    const float* __restrict__ row_in, int* flag, double* resid) {
+    const float* __restrict__ row_in, int* flag, double* resid, float vs) {
   extern __shared__ float4 proj_smem[];
   float* stage = reinterpret_cast<float*>(proj_smem);
   const int lane = threadIdx.x & 31;
@@ -509,6 +509,7 @@ __global__ void __launch_bounds__(STAGED ? kProjRows : 128) k_project(
   r.zero = zero + goff;
   r.wdump = nullptr;
   r.rs = (valid && row_in) ? row_in[row] : 1.f;
+  r.vs = vs;
   r.flag = flag;
   r.valid = valid;
   const float* mine = stage + lane * slot;
@@ -789,6 +790,7 @@ struct admmq_ctx {
   float* resid_part;    // [iters][tiles][4][2]
   float* obj_part;      // [tiles][4]
   float* rho_tab;       // [iters] rho_t, as the host computes it
+  float* vscale_tab;    // [iters] the dual's factor after iteration t (1 without rescaling)
   int* ready;           // [2][unit rows] ready counters of the fused schedule
   int ready_base;       // iterations counted in `ready` since admmq_init zeroed it
   int* ticket;          // [2] unit tickets of the fused launches, used alternately
@@ -852,7 +854,7 @@ Layout make_layout(int d, int m, int iters, int lwork) {
   L.V = take(4 * md);
   L.resid_part = take(4 * (size_t)(iters > 0 ? iters : 1) * tiles * 8);
   L.obj_part = take(4 * (size_t)tiles * 4);
-  L.rho_tab = take(4 * (size_t)(iters > 0 ? iters : 1));
+  L.rho_tab = take(4 * 2 * (size_t)(iters > 0 ? iters : 1));  // rho_t, then the dual factors
   L.ready = take(4 * (2 * (size_t)cdiv(m, 2 * kBM) + 2));  // counters, then 2 tickets
   L.row_in = take(4 * (size_t)m);
   L.row_out = take(4 * (size_t)m);
@@ -874,6 +876,15 @@ float rho_at(const admmq_params& p, int t) {
   return (float)((double)p.rho0 * pow((double)p.gamma, (double)t));
 }
 
+// Factor applied to V~ after iteration t: rho_t / rho_{t+1} (evaluated in
+// double, rounded once) with params.rescale_dual, else exactly 1.
+float vscale_at(const admmq_params& p, int t) {
+  if (!p.rescale_dual) return 1.f;
+  const double a = (double)p.rho0 * pow((double)p.gamma, (double)t);
+  const double b = (double)p.rho0 * pow((double)p.gamma, (double)(t + 1));
+  return (float)(a / b);
+}
+
 int check_params(int d, int m, const admmq_params* p) {
   if (!p) return ADMMQ_ERR_INVALID_ARG;
   if (d <= 0 || m <= 0 || d % 32 != 0) return ADMMQ_ERR_INVALID_ARG;
@@ -886,6 +897,7 @@ int check_params(int d, int m, const admmq_params* p) {
   if (p->split_mode < ADMMQ_SPLIT_AUTO || p->split_mode > ADMMQ_SPLIT_F16)
     return ADMMQ_ERR_INVALID_ARG;
   if (p->no_scaling != 0 && p->no_scaling != 1) return ADMMQ_ERR_INVALID_ARG;
+  if (p->rescale_dual != 0 && p->rescale_dual != 1) return ADMMQ_ERR_INVALID_ARG;
   if (p->schedule != ADMMQ_SCHEDULE_FUSED && p->schedule != ADMMQ_SCHEDULE_PER_GEMM)
     return ADMMQ_ERR_INVALID_ARG;
   return ADMMQ_OK;
@@ -979,6 +991,7 @@ cudaError_t launch_admm_loop(const admmq_ctx* c, const GemmGeom& g, const TUpdat
   x.p1 = p1;
   x.p2 = p2;
   x.rho = c->rho_tab;
+  x.vscale = c->vscale_tab;
   x.part0 = c->resid_part;
   x.part_stride = (long long)c->tiles_eig * 8;
   x.ready = c->ready;
@@ -1024,7 +1037,7 @@ const char* admmq_status_string(int s) {
   }
 }
 
-int admmq_version(void) { return 100; }
+int admmq_version(void) { return 101; }
 
 int64_t admmq_launch_count(void) { return (int64_t)__atomic_load_n(&g_launches, __ATOMIC_RELAXED); }
 
@@ -1123,6 +1136,7 @@ int admmq_create(admmq_ctx** out, int d, int m, const admmq_params* p, void* ws,
   c->resid_part = (float*)(b + L.resid_part);
   c->obj_part = (float*)(b + L.obj_part);
   c->rho_tab = (float*)(b + L.rho_tab);
+  c->vscale_tab = c->rho_tab + (p->iters > 0 ? p->iters : 1);
   c->ready = (int*)(b + L.ready);
   c->ticket = c->ready + 2 * cdiv(m, 2 * kBM);
   c->tiles_eig = eig_tiles(m, d);
@@ -1242,9 +1256,13 @@ int admmq_init(admmq_ctx* c, uint8_t* codes, float* scale, float* zero, void* st
         c->V, c->P_hi, c->P_lo, c->enc, c->row_in, flag);
   CK(cudaGetLastError());
   if (c->p.iters > 0) {
-    std::vector<float> rho(c->p.iters);
-    for (int t = 0; t < c->p.iters; ++t) rho[t] = rho_at(c->p, t);
-    CK(cudaMemcpyAsync(c->rho_tab, rho.data(), sizeof(float) * rho.size(), cudaMemcpyHostToDevice, st));
+    const int T = c->p.iters;
+    std::vector<float> tab(2 * (size_t)T);  // rho_t, then the dual factors (adjacent in the workspace)
+    for (int t = 0; t < T; ++t) {
+      tab[t] = rho_at(c->p, t);
+      tab[T + t] = vscale_at(c->p, t);
+    }
+    CK(cudaMemcpyAsync(c->rho_tab, tab.data(), sizeof(float) * tab.size(), cudaMemcpyHostToDevice, st));
   }
   CK(cudaMemsetAsync(c->ready, 0, sizeof(int) * (2 * cdiv(m, 2 * kBM) + 2), st));
   c->ready_base = 0;
@@ -1282,6 +1300,7 @@ int admmq_iterate(admmq_ctx* c, int t0, int count, uint8_t* codes, float* scale,
   p2.ld = d;
   p2.group = c->p.group;
   p2.L = c->L;
+  p2.vs = 1.f;
   auto new_event = [&](cudaEvent_t& e) -> int {
     CK(cudaEventCreate(&e));
     return ADMMQ_OK;
@@ -1335,6 +1354,7 @@ int admmq_iterate(admmq_ctx* c, int t0, int count, uint8_t* codes, float* scale,
                                                                                     c->mE, g, p1, st)));
     if (c->timing) CK(cudaEventRecord(rec.b, st));
     p2.part = c->resid_part + (size_t)t * c->tiles_eig * 8;
+    p2.vs = vscale_at(c->p, t);
     cudaError_t e;
     switch (c->p.grid_mode) {
       case ADMMQ_GRID_MINMAX:
@@ -1493,12 +1513,14 @@ int admmq_get_timing(admmq_ctx* c, double ms[2], int launches[2], int* iters_tim
 int admmq_project(const float* wt, float* V, const float* sig, const float* rsig,
                   const float* hd, int d, int m, int bits, int g, int mode, int split,
                   uint8_t* codes, float* scale, float* zero, void* p_hi, void* p_lo,
-                  const float* row_scale, int* range_flag, double* resid, void* stream) {
+                  const float* row_scale, int* range_flag, double* resid, float dual_scale,
+                  void* stream) {
   if (!wt || !V || !sig || !rsig || !hd || !codes || !scale || !zero || !p_hi || !p_lo || !resid)
     return ADMMQ_ERR_INVALID_ARG;
   if (d <= 0 || m <= 0 || d % 32 != 0 || !(g == 32 || g == 64 || g == 128) || d % g != 0 ||
       bits < 1 || bits > 8 || mode < ADMMQ_GRID_MINMAX || mode > ADMMQ_GRID_MSE ||
-      !(split == ADMMQ_SPLIT_3XTF32 || split == ADMMQ_SPLIT_MIXED || split == ADMMQ_SPLIT_F16))
+      !(split == ADMMQ_SPLIT_3XTF32 || split == ADMMQ_SPLIT_MIXED || split == ADMMQ_SPLIT_F16) ||
+      !(dual_scale > 0.f && dual_scale <= 1e30f))
     return ADMMQ_ERR_INVALID_ARG;
   if (!aligned32(V) || !aligned32(codes) || !aligned32(p_hi) || !aligned32(p_lo) ||
       ((uintptr_t)wt & 15) || ((uintptr_t)sig & 31) || ((uintptr_t)rsig & 31) || ((uintptr_t)hd & 31) ||
@@ -1515,7 +1537,7 @@ int admmq_project(const float* wt, float* V, const float* sig, const float* rsig
 #define PROJECT_ENC(MODE, ENC)                                                               \
   count_launch(), k_project<MODE, ENC, MODE != GRID_MSE><<<grid, block, smem, st>>>(         \
                       wt, V, sig, rsig, hd, m, d, g, L, codes, scale, zero, p_hi, p_lo,      \
-                      row_scale, range_flag, resid);
+                      row_scale, range_flag, resid, dual_scale);
 #define PROJECT_CASE(MODE)       \
   if (enc == ENC_MIX) {          \
     PROJECT_ENC(MODE, ENC_MIX)   \

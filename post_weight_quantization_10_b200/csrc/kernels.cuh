@@ -259,6 +259,7 @@ struct ProjRow {
   float* zero;
   float* wdump;        // optional raw W~ output
   float rs;            // the row's operand scale (fp16 split; 1 otherwise)
+  float vs;            // dual rescaling rho_t / rho_{t+1} (1 without it)
   int* flag;           // range flag of the fp16 split
   bool valid;
 };
@@ -433,7 +434,7 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, LoadV&& loadv, cons
         const float q = clampq(__fadd_rn(q8[k], z), Lf);
         const float D = __fmul_rn(s, __fsub_rn(q, z));
         const float dt = __fmul_rn(D, rr[k]);
-        vn[k] = __fsub_rn(t, dt);
+        vn[k] = __fmul_rn(__fsub_rn(t, dt), r.vs);
         pv[k] = __fsub_rn(dt, vn[k]);
         const int wi = (e + k) >> 2, sh = 8 * ((e + k) & 3);
         if (sh == 0) qw[wi] = 0u;
@@ -594,6 +595,7 @@ struct ProjParams {
   const float* hd;
   float* part;    // [tiles][4][2] for this iteration
   float* wdump;   // optional
+  float vs;       // dual rescaling of this iteration (1 without it)
   int ld;         // d_in
   int group;
   int L;
@@ -633,6 +635,7 @@ struct EpiProject {
       r.wdump = p.wdump ? p.wdump + off : nullptr;
       r.rs = ri;
       r.flag = p.flag;
+      r.vs = p.vs;
       r.valid = valid;
       // W~ = Q T: the accumulator carries the operands' scales (exact powers of two)
       auto loadw = [&](int c, float (&w)[32]) {

@@ -51,10 +51,11 @@ def _oracle(p, X, W, grid, iters=None):
     return H, Wm, res
 
 
-def _solver(A, p, X, W, grid, iters=None, split="auto", scaling=True, schedule="fused"):
+def _solver(A, p, X, W, grid, iters=None, split="auto", scaling=True, schedule="fused",
+            rescale_dual=False):
     prm = A.Params(bits=p.bits, group=p.group, iters=p.iters if iters is None else iters,
                    rho0=p.rho0, gamma=p.gamma, lambda_rel=p.lambda_rel, grid=grid, split=split,
-                   scaling=scaling, schedule=schedule)
+                   scaling=scaling, schedule=schedule, rescale_dual=rescale_dual)
     G = A.build_hessian(X)
     s = A.Solver(X.shape[1], W.shape[0], prm)
     s.prepare(G, W)
@@ -215,6 +216,70 @@ def test_free_running_solve(A, name, grid):
     r = s.resid.cpu().numpy()[: p.iters]
     np.testing.assert_allclose(r[:3, 0], res["r"][:3], rtol=1e-3)
     assert agree >= 0.9 and abs(rel) <= 0.2
+
+
+@pytest.mark.parametrize("name,split", [("tiny", "auto"), ("ragged", "auto"), ("ragged", "f16")])
+def test_rescaled_dual_teacher_forced(A, name, split):
+    """The dual-rescaling variant (V~ *= rho_t / rho_{t+1} after each
+    iteration): along the oracle's trajectory run with rescale_dual, one GPU
+    iteration gives W~ within 1e-4 and the codes within the step bar, and the
+    GPU's new V~ equals the oracle's rescaled one wherever the codes agree."""
+    p, X, W = _layer(name)
+    trace = []
+    H = O.hessian(X.float().cpu().numpy(), p.lambda_rel)
+    Wm = W.float().cpu().numpy().T.astype(np.float64)
+    O.admm_q(H, Wm, p.bits, p.group, p.iters, rho0=p.rho0, gamma=p.gamma, grid="lsq",
+             trace=trace, rescale_dual=True)
+    s = _solver(A, p, X, W, "lsq", split=split, rescale_dual=True)
+    s.init()
+    wt = torch.empty((W.shape[0], X.shape[1]), dtype=torch.float32, device="cuda")
+    s.dump_wtilde(wt)
+    for t in STEPS[name]:
+        e = trace[t]
+        _load_state(s, e)
+        s.iterate(t, 1)
+        torch.cuda.synchronize()
+        ref = e["W_tilde"].T
+        assert np.linalg.norm(wt.cpu().numpy() - ref) / np.linalg.norm(ref) <= 1e-4, t
+        c = s.codes.cpu().numpy()
+        agree = c == e["codes_out"].T
+        assert np.mean(~agree) <= 1e-3, t
+        V = s.buffer("V").cpu().numpy().astype(np.float64)
+        Vr = e["Vt_out"].T
+        err = np.abs(V - Vr)[agree].max()
+        assert err <= 1e-4 * np.abs(ref).max(), (t, err)
+    s.dump_wtilde(None)
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged"])
+def test_rescaled_dual_solve(A, name):
+    """The whole solve with rescale_dual: the fused and the per-GEMM
+    schedules give the same bits, the result is a valid solution close to
+    the oracle's own rescaled solve, and it differs from the default one
+    (gamma > 1 makes the factor differ from 1)."""
+    p, X, W = _layer(name)
+    runs = {}
+    for sched in ("per_gemm", "fused"):
+        s = _solver(A, p, X, W, "lsq", schedule=sched, rescale_dual=True)
+        s.solve()
+        torch.cuda.synchronize()
+        s.check()
+        runs[sched] = (s.codes.cpu().clone(), s.buffer("V").cpu().clone(), float(s.objective.cpu()))
+    assert torch.equal(runs["fused"][0], runs["per_gemm"][0])
+    assert torch.equal(runs["fused"][1], runs["per_gemm"][1])
+    assert runs["fused"][2] == runs["per_gemm"][2]
+    H = O.hessian(X.float().cpu().numpy(), p.lambda_rel)
+    Wm = W.float().cpu().numpy().T.astype(np.float64)
+    res = O.admm_q(H, Wm, p.bits, p.group, p.iters, rho0=p.rho0, gamma=p.gamma, grid="lsq",
+                   rescale_dual=True)
+    codes = runs["fused"][0].numpy()
+    agree = float(np.mean(codes == res["codes"].T))
+    rel = runs["fused"][2] / res["objective"] - 1.0
+    print(f"rescaled dual {name}: codes agree {agree:.5f}, objective rel {rel:+.3e}")
+    assert agree >= 0.9 and abs(rel) <= 0.2
+    plain = _solver(A, p, X, W, "lsq")
+    plain.solve()
+    assert not torch.equal(plain.buffer("V").cpu(), runs["fused"][1])
 
 
 @pytest.mark.parametrize("name", ["tiny", "ragged"])

@@ -651,6 +651,53 @@ def test_admm_beats_rtn_and_gptq_with_lsq_refresh():
 # ------------------------------------------------------------------------ pack
 
 
+def test_dual_rescaling_keeps_the_unscaled_dual():
+    """With rescale_dual the scaled dual is multiplied by rho_t / rho_{t+1}
+    after its update: rho_{t+1} V~_{t+1} = rho_t (V~_t + W~_t - D~_{t+1}), the
+    unscaled dual's ADMM update.  With gamma = 1 it changes nothing; with
+    gamma > 1 it changes the iterates."""
+    rng = np.random.default_rng(11)
+    X = rng.standard_normal((400, 16)) @ rng.standard_normal((16, 16))
+    H = O.hessian(X)
+    W_hat = rng.standard_normal((16, 3)) * 0.05
+    rho0, gamma = 0.1, 1.3
+    trace = []
+    res = O.admm_q(H, W_hat, 3, 8, 12, rho0=rho0, gamma=gamma, grid="minmax", trace=trace,
+                   rescale_dual=True)
+    sigma = res["sigma"][:, None]
+    for t in range(len(trace) - 1):
+        e, nxt = trace[t], trace[t + 1]
+        lhs = nxt["rho"] * e["Vt_out"]
+        rhs = e["rho"] * (e["Vt"] + e["W_tilde"] - nxt["Dt"])
+        np.testing.assert_allclose(lhs, rhs, rtol=1e-12, atol=1e-14 * np.abs(rhs).max())
+        assert nxt["Dt"] == pytest.approx(O.project(e["Y"], 3, 8, "minmax", np.diag(H), e["scale"],
+                                                    e["zero"])[3] / sigma, rel=1e-15)
+    a = O.admm_q(H, W_hat, 3, 8, 12, rho0=rho0, gamma=1.0, grid="minmax", rescale_dual=True)
+    b = O.admm_q(H, W_hat, 3, 8, 12, rho0=rho0, gamma=1.0, grid="minmax")
+    np.testing.assert_array_equal(a["V_tilde"], b["V_tilde"])
+    c = O.admm_q(H, W_hat, 3, 8, 12, rho0=rho0, gamma=gamma, grid="minmax")
+    assert not np.array_equal(res["V_tilde"], c["V_tilde"])
+
+
+def test_epilogue_step_dual_scale():
+    """The float32 statement with a dual scale r: V~' = fl(fl(t - D~) r) and
+    P = fl(D~ - V~'); r = 1 gives the unscaled step bit for bit."""
+    W, V, sig, rsig, hd, s0, z0, c0 = _epilogue_inputs(4, 64, 32, 3, seed=5)
+    base = P.epilogue_step(W, V, sig, rsig, hd, s0, z0, c0, 3, 32, "lsq")
+    one = P.epilogue_step(W, V, sig, rsig, hd, s0, z0, c0, 3, 32, "lsq", dual_scale=1.0)
+    for k in ("codes", "scale", "zero", "V", "P"):
+        np.testing.assert_array_equal(base[k], one[k])
+    r = np.float32(1 / 1.05)
+    out = P.epilogue_step(W, V, sig, rsig, hd, s0, z0, c0, 3, 32, "lsq", dual_scale=r)
+    np.testing.assert_array_equal(out["codes"], base["codes"])
+    f = np.float64
+    np.testing.assert_allclose(out["V"].astype(f), base["V"].astype(f) * f(r), rtol=1e-7, atol=0)
+    # P + V~' = D~ in both (the same D~: same codes and grid)
+    Dt = base["P"].astype(f) + base["V"].astype(f)
+    np.testing.assert_allclose(out["P"].astype(f) + out["V"].astype(f), Dt, rtol=0,
+                               atol=2e-7 * np.abs(Dt).max())
+
+
 def test_pack_hand_examples():
     c4 = np.array([[1, 2, 3, 4, 5, 6, 7, 8]])
     assert O.pack(c4, 4)[0, 0] == 0x87654321
