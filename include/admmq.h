@@ -104,6 +104,10 @@ typedef struct admmq_params {
                        unscaled dual rho V~ carries over when the penalty grows
                        (the pages say nothing on it; a variant for study); 0
                        (default): V~ += W~ - D~ only                             */
+  int fit_on_w;     /* 1: refresh the grid from Sigma W~ and round Sigma (W~ + V~)
+                       onto it (the pages' "current continuous iterate" read as
+                       W~; a variant for study); 0 (default): fit the grid on
+                       the point being projected, Sigma (W~ + V~)               */
 } admmq_params;
 
 typedef struct admmq_ctx admmq_ctx; /* opaque; host memory owned by the library */
@@ -300,7 +304,9 @@ int admmq_get_timing(admmq_ctx* ctx, double ms[2], int launches[2], int* iters_t
  * fp16's range; codes/scale/zero hold the previous D on entry and the new D
  * on exit; resid_dev fp64 [2] receives the two residual sums of squares;
  * dual_scale multiplies the new V~ (rho_t / rho_{t+1} under
- * admmq_params.rescale_dual; 1 otherwise; must be positive and finite).
+ * admmq_params.rescale_dual; 1 otherwise; must be positive and finite);
+ * fit_on_w = 1 refreshes the grid from sigma W~ alone (admmq_params.fit_on_w),
+ * 0 from sigma (W~ + V~).
  * V_dev, codes_dev, P_hi_dev, P_lo_dev, sigma_dev, rsig_dev and hdiag_dev
  * must be 32-byte aligned, wtilde_dev 16-byte aligned, row_scale_dev and
  * range_flag_dev 4-byte aligned (ADMMQ_ERR_INVALID_ARG otherwise). */
@@ -308,7 +314,8 @@ int admmq_project(const float* wtilde_dev, float* V_dev, const float* sigma_dev,
                   const float* rsig_dev, const float* hdiag_dev, int d_in, int d_out, int bits,
                   int group, int grid_mode, int split_mode, uint8_t* codes_dev, float* scale_dev,
                   float* zero_dev, void* P_hi_dev, void* P_lo_dev, const float* row_scale_dev,
-                  int* range_flag_dev, double* resid_dev, float dual_scale, void* stream);
+                  int* range_flag_dev, double* resid_dev, float dual_scale, int fit_on_w,
+                  void* stream);
 
 /* The split precision a context runs its eigenbasis GEMMs in
  * (ADMMQ_SPLIT_3XTF32, ADMMQ_SPLIT_MIXED or ADMMQ_SPLIT_F16; ADMMQ_SPLIT_AUTO

@@ -119,7 +119,7 @@ def rtn(W_hat: np.ndarray, bits: int, group: int):
 
 
 def project(Y: np.ndarray, bits: int, group: int, mode: str, hdiag: np.ndarray,
-            s_prev: np.ndarray, z_prev: np.ndarray):
+            s_prev: np.ndarray, z_prev: np.ndarray, Y_fit=None):
     """D-update: project Y = Sigma (W~ + V~) onto a per-group grid ([ADMM-Q] section 2).
 
     The decision is taken in float32 (the kernels' precision).  `mode` selects
@@ -132,21 +132,24 @@ def project(Y: np.ndarray, bits: int, group: int, mode: str, hdiag: np.ndarray,
                 heuristic by MSE grid search, [ADMM-Q] Methodology section 3,
                 modularity);
       "frozen": the previous grid is kept (GPTQ-style fixed grid).
+    `Y_fit` (optional): the grid is refreshed from Y_fit instead of Y, and Y
+    is rounded onto it.
     Returns (codes, scale, zero, D) like rtn().
     """
     d, m = Y.shape
     L = (1 << bits) - 1
     yg = _groups(np.asarray(Y, dtype=np.float32), group)
+    fg = yg if Y_fit is None else _groups(np.asarray(Y_fit, dtype=np.float32), group)
     sp = np.ascontiguousarray(np.asarray(s_prev, np.float32).T).reshape(-1)
     zp = np.ascontiguousarray(np.asarray(z_prev, np.float32).T).reshape(-1)
     if mode == "minmax":
-        s, z = p32.fit_minmax(yg, L)
+        s, z = p32.fit_minmax(fg, L)
     elif mode == "lsq":
         wg = np.broadcast_to(np.asarray(hdiag, np.float32).reshape(d // group, group)[None],
                              (m, d // group, group)).reshape(-1, group)
-        s, z = p32.fit_lsq(yg, wg, sp, zp, L)
+        s, z = p32.fit_lsq(fg, wg, sp, zp, L)
     elif mode == "mse":
-        s, z = p32.fit_mse(yg, L)
+        s, z = p32.fit_mse(fg, L)
     elif mode == "frozen":
         s, z = sp, zp
     else:
@@ -176,7 +179,7 @@ def w_update(Q: np.ndarray, lam: np.ndarray, B: np.ndarray, rho: float,
 def admm_q(H: np.ndarray, W_hat: np.ndarray, bits: int, group: int, iters: int,
            rho0: float = 0.1, gamma: float = 1.05, grid: str = "minmax",
            scaling: bool = True, eig=None, grid0=None, trace=None,
-           rescale_dual: bool = False) -> dict:
+           rescale_dual: bool = False, fit_on_w: bool = False) -> dict:
     """The ADMM-Q layer solve, step by step in the pages' order.
 
     1. Sigma = Diag(H)^(-1/2); H~ = Sigma H Sigma; W^~ = Sigma^-1 W_hat.
@@ -193,6 +196,9 @@ def admm_q(H: np.ndarray, W_hat: np.ndarray, bits: int, group: int, iters: int,
     that the unscaled dual rho V~ carries over unchanged when the penalty
     grows (the pages say nothing on this; without the flag V~ is literally
     V~ + W~ - D~, the reading the default follows).
+    `fit_on_w=True` refreshes the grid from Sigma W~ instead of the point
+    being projected, Sigma (W~ + V~) (the pages' "current continuous
+    iterate" read as W~; the default reads it as the projected point).
     `eig` optionally passes a precomputed (Lambda, Q) of H~; `grid0` an
     initial (scale, zero) pair ((d_in/group) x d_out each) replacing the RTN
     grid of W_hat (the start D is then W_hat rounded on that grid).
@@ -225,7 +231,8 @@ def admm_q(H: np.ndarray, W_hat: np.ndarray, bits: int, group: int, iters: int,
                          scale=s.copy(), zero=z.copy())
         Wt = w_update(Q, lam, B, rho, Dt, Vt)
         Y = sigma[:, None] * (Wt + Vt)
-        codes_new, s, z, D = project(Y, bits, group, grid, hdiag, s, z)
+        Y_fit = sigma[:, None] * Wt if fit_on_w else None
+        codes_new, s, z, D = project(Y, bits, group, grid, hdiag, s, z, Y_fit=Y_fit)
         Dt_new = D / sigma[:, None]
         Vt = Vt + Wt - Dt_new
         if rescale_dual:

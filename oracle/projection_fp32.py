@@ -260,7 +260,7 @@ def init_step(W_rows: np.ndarray, rsig: np.ndarray, bits: int, group: int, split
 def epilogue_step(W_acc: np.ndarray, V: np.ndarray, sigma: np.ndarray, rsig: np.ndarray,
                   hdiag: np.ndarray, s_prev: np.ndarray, z_prev: np.ndarray,
                   codes_prev: np.ndarray, bits: int, group: int, mode: str,
-                  split: str = "mixed", row_scale=None, dual_scale=None):
+                  split: str = "mixed", row_scale=None, dual_scale=None, fit_on_w=False):
     """One fused projection + dual update in memory layout ([d_out][d_in]).
 
     Per element (i = input channel):
@@ -270,6 +270,8 @@ def epilogue_step(W_acc: np.ndarray, V: np.ndarray, sigma: np.ndarray, rsig: np.
       V~' = t - D~          P  = D~ - V~'   (in the operand encoding of `split`)
     With `dual_scale` r (the dual rescaling rho_t / rho_{t+1}, a float32):
       V~' = (t - D~) r, rounded after the subtraction and after the product.
+    With `fit_on_w` the grid is fitted on y_w = sigma_i W~ (the dual left
+    out); y is still the point rounded onto it.
     Residual sums (float64 here; the kernels sum in float32, compared with a
     tolerance): r2 = sum (W~ - D~)^2 and s2 = sum (D~ - D~_prev)^2 where
     D~_prev = s_prev (q_prev - z_prev) * rsig.
@@ -280,16 +282,17 @@ def epilogue_step(W_acc: np.ndarray, V: np.ndarray, sigma: np.ndarray, rsig: np.
     t = _f(W_acc + V)
     y = _f(_f(sigma)[None, :] * t)
     yg = _rows_to_groups(y, group)
+    fg = _rows_to_groups(_f(_f(sigma)[None, :] * W_acc), group) if fit_on_w else yg
     sp = _f(s_prev).reshape(-1)
     zp = _f(z_prev).reshape(-1)
     if mode == "minmax":
-        s, z = fit_minmax(yg, L)
+        s, z = fit_minmax(fg, L)
     elif mode == "lsq":
         wg = np.broadcast_to(_f(hdiag).reshape(d // group, group)[None],
                              (m, d // group, group)).reshape(-1, group)
-        s, z = fit_lsq(yg, wg, sp, zp, L)
+        s, z = fit_lsq(fg, wg, sp, zp, L)
     elif mode == "mse":
-        s, z = fit_mse(yg, L)
+        s, z = fit_mse(fg, L)
     elif mode == "frozen":
         s, z = sp, zp
     else:

@@ -37,7 +37,8 @@ class _Params(ctypes.Structure):
                 ("rho0", ctypes.c_float), ("gamma", ctypes.c_float),
                 ("lambda_rel", ctypes.c_float), ("grid_mode", ctypes.c_int),
                 ("split_mode", ctypes.c_int), ("no_scaling", ctypes.c_int),
-                ("schedule", ctypes.c_int), ("rescale_dual", ctypes.c_int)]
+                ("schedule", ctypes.c_int), ("rescale_dual", ctypes.c_int),
+                ("fit_on_w", ctypes.c_int)]
 
 
 @dataclass
@@ -53,11 +54,12 @@ class Params:
     scaling: bool = True  # False: Sigma = I (the unscaled ablation)
     schedule: str = "fused"  # fused: one launch per iterate call | per_gemm: two per iteration
     rescale_dual: bool = False  # V~ *= rho_t / rho_{t+1} after each iteration (a study variant)
+    fit_on_w: bool = False  # refresh the grid from Sigma W~ instead of Sigma (W~ + V~) (a study variant)
 
     def c(self) -> _Params:
         return _Params(self.bits, self.group, self.iters, self.rho0, self.gamma, self.lambda_rel,
                        GRID_MODES[self.grid], SPLIT_MODES[self.split], int(not self.scaling),
-                       SCHEDULES[self.schedule], int(self.rescale_dual))
+                       SCHEDULES[self.schedule], int(self.rescale_dual), int(self.fit_on_w))
 
 
 _lib = None
@@ -112,7 +114,7 @@ def lib():
         "admmq_get_timing": (_i, [_vp, ctypes.POINTER(ctypes.c_double),
                                   ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
         "admmq_project": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp,
-                               _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _vp]),
+                               _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _i, _vp]),
         "admmq_split_mode": (_i, [_vp]),
         "admmq_check": (_i, [_vp, _vp]),
         "admmq_debug_skew_ready": (_i, [_vp, _i]),
@@ -328,12 +330,13 @@ def pack(codes: torch.Tensor, bits: int, out: torch.Tensor | None = None, stream
 
 def project(wtilde, V, sigma, rsig, hdiag, bits, group, grid, codes, scale, zero, P_hi, P_lo,
             resid=None, split="mixed", row_scale=None, range_flag=None, dual_scale=1.0,
-            stream=None):
+            fit_on_w=False, stream=None):
     """Stand-alone projection; P planes in the encoding of `split`: "3xtf32"
     fp32 [m][d] x2, "mixed" fp32 [m][d] + int16 (bf16 bit patterns) [m][2d],
     "f16" int16 (fp16 bit patterns) [m][d] x2 with the rows' scales
     `row_scale` (fp32 [m]; None = 1) and an optional int32 range flag;
-    `dual_scale` multiplies the new V~ (the dual rescaling)."""
+    `dual_scale` multiplies the new V~ (the dual rescaling); `fit_on_w`
+    refreshes the grid from sigma W~ alone."""
     m, d = wtilde.shape
     if resid is None:
         resid = torch.zeros(2, dtype=torch.float64, device=wtilde.device)
@@ -341,7 +344,7 @@ def project(wtilde, V, sigma, rsig, hdiag, bits, group, grid, codes, scale, zero
                                bits, group, GRID_MODES[grid], SPLIT_MODES[split], _ptr(codes),
                                _ptr(scale), _ptr(zero), _ptr(P_hi), _ptr(P_lo), _ptr(row_scale),
                                _ptr(range_flag), _ptr(resid), ctypes.c_float(dual_scale),
-                               _stream(stream)),
+                               int(fit_on_w), _stream(stream)),
            "admmq_project")
     return resid
 

@@ -451,7 +451,7 @@ __global__ void __launch_bounds__(STAGED ? kProjRows : 128) k_project(
     const float* __restrict__ wt, float* V, const float* __restrict__ sig,
     const float* __restrict__ rsig, const float* __restrict__ hd, int m, int d, int g, int L,
     uint8_t* codes, float* scale, float* zero, void* p_hi, void* p_lo,
-    const float* __restrict__ row_in, int* flag, double* resid, float vs) {
+    const float* __restrict__ row_in, int* flag, double* resid, float vs, int fit_w) {
   extern __shared__ float4 proj_smem[];
   float* stage = reinterpret_cast<float*>(proj_smem);
   const int lane = threadIdx.x & 31;
@@ -510,6 +510,7 @@ __global__ void __launch_bounds__(STAGED ? kProjRows : 128) k_project(
   r.wdump = nullptr;
   r.rs = (valid && row_in) ? row_in[row] : 1.f;
   r.vs = vs;
+  r.fit_w = fit_w;
   r.flag = flag;
   r.valid = valid;
   const float* mine = stage + lane * slot;
@@ -898,6 +899,7 @@ int check_params(int d, int m, const admmq_params* p) {
     return ADMMQ_ERR_INVALID_ARG;
   if (p->no_scaling != 0 && p->no_scaling != 1) return ADMMQ_ERR_INVALID_ARG;
   if (p->rescale_dual != 0 && p->rescale_dual != 1) return ADMMQ_ERR_INVALID_ARG;
+  if (p->fit_on_w != 0 && p->fit_on_w != 1) return ADMMQ_ERR_INVALID_ARG;
   if (p->schedule != ADMMQ_SCHEDULE_FUSED && p->schedule != ADMMQ_SCHEDULE_PER_GEMM)
     return ADMMQ_ERR_INVALID_ARG;
   return ADMMQ_OK;
@@ -1037,7 +1039,7 @@ const char* admmq_status_string(int s) {
   }
 }
 
-int admmq_version(void) { return 101; }
+int admmq_version(void) { return 102; }
 
 int64_t admmq_launch_count(void) { return (int64_t)__atomic_load_n(&g_launches, __ATOMIC_RELAXED); }
 
@@ -1301,6 +1303,7 @@ int admmq_iterate(admmq_ctx* c, int t0, int count, uint8_t* codes, float* scale,
   p2.group = c->p.group;
   p2.L = c->L;
   p2.vs = 1.f;
+  p2.fit_w = c->p.fit_on_w;
   auto new_event = [&](cudaEvent_t& e) -> int {
     CK(cudaEventCreate(&e));
     return ADMMQ_OK;
@@ -1514,13 +1517,13 @@ int admmq_project(const float* wt, float* V, const float* sig, const float* rsig
                   const float* hd, int d, int m, int bits, int g, int mode, int split,
                   uint8_t* codes, float* scale, float* zero, void* p_hi, void* p_lo,
                   const float* row_scale, int* range_flag, double* resid, float dual_scale,
-                  void* stream) {
+                  int fit_on_w, void* stream) {
   if (!wt || !V || !sig || !rsig || !hd || !codes || !scale || !zero || !p_hi || !p_lo || !resid)
     return ADMMQ_ERR_INVALID_ARG;
   if (d <= 0 || m <= 0 || d % 32 != 0 || !(g == 32 || g == 64 || g == 128) || d % g != 0 ||
       bits < 1 || bits > 8 || mode < ADMMQ_GRID_MINMAX || mode > ADMMQ_GRID_MSE ||
       !(split == ADMMQ_SPLIT_3XTF32 || split == ADMMQ_SPLIT_MIXED || split == ADMMQ_SPLIT_F16) ||
-      !(dual_scale > 0.f && dual_scale <= 1e30f))
+      !(dual_scale > 0.f && dual_scale <= 1e30f) || (fit_on_w != 0 && fit_on_w != 1))
     return ADMMQ_ERR_INVALID_ARG;
   if (!aligned32(V) || !aligned32(codes) || !aligned32(p_hi) || !aligned32(p_lo) ||
       ((uintptr_t)wt & 15) || ((uintptr_t)sig & 31) || ((uintptr_t)rsig & 31) || ((uintptr_t)hd & 31) ||
@@ -1537,7 +1540,7 @@ int admmq_project(const float* wt, float* V, const float* sig, const float* rsig
 #define PROJECT_ENC(MODE, ENC)                                                               \
   count_launch(), k_project<MODE, ENC, MODE != GRID_MSE><<<grid, block, smem, st>>>(         \
                       wt, V, sig, rsig, hd, m, d, g, L, codes, scale, zero, p_hi, p_lo,      \
-                      row_scale, range_flag, resid, dual_scale);
+                      row_scale, range_flag, resid, dual_scale, fit_on_w);
 #define PROJECT_CASE(MODE)       \
   if (enc == ENC_MIX) {          \
     PROJECT_ENC(MODE, ENC_MIX)   \

@@ -260,6 +260,7 @@ struct ProjRow {
   float* wdump;        // optional raw W~ output
   float rs;            // the row's operand scale (fp16 split; 1 otherwise)
   float vs;            // dual rescaling rho_t / rho_{t+1} (1 without it)
+  int fit_w;           // 1: refresh the grid from sigma W~ (V~ left out of the fit)
   int* flag;           // range flag of the fp16 split
   bool valid;
 };
@@ -294,7 +295,7 @@ __device__ __forceinline__ void mse_clip_grid(LoadW& loadw, LoadV& loadv, const 
 #pragma unroll
     for (int e = 0; e < 32; e += 8) {
       float vv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      loadv(c + e, vv);
+      if (!r.fit_w) loadv(c + e, vv);  // the grid fitted on sigma W~ alone (fit_w)
       float ss[8];
       load8_col<COLS_SMEM>(r.sig + c + e, ss);
 #pragma unroll
@@ -360,7 +361,7 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, LoadV&& loadv, cons
 #pragma unroll
       for (int e = 0; e < 32; e += 8) {
         float vv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        loadv(c + e, vv);
+        if (!r.fit_w) loadv(c + e, vv);  // the grid fitted on sigma W~ alone (fit_w)
         float ss[8], hh[8], y8[8], q8[8];
         load8_col<COLS_SMEM>(r.sig + c + e, ss);
         if (MODE == GRID_LSQ) load8_col<COLS_SMEM>(r.hd + c + e, hh);
@@ -596,6 +597,7 @@ struct ProjParams {
   float* part;    // [tiles][4][2] for this iteration
   float* wdump;   // optional
   float vs;       // dual rescaling of this iteration (1 without it)
+  int fit_w;      // grid refreshed from sigma W~ instead of sigma (W~ + V~)
   int ld;         // d_in
   int group;
   int L;
@@ -636,6 +638,7 @@ struct EpiProject {
       r.rs = ri;
       r.flag = p.flag;
       r.vs = p.vs;
+      r.fit_w = p.fit_w;
       r.valid = valid;
       // W~ = Q T: the accumulator carries the operands' scales (exact powers of two)
       auto loadw = [&](int c, float (&w)[32]) {

@@ -85,15 +85,18 @@ def _proj_inputs(m, d, g, bits, seed):
 @pytest.mark.parametrize("grid", ["minmax", "lsq", "mse", "frozen"])
 @pytest.mark.parametrize("bits,g,m,d", [(3, 128, 200, 384), (2, 64, 33, 128), (4, 32, 130, 96),
                                         (3, 64, 32, 64)])
-@pytest.mark.parametrize("dual", [None, np.float32(1 / 1.05)])  # the dual rescaling factor
-def test_projection_kernel_bitexact(A, grid, bits, g, m, d, split, dual):
+# the study variants: dual rescaling factor, grid fitted on sigma W~ alone
+@pytest.mark.parametrize("variant", ["plain", "dual", "fit_w"])
+def test_projection_kernel_bitexact(A, grid, bits, g, m, d, split, variant):
+    dual = np.float32(1 / 1.05) if variant == "dual" else None
+    fit_w = variant == "fit_w"
     x = _proj_inputs(m, d, g, bits, seed=bits * 100 + g + m)
     rng = np.random.default_rng(m + d)
     # the fp16 split's per-row powers of two (1 for the other encodings)
     rs = (np.ldexp(np.float32(1), rng.integers(-4, 5, m)).astype(np.float32) if split == "f16"
           else None)
     ref = P.epilogue_step(x["W"], x["V"], x["sig"], x["rsig"], x["hd"], x["s0"], x["z0"], x["c0"],
-                          bits, g, grid, split, row_scale=rs, dual_scale=dual)
+                          bits, g, grid, split, row_scale=rs, dual_scale=dual, fit_on_w=fit_w)
     cu = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
     V = cu(x["V"])
     codes, scale, zero = cu(x["c0"]), cu(x["s0"]), cu(x["z0"])
@@ -108,7 +111,7 @@ def test_projection_kernel_bitexact(A, grid, bits, g, m, d, split, dual):
     resid = A.project(cu(x["W"]), V, cu(x["sig"]), cu(x["rsig"]), cu(x["hd"]), bits, g, grid,
                       codes, scale, zero, phi, plo, split=split,
                       row_scale=cu(rs) if rs is not None else None, range_flag=flag,
-                      dual_scale=1.0 if dual is None else float(dual))
+                      dual_scale=1.0 if dual is None else float(dual), fit_on_w=fit_w)
     torch.cuda.synchronize()
     np.testing.assert_array_equal(codes.cpu().numpy(), ref["codes"])
     np.testing.assert_array_equal(scale.cpu().numpy().view(np.uint32), ref["scale"].view(np.uint32))

@@ -52,10 +52,11 @@ def _oracle(p, X, W, grid, iters=None):
 
 
 def _solver(A, p, X, W, grid, iters=None, split="auto", scaling=True, schedule="fused",
-            rescale_dual=False):
+            rescale_dual=False, fit_on_w=False):
     prm = A.Params(bits=p.bits, group=p.group, iters=p.iters if iters is None else iters,
                    rho0=p.rho0, gamma=p.gamma, lambda_rel=p.lambda_rel, grid=grid, split=split,
-                   scaling=scaling, schedule=schedule, rescale_dual=rescale_dual)
+                   scaling=scaling, schedule=schedule, rescale_dual=rescale_dual,
+                   fit_on_w=fit_on_w)
     G = A.build_hessian(X)
     s = A.Solver(X.shape[1], W.shape[0], prm)
     s.prepare(G, W)
@@ -280,6 +281,42 @@ def test_rescaled_dual_solve(A, name):
     plain = _solver(A, p, X, W, "lsq")
     plain.solve()
     assert not torch.equal(plain.buffer("V").cpu(), runs["fused"][1])
+
+
+@pytest.mark.parametrize("name,grid,split", [("tiny", "lsq", "auto"), ("ragged", "lsq", "f16"),
+                                             ("ragged", "mse", "auto"), ("tiny", "minmax", "auto")])
+def test_grid_fitted_on_w_teacher_forced(A, name, grid, split):
+    """The fit-on-W~ variant: along the oracle's trajectory run with
+    fit_on_w, one GPU iteration gives W~ within 1e-4 and the codes within the
+    step bar; the fused and the per-GEMM schedules then give the same bits
+    for the whole solve."""
+    p, X, W = _layer(name)
+    trace = []
+    H = O.hessian(X.float().cpu().numpy(), p.lambda_rel)
+    Wm = W.float().cpu().numpy().T.astype(np.float64)
+    O.admm_q(H, Wm, p.bits, p.group, p.iters, rho0=p.rho0, gamma=p.gamma, grid=grid,
+             trace=trace, fit_on_w=True)
+    s = _solver(A, p, X, W, grid, split=split, fit_on_w=True)
+    s.init()
+    wt = torch.empty((W.shape[0], X.shape[1]), dtype=torch.float32, device="cuda")
+    s.dump_wtilde(wt)
+    for t in STEPS[name]:
+        e = trace[t]
+        _load_state(s, e)
+        s.iterate(t, 1)
+        torch.cuda.synchronize()
+        ref = e["W_tilde"].T
+        assert np.linalg.norm(wt.cpu().numpy() - ref) / np.linalg.norm(ref) <= 1e-4, t
+        assert np.mean(s.codes.cpu().numpy() != e["codes_out"].T) <= 1e-3, t
+    s.dump_wtilde(None)
+    runs = []
+    for sched in ("per_gemm", "fused"):
+        s = _solver(A, p, X, W, grid, split=split, schedule=sched, fit_on_w=True)
+        s.solve()
+        torch.cuda.synchronize()
+        s.check()
+        runs.append((s.codes.cpu().clone(), s.buffer("V").cpu().clone()))
+    assert torch.equal(runs[0][0], runs[1][0]) and torch.equal(runs[0][1], runs[1][1])
 
 
 @pytest.mark.parametrize("name", ["tiny", "ragged"])

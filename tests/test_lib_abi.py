@@ -53,6 +53,9 @@ def test_argument_checks_without_gpu(lib):
     bad = admmq.Params(bits=3, group=128).c()
     bad.rescale_dual = 2
     assert lib.admmq_workspace_bytes(256, 8, ctypes.byref(bad)) == 0
+    bad = admmq.Params(bits=3, group=128).c()
+    bad.fit_on_w = -1
+    assert lib.admmq_workspace_bytes(256, 8, ctypes.byref(bad)) == 0
     assert lib.admmq_gram_workspace_bytes(100, 30) == 0
     assert lib.admmq_pack(None, 64, 4, 3, None, None) == -1
     assert lib.admmq_pack(ctypes.c_void_p(16), 48, 4, 3, ctypes.c_void_p(16), None) == -1
@@ -70,10 +73,10 @@ def test_alignment_checks_without_gpu(lib):
     device (the pointers below are never dereferenced)."""
     ok = [ctypes.c_void_p(0x10000 * (i + 1)) for i in range(12)]
     # wt V sig rsig hd | d m bits g mode split | codes scale zero p_hi p_lo | row_scale flag
-    # | resid dual_scale stream
-    def call(ptrs, split=2, mode=0, row_scale=None, flag=None, dual_scale=1.0):
+    # | resid dual_scale fit_on_w stream
+    def call(ptrs, split=2, mode=0, row_scale=None, flag=None, dual_scale=1.0, fit_on_w=0):
         return lib.admmq_project(*ptrs[:5], 256, 8, 3, 128, mode, split, *ptrs[5:10], row_scale,
-                                 flag, ptrs[10], ctypes.c_float(dual_scale), None)
+                                 flag, ptrs[10], ctypes.c_float(dual_scale), fit_on_w, None)
     for k in (1, 5, 8, 9):  # V, codes, P_hi, P_lo off by 16 bytes
         bad = list(ok)
         bad[k] = ctypes.c_void_p(ok[k].value + 16)
@@ -89,6 +92,7 @@ def test_alignment_checks_without_gpu(lib):
         assert call(list(ok), mode=mode) == -1, mode
     for r in (0.0, -1.0, float("nan"), float("inf")):  # the dual factor is positive and finite
         assert call(list(ok), dual_scale=r) == -1, r
+    assert call(list(ok), fit_on_w=2) == -1
     assert lib.admmq_split_mode(None) == -1
     assert lib.admmq_debug_dump_wtilde(None, None) == -1
 

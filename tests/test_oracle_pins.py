@@ -698,6 +698,38 @@ def test_epilogue_step_dual_scale():
                                atol=2e-7 * np.abs(Dt).max())
 
 
+@pytest.mark.parametrize("mode", ["minmax", "lsq", "mse"])
+def test_grid_fitted_on_w(mode):
+    """fit_on_w refreshes the grid from sigma W~ and rounds sigma (W~ + V~)
+    onto it: the memory-layout statement equals the float64 route's D-update
+    given the fit target separately; with V~ = 0 (the first iteration) it is
+    the default step; later iterates differ from the default solve's."""
+    W, V, sig, rsig, hd, s0, z0, c0 = _epilogue_inputs(5, 96, 32, 3, seed=9)
+    out = P.epilogue_step(W, V, sig, rsig, hd, s0, z0, c0, 3, 32, mode, fit_on_w=True)
+    y = (sig[None, :] * (W + V).astype(np.float32)).astype(np.float32)
+    yw = (sig[None, :] * W).astype(np.float32)
+    codes, sc, ze, _ = O.project(y.T, 3, 32, mode, hd, s0.T, z0.T, Y_fit=yw.T)
+    np.testing.assert_array_equal(out["codes"], codes.T)
+    np.testing.assert_array_equal(out["scale"], sc.T)
+    np.testing.assert_array_equal(out["zero"], ze.T)
+    default = P.epilogue_step(W, V, sig, rsig, hd, s0, z0, c0, 3, 32, mode)
+    assert not np.array_equal(out["scale"], default["scale"])
+    Z = np.zeros_like(V)
+    a = P.epilogue_step(W, Z, sig, rsig, hd, s0, z0, c0, 3, 32, mode, fit_on_w=True)
+    b = P.epilogue_step(W, Z, sig, rsig, hd, s0, z0, c0, 3, 32, mode)
+    for k in ("codes", "scale", "zero", "V", "P"):
+        np.testing.assert_array_equal(a[k], b[k])
+    rng = np.random.default_rng(12)
+    X = rng.standard_normal((300, 16)) @ rng.standard_normal((16, 16))
+    H = O.hessian(X)
+    W_hat = rng.standard_normal((16, 3)) * 0.05
+    one = O.admm_q(H, W_hat, 3, 8, 1, grid=mode, fit_on_w=True)
+    ref = O.admm_q(H, W_hat, 3, 8, 1, grid=mode)
+    np.testing.assert_array_equal(one["codes"], ref["codes"])
+    many = O.admm_q(H, W_hat, 3, 8, 30, grid=mode, fit_on_w=True)
+    assert not np.array_equal(many["V_tilde"], O.admm_q(H, W_hat, 3, 8, 30, grid=mode)["V_tilde"])
+
+
 def test_pack_hand_examples():
     c4 = np.array([[1, 2, 3, 4, 5, 6, 7, 8]])
     assert O.pack(c4, 4)[0, 0] == 0x87654321
