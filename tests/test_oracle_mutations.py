@@ -68,6 +68,9 @@ EPI = tuple((pins.test_epilogue_step_follows_the_d_and_dual_updates, (mode, 3, 3
             for mode in ("minmax", "lsq", "frozen"))
 INIT = (pins.test_init_step_is_rtn_in_memory_layout, (3, 32, 6, 96))
 PACK = (pins.test_pack_hand_examples, ())
+RESCALE = (pins.test_dual_rescaling_keeps_the_unscaled_dual, ())
+RESCALE_F32 = (pins.test_epilogue_step_dual_scale, ())
+FIT_W = tuple((pins.test_grid_fitted_on_w, (mode,)) for mode in ("minmax", "lsq", "mse"))
 PACK_BIG = (pins.test_pack_matches_big_integer_route, (3,))
 
 # name: (module, function, old text, new text, pins that should notice)
@@ -155,6 +158,14 @@ MISTAKES = {
                                        "y = _f(_f(sigma)[None, :] * W_acc)", list(EPI)),
     "epilogue_residual_against_v": (P, "epilogue_step", "np.sum((W_acc.astype(np.float64) - Dt) ** 2)",
                                     "np.sum((V.astype(np.float64) - Dt) ** 2)", list(EPI)),
+    "rescale_factor_inverted": (O, "admm_q", "Vt = Vt * (rho / (rho0 * gamma ** (t + 1)))",
+                                "Vt = Vt * ((rho0 * gamma ** (t + 1)) / rho)", [RESCALE]),
+    "epilogue_rescales_p_not_v": (P, "epilogue_step", "V_new = _f(V_new * f32(dual_scale))",
+                                  "V_new = V_new", [RESCALE_F32]),
+    "fit_target_ignored": (O, "project", "fg = yg if Y_fit is None else", "fg = yg if True else",
+                           list(FIT_W)),
+    "epilogue_fits_with_dual": (P, "epilogue_step", "_f(_f(sigma)[None, :] * W_acc), group) if fit_on_w",
+                                "_f(_f(sigma)[None, :] * t), group) if fit_on_w", list(FIT_W)),
     "init_forgets_scaling": (P, "init_step", "Dt = _f(D * _f(rsig)[None, :])", "Dt = _f(D)", [INIT]),
     "rows_grouped_by_column": (P, "_rows_to_groups", "A.reshape(m * (d // g), g)",
                                "np.ascontiguousarray(A.T).reshape(m * (d // g), g)", list(EPI) + [INIT]),
