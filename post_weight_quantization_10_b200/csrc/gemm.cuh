@@ -1,7 +1,7 @@
 // gemm.cuh -- persistent tcgen05 GEMM engine for sm_100a.
 //
 // D[M x N] = A[M x K] * B[K x N] with operands staged in shared memory by TMA
-// (128-byte swizzle, no multicast) and fp32 accumulation.  Operands are bf16
+// (128-byte swizzle, every CTA loading its own tiles) and fp32 accumulation.  Operands are bf16
 // (kind::f16) or tf32 held in fp32 words (kind::tf32); a shared-memory row is
 // always 128 bytes (64 bf16 or 32 fp32 along K) and one MMA consumes 32 bytes
 // of K.  Split-precision products for fp32-accurate GEMMs (NPL = 2 planes):
