@@ -158,7 +158,8 @@ class ClockSampler:
 class LayerRun:
     """Device-resident state of one layer solve through the C ABI binding."""
 
-    def __init__(self, A, p, grid, seed, device, split="auto", scaling=True, schedule="fused"):
+    def __init__(self, A, p, grid, seed, device, split="auto", scaling=True, schedule="fused",
+                 rescale_dual=False, fit_on_w=False):
         self.A, self.p = A, p
         self.X = workloads.make_activations(p, seed=seed, device=device)
         self.W = workloads.make_weights(p, seed=seed, device=device, dtype=torch.bfloat16)
@@ -167,7 +168,7 @@ class LayerRun:
                                    device=device)
         prm = A.Params(bits=p.bits, group=p.group, iters=p.iters, rho0=p.rho0, gamma=p.gamma,
                        lambda_rel=p.lambda_rel, grid=grid, split=split, scaling=scaling,
-                       schedule=schedule)
+                       schedule=schedule, rescale_dual=rescale_dual, fit_on_w=fit_on_w)
         self.s = A.Solver(p.d_in, p.d_out, prm, device=device)
         self.packed = torch.empty((p.d_out, p.d_in * p.bits // 32), dtype=torch.int32,
                                   device=device)
@@ -399,7 +400,8 @@ def run_ours(args, rank, world, device):
     if args.tokens:
         p = workloads.scaled(p, args.tokens, p.d_in, p.d_out)
     run = LayerRun(A, p, args.grid, seed=rank, device=device, split=args.split,
-                   scaling=not args.no_scaling, schedule=args.schedule)
+                   scaling=not args.no_scaling, schedule=args.schedule,
+                   rescale_dual=args.rescale_dual, fit_on_w=args.fit_on_w)
     clocks = ClockSampler(torch.cuda.current_device())
     clocks.start()
     eigh_s = run.setup_eigh()
@@ -490,8 +492,10 @@ def run_ours(args, rank, world, device):
         "vs_baseline": None,
         "dtype": DTYPES[split],
         "data": "synthetic (seeded Qwen3-8B-shaped activations and weights; no dataset)",
-        "config": {"workload": workload_desc(p, args.grid) + (" Sigma=I (unscaled ablation)"
-                                                              if args.no_scaling else ""),
+        "config": {"workload": workload_desc(p, args.grid)
+                   + (" Sigma=I (unscaled ablation)" if args.no_scaling else "")
+                   + (" dual rescaled by rho_t/rho_t+1" if args.rescale_dual else "")
+                   + (" grid fitted on W~" if args.fit_on_w else ""),
                    "parallelism": f"independent layers x{world}",
                    "l2": "inputs larger than L2 (X is %.1f GiB)" % (n * d * 2 / 2**30),
                    "eigh": "one-time setup outside the step (eigh_s)",
@@ -745,6 +749,10 @@ def main():
     ap.add_argument("--bits", type=int, default=0, help="decoder workload: W2/W3/W4 (default 3)")
     ap.add_argument("--no-scaling", action="store_true",
                     help="Sigma = I: the unscaled ablation (objective comparison)")
+    ap.add_argument("--rescale-dual", action="store_true",
+                    help="variant: V~ *= rho_t / rho_{t+1} after each iteration")
+    ap.add_argument("--fit-on-w", action="store_true",
+                    help="variant: refresh the grid from Sigma W~ instead of Sigma (W~ + V~)")
     ap.add_argument("--shard", action="store_true",
                     help="split ONE layer over the ranks (tokens and output rows; H all-reduced)")
     ap.add_argument("--grid", default="lsq", choices=["lsq", "minmax", "mse", "frozen"])
