@@ -131,7 +131,11 @@ int64_t admmq_launch_count(void);
  *              (so X may be streamed in chunks of tokens).
  *   ws_dev     scratch of at least admmq_gram_workspace_bytes(n, d_in) bytes.
  * bf16 products are exact in fp32; sums are fp32 (tensor cores), combined in a
- * fixed order, so the result is deterministic for a given device and shape. */
+ * fixed order, so the result is deterministic for a given device and shape.
+ * Failure: the Gram kernel's pipeline waits are bounded; one that gives up
+ * sets the int32 status word at the start of ws_dev (non-zero) and the Gram
+ * writes NaN on the diagonal of H, so admmq_prepare() on that H returns
+ * ADMMQ_ERR_NONFINITE. */
 size_t admmq_gram_workspace_bytes(int64_t n, int d_in);
 int admmq_build_hessian(const void* X_dev, int64_t n, int d_in, float* H_dev, int accumulate,
                         void* ws_dev, size_t ws_bytes, void* stream);
@@ -140,9 +144,9 @@ int admmq_build_hessian(const void* X_dev, int64_t n, int d_in, float* H_dev, in
  * this is an interface for callers, not a step of the method).
  * Some callers cannot allocate device memory at the moment they need the
  * Hessian: a serving or training framework that has already reserved all
- * device memory for its own pool, or code that must not call cudaMalloc
- * (it can synchronise the device and is not allowed while a stream is being
- * captured).  This entry point takes no workspace: its scratch (the k-split
+ * device memory for its own pool, or code on a latency-bound path that must
+ * not call cudaMalloc (which can synchronise the whole device).  This entry
+ * point takes no workspace: its scratch (the k-split
  * partial sums and a status word) lives in one file-scope device array of
  * ADMMQ_STATIC_SCRATCH_BYTES, which every GPU that loads the library holds
  * until the process exits.  It computes the same X^T X as
@@ -153,7 +157,16 @@ int admmq_build_hessian(const void* X_dev, int64_t n, int d_in, float* H_dev, in
  *   is launched.
  *   The first call on a device looks the array's device address up
  *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.  Nothing is allocated, here or later.
+ *   before any stream capture.  The address belongs to the device's current
+ *   CUDA context: after cudaDeviceReset, or any other teardown and re-creation
+ *   of that context, the next call looks it up again (and counts as a first
+ *   call once more).  Nothing is allocated, here or later.
+ *   Failure: the status word lives in the library's array, out of the
+ *   caller's reach; a Gram whose bounded waits gave up is reported by NaN on
+ *   the diagonal of H, which admmq_prepare() turns into ADMMQ_ERR_NONFINITE.
+ *   Speed: the partial sums of the k-split must fit the array, so from
+ *   d_in = 2048 up the split count falls (to 1 at d_in = 4096) and such a
+ *   call can be slower than admmq_build_hessian on the same input.
  *   All calls share the array and it keeps the last call's contents (the
  *   status word is cleared at the start of every call): calls that overlap on
  *   the GPU -- on different streams, or from different threads -- race on it

@@ -12,6 +12,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <mutex>
 #include <type_traits>
 #include <vector>
 
@@ -1711,22 +1712,67 @@ namespace {
 __device__ __align__(256) uint8_t g_static_scratch[ADMMQ_STATIC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
-void* g_static_ptr[kMaxDevices] = {};
-bool g_static_ready[kMaxDevices] = {};
 
-// Device address of g_static_scratch for the current device (looked up once
-// per device with that device current).
+// The array's device address belongs to the context the module was loaded
+// into: after cudaDeviceReset (or any other teardown of the primary context)
+// the module is loaded again and the array may sit elsewhere.  So the address
+// is cached per device together with the unique id of the context it was
+// looked up in, and looked up again whenever the current context differs.
+struct StaticSlot {
+  unsigned long long ctx_id;  // 0: nothing cached
+  void* ptr;
+};
+StaticSlot g_static_slot[kMaxDevices] = {};
+std::mutex g_static_mu;
+
+// Unique id of the calling thread's current context, or 0 when there is none
+// (or it was destroyed).  Driver entry points resolved through the runtime,
+// so the library needs no link to libcuda.
+unsigned long long current_ctx_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static bool resolved = false;
+  if (!resolved) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+    resolved = true;
+  }
+  if (!get_cur || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_cur(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of g_static_scratch in the current device's current
+// context: looked up with cudaGetSymbolAddress on the first call in a
+// context (which also creates the primary context if none is current), then
+// taken from the cache while that context stays current.
 int static_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return ADMMQ_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return ADMMQ_ERR_UNSUPPORTED;
-  if (!__atomic_load_n(&g_static_ready[dev], __ATOMIC_ACQUIRE)) {
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  const unsigned long long id = current_ctx_id();
+  StaticSlot& slot = g_static_slot[dev];
+  if (id == 0 || slot.ctx_id != id) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return ADMMQ_ERR_CUDA;
-    g_static_ptr[dev] = p;
-    __atomic_store_n(&g_static_ready[dev], true, __ATOMIC_RELEASE);
+    const unsigned long long now = current_ctx_id();  // the context the lookup ran in
+    slot.ptr = p;
+    slot.ctx_id = now;
+    *out = p;
+    return ADMMQ_OK;
   }
-  *out = g_static_ptr[dev];
+  *out = slot.ptr;
   return ADMMQ_OK;
 }
 

@@ -2,14 +2,15 @@
 
 Some callers cannot allocate device memory at the moment they need the
 Hessian: a framework whose memory pool already holds all of the device
-memory, or code that must not call cudaMalloc (it can synchronise the device
-and is not allowed while a stream is being captured).  This entry point keeps
+memory, or code on a latency-bound path that must not call cudaMalloc
+(which can synchronise the whole device).  This entry point keeps
 its scratch in a fixed device array inside the library instead of taking a
 workspace.  Called through the C ABI, it must return the same X^T X as the
 allocating admmq_build_hessian (within the 1e-4 relative Frobenius tolerance
 the Gram tests use), on two calls in a row, since the shared array keeps the
 previous call's contents; and it must refuse a d_in whose partial sums do not
-fit, before launching anything.
+fit, before launching anything.  Once the first call has loaded the
+library's code, a call leaves the device's free memory unchanged.
 
 This file is collected last so that a run stopping at the first failure has
 run every other test already.
@@ -47,8 +48,14 @@ def test_static_gram_equals_allocating_gram_twice():
         X = _acts(n, d, seed)
         ref = admmq.build_hessian(X)
         H = torch.full((d, d), float("nan"), dtype=torch.float32, device="cuda")
+        torch.cuda.synchronize()
+        free0 = torch.cuda.mem_get_info()[0]
         assert f(X.data_ptr(), n, d, H.data_ptr(), 0, stream) == 0
         torch.cuda.synchronize()
+        if seed == 12:
+            # the second call: the library's code is loaded by now, and the
+            # call takes no device memory of its own
+            assert torch.cuda.mem_get_info()[0] == free0
         assert torch.isfinite(H).all()
         assert torch.equal(H, H.T)
         err = float((H.double() - ref.double()).norm() / ref.double().norm())
