@@ -338,8 +338,24 @@ int admmq_split_mode(const admmq_ctx* ctx);
 
 /* Synchronises the stream and reads the kernel status words: ADMMQ_OK,
  * ADMMQ_ERR_TIMEOUT (a bounded wait gave up) or ADMMQ_ERR_RANGE (an fp16-split
- * operand left fp16's range; rerun with ADMMQ_SPLIT_MIXED or _3XTF32). */
+ * operand left fp16's range: the solve's result is not valid; switch the
+ * context with admmq_set_split and solve again). */
 int admmq_check(admmq_ctx* ctx, void* stream);
+
+/* Switch a context whose eigendecomposition is done (admmq_eigh) to another
+ * split precision (ADMMQ_SPLIT_3XTF32, _MIXED or _F16; not _AUTO): the
+ * eigenvector planes are encoded again from the float64 eigenvectors kept in
+ * the workspace and the scaled weights from W_hat, in the same buffers, and
+ * the timeout and range status words are cleared.  The iterate is not
+ * converted: admmq_init (or admmq_solve) must come next; admmq_iterate and
+ * admmq_finish return ADMMQ_ERR_INVALID_ARG until then.  A solve after the
+ * switch gives the same bits as a context created with that split.
+ * The fp16 split's operands carry 64x headroom over each row's scaled weight
+ * norm; a row whose iterate grows past it (seen on layers where the min/max
+ * grid refresh lets a row drift) sets the range word.  The recovery is this
+ * call with ADMMQ_SPLIT_MIXED, then the solve again.
+ * Asynchronous on `stream`; nothing is allocated. */
+int admmq_set_split(admmq_ctx* ctx, int split_mode, void* stream);
 
 /* Test hook for the failure path: pretend `iterations` more iterations have
  * been counted, so that the next fused launch's GEMM-2 tiles wait for GEMM-1

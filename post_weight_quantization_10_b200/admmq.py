@@ -116,6 +116,7 @@ def lib():
         "admmq_project": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp,
                                _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _i, _vp]),
         "admmq_split_mode": (_i, [_vp]),
+        "admmq_set_split": (_i, [_vp, _i, _vp]),
         "admmq_check": (_i, [_vp, _vp]),
         "admmq_debug_skew_ready": (_i, [_vp, _i]),
         "admmq_debug_rint_div": (_i, [_vp, _vp, _i64, _vp, _vp]),
@@ -297,9 +298,15 @@ class Solver:
 
     @property
     def split(self) -> str:
-        """The eigenbasis GEMMs' split precision ("3xtf32" or "mixed")."""
+        """The eigenbasis GEMMs' split precision: "3xtf32", "mixed" or "f16"."""
         mode = int(lib().admmq_split_mode(self._ctx))
         return {1: "3xtf32", 2: "mixed", 3: "f16"}[mode]
+
+    def set_split(self, split: str, stream=None):
+        """Switch to another split precision after eigh(); init() or solve()
+        must come next (see admmq_set_split in include/admmq.h)."""
+        _check(lib().admmq_set_split(self._ctx, SPLIT_MODES[split], _stream(stream)),
+               "admmq_set_split")
 
     def dump_wtilde(self, out: torch.Tensor | None):
         _check(lib().admmq_debug_dump_wtilde(self._ctx, _ptr(out)), "admmq_debug_dump_wtilde")
@@ -379,10 +386,21 @@ def gptq(G: torch.Tensor, W_hat: torch.Tensor, bits: int, group: int, lambda_rel
 
 def solve_layer(X: torch.Tensor, W_hat: torch.Tensor, params: Params, stream=None) -> Solver:
     """Gram -> setup -> solve for one layer; the Solver holds codes/scale/zero,
-    the residual history and the objective."""
+    the residual history and the objective.  Synchronises once at the end to
+    read the status words: when the fp16 split's range word is set, the layer
+    is solved again with the mixed split (admmq_set_split); any other error
+    raises AdmmqError."""
     H = build_hessian(X, stream=stream)
     s = Solver(X.shape[1], W_hat.shape[0], params, device=X.device)
     s.prepare(H, W_hat, stream)
     s.eigh(stream)
     s.solve(stream)
+    try:
+        s.check(stream)
+    except AdmmqError as e:
+        if e.status != ERR_RANGE:
+            raise
+        s.set_split("mixed", stream)
+        s.solve(stream)
+        s.check(stream)
     return s

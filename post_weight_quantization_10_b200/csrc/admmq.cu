@@ -1570,6 +1570,58 @@ int admmq_split_mode(const admmq_ctx* c) {
   return c->enc == ENC_MIX ? ADMMQ_SPLIT_MIXED : (c->enc == ENC_F16 ? ADMMQ_SPLIT_F16 : ADMMQ_SPLIT_3XTF32);
 }
 
+int admmq_set_split(admmq_ctx* c, int split_mode, void* stream) {
+  if (!c || !c->eig_done) return ADMMQ_ERR_INVALID_ARG;
+  if (!(split_mode == ADMMQ_SPLIT_3XTF32 || split_mode == ADMMQ_SPLIT_MIXED ||
+        split_mode == ADMMQ_SPLIT_F16))
+    return ADMMQ_ERR_INVALID_ARG;
+  const int enc = split_mode == ADMMQ_SPLIT_MIXED ? ENC_MIX
+                  : split_mode == ADMMQ_SPLIT_F16 ? ENC_F16
+                                                  : ENC_TF32X3;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int d = c->d, m = c->m;
+  // the operand maps of the new encoding (same buffers: every encoding fits
+  // 4 bytes per element per plane)
+  CUtensorMap mWt[2], mP[2], mT[2], mE[2], mQ[2];
+  bool ok = make_plane_maps(mWt, c->Wt_hi, c->Wt_lo, d, m, kBM, enc) &&
+            make_plane_maps(mP, c->P_hi, c->P_lo, d, m, kBM, enc) &&
+            make_plane_maps(mT, c->T_hi, c->T_lo, d, m, kBM, enc) &&
+            make_plane_maps(mE, c->E_hi, c->E_lo, d, d, EigCfg::B_ROWS, enc) &&
+            make_plane_maps(mQ, c->Q_hi, c->Q_lo, d, d, EigCfg::B_ROWS, enc);
+  if (!ok) return ADMMQ_ERR_CUDA;
+  // clear the timeout and range words; the setup and eigenvalue words stay
+  CK(cudaMemsetAsync(c->status, 0, sizeof(int), st));
+  CK(cudaMemsetAsync(c->status + 3, 0, sizeof(int), st));
+  const long long md = (long long)m * d;
+  int* flag = c->status + 3;
+  if (c->w_dtype == ADMMQ_DTYPE_F32) {
+    count_launch(), k_row_scales<float><<<grid_for(m, 8), 256, 0, st>>>(
+        (const float*)c->W_hat, c->rsig, m, d, enc, c->row_in, c->row_out);
+    count_launch(), k_scale_weights<float><<<grid_for(md), 256, 0, st>>>(
+        (const float*)c->W_hat, c->rsig, d, md, c->Wt_hi, c->Wt_lo, enc, c->row_in, flag);
+  } else {
+    count_launch(), k_row_scales<__nv_bfloat16><<<grid_for(m, 8), 256, 0, st>>>(
+        (const __nv_bfloat16*)c->W_hat, c->rsig, m, d, enc, c->row_in, c->row_out);
+    count_launch(), k_scale_weights<__nv_bfloat16><<<grid_for(md), 256, 0, st>>>(
+        (const __nv_bfloat16*)c->W_hat, c->rsig, d, md, c->Wt_hi, c->Wt_lo, enc, c->row_in,
+        flag);
+  }
+  CK(cudaGetLastError());
+  count_launch(), k_split_eigvecs<<<dim3(cdiv(d, 32), cdiv(d, 32)), dim3(32, 8), 0, st>>>(
+      c->Ht, d, c->E_hi, c->E_lo, c->Q_hi, c->Q_lo, enc);
+  CK(cudaGetLastError());
+  c->enc = enc;
+  for (int p = 0; p < 2; ++p) {
+    c->mWt[p] = mWt[p];
+    c->mP[p] = mP[p];
+    c->mT[p] = mT[p];
+    c->mE[p] = mE[p];
+    c->mQ[p] = mQ[p];
+  }
+  c->inited = false;  // the iterate's planes are in the old encoding: admmq_init next
+  return ADMMQ_OK;
+}
+
 int admmq_debug_rint_div(const float* y, const float* s, long long n, float* out, void* stream) {
   if (!y || !s || !out || n < 0 || n % 8 != 0) return ADMMQ_ERR_INVALID_ARG;
   if (n == 0) return ADMMQ_OK;

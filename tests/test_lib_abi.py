@@ -94,6 +94,7 @@ def test_alignment_checks_without_gpu(lib):
         assert call(list(ok), dual_scale=r) == -1, r
     assert call(list(ok), fit_on_w=2) == -1
     assert lib.admmq_split_mode(None) == -1
+    assert lib.admmq_set_split(None, 2, None) == -1
     assert lib.admmq_debug_dump_wtilde(None, None) == -1
 
 
