@@ -8,13 +8,16 @@ weight rows, weights with outliers over six orders of magnitude under the
 fp16 split's power-of-two row scales, and T = 0 (the solve is the RTN start).
 Each result must be a valid solution (codes in [0, L], positive scales,
 integer zero points in [0, L], the reported objective equal to the objective
-of the returned codes), close to the float64 oracle's free-running solve by
-the bar of the free-running tests, and exact where the method fixes it.
+of the returned codes), within the acceptance bar of the float64 oracle's
+free-running solve (widened only as far as the oracle's own spread under
+noise of the GPU's per-step size requires, as in the free-running tests),
+and exact where the method fixes it.
 """
 import numpy as np
 import pytest
 import torch
 
+import _spread as S
 from oracle import admmq_oracle as O
 from post_weight_quantization_10_b200 import workloads
 
@@ -82,12 +85,15 @@ def test_degenerate_layer_solves(A, name):
     s = _solve(A, p, split, X, W)
     H = O.hessian(X.float().cpu().numpy(), p.lambda_rel)
     Wm = W.float().cpu().numpy().T.astype(np.float64)
-    res = O.admm_q(H, Wm, p.bits, p.group, p.iters, rho0=p.rho0, gamma=p.gamma, grid="lsq")
+    eps = max(S.step0_error(A, p, X, W, H, Wm, "lsq", split=split), S.EPS_FLOOR)
+    res, runs = S.noisy_runs(H, Wm, p, "lsq", eps, seeds=16)
     codes, obj = _valid(p, s, H, Wm)
     agree = float(np.mean(codes == res["codes"].T))
     rel = obj / res["objective"] - 1.0 if res["objective"] > 0 else obj
-    print(f"{name}: split {s.split}, codes agree {agree:.5f}, objective rel {rel:+.3e}")
-    assert agree >= 0.9 and abs(rel) <= 0.2
+    agree_bar, rel_bar, lo, hi = S.bars(res, runs)
+    print(f"{name}: split {s.split}, codes agree {agree:.5f}, objective rel {rel:+.3e}; "
+          f"oracle at noise {eps:.1e}: agree >= {lo:.5f}, |rel| <= {hi:.2e}")
+    assert agree >= agree_bar and abs(rel) <= rel_bar
     if name == "zero_rows":
         # a zero row stays on its RTN grid (s = 1, z = 0) with every code 0
         for r in (5, 17):
@@ -115,17 +121,21 @@ def test_zero_iterations_is_the_rtn_start(A, split):
 @pytest.mark.parametrize("split", ["auto", "f16"])
 def test_extreme_bit_widths(A, bits, split):
     """b = 1 (two levels per group) and b = 8 (256 levels): valid solutions
-    close to the oracle's, with codes spanning the whole range [0, 2^b - 1]."""
+    within the bar of the free-running tests, with codes spanning the whole
+    range [0, 2^b - 1]."""
     p = workloads.scaled(BASE, 2048, 256, 64, group=64, bits=bits, iters=40, rank=16)
     X = workloads.make_activations(p, seed=6, device="cuda")
     W = workloads.make_weights(p, seed=6, device="cuda", dtype=torch.float32)
     s = _solve(A, p, split, X, W)
     H = O.hessian(X.float().cpu().numpy(), p.lambda_rel)
     Wm = W.float().cpu().numpy().T.astype(np.float64)
-    res = O.admm_q(H, Wm, p.bits, p.group, p.iters, rho0=p.rho0, gamma=p.gamma, grid="lsq")
+    eps = max(S.step0_error(A, p, X, W, H, Wm, "lsq", split=split), S.EPS_FLOOR)
+    res, runs = S.noisy_runs(H, Wm, p, "lsq", eps, seeds=16)
     codes, obj = _valid(p, s, H, Wm)
     assert codes.min() == 0 and codes.max() == (1 << bits) - 1
     agree = float(np.mean(codes == res["codes"].T))
     rel = obj / res["objective"] - 1.0
-    print(f"bits {bits} / {s.split}: codes agree {agree:.5f}, objective rel {rel:+.3e}")
-    assert agree >= 0.9 and abs(rel) <= 0.2
+    agree_bar, rel_bar, lo, hi = S.bars(res, runs)
+    print(f"bits {bits} / {s.split}: codes agree {agree:.5f}, objective rel {rel:+.3e}; "
+          f"oracle at noise {eps:.1e}: agree >= {lo:.5f}, |rel| <= {hi:.2e}")
+    assert agree >= agree_bar and abs(rel) <= rel_bar

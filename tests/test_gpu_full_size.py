@@ -15,6 +15,7 @@ import numpy as np
 import pytest
 import torch
 
+import _spread as S
 from oracle import admmq_oracle as O
 from oracle import projection_fp32 as P
 from post_weight_quantization_10_b200 import workloads
@@ -131,45 +132,31 @@ def test_full_size_teacher_forced(A, full_setup, grid, split):
     s.dump_wtilde(None)
 
 
-def _oracle_spread(full_setup, grid, res, monkeypatch, rel_noise=4e-6, seeds=(0, 1, 2)):
-    """How far the float64 oracle's own result moves on this layer when its
-    W-update carries relative noise of `rel_noise` (the GPU's per-step W~
-    error at this size is ~4e-6): (lowest code agreement, largest objective
-    change) over a few noise seeds."""
-    p, X, W, H, Wm, eig, _ = full_setup
-    w_update = O.w_update
-    agrees, rels = [], []
-    for seed in seeds:
-        rng = np.random.default_rng(seed)
-
-        def noisy(*a, rng=rng):
-            Wt = w_update(*a)
-            return Wt * (1.0 + rel_noise * rng.standard_normal(Wt.shape))
-
-        monkeypatch.setattr(O, "w_update", noisy)
-        r = O.admm_q(H, Wm, p.bits, p.group, p.iters, rho0=p.rho0, gamma=p.gamma, grid=grid,
-                     eig=eig)
-        monkeypatch.setattr(O, "w_update", w_update)
-        agrees.append(float(np.mean(r["codes"] == res["codes"])))
-        rels.append(abs(r["objective"] / res["objective"] - 1.0))
-    return min(agrees), max(rels)
-
-
 @pytest.mark.parametrize("grid", ["lsq", "minmax"])
-def test_full_size_free_running(A, full_setup, grid, monkeypatch):
+def test_full_size_free_running(A, full_setup, grid):
     """The whole T = 100 solve at 4096 x 4096: valid codes and grids, and on
-    the sampled rows codes and objective inside the spread the method itself
-    shows at this size.  The trajectory amplifies last-bit differences (step
-    parity is the teacher-forced test above), so the bar is the oracle's own
-    spread on this layer under W-update noise of the GPU's size, with margin:
-    codes agree >= (lowest noisy agreement - 0.05), objective within
-    2 x (largest noisy change) + 1e-3."""
-    p, X, W, H, Wm, _, _ = full_setup
-    res, _ = _oracle_run(full_setup, grid)
+    the sampled rows codes and objective within the acceptance bar, widened
+    only as far as the method's own spread at this size requires: the oracle
+    re-run on the same rows with its W-update perturbed by relative noise of
+    the GPU's measured per-step size (the W~ difference after iteration 0 on
+    the sampled rows), three seeds.  The trajectory amplifies last-bit
+    differences; step parity is the teacher-forced test above."""
+    p, X, W, H, Wm, eig, _ = full_setup
+    res, trace = _oracle_run(full_setup, grid)
     s = _solver(A, p, X, W, grid)
+    rows = torch.from_numpy(ROWS).cuda()
+    s.init()
+    wt = torch.empty((D, D), dtype=torch.float32, device="cuda")
+    s.dump_wtilde(wt)
+    s.iterate(0, 1)
+    s.dump_wtilde(None)
+    torch.cuda.synchronize()
+    ref0 = trace[0]["W_tilde"].T
+    eps = float(np.linalg.norm(wt[rows].cpu().numpy().astype(np.float64) - ref0)
+                / np.linalg.norm(ref0))
+    del wt
     s.solve()
     torch.cuda.synchronize()
-    rows = torch.from_numpy(ROWS).cuda()
     codes = s.codes[rows].cpu().numpy()
     sc, ze = s.scale[rows].cpu().numpy(), s.zero[rows].cpu().numpy()
     L = (1 << p.bits) - 1
@@ -179,11 +166,13 @@ def test_full_size_free_running(A, full_setup, grid, monkeypatch):
     obj_gpu = O.objective(H, Dg.T.astype(np.float64), Wm)
     rel = obj_gpu / res["objective"] - 1.0
     agree = float(np.mean(codes == res["codes"].T))
-    min_agree, max_rel = _oracle_spread(full_setup, grid, res, monkeypatch)
+    _, runs = S.noisy_runs(H, Wm, p, grid, max(eps, S.EPS_FLOOR), seeds=3, eig=eig)
+    agree_bar, rel_bar, lo, hi = S.bars(res, runs)
     print(f"full-size free-running {grid}: codes agree {agree:.5f}, objective rel {rel:+.3e}; "
-          f"oracle under noise: agree >= {min_agree:.5f}, |rel| <= {max_rel:.3e}")
-    assert agree >= min_agree - 0.05
-    assert abs(rel) <= 2.0 * max_rel + 1e-3
+          f"oracle at noise {eps:.1e}: agree >= {lo:.5f}, |rel| <= {hi:.3e}; "
+          f"bar: agree >= {agree_bar:.5f}, |rel| <= {rel_bar:.3e}")
+    assert agree >= agree_bar
+    assert abs(rel) <= rel_bar
 
 
 FIRST_ITERATION_SHAPES = {

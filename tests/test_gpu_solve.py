@@ -10,6 +10,7 @@ import numpy as np
 import pytest
 import torch
 
+import _spread as S
 from oracle import admmq_oracle as O
 from oracle import projection_fp32 as P
 from post_weight_quantization_10_b200 import workloads
@@ -192,17 +193,22 @@ def test_teacher_forced_iterations(A, name, grid, split):
 @pytest.mark.parametrize("name", ["tiny", "ragged", "down_small"])
 @pytest.mark.parametrize("grid", ["minmax", "lsq", "mse", "frozen"])
 def test_free_running_solve(A, name, grid):
-    """The whole solve, free-running on both sides.  The trajectory is
-    sensitive to rounding at the 1e-7 level (the float64 oracle itself only
-    reproduces ~99.6-99.95% of its codes under 1e-7..1e-6 relative noise), so
-    the per-step bar is checked above; here the GPU result must be a valid
-    solution, report the objective of its own codes, and stay close to the
-    oracle's."""
+    """The whole solve, free-running on both sides.  The GPU result must be a
+    valid solution and report the objective of its own codes.  Its codes and
+    objective are then held to the acceptance bar (>= 99.9% equal, objective
+    within 1e-3), widened only as far as the oracle's own spread on this
+    layer requires: the oracle re-run with its W-update perturbed by relative
+    noise of the GPU's measured per-step size (the trajectory amplifies
+    last-bit differences; step parity is the teacher-forced test above)."""
     p, X, W = _layer(name)
     s = _solver(A, p, X, W, grid)
     s.solve()
     torch.cuda.synchronize()
-    H, Wm, res = _oracle(p, X, W, grid)
+    Xn = X.float().cpu().numpy()
+    H = O.hessian(Xn, p.lambda_rel)
+    Wm = W.float().cpu().numpy().T.astype(np.float64)
+    eps = max(S.step0_error(A, p, X, W, H, Wm, grid), S.EPS_FLOOR)
+    res, runs = S.noisy_runs(H, Wm, p, grid, eps, seeds=16)
     codes = s.codes.cpu().numpy()
     L = (1 << p.bits) - 1
     assert codes.max() <= L
@@ -213,10 +219,13 @@ def test_free_running_solve(A, name, grid):
     assert O.objective(H, Dg.T, Wm) == pytest.approx(obj, rel=1e-4)
     agree = float(np.mean(codes == res["codes"].T))
     rel = obj / res["objective"] - 1.0
-    print(f"free-running {name}/{grid}: codes agree {agree:.5f}, objective rel {rel:+.3e}")
+    agree_bar, rel_bar, lo, hi = S.bars(res, runs)
+    print(f"free-running {name}/{grid}: codes agree {agree:.5f}, objective rel {rel:+.3e}; "
+          f"oracle at noise {eps:.1e}: agree >= {lo:.5f}, |rel| <= {hi:.2e}; "
+          f"bar: agree >= {agree_bar:.5f}, |rel| <= {rel_bar:.2e}")
     r = s.resid.cpu().numpy()[: p.iters]
     np.testing.assert_allclose(r[:3, 0], res["r"][:3], rtol=1e-3)
-    assert agree >= 0.9 and abs(rel) <= 0.2
+    assert agree >= agree_bar and abs(rel) <= rel_bar
 
 
 @pytest.mark.parametrize("name,split", [("tiny", "auto"), ("ragged", "auto"), ("ragged", "f16")])
@@ -255,8 +264,9 @@ def test_rescaled_dual_teacher_forced(A, name, split):
 @pytest.mark.parametrize("name", ["tiny", "ragged"])
 def test_rescaled_dual_solve(A, name):
     """The whole solve with rescale_dual: the fused and the per-GEMM
-    schedules give the same bits, the result is a valid solution close to
-    the oracle's own rescaled solve, and it differs from the default one
+    schedules give the same bits, the result is within the acceptance bar of
+    the oracle's own rescaled solve (widened only to the oracle's spread under
+    noise of the GPU's per-step size), and it differs from the default one
     (gamma > 1 makes the factor differ from 1)."""
     p, X, W = _layer(name)
     runs = {}
@@ -271,13 +281,15 @@ def test_rescaled_dual_solve(A, name):
     assert runs["fused"][2] == runs["per_gemm"][2]
     H = O.hessian(X.float().cpu().numpy(), p.lambda_rel)
     Wm = W.float().cpu().numpy().T.astype(np.float64)
-    res = O.admm_q(H, Wm, p.bits, p.group, p.iters, rho0=p.rho0, gamma=p.gamma, grid="lsq",
-                   rescale_dual=True)
+    eps = max(S.step0_error(A, p, X, W, H, Wm, "lsq", rescale_dual=True), S.EPS_FLOOR)
+    res, noisy = S.noisy_runs(H, Wm, p, "lsq", eps, seeds=16, rescale_dual=True)
     codes = runs["fused"][0].numpy()
     agree = float(np.mean(codes == res["codes"].T))
     rel = runs["fused"][2] / res["objective"] - 1.0
-    print(f"rescaled dual {name}: codes agree {agree:.5f}, objective rel {rel:+.3e}")
-    assert agree >= 0.9 and abs(rel) <= 0.2
+    agree_bar, rel_bar, lo, hi = S.bars(res, noisy)
+    print(f"rescaled dual {name}: codes agree {agree:.5f}, objective rel {rel:+.3e}; "
+          f"oracle at noise {eps:.1e}: agree >= {lo:.5f}, |rel| <= {hi:.2e}")
+    assert agree >= agree_bar and abs(rel) <= rel_bar
     plain = _solver(A, p, X, W, "lsq")
     plain.solve()
     assert not torch.equal(plain.buffer("V").cpu(), runs["fused"][1])
@@ -462,3 +474,50 @@ def test_bounded_wait_timeout_reports_and_recovers(A, name, split):
     ref.check()
     assert torch.equal(s.codes, ref.codes) and torch.equal(s.scale, ref.scale)
     assert float(s.objective.cpu()) == float(ref.objective.cpu())
+
+
+@pytest.mark.parametrize("name,grid,first,second", [("ragged", "lsq", "f16", "mixed"),
+                                                     ("tiny", "minmax", "3xtf32", "f16")])
+def test_set_split_equals_fresh_context(A, name, grid, first, second):
+    """admmq_set_split re-encodes a context's planes for another split
+    precision; a solve after the switch gives the bits of a context created
+    with that split (codes, grid, dual, objective, residual history)."""
+    p, X, W = _layer(name)
+    s = _solver(A, p, X, W, grid, split=first)
+    s.solve()
+    s.check()
+    s.set_split(second)
+    assert s.split == second
+    with pytest.raises(A.AdmmqError):
+        s.iterate(0, 1)        # the iterate must be started again first
+    s.solve()
+    s.check()
+    ref = _solver(A, p, X, W, grid, split=second)
+    ref.solve()
+    ref.check()
+    for k in ("codes", "scale", "zero", "resid", "objective"):
+        assert torch.equal(getattr(s, k), getattr(ref, k)), k
+    assert torch.equal(s.buffer("V"), ref.buffer("V"))
+
+
+def test_fp16_range_falls_back_to_mixed(A):
+    """The fp16 split's operands carry 64x headroom over each row's scaled
+    weight norm.  On the down_proj-like layer, the min/max refresh lets one
+    row drift until its iterate leaves that range: the solve reports
+    ADMMQ_ERR_RANGE.  solve_layer then switches to the mixed split and solves
+    again, which gives the bits of a mixed-split solve."""
+    p, X, W = _layer("down_small")
+    prm = A.Params(bits=p.bits, group=p.group, iters=p.iters, rho0=p.rho0, gamma=p.gamma,
+                   lambda_rel=p.lambda_rel, grid="minmax", split="f16")
+    raw = _solver(A, p, X, W, "minmax", split="f16")
+    raw.solve()
+    with pytest.raises(A.AdmmqError) as ei:
+        raw.check()
+    assert ei.value.status == A.ERR_RANGE
+    s = A.solve_layer(X, W, prm)
+    assert s.split == "mixed"
+    ref = _solver(A, p, X, W, "minmax", split="mixed")
+    ref.solve()
+    ref.check()
+    for k in ("codes", "scale", "zero", "objective"):
+        assert torch.equal(getattr(s, k), getattr(ref, k)), k
