@@ -7,8 +7,10 @@ its Python binding) never calls it: there is no CPU fallback.
   admmq_oracle     float64 Hessian, scaling, ADMM-Q, RTN, GPTQ, Babai, pack
   projection_fp32  float32 op-by-op grid fit / projection / fused epilogue,
                    the bit-exact specification of the projection kernels
+  spread           the oracle's own spread under W-update noise, which sets
+                   the bar for free-running GPU solves
 
 Pinned by tests/test_oracle_pins.py; "parity unpinned" parts are listed in the
 admmq_oracle module docstring.
 """
-from . import admmq_oracle, projection_fp32  # noqa: F401
+from . import admmq_oracle, projection_fp32, spread  # noqa: F401

@@ -18,21 +18,25 @@ import torch
 
 
 class InputPipeline:
-    """Two device slots for a fixed set of input tensors (shapes, dtypes)."""
+    """Device slots (two by default) for a fixed set of input tensors (shapes,
+    dtypes).  One slot is enough when something else runs between a slot's
+    use and its next copy (e.g. one pipeline per solve of a decoder layer,
+    the copy for solve i + 1 running during solve i)."""
 
-    def __init__(self, like: list[torch.Tensor], device):
+    def __init__(self, like: list[torch.Tensor], device, slots: int = 2,
+                 copy_stream: torch.cuda.Stream | None = None):
         self.slots = [[torch.empty(t.shape, dtype=t.dtype, device=device) for t in like]
-                      for _ in range(2)]
-        self.copy_stream = torch.cuda.Stream(device=device)
-        self.copied = [torch.cuda.Event() for _ in range(2)]
-        self.used = [torch.cuda.Event() for _ in range(2)]
+                      for _ in range(slots)]
+        self.copy_stream = copy_stream or torch.cuda.Stream(device=device)
+        self.copied = [torch.cuda.Event() for _ in range(slots)]
+        self.used = [torch.cuda.Event() for _ in range(slots)]
         self.next = 0
 
     def prefetch(self, host: list[torch.Tensor]) -> int:
         """Enqueue the copy of `host` (pinned tensors) into the next slot on the
         copy stream; returns the slot."""
         slot = self.next
-        self.next ^= 1
+        self.next = (self.next + 1) % len(self.slots)
         with torch.cuda.stream(self.copy_stream):
             self.copy_stream.wait_event(self.used[slot])  # its previous readers are done
             for dst, src in zip(self.slots[slot], host):
