@@ -58,10 +58,12 @@ def peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, src="fallback")
 
 
-# Source files each measured kernel is compiled from: its DRAM traffic figure
-# (profiles/traffic.json) stands only while these are unchanged.
+# Source files each measured kernel is compiled and launched from (its
+# launch geometry, e.g. the tile visiting order, is set in admmq.cu): its
+# DRAM traffic figure (profiles/traffic.json) stands only while these are
+# unchanged.
 KERNEL_SOURCES = {
-    "admm_loop": ["ptx.cuh", "gemm.cuh", "kernels.cuh", "admm_loop.cuh"],
+    "admm_loop": ["ptx.cuh", "gemm.cuh", "kernels.cuh", "admm_loop.cuh", "admmq.cu"],
     "project": ["ptx.cuh", "gemm.cuh", "kernels.cuh", "admmq.cu"],
     "pack": ["admmq.cu"],
 }

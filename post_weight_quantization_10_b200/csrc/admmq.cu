@@ -639,10 +639,24 @@ GemmGeom make_geom(int M, int N, long long K, int BN, int BK, int splits, bool t
 }
 
 // Geometry of an eigenbasis GEMM [rows][d] x [d][d] for an encoding (its K
-// per stage: 32 fp32 or 64 fp16 elements).
+// per stage: 32 fp32 or 64 fp16 elements).  A band's A panels (band unit
+// rows x d x the encoding's bytes per element, both planes) are re-read for
+// every tile column of the band, so they should stay in L2: the band is the
+// most unit rows (at most 8) whose panels fit 48 MiB.  Measured per fused
+// launch at d = 12288 (down_proj, fp16 split, 12.6 MB of A per unit row):
+// bands 2 / 3 / 4 / 5 / 6 / 8 took 612-619 / 602-604 / 598-599 / 602 /
+// 599-604 / 615-616 ms; at d = 4096 (4 MB per unit row) bands 4-12 are
+// within 1% and 8 is kept.
 GemmGeom eig_geom(int enc, int rows, int d, int* status) {
-  return enc == ENC_F16 ? make_geom(rows, d, d, EigCfgF::BN, EigCfgF::BK, 1, false, status, EigCfgF::UNIT_M)
-                        : make_geom(rows, d, d, EigCfg::BN, EigCfg::BK, 1, false, status, EigCfg::UNIT_M);
+  GemmGeom g = enc == ENC_F16
+                   ? make_geom(rows, d, d, EigCfgF::BN, EigCfgF::BK, 1, false, status, EigCfgF::UNIT_M)
+                   : make_geom(rows, d, d, EigCfg::BN, EigCfg::BK, 1, false, status, EigCfg::UNIT_M);
+  const long long unit_m = enc == ENC_F16 ? EigCfgF::UNIT_M : EigCfg::UNIT_M;
+  const long long elem = enc == ENC_F16 ? 4 : 8;  // bytes per A element over both planes
+  const long long fit = (48ll << 20) / (unit_m * (long long)d * elem);
+  const int cap = fit < 1 ? 1 : (fit > 8 ? 8 : (int)fit);
+  if (g.band > cap) g.band = cap;
+  return g;
 }
 
 // Launches k_gemm<Cfg, Work> over `units` work units: one CTA per SM, or one
