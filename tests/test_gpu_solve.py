@@ -521,3 +521,27 @@ def test_fp16_range_falls_back_to_mixed(A):
     ref.check()
     for k in ("codes", "scale", "zero", "objective"):
         assert torch.equal(getattr(s, k), getattr(ref, k)), k
+
+
+def test_solve_overlapped_matches_separate_solves(A):
+    """pipeline.solve_overlapped (the largest eigendecomposition on a second
+    stream while the other layers are solved) gives every layer the bits of
+    solving it alone."""
+    from post_weight_quantization_10_b200 import pipeline
+    layers = []
+    for name in ("ragged", "down_small", "tiny"):
+        p, X, W = _layer(name)
+        layers.append((p, X, W))
+    jobs, refs = [], []
+    for p, X, W in layers:
+        prm = A.Params(bits=p.bits, group=p.group, iters=p.iters, rho0=p.rho0, gamma=p.gamma,
+                       lambda_rel=p.lambda_rel, grid="lsq")
+        G = A.build_hessian(X)
+        jobs.append((A.Solver(X.shape[1], W.shape[0], prm), G, W))
+        refs.append(A.solve_layer(X, W, prm))
+    pipeline.solve_overlapped(jobs)
+    torch.cuda.synchronize()
+    for (s, _, _), ref in zip(jobs, refs):
+        s.check()
+        for k in ("codes", "scale", "zero", "objective"):
+            assert torch.equal(getattr(s, k), getattr(ref, k)), k
