@@ -60,6 +60,8 @@ MSE_EXACT = (pins.test_mse_clip_exact_grid_keeps_minmax, ())
 MSE_F64 = (pins.test_mse_clip_search_against_float64, (3,))
 LSQ_EXACT = (pins.test_lsq_refit_recovers_exact_grid, ())
 LSQ_DOWN = (pins.test_lsq_refit_does_not_increase_weighted_error, ())
+LSQ_STAGES = (pins.test_lsq_refit_stages_against_lstsq, ())
+LSQ_MIN = (pins.test_lsq_refit_scale_is_a_weighted_minimum, ())
 TF32 = (pins.test_tf32_split_reconstructs_float32, ())
 F16 = (pins.test_f16_split_encoding, ())
 F16_ROWS = (pins.test_f16_row_scales, ())
@@ -140,7 +142,16 @@ MISTAKES = {
                                  [LSQ_EXACT, LSQ_DOWN]),
     "lsq_variance_uses_mean_y": (P, "fit_lsq", "var = _f(Sqq - _f(Sq * qm))", "var = _f(Sqq - _f(Sq * ym))",
                                  [LSQ_EXACT, LSQ_DOWN]),
-    "lsq_zero_point_sign": (P, "fit_lsq", "_f(qm - _f(ym /", "_f(qm + _f(ym /", [LSQ_EXACT, LSQ_DOWN]),
+    "lsq_zero_point_sign": (P, "fit_lsq", "_f(qm - _f(ym /", "_f(qm + _f(ym /",
+                            [LSQ_EXACT, LSQ_DOWN, LSQ_STAGES]),
+    "lsq_second_fit_drops_factor_2": (P, "fit_lsq", "_f(f32(2) * zc)", "zc", [LSQ_STAGES, LSQ_MIN]),
+    "lsq_second_fit_wrong_cross_term": (P, "fit_lsq", "num = _f(Sqy - _f(zc * Sy))",
+                                        "num = _f(Sqy - _f(zc * Sq))", [LSQ_STAGES, LSQ_MIN]),
+    "lsq_zero_point_floor": (P, "fit_lsq", "np.clip(np.rint(_f(qm", "np.clip(np.floor(_f(qm",
+                             [LSQ_STAGES]),
+    "lsq_keeps_first_slope": (P, "fit_lsq", "s = np.where(ok, s2, s0)", "s = np.where(ok, s1, s0)",
+                              [LSQ_STAGES, LSQ_MIN]),
+    "lsq_unweighted_mean": (P, "fit_lsq", "Sw = _f(Sw + w)", "Sw = _f(Sw + f32(1))", [LSQ_STAGES]),
     # operand encodings
     "tf32_truncates": (P, "tf32_round", "((b + 0xFFF + lsb) >> 13) << 13", "(b >> 13) << 13", [TF32]),
     "f16_low_part_unscaled": (P, "split_f16", "_f(xs - hi.astype(np.float32))",

@@ -385,6 +385,67 @@ def test_lsq_refit_does_not_increase_weighted_error():
     assert e1.sum() < e0.sum()
 
 
+def test_lsq_refit_stages_against_lstsq():
+    """Each stage of the least-squares refresh against numpy's least-squares
+    solver in float64 on the same data (an independent route; the refit
+    itself sums in float32, element order):
+    1. with the codes q of the previous grid, the weighted straight-line fit
+       y ~ s1 q + b gives the slope s1 and the zero point z = -b / s1, which
+       is rounded and clamped to an integer zc;
+    2. with zc fixed, the scale minimises sum w (y - s (q - zc))^2.
+    Groups whose fit falls back (a non-positive slope) keep the previous
+    grid."""
+    rng = np.random.default_rng(31)
+    L = 7
+    G, g = 300, 128
+    y = (rng.standard_normal((G, g)) * 0.05 + rng.standard_normal((G, 1)) * 0.02).astype(np.float32)
+    w = np.exp(rng.standard_normal((G, g))).astype(np.float32)
+    s0, z0 = P.fit_minmax((y * 1.2).astype(np.float32), L)
+    s, z = P.fit_lsq(y, w, s0, z0, L)
+    q = P.round_to_grid(y, s0, z0, L).astype(np.float64)
+    yd, wd = y.astype(np.float64), w.astype(np.float64)
+    checked = 0
+    for i in range(G):
+        rw = np.sqrt(wd[i])
+        A = np.stack([q[i], np.ones(g)], axis=1) * rw[:, None]
+        slope, icpt = np.linalg.lstsq(A, yd[i] * rw, rcond=None)[0]
+        if slope <= 0:
+            assert s[i] == s0[i] and z[i] == z0[i]
+            continue
+        zc = float(np.clip(np.rint(-icpt / slope), 0, L))
+        if abs(-icpt / slope - np.rint(-icpt / slope)) < 1e-3:
+            continue  # a zero point within float32 reach of a rounding tie
+        assert z[i] == zc, (i, z[i], zc)
+        a = (q[i] - zc) * rw
+        s_ref = np.linalg.lstsq(a[:, None], yd[i] * rw, rcond=None)[0][0]
+        if s_ref > 0:
+            assert s[i] == pytest.approx(s_ref, rel=2e-5), i
+        checked += 1
+    assert checked > 0.8 * G
+
+
+def test_lsq_refit_scale_is_a_weighted_minimum():
+    """The refitted scale minimises the weighted squared error of the codes
+    it was fitted from, at the refitted zero point: moving it by 1e-3
+    either way increases sum w (y - s (q - z))^2."""
+    rng = np.random.default_rng(32)
+    L = 3
+    y = (rng.standard_normal((100, 64)) * 0.05).astype(np.float32)
+    w = np.exp(rng.standard_normal((100, 64))).astype(np.float32)
+    s0, z0 = P.fit_minmax(y, L)
+    s, z = P.fit_lsq(y, w, s0, z0, L)
+    q = P.round_to_grid(y, s0, z0, L).astype(np.float64)
+    yd, wd = y.astype(np.float64), w.astype(np.float64)
+
+    def e(sc):
+        return np.sum(wd * (yd - sc[:, None] * (q - z.astype(np.float64)[:, None])) ** 2, axis=1)
+    sd = s.astype(np.float64)
+    moved = (s != s0) | (z != z0)
+    assert moved.mean() > 0.5
+    assert np.all((e(sd) <= e(sd * (1 + 1e-3)))[moved])
+    assert np.all((e(sd) <= e(sd * (1 - 1e-3)))[moved])
+
+
 def _epilogue_inputs(m, d, g, bits, seed):
     """A [d_out][d_in] tile of W~ and V~ with a scaling vector, its inverse,
     diag(H) = 1/sigma^2, and a previous grid and codes (the min/max RTN grid
