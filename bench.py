@@ -800,8 +800,12 @@ def run_ours(args, rank, world, device):
 def stream_kernels(A, grid, device, reps=10):
     """HBM-bound kernels timed on their own, on buffers larger than L2: the
     standalone projection (the fused epilogue's float32 arithmetic reading W~
-    from memory) and the b-bit pack.  Algorithmic bytes per element: W~ 4,
-    V 4 + 4, codes 1 + 1, P planes 8 (projection); codes 1 + b/8 (pack)."""
+    from memory) and the b-bit pack.  The projection writes P in the fp16
+    split, the encoding the solve uses at this shape (d_in >= 2048); its
+    algorithmic bytes per element: W~ 4, V 4 + 4, codes 1 + 1, P planes 2 + 2
+    (18).  `project_by_grid` times every grid refresh in that encoding, and
+    the least-squares one also in the mixed encoding (P planes 4 + 4, 22
+    bytes).  The pack: codes 1 + b/8 bytes per element."""
     pk = peaks()
     m, d, g, bits = 25600, 5120, 128, 3          # the up_proj 32B layer shape
     gen = torch.Generator(device=device).manual_seed(7)
@@ -814,16 +818,27 @@ def stream_kernels(A, grid, device, reps=10):
     codes = torch.randint(0, L + 1, (m, d), generator=gen, device=device, dtype=torch.uint8)
     scale = torch.full((m, d // g), 0.01, device=device)
     zero = torch.full((m, d // g), 3.0, device=device)
-    phi = torch.empty((m, d), device=device)
-    plo = torch.empty((m, 2 * d), dtype=torch.int16, device=device)  # bf16 correction rows
+    # row scales of the fp16 split: 2^e with |row| 2^e in [2^9, 2^10)
+    rows = torch.linalg.vector_norm(wt, dim=1)
+    row_scale = torch.exp2(torch.ceil(9.0 - torch.log2(rows)))
+    flag = torch.zeros(1, dtype=torch.int32, device=device)
+    phi = torch.empty((m, d), device=device)     # mixed: fp32 plane, bf16 correction rows
+    plo = torch.empty((m, 2 * d), dtype=torch.int16, device=device)
+    f16_hi = torch.empty((m, d), dtype=torch.int16, device=device)
+    f16_lo = torch.empty((m, d), dtype=torch.int16, device=device)
     resid = torch.zeros(2, dtype=torch.float64, device=device)
     big = torch.randint(0, L + 1, (4 * m, d), generator=gen, device=device, dtype=torch.uint8)
     packed = torch.empty((4 * m, d * bits // 32), dtype=torch.int32, device=device)
-    out = {}
-    for name, fn, nbytes, shape in (
-            ("project", lambda: A.project(wt, V, sig, rsig, hd, bits, g, grid, codes, scale, zero,
-                                          phi, plo, resid=resid), 22.0 * m * d, [m, d]),
-            ("pack", lambda: A.pack(big, bits, out=packed), (1 + bits / 8) * 4 * m * d, [4 * m, d])):
+
+    def proj(gr, split):
+        if split == "f16":
+            return lambda: A.project(wt, V, sig, rsig, hd, bits, g, gr, codes, scale, zero,
+                                     f16_hi, f16_lo, resid=resid, split="f16",
+                                     row_scale=row_scale, range_flag=flag)
+        return lambda: A.project(wt, V, sig, rsig, hd, bits, g, gr, codes, scale, zero,
+                                 phi, plo, resid=resid, split="mixed")
+
+    def timed(fn):
         fn()
         torch.cuda.synchronize()
         a = torch.cuda.Event(enable_timing=True)
@@ -833,11 +848,28 @@ def stream_kernels(A, grid, device, reps=10):
             fn()
         b.record()
         torch.cuda.synchronize()
-        ms = a.elapsed_time(b) / reps
+        return a.elapsed_time(b) / reps
+
+    def entry(ms, nbytes, shape, traffic):
         gbs = nbytes / (ms / 1e3) / 1e9
-        out[name] = {"shape": shape, "bits": bits, "alg_bytes": nbytes, "ms": ms, "gbs": gbs,
-                     "frac_hbm": gbs / pk["hbm"], "traffic": measured_traffic(name, "stream")}
-    del wt, V, codes, phi, plo, big, packed
+        return {"shape": shape, "bits": bits, "alg_bytes": nbytes, "ms": ms, "gbs": gbs,
+                "frac_hbm": gbs / pk["hbm"], "traffic": traffic}
+
+    out = {}
+    out["project"] = entry(timed(proj(grid, "f16")), 18.0 * m * d, [m, d],
+                           measured_traffic("project", "stream") if grid == "lsq" else None)
+    out["project"].update(grid=grid, split="f16")
+    by = {}
+    for gr, split, nb in (("lsq", "f16", 18.0), ("minmax", "f16", 18.0), ("frozen", "f16", 18.0),
+                          ("mse", "f16", 18.0), ("lsq", "mixed", 22.0)):
+        e = entry(timed(proj(gr, split)), nb * m * d, [m, d], None)
+        by[f"{gr}/{split}"] = {k: e[k] for k in ("ms", "gbs", "frac_hbm", "alg_bytes")}
+    out["project_by_grid"] = by
+    out["pack"] = entry(timed(lambda: A.pack(big, bits, out=packed)), (1 + bits / 8) * 4 * m * d,
+                        [4 * m, d], measured_traffic("pack", "stream"))
+    if int(flag.item()) != 0:
+        raise RuntimeError("stream projection: fp16 range flag set")
+    del wt, V, codes, phi, plo, f16_hi, f16_lo, big, packed
     torch.cuda.empty_cache()
     return out
 

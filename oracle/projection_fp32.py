@@ -20,7 +20,12 @@ Grid semantics (our reading; the pages do not define the fit):
           y ~ s (q - z) with weights w = diag(H) (the metric of the scaled
           problem): first slope and offset, then the integer zero point, then
           the slope again for that zero point.  Groups whose fit is degenerate
-          keep the previous grid.
+          keep the previous grid.  Each of the fit's five sums is taken over
+          consecutive blocks of 32 columns, each block in element order, and
+          the block sums are then added pairwise ((B0 + B1) + (B2 + B3) for a
+          group of 128, B0 + B1 for 64, B0 alone for 32): the pages state the
+          fit in exact arithmetic, so the float32 summation order is ours to
+          fix, and blocks let one thread per block share a group.
   mse     clipping search: for each ratio a in CLIP_RATIOS (1, 31/32, ..., 17/32,
           exact in float32) the min/max grid of the clipped range
           (a * mn, a * mx); each candidate's squared error sum (y - D)^2 is
@@ -88,22 +93,43 @@ def fit_mse(yg: np.ndarray, L: int, return_error: bool = False):
     return tuple(best) if return_error else (best[0], best[1])
 
 
+LSQ_BLOCK = 32  # columns per element-ordered block of the least-squares sums
+
+
+def _pairwise(parts):
+    """Adjacent block sums added pairwise, level by level (an odd last one
+    moves up a level unchanged)."""
+    while len(parts) > 1:
+        nxt = [tuple(_f(a + b) for a, b in zip(parts[i], parts[i + 1]))
+               for i in range(0, len(parts) - 1, 2)]
+        if len(parts) % 2:
+            nxt.append(parts[-1])
+        parts = nxt
+    return parts[0]
+
+
 def fit_lsq(yg: np.ndarray, wg: np.ndarray, s_prev: np.ndarray, z_prev: np.ndarray, L: int):
-    """Weighted least-squares grid refit, sums taken in element order."""
+    """Weighted least-squares grid refit; each sum is the pairwise float32 sum
+    of its 32-column block sums, each block taken in element order."""
     yg, wg = _f(yg), _f(wg)
     s0, z0 = _f(s_prev), _f(z_prev)
     q = round_to_grid(yg, s0, z0, L)
     G, g = yg.shape
-    Sw = np.zeros(G, f32); Sq = np.zeros(G, f32); Sqq = np.zeros(G, f32)
-    Sy = np.zeros(G, f32); Sqy = np.zeros(G, f32)
-    for i in range(g):
-        w, qi, yi = wg[:, i], q[:, i], yg[:, i]
-        wq = _f(w * qi)
-        Sw = _f(Sw + w)
-        Sq = _f(Sq + wq)
-        Sqq = _f(Sqq + _f(wq * qi))
-        Sy = _f(Sy + _f(w * yi))
-        Sqy = _f(Sqy + _f(wq * yi))
+    blocks = []
+    for lo in range(0, g, LSQ_BLOCK):
+        hi = min(lo + LSQ_BLOCK, g)
+        Sw = np.zeros(G, f32); Sq = np.zeros(G, f32); Sqq = np.zeros(G, f32)
+        Sy = np.zeros(G, f32); Sqy = np.zeros(G, f32)
+        for i in range(lo, hi):
+            w, qi, yi = wg[:, i], q[:, i], yg[:, i]
+            wq = _f(w * qi)
+            Sw = _f(Sw + w)
+            Sq = _f(Sq + wq)
+            Sqq = _f(Sqq + _f(wq * qi))
+            Sy = _f(Sy + _f(w * yi))
+            Sqy = _f(Sqy + _f(wq * yi))
+        blocks.append((Sw, Sq, Sqq, Sy, Sqy))
+    Sw, Sq, Sqq, Sy, Sqy = _pairwise(blocks)
     qm = _f(Sq / Sw)
     ym = _f(Sy / Sw)
     var = _f(Sqq - _f(Sq * qm))

@@ -430,33 +430,39 @@ __global__ void k_rint_div(const float* __restrict__ y, const float* __restrict_
   }
 }
 
-// Standalone projection: one thread per (row, group), W~ read from memory.
-// The passes over a group read each of its elements two or three times, and
-// once enough warps run to cover the memory latency their groups (2 x g
-// floats each) no longer stay in L1, so by default a block is one warp of 32
-// rows that first copies its rows' W~ and V~ segments into shared memory
-// (coalesced 16-byte asynchronous copies, a whole row segment per
-// instruction for g = 128); the passes read them from there and DRAM sees
-// each input once.  The 16-candidate error search of GRID_MSE is bound by
-// arithmetic rather than memory, so it keeps more warps per SM by reading W~
-// and V~ from global memory (STAGED = false, 128-thread blocks).
-constexpr int kProjRows = 32;
+// Standalone projection, W~ read from memory.  The passes over a group read
+// each of its elements two or three times, and once enough warps run to
+// cover the memory latency their groups (2 x g floats each) no longer stay
+// in L1, so by default a block is one warp that first copies its rows' W~
+// and V~ segments into shared memory (coalesced 16-byte asynchronous copies,
+// a whole row segment per instruction for g = 128); the passes read them
+// from there and DRAM sees each input once.  A lane takes one 32-column block
+// of a (row, group): TPG = g / 32 lanes share a group and a warp holds 32 /
+// TPG rows (8 for g = 128), so a warp stages about 9 KB whatever g is and
+// many warps fit on an SM.  The 16-candidate error search of GRID_MSE is
+// bound by arithmetic rather than memory, so it reads W~ and V~ from global
+// memory (STAGED = false, 128-thread blocks, a thread per (row, group)).
+__host__ __device__ constexpr int proj_rows(int tpg) { return 32 / tpg; }
 // floats per row slot: W~ (g), V~ (g), 4 of padding so that the rows' 16-byte
-// reads at one column spread over the banks; after the 32 row slots, the
+// reads at one column spread over the banks; after the row slots, the
 // group's sigma, 1/sigma and diag(H) (g each), shared by the block's rows
 __host__ __device__ constexpr int proj_slot(int g) { return 2 * g + 4; }
-__host__ __device__ constexpr int proj_floats(int g) { return kProjRows * proj_slot(g) + 3 * g; }
+__host__ __device__ constexpr int proj_floats(int g, int tpg) {
+  return proj_rows(tpg) * proj_slot(g) + 3 * g;
+}
 
-template <int MODE, int ENC, bool STAGED>
-__global__ void __launch_bounds__(STAGED ? kProjRows : 128) k_project(
+template <int MODE, int ENC, bool STAGED, int TPG>
+__global__ void __launch_bounds__(STAGED ? 32 : 128) k_project(
     const float* __restrict__ wt, float* V, const float* __restrict__ sig,
     const float* __restrict__ rsig, const float* __restrict__ hd, int m, int d, int g, int L,
     uint8_t* codes, float* scale, float* zero, void* p_hi, void* p_lo,
     const float* __restrict__ row_in, int* flag, double* resid, float vs, int fit_w) {
+  static_assert(TPG == 1 || STAGED, "lanes that share a group share staged rows");
+  constexpr int kRows = STAGED ? proj_rows(TPG) : 128;
   extern __shared__ float4 proj_smem[];
   float* stage = reinterpret_cast<float*>(proj_smem);
   const int lane = threadIdx.x & 31;
-  const int row0 = blockIdx.x * blockDim.x;
+  const int row0 = blockIdx.x * kRows;
   const int grp = blockIdx.y;
   const int col0 = grp * g;
   const int slot = proj_slot(g);
@@ -464,7 +470,7 @@ __global__ void __launch_bounds__(STAGED ? kProjRows : 128) k_project(
     // rows past m are filled with zeros (they are projected, never stored)
     const int per_row = g / 2;  // float4 pieces of W~ and V~ in one row
     const uint32_t sbase = smem_u32(stage);
-    for (int i = lane; i < kProjRows * per_row; i += 32) {
+    for (int i = lane; i < kRows * per_row; i += 32) {
       const int rr = i / per_row, piece = i - rr * per_row;
       const int arr = piece >= g / 4 ? 1 : 0;
       const int k = 4 * (piece - arr * (g / 4));
@@ -476,36 +482,41 @@ __global__ void __launch_bounds__(STAGED ? kProjRows : 128) k_project(
         *reinterpret_cast<float4*>(stage + off_s) = make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
-    float* cols = stage + kProjRows * slot;
+    float* cols = stage + kRows * slot;
     for (int i = lane; i < 3 * (g / 4); i += 32) {
       const int v = i / (g / 4), k = 4 * (i - v * (g / 4));
       const float* src = (v == 0 ? sig : v == 1 ? rsig : hd) + col0 + k;
       cp_async16(smem_u32(cols + v * g + k), src);
     }
-    // the codes of this lane's row, read in the projection pass
-    if (row0 + lane < m) prefetch_l2_bulk(codes + (long long)(row0 + lane) * d + col0, (uint32_t)g);
+    // the codes of this block's rows, read in the projection pass
+    if (lane < kRows && row0 + lane < m)
+      prefetch_l2_bulk(codes + (long long)(row0 + lane) * d + col0, (uint32_t)g);
     cp_async_wait_all();
     __syncwarp();
   }
-  const int row = row0 + (int)threadIdx.x;
+  // this thread's row of the block and its 32-column block of the group
+  const int rr = TPG > 1 ? lane % kRows : (int)threadIdx.x;
+  const int blk = TPG > 1 ? lane / kRows : 0;
+  const int hc = 32 * blk;  // first column of this thread within the group
+  const int row = row0 + rr;
   const bool valid = row < m;
-  const long long off = (long long)(valid ? row : 0) * d + col0;
+  const long long off = (long long)(valid ? row : 0) * d + col0 + hc;
   const long long goff = (long long)(valid ? row : 0) * (d / g) + grp;
   ProjRow r;
   r.V = V + off;
   if (STAGED) {
-    const float* cols = stage + kProjRows * slot;
-    r.sig = cols;
-    r.rsig = cols + g;
-    r.hd = cols + 2 * g;
+    const float* cols = stage + kRows * slot;
+    r.sig = cols + hc;
+    r.rsig = cols + g + hc;
+    r.hd = cols + 2 * g + hc;
   } else {
     r.sig = sig + col0;
     r.rsig = rsig + col0;
     r.hd = hd + col0;
   }
   r.codes = codes + off;
-  r.phi = plane0_at(ENC, p_hi, valid ? row : 0, d, col0);
-  r.plo = plane1_at(ENC, p_lo, valid ? row : 0, d, col0);
+  r.phi = plane0_at(ENC, p_hi, valid ? row : 0, d, col0 + hc);
+  r.plo = plane1_at(ENC, p_lo, valid ? row : 0, d, col0 + hc);
   r.scale = scale + goff;
   r.zero = zero + goff;
   r.wdump = nullptr;
@@ -514,7 +525,8 @@ __global__ void __launch_bounds__(STAGED ? kProjRows : 128) k_project(
   r.fit_w = fit_w;
   r.flag = flag;
   r.valid = valid;
-  const float* mine = stage + lane * slot;
+  r.grid_out = blk == 0;
+  const float* mine = stage + rr * slot + hc;
   auto loadw = [&](int c, float (&w)[32]) {
 #pragma unroll
     for (int k = 0; k < 32; k += 4) {
@@ -537,7 +549,7 @@ __global__ void __launch_bounds__(STAGED ? kProjRows : 128) k_project(
     }
   };
   float r2 = 0.f, s2 = 0.f;
-  project_group<MODE, ENC, STAGED>(loadw, loadv, r, g, L, r2, s2);
+  project_group<MODE, ENC, STAGED, TPG>(loadw, loadv, r, g, L, r2, s2);
   r2 = warp_sum(r2);
   s2 = warp_sum(s2);
   if (lane == 0) {
@@ -1547,34 +1559,47 @@ int admmq_project(const float* wt, float* V, const float* sig, const float* rsig
   cudaStream_t st = (cudaStream_t)stream;
   CK(cudaMemsetAsync(resid, 0, 2 * sizeof(double), st));
   const bool staged = mode != ADMMQ_GRID_MSE;
-  const int block = staged ? kProjRows : 128;
-  dim3 grid(cdiv(m, block), d / g);
-  const size_t smem = staged ? sizeof(float) * proj_floats(g) : 0;  // <= 34,816 bytes
+  const int tpg = staged ? g / 32 : 1;
+  const int rows = staged ? proj_rows(tpg) : 128;
+  const int block = staged ? 32 : 128;
+  dim3 grid(cdiv(m, rows), d / g);
+  const size_t smem = staged ? sizeof(float) * proj_floats(g, tpg) : 0;  // <= 9,856 bytes
   const int L = (1 << bits) - 1;
   const int enc = split == ADMMQ_SPLIT_MIXED ? ENC_MIX : (split == ADMMQ_SPLIT_F16 ? ENC_F16 : ENC_TF32X3);
-#define PROJECT_ENC(MODE, ENC)                                                               \
-  count_launch(), k_project<MODE, ENC, MODE != GRID_MSE><<<grid, block, smem, st>>>(         \
-                      wt, V, sig, rsig, hd, m, d, g, L, codes, scale, zero, p_hi, p_lo,      \
+#define PROJECT_LAUNCH(MODE, ENC, STAGED, TPG)                                           \
+  count_launch(), k_project<MODE, ENC, STAGED, TPG><<<grid, block, smem, st>>>(          \
+                      wt, V, sig, rsig, hd, m, d, g, L, codes, scale, zero, p_hi, p_lo,  \
                       row_scale, range_flag, resid, dual_scale, fit_on_w);
-#define PROJECT_CASE(MODE)       \
+#define PROJECT_STAGED(MODE, ENC)      \
+  if (tpg == 4) {                      \
+    PROJECT_LAUNCH(MODE, ENC, true, 4) \
+  } else if (tpg == 2) {               \
+    PROJECT_LAUNCH(MODE, ENC, true, 2) \
+  } else {                             \
+    PROJECT_LAUNCH(MODE, ENC, true, 1) \
+  }
+#define PROJECT_GLOBAL(MODE, ENC) PROJECT_LAUNCH(MODE, ENC, false, 1)
+#define PROJECT_CASE(MODE, KIND) \
   if (enc == ENC_MIX) {          \
-    PROJECT_ENC(MODE, ENC_MIX)   \
+    KIND(MODE, ENC_MIX)          \
   } else if (enc == ENC_F16) {   \
-    PROJECT_ENC(MODE, ENC_F16)   \
+    KIND(MODE, ENC_F16)          \
   } else {                       \
-    PROJECT_ENC(MODE, ENC_TF32X3) \
+    KIND(MODE, ENC_TF32X3)       \
   }
   if (mode == ADMMQ_GRID_MINMAX) {
-    PROJECT_CASE(GRID_MINMAX)
+    PROJECT_CASE(GRID_MINMAX, PROJECT_STAGED)
   } else if (mode == ADMMQ_GRID_LSQ) {
-    PROJECT_CASE(GRID_LSQ)
+    PROJECT_CASE(GRID_LSQ, PROJECT_STAGED)
   } else if (mode == ADMMQ_GRID_MSE) {
-    PROJECT_CASE(GRID_MSE)
+    PROJECT_CASE(GRID_MSE, PROJECT_GLOBAL)
   } else {
-    PROJECT_CASE(GRID_FROZEN)
+    PROJECT_CASE(GRID_FROZEN, PROJECT_STAGED)
   }
 #undef PROJECT_CASE
-#undef PROJECT_ENC
+#undef PROJECT_STAGED
+#undef PROJECT_GLOBAL
+#undef PROJECT_LAUNCH
   CK(cudaGetLastError());
   return ADMMQ_OK;
 }

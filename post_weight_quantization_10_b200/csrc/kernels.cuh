@@ -60,6 +60,10 @@ __device__ __forceinline__ void split_f16(float xs, uint16_t& hb, uint16_t& lb) 
   hb = __half_as_ushort(h);
   lb = __half_as_ushort(__float2half_rn(__fsub_rn(xs, __half2float(h))));
 }
+__device__ __forceinline__ uint32_t half2_bits(__half2 h) {
+  return (uint32_t)__half_as_ushort(__low2half(h)) |
+         ((uint32_t)__half_as_ushort(__high2half(h)) << 16);
+}
 // Index of column c's hi entry in its correction row (lo is 32 further on
 // for A operands, 32 before for B operands).
 __device__ __forceinline__ long long cplane_hi(long long c, bool b_side) {
@@ -100,16 +104,26 @@ template <int ENC>
 __device__ __forceinline__ void put_operand8(void* hi_row, void* lo_row, long long c,
                                              const float (&x)[8], float s, int* flag) {
   if (ENC == ENC_F16) {
-    uint16_t hb[8], lb[8];
+    // two elements per conversion: cvt.rn.f16x2.f32 rounds each one to
+    // nearest even, as split_f16 does, and leaves them packed (element 2j
+    // in the low half, the layout of the plane)
+    uint32_t hw[4], lw[4];
     bool bad = false;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const float xs = __fmul_rn(x[k], s);
-      bad |= !(fabsf(xs) < kF16Limit);
-      split_f16(xs, hb[k], lb[k]);
+    for (int j = 0; j < 4; ++j) {
+      const float a = __fmul_rn(x[2 * j], s), b = __fmul_rn(x[2 * j + 1], s);
+      bad |= !(fabsf(a) < kF16Limit);
+      bad |= !(fabsf(b) < kF16Limit);
+      const __half2 h = __floats2half2_rn(a, b);
+      const float2 hf = __half22float2(h);
+      const __half2 l = __floats2half2_rn(__fsub_rn(a, hf.x), __fsub_rn(b, hf.y));
+      hw[j] = half2_bits(h);
+      lw[j] = half2_bits(l);
     }
-    st_u16x8(reinterpret_cast<uint16_t*>(hi_row) + c, hb);
-    st_u16x8(reinterpret_cast<uint16_t*>(lo_row) + c, lb);
+    *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(hi_row) + c) =
+        make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(lo_row) + c) =
+        make_uint4(lw[0], lw[1], lw[2], lw[3]);
     if (bad && flag) *flag = 1;
     return;
   }
@@ -182,28 +196,40 @@ __device__ __forceinline__ float clampq(float q, float L) {
 // correctly rounded first (the same integers as rintf(__fdiv_rn(y, s))), from
 // r = __frcp_rn(s).  t = y r differs from the rounded quotient by at most
 // 1.5 * 2^-23 |y / s| (the reciprocal's and the product's roundings, 2^-24
-// each, and the quotient's own), so when t lies farther than 2^-21 |t| from
-// the nearest half-integer both round to the same integer.  Otherwise (a
-// near-tie, or a non-finite t) that value is divided exactly.  The eight
-// fast paths are straight-line code; the exact divisions are rare.
+// each, and the quotient's own), so when |t - rint(t)| is below the
+// threshold 0.5 - 2^-21 |t| (one fused multiply-add, rounded once) both
+// round to the same integer.  Otherwise (a near-tie, a negative threshold
+// for |t| >= 2^20, or a non-finite t) that value is divided exactly.  The
+// eight fast paths are straight-line code; the exact divisions are rare.
+__device__ __forceinline__ bool rint_fast_ok(float t, float q) {
+  return fabsf(__fsub_rn(t, q)) < __fmaf_rn(-4.76837158203125e-7f, fabsf(t), 0.5f);  // 2^-21
+}
 __device__ __forceinline__ void rint_div8(const float (&y)[8], float s, float r, float (&q)[8]) {
   bool exact = false;
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
     const float t = __fmul_rn(y[k], r);
     q[k] = rintf(t);
-    const float off = fabsf(__fsub_rn(t, q[k]));
-    exact |= !(off < __fsub_rn(0.5f, __fmul_rn(fabsf(t), 4.76837158203125e-7f)));  // 2^-21
+    exact |= !rint_fast_ok(t, q[k]);
   }
   if (exact) {
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const float t = __fmul_rn(y[k], r);
-      const float off = fabsf(__fsub_rn(t, rintf(t)));
-      if (!(off < __fsub_rn(0.5f, __fmul_rn(fabsf(t), 4.76837158203125e-7f))))
-        q[k] = rintf(__fdiv_rn(y[k], s));
+      if (!rint_fast_ok(t, rintf(t))) q[k] = rintf(__fdiv_rn(y[k], s));
     }
   }
+}
+
+// Codes as bytes without float-to-integer conversions: for an integer q in
+// [0, 255], q + 2^23 is exact and its low byte is q; for a byte b, the word
+// 0x4B0000bb is 2^23 + b.
+__device__ __forceinline__ uint32_t code_word(float q) { return __float_as_uint(__fadd_rn(q, 8388608.f)); }
+__device__ __forceinline__ uint32_t pack_codes4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+__device__ __forceinline__ float code_at(uint32_t w, int k) {  // byte k (0..3) of w
+  return __fsub_rn(__uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540u + (uint32_t)k)), 8388608.f);
 }
 
 // eight consecutive read-only floats (per-column vectors: sigma, 1/sigma, diag H)
@@ -243,7 +269,8 @@ __device__ __forceinline__ float warp_sum(float v) {
 //   minmax: mn = min(0, min y), mx = max(0, max y), s = (mx - mn)/L,
 //           z = rint(-mn/s)   (s = 1, z = 0 when mx = mn)
 //   lsq:    q0 = clamp(rint(y/s_prev) + z_prev); weighted sums (w = diag H)
-//           in element order; slope/offset, integer zero point, slope again
+//           over each half group in element order, then the two halves
+//           added; slope/offset, integer zero point, slope again
 //   q = clamp(rint(y/s) + z, 0, L);  D = s (q - z);  D~ = D rsig
 //   V~' = t - D~;  P = D~ - V~'  (stored in the GEMM operand encoding)
 
@@ -263,6 +290,7 @@ struct ProjRow {
   int fit_w;           // 1: refresh the grid from sigma W~ (V~ left out of the fit)
   int* flag;           // range flag of the fp16 split
   bool valid;
+  bool grid_out;       // this thread stores the group's scale and zero point
 };
 
 // Grid spanning [mn, mx] (mn <= 0 <= mx): s = (mx - mn) / L, z = rint(-mn / s);
@@ -340,10 +368,22 @@ __device__ __forceinline__ void mse_clip_grid(LoadW& loadw, LoadV& loadv, const 
 // v[8]) the dual V~ at c .. c + 7 (left at zero for an invalid row); the new
 // V~ is stored through r.V.  COLS_SMEM: r.sig, r.rsig and r.hd point into
 // shared memory.
-template <int MODE, int ENC, bool COLS_SMEM = false, class LoadW, class LoadV>
+//
+// The least-squares sums are taken over consecutive 32-column blocks, each in
+// element order, and the block sums are then added pairwise: (B0 + B1) +
+// (B2 + B3) for g = 128, B0 + B1 for 64, B0 for 32.  TPG > 1: that many lanes
+// share the group (TPG = g / 32), one block each (columns 0 .. 31 of r's
+// pointers, which the caller offsets to the block), lanes rr + (32 / TPG) j
+// for block j; the block sums (and min/max) are combined by shuffles in the
+// same pairwise order, every lane fits the same grid, and the lane with
+// r.grid_out stores it.  Every lane of the warp must call it then.
+template <int MODE, int ENC, bool COLS_SMEM = false, int TPG = 1, class LoadW, class LoadV>
 __device__ __forceinline__ void project_group(LoadW&& loadw, LoadV&& loadv, const ProjRow& r,
                                               int g, int L, float& r2, float& s2) {
+  static_assert(TPG == 1 || MODE != GRID_MSE, "the clipping search keeps one thread per group");
+  static_assert(TPG == 1 || TPG == 2 || TPG == 4, "one to four 32-column blocks per group");
   const float Lf = (float)L;
+  const int n = TPG > 1 ? 32 : g;  // columns of this thread
   float s0 = 1.f, z0 = 0.f;
   if (r.valid) {  // L2 reads: another SM may have written them in this launch
     s0 = __ldcg(r.scale);
@@ -354,8 +394,11 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, LoadV&& loadv, cons
   if (MODE != GRID_FROZEN) {
     float mn = 0.f, mx = 0.f;
     float Sw = 0.f, Sq = 0.f, Sqq = 0.f, Sy = 0.f, Sqy = 0.f;
+    // one thread per group: the last even block (E) and the first pair (A)
+    float Ew = 0.f, Eq = 0.f, Eqq = 0.f, Ey = 0.f, Eqy = 0.f;
+    float Aw = 0.f, Aq = 0.f, Aqq = 0.f, Ay = 0.f, Aqy = 0.f;
 #pragma unroll
-    for (int c = 0; c < g; c += 32) {
+    for (int c = 0; c < n; c += 32) {
       float w[32];
       loadw(c, w);
 #pragma unroll
@@ -386,6 +429,46 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, LoadV&& loadv, cons
           }
         }
       }
+      if (MODE == GRID_LSQ && TPG == 1) {  // block c / 32 ends: pairwise combination
+        if (c & 32) {  // odd block: its pair is E + S
+          Sw = __fadd_rn(Ew, Sw); Sq = __fadd_rn(Eq, Sq); Sqq = __fadd_rn(Eqq, Sqq);
+          Sy = __fadd_rn(Ey, Sy); Sqy = __fadd_rn(Eqy, Sqy);
+          if (c & 64) {  // the second pair: the total of four blocks stays in S
+            Sw = __fadd_rn(Aw, Sw); Sq = __fadd_rn(Aq, Sq); Sqq = __fadd_rn(Aqq, Sqq);
+            Sy = __fadd_rn(Ay, Sy); Sqy = __fadd_rn(Aqy, Sqy);
+          } else {
+            Aw = Sw; Aq = Sq; Aqq = Sqq; Ay = Sy; Aqy = Sqy;
+            Sw = 0.f; Sq = 0.f; Sqq = 0.f; Sy = 0.f; Sqy = 0.f;
+          }
+        } else {
+          Ew = Sw; Eq = Sq; Eqq = Sqq; Ey = Sy; Eqy = Sqy;
+          Sw = 0.f; Sq = 0.f; Sqq = 0.f; Sy = 0.f; Sqy = 0.f;
+        }
+      }
+    }
+    if (MODE == GRID_LSQ) {
+      if (TPG == 1) {
+        if (g == 32) {
+          Sw = Ew; Sq = Eq; Sqq = Eqq; Sy = Ey; Sqy = Eqy;
+        } else if (g == 64) {
+          Sw = Aw; Sq = Aq; Sqq = Aqq; Sy = Ay; Sqy = Aqy;
+        }
+      } else {  // lanes 32/TPG apart hold adjacent blocks; the sums are commutative
+#pragma unroll
+        for (int o = 32 / TPG; o < 32; o <<= 1) {
+          Sw = __fadd_rn(Sw, __shfl_xor_sync(0xffffffffu, Sw, o));
+          Sq = __fadd_rn(Sq, __shfl_xor_sync(0xffffffffu, Sq, o));
+          Sqq = __fadd_rn(Sqq, __shfl_xor_sync(0xffffffffu, Sqq, o));
+          Sy = __fadd_rn(Sy, __shfl_xor_sync(0xffffffffu, Sy, o));
+          Sqy = __fadd_rn(Sqy, __shfl_xor_sync(0xffffffffu, Sqy, o));
+        }
+      }
+    } else if (TPG > 1 && MODE == GRID_MINMAX) {
+#pragma unroll
+      for (int o = 32 / TPG; o < 32; o <<= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      }
     }
     if (MODE == GRID_MINMAX) {
       range_grid(mn, mx, Lf, s, z);
@@ -409,7 +492,7 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, LoadV&& loadv, cons
   }
   const float rs = __frcp_rn(s);
 #pragma unroll
-  for (int c = 0; c < g; c += 32) {
+  for (int c = 0; c < n; c += 32) {
     float w[32];
     loadw(c, w);
     uint32_t cw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // the 32 previous codes
@@ -423,6 +506,7 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, LoadV&& loadv, cons
       load8_col<COLS_SMEM>(r.sig + c + e, ss);
       load8_col<COLS_SMEM>(r.rsig + c + e, rr);
       float vn[8], pv[8];
+      uint32_t qb[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         t8[k] = __fadd_rn(w[e + k], vv[k]);
@@ -437,16 +521,17 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, LoadV&& loadv, cons
         const float dt = __fmul_rn(D, rr[k]);
         vn[k] = __fmul_rn(__fsub_rn(t, dt), r.vs);
         pv[k] = __fsub_rn(dt, vn[k]);
-        const int wi = (e + k) >> 2, sh = 8 * ((e + k) & 3);
-        if (sh == 0) qw[wi] = 0u;
-        qw[wi] |= (uint32_t)q << sh;
+        qb[k] = code_word(q);
         const float e1 = w[e + k] - dt;
         r2 += e1 * e1;
-        const float qp = (float)((cw[wi] >> sh) & 0xFFu);
+        // the previous iterate D~_prev = s0 (q_prev - z0) rsig, for the residual
+        const float qp = code_at(cw[(e + k) >> 2], (e + k) & 3);
         const float dtp = __fmul_rn(__fmul_rn(s0, __fsub_rn(qp, z0)), rr[k]);
         const float e2 = dt - dtp;
         s2 += e2 * e2;
       }
+      qw[e / 4] = pack_codes4(qb[0], qb[1], qb[2], qb[3]);
+      qw[e / 4 + 1] = pack_codes4(qb[4], qb[5], qb[6], qb[7]);
       if (r.valid) {
         st_v8f(r.V + c + e, vn);
         put_operand8<ENC>(r.phi, r.plo, c + e, pv, r.rs, r.flag);  // P, A side
@@ -460,7 +545,7 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, LoadV&& loadv, cons
     }
     if (r.valid) st_v8(r.codes + c, qw);
   }
-  if (r.valid) {
+  if (r.valid && r.grid_out) {
     *r.scale = s;
     *r.zero = z;
   }
@@ -640,6 +725,7 @@ struct EpiProject {
       r.vs = p.vs;
       r.fit_w = p.fit_w;
       r.valid = valid;
+      r.grid_out = true;
       // W~ = Q T: the accumulator carries the operands' scales (exact powers of two)
       auto loadw = [&](int c, float (&w)[32]) {
         tmem_ld32(taddr + c0 + c, w);

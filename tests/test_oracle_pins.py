@@ -388,7 +388,7 @@ def test_lsq_refit_does_not_increase_weighted_error():
 def test_lsq_refit_stages_against_lstsq():
     """Each stage of the least-squares refresh against numpy's least-squares
     solver in float64 on the same data (an independent route; the refit
-    itself sums in float32, element order):
+    itself sums in float32, by 32-column blocks):
     1. with the codes q of the previous grid, the weighted straight-line fit
        y ~ s1 q + b gives the slope s1 and the zero point z = -b / s1, which
        is rounded and clamped to an integer zc;
