@@ -459,6 +459,8 @@ __global__ void __launch_bounds__(STAGED ? 32 : 128) k_project(
     const float* __restrict__ row_in, int* flag, double* resid, float vs, int fit_w) {
   static_assert(TPG == 1 || STAGED, "lanes that share a group share staged rows");
   constexpr int kRows = STAGED ? proj_rows(TPG) : 128;
+  // staged launches have g = 32 TPG: a constant, so every index below folds
+  if (STAGED) g = 32 * TPG;
   extern __shared__ float4 proj_smem[];
   float* stage = reinterpret_cast<float*>(proj_smem);
   const int lane = threadIdx.x & 31;
@@ -470,6 +472,7 @@ __global__ void __launch_bounds__(STAGED ? 32 : 128) k_project(
     // rows past m are filled with zeros (they are projected, never stored)
     const int per_row = g / 2;  // float4 pieces of W~ and V~ in one row
     const uint32_t sbase = smem_u32(stage);
+#pragma unroll
     for (int i = lane; i < kRows * per_row; i += 32) {
       const int rr = i / per_row, piece = i - rr * per_row;
       const int arr = piece >= g / 4 ? 1 : 0;
@@ -483,6 +486,7 @@ __global__ void __launch_bounds__(STAGED ? 32 : 128) k_project(
       }
     }
     float* cols = stage + kRows * slot;
+#pragma unroll
     for (int i = lane; i < 3 * (g / 4); i += 32) {
       const int v = i / (g / 4), k = 4 * (i - v * (g / 4));
       const float* src = (v == 0 ? sig : v == 1 ? rsig : hd) + col0 + k;

@@ -204,6 +204,10 @@ __device__ __forceinline__ float clampq(float q, float L) {
 __device__ __forceinline__ bool rint_fast_ok(float t, float q) {
   return fabsf(__fsub_rn(t, q)) < __fmaf_rn(-4.76837158203125e-7f, fabsf(t), 0.5f);  // 2^-21
 }
+// The rare exact path, out of line: inlined, its eight divisions per batch
+// would sit between the hot instructions and spread them in the
+// instruction cache.
+__device__ __noinline__ float rint_div_exact(float y, float s) { return rintf(__fdiv_rn(y, s)); }
 __device__ __forceinline__ void rint_div8(const float (&y)[8], float s, float r, float (&q)[8]) {
   bool exact = false;
 #pragma unroll
@@ -216,7 +220,7 @@ __device__ __forceinline__ void rint_div8(const float (&y)[8], float s, float r,
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const float t = __fmul_rn(y[k], r);
-      if (!rint_fast_ok(t, rintf(t))) q[k] = rintf(__fdiv_rn(y[k], s));
+      if (!rint_fast_ok(t, rintf(t))) q[k] = rint_div_exact(y[k], s);
     }
   }
 }
@@ -470,9 +474,9 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, LoadV&& loadv, cons
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       }
     }
-    if (MODE == GRID_MINMAX) {
+    if constexpr (MODE == GRID_MINMAX) {
       range_grid(mn, mx, Lf, s, z);
-    } else if (MODE == GRID_MSE) {
+    } else if constexpr (MODE == GRID_MSE) {
       mse_clip_grid<COLS_SMEM>(loadw, loadv, r, g, Lf, mn, mx, s, z);
     } else {
       const float qm = __fdiv_rn(Sq, Sw);
