@@ -36,6 +36,9 @@ def _layer(name, seed=0):
         # the end), which is where the codes are a well-posed comparison
         "ragged": ("q_proj", 4096, 384, 200, dict(rank=16)),
         "down_small": ("down_proj", 4096, 256, 130, dict()),
+        # groups of 32 (one 32-column block per group) and 64 (two)
+        "ragged_g32": ("q_proj", 4096, 384, 200, dict(rank=16, group=32)),
+        "ragged_g64": ("q_proj", 4096, 384, 200, dict(rank=16, group=64)),
     }[name]
     p = workloads.scaled(workloads.PRESETS[base], n, d, m, **extra)
     X = workloads.make_activations(p, seed=seed, device="cuda")
@@ -96,7 +99,7 @@ def test_rtn_start_bitexact(A, name):
     np.testing.assert_array_equal(s.scale.cpu().numpy(), s_o.T)
 
 
-@pytest.mark.parametrize("name", ["tiny", "ragged"])
+@pytest.mark.parametrize("name", ["tiny", "ragged", "ragged_g32", "ragged_g64"])
 @pytest.mark.parametrize("grid", ["minmax", "lsq"])
 def test_first_iteration_w_update(A, name, grid):
     """W~ after iteration 0 (from the bit-exact RTN start) within 1e-4 relative
