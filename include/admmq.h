@@ -53,7 +53,9 @@ enum {
 /* Grid refresh used by the D-update (the pages do not fix the fit). */
 enum {
   ADMMQ_GRID_MINMAX = 0, /* scale/zero from the group's min/max, 0 included    */
-  ADMMQ_GRID_LSQ = 1,    /* weighted least-squares refit, weights diag(H)       */
+  ADMMQ_GRID_LSQ = 1,    /* weighted least-squares refit, weights diag(H); its
+                            float32 sums are taken per 32-column block in
+                            element order and the block sums added pairwise */
   ADMMQ_GRID_FROZEN = 2, /* keep the start grid (RTN grid of W_hat)             */
   ADMMQ_GRID_MSE = 3     /* MSE clipping search: the min/max grid of the range
                             clipped by a = (32 - k) / 32, k < 16, whose float32
