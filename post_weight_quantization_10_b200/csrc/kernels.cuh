@@ -273,8 +273,8 @@ __device__ __forceinline__ float warp_sum(float v) {
 //   minmax: mn = min(0, min y), mx = max(0, max y), s = (mx - mn)/L,
 //           z = rint(-mn/s)   (s = 1, z = 0 when mx = mn)
 //   lsq:    q0 = clamp(rint(y/s_prev) + z_prev); weighted sums (w = diag H)
-//           over each half group in element order, then the two halves
-//           added; slope/offset, integer zero point, slope again
+//           per 32-column block in element order, block sums added
+//           pairwise; slope/offset, integer zero point, slope again
 //   q = clamp(rint(y/s) + z, 0, L);  D = s (q - z);  D~ = D rsig
 //   V~' = t - D~;  P = D~ - V~'  (stored in the GEMM operand encoding)
 
