@@ -445,10 +445,19 @@ __global__ void k_rint_div(const float* __restrict__ y, const float* __restrict_
 __host__ __device__ constexpr int proj_rows(int tpg) { return 32 / tpg; }
 // floats per row slot: W~ (g), V~ (g), 4 of padding so that the rows' 16-byte
 // reads at one column spread over the banks; after the row slots, the
-// group's sigma, 1/sigma and diag(H) (g each), shared by the block's rows
+// group's sigma, 1/sigma and diag(H) (g each), shared by the block's rows;
+// then the rows' previous codes (g bytes each) and their scale and zero point
 __host__ __device__ constexpr int proj_slot(int g) { return 2 * g + 4; }
+__host__ __device__ constexpr int proj_cols(int g, int tpg) { return proj_rows(tpg) * proj_slot(g); }
+__host__ __device__ constexpr int proj_codes(int g, int tpg) { return proj_cols(g, tpg) + 3 * g; }
+// a row's codes take g + 16 bytes, so the lanes of one 16-byte read phase
+// (8 rows, the same column) fall on different banks
+__host__ __device__ constexpr int proj_code_row(int g) { return g + 16; }
+__host__ __device__ constexpr int proj_grid(int g, int tpg) {
+  return proj_codes(g, tpg) + proj_rows(tpg) * proj_code_row(g) / 4;
+}
 __host__ __device__ constexpr int proj_floats(int g, int tpg) {
-  return proj_rows(tpg) * proj_slot(g) + 3 * g;
+  return proj_grid(g, tpg) + 2 * proj_rows(tpg);
 }
 
 template <int MODE, int ENC, bool STAGED, int TPG>
@@ -456,7 +465,8 @@ __global__ void __launch_bounds__(STAGED ? 32 : 128) k_project(
     const float* __restrict__ wt, float* V, const float* __restrict__ sig,
     const float* __restrict__ rsig, const float* __restrict__ hd, int m, int d, int g, int L,
     uint8_t* codes, float* scale, float* zero, void* p_hi, void* p_lo,
-    const float* __restrict__ row_in, int* flag, double* resid, float vs, int fit_w) {
+    const float* __restrict__ row_in, int* flag, double* resid, float vs, int fit_w,
+    int ahead) {
   static_assert(TPG == 1 || STAGED, "lanes that share a group share staged rows");
   constexpr int kRows = STAGED ? proj_rows(TPG) : 128;
   // staged launches have g = 32 TPG: a constant, so every index below folds
@@ -492,9 +502,36 @@ __global__ void __launch_bounds__(STAGED ? 32 : 128) k_project(
       const float* src = (v == 0 ? sig : v == 1 ? rsig : hd) + col0 + k;
       cp_async16(smem_u32(cols + v * g + k), src);
     }
-    // the codes of this block's rows, read in the projection pass
-    if (lane < kRows && row0 + lane < m)
-      prefetch_l2_bulk(codes + (long long)(row0 + lane) * d + col0, (uint32_t)g);
+    // the previous codes of this block's rows and their scale and zero point
+    uint8_t* cs = reinterpret_cast<uint8_t*>(stage + proj_codes(g, TPG));
+#pragma unroll
+    for (int i = lane; i < kRows * (g / 16); i += 32) {
+      const int rr = i / (g / 16), k = 16 * (i - rr * (g / 16));
+      if (row0 + rr < m)
+        cp_async16(smem_u32(cs + rr * proj_code_row(g) + k),
+                   codes + (long long)(row0 + rr) * d + col0 + k);
+    }
+    float* gs = stage + proj_grid(g, TPG);
+    if (lane < kRows && row0 + lane < m) {
+      const long long gi = (long long)(row0 + lane) * (d / g) + grp;
+      cp_async4(smem_u32(gs + lane), scale + gi);
+      cp_async4(smem_u32(gs + kRows + lane), zero + gi);
+    }
+    // Blocks start in the order of their linear index, so the block `ahead`
+    // (one resident wave) later will run on an SM about when this one ends:
+    // bring its rows into L2 now, so that its copies find them there.
+    if (ahead > 0) {
+      const long long lin = blockIdx.x + (long long)blockIdx.y * gridDim.x + ahead;
+      if (lin < (long long)gridDim.x * gridDim.y) {
+        const int r0 = (int)(lin % gridDim.x) * kRows, c0 = (int)(lin / gridDim.x) * g;
+        if (lane < kRows && r0 + lane < m) {
+          const long long o = (long long)(r0 + lane) * d + c0;
+          prefetch_l2_bulk(wt + o, 4u * (uint32_t)g);
+          prefetch_l2_bulk(V + o, 4u * (uint32_t)g);
+          prefetch_l2_bulk(codes + o, (uint32_t)g);
+        }
+      }
+    }
     cp_async_wait_all();
     __syncwarp();
   }
@@ -530,6 +567,15 @@ __global__ void __launch_bounds__(STAGED ? 32 : 128) k_project(
   r.flag = flag;
   r.valid = valid;
   r.grid_out = blk == 0;
+  if (STAGED) {
+    r.codes_in = reinterpret_cast<const uint8_t*>(stage + proj_codes(g, TPG)) + rr * proj_code_row(g) + hc;
+    r.scale_in = stage + proj_grid(g, TPG) + rr;
+    r.zero_in = stage + proj_grid(g, TPG) + kRows + rr;
+  } else {
+    r.codes_in = nullptr;
+    r.scale_in = nullptr;
+    r.zero_in = nullptr;
+  }
   const float* mine = stage + rr * slot + hc;
   auto loadw = [&](int c, float (&w)[32]) {
 #pragma unroll
@@ -1567,13 +1613,22 @@ int admmq_project(const float* wt, float* V, const float* sig, const float* rsig
   const int rows = staged ? proj_rows(tpg) : 128;
   const int block = staged ? 32 : 128;
   dim3 grid(cdiv(m, rows), d / g);
-  const size_t smem = staged ? sizeof(float) * proj_floats(g, tpg) : 0;  // <= 9,856 bytes
+  const size_t smem = staged ? sizeof(float) * proj_floats(g, tpg) : 0;  // <= 11,072 bytes
   const int L = (1 << bits) - 1;
   const int enc = split == ADMMQ_SPLIT_MIXED ? ENC_MIX : (split == ADMMQ_SPLIT_F16 ? ENC_F16 : ENC_TF32X3);
-#define PROJECT_LAUNCH(MODE, ENC, STAGED, TPG)                                           \
-  count_launch(), k_project<MODE, ENC, STAGED, TPG><<<grid, block, smem, st>>>(          \
-                      wt, V, sig, rsig, hd, m, d, g, L, codes, scale, zero, p_hi, p_lo,  \
-                      row_scale, range_flag, resid, dual_scale, fit_on_w);
+#define PROJECT_LAUNCH(MODE, ENC, STAGED, TPG)                                             \
+  {                                                                                         \
+    int per_sm = 0;                                                                         \
+    if (STAGED)                                                                             \
+      CK(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_project<MODE, ENC, STAGED, TPG>, \
+                                                       block, smem));                       \
+    /* the L2 prefetch pays for the fp16 split's 4-byte P planes (measured: least  */     \
+    /* squares +10%, min/max and frozen +6%); with 8-byte planes it cost 2%         */     \
+    const int ahead = ENC == ENC_F16 ? num_sms() * per_sm : 0;                              \
+    count_launch(), k_project<MODE, ENC, STAGED, TPG><<<grid, block, smem, st>>>(            \
+                        wt, V, sig, rsig, hd, m, d, g, L, codes, scale, zero, p_hi, p_lo,   \
+                        row_scale, range_flag, resid, dual_scale, fit_on_w, ahead);         \
+  }
 #define PROJECT_STAGED(MODE, ENC)      \
   if (tpg == 4) {                      \
     PROJECT_LAUNCH(MODE, ENC, true, 4) \

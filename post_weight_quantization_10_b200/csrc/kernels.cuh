@@ -288,6 +288,11 @@ struct ProjRow {
   void* plo;           // P plane 1 at the group's first column
   float* scale;        // this group's scale / zero
   float* zero;
+  // COLS_SMEM: copies of the previous codes (the row's, at the group's first
+  // column) and of the group's scale and zero point in shared memory
+  const uint8_t* codes_in;
+  const float* scale_in;
+  const float* zero_in;
   float* wdump;        // optional raw W~ output
   float rs;            // the row's operand scale (fp16 split; 1 otherwise)
   float vs;            // dual rescaling rho_t / rho_{t+1} (1 without it)
@@ -390,8 +395,8 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, LoadV&& loadv, cons
   const int n = TPG > 1 ? 32 : g;  // columns of this thread
   float s0 = 1.f, z0 = 0.f;
   if (r.valid) {  // L2 reads: another SM may have written them in this launch
-    s0 = __ldcg(r.scale);
-    z0 = __ldcg(r.zero);
+    s0 = COLS_SMEM ? *r.scale_in : __ldcg(r.scale);
+    z0 = COLS_SMEM ? *r.zero_in : __ldcg(r.zero);
   }
   float s = s0, z = z0;
   const float r0 = __frcp_rn(s0);
@@ -500,7 +505,16 @@ __device__ __forceinline__ void project_group(LoadW&& loadw, LoadV&& loadv, cons
     float w[32];
     loadw(c, w);
     uint32_t cw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // the 32 previous codes
-    if (r.valid) ld_v8(r.codes + c, cw);
+    if (r.valid) {
+      if (COLS_SMEM) {
+        const uint4 a = *reinterpret_cast<const uint4*>(r.codes_in + c);
+        const uint4 b = *reinterpret_cast<const uint4*>(r.codes_in + c + 16);
+        cw[0] = a.x; cw[1] = a.y; cw[2] = a.z; cw[3] = a.w;
+        cw[4] = b.x; cw[5] = b.y; cw[6] = b.z; cw[7] = b.w;
+      } else {
+        ld_v8(r.codes + c, cw);
+      }
+    }
     uint32_t qw[8];
 #pragma unroll
     for (int e = 0; e < 32; e += 8) {
@@ -730,6 +744,9 @@ struct EpiProject {
       r.fit_w = p.fit_w;
       r.valid = valid;
       r.grid_out = true;
+      r.codes_in = nullptr;  // read from global memory (COLS_SMEM = false)
+      r.scale_in = nullptr;
+      r.zero_in = nullptr;
       // W~ = Q T: the accumulator carries the operands' scales (exact powers of two)
       auto loadw = [&](int c, float (&w)[32]) {
         tmem_ld32(taddr + c0 + c, w);
