@@ -520,9 +520,9 @@ __global__ void __launch_bounds__(STAGED ? 32 : 128) k_project(
     // Blocks start in the order of their linear index, so the block `ahead`
     // (one resident wave) later will run on an SM about when this one ends:
     // bring its rows into L2 now, so that its copies find them there.
-    if (ahead > 0) {
-      const long long lin = blockIdx.x + (long long)blockIdx.y * gridDim.x + ahead;
-      if (lin < (long long)gridDim.x * gridDim.y) {
+    if (ahead > 0) {  // the grid has fewer than 2^31 blocks (the host checks)
+      const unsigned lin = blockIdx.x + blockIdx.y * gridDim.x + (unsigned)ahead;
+      if (lin < gridDim.x * gridDim.y) {
         const int r0 = (int)(lin % gridDim.x) * kRows, c0 = (int)(lin / gridDim.x) * g;
         if (lane < kRows && r0 + lane < m) {
           const long long o = (long long)(r0 + lane) * d + c0;
@@ -1624,7 +1624,8 @@ int admmq_project(const float* wt, float* V, const float* sig, const float* rsig
                                                        block, smem));                       \
     /* the L2 prefetch pays for the fp16 split's 4-byte P planes (measured: least  */     \
     /* squares +10%, min/max and frozen +6%); with 8-byte planes it cost 2%         */     \
-    const int ahead = ENC == ENC_F16 ? num_sms() * per_sm : 0;                              \
+    const int ahead = (ENC == ENC_F16 && (long long)grid.x * grid.y < (1ll << 31))          \
+                          ? num_sms() * per_sm : 0;                                        \
     count_launch(), k_project<MODE, ENC, STAGED, TPG><<<grid, block, smem, st>>>(            \
                         wt, V, sig, rsig, hd, m, d, g, L, codes, scale, zero, p_hi, p_lo,   \
                         row_scale, range_flag, resid, dual_scale, fit_on_w, ahead);         \
