@@ -438,15 +438,18 @@ __global__ void k_rint_div(const float* __restrict__ y, const float* __restrict_
 // a whole row segment per instruction for g = 128); the passes read them
 // from there and DRAM sees each input once.  A lane takes one 32-column block
 // of a (row, group): TPG = g / 32 lanes share a group and a warp holds 32 /
-// TPG rows (8 for g = 128), so a warp stages about 9 KB whatever g is and
-// many warps fit on an SM.  The 16-candidate error search of GRID_MSE is
-// bound by arithmetic rather than memory, so it reads W~ and V~ from global
-// memory (STAGED = false, 128-thread blocks, a thread per (row, group)).
+// TPG rows (8 for g = 128), so a warp stages about 11 KB whatever g is and
+// many warps fit on an SM.  The rows' previous codes, scales and zero points
+// are staged too, so the passes wait on no global load.  The 16-candidate
+// error search of GRID_MSE is bound by arithmetic rather than memory, so it
+// reads W~ and V~ from global memory (STAGED = false, 128-thread blocks, a
+// thread per (row, group)).
 __host__ __device__ constexpr int proj_rows(int tpg) { return 32 / tpg; }
 // floats per row slot: W~ (g), V~ (g), 4 of padding so that the rows' 16-byte
 // reads at one column spread over the banks; after the row slots, the
 // group's sigma, 1/sigma and diag(H) (g each), shared by the block's rows;
-// then the rows' previous codes (g bytes each) and their scale and zero point
+// then the rows' previous codes (g + 16 bytes each) and their scales and zero
+// points
 __host__ __device__ constexpr int proj_slot(int g) { return 2 * g + 4; }
 __host__ __device__ constexpr int proj_cols(int g, int tpg) { return proj_rows(tpg) * proj_slot(g); }
 __host__ __device__ constexpr int proj_codes(int g, int tpg) { return proj_cols(g, tpg) + 3 * g; }
